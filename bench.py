@@ -1,0 +1,386 @@
+"""Benchmark of windowed INT8 delta-rule decode on B200.
+
+`python bench.py --gpus N --steps K --warmup W [--workload NAME] [--impl ours|reference]`
+
+One step = one window of the workload on every head of the batch: W decode
+calls through the C ABI (the W-th also reconstructs, re-extracts the
+compensators, smooths and requantizes the state), replayed from a CUDA graph.
+Prints ONE JSON line (rank 0).  Default workload: GDN, 1024 independent
+states x 16 heads, d = 128, W = 64, r = 4 (state + buffers ~1.3 GB, larger
+than L2, so no L2 flush is needed between steps).
+
+--impl reference times the CPU oracle (the plain C implementation the parity
+tests compare against) on a bounded sample of heads of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_recurrent_state_lq_b200 import configs, inputs as gen, lq, runner, traffic  # noqa: E402
+
+METRIC = "state updates/s (batch·head·token) and achieved HBM TB/s vs ~8 TB/s B200 peak"
+UNIT = "state updates/s"
+DEFAULT_WL = configs.GDN_PREFIX_CACHE.name
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+            0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons of this process's GPU through NVML."""
+
+    def __init__(self, device: int, period: float = 0.05):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            p = torch.cuda.get_device_properties(device)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nv = pynvml
+        except Exception:  # NVML unavailable: report no clocks
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in _REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._h is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return None
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+        pg = dist
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local, pg
+
+
+def max_over_ranks(x: float, pg) -> float:
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample_seconds(wl, heads: int, threads: int, seed_offset: int = 0):
+    """Time the oracle on `heads` heads of the workload for one window (W tokens
+    and the flush).  Initial states: a short oracle prefill plus the workload's
+    outliers (the decode's CPU work does not depend on the values)."""
+    import numpy as np
+    from oracle import oracle as O
+    sw = wl.with_(B=max(1, heads // wl.H + (heads % wl.H > 0)), seed=wl.seed + seed_offset)
+    oc = O.Cfg(dk=wl.dk, dv=wl.dv, gate=wl.gate, W=wl.W, r=wl.r, K=wl.K, smoothing=wl.smoothing, P=wl.P)
+    pre = gen.token_inputs(sw, 16, stream="prefill")
+    S0 = O.prefill(O.Cfg(dk=wl.dk, dv=wl.dv, gate=wl.gate, quantize=0), O.per_head_inputs(pre, wl.H),
+                   nthreads=threads).astype(np.float32).reshape(sw.B, wl.H, wl.dk, wl.dv)
+    S0 = gen.apply_outliers(torch.from_numpy(S0), sw).numpy().reshape(-1, wl.dk, wl.dv)[:heads]
+    tok = O.per_head_inputs(gen.token_inputs(sw, wl.W), wl.H)
+    tok = {k: np.ascontiguousarray(v[:, :heads]) for k, v in tok.items()}
+    rows = None
+    if wl.P:
+        rows = np.tile(np.arange(wl.P, dtype=np.int32) * (wl.dk // wl.P), (heads, 1))
+    t0 = time.perf_counter()
+    O.run(oc, tok, S0=S0, hp_rows=rows, flush_last=True, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return dt
+
+
+def cpu_baseline(wl, target_s: float = 12.0):
+    threads = os.cpu_count() or 1
+    probe = 32
+    dt = oracle_sample_seconds(wl, probe, threads)
+    heads = int(max(probe, min(100000, probe * target_s / max(dt, 1e-3))))
+    dt = oracle_sample_seconds(wl, heads, threads, seed_offset=1)
+    value = heads * wl.W / dt
+    return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{heads} heads of {wl.name} x one window ({wl.W} tokens + flush), "
+                      f"includes the oracle's initial quantization; {dt:.1f} s"}
+
+
+def run_reference(args, wl, world, rank, pg):
+    if rank != 0:
+        return 0
+    threads = os.cpu_count() or 1
+    probe = 16
+    dt = oracle_sample_seconds(wl, probe, threads)
+    heads = int(max(probe, min(100000, probe * 2.5 / max(dt, 1e-3))))   # ~2.5 s per step
+    for _ in range(args.warmup):
+        oracle_sample_seconds(wl, heads, threads)
+    times = [oracle_sample_seconds(wl, heads, threads, seed_offset=1 + k) for k in range(args.steps)]
+    t = sum(times)
+    value = heads * wl.W * args.steps / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "sample_heads": heads},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"{heads} heads x one window of {wl.W} tokens per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def profile_traffic(wl):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel sources; else None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "decode_window_traffic.txt")
+    try:
+        kv = dict(line.split(":", 1) for line in open(path) if ":" in line)
+    except OSError:
+        return None
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "quantized_recurrent_state_lq_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    if kv.get("csrc_sha256", "").strip() != h.hexdigest()[:16] or kv.get("workload", "").strip() != wl.name:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch_full"])
+    except (KeyError, ValueError):
+        return None
+
+
+def time_graph_steps(r: runner.WindowRunner, K: int, start: int, stream) -> float:
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for k in range(K):
+        r.replay(start + k)
+    ev1.record(stream)
+    ev1.synchronize()
+    return ev0.elapsed_time(ev1) / 1e3
+
+
+def kernel_times(r: runner.WindowRunner, windows: int, stream):
+    """Mean device time of the buffering decode launches and of the flushing
+    launch, each bracketed by CUDA events on the launching stream."""
+    W = r.W
+    evs = []
+    for w in range(windows):
+        for t in range(W):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            r.step_call(w * W + t)
+            b.record(stream)
+            evs.append((t, a, b))
+    torch.cuda.synchronize()
+    buf = [a.elapsed_time(b) / 1e3 for t, a, b in evs if t < W - 1]
+    fl = [a.elapsed_time(b) / 1e3 for t, a, b in evs if t == W - 1]
+    return (statistics.mean(buf) if buf else None), statistics.mean(fl)
+
+
+def e2e_measure(r: runner.WindowRunner, steps: int, stream):
+    """Whole windows through the C ABI with HOST inputs and outputs: pinned
+    host -> device copy of the window's inputs, the W calls, and the device ->
+    host copy of its outputs, all inside the timed region."""
+    W = r.W
+    keys = ["q", "k", "v", "beta", "alpha"]
+    host_in = {k: torch.empty_like(r.tok[k][:W], device="cpu").pin_memory() for k in keys}
+    for k in keys:
+        host_in[k].copy_(r.tok[k][:W])
+    host_out = torch.empty_like(r.out[:W], device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for k in range(steps):
+        for key in keys:
+            r.tok[key][:W].copy_(host_in[key], non_blocking=True)
+        r.replay(0)
+        host_out.copy_(r.out[:W], non_blocking=True)
+    ev1.record(stream)
+    ev1.synchronize()
+    dt = ev0.elapsed_time(ev1) / 1e3
+    return dt, h2d, d2h
+
+
+def mode_throughput(wl, S0, mode: str, windows: int, stream):
+    """Throughput of a reference mode on the same inputs (FP32 state or
+    per-step INT8), timed over whole graph-replayed windows."""
+    r = runner.WindowRunner(wl, S0, mode=mode, tokens=wl.W * min(2, wl.T // wl.W))
+    r.capture()
+    for k in range(2):
+        r.replay(k)
+    torch.cuda.synchronize()
+    dt = time_graph_steps(r, windows, 0, stream)
+    v = wl.heads * wl.W * windows / dt
+    del r
+    torch.cuda.empty_cache()
+    return v
+
+
+def run_ours(args, wl, world, rank, pg):
+    dev = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = measured_peaks()
+    rows = runner.damp_rows(wl) if wl.P else None
+    S0, _ = runner.initial_state(wl)
+    r = runner.WindowRunner(wl, S0, hp_rows=rows)
+    r.capture()
+    for k in range(args.warmup):
+        r.replay(k)
+    torch.cuda.synchronize()
+    barrier(pg)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        dt = time_graph_steps(r, args.steps, args.warmup, stream)
+    torch.cuda.synchronize()
+    barrier(pg)
+    dt_max = max_over_ranks(dt, pg)
+    rc = lq.lq_get_status(r.st)
+    if rc != lq.LQ_OK:
+        raise lq.LqError(rc, "decode status")
+
+    updates = wl.heads * wl.W * args.steps * world
+    value = updates / dt_max
+    step_bytes = traffic.window_bytes(wl) * wl.heads
+    t_buf, t_flush = kernel_times(r, 2, stream)
+    launch_bytes = traffic.nonflush_launch_bytes(wl) * wl.heads
+    achieved = launch_bytes / t_buf / 1e9
+    tr = profile_traffic(wl)
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": tr,
+            "kernel": "decode_kernel (buffering launches, n = 0..W-2)",
+            "algorithmic_bytes_per_launch": launch_bytes, "mean_launch_s": t_buf,
+            "peak_source": f"{peak_src} hbm_gbs (copy kernel)"}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "state_dtype": "int8", "data": "synthetic",
+            "config": {"workload": wl.name, "gate": wl.gate, "B": wl.B, "H": wl.H, "Hk": wl.Hk, "dk": wl.dk,
+                       "dv": wl.dv, "W": wl.W, "r": wl.r, "K": wl.K, "P": wl.P, "step": "one window per head",
+                       "l2": "state + buffers + inputs larger than L2 (no flush needed)",
+                       "parallelism": f"dp{world} (independent heads, no collective)"},
+            "hbm": {"achieved_tbs": step_bytes * args.steps / dt / 1e12,
+                    "frac_of_8tbs": step_bytes * args.steps / dt / 8e12,
+                    "frac_of_measured": step_bytes * args.steps / dt / 1e9 / peaks["hbm_gbs"],
+                    "algorithmic_bytes_per_step": step_bytes},
+            "kernels": {"decode_buffering_mean_s": t_buf, "decode_flushing_mean_s": t_flush},
+            "roofline": roof, "gpu_launches": wl.W * args.steps, "clocks": clk.summary()}
+
+    e2e_steps = max(1, min(args.steps, 5))
+    dte, h2d, d2h = e2e_measure(r, e2e_steps, stream)
+    dte = max_over_ranks(dte, pg)
+    line["e2e"] = {"value": wl.heads * wl.W * e2e_steps * world / dte, "unit": UNIT,
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del r
+    torch.cuda.empty_cache()
+
+    if not args.no_modes and wl.P == 0:
+        modes = {"window_int8": value / world}
+        modes["fp32_state"] = mode_throughput(wl, S0, "fp32", 4, stream)
+        modes["per_step_int8"] = mode_throughput(wl, S0, "step", 2, stream)
+        nv = wl.with_(r=0, smoothing=0)
+        modes["naive_per_step_int8"] = mode_throughput(nv, S0, "step", 2, stream)
+        modes["window_vs_fp32_speedup"] = modes["window_int8"] / modes["fp32_state"]
+        line["modes_per_gpu"] = modes
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WL, choices=sorted(configs.BY_NAME))
+    ap.add_argument("--no-modes", action="store_true", help="skip the FP32 / per-step INT8 context lines")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    wl = configs.BY_NAME[args.workload]
+    world, rank, local, pg = dist_setup()
+    try:
+        if args.impl == "reference":
+            rc = run_reference(args, wl, world, rank, pg)
+        else:
+            rc = run_ours(args, wl, world, rank, pg)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,199 @@
+/*
+ * lq_state.h -- C ABI of the windowed low-bit recurrent-state decode library
+ * (liblq.so), for Gated DeltaNet (one decay per head) and KDA (one decay per
+ * key channel) on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow these passages:
+ *  - recurrence: "LinQuant: Functional Invariances for Low-Precision Linear
+ *    Recurrences", appendix Table 3 (Gated DeltaNet and Kimi Delta Attention
+ *    rows).  The state is kept as S (d_k x d_v, key rows, value columns), the
+ *    transpose of the table's form:  S_t = (I - b_t k_t k_t^T) D_t S_{t-1}
+ *    + b_t k_t v_t^T,  o_t = S_t^T q_t,  D_t = a_t I (GDN) or diag(a_t) (KDA).
+ *  - windowed quantization: "LeapQuant: Efficient Linear Attention with
+ *    Accurate Recurrent State Quantization" (project page), paragraph on
+ *    leaping over a window: the state is stored in low precision at the
+ *    window start and held fixed; higher-precision token updates are
+ *    buffered; each output comes from the fixed state plus the buffer; at the
+ *    window end the full state is reconstructed and quantized again.
+ *  - Compensator Tokens: same page, next paragraph: a few high-precision
+ *    rank-one outer products keep the largest outliers and share the real
+ *    tokens' update path.
+ *  - smoothing: same page, following paragraph: per-key-row scales balance
+ *    the residual before quantizing, recomputed at every window boundary;
+ *    key-row and value-column scales also in "How does STEPQuant compress
+ *    recurrent states without losing accuracy?".
+ *  - BF16 rows: "DAMP: Decay-Aware Mixed-Precision Recurrent-State
+ *    Quantization", abstract: high-risk channels stored at higher precision,
+ *    the rest in INT8.
+ *
+ * Conventions for every call:
+ *  - d_* arguments are DEVICE pointers owned by the caller (for instance the
+ *    data_ptr() of torch tensors); h_* arguments are HOST pointers.  Nothing
+ *    is freed by the library except the opaque handle in lq_state_destroy.
+ *  - Floating-point tensors are float32, C-contiguous, in the shapes given.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Compute
+ *    calls are asynchronous on it unless their comment says they synchronize.
+ *  - Every call returns LQ_OK (0) or a negative lq_status; argument errors are
+ *    detected on the host before anything is launched, and a call that
+ *    returns an error has launched nothing.  No C++ exception crosses the ABI.
+ *  - Supported head sizes: d_k, d_v in {64, 128}.
+ */
+#ifndef LQ_STATE_H
+#define LQ_STATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LQ_OK = 0,
+    LQ_ERR_INVALID_ARG = -1,  /* null pointer, bad enum, W < 1, r > min(dk,dv), ... */
+    LQ_ERR_SHAPE = -2,        /* B, H, Hk, dk, dv inconsistent or Hk does not divide H */
+    LQ_ERR_WORKSPACE = -3,    /* workspace too small or not 256-byte aligned */
+    LQ_ERR_WINDOW_FULL = -4,  /* lq_decode_step with W tokens already buffered */
+    LQ_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed */
+    LQ_ERR_NONFINITE = -6,    /* a kernel saw a NaN/Inf output (lq_get_status) */
+    LQ_ERR_UNSUPPORTED = -7,  /* head size or combination not built */
+    LQ_ERR_TIMEOUT = -8       /* a bounded device wait gave up (lq_get_status) */
+} lq_status;
+
+typedef enum { LQ_GATE_SCALAR = 0 /* GDN */, LQ_GATE_CHANNEL = 1 /* KDA */ } lq_gate;
+
+typedef enum {
+    LQ_MODE_FP32 = 0,        /* FP32 state, read and written every token (baseline) */
+    LQ_MODE_INT8_STEP = 1,   /* INT8 state requantized after every token (W must be 1) */
+    LQ_MODE_INT8_WINDOW = 2  /* INT8 state quantized once per window of W tokens */
+} lq_mode;
+
+typedef struct {
+    int32_t B, H, Hk;       /* batch, value heads, q/k heads (Hk divides H; GQA map h -> h*Hk/H) */
+    int32_t dk, dv;         /* key / value head size */
+    int32_t gate;           /* lq_gate */
+    int32_t mode;           /* lq_mode */
+    int32_t W;              /* window length (tokens per quantization) */
+    int32_t r;              /* compensator tokens per head, 0..min(dk,dv) */
+    int32_t power_iters;    /* power-iteration steps per compensator (K), >= 0 */
+    int32_t n_hp_rows;      /* P: BF16 key rows per head (DAMP layout), 0 = all INT8 */
+    int32_t smoothing;      /* 1: per-key-row RMS smoothing; 0: none (m = 1) */
+    int32_t fused_flush;    /* 1: the call that buffers the W-th token also flushes */
+} lq_config;
+
+/* A quantized state in plain arrays (all device pointers, caller-owned):
+ *   codes     int8   [B,H,dk-P,dv]  INT8 key rows in increasing row order, dv contiguous
+ *   bf16_rows uint16 [B,H,P,dv]     BF16 bit patterns of the rows listed in hp_row_ids
+ *   m         float  [B,H,dk]       smoothing scale per key row (1 on BF16 rows)
+ *   s         float  [B,H,dv]       quantization scale per value column
+ *   comp_k    float  [B,H,r,dk]     compensator key-side vectors c_j
+ *   comp_v    float  [B,H,r,dv]     compensator value-side vectors w_j
+ * The represented state is  S_ic = (C_ic * s_c) * m_i  (float, in that order) on
+ * INT8 rows, bf16(B_pc) on BF16 rows, plus sum_j c_j[i] w_j[c].
+ * bf16_rows may be NULL when P = 0; comp_k/comp_v may be NULL when r = 0. */
+typedef struct {
+    int8_t *codes;
+    uint16_t *bf16_rows;
+    float *m;
+    float *s;
+    float *comp_k;
+    float *comp_v;
+} lq_qstate_view;
+
+typedef struct lq_state lq_state; /* opaque; host memory owned by the library */
+
+/* Bytes of device workspace lq_state_init needs for cfg (0 if cfg is invalid). */
+size_t lq_workspace_bytes(const lq_config *cfg);
+
+/* Check a config without touching the GPU; returns LQ_OK or the error code. */
+int lq_config_check(const lq_config *cfg);
+
+/*
+ * Create a decode state in caller-owned device memory d_workspace (>=
+ * lq_workspace_bytes(cfg) bytes, 256-byte aligned) from an FP32 initial state
+ * d_S0 [B,H,dk,dv].  INT8 modes quantize it (compensators, smoothing, codes);
+ * FP32 mode copies it.  h_hp_row_ids [H,P] (HOST, required iff P > 0) lists
+ * each head's BF16 key rows, distinct and in [0,dk); the same rows serve every
+ * batch entry.  Synchronizes `stream` once (status word reset).  The handle
+ * must be released with lq_state_destroy; the workspace must outlive it.
+ */
+int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_t bytes,
+                  const float *d_S0, const int32_t *h_hp_row_ids, void *stream);
+
+/*
+ * Decode one token for all B*H heads:  q, k [B,Hk,dk], v [B,H,dv], beta [B,H],
+ * alpha [B,H] (GDN) or [B,H,dk] (KDA)  ->  o [B,H,dv].
+ * INT8_WINDOW: the output comes from the window-start INT8 state, its
+ * compensators and the buffered updates; the new update (k_t / Gamma_t, u_t)
+ * is appended to the buffer and the INT8 state is not written.  With
+ * fused_flush = 1 the call that buffers the W-th token also reconstructs and
+ * requantizes the state (the window ends); with fused_flush = 0 a call with W
+ * tokens already buffered returns LQ_ERR_WINDOW_FULL and launches nothing.
+ * INT8_STEP: decode and requantize in the same launch, every token.
+ * FP32: read, update and write the FP32 state.
+ */
+int lq_decode_step(lq_state *st, const float *d_q, const float *d_k, const float *d_v,
+                   const float *d_beta, const float *d_alpha, float *d_o, void *stream);
+
+/* End the current window: reconstruct S = Gamma (Deq + comps + buffer) and
+ * quantize it (new compensators, smoothing, codes); resets the buffer.  A no-op
+ * with nothing buffered and in FP32 / INT8_STEP modes. */
+int lq_window_flush(lq_state *st, void *stream);
+
+/* Tokens buffered in the current window (host counter, no synchronization). */
+int lq_state_buffered(const lq_state *st);
+
+/* Write the exact current state, Gamma (Deq + comps + buffer) in INT8 modes or
+ * the FP32 state, to d_S [B,H,dk,dv].  Does not change the state. */
+int lq_state_export_fp32(const lq_state *st, float *d_S, void *stream);
+
+/* Copy the window-start quantized state out to / in from plain arrays (layout of
+ * lq_qstate_view, for this state's B and H).  Import starts a new window
+ * (buffer emptied, Gamma = 1).  INT8 modes only.  Used for checkpoint/resume. */
+int lq_state_export_view(const lq_state *st, const lq_qstate_view *out, void *stream);
+int lq_state_import_view(lq_state *st, const lq_qstate_view *in, void *stream);
+
+/*
+ * Stateless codec on B*H heads.  lq_quantize_state: d_S [B,H,dk,dv] -> out
+ * (compensators by power iteration, smoothing, per-column scales, INT8 codes,
+ * BF16 rows).  lq_dequantize_state: in -> d_S.  cfg supplies B, H, dk, dv, r,
+ * power_iters, smoothing and P; h_hp_row_ids [H,P] is a HOST array (NULL iff
+ * P = 0), checked on the host; when P > 0 a device copy of it lives in a
+ * stream-ordered temporary (cudaMallocAsync / cudaFreeAsync on `stream`).
+ */
+int lq_quantize_state(const lq_config *cfg, const float *d_S, const int32_t *h_hp_row_ids,
+                      lq_qstate_view *out, void *stream);
+int lq_dequantize_state(const lq_config *cfg, const lq_qstate_view *in,
+                        const int32_t *h_hp_row_ids, float *d_S, void *stream);
+
+/*
+ * DAMP channel risk (offline calibration; DAMP abstract: error energy and
+ * decay-based persistence pick the high-risk channels).  For each head h:
+ *   E[h,i]  = sum_n sum_c (R - Deq(R))_ic^2 over the n_states FP32 states
+ *             d_states [n_states,H,dk,dv], R being the residual after cfg->r
+ *             compensators and Deq its INT8 reconstruction (no BF16 rows,
+ *             smoothing per cfg->smoothing);
+ *   score   = E[h,i] / (1 - mean decay), the mean taken over the
+ *             n_gate_samples calibration gates d_gates [n_gate_samples,H,ga]
+ *             (ga = 1 for GDN: one mean per head; ga = dk for KDA: per row);
+ *   d_rows [H,P] <- the P = cfg->n_hp_rows best rows per head (ties to the
+ *             lower index) in increasing row order; d_energy [H,dk] <- E.
+ * Uses cfg's H, dk, dv, gate, r, power_iters, smoothing, n_hp_rows (>= 1).
+ */
+int lq_damp_select(const lq_config *cfg, int32_t n_states, const float *d_states,
+                   int32_t n_gate_samples, const float *d_gates, double *d_energy,
+                   int32_t *d_rows, void *stream);
+
+/* Synchronize `stream` and return the sticky device status of this state:
+ * LQ_OK, LQ_ERR_NONFINITE or LQ_ERR_TIMEOUT. */
+int lq_get_status(lq_state *st, void *stream);
+
+void lq_state_destroy(lq_state *st);
+
+const char *lq_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LQ_STATE_H */

@@ -1,0 +1,387 @@
+// lq_api.cu -- the C ABI declared in include/lq_state.h: argument checks,
+// workspace carving, the host-side window counter and kernel sequencing.
+// Every entry point validates on the host first and launches nothing on error.
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "../../include/lq_state.h"
+#include "lq_kernels.h"
+
+using lq::Layout;
+
+struct lq_state {
+    lq_config cfg;
+    Layout L;
+    unsigned char *ws;
+    size_t bytes;
+    int *status;
+    int *hp_rows;
+    unsigned char *rec;
+    size_t heads;
+    int n;  // tokens buffered in the current window
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kMaxSmem = 227 * 1024;
+
+size_t align_sz(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool is_int8(const lq_config *c) { return c->mode == LQ_MODE_INT8_STEP || c->mode == LQ_MODE_INT8_WINDOW; }
+
+Layout layout_of(const lq_config *c) {
+    const int W = c->mode == LQ_MODE_INT8_STEP ? 1 : c->W;
+    return lq::make_layout(c->dk, c->dv, c->n_hp_rows, c->r, W, c->gate == LQ_GATE_CHANNEL);
+}
+
+int check_codec_fields(const lq_config *c) {
+    if (c->dk != 64 && c->dk != 128) return LQ_ERR_UNSUPPORTED;
+    if (c->dv != 64 && c->dv != 128) return LQ_ERR_UNSUPPORTED;
+    if (c->r < 0 || c->r > (c->dk < c->dv ? c->dk : c->dv)) return LQ_ERR_INVALID_ARG;
+    if (c->power_iters < 0 || c->power_iters > 1000) return LQ_ERR_INVALID_ARG;
+    if (c->n_hp_rows < 0 || c->n_hp_rows >= c->dk) return LQ_ERR_INVALID_ARG;
+    if (c->smoothing != 0 && c->smoothing != 1) return LQ_ERR_INVALID_ARG;
+    return LQ_OK;
+}
+
+int check_config(const lq_config *c) {
+    if (!c) return LQ_ERR_INVALID_ARG;
+    if (c->B < 1 || c->H < 1 || c->Hk < 1) return LQ_ERR_SHAPE;
+    if (c->Hk > c->H || c->H % c->Hk != 0) return LQ_ERR_SHAPE;
+    if ((long long)c->B * c->H > (1ll << 31) - 1) return LQ_ERR_SHAPE;
+    if (c->gate != LQ_GATE_SCALAR && c->gate != LQ_GATE_CHANNEL) return LQ_ERR_INVALID_ARG;
+    if (c->mode != LQ_MODE_FP32 && c->mode != LQ_MODE_INT8_STEP && c->mode != LQ_MODE_INT8_WINDOW)
+        return LQ_ERR_INVALID_ARG;
+    if (c->fused_flush != 0 && c->fused_flush != 1) return LQ_ERR_INVALID_ARG;
+    int rc = check_codec_fields(c);
+    if (rc) return rc;
+    if (is_int8(c)) {
+        if (c->W < 1) return LQ_ERR_INVALID_ARG;
+        if (c->mode == LQ_MODE_INT8_STEP && c->W != 1) return LQ_ERR_INVALID_ARG;
+        if (lq::decode_smem_bytes(c->dk, c->dv, layout_of(c)) > kMaxSmem) return LQ_ERR_UNSUPPORTED;
+    } else if (c->n_hp_rows != 0) {
+        return LQ_ERR_INVALID_ARG;
+    }
+    return LQ_OK;
+}
+
+size_t hp_bytes(const lq_config *c) { return align_sz((size_t)c->H * c->n_hp_rows * 4, kAlign); }
+
+size_t record_bytes(const lq_config *c) {
+    if (is_int8(c)) return (size_t)layout_of(c).rec_bytes;
+    return (size_t)c->dk * c->dv * 4;
+}
+
+int check_hp_rows(const lq_config *c, const int32_t *rows) {
+    if (c->n_hp_rows == 0) return LQ_OK;
+    if (!rows) return LQ_ERR_INVALID_ARG;
+    for (int h = 0; h < c->H; ++h) {
+        const int32_t *r = rows + (size_t)h * c->n_hp_rows;
+        for (int p = 0; p < c->n_hp_rows; ++p) {
+            if (r[p] < 0 || r[p] >= c->dk) return LQ_ERR_INVALID_ARG;
+            for (int q = 0; q < p; ++q)
+                if (r[q] == r[p]) return LQ_ERR_INVALID_ARG;
+        }
+    }
+    return LQ_OK;
+}
+
+lq::QPtrs record_ptrs(const lq_state *st) {
+    const Layout &L = st->L;
+    lq::QPtrs q{};
+    const size_t hs = (size_t)L.rec_bytes;
+    q.codes = st->rec; q.codes_hs = hs;
+    q.hp = st->rec + L.off_hp; q.hp_hs = hs;
+    q.m = st->rec + L.off_m; q.m_hs = hs;
+    q.s = st->rec + L.off_s; q.s_hs = hs;
+    q.ck = st->rec + L.off_ent; q.ck_hs = hs; q.ck_js = L.dk + L.dv;
+    q.cw = st->rec + L.off_ent + (size_t)L.dk * 4; q.cw_hs = hs; q.cw_js = L.dk + L.dv;
+    q.gam = st->rec + L.off_gam; q.gam_hs = hs; q.gam_n = L.kda ? L.dk : 1;
+    return q;
+}
+
+lq::QPtrs view_ptrs(const lq_config *c, const lq_qstate_view *v) {
+    lq::QPtrs q{};
+    const int dk = c->dk, dv = c->dv, P = c->n_hp_rows, r = c->r;
+    q.codes = reinterpret_cast<unsigned char *>(v->codes); q.codes_hs = (size_t)(dk - P) * dv;
+    q.hp = reinterpret_cast<unsigned char *>(v->bf16_rows); q.hp_hs = (size_t)P * dv * 2;
+    q.m = reinterpret_cast<unsigned char *>(v->m); q.m_hs = (size_t)dk * 4;
+    q.s = reinterpret_cast<unsigned char *>(v->s); q.s_hs = (size_t)dv * 4;
+    q.ck = reinterpret_cast<unsigned char *>(v->comp_k); q.ck_hs = (size_t)r * dk * 4; q.ck_js = dk;
+    q.cw = reinterpret_cast<unsigned char *>(v->comp_v); q.cw_hs = (size_t)r * dv * 4; q.cw_js = dv;
+    return q;
+}
+
+int check_view(const lq_config *c, const lq_qstate_view *v) {
+    if (!v || !v->codes || !v->m || !v->s) return LQ_ERR_INVALID_ARG;
+    if (c->n_hp_rows > 0 && !v->bf16_rows) return LQ_ERR_INVALID_ARG;
+    if (c->r > 0 && (!v->comp_k || !v->comp_v)) return LQ_ERR_INVALID_ARG;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(v->codes) | reinterpret_cast<uintptr_t>(v->m) |
+                        reinterpret_cast<uintptr_t>(v->s) | reinterpret_cast<uintptr_t>(v->bf16_rows);
+    if (a & 15) return LQ_ERR_INVALID_ARG;  // 16-byte vector access
+    return LQ_OK;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? LQ_OK : LQ_ERR_CUDA; }
+
+lq::DecodeArgs decode_args(const lq_state *st) {
+    lq::DecodeArgs a{};
+    a.L = st->L;
+    a.rec = st->rec;
+    a.B = st->cfg.B; a.H = st->cfg.H; a.Hk = st->cfg.Hk;
+    a.K = st->cfg.power_iters;
+    a.smoothing = st->cfg.smoothing;
+    a.n = st->n;
+    a.hp_rows = st->hp_rows;
+    a.status = st->status;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lq_config_check(const lq_config *cfg) { return check_config(cfg); }
+
+size_t lq_workspace_bytes(const lq_config *cfg) {
+    if (check_config(cfg) != LQ_OK) return 0;
+    return kAlign + hp_bytes(cfg) + (size_t)cfg->B * cfg->H * record_bytes(cfg);
+}
+
+int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_t bytes, const float *d_S0,
+                  const int32_t *h_hp_row_ids, void *stream) {
+    if (!out) return LQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!d_workspace || !d_S0) return LQ_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(d_workspace) % kAlign) return LQ_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(d_S0) % 16) return LQ_ERR_INVALID_ARG;
+    if (bytes < lq_workspace_bytes(cfg)) return LQ_ERR_WORKSPACE;
+    rc = check_hp_rows(cfg, h_hp_row_ids);
+    if (rc) return rc;
+    lq_state *st = new (std::nothrow) lq_state;
+    if (!st) return LQ_ERR_INVALID_ARG;
+    st->cfg = *cfg;
+    if (cfg->mode == LQ_MODE_INT8_STEP) st->cfg.W = 1;
+    st->L = layout_of(cfg);
+    st->ws = static_cast<unsigned char *>(d_workspace);
+    st->bytes = bytes;
+    st->status = reinterpret_cast<int *>(st->ws);
+    st->hp_rows = reinterpret_cast<int *>(st->ws + kAlign);
+    st->rec = st->ws + kAlign + hp_bytes(cfg);
+    st->heads = (size_t)cfg->B * cfg->H;
+    st->n = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(st->status, 0, sizeof(int), s);
+    if (e == cudaSuccess && cfg->n_hp_rows > 0)
+        e = cudaMemcpyAsync(st->hp_rows, h_hp_row_ids, (size_t)cfg->H * cfg->n_hp_rows * 4,
+                            cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) {
+        if (is_int8(cfg)) {
+            lq::CodecArgs a{};
+            a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing;
+            a.P = cfg->n_hp_rows; a.hp_rows = st->hp_rows; a.S_in = d_S0;
+            a.q = record_ptrs(st);
+            a.status = st->status;
+            e = lq::launch_quantize(a, cfg->dk, cfg->dv, (int)st->heads, s);
+        } else {
+            e = cudaMemcpyAsync(st->rec, d_S0, st->heads * record_bytes(cfg), cudaMemcpyDeviceToDevice, s);
+        }
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        delete st;
+        return LQ_ERR_CUDA;
+    }
+    *out = st;
+    return LQ_OK;
+}
+
+int lq_decode_step(lq_state *st, const float *d_q, const float *d_k, const float *d_v, const float *d_beta,
+                   const float *d_alpha, float *d_o, void *stream) {
+    if (!st || !d_q || !d_k || !d_v || !d_beta || !d_alpha || !d_o) return LQ_ERR_INVALID_ARG;
+    const lq_config &c = st->cfg;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool kda = c.gate == LQ_GATE_CHANNEL;
+    if (c.mode == LQ_MODE_FP32) {
+        lq::Fp32Args a{};
+        a.S = reinterpret_cast<float *>(st->rec);
+        a.B = c.B; a.H = c.H; a.Hk = c.Hk;
+        a.q = d_q; a.k = d_k; a.v = d_v; a.beta = d_beta; a.alpha = d_alpha; a.o = d_o;
+        a.status = st->status;
+        return cuda_rc(lq::launch_fp32_step(a, c.dk, c.dv, (int)st->heads, kda, s));
+    }
+    if (st->n >= st->L.W) return LQ_ERR_WINDOW_FULL;
+    const bool flush = (c.mode == LQ_MODE_INT8_STEP) || (c.fused_flush && st->n + 1 == st->L.W);
+    lq::DecodeArgs a = decode_args(st);
+    a.q = d_q; a.k = d_k; a.v = d_v; a.beta = d_beta; a.alpha = d_alpha; a.o = d_o;
+    const int rc = cuda_rc(lq::launch_decode(a, c.dk, c.dv, (int)st->heads, kda, flush, c.n_hp_rows > 0, s));
+    if (rc == LQ_OK) st->n = flush ? 0 : st->n + 1;
+    return rc;
+}
+
+int lq_window_flush(lq_state *st, void *stream) {
+    if (!st) return LQ_ERR_INVALID_ARG;
+    if (st->cfg.mode != LQ_MODE_INT8_WINDOW || st->n == 0) return LQ_OK;
+    lq::DecodeArgs a = decode_args(st);
+    const int rc = cuda_rc(lq::launch_flush(a, st->cfg.dk, st->cfg.dv, (int)st->heads,
+                                            st->cfg.gate == LQ_GATE_CHANNEL, st->cfg.n_hp_rows > 0, false,
+                                            static_cast<cudaStream_t>(stream)));
+    if (rc == LQ_OK) st->n = 0;
+    return rc;
+}
+
+int lq_state_buffered(const lq_state *st) { return st ? st->n : 0; }
+
+int lq_state_export_fp32(const lq_state *st, float *d_S, void *stream) {
+    if (!st || !d_S) return LQ_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(d_S) % 16) return LQ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (st->cfg.mode == LQ_MODE_FP32)
+        return cuda_rc(cudaMemcpyAsync(d_S, st->rec, st->heads * record_bytes(&st->cfg), cudaMemcpyDeviceToDevice, s));
+    lq::DecodeArgs a = decode_args(st);
+    a.S_out = d_S;
+    return cuda_rc(lq::launch_flush(a, st->cfg.dk, st->cfg.dv, (int)st->heads, st->cfg.gate == LQ_GATE_CHANNEL,
+                                    st->cfg.n_hp_rows > 0, true, s));
+}
+
+int lq_state_export_view(const lq_state *st, const lq_qstate_view *out, void *stream) {
+    if (!st) return LQ_ERR_INVALID_ARG;
+    if (!is_int8(&st->cfg)) return LQ_ERR_INVALID_ARG;
+    int rc = check_view(&st->cfg, out);
+    if (rc) return rc;
+    lq::CodecArgs a{};
+    a.H = st->cfg.H; a.r = st->cfg.r; a.P = st->cfg.n_hp_rows;
+    a.q = record_ptrs(st);
+    a.q.gam = nullptr;
+    a.q2 = view_ptrs(&st->cfg, out);
+    return cuda_rc(lq::launch_qcopy(a, st->cfg.dk, st->cfg.dv, (int)st->heads, static_cast<cudaStream_t>(stream)));
+}
+
+int lq_state_import_view(lq_state *st, const lq_qstate_view *in, void *stream) {
+    if (!st) return LQ_ERR_INVALID_ARG;
+    if (!is_int8(&st->cfg)) return LQ_ERR_INVALID_ARG;
+    int rc = check_view(&st->cfg, in);
+    if (rc) return rc;
+    lq::CodecArgs a{};
+    a.H = st->cfg.H; a.r = st->cfg.r; a.P = st->cfg.n_hp_rows;
+    a.q = view_ptrs(&st->cfg, in);
+    a.q2 = record_ptrs(st);
+    rc = cuda_rc(lq::launch_qcopy(a, st->cfg.dk, st->cfg.dv, (int)st->heads, static_cast<cudaStream_t>(stream)));
+    if (rc == LQ_OK) st->n = 0;
+    return rc;
+}
+
+static int codec_common(const lq_config *cfg, const int32_t *h_rows, lq::CodecArgs &a, int **d_rows,
+                        cudaStream_t s) {
+    if (!cfg) return LQ_ERR_INVALID_ARG;
+    if (cfg->B < 1 || cfg->H < 1) return LQ_ERR_SHAPE;
+    int rc = check_codec_fields(cfg);
+    if (rc) return rc;
+    rc = check_hp_rows(cfg, h_rows);
+    if (rc) return rc;
+    a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing; a.P = cfg->n_hp_rows;
+    *d_rows = nullptr;
+    if (cfg->n_hp_rows > 0) {
+        const size_t nb = (size_t)cfg->H * cfg->n_hp_rows * 4;
+        if (cudaMallocAsync(reinterpret_cast<void **>(d_rows), nb, s) != cudaSuccess) return LQ_ERR_CUDA;
+        if (cudaMemcpyAsync(*d_rows, h_rows, nb, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+            cudaFreeAsync(*d_rows, s);
+            return LQ_ERR_CUDA;
+        }
+        a.hp_rows = *d_rows;
+    }
+    return LQ_OK;
+}
+
+int lq_quantize_state(const lq_config *cfg, const float *d_S, const int32_t *h_hp_row_ids, lq_qstate_view *out,
+                      void *stream) {
+    if (!d_S || (reinterpret_cast<uintptr_t>(d_S) % 16)) return LQ_ERR_INVALID_ARG;
+    if (!cfg) return LQ_ERR_INVALID_ARG;
+    int rc = check_view(cfg, out);
+    if (rc) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    lq::CodecArgs a{};
+    int *d_rows = nullptr;
+    rc = codec_common(cfg, h_hp_row_ids, a, &d_rows, s);
+    if (rc) return rc;
+    a.S_in = d_S;
+    a.q = view_ptrs(cfg, out);
+    rc = cuda_rc(lq::launch_quantize(a, cfg->dk, cfg->dv, cfg->B * cfg->H, s));
+    if (d_rows) cudaFreeAsync(d_rows, s);
+    return rc;
+}
+
+int lq_dequantize_state(const lq_config *cfg, const lq_qstate_view *in, const int32_t *h_hp_row_ids, float *d_S,
+                        void *stream) {
+    if (!d_S || (reinterpret_cast<uintptr_t>(d_S) % 16)) return LQ_ERR_INVALID_ARG;
+    if (!cfg) return LQ_ERR_INVALID_ARG;
+    int rc = check_view(cfg, in);
+    if (rc) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    lq::CodecArgs a{};
+    int *d_rows = nullptr;
+    rc = codec_common(cfg, h_hp_row_ids, a, &d_rows, s);
+    if (rc) return rc;
+    a.S_out = d_S;
+    a.q = view_ptrs(cfg, in);
+    rc = cuda_rc(lq::launch_dequantize(a, cfg->dk, cfg->dv, cfg->B * cfg->H, s));
+    if (d_rows) cudaFreeAsync(d_rows, s);
+    return rc;
+}
+
+int lq_damp_select(const lq_config *cfg, int32_t n_states, const float *d_states, int32_t n_gate_samples,
+                   const float *d_gates, double *d_energy, int32_t *d_rows, void *stream) {
+    if (!cfg || !d_states || !d_gates || !d_energy || !d_rows) return LQ_ERR_INVALID_ARG;
+    if (n_states < 1 || n_gate_samples < 1) return LQ_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(d_states) % 16) return LQ_ERR_INVALID_ARG;
+    if (cfg->H < 1) return LQ_ERR_SHAPE;
+    if (cfg->gate != LQ_GATE_SCALAR && cfg->gate != LQ_GATE_CHANNEL) return LQ_ERR_INVALID_ARG;
+    int rc = check_codec_fields(cfg);
+    if (rc) return rc;
+    if (cfg->n_hp_rows < 1) return LQ_ERR_INVALID_ARG;
+    lq::CodecArgs a{};
+    a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing; a.P = cfg->n_hp_rows;
+    a.S_in = d_states;
+    a.n_states = n_states;
+    a.n_gate_samples = n_gate_samples;
+    a.gate_per_channel = cfg->gate == LQ_GATE_CHANNEL;
+    a.gates = d_gates;
+    a.energy = d_energy;
+    a.rows_out = d_rows;
+    return cuda_rc(lq::launch_damp_select(a, cfg->dk, cfg->dv, static_cast<cudaStream_t>(stream)));
+}
+
+int lq_get_status(lq_state *st, void *stream) {
+    if (!st) return LQ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int h = 0;
+    if (cudaMemcpyAsync(&h, st->status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return LQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LQ_ERR_CUDA;
+    if (h & lq::kStatusTimeout) return LQ_ERR_TIMEOUT;
+    if (h & lq::kStatusNonFinite) return LQ_ERR_NONFINITE;
+    return LQ_OK;
+}
+
+void lq_state_destroy(lq_state *st) { delete st; }
+
+const char *lq_strerror(int status) {
+    switch (status) {
+        case LQ_OK: return "ok";
+        case LQ_ERR_INVALID_ARG: return "invalid argument";
+        case LQ_ERR_SHAPE: return "inconsistent shape";
+        case LQ_ERR_WORKSPACE: return "workspace too small or misaligned";
+        case LQ_ERR_WINDOW_FULL: return "window full: flush before decoding another token";
+        case LQ_ERR_CUDA: return "CUDA runtime error";
+        case LQ_ERR_NONFINITE: return "non-finite value produced on the device";
+        case LQ_ERR_UNSUPPORTED: return "unsupported head size or configuration";
+        case LQ_ERR_TIMEOUT: return "a bounded device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,236 @@
+// lq_codec.cu -- stateless codec kernels: quantize an FP32 state (window-start
+// quantizer of the LeapQuant project page, with the DAMP BF16 rows),
+// dequantize it, copy a quantized state between the workspace record and plain
+// arrays, and the DAMP channel-risk selection.  One CTA of 256 threads per head.
+#include "lq_codec.cuh"
+#include "lq_kernels.h"
+
+namespace lq {
+
+template <int DK, int DV>
+struct QSmem {
+    CodecSmem<DK, DV> cs;
+    int map[DK];
+    int wscr[kWarps];
+};
+
+template <int DK, int DV>
+__device__ __forceinline__ void tile_load_global(float (&R)[Tile<DK, DV>::RPT][16], const float *src) {
+    using T = Tile<DK, DV>;
+    const int t = threadIdx.x, cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(src + (size_t)(row0 + r) * DV + cg * 16) + q);
+            R[r][4 * q] = f.x; R[r][4 * q + 1] = f.y; R[r][4 * q + 2] = f.z; R[r][4 * q + 3] = f.w;
+        }
+}
+
+template <int DK, int DV>
+__device__ __forceinline__ void tile_store_global(const float (&R)[Tile<DK, DV>::RPT][16], float *dst) {
+    using T = Tile<DK, DV>;
+    const int t = threadIdx.x, cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            reinterpret_cast<float4 *>(dst + (size_t)(row0 + r) * DV + cg * 16)[q] =
+                make_float4(R[r][4 * q], R[r][4 * q + 1], R[r][4 * q + 2], R[r][4 * q + 3]);
+}
+
+__device__ __forceinline__ CodecOut codec_out_of(const QPtrs &q, int head) {
+    CodecOut o;
+    o.codes = reinterpret_cast<int8_t *>(q.codes + (size_t)head * q.codes_hs);
+    o.hp = reinterpret_cast<uint16_t *>(q.hp ? q.hp + (size_t)head * q.hp_hs : nullptr);
+    o.m = reinterpret_cast<float *>(q.m + (size_t)head * q.m_hs);
+    o.s = reinterpret_cast<float *>(q.s + (size_t)head * q.s_hs);
+    o.ck = reinterpret_cast<float *>(q.ck ? q.ck + (size_t)head * q.ck_hs : nullptr);
+    o.ck_stride = q.ck_js;
+    o.cw = reinterpret_cast<float *>(q.cw ? q.cw + (size_t)head * q.cw_hs : nullptr);
+    o.cw_stride = q.cw_js;
+    return o;
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const CodecArgs a) {
+    __shared__ QSmem<DK, DV> sm;
+    using T = Tile<DK, DV>;
+    const int head = blockIdx.x, h = head % a.H;
+    if (a.P > 0) build_row_map<DK>(a.hp_rows + (size_t)h * a.P, a.P, sm.map, sm.wscr);
+    float R[T::RPT][16];
+    tile_load_global<DK, DV>(R, a.S_in + (size_t)head * DK * DV);
+    const CodecOut out = codec_out_of(a.q, head);
+    double eacc[T::RPT];
+    codec_quantize<DK, DV, false>(R, a.r, a.K, a.smoothing, a.P, a.P > 0 ? sm.map : nullptr, sm.cs, out, eacc);
+    if (a.q.gam) {
+        float *g = reinterpret_cast<float *>(a.q.gam + (size_t)head * a.q.gam_hs);
+        for (int i = threadIdx.x; i < a.q.gam_n; i += kThreads) g[i] = 1.0f;
+    }
+}
+
+// S = Deq(C, m, s) [BF16 rows widened] + sum_j c_j w_j^T.
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads) dequantize_kernel(const CodecArgs a) {
+    __shared__ QSmem<DK, DV> sm;
+    using T = Tile<DK, DV>;
+    const int head = blockIdx.x, h = head % a.H;
+    const int t = threadIdx.x, cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
+    if (a.P > 0) build_row_map<DK>(a.hp_rows + (size_t)h * a.P, a.P, sm.map, sm.wscr);
+    const QPtrs &q = a.q;
+    const int8_t *codes = reinterpret_cast<const int8_t *>(q.codes + (size_t)head * q.codes_hs);
+    const uint16_t *hp = q.hp ? reinterpret_cast<const uint16_t *>(q.hp + (size_t)head * q.hp_hs) : nullptr;
+    const float *m = reinterpret_cast<const float *>(q.m + (size_t)head * q.m_hs);
+    const float *s = reinterpret_cast<const float *>(q.s + (size_t)head * q.s_hs);
+    float R[T::RPT][16];
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r) {
+        const int i = row0 + r;
+        const int mp = a.P > 0 ? sm.map[i] : i;
+        if (mp >= 0) {
+            const float mi = m[i];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const int col = cg * 16 + c;
+                R[r][c] = ((float)codes[(size_t)mp * DV + col] * s[col]) * mi;
+            }
+        } else {
+            const int p = -1 - mp;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) R[r][c] = bf16_to_f(hp[(size_t)p * DV + cg * 16 + c]);
+        }
+    }
+    for (int j = 0; j < a.r; ++j) {
+        const float *ck = reinterpret_cast<const float *>(q.ck + (size_t)head * q.ck_hs) + (size_t)j * q.ck_js;
+        const float *cw = reinterpret_cast<const float *>(q.cw + (size_t)head * q.cw_hs) + (size_t)j * q.cw_js;
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const float c = ck[row0 + r];
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) R[r][cc] = fmaf(c, cw[cg * 16 + cc], R[r][cc]);
+        }
+    }
+    tile_store_global<DK, DV>(R, a.S_out + (size_t)head * DK * DV);
+}
+
+// Copy a quantized state from q to q2 (same head numbering), setting q2's
+// Gamma to 1 when it has one.
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads) qcopy_kernel(const CodecArgs a) {
+    const int head = blockIdx.x, t = threadIdx.x;
+    const QPtrs &x = a.q, &y = a.q2;
+    const int P = a.P;
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x.codes + (size_t)head * x.codes_hs);
+        uint4 *dst = reinterpret_cast<uint4 *>(y.codes + (size_t)head * y.codes_hs);
+        const int n16 = (DK - P) * DV / 16;
+        for (int e = t; e < n16; e += kThreads) dst[e] = src[e];
+    }
+    if (P > 0) {
+        const uint16_t *src = reinterpret_cast<const uint16_t *>(x.hp + (size_t)head * x.hp_hs);
+        uint16_t *dst = reinterpret_cast<uint16_t *>(y.hp + (size_t)head * y.hp_hs);
+        for (int e = t; e < P * DV; e += kThreads) dst[e] = src[e];
+    }
+    {
+        const float *src = reinterpret_cast<const float *>(x.m + (size_t)head * x.m_hs);
+        float *dst = reinterpret_cast<float *>(y.m + (size_t)head * y.m_hs);
+        for (int e = t; e < DK; e += kThreads) dst[e] = src[e];
+        src = reinterpret_cast<const float *>(x.s + (size_t)head * x.s_hs);
+        dst = reinterpret_cast<float *>(y.s + (size_t)head * y.s_hs);
+        for (int e = t; e < DV; e += kThreads) dst[e] = src[e];
+    }
+    for (int j = 0; j < a.r; ++j) {
+        const float *sk = reinterpret_cast<const float *>(x.ck + (size_t)head * x.ck_hs) + (size_t)j * x.ck_js;
+        float *dk_ = reinterpret_cast<float *>(y.ck + (size_t)head * y.ck_hs) + (size_t)j * y.ck_js;
+        for (int e = t; e < DK; e += kThreads) dk_[e] = sk[e];
+        const float *sw = reinterpret_cast<const float *>(x.cw + (size_t)head * x.cw_hs) + (size_t)j * x.cw_js;
+        float *dw = reinterpret_cast<float *>(y.cw + (size_t)head * y.cw_hs) + (size_t)j * y.cw_js;
+        for (int e = t; e < DV; e += kThreads) dw[e] = sw[e];
+    }
+    if (y.gam) {
+        float *g = reinterpret_cast<float *>(y.gam + (size_t)head * y.gam_hs);
+        for (int i = t; i < y.gam_n; i += kThreads) g[i] = 1.0f;
+    }
+}
+
+// DAMP channel risk: per head, sum over the calibration states of the per-row
+// INT8 error energy, times the row's persistence 1 / (1 - mean decay); keep the
+// top P rows (ties to the lower index), listed in increasing order.
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads) damp_select_kernel(const CodecArgs a) {
+    __shared__ CodecSmem<DK, DV> cs;
+    __shared__ double score[DK];
+    __shared__ int sel[DK];
+    using T = Tile<DK, DV>;
+    const int h = blockIdx.x, t = threadIdx.x;
+    const int cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
+    double eacc[T::RPT];
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r) eacc[r] = 0.0;
+    CodecOut none{};
+    for (int n = 0; n < a.n_states; ++n) {
+        float R[T::RPT][16];
+        tile_load_global<DK, DV>(R, a.S_in + ((size_t)n * a.H + h) * DK * DV);
+        codec_quantize<DK, DV, true>(R, a.r, a.K, a.smoothing, 0, nullptr, cs, none, eacc);
+    }
+    if (cg == 0) {
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) score[row0 + r] = eacc[r];
+    }
+    __syncthreads();
+    if (t < DK) {
+        const double E = score[t];
+        a.energy[(size_t)h * DK + t] = E;
+        double mean = 0.0;
+        const int ga = a.gate_per_channel ? DK : 1;
+        const int col = a.gate_per_channel ? t : 0;
+        for (int sidx = 0; sidx < a.n_gate_samples; ++sidx)
+            mean += (double)a.gates[((size_t)sidx * a.H + h) * ga + col];
+        mean /= (double)a.n_gate_samples;
+        score[t] = E * (1.0 / (1.0 - mean));
+    }
+    __syncthreads();
+    if (t < DK) {
+        const double mine = score[t];
+        int rank = 0;
+        for (int j = 0; j < DK; ++j) {
+            const double o = score[j];
+            rank += (o > mine) || (o == mine && j < t);
+        }
+        sel[t] = rank < a.P;
+    }
+    __syncthreads();
+    if (t < DK && sel[t]) {
+        int pos = 0;
+        for (int j = 0; j < t; ++j) pos += sel[j];
+        a.rows_out[(size_t)h * a.P + pos] = t;
+    }
+}
+
+#define LQ_PICK(dk, dv, KERN)                          \
+    (((dk) == 128 && (dv) == 128)  ? KERN<128, 128>    \
+     : ((dk) == 64 && (dv) == 64)  ? KERN<64, 64>      \
+     : ((dk) == 64 && (dv) == 128) ? KERN<64, 128>     \
+                                   : KERN<128, 64>)
+
+cudaError_t launch_quantize(const CodecArgs &a, int dk, int dv, int heads, cudaStream_t s) {
+    LQ_PICK(dk, dv, quantize_kernel)<<<heads, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const CodecArgs &a, int dk, int dv, int heads, cudaStream_t s) {
+    LQ_PICK(dk, dv, dequantize_kernel)<<<heads, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_qcopy(const CodecArgs &a, int dk, int dv, int heads, cudaStream_t s) {
+    LQ_PICK(dk, dv, qcopy_kernel)<<<heads, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_damp_select(const CodecArgs &a, int dk, int dv, cudaStream_t s) {
+    LQ_PICK(dk, dv, damp_select_kernel)<<<a.H, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace lq

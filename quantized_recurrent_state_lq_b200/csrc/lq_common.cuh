@@ -1,0 +1,197 @@
+// lq_common.cuh -- device helpers shared by the decode, flush and codec kernels:
+// the per-head record layout, bulk-copy (TMA, non-tensor) staging with a
+// bounded mbarrier wait, warp/block reductions and BF16 rounding.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lq {
+
+constexpr int kThreads = 256;  // every kernel here runs 8 warps per CTA
+constexpr int kWarps = kThreads / 32;
+
+// Sticky device status bits (reported by lq_get_status).
+constexpr int kStatusNonFinite = 1;
+constexpr int kStatusTimeout = 2;
+
+// ---------------------------------------------------------------------------
+// Per-head record in the workspace (INT8 modes).  One contiguous, 128-byte
+// aligned slab per (batch, head), so that a decode step stages everything it
+// reads for a head -- codes, BF16 rows, m, s, compensators and the buffered
+// tokens -- with ONE bulk copy of the slab's prefix:
+//   codes   int8  [dk-P][dv]        INT8 rows in increasing key-row order
+//   hp      u16   [P][dv]           BF16 rows (order of the head's row list)
+//   m       f32   [dk]              smoothing scale per key row (1 on BF16 rows)
+//   s       f32   [dv]              quantization scale per value column
+//   ent     f32   [r+W][dk+dv]      entry e = (key side [dk], value side [dv]);
+//                                   e < r: compensator (c_e, w_e);
+//                                   r <= e < r+n: buffered token (k/Gamma, u)
+//   gam     f32   [dk] (KDA) / [4] (GDN)   cumulative decay since window start
+// ---------------------------------------------------------------------------
+struct Layout {
+    int dk, dv, P, r, W, kda;
+    int off_hp, off_m, off_s, off_ent, off_gam;
+    int rec_bytes;
+};
+
+__host__ __device__ inline int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+__host__ inline Layout make_layout(int dk, int dv, int P, int r, int W, int kda) {
+    Layout L;
+    L.dk = dk; L.dv = dv; L.P = P; L.r = r; L.W = W; L.kda = kda;
+    int o = align_up((dk - P) * dv, 16);
+    L.off_hp = o;
+    o = align_up(o + P * dv * 2, 16);
+    L.off_m = o;
+    o += dk * 4;
+    L.off_s = o;
+    o += dv * 4;
+    L.off_ent = align_up(o, 16);
+    o = L.off_ent + (r + W) * (dk + dv) * 4;
+    L.off_gam = align_up(o, 16);
+    o = L.off_gam + (kda ? dk : 4) * 4;
+    L.rec_bytes = align_up(o, 128);
+    return L;
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers: mbarrier + cp.async.bulk (global -> shared, no multicast).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of `bar` for at most ~limit_ns.  On a timeout, raise
+// the status bit, then keep waiting (again bounded) so that the copy in flight
+// lands before the caller's shared memory is released, and report failure.
+__device__ inline bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int *status,
+                                         uint64_t limit_ns = 1000000000ull) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > limit_ns) {
+            if (status) atomicOr(status, kStatusTimeout);
+            uint64_t t1 = global_ns();
+            while (!mbar_try_wait(bar, parity)) {
+                if (global_ns() - t1 > 4 * limit_ns) break;
+            }
+            return false;
+        }
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// Reductions.
+// ---------------------------------------------------------------------------
+template <int WIDTH>
+__device__ __forceinline__ float shfl_xor_sum(float v) {
+#pragma unroll
+    for (int m = WIDTH / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) { return shfl_xor_sum<32>(v); }
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+    return v;
+}
+
+// Sum of one double per thread over the CTA; every thread gets the result.
+// `scratch` holds kWarps doubles; the call begins and ends with a barrier.
+__device__ inline double block_sum_d(double v, double *scratch) {
+    v = warp_sum_d(v);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
+    __syncthreads();
+    double s = 0.0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) s += scratch[w];
+    return s;
+}
+
+// ---------------------------------------------------------------------------
+// BF16 round-to-nearest-even from float bits, and back.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint16_t bf16_rne(float x) {
+    uint32_t u = __float_as_uint(x);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) return (uint16_t)((u >> 16) | 0x0040u);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+__device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+// Signed bytes of a 32-bit word -> floats (exact).
+__device__ __forceinline__ void s8x4_to_f(uint32_t w, float f[4]) {
+    f[0] = (float)(int8_t)(w & 0xff);
+    f[1] = (float)(int8_t)((w >> 8) & 0xff);
+    f[2] = (float)(int8_t)((w >> 16) & 0xff);
+    f[3] = (float)(int8_t)(w >> 24);
+}
+
+// Build the key-row map of one head in shared memory: map[i] = INT8 slot of
+// row i (rows in increasing order, BF16 rows skipped) or -1-p for the p-th
+// BF16 row.  Needs DK <= kThreads.  Ends with a barrier.
+template <int DK>
+__device__ inline void build_row_map(const int *hp_rows_h, int P, int *map, int *scratch_w) {
+    const int i = threadIdx.x;
+    int p_of = -1;
+    if (i < DK) {
+        for (int p = 0; p < P; ++p)
+            if (hp_rows_h[p] == i) p_of = p;
+    }
+    const bool hp = (i < DK) && (p_of >= 0);
+    const uint32_t bal = __ballot_sync(0xffffffffu, hp);
+    const int lane = i & 31, warp = i >> 5;
+    if (lane == 0) scratch_w[warp] = __popc(bal);
+    __syncthreads();
+    int before = __popc(bal & ((1u << lane) - 1u));
+    for (int w = 0; w < warp; ++w) before += scratch_w[w];
+    if (i < DK) map[i] = hp ? (-1 - p_of) : (i - before);
+    __syncthreads();
+}
+
+}  // namespace lq

@@ -1,0 +1,297 @@
+"""Thin Python binding of liblq.so (include/lq_state.h), same names as the C ABI.
+
+Argument marshalling only: torch tensors are checked for device, dtype, shape
+and contiguity and passed as raw device pointers together with torch's current
+CUDA stream.  Every computation happens in the CUDA library; if liblq.so is
+missing this module raises on import of the library instead of falling back.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblq.so")
+
+LQ_OK = 0
+LQ_ERR_INVALID_ARG = -1
+LQ_ERR_SHAPE = -2
+LQ_ERR_WORKSPACE = -3
+LQ_ERR_WINDOW_FULL = -4
+LQ_ERR_CUDA = -5
+LQ_ERR_NONFINITE = -6
+LQ_ERR_UNSUPPORTED = -7
+LQ_ERR_TIMEOUT = -8
+
+LQ_GATE_SCALAR, LQ_GATE_CHANNEL = 0, 1
+LQ_MODE_FP32, LQ_MODE_INT8_STEP, LQ_MODE_INT8_WINDOW = 0, 1, 2
+
+EXPORTED = ["lq_workspace_bytes", "lq_config_check", "lq_state_init", "lq_decode_step",
+            "lq_window_flush", "lq_state_buffered", "lq_state_export_fp32",
+            "lq_state_export_view", "lq_state_import_view", "lq_quantize_state",
+            "lq_dequantize_state", "lq_damp_select", "lq_get_status", "lq_state_destroy",
+            "lq_strerror"]
+
+
+class LqError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)} ({code})")
+
+
+class lq_config(C.Structure):
+    _fields_ = [(n, C.c_int32) for n in ("B", "H", "Hk", "dk", "dv", "gate", "mode", "W", "r",
+                                          "power_iters", "n_hp_rows", "smoothing", "fused_flush")]
+
+
+class lq_qstate_view(C.Structure):
+    _fields_ = [("codes", C.c_void_p), ("bf16_rows", C.c_void_p), ("m", C.c_void_p),
+                ("s", C.c_void_p), ("comp_k", C.c_void_p), ("comp_v", C.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Load liblq.so (building it in-tree first if it is missing or stale)."""
+    global _lib
+    if _lib is None:
+        from . import build as _build
+        if not os.path.exists(LIB_PATH) or _build._stale():
+            _build.build()
+        L = C.CDLL(LIB_PATH)
+        vp, i32, sz = C.c_void_p, C.c_int32, C.c_size_t
+        cfgp = C.POINTER(lq_config)
+        viewp = C.POINTER(lq_qstate_view)
+        sig = {
+            "lq_workspace_bytes": (sz, [cfgp]),
+            "lq_config_check": (C.c_int, [cfgp]),
+            "lq_state_init": (C.c_int, [C.POINTER(vp), cfgp, vp, sz, vp, vp, vp]),
+            "lq_decode_step": (C.c_int, [vp, vp, vp, vp, vp, vp, vp, vp]),
+            "lq_window_flush": (C.c_int, [vp, vp]),
+            "lq_state_buffered": (C.c_int, [vp]),
+            "lq_state_export_fp32": (C.c_int, [vp, vp, vp]),
+            "lq_state_export_view": (C.c_int, [vp, viewp, vp]),
+            "lq_state_import_view": (C.c_int, [vp, viewp, vp]),
+            "lq_quantize_state": (C.c_int, [cfgp, vp, vp, viewp, vp]),
+            "lq_dequantize_state": (C.c_int, [cfgp, viewp, vp, vp, vp]),
+            "lq_damp_select": (C.c_int, [cfgp, i32, vp, i32, vp, vp, vp, vp]),
+            "lq_get_status": (C.c_int, [vp, vp]),
+            "lq_state_destroy": (None, [vp]),
+            "lq_strerror": (C.c_char_p, [C.c_int]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().lq_strerror(code).decode()
+
+
+def _chk(rc: int, what: str):
+    if rc != LQ_OK:
+        raise LqError(rc, what)
+
+
+@dataclass
+class Config:
+    B: int
+    H: int
+    Hk: int
+    dk: int
+    dv: int
+    gate: str = "gdn"            # "gdn" | "kda"
+    mode: str = "window"         # "fp32" | "step" | "window"
+    W: int = 32
+    r: int = 4
+    power_iters: int = 8
+    n_hp_rows: int = 0
+    smoothing: int = 1
+    fused_flush: int = 1
+
+    def c(self) -> lq_config:
+        gate = {"gdn": LQ_GATE_SCALAR, "kda": LQ_GATE_CHANNEL}[self.gate]
+        mode = {"fp32": LQ_MODE_FP32, "step": LQ_MODE_INT8_STEP, "window": LQ_MODE_INT8_WINDOW}[self.mode]
+        return lq_config(self.B, self.H, self.Hk, self.dk, self.dv, gate, mode, self.W, self.r,
+                         self.power_iters, self.n_hp_rows, self.smoothing, self.fused_flush)
+
+    @property
+    def heads(self) -> int:
+        return self.B * self.H
+
+    @property
+    def ga(self) -> int:
+        return self.dk if self.gate == "kda" else 1
+
+    @staticmethod
+    def from_workload(wl, mode: str = "window", **kw) -> "Config":
+        base = dict(B=wl.B, H=wl.H, Hk=wl.Hk, dk=wl.dk, dv=wl.dv, gate=wl.gate, mode=mode,
+                    W=(1 if mode == "step" else wl.W), r=wl.r, power_iters=wl.K,
+                    n_hp_rows=(wl.P if mode != "fp32" else 0), smoothing=wl.smoothing)
+        base.update(kw)
+        return Config(**base)
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str, shape=None, dtype=torch.float32) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t.data_ptr()
+
+
+def _host_rows(cfg: Config, hp_rows):
+    if cfg.n_hp_rows == 0:
+        return None, None
+    arr = torch.as_tensor(hp_rows, dtype=torch.int32).cpu().contiguous()
+    if tuple(arr.shape) != (cfg.H, cfg.n_hp_rows):
+        raise ValueError(f"hp_rows must be [H, P] = {(cfg.H, cfg.n_hp_rows)}")
+    return arr, C.c_void_p(arr.data_ptr())
+
+
+def view_shapes(cfg: Config) -> dict:
+    B, H, dk, dv, P, r = cfg.B, cfg.H, cfg.dk, cfg.dv, cfg.n_hp_rows, cfg.r
+    return {"codes": ((B, H, dk - P, dv), torch.int8), "bf16_rows": ((B, H, P, dv), torch.int16),
+            "m": ((B, H, dk), torch.float32), "s": ((B, H, dv), torch.float32),
+            "comp_k": ((B, H, r, dk), torch.float32), "comp_v": ((B, H, r, dv), torch.float32)}
+
+
+def alloc_view(cfg: Config, device="cuda") -> dict:
+    return {k: torch.zeros(shape, dtype=dt, device=device) for k, (shape, dt) in view_shapes(cfg).items()}
+
+
+def _view_struct(cfg: Config, view: dict) -> lq_qstate_view:
+    ptr = {}
+    for k, (shape, dt) in view_shapes(cfg).items():
+        t = view[k]
+        ptr[k] = _dev(t, k, shape, dt) if t.numel() else None
+    return lq_qstate_view(ptr["codes"], ptr["bf16_rows"], ptr["m"], ptr["s"], ptr["comp_k"], ptr["comp_v"])
+
+
+def lq_config_check(cfg: Config) -> int:
+    return lib().lq_config_check(C.byref(cfg.c()))
+
+
+def lq_workspace_bytes(cfg: Config) -> int:
+    return lib().lq_workspace_bytes(C.byref(cfg.c()))
+
+
+class LqState:
+    """Owns the opaque handle and keeps the workspace tensor alive."""
+
+    def __init__(self, cfg: Config, handle: int, workspace: torch.Tensor, rows):
+        self.cfg = cfg
+        self.handle = C.c_void_p(handle)
+        self.workspace = workspace
+        self._rows = rows
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.lq_state_destroy(h)
+            self.handle = C.c_void_p(0)
+
+
+def lq_state_init(cfg: Config, S0: torch.Tensor, hp_rows=None, workspace: torch.Tensor | None = None,
+                  stream=None) -> LqState:
+    nbytes = lq_workspace_bytes(cfg)
+    if nbytes == 0:
+        _chk(lq_config_check(cfg), "lq_config_check")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=S0.device)
+    p_s0 = _dev(S0, "S0", (cfg.B, cfg.H, cfg.dk, cfg.dv))
+    rows, p_rows = _host_rows(cfg, hp_rows)
+    h = C.c_void_p()
+    _chk(lib().lq_state_init(C.byref(h), C.byref(cfg.c()), C.c_void_p(workspace.data_ptr()),
+                             workspace.numel() * workspace.element_size(), C.c_void_p(p_s0), p_rows,
+                             C.c_void_p(_stream(stream))), "lq_state_init")
+    return LqState(cfg, h.value, workspace, rows)
+
+
+def lq_decode_step(st: LqState, q, k, v, beta, alpha, o, stream=None):
+    c = st.cfg
+    args = [_dev(q, "q", (c.B, c.Hk, c.dk)), _dev(k, "k", (c.B, c.Hk, c.dk)),
+            _dev(v, "v", (c.B, c.H, c.dv)), _dev(beta, "beta", (c.B, c.H)),
+            _dev(alpha, "alpha", (c.B, c.H) if c.gate == "gdn" else (c.B, c.H, c.dk)),
+            _dev(o, "o", (c.B, c.H, c.dv))]
+    _chk(lib().lq_decode_step(st.handle, *[C.c_void_p(a) for a in args], C.c_void_p(_stream(stream))),
+         "lq_decode_step")
+
+
+def lq_window_flush(st: LqState, stream=None):
+    _chk(lib().lq_window_flush(st.handle, C.c_void_p(_stream(stream))), "lq_window_flush")
+
+
+def lq_state_buffered(st: LqState) -> int:
+    return lib().lq_state_buffered(st.handle)
+
+
+def lq_state_export_fp32(st: LqState, S: torch.Tensor, stream=None):
+    c = st.cfg
+    _chk(lib().lq_state_export_fp32(st.handle, C.c_void_p(_dev(S, "S", (c.B, c.H, c.dk, c.dv))),
+                                    C.c_void_p(_stream(stream))), "lq_state_export_fp32")
+
+
+def lq_state_export_view(st: LqState, view: dict, stream=None):
+    v = _view_struct(st.cfg, view)
+    _chk(lib().lq_state_export_view(st.handle, C.byref(v), C.c_void_p(_stream(stream))), "lq_state_export_view")
+
+
+def lq_state_import_view(st: LqState, view: dict, stream=None):
+    v = _view_struct(st.cfg, view)
+    _chk(lib().lq_state_import_view(st.handle, C.byref(v), C.c_void_p(_stream(stream))), "lq_state_import_view")
+
+
+def lq_quantize_state(cfg: Config, S: torch.Tensor, view: dict, hp_rows=None, stream=None):
+    p = _dev(S, "S", (cfg.B, cfg.H, cfg.dk, cfg.dv))
+    rows, p_rows = _host_rows(cfg, hp_rows)
+    v = _view_struct(cfg, view)
+    _chk(lib().lq_quantize_state(C.byref(cfg.c()), C.c_void_p(p), p_rows, C.byref(v),
+                                 C.c_void_p(_stream(stream))), "lq_quantize_state")
+
+
+def lq_dequantize_state(cfg: Config, view: dict, S: torch.Tensor, hp_rows=None, stream=None):
+    p = _dev(S, "S", (cfg.B, cfg.H, cfg.dk, cfg.dv))
+    rows, p_rows = _host_rows(cfg, hp_rows)
+    v = _view_struct(cfg, view)
+    _chk(lib().lq_dequantize_state(C.byref(cfg.c()), C.byref(v), p_rows, C.c_void_p(p),
+                                   C.c_void_p(_stream(stream))), "lq_dequantize_state")
+
+
+def lq_damp_select(cfg: Config, states: torch.Tensor, gates: torch.Tensor, energy: torch.Tensor,
+                   rows: torch.Tensor, stream=None):
+    n = states.shape[0]
+    ps = _dev(states, "states", (n, cfg.H, cfg.dk, cfg.dv))
+    ng = gates.shape[0]
+    pg = _dev(gates, "gates", (ng, cfg.H, cfg.ga))
+    pe = _dev(energy, "energy", (cfg.H, cfg.dk), torch.float64)
+    pr = _dev(rows, "rows", (cfg.H, cfg.n_hp_rows), torch.int32)
+    _chk(lib().lq_damp_select(C.byref(cfg.c()), n, C.c_void_p(ps), ng, C.c_void_p(pg), C.c_void_p(pe),
+                              C.c_void_p(pr), C.c_void_p(_stream(stream))), "lq_damp_select")
+
+
+def lq_get_status(st: LqState, stream=None) -> int:
+    return lib().lq_get_status(st.handle, C.c_void_p(_stream(stream)))
+
+
+def lq_state_destroy(st: LqState):
+    if st.handle.value:
+        lib().lq_state_destroy(st.handle)
+        st.handle = C.c_void_p(0)

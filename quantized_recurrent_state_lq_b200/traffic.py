@@ -1,0 +1,62 @@
+"""Algorithmic HBM bytes of the decode path -- what the method must move, not
+what a kernel happens to move -- used for the roofline figures.
+
+Per head and token of a window (n tokens already buffered, 0 <= n < W):
+  IO      q, k read once per q/k head (shared by H/Hk value heads), v and o,
+          beta, the gate (1 or dk floats)
+  state   INT8 codes (dk-P)*dv, BF16 rows 2*P*dv, m and s (dk+dv)*4,
+          r compensators r*(dk+dv)*4, the n buffered entries n*(dk+dv)*4
+  append  one entry (dk+dv)*4 and Gamma written (read too when n > 0)
+At the window end the new state is written once: codes, BF16 rows, m, s and
+the compensators.
+"""
+from __future__ import annotations
+
+from .configs import Workload
+
+
+def io_bytes(wl: Workload) -> float:
+    G = wl.H // wl.Hk
+    gate = wl.dk if wl.gate == "kda" else 1
+    return 2 * wl.dk * 4 / G + 2 * wl.dv * 4 + 4 + gate * 4
+
+
+def state_bytes(wl: Workload, P: int | None = None) -> int:
+    P = wl.P if P is None else P
+    return (wl.dk - P) * wl.dv + 2 * P * wl.dv + 4 * (wl.dk + wl.dv) + 4 * wl.r * (wl.dk + wl.dv)
+
+
+def gamma_bytes(wl: Workload, n: int) -> int:
+    g = wl.dk if wl.gate == "kda" else 1
+    return 4 * g * (2 if n > 0 else 1)
+
+
+def decode_launch_bytes(wl: Workload, n: int, flush: bool = False) -> float:
+    """Bytes per head of the decode launch that buffers token n+1 of a window."""
+    e = 4 * (wl.dk + wl.dv)
+    b = io_bytes(wl) + state_bytes(wl) + n * e
+    if flush:
+        b += state_bytes(wl)           # the new window-start state is written once
+    else:
+        b += e + gamma_bytes(wl, n)    # append the entry, keep Gamma
+    return b
+
+
+def window_bytes(wl: Workload) -> float:
+    """Bytes per head for one whole window (W decode tokens, the last one flushing)."""
+    return sum(decode_launch_bytes(wl, n, flush=(n == wl.W - 1)) for n in range(wl.W))
+
+
+def nonflush_launch_bytes(wl: Workload) -> float:
+    """Mean bytes per head of the W-1 launches that only buffer (n = 0 .. W-2)."""
+    if wl.W < 2:
+        return 0.0
+    return sum(decode_launch_bytes(wl, n) for n in range(wl.W - 1)) / (wl.W - 1)
+
+
+def fp32_step_bytes(wl: Workload) -> float:
+    return io_bytes(wl) + 8 * wl.dk * wl.dv
+
+
+def step_int8_bytes(wl: Workload) -> float:
+    return io_bytes(wl) + 2 * state_bytes(wl)

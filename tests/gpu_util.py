@@ -1,0 +1,125 @@
+"""Helpers for the GPU parity tests: run the CUDA path through the C ABI and the
+oracle on the same seeded inputs, map between the two layouts, compare.
+
+Directions of data flow: inputs come from the seeded generator (or from the
+oracle, e.g. an oracle window-start state imported into the GPU state to
+teacher-force a window); nothing computed by the CUDA path is ever fed to the
+oracle."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from quantized_recurrent_state_lq_b200 import configs, inputs as gen, lq
+
+f32 = np.float32
+
+
+def require_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def ocfg(cfg: lq.Config, quantize: int = 1) -> O.Cfg:
+    return O.Cfg(dk=cfg.dk, dv=cfg.dv, gate=cfg.gate, W=cfg.W, r=cfg.r, K=cfg.power_iters,
+                 smoothing=cfg.smoothing, P=cfg.n_hp_rows, quantize=quantize)
+
+
+def head_rows(cfg: lq.Config, hp_rows):
+    """[H, P] row lists -> per (b, h) head [B*H, P] for the oracle."""
+    if cfg.n_hp_rows == 0:
+        return None
+    hr = np.asarray(hp_rows, np.int32)
+    return np.ascontiguousarray(np.tile(hr, (cfg.B, 1)))
+
+
+def gpu_view_to_oracle(cfg: lq.Config, view: dict, hp_rows) -> dict:
+    """GPU view (compact INT8 rows) -> oracle view (full [dk, dv] codes, zero on BF16 rows)."""
+    B, H, dk, dv, P = cfg.B, cfg.H, cfg.dk, cfg.dv, cfg.n_hp_rows
+    nh = B * H
+    codes_c = view["codes"].cpu().numpy().reshape(nh, dk - P, dv)
+    codes = np.zeros((nh, dk, dv), np.int8)
+    for b in range(B):
+        for h in range(H):
+            keep = np.setdiff1d(np.arange(dk), np.asarray(hp_rows[h])) if P else np.arange(dk)
+            codes[b * H + h, keep] = codes_c[b * H + h]
+    out = {"codes": codes,
+           "m": view["m"].cpu().numpy().reshape(nh, dk).copy(),
+           "s": view["s"].cpu().numpy().reshape(nh, dv).copy(),
+           "c": view["comp_k"].cpu().numpy().reshape(nh, cfg.r, dk).copy(),
+           "w": view["comp_v"].cpu().numpy().reshape(nh, cfg.r, dv).copy(),
+           "hp": np.zeros((nh, max(P, 1), dv), np.uint16)}
+    if P:
+        out["hp"] = view["bf16_rows"].cpu().numpy().view(np.uint16).reshape(nh, P, dv).copy()
+    return out
+
+
+def oracle_view_to_gpu(cfg: lq.Config, ov: dict, hp_rows, device="cuda") -> dict:
+    B, H, dk, dv, P = cfg.B, cfg.H, cfg.dk, cfg.dv, cfg.n_hp_rows
+    nh = B * H
+    codes = np.zeros((nh, dk - P, dv), np.int8)
+    for b in range(B):
+        for h in range(H):
+            keep = np.setdiff1d(np.arange(dk), np.asarray(hp_rows[h])) if P else np.arange(dk)
+            codes[b * H + h] = ov["codes"][b * H + h][keep]
+    v = lq.alloc_view(cfg, device)
+    v["codes"].copy_(torch.from_numpy(codes.reshape(B, H, dk - P, dv)))
+    v["m"].copy_(torch.from_numpy(np.asarray(ov["m"], f32).reshape(B, H, dk)))
+    v["s"].copy_(torch.from_numpy(np.asarray(ov["s"], f32).reshape(B, H, dv)))
+    if cfg.r:
+        v["comp_k"].copy_(torch.from_numpy(np.asarray(ov["c"], f32).reshape(B, H, cfg.r, dk)))
+        v["comp_v"].copy_(torch.from_numpy(np.asarray(ov["w"], f32).reshape(B, H, cfg.r, dv)))
+    if P:
+        hp = np.asarray(ov["hp"], np.uint16)[:, :P].reshape(B, H, P, dv).view(np.int16)
+        v["bf16_rows"].copy_(torch.from_numpy(hp.copy()))
+    return v
+
+
+def rel_inf_rows(a: np.ndarray, ref: np.ndarray, axis=-1) -> np.ndarray:
+    """||a - ref||_inf / ||ref||_inf along `axis` (one value per vector)."""
+    num = np.abs(np.asarray(a, np.float64) - ref).max(axis=axis)
+    den = np.abs(ref).max(axis=axis)
+    return num / np.maximum(den, 1e-30)
+
+
+def compare_codes(gpu: np.ndarray, orc: np.ndarray, ratio: np.ndarray | None, tie_eps: float):
+    """Codes must agree except 1-LSB flips at values within tie_eps of a rounding tie.
+
+    Returns (n_mismatch, n_total, all_mismatches_explained)."""
+    d = gpu.astype(np.int32) - orc.astype(np.int32)
+    mism = d != 0
+    n = int(mism.sum())
+    if n == 0:
+        return 0, gpu.size, True
+    if np.abs(d).max() > 1:
+        return n, gpu.size, False
+    if ratio is None:
+        return n, gpu.size, False
+    frac = np.abs(ratio - np.trunc(ratio))
+    near = np.abs(frac - 0.5) < tie_eps
+    return n, gpu.size, bool(np.all(near[mism]))
+
+
+def oracle_ratios(cfg: lq.Config, S_heads: np.ndarray, hp_rows_heads) -> np.ndarray:
+    """x/s behind every oracle code, for float32 states S_heads [nh, dk, dv]."""
+    oc = ocfg(cfg)
+    out = np.zeros(S_heads.shape, np.float64)
+    for h in range(S_heads.shape[0]):
+        rows = None if hp_rows_heads is None else hp_rows_heads[h]
+        out[h] = O.quantize(oc, S_heads[h].astype(f32), hp_rows=rows, want_ratio=True)["ratio"]
+    return out
+
+
+def prefill_state(wl: configs.Workload, tokens: int, heads=None) -> np.ndarray:
+    """Oracle prefill from zero over `tokens` generator tokens, then the
+    workload's outliers; returns float32 [B, H, dk, dv] (or the listed heads)."""
+    pre = gen.token_inputs(wl, tokens, stream="prefill")
+    oc = O.Cfg(dk=wl.dk, dv=wl.dv, gate=wl.gate, quantize=0)
+    S = O.prefill(oc, O.per_head_inputs(pre, wl.H)).astype(f32).reshape(wl.B, wl.H, wl.dk, wl.dv)
+    return gen.apply_outliers(torch.from_numpy(S), wl).numpy()
+
+
+def step_args(tok: dict, t: int):
+    return (tok["q"][t], tok["k"][t], tok["v"][t], tok["beta"][t], tok["alpha"][t])

@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/lq_state.h declares, validates configs and rejects
+bad arguments before launching anything."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+from quantized_recurrent_state_lq_b200 import configs, lq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lq_state.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    return lq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ["lq_state_init", "lq_decode_step", "lq_window_flush", "lq_quantize_state",
+                 "lq_dequantize_state"]:
+        assert must in names
+    assert sorted(lq.EXPORTED) == names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", lq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r" T (lq_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert getattr(L, n) is not None
+
+
+@pytest.mark.parametrize("wl", configs.WORKLOADS, ids=lambda w: w.name)
+@pytest.mark.parametrize("mode", ["fp32", "step", "window"])
+def test_workload_configs_are_valid(L, wl, mode):
+    cfg = lq.Config.from_workload(wl, mode=mode)
+    assert lq.lq_config_check(cfg) == lq.LQ_OK
+    assert lq.lq_workspace_bytes(cfg) > 0
+
+
+def test_workspace_size_matches_record_layout(L):
+    wl = configs.KDA_B256
+    cfg = lq.Config.from_workload(wl)
+    dk, dv, r, W = wl.dk, wl.dv, wl.r, wl.W
+    payload = (dk * dv) + 4 * (dk + dv) + 4 * (r + W) * (dk + dv) + 4 * dk
+    per_head = (lq.lq_workspace_bytes(cfg) - 256) / wl.heads
+    assert payload <= per_head <= payload + 128 + 64
+    fp = lq.Config.from_workload(wl, mode="fp32")
+    assert lq.lq_workspace_bytes(fp) == 256 + wl.heads * dk * dv * 4
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("dk", 96, lq.LQ_ERR_UNSUPPORTED), ("dv", 256, lq.LQ_ERR_UNSUPPORTED),
+    ("Hk", 3, lq.LQ_ERR_SHAPE), ("B", 0, lq.LQ_ERR_SHAPE), ("H", 0, lq.LQ_ERR_SHAPE),
+    ("W", 0, lq.LQ_ERR_INVALID_ARG), ("r", 129, lq.LQ_ERR_INVALID_ARG), ("r", -1, lq.LQ_ERR_INVALID_ARG),
+    ("power_iters", -1, lq.LQ_ERR_INVALID_ARG), ("n_hp_rows", 128, lq.LQ_ERR_INVALID_ARG),
+    ("smoothing", 2, lq.LQ_ERR_INVALID_ARG), ("fused_flush", 7, lq.LQ_ERR_INVALID_ARG),
+    ("W", 400, lq.LQ_ERR_UNSUPPORTED),
+])
+def test_config_errors(L, field, value, code):
+    cfg = lq.Config.from_workload(configs.GDN_SERVING)
+    setattr(cfg, field, value)
+    assert lq.lq_config_check(cfg) == code
+    assert lq.lq_workspace_bytes(cfg) == 0
+
+
+def test_step_mode_requires_window_one(L):
+    cfg = lq.Config.from_workload(configs.GDN_SERVING, mode="step")
+    assert lq.lq_config_check(cfg) == lq.LQ_OK
+    cfg.W = 4
+    assert lq.lq_config_check(cfg) == lq.LQ_ERR_INVALID_ARG
+
+
+def _init(L, cfg, ws, nbytes, s0, rows=None):
+    h = C.c_void_p()
+    return L.lq_state_init(C.byref(h), C.byref(cfg.c()), C.c_void_p(ws), nbytes, C.c_void_p(s0), rows, None)
+
+
+def test_state_init_rejects_bad_arguments_without_launching(L):
+    """All of these fail on the host; the fake device addresses are never touched."""
+    cfg = lq.Config.from_workload(configs.TINY_GDN)
+    need = lq.lq_workspace_bytes(cfg)
+    fake_ws, fake_s0 = 0x7f0000000000, 0x7f1000000000
+    h = C.c_void_p()
+    assert L.lq_state_init(None, C.byref(cfg.c()), C.c_void_p(fake_ws), need, C.c_void_p(fake_s0), None, None) \
+        == lq.LQ_ERR_INVALID_ARG
+    assert _init(L, cfg, None, need, fake_s0) == lq.LQ_ERR_INVALID_ARG
+    assert _init(L, cfg, fake_ws, need, None) == lq.LQ_ERR_INVALID_ARG
+    assert _init(L, cfg, fake_ws + 64, need, fake_s0) == lq.LQ_ERR_WORKSPACE
+    assert _init(L, cfg, fake_ws, need - 1, fake_s0) == lq.LQ_ERR_WORKSPACE
+    bad = lq.Config.from_workload(configs.TINY_GDN)
+    bad.Hk = 3
+    assert _init(L, bad, fake_ws, need, fake_s0) == lq.LQ_ERR_SHAPE
+
+
+def test_state_init_checks_bf16_row_lists(L):
+    cfg = lq.Config.from_workload(configs.TINY_GDN, n_hp_rows=2)
+    need = lq.lq_workspace_bytes(cfg)
+    fake_ws, fake_s0 = 0x7f0000000000, 0x7f1000000000
+    assert _init(L, cfg, fake_ws, need, fake_s0, None) == lq.LQ_ERR_INVALID_ARG
+    dup = (C.c_int32 * 4)(1, 1, 2, 3)
+    assert _init(L, cfg, fake_ws, need, fake_s0, dup) == lq.LQ_ERR_INVALID_ARG
+    oob = (C.c_int32 * 4)(1, 64, 2, 3)
+    assert _init(L, cfg, fake_ws, need, fake_s0, oob) == lq.LQ_ERR_INVALID_ARG
+    neg = (C.c_int32 * 4)(-1, 5, 2, 3)
+    assert _init(L, cfg, fake_ws, need, fake_s0, neg) == lq.LQ_ERR_INVALID_ARG
+
+
+def test_null_handles_and_pointers(L):
+    assert L.lq_decode_step(None, *([C.c_void_p(16)] * 6), None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_window_flush(None, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_state_export_fp32(None, C.c_void_p(16), None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_get_status(None, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_state_buffered(None) == 0
+    L.lq_state_destroy(None)
+    cfg = lq.Config.from_workload(configs.TINY_GDN)
+    view = lq.lq_qstate_view(None, None, None, None, None, None)
+    assert L.lq_quantize_state(C.byref(cfg.c()), C.c_void_p(256), None, C.byref(view), None) \
+        == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_damp_select(C.byref(cfg.c()), 0, C.c_void_p(256), 1, C.c_void_p(256), C.c_void_p(256),
+                            C.c_void_p(256), None) == lq.LQ_ERR_INVALID_ARG
+
+
+def test_strerror_covers_every_status(L):
+    for code in range(-8, 1):
+        assert lq.strerror(code) != "unknown status"
+    assert lq.strerror(-99) == "unknown status"

@@ -1,0 +1,117 @@
+"""GPU codec parity (identical FP32 input to both sides): lq_quantize_state and
+lq_dequantize_state against the oracle's quantizer, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from quantized_recurrent_state_lq_b200 import inputs as gen, lq
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+# Codes: bit-exact except 1-LSB flips at rounding ties, on at most 0.01% of
+# entries.  Scales, smoothing factors and compensator products: relative 1e-5.
+CODE_FLIP_FRAC = 1e-4
+TIE_EPS = 1e-3
+REL = 1e-5
+
+CASES = [
+    # (B, H, dk, dv, r, K, smoothing, P)
+    (2, 3, 128, 128, 4, 8, 1, 0),
+    (1, 5, 64, 64, 2, 8, 1, 0),
+    (2, 2, 64, 128, 2, 8, 1, 0),
+    (2, 2, 128, 64, 3, 8, 1, 0),
+    (2, 3, 128, 128, 0, 8, 0, 0),      # naive INT8: no compensators, no smoothing
+    (2, 3, 128, 128, 0, 8, 1, 0),
+    (2, 4, 128, 128, 2, 8, 1, 16),     # DAMP BF16 rows
+    (1, 3, 128, 128, 4, 0, 1, 0),      # K = 0: c = R w0
+]
+
+
+def _rows(H, dk, P, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.stack([torch.sort(torch.randperm(dk, generator=g)[:P]).values for _ in range(H)]).int().numpy()
+
+
+@pytest.mark.parametrize("B,H,dk,dv,r,K,smoothing,P", CASES)
+def test_quantize_matches_oracle(B, H, dk, dv, r, K, smoothing, P):
+    U.require_gpu()
+    cfg = lq.Config(B=B, H=H, Hk=H, dk=dk, dv=dv, r=r, power_iters=K, smoothing=smoothing, n_hp_rows=P)
+    S = gen.random_state(B * H, dk, dv, seed=11 + dk + dv + r + P).reshape(B, H, dk, dv)
+    rows = _rows(H, dk, P, 5) if P else None
+    view = lq.alloc_view(cfg)
+    lq.lq_quantize_state(cfg, S.cuda(), view, hp_rows=rows)
+    torch.cuda.synchronize()
+    got = U.gpu_view_to_oracle(cfg, view, rows)
+    oc = U.ocfg(cfg)
+    hr = U.head_rows(cfg, rows)
+    Sn = S.numpy().reshape(B * H, dk, dv)
+    flips = total = 0
+    for h in range(B * H):
+        want = O.quantize(oc, Sn[h], hp_rows=None if hr is None else hr[h], want_ratio=True)
+        n, tot, ok = U.compare_codes(got["codes"][h], want["codes"], want["ratio"], TIE_EPS)
+        assert ok, f"head {h}: {n} code mismatches not explained by rounding ties"
+        flips += n
+        total += tot
+        np.testing.assert_allclose(got["m"][h], want["m"], rtol=REL)
+        np.testing.assert_allclose(got["s"][h], want["s"], rtol=REL, atol=1e-30)
+        scale = np.abs(Sn[h]).max()
+        for j in range(r):
+            pg = np.outer(got["c"][h][j], got["w"][h][j])
+            pw = np.outer(want["c"][j], want["w"][j])
+            assert np.abs(pg - pw).max() <= REL * scale, (h, j, np.abs(pg - pw).max() / scale)
+        if P:
+            np.testing.assert_array_equal(got["hp"][h][:P], want["hp"][:P])
+    print(f"codec parity {cfg.B}x{cfg.H} d{dk}x{dv} r{r}: {flips}/{total} tie flips")
+    assert flips <= CODE_FLIP_FRAC * total + 1
+
+
+@pytest.mark.parametrize("B,H,dk,dv,r,K,smoothing,P", CASES[:3] + CASES[6:7])
+def test_dequantize_matches_oracle(B, H, dk, dv, r, K, smoothing, P):
+    U.require_gpu()
+    cfg = lq.Config(B=B, H=H, Hk=H, dk=dk, dv=dv, r=r, power_iters=K, smoothing=smoothing, n_hp_rows=P)
+    S = gen.random_state(B * H, dk, dv, seed=3).numpy()
+    rows = _rows(H, dk, P, 7) if P else None
+    hr = U.head_rows(cfg, rows)
+    oc = U.ocfg(cfg)
+    ov = O.empty_views(oc, B * H)
+    want = np.zeros((B * H, dk, dv))
+    for h in range(B * H):
+        q = O.quantize(oc, S[h], hp_rows=None if hr is None else hr[h])
+        for k in ov:
+            ov[k][h][...] = np.asarray(q[k]).reshape(ov[k][h].shape)
+        want[h] = O.dequantize(oc, q, hp_rows=None if hr is None else hr[h])
+    view = U.oracle_view_to_gpu(cfg, ov, rows)
+    out = torch.empty((B, H, dk, dv), device="cuda")
+    lq.lq_dequantize_state(cfg, view, out, hp_rows=rows)
+    got = out.cpu().numpy().reshape(B * H, dk, dv)
+    err = U.rel_inf_rows(got.reshape(B * H, -1), want.reshape(B * H, -1))
+    assert err.max() < 1e-6, err.max()
+
+
+def test_view_export_import_roundtrip():
+    U.require_gpu()
+    cfg = lq.Config(B=2, H=3, Hk=3, dk=128, dv=128, W=4, r=2, n_hp_rows=8)
+    rows = _rows(3, 128, 8, 9)
+    S0 = gen.random_state(6, 128, 128, seed=4).reshape(2, 3, 128, 128).cuda()
+    st = lq.lq_state_init(cfg, S0, hp_rows=rows)
+    v1 = lq.alloc_view(cfg)
+    lq.lq_state_export_view(st, v1)
+    v2 = lq.alloc_view(cfg)
+    lq.lq_quantize_state(cfg, S0, v2, hp_rows=rows)
+    for k in v1:
+        assert torch.equal(v1[k], v2[k]), k
+    v3 = {k: t.clone() for k, t in v1.items()}
+    v3["s"].mul_(2.0)
+    lq.lq_state_import_view(st, v3)
+    v4 = lq.alloc_view(cfg)
+    lq.lq_state_export_view(st, v4)
+    for k in v3:
+        assert torch.equal(v3[k], v4[k]), k
+    # export of the FP32 state at a window start equals dequantize of the view
+    a = torch.empty_like(S0)
+    b = torch.empty_like(S0)
+    lq.lq_state_export_fp32(st, a)
+    lq.lq_dequantize_state(cfg, v4, b, hp_rows=rows)
+    torch.testing.assert_close(a, b, rtol=1e-6, atol=1e-6 * b.abs().max().item())

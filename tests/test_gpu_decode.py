@@ -1,0 +1,235 @@
+"""GPU decode parity through the C ABI against the oracle on the same seeded
+inputs: FP32-state mode, windowed INT8 (teacher-forced per window: each window
+starts from the oracle's window-start view, imported into the GPU state),
+per-step INT8, naive INT8, DAMP rows, partial windows and error paths."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from quantized_recurrent_state_lq_b200 import configs, inputs as gen, lq
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+OUT_REL = 1e-3     # outputs: max relative error per output vector (b, h, t)
+STATE_REL = 1e-3   # FP32 state: max relative error per head
+TIE_EPS = 0.05     # post-flush codes may flip 1 LSB only this close to a tie
+FLUSH_FLIP_FRAC = 2e-3
+
+
+def _workload(gate, B, H, Hk, dk, dv, W, r, seed, P=0):
+    return configs.TINY_GDN.with_(gate=gate, B=B, H=H, Hk=Hk, dk=dk, dv=dv, W=W, r=r, seed=seed, P=P,
+                                  n_out_rows=3, n_out_cols=3, out_lo=10.0, out_hi=50.0)
+
+
+def _rows_for(wl):
+    if not wl.P:
+        return None
+    g = torch.Generator().manual_seed(wl.seed + 77)
+    return torch.stack([torch.sort(torch.randperm(wl.dk, generator=g)[:wl.P]).values
+                        for _ in range(wl.H)]).int().numpy()
+
+
+@pytest.mark.parametrize("gate,B,H,Hk,dk,dv", [("gdn", 2, 4, 2, 128, 128), ("kda", 1, 3, 3, 64, 128),
+                                               ("gdn", 1, 2, 2, 64, 64), ("kda", 2, 2, 1, 128, 64)])
+def test_fp32_mode_matches_oracle(gate, B, H, Hk, dk, dv):
+    U.require_gpu()
+    wl = _workload(gate, B, H, Hk, dk, dv, 8, 0, seed=21)
+    T = 96
+    S0 = U.prefill_state(wl, 64)
+    tok = gen.token_inputs(wl, T, device="cuda")
+    cfg = lq.Config.from_workload(wl, mode="fp32")
+    st = lq.lq_state_init(cfg, torch.from_numpy(S0).cuda())
+    outs = torch.empty((T, B, H, dv), device="cuda")
+    for t in range(T):
+        lq.lq_decode_step(st, *U.step_args(tok, t), outs[t])
+    S = torch.empty((B, H, dk, dv), device="cuda")
+    lq.lq_state_export_fp32(st, S)
+    assert lq.lq_get_status(st) == lq.LQ_OK
+    ref = O.run(U.ocfg(cfg, quantize=0), O.per_head_inputs(tok, H), S0=S0.reshape(-1, dk, dv))
+    got = outs.cpu().numpy().reshape(T, B * H, dv)
+    err = U.rel_inf_rows(got, ref["o"])
+    print(f"fp32 mode {gate} d{dk}x{dv}: max out rel err {err.max():.2e}")
+    assert err.max() < OUT_REL
+    serr = U.rel_inf_rows(S.cpu().numpy().reshape(B * H, -1), ref["S"].reshape(B * H, -1))
+    assert serr.max() < STATE_REL
+
+
+def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label=""):
+    """Run T tokens window by window; each window starts from the oracle's view."""
+    cfg = lq.Config.from_workload(wl, mode=mode, fused_flush=int(fused), smoothing=smoothing)
+    if mode == "step":
+        cfg.W = 1
+    rows = _rows_for(wl)
+    hr = U.head_rows(cfg, rows)
+    nh = wl.B * wl.H
+    S0 = U.prefill_state(wl, 64)
+    tok = gen.token_inputs(wl, T, device="cuda")
+    ph = O.per_head_inputs(tok, wl.H)
+    oc = U.ocfg(cfg)
+    st = lq.lq_state_init(cfg, torch.from_numpy(S0).cuda(), hp_rows=rows)
+    # window-start view of the oracle
+    ov = O.empty_views(oc, nh)
+    for h in range(nh):
+        q = O.quantize(oc, S0.reshape(nh, wl.dk, wl.dv)[h], hp_rows=None if hr is None else hr[h])
+        for k in ov:
+            ov[k][h][...] = np.asarray(q[k]).reshape(ov[k][h].shape)
+    W = cfg.W
+    stats = {"out": 0.0, "state": 0.0, "flips": 0, "codes": 0}
+    o = torch.empty((wl.B, wl.H, wl.dv), device="cuda")
+    t0 = 0
+    while t0 < T:
+        n = min(W, T - t0)
+        sl = {k: v[t0:t0 + n] for k, v in ph.items()}
+        ref = O.run(oc, sl, view=ov, hp_rows=hr, flush_last=(n == W))
+        lq.lq_state_import_view(st, U.oracle_view_to_gpu(cfg, ov, rows))
+        for t in range(n):
+            last = t == n - 1
+            if last and n == W and not fused and mode == "window":
+                lq.lq_decode_step(st, *U.step_args(tok, t0 + t), o)
+                S = torch.empty((wl.B, wl.H, wl.dk, wl.dv), device="cuda")
+                lq.lq_state_export_fp32(st, S)
+                e = U.rel_inf_rows(S.cpu().numpy().reshape(nh, -1), ref["S_pre"].reshape(nh, -1))
+                stats["state"] = max(stats["state"], float(e.max()))
+                lq.lq_window_flush(st)
+            else:
+                lq.lq_decode_step(st, *U.step_args(tok, t0 + t), o)
+            e = U.rel_inf_rows(o.cpu().numpy().reshape(nh, wl.dv), ref["o"][t])
+            stats["out"] = max(stats["out"], float(e.max()))
+        assert lq.lq_state_buffered(st) == (0 if n == W else n)
+        if n == W:
+            gv = lq.alloc_view(cfg)
+            lq.lq_state_export_view(st, gv)
+            got = U.gpu_view_to_oracle(cfg, gv, rows)
+            ratio = U.oracle_ratios(cfg, ref["S_pre"].astype(np.float32), hr)
+            nflip, ntot, ok = U.compare_codes(got["codes"], ref["view"]["codes"], ratio, TIE_EPS)
+            assert ok, f"{label}: code mismatches beyond 1-LSB rounding ties at window {t0 // W}"
+            stats["flips"] += nflip
+            stats["codes"] += ntot
+            np.testing.assert_allclose(got["m"], ref["view"]["m"], rtol=STATE_REL)
+            np.testing.assert_allclose(got["s"], ref["view"]["s"], rtol=STATE_REL)
+            scale = np.abs(ref["S_pre"]).max(axis=(1, 2))
+            for j in range(cfg.r):
+                pg = np.einsum("hi,hc->hic", got["c"][:, j], got["w"][:, j])
+                pw = np.einsum("hi,hc->hic", ref["view"]["c"][:, j], ref["view"]["w"][:, j])
+                assert (np.abs(pg - pw).max(axis=(1, 2)) <= STATE_REL * scale).all()
+            if cfg.n_hp_rows:
+                hpg = got["hp"][:, :cfg.n_hp_rows].view(np.int16).astype(np.int32)
+                hpw = ref["view"]["hp"][:, :cfg.n_hp_rows].view(np.int16).astype(np.int32)
+                assert np.abs(hpg - hpw).max() <= 1   # one bf16 ulp at a rounding tie
+        ov = ref["view"]
+        t0 += n
+    assert lq.lq_get_status(st) == lq.LQ_OK
+    print(f"{label}: out {stats['out']:.2e} state {stats['state']:.2e} "
+          f"flips {stats['flips']}/{stats['codes']}")
+    assert stats["out"] < OUT_REL
+    assert stats["state"] < STATE_REL
+    assert stats["flips"] <= FLUSH_FLIP_FRAC * max(stats["codes"], 1) + 1
+    return stats
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("gate,B,H,Hk,dk,dv,W,r", [
+    ("gdn", 1, 2, 2, 64, 64, 16, 2),        # the tiny workload's shape
+    ("gdn", 2, 4, 2, 128, 128, 8, 4),       # GQA, d = 128
+    ("kda", 2, 3, 3, 128, 128, 8, 4),
+    ("kda", 1, 3, 3, 64, 128, 5, 2),        # dk != dv, odd window
+    ("gdn", 2, 2, 2, 128, 64, 6, 3),
+])
+def test_windowed_teacher_forced(fused, gate, B, H, Hk, dk, dv, W, r):
+    U.require_gpu()
+    wl = _workload(gate, B, H, Hk, dk, dv, W, r, seed=31 + W)
+    T = 3 * W + W // 2   # three windows and a ragged tail
+    _teacher_forced(wl, T, fused, label=f"window {gate} d{dk}x{dv} W{W} r{r} fused{int(fused)}")
+
+
+def test_damp_rows_teacher_forced():
+    U.require_gpu()
+    wl = _workload("gdn", 2, 3, 3, 128, 128, 8, 2, seed=41, P=16)
+    _teacher_forced(wl, 2 * 8 + 3, True, label="damp P16")
+
+
+def test_per_step_int8_mode():
+    U.require_gpu()
+    wl = _workload("kda", 1, 3, 3, 128, 128, 1, 4, seed=43)
+    _teacher_forced(wl, 12, True, mode="step", label="per-step int8")
+
+
+def test_naive_int8_mode():
+    U.require_gpu()
+    wl = _workload("gdn", 2, 2, 2, 128, 128, 1, 0, seed=44)
+    _teacher_forced(wl, 12, True, mode="step", smoothing=0, label="naive int8")
+
+
+def test_free_running_tiny_workload():
+    """The tiny GDN workload end to end (no teacher forcing): the GPU and the
+    oracle each run the whole decode from the same initial state."""
+    U.require_gpu()
+    wl = configs.TINY_GDN
+    S0 = U.prefill_state(wl, wl.prefill)
+    tok = gen.token_inputs(wl, wl.T, device="cuda")
+    cfg = lq.Config.from_workload(wl)
+    st = lq.lq_state_init(cfg, torch.from_numpy(S0).cuda())
+    outs = torch.empty((wl.T, wl.B, wl.H, wl.dv), device="cuda")
+    for t in range(wl.T):
+        lq.lq_decode_step(st, *U.step_args(tok, t), outs[t])
+    ref = O.run(U.ocfg(cfg), O.per_head_inputs(tok, wl.H), S0=S0.reshape(-1, wl.dk, wl.dv))
+    fp = O.run(U.ocfg(cfg, quantize=0), O.per_head_inputs(tok, wl.H), S0=S0.reshape(-1, wl.dk, wl.dv))
+    got = outs.cpu().numpy().reshape(wl.T, -1, wl.dv)
+    err = U.rel_inf_rows(got, ref["o"])
+    q_err = U.rel_inf_rows(ref["o"], fp["o"])
+    print(f"free-running tiny: max rel err vs oracle {err.max():.2e} (mean {err.mean():.2e}); "
+          f"oracle's own quantization error vs FP {q_err.mean():.2e}")
+    # Any code flip at a window boundary propagates; bound by a fraction of the
+    # method's own quantization error.
+    assert err.mean() < 0.25 * q_err.mean() + 1e-6
+
+
+def test_partial_window_flush_and_window_full():
+    U.require_gpu()
+    wl = _workload("gdn", 1, 2, 2, 128, 128, 4, 2, seed=50)
+    cfg = lq.Config.from_workload(wl, fused_flush=0)
+    S0 = torch.from_numpy(U.prefill_state(wl, 32)).cuda()
+    tok = gen.token_inputs(wl, 8, device="cuda")
+    st = lq.lq_state_init(cfg, S0)
+    o = torch.empty((1, 2, 128), device="cuda")
+    for t in range(4):
+        lq.lq_decode_step(st, *U.step_args(tok, t), o)
+    with pytest.raises(lq.LqError) as ei:
+        lq.lq_decode_step(st, *U.step_args(tok, 4), o)
+    assert ei.value.code == lq.LQ_ERR_WINDOW_FULL
+    lq.lq_window_flush(st)
+    assert lq.lq_state_buffered(st) == 0
+    lq.lq_decode_step(st, *U.step_args(tok, 4), o)
+    lq.lq_decode_step(st, *U.step_args(tok, 5), o)
+    assert lq.lq_state_buffered(st) == 2
+    # oracle: window of 4, flush, then 2 tokens and a flush after 2
+    oc = U.ocfg(cfg)
+    ph = O.per_head_inputs(tok, 2)
+    a = O.run(oc, {k: v[:4] for k, v in ph.items()}, S0=S0.cpu().numpy().reshape(2, 128, 128), flush_last=True)
+    b = O.run(O.Cfg(**{**oc.__dict__, "W": 2}), {k: v[4:6] for k, v in ph.items()}, view=a["view"],
+              flush_last=True)
+    lq.lq_window_flush(st)
+    S = torch.empty_like(S0)
+    lq.lq_state_export_fp32(st, S)
+    deq = np.stack([O.dequantize(oc, {k: b["view"][k][h] for k in b["view"]}) for h in range(2)])
+    err = U.rel_inf_rows(S.cpu().numpy().reshape(2, -1), deq.reshape(2, -1))
+    # every window boundary may flip a few codes; compare within a few LSB-sized steps
+    assert err.max() < 2e-2, err
+    lq.lq_window_flush(st)   # nothing buffered: no-op
+    assert lq.lq_get_status(st) == lq.LQ_OK
+
+
+def test_nonfinite_inputs_raise_status():
+    U.require_gpu()
+    wl = _workload("gdn", 1, 2, 2, 64, 64, 4, 1, seed=60)
+    cfg = lq.Config.from_workload(wl)
+    S0 = torch.from_numpy(U.prefill_state(wl, 16)).cuda()
+    st = lq.lq_state_init(cfg, S0)
+    tok = gen.token_inputs(wl, 2, device="cuda")
+    v = tok["v"][0].clone()
+    v[0, 1, 3] = float("nan")
+    o = torch.empty((1, 2, 64), device="cuda")
+    lq.lq_decode_step(st, tok["q"][0], tok["k"][0], v, tok["beta"][0], tok["alpha"][0], o)
+    assert lq.lq_get_status(st) == lq.LQ_ERR_NONFINITE

@@ -322,7 +322,7 @@ def run_ours(args, wl, world, rank, pg):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * dt_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "state_dtype": "int8", "data": "synthetic",
-            "config": {"workload": wl.name, "gate": wl.gate, "B": wl.B, "H": wl.H, "Hk": wl.Hk, "dk": wl.dk,
+            "config": {"workload": wl.name, "gate": wl.gate, "prefill": wl.prefill, "B": wl.B, "H": wl.H, "Hk": wl.Hk, "dk": wl.dk,
                        "dv": wl.dv, "W": wl.W, "r": wl.r, "K": wl.K, "P": wl.P, "step": "one window per head",
                        "l2": "state + buffers + inputs larger than L2 (no flush needed)",
                        "parallelism": f"dp{world} (independent heads, no collective)"},
@@ -366,10 +366,16 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WL, choices=sorted(configs.BY_NAME))
     ap.add_argument("--no-modes", action="store_true", help="skip the FP32 / per-step INT8 context lines")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")
+    ap.add_argument("--prefill", type=int, default=None, help="override the prefill length (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     wl = configs.BY_NAME[args.workload]
+    if args.batch is not None:
+        wl = wl.with_(B=args.batch)
+    if args.prefill is not None:
+        wl = wl.with_(prefill=args.prefill)
     world, rank, local, pg = dist_setup()
     try:
         if args.impl == "reference":

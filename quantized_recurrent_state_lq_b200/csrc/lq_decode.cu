@@ -391,11 +391,11 @@ __global__ void __launch_bounds__(kThreads) fp32_step_kernel(const Fp32Args a) {
 // ---------------------------------------------------------------------------
 // Host-side launchers (called from the C ABI).
 // ---------------------------------------------------------------------------
-// Raise a kernel's dynamic shared memory limit once per size it is launched
-// with (the attribute is only set when a larger size is first needed).
+// Raise a kernel's dynamic shared memory limit when a launch first needs more
+// than it was set to.  `done` must be distinct for every kernel, so each
+// launcher below keeps its own.
 template <typename K>
-static cudaError_t set_smem(K kern, size_t bytes) {
-    static size_t done = 0;  // one per kernel instantiation
+static cudaError_t set_smem(K kern, size_t bytes, size_t &done) {
     if (bytes <= done) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e == cudaSuccess) done = bytes;
@@ -406,7 +406,8 @@ template <int DK, int DV, bool KDA, bool FLUSH, bool DAMP>
 static cudaError_t launch_decode_t(const DecodeArgs &a, int heads, cudaStream_t s) {
     const size_t sm = decode_smem_bytes(DK, DV, a.L);
     auto kern = decode_kernel<DK, DV, KDA, FLUSH, DAMP>;
-    cudaError_t e = set_smem(kern, sm);
+    static size_t done = 0;  // one per instantiation of this launcher
+    cudaError_t e = set_smem(kern, sm, done);
     if (e != cudaSuccess) return e;
     kern<<<heads, kThreads, sm, s>>>(a);
     return cudaGetLastError();
@@ -416,7 +417,8 @@ template <int DK, int DV, bool KDA, bool DAMP, bool EXPORT>
 static cudaError_t launch_flush_t(const DecodeArgs &a, int heads, cudaStream_t s) {
     const size_t sm = decode_smem_bytes(DK, DV, a.L);
     auto kern = flush_kernel<DK, DV, KDA, DAMP, EXPORT>;
-    cudaError_t e = set_smem(kern, sm);
+    static size_t done = 0;  // one per instantiation of this launcher
+    cudaError_t e = set_smem(kern, sm, done);
     if (e != cudaSuccess) return e;
     kern<<<heads, kThreads, sm, s>>>(a);
     return cudaGetLastError();

@@ -1,0 +1,108 @@
+"""Parity at the workloads' full sizes, in the launch configuration bench.py
+times (whole batch, CUDA-graph replay of one window, fused flush), on a sample
+of heads the oracle recomputes one by one.
+
+1. The GPU prefill (FP32-state kernel, all heads, the full prefill length) is
+   compared with the oracle's prefill of the sampled heads on the same inputs.
+2. The sampled heads' initial states are replaced by the oracle's, both sides
+   quantize them (codes compared with the rounding-tie slack).
+3. The sampled heads' window-start views are set to the oracle's (teacher
+   forcing) and one window is replayed from the captured graph; outputs and the
+   flushed state of the sampled heads are compared with the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from quantized_recurrent_state_lq_b200 import configs, inputs as gen, lq, runner
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+
+def _sample(wl, n=6):
+    g = torch.Generator().manual_seed(wl.seed + 1000)
+    pts = {(0, 0), (wl.B - 1, wl.H - 1)}
+    while len(pts) < n:
+        pts.add((int(torch.randint(wl.B, (1,), generator=g)), int(torch.randint(wl.H, (1,), generator=g))))
+    return sorted(pts)
+
+
+def _rows(wl):
+    if not wl.P:
+        return None
+    g = torch.Generator().manual_seed(wl.seed + 2000)
+    return torch.stack([torch.sort(torch.randperm(wl.dk, generator=g)[:wl.P]).values
+                        for _ in range(wl.H)]).int().numpy()
+
+
+@pytest.mark.parametrize("wl", configs.WORKLOADS[1:], ids=lambda w: w.name)
+def test_full_size_sampled_heads(wl):
+    U.require_gpu()
+    heads = _sample(wl)
+    S, cap = runner.gpu_prefill(wl, capture_heads=heads)
+    bsel = sorted({b for b, _ in heads})
+    local = [(bsel.index(b), h) for b, h in heads]
+    oc0 = O.Cfg(dk=wl.dk, dv=wl.dv, gate=wl.gate, quantize=0)
+    pre = O.prefill(oc0, O.per_head_inputs(cap, wl.H, heads=local))
+    idx_b = torch.tensor([b for b, _ in heads])
+    idx_h = torch.tensor([h for _, h in heads])
+    got0 = S[idx_b.cuda(), idx_h.cuda()].cpu().numpy()
+    e0 = U.rel_inf_rows(got0.reshape(len(heads), -1), pre.reshape(len(heads), -1))
+    print(f"{wl.name}: prefill ({wl.prefill} tokens, FP32 kernel) max rel err {e0.max():.2e}")
+    assert e0.max() < 1e-3
+
+    # both sides start from the oracle's prefilled state of the sampled heads
+    S[idx_b.cuda(), idx_h.cuda()] = torch.from_numpy(pre.astype(np.float32)).cuda()
+    S = gen.apply_outliers(S, wl)
+    S_s = S[idx_b.cuda(), idx_h.cuda()].cpu().numpy()
+    rows = _rows(wl)
+    hr = None if rows is None else np.ascontiguousarray(rows[idx_h.numpy()])
+    r = runner.WindowRunner(wl, S, hp_rows=rows, tokens=wl.W)
+    cfg = r.cfg
+    oc = U.ocfg(cfg)
+    ns = len(heads)
+    ov = O.empty_views(oc, ns)
+    for i in range(ns):
+        q = O.quantize(oc, S_s[i], hp_rows=None if hr is None else hr[i], want_ratio=True)
+        for k in ov:
+            ov[k][i][...] = np.asarray(q[k]).reshape(ov[k][i].shape)
+        ov.setdefault("ratio", np.zeros((ns, wl.dk, wl.dv)))[i] = q["ratio"]
+    ratio0 = ov.pop("ratio")
+    gv = lq.alloc_view(cfg)
+    lq.lq_state_export_view(r.st, gv)
+    sub = lq.Config(**{**cfg.__dict__, "B": 1, "H": ns})
+    pick = {k: v[idx_b.cuda(), idx_h.cuda()].unsqueeze(0).contiguous() for k, v in gv.items()}
+    got = U.gpu_view_to_oracle(sub, pick, None if hr is None else hr)
+    c = U.compare_codes(got["codes"], ov["codes"], ratio0)
+    print(f"{wl.name}: initial codes {c}")
+    U.assert_code_bar(c, wl.name + " initial")
+
+    # teacher forcing: the sampled heads start the window from the oracle's view
+    r.capture()
+    lq.lq_state_export_view(r.st, gv)
+    ovg = U.oracle_view_to_gpu(sub, ov, None if hr is None else hr)
+    for k in gv:
+        gv[k][idx_b.cuda(), idx_h.cuda()] = ovg[k][0]
+    lq.lq_state_import_view(r.st, gv)
+    r.replay(0)
+    torch.cuda.synchronize()
+    assert lq.lq_get_status(r.st) == lq.LQ_OK
+    assert torch.isfinite(r.out[: wl.W]).all()
+    tok_s = O.per_head_inputs(r.tok, wl.H, heads=heads)
+    tok_s = {k: v[: wl.W] for k, v in tok_s.items()}
+    ref = O.run(oc, tok_s, view=ov, hp_rows=hr, flush_last=True)
+    out = r.out[: wl.W][:, idx_b.cuda(), idx_h.cuda()].cpu().numpy()
+    e = U.rel_inf_rows(out, ref["o"])
+    print(f"{wl.name}: window outputs max rel err {e.max():.2e}")
+    assert e.max() < 1e-3
+    lq.lq_state_export_view(r.st, gv)
+    pick = {k: v[idx_b.cuda(), idx_h.cuda()].unsqueeze(0).contiguous() for k, v in gv.items()}
+    got = U.gpu_view_to_oracle(sub, pick, None if hr is None else hr)
+    ratio = U.oracle_ratios(sub, ref["S_pre"].astype(np.float32), hr)
+    c = U.compare_codes(got["codes"], ref["view"]["codes"], ratio)
+    print(f"{wl.name}: flushed codes {c}")
+    U.assert_code_bar(c, wl.name + " flushed")
+    np.testing.assert_allclose(got["s"], ref["view"]["s"], rtol=1e-3)
+    np.testing.assert_allclose(got["m"], ref["view"]["m"], rtol=1e-3)

@@ -18,6 +18,7 @@ struct lq_state {
     size_t bytes;
     int *status;
     int *hp_rows;
+    int *slot_rows;
     unsigned char *rec;
     size_t heads;
     int n;  // tokens buffered in the current window
@@ -70,6 +71,10 @@ int check_config(const lq_config *c) {
 
 size_t hp_bytes(const lq_config *c) { return align_sz((size_t)c->H * c->n_hp_rows * 4, kAlign); }
 
+size_t slot_bytes(const lq_config *c) {
+    return c->n_hp_rows > 0 ? align_sz((size_t)c->H * c->dk * 4, kAlign) : 0;
+}
+
 size_t record_bytes(const lq_config *c) {
     if (is_int8(c)) return (size_t)layout_of(c).rec_bytes;
     return (size_t)c->dk * c->dv * 4;
@@ -93,7 +98,7 @@ lq::QPtrs record_ptrs(const lq_state *st) {
     const Layout &L = st->L;
     lq::QPtrs q{};
     const size_t hs = (size_t)L.rec_bytes;
-    q.codes = st->rec; q.codes_hs = hs;
+    q.codes = st->rec + L.off_codes; q.codes_hs = hs;
     q.hp = st->rec + L.off_hp; q.hp_hs = hs;
     q.m = st->rec + L.off_m; q.m_hs = hs;
     q.s = st->rec + L.off_s; q.s_hs = hs;
@@ -120,7 +125,8 @@ int check_view(const lq_config *c, const lq_qstate_view *v) {
     if (c->n_hp_rows > 0 && !v->bf16_rows) return LQ_ERR_INVALID_ARG;
     if (c->r > 0 && (!v->comp_k || !v->comp_v)) return LQ_ERR_INVALID_ARG;
     const uintptr_t a = reinterpret_cast<uintptr_t>(v->codes) | reinterpret_cast<uintptr_t>(v->m) |
-                        reinterpret_cast<uintptr_t>(v->s) | reinterpret_cast<uintptr_t>(v->bf16_rows);
+                        reinterpret_cast<uintptr_t>(v->s) | reinterpret_cast<uintptr_t>(v->bf16_rows) |
+                        reinterpret_cast<uintptr_t>(v->comp_k) | reinterpret_cast<uintptr_t>(v->comp_v);
     if (a & 15) return LQ_ERR_INVALID_ARG;  // 16-byte vector access
     return LQ_OK;
 }
@@ -136,6 +142,7 @@ lq::DecodeArgs decode_args(const lq_state *st) {
     a.smoothing = st->cfg.smoothing;
     a.n = st->n;
     a.hp_rows = st->hp_rows;
+    a.slot_rows = st->slot_rows;
     a.status = st->status;
     return a;
 }
@@ -148,7 +155,7 @@ int lq_config_check(const lq_config *cfg) { return check_config(cfg); }
 
 size_t lq_workspace_bytes(const lq_config *cfg) {
     if (check_config(cfg) != LQ_OK) return 0;
-    return kAlign + hp_bytes(cfg) + (size_t)cfg->B * cfg->H * record_bytes(cfg);
+    return kAlign + hp_bytes(cfg) + slot_bytes(cfg) + (size_t)cfg->B * cfg->H * record_bytes(cfg);
 }
 
 int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_t bytes, const float *d_S0,
@@ -172,14 +179,37 @@ int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_
     st->bytes = bytes;
     st->status = reinterpret_cast<int *>(st->ws);
     st->hp_rows = reinterpret_cast<int *>(st->ws + kAlign);
-    st->rec = st->ws + kAlign + hp_bytes(cfg);
+    st->slot_rows = reinterpret_cast<int *>(st->ws + kAlign + hp_bytes(cfg));
+    st->rec = st->ws + kAlign + hp_bytes(cfg) + slot_bytes(cfg);
     st->heads = (size_t)cfg->B * cfg->H;
     st->n = 0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // Per head: the key row of every INT8 slot (increasing), then of every BF16 row.
+    int32_t *slots = nullptr;
+    if (cfg->n_hp_rows > 0) {
+        slots = static_cast<int32_t *>(malloc((size_t)cfg->H * cfg->dk * 4));
+        if (!slots) {
+            delete st;
+            return LQ_ERR_INVALID_ARG;
+        }
+        for (int h = 0; h < cfg->H; ++h) {
+            const int32_t *hr = h_hp_row_ids + (size_t)h * cfg->n_hp_rows;
+            int32_t *out_h = slots + (size_t)h * cfg->dk;
+            int j = 0;
+            for (int i = 0; i < cfg->dk; ++i) {
+                bool hp = false;
+                for (int p = 0; p < cfg->n_hp_rows; ++p) hp = hp || hr[p] == i;
+                if (!hp) out_h[j++] = i;
+            }
+            for (int p = 0; p < cfg->n_hp_rows; ++p) out_h[j++] = hr[p];
+        }
+    }
     cudaError_t e = cudaMemsetAsync(st->status, 0, sizeof(int), s);
     if (e == cudaSuccess && cfg->n_hp_rows > 0)
         e = cudaMemcpyAsync(st->hp_rows, h_hp_row_ids, (size_t)cfg->H * cfg->n_hp_rows * 4,
                             cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && cfg->n_hp_rows > 0)
+        e = cudaMemcpyAsync(st->slot_rows, slots, (size_t)cfg->H * cfg->dk * 4, cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) {
         if (is_int8(cfg)) {
             lq::CodecArgs a{};
@@ -193,6 +223,7 @@ int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_
         }
     }
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    free(slots);
     if (e != cudaSuccess) {
         delete st;
         return LQ_ERR_CUDA;
@@ -205,6 +236,11 @@ int lq_decode_step(lq_state *st, const float *d_q, const float *d_k, const float
                    const float *d_alpha, float *d_o, void *stream) {
     if (!st || !d_q || !d_k || !d_v || !d_beta || !d_alpha || !d_o) return LQ_ERR_INVALID_ARG;
     const lq_config &c = st->cfg;
+    // q, k, v and a per-channel gate are fetched with 16-byte bulk copies.
+    const uintptr_t al = reinterpret_cast<uintptr_t>(d_q) | reinterpret_cast<uintptr_t>(d_k) |
+                         reinterpret_cast<uintptr_t>(d_v) |
+                         (c.gate == LQ_GATE_CHANNEL ? reinterpret_cast<uintptr_t>(d_alpha) : 0);
+    if (al & 15) return LQ_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool kda = c.gate == LQ_GATE_CHANNEL;
     if (c.mode == LQ_MODE_FP32) {

@@ -14,31 +14,6 @@ struct QSmem {
     int wscr[kWarps];
 };
 
-template <int DK, int DV>
-__device__ __forceinline__ void tile_load_global(float (&R)[Tile<DK, DV>::RPT][16], const float *src) {
-    using T = Tile<DK, DV>;
-    const int t = threadIdx.x, cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
-#pragma unroll
-    for (int r = 0; r < T::RPT; ++r)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 f = __ldg(reinterpret_cast<const float4 *>(src + (size_t)(row0 + r) * DV + cg * 16) + q);
-            R[r][4 * q] = f.x; R[r][4 * q + 1] = f.y; R[r][4 * q + 2] = f.z; R[r][4 * q + 3] = f.w;
-        }
-}
-
-template <int DK, int DV>
-__device__ __forceinline__ void tile_store_global(const float (&R)[Tile<DK, DV>::RPT][16], float *dst) {
-    using T = Tile<DK, DV>;
-    const int t = threadIdx.x, cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
-#pragma unroll
-    for (int r = 0; r < T::RPT; ++r)
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            reinterpret_cast<float4 *>(dst + (size_t)(row0 + r) * DV + cg * 16)[q] =
-                make_float4(R[r][4 * q], R[r][4 * q + 1], R[r][4 * q + 2], R[r][4 * q + 3]);
-}
-
 __device__ __forceinline__ CodecOut codec_out_of(const QPtrs &q, int head) {
     CodecOut o;
     o.codes = reinterpret_cast<int8_t *>(q.codes + (size_t)head * q.codes_hs);
@@ -87,27 +62,28 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(const CodecArgs a)
     for (int r = 0; r < T::RPT; ++r) {
         const int i = row0 + r;
         const int mp = a.P > 0 ? sm.map[i] : i;
-        if (mp >= 0) {
-            const float mi = m[i];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const int col = cg * 16 + c;
-                R[r][c] = ((float)codes[(size_t)mp * DV + col] * s[col]) * mi;
+        for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int col = T::col(cg, qq) + u;
+                R[r][4 * qq + u] = mp >= 0 ? ((float)codes[(size_t)mp * DV + col] * s[col]) * m[i]
+                                           : bf16_to_f(hp[(size_t)(-1 - mp) * DV + col]);
             }
-        } else {
-            const int p = -1 - mp;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) R[r][c] = bf16_to_f(hp[(size_t)p * DV + cg * 16 + c]);
-        }
     }
     for (int j = 0; j < a.r; ++j) {
         const float *ck = reinterpret_cast<const float *>(q.ck + (size_t)head * q.ck_hs) + (size_t)j * q.ck_js;
         const float *cw = reinterpret_cast<const float *>(q.cw + (size_t)head * q.cw_hs) + (size_t)j * q.cw_js;
+        float wv[16];
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) wv[4 * qq + u] = cw[T::col(cg, qq) + u];
 #pragma unroll
         for (int r = 0; r < T::RPT; ++r) {
             const float c = ck[row0 + r];
 #pragma unroll
-            for (int cc = 0; cc < 16; ++cc) R[r][cc] = fmaf(c, cw[cg * 16 + cc], R[r][cc]);
+            for (int cc = 0; cc < 16; ++cc) R[r][cc] = fmaf(c, wv[cc], R[r][cc]);
         }
     }
     tile_store_global<DK, DV>(R, a.S_out + (size_t)head * DK * DV);

@@ -1,21 +1,26 @@
 // lq_codec.cuh -- the window-boundary quantizer on one head's FP32 state held
-// in registers across a 256-thread CTA.
+// in registers across the 256 compute threads of a CTA.
 //
 // Steps (LeapQuant project page: Compensator Tokens paragraph, then the
 // smoothing paragraph; STEPQuant article for key-row / value-column scales;
 // DAMP abstract for the BF16 rows):
 //   1. r compensators by deflated power iteration on the residual R:
-//      w = 1/sqrt(dv); K times { z = R w / |R w| ; w = R^T z / |R^T z| };
-//      c = R w;  R <- R - c w^T.   (norms accumulated in double)
+//      w = 1/sqrt(dv); K times { w = R^T (R w), normalised };  c = R w;
+//      R <- R - c w^T.  (R^T R w normalised is the oracle's z = Rw/|Rw|,
+//      w = R^T z/|R^T z| without the intermediate scaling, which only changes
+//      rounding; norms are accumulated in double.)
 //   2. BF16 rows: bf16_rne(R_i) for the head's listed key rows.
 //   3. m_i = sqrt(mean_c R_ic^2) (double accumulation), 1 if zero or if
 //      smoothing is off;  x = R / m.
 //   4. s_c = max_i |x_ic| / 127 over INT8 rows;  C = clamp(rne(x / s), +-127).
 //
-// Tile layout: a thread owns RPT consecutive key rows x 16 consecutive value
-// columns; CG = dv/16 column groups, RG = 256/CG row groups; thread t has
-// column group t % CG and row group t / CG, so the CG threads sharing rows are
-// adjacent lanes and the codes of one row segment leave as one 16-byte store.
+// Tile layout: a thread owns RPT consecutive key rows and 16 value columns, in
+// four groups of four adjacent columns spaced CG*4 apart:
+//   cols(cg, q, u) = 4*cg + 4*CG*q + u,  q, u in [0, 4),
+// with CG = dv/16 column groups and thread t in column group t % CG, row group
+// t / CG.  The CG threads sharing rows are adjacent lanes, so every 16-byte
+// shared-memory access of a column group touches consecutive words (no bank
+// conflicts) and code rows leave as 32-byte contiguous segments.
 #pragma once
 
 #include "lq_common.cuh"
@@ -27,14 +32,16 @@ struct Tile {
     static constexpr int CG = DV / 16;
     static constexpr int RG = kThreads / CG;
     static constexpr int RPT = DK / RG;
+    static constexpr int RGW = 32 / CG;  // row groups per warp
     static_assert(RPT >= 1 && RG * RPT == DK, "tile shape");
     static_assert(CG <= 32 && (32 % CG) == 0, "column groups per warp");
+    __device__ static int col(int cg, int q) { return 4 * cg + 4 * CG * q; }
 };
 
 template <int DK, int DV>
 struct CodecSmem {
-    float w[DV];
-    float red[kWarps][DV];
+    float red[2][kWarps][DV];   // cross-warp partial column sums (double-buffered)
+    float wv[kWarps][DV];       // per-warp copy of the current power-iteration vector
     float sc[DV];
     double dred[kWarps];
 };
@@ -51,33 +58,39 @@ struct CodecOut {
     int cw_stride;
 };
 
-// z[r] = sum_c R[r][c] w[c] for the thread's rows; all CG lanes of a row group
-// end with the full sums.
 template <int DK, int DV>
-__device__ __forceinline__ void tile_rows_matvec(const float (&R)[Tile<DK, DV>::RPT][16], const float *w_s,
-                                                 float (&z)[Tile<DK, DV>::RPT]) {
+__device__ __forceinline__ void load_cols16(const float *v, float (&o)[16]) {
     using T = Tile<DK, DV>;
     const int cg = threadIdx.x % T::CG;
-    float wv[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const float4 f = reinterpret_cast<const float4 *>(w_s + cg * 16)[q];
-        wv[4 * q] = f.x; wv[4 * q + 1] = f.y; wv[4 * q + 2] = f.z; wv[4 * q + 3] = f.w;
+        const float4 f = *reinterpret_cast<const float4 *>(v + T::col(cg, q));
+        o[4 * q] = f.x; o[4 * q + 1] = f.y; o[4 * q + 2] = f.z; o[4 * q + 3] = f.w;
     }
+}
+
+// z[r] = sum_c R[r][c] w[c] for the thread's rows (w: the thread's 16 column
+// values); all CG lanes of a row group end with the full sums.
+template <int DK, int DV>
+__device__ __forceinline__ void tile_rows_matvec(const float (&R)[Tile<DK, DV>::RPT][16], const float (&w)[16],
+                                                 float (&z)[Tile<DK, DV>::RPT]) {
+    using T = Tile<DK, DV>;
 #pragma unroll
     for (int r = 0; r < T::RPT; ++r) {
         float acc = 0.f;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) acc = fmaf(R[r][c], wv[c], acc);
+        for (int c = 0; c < 16; ++c) acc = fmaf(R[r][c], w[c], acc);
         z[r] = shfl_xor_sum<T::CG>(acc);
     }
 }
 
-// out_s[c] = sum_i R[i][c] z[i] over the whole tile.  Barrier at the end.
+// Column sums of R weighted by z, reduced over the tile.  Each warp ends with
+// the full vector y[DV] in its own wv[warp] (and lane-distributed in `mine`:
+// lane l holds y[4l .. 4l+3] for l < DV/4).  One barrier.
 template <int DK, int DV>
 __device__ __forceinline__ void tile_cols_matvec(const float (&R)[Tile<DK, DV>::RPT][16],
-                                                 const float (&z)[Tile<DK, DV>::RPT], float (*red)[DV],
-                                                 float *out_s) {
+                                                 const float (&z)[Tile<DK, DV>::RPT], CodecSmem<DK, DV> &cs,
+                                                 int buf, float4 &mine) {
     using T = Tile<DK, DV>;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5, cg = t % T::CG;
     float acc[16];
@@ -93,23 +106,24 @@ __device__ __forceinline__ void tile_cols_matvec(const float (&R)[Tile<DK, DV>::
     if (lane < T::CG) {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-            reinterpret_cast<float4 *>(&red[warp][cg * 16])[q] =
+            *reinterpret_cast<float4 *>(&cs.red[buf][warp][T::col(cg, q)]) =
                 make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
     }
-    __syncthreads();
-    if (t < DV) {
-        float s = 0.f;
+    cbar();
+    mine = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane < DV / 4) {
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) s += red[w][t];
-        out_s[t] = s;
+        for (int w = 0; w < kWarps; ++w) {
+            const float4 p = *reinterpret_cast<const float4 *>(&cs.red[buf][w][4 * lane]);
+            mine.x += p.x; mine.y += p.y; mine.z += p.z; mine.w += p.w;
+        }
     }
-    __syncthreads();
 }
 
 // Full codec on the register tile R (destroyed).  `map` is the shared row map
 // (slot >= 0 for INT8 rows, -1-p for BF16 row p); with P == 0 it may be null.
 // ENERGY: instead of writing codes, add sum_c (R - Deq)^2 of the residual to
-// eacc[r] (DAMP calibration); in that mode only m/s/compensators are computed.
+// eacc[r] (DAMP calibration); in that mode nothing is written.
 template <int DK, int DV, bool ENERGY>
 __device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, int K, int smoothing, int P,
                                const int *map, CodecSmem<DK, DV> &cs, const CodecOut &out,
@@ -119,59 +133,60 @@ __device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, in
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int cg = t % CG, rg = t / CG;
     const int row0 = rg * RPT;
+    int buf = 0;
 
     // 1. Compensator tokens.
     for (int j = 0; j < r_comp; ++j) {
-        if (t < DV) cs.w[t] = (float)(1.0 / sqrt((double)DV));
-        __syncthreads();
+        float w[16];
+        const float w0 = (float)(1.0 / sqrt((double)DV));
+#pragma unroll
+        for (int c = 0; c < 16; ++c) w[c] = w0;
         bool zero = false;
         for (int it = 0; it < K; ++it) {
             float z[RPT];
-            tile_rows_matvec<DK, DV>(R, cs.w, z);
-            double ss = 0.0;
-            if (cg == 0) {
-#pragma unroll
-                for (int r = 0; r < RPT; ++r) ss += (double)z[r] * (double)z[r];
-            }
-            const double nz = sqrt(block_sum_d(ss, cs.dred));
-            if (nz == 0.0) { zero = true; break; }
-#pragma unroll
-            for (int r = 0; r < RPT; ++r) z[r] = (float)((double)z[r] / nz);
-            tile_cols_matvec<DK, DV>(R, z, cs.red, cs.w);
-            const double sw = (t < DV) ? (double)cs.w[t] * (double)cs.w[t] : 0.0;
-            const double nw = sqrt(block_sum_d(sw, cs.dred));
+            tile_rows_matvec<DK, DV>(R, w, z);
+            float4 y;
+            tile_cols_matvec<DK, DV>(R, z, cs, buf, y);
+            buf ^= 1;
+            double ss = (double)y.x * y.x + (double)y.y * y.y + (double)y.z * y.z + (double)y.w * y.w;
+            const double nw = sqrt(warp_sum_d(ss));   // identical in every warp
             if (nw == 0.0) { zero = true; break; }
-            if (t < DV) cs.w[t] = (float)((double)cs.w[t] / nw);
-            __syncthreads();
+            const double inv = 1.0 / nw;
+            if (lane < DV / 4)
+                *reinterpret_cast<float4 *>(&cs.wv[warp][4 * lane]) =
+                    make_float4((float)(y.x * inv), (float)(y.y * inv), (float)(y.z * inv), (float)(y.w * inv));
+            __syncwarp();
+            load_cols16<DK, DV>(cs.wv[warp], w);
+            __syncwarp();
         }
         if (zero) {
             if (!ENERGY) {
                 if (t < DV) out.cw[j * out.cw_stride + t] = 0.f;
                 if (t < DK) out.ck[j * out.ck_stride + t] = 0.f;
             }
-            __syncthreads();
             continue;
         }
         float c[RPT];
-        tile_rows_matvec<DK, DV>(R, cs.w, c);
+        tile_rows_matvec<DK, DV>(R, w, c);
         if (!ENERGY) {
-            if (t < DV) out.cw[j * out.cw_stride + t] = cs.w[t];
+            if (warp == 0 && lane < CG) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<float4 *>(out.cw + j * out.cw_stride + T::col(cg, q)) =
+                        make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            }
             if (cg == 0) {
 #pragma unroll
                 for (int r = 0; r < RPT; ++r) out.ck[j * out.ck_stride + row0 + r] = c[r];
             }
         }
-        float wv[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) wv[q] = cs.w[cg * 16 + q];
 #pragma unroll
         for (int r = 0; r < RPT; ++r)
 #pragma unroll
-            for (int q = 0; q < 16; ++q) R[r][q] = fmaf(-c[r], wv[q], R[r][q]);
-        __syncthreads();
+            for (int q = 0; q < 16; ++q) R[r][q] = fmaf(-c[r], w[q], R[r][q]);
     }
 
-    // 2. BF16 rows and 3. smoothing scales.
+    // 2. BF16 rows and 3. smoothing scales; x = R / m in place (ENERGY keeps R).
     float m[RPT];
     bool int8row[RPT];
 #pragma unroll
@@ -181,13 +196,12 @@ __device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, in
         int8row[r] = mp >= 0;
         if (!ENERGY && mp < 0) {
             const int p = -1 - mp;
-            uint32_t pk[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                pk[q] = (uint32_t)bf16_rne(R[r][2 * q]) | ((uint32_t)bf16_rne(R[r][2 * q + 1]) << 16);
-            uint4 *dst = reinterpret_cast<uint4 *>(out.hp + (size_t)p * DV + cg * 16);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t lo = (uint32_t)bf16_rne(R[r][4 * q]) | ((uint32_t)bf16_rne(R[r][4 * q + 1]) << 16);
+                const uint32_t hi = (uint32_t)bf16_rne(R[r][4 * q + 2]) | ((uint32_t)bf16_rne(R[r][4 * q + 3]) << 16);
+                *reinterpret_cast<uint2 *>(out.hp + (size_t)p * DV + T::col(cg, q)) = make_uint2(lo, hi);
+            }
         }
         double ss = 0.0;
 #pragma unroll
@@ -202,6 +216,15 @@ __device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, in
         m[r] = mi;
         if (!ENERGY && cg == 0) out.m[i] = mi;
     }
+    // x = R / m (IEEE division, as the oracle); in place unless R is still
+    // needed for the error energy.
+    if (!ENERGY) {
+#pragma unroll
+        for (int r = 0; r < RPT; ++r)
+#pragma unroll
+            for (int q = 0; q < 16; ++q) R[r][q] = R[r][q] / m[r];
+    }
+    auto X = [&](int r, int q) -> float { return ENERGY ? R[r][q] / m[r] : R[r][q]; };
 
     // 4. Column scales over INT8 rows.
     {
@@ -212,7 +235,7 @@ __device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, in
         for (int r = 0; r < RPT; ++r) {
             if (!int8row[r]) continue;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) am[q] = fmaxf(am[q], fabsf(R[r][q] / m[r]));
+            for (int q = 0; q < 16; ++q) am[q] = fmaxf(am[q], fabsf(X(r, q)));
         }
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
@@ -223,24 +246,25 @@ __device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, in
         }
         if (lane < CG) {
 #pragma unroll
-            for (int q = 0; q < 16; ++q) cs.red[warp][cg * 16 + q] = am[q];
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<float4 *>(&cs.red[buf][warp][T::col(cg, q)]) =
+                    make_float4(am[4 * q], am[4 * q + 1], am[4 * q + 2], am[4 * q + 3]);
         }
-        __syncthreads();
+        cbar();
         if (t < DV) {
             float a = 0.f;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) a = fmaxf(a, cs.red[w][t]);
+            for (int w = 0; w < kWarps; ++w) a = fmaxf(a, cs.red[buf][w][t]);
             const float sc = a / 127.0f;
             cs.sc[t] = sc;
             if (!ENERGY) out.s[t] = sc;
         }
-        __syncthreads();
+        cbar();
     }
 
     // Codes (or the error energy of the INT8 reconstruction).
     float sv[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) sv[q] = cs.sc[cg * 16 + q];
+    load_cols16<DK, DV>(cs.sc, sv);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         if (!int8row[r]) continue;
@@ -249,9 +273,8 @@ __device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, in
         double e = 0.0;
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-            const float x = R[r][q] / m[r];
             float code = 0.f;
-            if (sv[q] != 0.f) code = fminf(fmaxf(rintf(x / sv[q]), -127.f), 127.f);
+            if (sv[q] != 0.f) code = fminf(fmaxf(rintf(X(r, q) / sv[q]), -127.f), 127.f);
             if (ENERGY) {
                 const float dq = (code * sv[q]) * m[r];
                 const double d = (double)R[r][q] - (double)dq;
@@ -266,67 +289,62 @@ __device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, in
             eacc[r] += e;
         } else {
             const int slot = (P > 0) ? map[i] : i;
-            *reinterpret_cast<uint4 *>(out.codes + (size_t)slot * DV + cg * 16) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            uint32_t *dst = reinterpret_cast<uint32_t *>(out.codes + (size_t)slot * DV);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[T::col(cg, q) / 4] = pk[q];
         }
     }
-    __syncthreads();
+    cbar();
 }
 
-// Reconstruct a head's current state into the tile from a staged record:
+// Reconstruct a head's current state into the tile:
 // R = Gamma * ( Deq(C, m, s) [or BF16 rows] + sum_{e<E} ktil_e u_e^T ).
-// stage points at the record prefix in shared memory; gam_s holds Gamma per
-// key row (shared memory, DK floats).  Returns true if every value is finite.
+// The arrays may live in shared or global memory: m_s [DK], s_s [DV],
+// hp_s [P][DV], codes_s [DK-P][DV], ent [E][DK+DV], gam_s [DK].
+// Returns true if every value is finite.
 template <int DK, int DV>
-__device__ __forceinline__ bool tile_from_stage(float (&R)[Tile<DK, DV>::RPT][16], const unsigned char *stage,
-                                                const Layout &L, int P, const int *map, int E,
-                                                const float *gam_s) {
+__device__ __forceinline__ bool tile_reconstruct(float (&R)[Tile<DK, DV>::RPT][16], const float *m_s,
+                                                 const float *s_s, const uint16_t *hp_s, const int8_t *codes_s,
+                                                 const float *ent, int P, const int *map, int E,
+                                                 const float *gam_s) {
     using T = Tile<DK, DV>;
     constexpr int RPT = T::RPT;
     const int t = threadIdx.x, cg = t % T::CG, rg = t / T::CG, row0 = rg * RPT;
-    const float *m_s = reinterpret_cast<const float *>(stage + L.off_m);
-    const float *s_s = reinterpret_cast<const float *>(stage + L.off_s);
-    const uint16_t *hp_s = reinterpret_cast<const uint16_t *>(stage + L.off_hp);
-    const float *ent = reinterpret_cast<const float *>(stage + L.off_ent);
     float sv[16];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float4 f = reinterpret_cast<const float4 *>(s_s + cg * 16)[q];
-        sv[4 * q] = f.x; sv[4 * q + 1] = f.y; sv[4 * q + 2] = f.z; sv[4 * q + 3] = f.w;
-    }
+    load_cols16<DK, DV>(s_s, sv);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         const int i = row0 + r;
         const int mp = (P > 0) ? map[i] : i;
         if (mp >= 0) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(stage + (size_t)mp * DV + cg * 16);
-            const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
             const float mi = m_s[i];
+            const uint32_t *row = reinterpret_cast<const uint32_t *>(codes_s + (size_t)mp * DV);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 float f[4];
-                s8x4_to_f(wd[q], f);
+                s8x4_to_f(row[T::col(cg, q) / 4], f);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) R[r][4 * q + u] = (f[u] * sv[4 * q + u]) * mi;
             }
         } else {
             const int p = -1 - mp;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) R[r][q] = bf16_to_f(hp_s[(size_t)p * DV + cg * 16 + q]);
+            for (int q = 0; q < 4; ++q) {
+                const uint2 h = *reinterpret_cast<const uint2 *>(hp_s + (size_t)p * DV + T::col(cg, q));
+                R[r][4 * q] = bf16_to_f((uint16_t)(h.x & 0xffff));
+                R[r][4 * q + 1] = bf16_to_f((uint16_t)(h.x >> 16));
+                R[r][4 * q + 2] = bf16_to_f((uint16_t)(h.y & 0xffff));
+                R[r][4 * q + 3] = bf16_to_f((uint16_t)(h.y >> 16));
+            }
         }
     }
     for (int e = 0; e < E; ++e) {
         const float *kt = ent + (size_t)e * (DK + DV);
-        const float *ut = kt + DK;
         float kv[RPT];
 #pragma unroll
         for (int r = 0; r < RPT; ++r) kv[r] = kt[row0 + r];
         float uv[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 f = reinterpret_cast<const float4 *>(ut + cg * 16)[q];
-            uv[4 * q] = f.x; uv[4 * q + 1] = f.y; uv[4 * q + 2] = f.z; uv[4 * q + 3] = f.w;
-        }
+        load_cols16<DK, DV>(kt + DK, uv);
 #pragma unroll
         for (int r = 0; r < RPT; ++r)
 #pragma unroll
@@ -343,6 +361,32 @@ __device__ __forceinline__ bool tile_from_stage(float (&R)[Tile<DK, DV>::RPT][16
         }
     }
     return finite;
+}
+
+// Tile <-> row-major [DK][DV] global arrays.
+template <int DK, int DV>
+__device__ __forceinline__ void tile_load_global(float (&R)[Tile<DK, DV>::RPT][16], const float *src) {
+    using T = Tile<DK, DV>;
+    const int t = threadIdx.x, cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(src + (size_t)(row0 + r) * DV + T::col(cg, q)));
+            R[r][4 * q] = f.x; R[r][4 * q + 1] = f.y; R[r][4 * q + 2] = f.z; R[r][4 * q + 3] = f.w;
+        }
+}
+
+template <int DK, int DV>
+__device__ __forceinline__ void tile_store_global(const float (&R)[Tile<DK, DV>::RPT][16], float *dst) {
+    using T = Tile<DK, DV>;
+    const int t = threadIdx.x, cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<float4 *>(dst + (size_t)(row0 + r) * DV + T::col(cg, q)) =
+                make_float4(R[r][4 * q], R[r][4 * q + 1], R[r][4 * q + 2], R[r][4 * q + 3]);
 }
 
 }  // namespace lq

@@ -17,21 +17,21 @@ constexpr int kStatusTimeout = 2;
 
 // ---------------------------------------------------------------------------
 // Per-head record in the workspace (INT8 modes).  One contiguous, 128-byte
-// aligned slab per (batch, head), so that a decode step stages everything it
-// reads for a head -- codes, BF16 rows, m, s, compensators and the buffered
-// tokens -- with ONE bulk copy of the slab's prefix:
-//   codes   int8  [dk-P][dv]        INT8 rows in increasing key-row order
-//   hp      u16   [P][dv]           BF16 rows (order of the head's row list)
+// aligned slab per (batch, head):
 //   m       f32   [dk]              smoothing scale per key row (1 on BF16 rows)
 //   s       f32   [dv]              quantization scale per value column
+//   hp      u16   [P][dv]           BF16 rows (order of the head's row list)
+//   codes   int8  [dk-P][dv]        INT8 rows in increasing key-row order
 //   ent     f32   [r+W][dk+dv]      entry e = (key side [dk], value side [dv]);
 //                                   e < r: compensator (c_e, w_e);
 //                                   r <= e < r+n: buffered token (k/Gamma, u)
 //   gam     f32   [dk] (KDA) / [4] (GDN)   cumulative decay since window start
+// A decode step reads [hp, codes, r+n entries] -- one contiguous byte range --
+// as a stream of bulk copies; m, s are read with the step's small vectors.
 // ---------------------------------------------------------------------------
 struct Layout {
     int dk, dv, P, r, W, kda;
-    int off_hp, off_m, off_s, off_ent, off_gam;
+    int off_m, off_s, off_hp, off_codes, off_ent, off_gam;
     int rec_bytes;
 };
 
@@ -40,20 +40,22 @@ __host__ __device__ inline int align_up(int x, int a) { return (x + a - 1) / a *
 __host__ inline Layout make_layout(int dk, int dv, int P, int r, int W, int kda) {
     Layout L;
     L.dk = dk; L.dv = dv; L.P = P; L.r = r; L.W = W; L.kda = kda;
-    int o = align_up((dk - P) * dv, 16);
-    L.off_hp = o;
-    o = align_up(o + P * dv * 2, 16);
-    L.off_m = o;
-    o += dk * 4;
-    L.off_s = o;
-    o += dv * 4;
-    L.off_ent = align_up(o, 16);
-    o = L.off_ent + (r + W) * (dk + dv) * 4;
+    L.off_m = 0;
+    L.off_s = dk * 4;
+    L.off_hp = (dk + dv) * 4;
+    L.off_codes = L.off_hp + P * dv * 2;
+    L.off_ent = align_up(L.off_codes + (dk - P) * dv, 16);
+    int o = L.off_ent + (r + W) * (dk + dv) * 4;
     L.off_gam = align_up(o, 16);
     o = L.off_gam + (kda ? dk : 4) * 4;
     L.rec_bytes = align_up(o, 128);
     return L;
 }
+
+// Named barrier over the 256 compute threads (warps 0..7) of a CTA; with a
+// 256-thread CTA it is a full barrier, with an extra producer warp it leaves
+// the producer out.
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // PTX wrappers: mbarrier + cp.async.bulk (global -> shared, no multicast).
@@ -139,13 +141,13 @@ __device__ __forceinline__ double warp_sum_d(double v) {
     return v;
 }
 
-// Sum of one double per thread over the CTA; every thread gets the result.
-// `scratch` holds kWarps doubles; the call begins and ends with a barrier.
+// Sum of one double per compute thread (warps 0..7); every compute thread
+// gets the result.  `scratch` holds kWarps doubles; two barriers inside.
 __device__ inline double block_sum_d(double v, double *scratch) {
     v = warp_sum_d(v);
-    __syncthreads();
+    cbar();
     if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
-    __syncthreads();
+    cbar();
     double s = 0.0;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) s += scratch[w];
@@ -164,17 +166,23 @@ __device__ __forceinline__ uint16_t bf16_rne(float x) {
 
 __device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
-// Signed bytes of a 32-bit word -> floats (exact).
+// Signed bytes of a 32-bit word -> floats (exact).  Each byte, offset to
+// unsigned, is placed in the low mantissa byte of 2^23 (bit pattern
+// 0x4B0000xx) with one byte permute, and 2^23 + 128 is subtracted: the
+// integer-to-float bias trick, two ALU operations per value instead of a
+// conversion instruction.
 __device__ __forceinline__ void s8x4_to_f(uint32_t w, float f[4]) {
-    f[0] = (float)(int8_t)(w & 0xff);
-    f[1] = (float)(int8_t)((w >> 8) & 0xff);
-    f[2] = (float)(int8_t)((w >> 16) & 0xff);
-    f[3] = (float)(int8_t)(w >> 24);
+    const uint32_t u = w ^ 0x80808080u;
+    f[0] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u)) - 8388736.0f;
+    f[1] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541u)) - 8388736.0f;
+    f[2] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542u)) - 8388736.0f;
+    f[3] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543u)) - 8388736.0f;
 }
 
 // Build the key-row map of one head in shared memory: map[i] = INT8 slot of
 // row i (rows in increasing order, BF16 rows skipped) or -1-p for the p-th
-// BF16 row.  Needs DK <= kThreads.  Ends with a barrier.
+// BF16 row.  Run by the 256 compute threads; needs DK <= 256.  Ends with a
+// barrier over them.
 template <int DK>
 __device__ inline void build_row_map(const int *hp_rows_h, int P, int *map, int *scratch_w) {
     const int i = threadIdx.x;
@@ -187,11 +195,11 @@ __device__ inline void build_row_map(const int *hp_rows_h, int P, int *map, int 
     const uint32_t bal = __ballot_sync(0xffffffffu, hp);
     const int lane = i & 31, warp = i >> 5;
     if (lane == 0) scratch_w[warp] = __popc(bal);
-    __syncthreads();
+    cbar();
     int before = __popc(bal & ((1u << lane) - 1u));
     for (int w = 0; w < warp; ++w) before += scratch_w[w];
     if (i < DK) map[i] = hp ? (-1 - p_of) : (i - before);
-    __syncthreads();
+    cbar();
 }
 
 }  // namespace lq

@@ -12,66 +12,71 @@
 //   u_t = beta_t (v_t - y_k),   o_t = y_q + u_t (k_t . q_t),
 // and (k_t / Gamma_t, u_t) is appended to the buffer.
 //
-// One CTA per (batch, head).  Thread 0 stages the head's record prefix (codes,
-// BF16 rows, m, s and the r + n buffered entries -- one contiguous range) into
-// shared memory with a single cp.async.bulk; meanwhile the other threads load
-// q, k, v, beta, alpha and form Gamma_t.  The codes are consumed as one 32-bit
-// word (4 columns) per lane and row, a warp covering whole 128-byte rows.
+// Buffering steps run decode_buffer_kernel (one CTA per head, the record head
+// staged by one bulk copy, the buffered entries streamed from global memory);
+// the step that ends a window runs decode_flush_kernel (one CTA per head,
+// state rebuilt in registers and requantized).
 #include "lq_codec.cuh"
 #include "lq_kernels.h"
 
 namespace lq {
 
+// Shared memory of a buffering step (everything but the staged codes).
 template <int DK, int DV>
-struct DecSmem {
-    float2 x2[DK];     // (Gamma*k, Gamma*q)
-    float2 a2[DK];     // (m*Gamma*k, m*Gamma*q) by INT8 slot
-    float k[DK];
-    float gam[DK];
+struct BufSmem {
+    float2 x2[DK];              // (Gamma k, Gamma q) by key row
+    float2 a2[DK];              // m * x2, by INT8 slot
+    float2 red[kWarps][DV];     // per-warp partial column sums
+    int rows[DK];               // DAMP: key row of INT8 slot j, then of BF16 row p
     float v[DV];
-    float2 red[kWarps * (128 / DV)][DV];
-    int map[DK];
-    int wscr[kWarps];
+    float gt[DK];               // Gamma_t (GDN: gt[0])
+    float kk[DK];
     float kqw[kWarps];
-    CodecSmem<DK, DV> cs;
     uint64_t mbar;
 };
 
 template <int DK, int DV>
-__host__ __device__ constexpr size_t dec_fixed_bytes() {
-    return (sizeof(DecSmem<DK, DV>) + 15) / 16 * 16;
+__host__ __device__ constexpr size_t buf_fixed_bytes() {
+    return (sizeof(BufSmem<DK, DV>) + 127) / 128 * 128;
 }
 
-size_t decode_smem_bytes(int dk, int dv, const Layout &L) {
+size_t buffer_smem_bytes(int dk, int dv, const Layout &L) {
     size_t fixed = 0;
-    if (dk == 64 && dv == 64) fixed = dec_fixed_bytes<64, 64>();
-    if (dk == 64 && dv == 128) fixed = dec_fixed_bytes<64, 128>();
-    if (dk == 128 && dv == 64) fixed = dec_fixed_bytes<128, 64>();
-    if (dk == 128 && dv == 128) fixed = dec_fixed_bytes<128, 128>();
-    const size_t stage = (size_t)align_up(L.off_ent + (L.r + L.W) * (L.dk + L.dv) * 4, 16);
-    const size_t dots = (size_t)(L.r + L.W + 1) * sizeof(float2);
-    return stage + fixed + align_up((int)dots, 16);
+    if (dk == 64 && dv == 64) fixed = buf_fixed_bytes<64, 64>();
+    if (dk == 64 && dv == 128) fixed = buf_fixed_bytes<64, 128>();
+    if (dk == 128 && dv == 64) fixed = buf_fixed_bytes<128, 64>();
+    if (dk == 128 && dv == 128) fixed = buf_fixed_bytes<128, 128>();
+    return fixed + (size_t)align_up(L.off_ent, 128);
 }
 
-// Decode one token of one head; FLUSH also ends the window in the same launch.
-template <int DK, int DV, bool KDA, bool FLUSH, bool DAMP>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a) {
+// One buffering token of one head (n < W-1 tokens already buffered, or any n
+// with the flush left to lq_window_flush).  One CTA per head, 256 threads.
+//   * thread 0 stages the record head [m | s | BF16 rows | codes] with one
+//     cp.async.bulk (17 KB at d = 128) into shared memory;
+//   * the r + n buffered entries are read straight from global memory, one
+//     entry per warp (32 lanes x 16 bytes per half), two entries in flight per
+//     warp, while the codes are still arriving;
+//   * codes: one 32-bit word (4 columns) per lane and row, a warp per row.
+// The small footprint (~28 KB of shared memory, <= 64 registers) keeps 4+
+// CTAs resident per SM, which is what hides the load latency.
+template <int DK, int DV, bool KDA, bool DAMP>
+__global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
+    BufSmem<DK, DV> &S = *reinterpret_cast<BufSmem<DK, DV> *>(smem);
+    unsigned char *stage = smem + buf_fixed_bytes<DK, DV>();
     const Layout &L = a.L;
     const int head = blockIdx.x;
-    const int b = head / a.H, h = head - b * a.H;
-    const int g = (h * a.Hk) / a.H;
+    const int b = head / a.H, h = head - b * a.H, g = (h * a.Hk) / a.H;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int P = DAMP ? L.P : 0;
     const int NI = DK - P;
-    const int E = L.r + a.n;  // entries present before this token
-    const size_t stage_bytes = (size_t)align_up(L.off_ent + (L.r + L.W) * (DK + DV) * 4, 16);
-    unsigned char *stage = smem;
-    DecSmem<DK, DV> &S = *reinterpret_cast<DecSmem<DK, DV> *>(smem + stage_bytes);
-    float2 *dots = reinterpret_cast<float2 *>(smem + stage_bytes + dec_fixed_bytes<DK, DV>());
+    const int E = L.r + a.n;
+    const size_t hv = (size_t)b * a.H + h;
     unsigned char *rec = a.rec + (size_t)head * L.rec_bytes;
+    const float *ent_g = reinterpret_cast<const float *>(rec + L.off_ent);
     float *rec_ent = reinterpret_cast<float *>(rec + L.off_ent);
     float *rec_gam = reinterpret_cast<float *>(rec + L.off_gam);
+    constexpr int XPL = DK / 32;   // key elements per lane in an entry's dot product
 
     if (t == 0) {
         mbar_init(&S.mbar, 1);
@@ -79,220 +84,331 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a) {
     }
     __syncthreads();
     if (t == 0) {
-        const uint32_t bytes = (uint32_t)(L.off_ent + E * (DK + DV) * 4);
-        mbar_arrive_expect_tx(&S.mbar, bytes);
-        bulk_g2s(stage, rec, bytes, &S.mbar);
+        mbar_arrive_expect_tx(&S.mbar, (uint32_t)L.off_ent);
+        bulk_g2s(stage, rec, (uint32_t)L.off_ent, &S.mbar);
     }
 
-    // Step inputs and the cumulative gate while the stage is in flight.
-    const size_t hv = (size_t)b * a.H + h;
-    const size_t qk = ((size_t)b * a.Hk + g) * DK;
+    // First two entries of this warp, in flight while the rest is set up.
+    float4 kbuf[2], ubuf[2];
+    float2 kbuf2[2];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        const int e = warp + p * kWarps;
+        if (e < E) {
+            const float *kt = ent_g + (size_t)e * (DK + DV);
+            if (XPL == 4) kbuf[p] = __ldcs(reinterpret_cast<const float4 *>(kt) + lane);
+            else kbuf2[p] = __ldcs(reinterpret_cast<const float2 *>(kt) + lane);
+            if (lane < DV / 4) ubuf[p] = __ldcs(reinterpret_cast<const float4 *>(kt + DK) + lane);
+        }
+    }
+
+    // Step inputs and Gamma_t.
     float kqp = 0.f;
     if (t < DK) {
+        const size_t qk = ((size_t)b * a.Hk + g) * DK;
         const float kk = a.k[qk + t], qq = a.q[qk + t];
-        const float al = KDA ? a.alpha[hv * DK + t] : a.alpha[hv];
-        float gp = 1.0f;
-        if (a.n > 0) gp = KDA ? rec_gam[t] : rec_gam[0];
-        const float gt = al * gp;
-        S.k[t] = kk;
-        S.gam[t] = gt;
+        const float gp = a.n > 0 ? (KDA ? rec_gam[t] : rec_gam[0]) : 1.0f;
+        const float gt = (KDA ? a.alpha[hv * DK + t] : a.alpha[hv]) * gp;
         S.x2[t] = make_float2(gt * kk, gt * qq);
+        S.gt[t] = gt;
+        S.kk[t] = kk;
         kqp = kk * qq;
+        if (DAMP) S.rows[t] = a.slot_rows[(size_t)h * DK + t];
     }
     if (t < DV) S.v[t] = a.v[hv * DV + t];
+    const float beta = a.beta[hv];
     kqp = warp_sum(kqp);
     if (lane == 0) S.kqw[warp] = kqp;
-    if (DAMP) build_row_map<DK>(a.hp_rows + (size_t)h * P, P, S.map, S.wscr);
     __syncthreads();
     float kq = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) kq += S.kqw[w];
+    // This lane's x values for the entry dot products.
+    float xk[XPL], xq[XPL];
+#pragma unroll
+    for (int u = 0; u < XPL; ++u) {
+        const float2 x = S.x2[XPL * lane + u];
+        xk[u] = x.x;
+        xq[u] = x.y;
+    }
 
-    const bool ok = mbar_wait_bounded(&S.mbar, 0, a.status);
-    if (__syncthreads_or(!ok)) return;
-
-    const float *m_s = reinterpret_cast<const float *>(stage + L.off_m);
-    const float *s_s = reinterpret_cast<const float *>(stage + L.off_s);
-    const uint16_t *hp_s = reinterpret_cast<const uint16_t *>(stage + L.off_hp);
-    const float *ent = reinterpret_cast<const float *>(stage + L.off_ent);
-
-    if (t < DK) {
-        const int j = DAMP ? S.map[t] : t;
-        if (j >= 0) {
-            const float mi = m_s[t];
-            const float2 x = S.x2[t];
-            S.a2[j] = make_float2(mi * x.x, mi * x.y);
+    // Entries: y += u_e (ktil_e . x), one warp per entry, loads kept two ahead.
+    float ek[4] = {0.f, 0.f, 0.f, 0.f}, eq[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int e0 = warp; e0 < E; e0 += 2 * kWarps) {
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const int e = e0 + p * kWarps;
+            if (e >= E) break;
+            float dk_, dq_;
+            if (XPL == 4) {
+                const float4 kv = kbuf[p];
+                dk_ = fmaf(kv.x, xk[0], fmaf(kv.y, xk[1 % XPL], fmaf(kv.z, xk[2 % XPL], kv.w * xk[3 % XPL])));
+                dq_ = fmaf(kv.x, xq[0], fmaf(kv.y, xq[1 % XPL], fmaf(kv.z, xq[2 % XPL], kv.w * xq[3 % XPL])));
+            } else {
+                const float2 kv = kbuf2[p];
+                dk_ = fmaf(kv.x, xk[0], kv.y * xk[1 % XPL]);
+                dq_ = fmaf(kv.x, xq[0], kv.y * xq[1 % XPL]);
+            }
+            const float4 uv = ubuf[p];
+            const int en = e + 2 * kWarps;   // refill this slot
+            if (en < E) {
+                const float *kt = ent_g + (size_t)en * (DK + DV);
+                if (XPL == 4) kbuf[p] = __ldcs(reinterpret_cast<const float4 *>(kt) + lane);
+                else kbuf2[p] = __ldcs(reinterpret_cast<const float2 *>(kt) + lane);
+                if (lane < DV / 4) ubuf[p] = __ldcs(reinterpret_cast<const float4 *>(kt + DK) + lane);
+            }
+            dk_ = warp_sum(dk_);
+            dq_ = warp_sum(dq_);
+            if (lane < DV / 4) {
+                ek[0] = fmaf(uv.x, dk_, ek[0]); ek[1] = fmaf(uv.y, dk_, ek[1]);
+                ek[2] = fmaf(uv.z, dk_, ek[2]); ek[3] = fmaf(uv.w, dk_, ek[3]);
+                eq[0] = fmaf(uv.x, dq_, eq[0]); eq[1] = fmaf(uv.y, dq_, eq[1]);
+                eq[2] = fmaf(uv.z, dq_, eq[2]); eq[3] = fmaf(uv.w, dq_, eq[3]);
+            }
         }
     }
-    __syncthreads();
 
-    // Dual GEMV over the INT8 rows.
-    constexpr int LPR = DV / 4;    // lanes per row
-    constexpr int RPP = 32 / LPR;  // rows per warp pass
+    // Codes staged: a = m * x by INT8 slot, then the dual GEMV.
+    const bool ok = mbar_wait_bounded(&S.mbar, 0, a.status);
+    if (__syncthreads_or(!ok)) return;
+    const float *m_s = reinterpret_cast<const float *>(stage + L.off_m);
+    const float *s_s = reinterpret_cast<const float *>(stage + L.off_s);
+    if (t < NI) {
+        const int row = DAMP ? S.rows[t] : t;
+        const float mi = m_s[row];
+        const float2 x = S.x2[row];
+        S.a2[t] = make_float2(mi * x.x, mi * x.y);
+    }
+    __syncthreads();
+    constexpr int LPR = DV / 4, RPP = 32 / LPR;
+    float ak[4] = {0.f, 0.f, 0.f, 0.f}, aq[4] = {0.f, 0.f, 0.f, 0.f};
     {
         const int cq = lane % LPR, rsub = lane / LPR;
-        float ak[4] = {0.f, 0.f, 0.f, 0.f}, aq[4] = {0.f, 0.f, 0.f, 0.f};
+        const unsigned char *codes = stage + L.off_codes;
+#pragma unroll 4
         for (int j = warp * RPP + rsub; j < NI; j += kWarps * RPP) {
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(stage + (size_t)j * DV + cq * 4);
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(codes + (size_t)j * DV + 4 * cq);
+            const float2 av = S.a2[j];
             float f[4];
             s8x4_to_f(w, f);
-            const float2 av = S.a2[j];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 ak[u] = fmaf(f[u], av.x, ak[u]);
                 aq[u] = fmaf(f[u], av.y, aq[u]);
             }
         }
-        float2 *red = S.red[warp * RPP + rsub];
+        if (RPP == 2) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) red[cq * 4 + u] = make_float2(ak[u], aq[u]);
-    }
-    // Buffer / compensator dot products, one warp per entry.
-    for (int e = warp; e < E; e += kWarps) {
-        const float *kt = ent + (size_t)e * (DK + DV);
-        float dk_ = 0.f, dq_ = 0.f;
-#pragma unroll
-        for (int i = lane; i < DK; i += 32) {
-            const float kv = kt[i];
-            const float2 x = S.x2[i];
-            dk_ = fmaf(kv, x.x, dk_);
-            dq_ = fmaf(kv, x.y, dq_);
+            for (int u = 0; u < 4; ++u) {
+                ak[u] += __shfl_xor_sync(0xffffffffu, ak[u], 16);
+                aq[u] += __shfl_xor_sync(0xffffffffu, aq[u], 16);
+            }
         }
-        dk_ = warp_sum(dk_);
-        dq_ = warp_sum(dq_);
-        if (lane == 0) dots[e] = make_float2(dk_, dq_);
+    }
+    if (DAMP) {   // BF16 rows: one per warp, 4 columns per lane, unscaled x
+        const uint16_t *hp = reinterpret_cast<const uint16_t *>(stage + L.off_hp);
+        for (int p = warp; p < P; p += kWarps) {
+            if (lane < DV / 4) {
+                const uint2 hb = *reinterpret_cast<const uint2 *>(hp + (size_t)p * DV + 4 * lane);
+                const float2 x = S.x2[S.rows[NI + p]];
+                const float f0 = bf16_to_f((uint16_t)(hb.x & 0xffff)), f1 = bf16_to_f((uint16_t)(hb.x >> 16));
+                const float f2 = bf16_to_f((uint16_t)(hb.y & 0xffff)), f3 = bf16_to_f((uint16_t)(hb.y >> 16));
+                ek[0] = fmaf(f0, x.x, ek[0]); ek[1] = fmaf(f1, x.x, ek[1]);
+                ek[2] = fmaf(f2, x.x, ek[2]); ek[3] = fmaf(f3, x.x, ek[3]);
+                eq[0] = fmaf(f0, x.y, eq[0]); eq[1] = fmaf(f1, x.y, eq[1]);
+                eq[2] = fmaf(f2, x.y, eq[2]); eq[3] = fmaf(f3, x.y, eq[3]);
+            }
+        }
+    }
+    // Per warp: s * (codes part) + (BF16 rows + entries part); one barrier.
+    if (lane < DV / 4) {
+        const float4 sc = *reinterpret_cast<const float4 *>(s_s + 4 * lane);
+        const float s4[4] = {sc.x, sc.y, sc.z, sc.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            S.red[warp][4 * lane + u] = make_float2(fmaf(s4[u], ak[u], ek[u]), fmaf(s4[u], aq[u], eq[u]));
     }
     __syncthreads();
-
-    // Per value column: finish y_k, y_q; output; the new buffer entry.
-    const int En = E;  // slot of the new entry
     if (t < DV) {
         float yk = 0.f, yq = 0.f;
 #pragma unroll
-        for (int sl = 0; sl < kWarps * RPP; ++sl) {
-            const float2 p = S.red[sl][t];
+        for (int w = 0; w < kWarps; ++w) {
+            const float2 p = S.red[w][t];
             yk += p.x;
             yq += p.y;
         }
-        const float sc = s_s[t];
-        yk *= sc;
-        yq *= sc;
-        if (DAMP) {
-            for (int p = 0; p < P; ++p) {
-                const int i = a.hp_rows[(size_t)h * P + p];
-                const float bv = bf16_to_f(hp_s[(size_t)p * DV + t]);
-                const float2 x = S.x2[i];
-                yk = fmaf(bv, x.x, yk);
-                yq = fmaf(bv, x.y, yq);
-            }
-        }
-        for (int e = 0; e < E; ++e) {
-            const float u = ent[(size_t)e * (DK + DV) + DK + t];
-            const float2 d = dots[e];
-            yk = fmaf(u, d.x, yk);
-            yq = fmaf(u, d.y, yq);
-        }
-        const float beta = a.beta[hv];
         const float ut = beta * (S.v[t] - yk);
         const float o = fmaf(ut, kq, yq);
         a.o[hv * DV + t] = o;
+        rec_ent[(size_t)E * (DK + DV) + DK + t] = ut;
         if (!isfinite(o) || !isfinite(ut)) atomicOr(a.status, kStatusNonFinite);
-        if (FLUSH) {
-            reinterpret_cast<float *>(stage + L.off_ent)[(size_t)En * (DK + DV) + DK + t] = ut;
-        } else {
-            rec_ent[(size_t)En * (DK + DV) + DK + t] = ut;
-        }
     }
     if (t < DK) {
-        const float kt = S.k[t] / S.gam[t];
-        if (FLUSH) {
-            reinterpret_cast<float *>(stage + L.off_ent)[(size_t)En * (DK + DV) + t] = kt;
-        } else {
-            rec_ent[(size_t)En * (DK + DV) + t] = kt;
-            if (KDA) rec_gam[t] = S.gam[t];
-            else if (t == 0) rec_gam[0] = S.gam[0];
-        }
-    }
-    if (!FLUSH) return;
-
-    // ---- window end: reconstruct, re-extract compensators, smooth, pack ----
-    __syncthreads();
-    using T = Tile<DK, DV>;
-    float R[T::RPT][16];
-    const bool fin = tile_from_stage<DK, DV>(R, stage, L, P, DAMP ? S.map : nullptr, E + 1, S.gam);
-    if (!fin) atomicOr(a.status, kStatusNonFinite);
-    CodecOut out;
-    out.codes = reinterpret_cast<int8_t *>(rec);
-    out.hp = reinterpret_cast<uint16_t *>(rec + L.off_hp);
-    out.m = reinterpret_cast<float *>(rec + L.off_m);
-    out.s = reinterpret_cast<float *>(rec + L.off_s);
-    out.ck = rec_ent;
-    out.ck_stride = DK + DV;
-    out.cw = rec_ent + DK;
-    out.cw_stride = DK + DV;
-    double eacc[T::RPT];
-    codec_quantize<DK, DV, false>(R, L.r, a.K, a.smoothing, P, DAMP ? S.map : nullptr, S.cs, out, eacc);
-    if (KDA) {
-        if (t < DK) rec_gam[t] = 1.0f;
-    } else if (t == 0) {
-        rec_gam[0] = 1.0f;
+        rec_ent[(size_t)E * (DK + DV) + t] = S.kk[t] / S.gt[t];
+        if (KDA) rec_gam[t] = S.gt[t];
+        else if (t == 0) rec_gam[0] = S.gt[0];
     }
 }
 
-// Stage a head's record prefix with E entries (used by flush / export).
+// ---------------------------------------------------------------------------
+// Window-end step: one CTA per head.  The record prefix (m, s, BF16 rows,
+// codes, r+n entries) is staged with one bulk copy; the tile
+//   S' = Gamma_t [Deq + sum_e ktil_e u_e^T]
+// is built in registers, the step's outputs come from it (y_k = S'^T k_t,
+// y_q = S'^T q_t), S_t = S' + k_t u_t^T is quantized in place (new
+// compensators, smoothing, codes) and Gamma restarts at 1.
+// kExport instead writes the current state Gamma [Deq + buffer] (no token);
+// kFlushOnly ends the window without a token (lq_window_flush).
+// ---------------------------------------------------------------------------
 template <int DK, int DV>
-__device__ inline bool stage_record(unsigned char *stage, const unsigned char *rec, const Layout &L, int E,
-                                    uint64_t *mbar, int *status) {
-    if (threadIdx.x == 0) {
-        mbar_init(mbar, 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t bytes = (uint32_t)(L.off_ent + E * (DK + DV) * 4);
-        mbar_arrive_expect_tx(mbar, bytes);
-        bulk_g2s(stage, rec, bytes, mbar);
-    }
-    const bool ok = mbar_wait_bounded(mbar, 0, status);
-    return !__syncthreads_or(!ok);
+struct FlushSmem {
+    float k[DK], q[DK], gam[DK];
+    float u[DV];
+    float kqw[kWarps];
+    int map[DK];
+    int wscr[kWarps];
+    CodecSmem<DK, DV> cs;
+    uint64_t mbar;
+};
+
+template <int DK, int DV>
+__host__ __device__ constexpr size_t flush_fixed_bytes() {
+    return (sizeof(FlushSmem<DK, DV>) + 127) / 128 * 128;
 }
 
-// End a window (n >= 1 tokens buffered), or (EXPORT) write the current state.
-template <int DK, int DV, bool KDA, bool DAMP, bool EXPORT>
-__global__ void __launch_bounds__(kThreads) flush_kernel(const DecodeArgs a) {
+size_t flush_smem_bytes(int dk, int dv, const Layout &L) {
+    size_t fixed = 0;
+    if (dk == 64 && dv == 64) fixed = flush_fixed_bytes<64, 64>();
+    if (dk == 64 && dv == 128) fixed = flush_fixed_bytes<64, 128>();
+    if (dk == 128 && dv == 64) fixed = flush_fixed_bytes<128, 64>();
+    if (dk == 128 && dv == 128) fixed = flush_fixed_bytes<128, 128>();
+    return fixed + (size_t)align_up(L.off_ent + (L.r + L.W) * (L.dk + L.dv) * 4, 128);
+}
+
+enum { kFlushStep = 0, kFlushOnly = 1, kExport = 2 };
+
+template <int DK, int DV, bool KDA, bool DAMP, int MODE>
+__global__ void __launch_bounds__(kThreads) decode_flush_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
+    using T = Tile<DK, DV>;
+    FlushSmem<DK, DV> &F = *reinterpret_cast<FlushSmem<DK, DV> *>(smem);
+    unsigned char *stage = smem + flush_fixed_bytes<DK, DV>();
     const Layout &L = a.L;
     const int head = blockIdx.x;
-    const int h = head % a.H;
-    const int t = threadIdx.x;
+    const int b = head / a.H, h = head - b * a.H, g = (h * a.Hk) / a.H;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
     const int P = DAMP ? L.P : 0;
     const int E = L.r + a.n;
-    const size_t stage_bytes = (size_t)align_up(L.off_ent + (L.r + L.W) * (DK + DV) * 4, 16);
-    unsigned char *stage = smem;
-    DecSmem<DK, DV> &S = *reinterpret_cast<DecSmem<DK, DV> *>(smem + stage_bytes);
     unsigned char *rec = a.rec + (size_t)head * L.rec_bytes;
     float *rec_ent = reinterpret_cast<float *>(rec + L.off_ent);
     float *rec_gam = reinterpret_cast<float *>(rec + L.off_gam);
-    if (t < DK) S.gam[t] = (a.n == 0) ? 1.0f : (KDA ? rec_gam[t] : rec_gam[0]);
-    if (DAMP) build_row_map<DK>(a.hp_rows + (size_t)h * P, P, S.map, S.wscr);
-    if (!stage_record<DK, DV>(stage, rec, L, E, &S.mbar, a.status)) return;
-    using T = Tile<DK, DV>;
+    const size_t hv = (size_t)b * a.H + h;
+
+    if (t == 0) {
+        mbar_init(&F.mbar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (t == 0) {
+        const uint32_t bytes = (uint32_t)(L.off_ent + E * (DK + DV) * 4);
+        mbar_arrive_expect_tx(&F.mbar, bytes);
+        bulk_g2s(stage, rec, bytes, &F.mbar);
+    }
+    float kqp = 0.f;
+    if (t < DK) {
+        const float gp = a.n > 0 ? (KDA ? rec_gam[t] : rec_gam[0]) : 1.0f;
+        float gt = gp;
+        if (MODE == kFlushStep) {
+            const size_t qk = ((size_t)b * a.Hk + g) * DK;
+            const float kk = a.k[qk + t], qq = a.q[qk + t];
+            gt = (KDA ? a.alpha[hv * DK + t] : a.alpha[hv]) * gp;
+            F.k[t] = kk;
+            F.q[t] = qq;
+            kqp = kk * qq;
+        }
+        F.gam[t] = gt;
+    }
+    kqp = warp_sum(kqp);
+    if (lane == 0) F.kqw[warp] = kqp;
+    if (DAMP) build_row_map<DK>(a.hp_rows + (size_t)h * P, P, F.map, F.wscr);
+    const bool okw = mbar_wait_bounded(&F.mbar, 0, a.status);
+    if (__syncthreads_or(!okw)) return;
+
     float R[T::RPT][16];
-    const bool fin = tile_from_stage<DK, DV>(R, stage, L, P, DAMP ? S.map : nullptr, E, S.gam);
+    const bool fin = tile_reconstruct<DK, DV>(
+        R, reinterpret_cast<const float *>(stage + L.off_m), reinterpret_cast<const float *>(stage + L.off_s),
+        reinterpret_cast<const uint16_t *>(stage + L.off_hp), reinterpret_cast<const int8_t *>(stage + L.off_codes),
+        reinterpret_cast<const float *>(stage + L.off_ent), P, DAMP ? F.map : nullptr, E, F.gam);
     if (!fin) atomicOr(a.status, kStatusNonFinite);
-    if (EXPORT) {
-        const int cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
-        float *dst = a.S_out + (size_t)head * DK * DV;
-#pragma unroll
-        for (int r = 0; r < T::RPT; ++r)
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                reinterpret_cast<float4 *>(dst + (size_t)(row0 + r) * DV + cg * 16)[q] =
-                    make_float4(R[r][4 * q], R[r][4 * q + 1], R[r][4 * q + 2], R[r][4 * q + 3]);
+
+    if (MODE == kExport) {
+        tile_store_global<DK, DV>(R, a.S_out + (size_t)head * DK * DV);
         return;
     }
+    if (MODE == kFlushStep) {
+        // y_k = S'^T k, y_q = S'^T q over the tile, one barrier.
+        float zk[T::RPT], zq[T::RPT];
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            zk[r] = F.k[row0 + r];
+            zq[r] = F.q[row0 + r];
+        }
+        float acc[2][16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            float x = 0.f, y = 0.f;
+#pragma unroll
+            for (int r = 0; r < T::RPT; ++r) {
+                x = fmaf(R[r][c], zk[r], x);
+                y = fmaf(R[r][c], zq[r], y);
+            }
+#pragma unroll
+            for (int m = T::CG; m < 32; m <<= 1) {
+                x += __shfl_xor_sync(0xffffffffu, x, m);
+                y += __shfl_xor_sync(0xffffffffu, y, m);
+            }
+            acc[0][c] = x;
+            acc[1][c] = y;
+        }
+        float(*rk)[DV] = F.cs.red[0];
+        float(*rq)[DV] = F.cs.red[1];
+        if (lane < T::CG) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                *reinterpret_cast<float4 *>(&rk[warp][T::col(cg, q)]) =
+                    make_float4(acc[0][4 * q], acc[0][4 * q + 1], acc[0][4 * q + 2], acc[0][4 * q + 3]);
+                *reinterpret_cast<float4 *>(&rq[warp][T::col(cg, q)]) =
+                    make_float4(acc[1][4 * q], acc[1][4 * q + 1], acc[1][4 * q + 2], acc[1][4 * q + 3]);
+            }
+        }
+        cbar();
+        if (t < DV) {
+            float yk = 0.f, yq = 0.f, kq = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                yk += rk[w][t];
+                yq += rq[w][t];
+                kq += F.kqw[w];
+            }
+            const float ut = a.beta[hv] * (a.v[hv * DV + t] - yk);
+            const float o = fmaf(ut, kq, yq);
+            a.o[hv * DV + t] = o;
+            F.u[t] = ut;
+            if (!isfinite(o) || !isfinite(ut)) atomicOr(a.status, kStatusNonFinite);
+        }
+        cbar();
+        float uv[16];
+        load_cols16<DK, DV>(F.u, uv);
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const float kk = F.k[row0 + r];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) R[r][c] = fmaf(kk, uv[c], R[r][c]);
+        }
+    }
     CodecOut out;
-    out.codes = reinterpret_cast<int8_t *>(rec);
+    out.codes = reinterpret_cast<int8_t *>(rec + L.off_codes);
     out.hp = reinterpret_cast<uint16_t *>(rec + L.off_hp);
     out.m = reinterpret_cast<float *>(rec + L.off_m);
     out.s = reinterpret_cast<float *>(rec + L.off_s);
@@ -301,7 +417,7 @@ __global__ void __launch_bounds__(kThreads) flush_kernel(const DecodeArgs a) {
     out.cw = rec_ent + DK;
     out.cw_stride = DK + DV;
     double eacc[T::RPT];
-    codec_quantize<DK, DV, false>(R, L.r, a.K, a.smoothing, P, DAMP ? S.map : nullptr, S.cs, out, eacc);
+    codec_quantize<DK, DV, false>(R, L.r, a.K, a.smoothing, P, DAMP ? F.map : nullptr, F.cs, out, eacc);
     if (KDA) {
         if (t < DK) rec_gam[t] = 1.0f;
     } else if (t == 0) {
@@ -319,6 +435,7 @@ __global__ void __launch_bounds__(kThreads) fp32_step_kernel(const Fp32Args a) {
     __shared__ float k_s[DK], q_s[DK], d_s[DK];
     __shared__ float2 red[kWarps * RPP][DV];
     __shared__ float kqw[kWarps];
+    __shared__ float u_s[DV];
     const int head = blockIdx.x;
     const int b = head / a.H, h = head - b * a.H, g = (h * a.Hk) / a.H;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -358,7 +475,6 @@ __global__ void __launch_bounds__(kThreads) fp32_step_kernel(const Fp32Args a) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) red[warp * RPP + rsub][cq * 4 + u] = make_float2(yk[u], yq[u]);
     __syncthreads();
-    __shared__ float u_s[DV];
     if (t < DV) {
         float a_k = 0.f, a_q = 0.f;
 #pragma unroll
@@ -391,6 +507,7 @@ __global__ void __launch_bounds__(kThreads) fp32_step_kernel(const Fp32Args a) {
 // ---------------------------------------------------------------------------
 // Host-side launchers (called from the C ABI).
 // ---------------------------------------------------------------------------
+
 // Raise a kernel's dynamic shared memory limit when a launch first needs more
 // than it was set to.  `done` must be distinct for every kernel, so each
 // launcher below keeps its own.
@@ -402,22 +519,22 @@ static cudaError_t set_smem(K kern, size_t bytes, size_t &done) {
     return e;
 }
 
-template <int DK, int DV, bool KDA, bool FLUSH, bool DAMP>
-static cudaError_t launch_decode_t(const DecodeArgs &a, int heads, cudaStream_t s) {
-    const size_t sm = decode_smem_bytes(DK, DV, a.L);
-    auto kern = decode_kernel<DK, DV, KDA, FLUSH, DAMP>;
-    static size_t done = 0;  // one per instantiation of this launcher
+template <int DK, int DV, bool KDA, bool DAMP>
+static cudaError_t launch_buffer_t(const DecodeArgs &a, int heads, cudaStream_t s) {
+    const size_t sm = buffer_smem_bytes(DK, DV, a.L);
+    auto kern = decode_buffer_kernel<DK, DV, KDA, DAMP>;
+    static size_t done = 0;
     cudaError_t e = set_smem(kern, sm, done);
     if (e != cudaSuccess) return e;
     kern<<<heads, kThreads, sm, s>>>(a);
     return cudaGetLastError();
 }
 
-template <int DK, int DV, bool KDA, bool DAMP, bool EXPORT>
+template <int DK, int DV, bool KDA, bool DAMP, int MODE>
 static cudaError_t launch_flush_t(const DecodeArgs &a, int heads, cudaStream_t s) {
-    const size_t sm = decode_smem_bytes(DK, DV, a.L);
-    auto kern = flush_kernel<DK, DV, KDA, DAMP, EXPORT>;
-    static size_t done = 0;  // one per instantiation of this launcher
+    const size_t sm = flush_smem_bytes(DK, DV, a.L);
+    auto kern = decode_flush_kernel<DK, DV, KDA, DAMP, MODE>;
+    static size_t done = 0;
     cudaError_t e = set_smem(kern, sm, done);
     if (e != cudaSuccess) return e;
     kern<<<heads, kThreads, sm, s>>>(a);
@@ -431,33 +548,24 @@ static cudaError_t launch_flush_t(const DecodeArgs &a, int heads, cudaStream_t s
                                    : FN<128, 64>)
 
 template <int DK, int DV>
-static cudaError_t decode_dispatch(const DecodeArgs &a, int heads, bool kda, bool flush, bool damp,
-                                   cudaStream_t s) {
-    if (kda) {
-        if (flush) return damp ? launch_decode_t<DK, DV, true, true, true>(a, heads, s)
-                               : launch_decode_t<DK, DV, true, true, false>(a, heads, s);
-        return damp ? launch_decode_t<DK, DV, true, false, true>(a, heads, s)
-                    : launch_decode_t<DK, DV, true, false, false>(a, heads, s);
-    }
-    if (flush) return damp ? launch_decode_t<DK, DV, false, true, true>(a, heads, s)
-                           : launch_decode_t<DK, DV, false, true, false>(a, heads, s);
-    return damp ? launch_decode_t<DK, DV, false, false, true>(a, heads, s)
-                : launch_decode_t<DK, DV, false, false, false>(a, heads, s);
+static cudaError_t buffer_dispatch(const DecodeArgs &a, int heads, bool kda, bool damp, cudaStream_t s) {
+    if (kda) return damp ? launch_buffer_t<DK, DV, true, true>(a, heads, s) : launch_buffer_t<DK, DV, true, false>(a, heads, s);
+    return damp ? launch_buffer_t<DK, DV, false, true>(a, heads, s) : launch_buffer_t<DK, DV, false, false>(a, heads, s);
+}
+
+template <int DK, int DV, int MODE>
+static cudaError_t flush_mode_dispatch(const DecodeArgs &a, int heads, bool kda, bool damp, cudaStream_t s) {
+    if (kda) return damp ? launch_flush_t<DK, DV, true, true, MODE>(a, heads, s)
+                         : launch_flush_t<DK, DV, true, false, MODE>(a, heads, s);
+    return damp ? launch_flush_t<DK, DV, false, true, MODE>(a, heads, s)
+                : launch_flush_t<DK, DV, false, false, MODE>(a, heads, s);
 }
 
 template <int DK, int DV>
-static cudaError_t flush_dispatch(const DecodeArgs &a, int heads, bool kda, bool damp, bool exp,
-                                  cudaStream_t s) {
-    if (exp) {
-        if (kda) return damp ? launch_flush_t<DK, DV, true, true, true>(a, heads, s)
-                             : launch_flush_t<DK, DV, true, false, true>(a, heads, s);
-        return damp ? launch_flush_t<DK, DV, false, true, true>(a, heads, s)
-                    : launch_flush_t<DK, DV, false, false, true>(a, heads, s);
-    }
-    if (kda) return damp ? launch_flush_t<DK, DV, true, true, false>(a, heads, s)
-                         : launch_flush_t<DK, DV, true, false, false>(a, heads, s);
-    return damp ? launch_flush_t<DK, DV, false, true, false>(a, heads, s)
-                : launch_flush_t<DK, DV, false, false, false>(a, heads, s);
+static cudaError_t flush_dispatch(const DecodeArgs &a, int heads, bool kda, bool damp, int mode, cudaStream_t s) {
+    if (mode == kFlushStep) return flush_mode_dispatch<DK, DV, kFlushStep>(a, heads, kda, damp, s);
+    if (mode == kFlushOnly) return flush_mode_dispatch<DK, DV, kFlushOnly>(a, heads, kda, damp, s);
+    return flush_mode_dispatch<DK, DV, kExport>(a, heads, kda, damp, s);
 }
 
 template <int DK, int DV>
@@ -469,16 +577,22 @@ static cudaError_t fp32_dispatch(const Fp32Args &a, int heads, bool kda, cudaStr
 
 cudaError_t launch_decode(const DecodeArgs &a, int dk, int dv, int heads, bool kda, bool flush, bool damp,
                           cudaStream_t s) {
-    return LQ_DISPATCH_DKDV(dk, dv, decode_dispatch)(a, heads, kda, flush, damp, s);
+    if (flush) return LQ_DISPATCH_DKDV(dk, dv, flush_dispatch)(a, heads, kda, damp, kFlushStep, s);
+    return LQ_DISPATCH_DKDV(dk, dv, buffer_dispatch)(a, heads, kda, damp, s);
 }
 
 cudaError_t launch_flush(const DecodeArgs &a, int dk, int dv, int heads, bool kda, bool damp, bool exp,
                          cudaStream_t s) {
-    return LQ_DISPATCH_DKDV(dk, dv, flush_dispatch)(a, heads, kda, damp, exp, s);
+    return LQ_DISPATCH_DKDV(dk, dv, flush_dispatch)(a, heads, kda, damp, exp ? kExport : kFlushOnly, s);
 }
 
 cudaError_t launch_fp32_step(const Fp32Args &a, int dk, int dv, int heads, bool kda, cudaStream_t s) {
     return LQ_DISPATCH_DKDV(dk, dv, fp32_dispatch)(a, heads, kda, s);
+}
+
+size_t decode_smem_bytes(int dk, int dv, const Layout &L) {
+    const size_t a = flush_smem_bytes(dk, dv, L), b = buffer_smem_bytes(dk, dv, L);
+    return a > b ? a : b;
 }
 
 }  // namespace lq

@@ -17,6 +17,7 @@ struct DecodeArgs {
     const float *q, *k, *v, *beta, *alpha;
     float *o;
     const int *hp_rows;   // [H][P] (device)
+    const int *slot_rows; // [H][dk] (device): key row of INT8 slot j, then of BF16 row p
     int *status;
     float *S_out;         // export target [heads][dk][dv]
 };

@@ -10,14 +10,16 @@ from tests import gpu_util as U
 
 pytestmark = pytest.mark.gpu
 
-# Codes: bit-exact except 1-LSB flips at rounding ties, on at most 0.01% of
-# entries.  Compensator products: 1e-5 of the state's max magnitude.  Scales m
-# and s: relative 1e-4 -- the residual left after removing compensators of
-# outlier magnitude is up to ~100x smaller than the state, so its FP32
-# rounding (kernel) against double (oracle) is amplified by that ratio.
+# Codes: bit-exact except 1 LSB on at most 0.01% of entries.  Compensator
+# products: 1e-4 of the state's max magnitude -- K = 8 power steps do not
+# converge when the next singular value is close, and the unconverged iterate
+# amplifies FP32 rounding (kernel) against double (oracle) by up to
+# 1/(1 - sigma_{j+1}/sigma_j).  Scales m and s: relative 1e-4 -- the residual
+# left after removing compensators of outlier magnitude is up to ~100x smaller
+# than the state, so its rounding is amplified by that ratio.
 CODE_FLIP_FRAC = 1e-4
 TIE_EPS = 1e-3
-REL = 1e-5
+REL = 1e-4
 SCALE_REL = 1e-4
 
 CASES = [

@@ -102,35 +102,11 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- distributed
 
-def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        backend = "nccl" if torch.cuda.is_available() else "gloo"
-        if torch.cuda.is_available():
-            torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
-        pg = dist
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(0)
-    return world, rank, local, pg
+from quantized_recurrent_state_lq_b200 import dist as D  # noqa: E402
 
-
-def max_over_ranks(x: float, pg) -> float:
-    if pg is None:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
-    pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    return float(t.item())
-
-
-def barrier(pg):
-    if pg is not None:
-        pg.barrier()
+dist_setup = D.setup
+max_over_ranks = D.max_over_ranks
+barrier = D.barrier
 
 
 # ---------------------------------------------------------------- CPU oracle leg
@@ -307,8 +283,7 @@ def run_ours(args, wl, world, rank, pg):
     if rc != lq.LQ_OK:
         raise lq.LqError(rc, "decode status")
 
-    updates = wl.heads * wl.W * args.steps * world
-    value = updates / dt_max
+    value = D.weak_scaling_value(wl.heads * wl.W * args.steps, world, dt_max)
     step_bytes = traffic.window_bytes(wl) * wl.heads
     t_buf, t_flush = kernel_times(r, 2, stream)
     launch_bytes = traffic.nonflush_launch_bytes(wl) * wl.heads
@@ -383,8 +358,7 @@ def main():
         else:
             rc = run_ours(args, wl, world, rank, pg)
     finally:
-        if pg is not None:
-            pg.destroy_process_group()
+        D.teardown(pg)
     return rc
 
 

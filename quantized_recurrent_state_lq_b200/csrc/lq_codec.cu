@@ -30,6 +30,8 @@ __device__ __forceinline__ CodecOut codec_out_of(const QPtrs &q, int head) {
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const CodecArgs a) {
     __shared__ QSmem<DK, DV> sm;
+    extern __shared__ __align__(16) unsigned char dyn[];
+    ExactSmem<DK, DV> &X = *reinterpret_cast<ExactSmem<DK, DV> *>(dyn);
     using T = Tile<DK, DV>;
     const int head = blockIdx.x, h = head % a.H;
     if (a.P > 0) build_row_map<DK>(a.hp_rows + (size_t)h * a.P, a.P, sm.map, sm.wscr);
@@ -37,7 +39,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const CodecArgs a) {
     tile_load_global<DK, DV>(R, a.S_in + (size_t)head * DK * DV);
     const CodecOut out = codec_out_of(a.q, head);
     double eacc[T::RPT];
-    codec_quantize<DK, DV, false>(R, a.r, a.K, a.smoothing, a.P, a.P > 0 ? sm.map : nullptr, sm.cs, out, eacc);
+    codec_quantize_exact<DK, DV, false>(R, a.r, a.K, a.smoothing, a.P, a.P > 0 ? sm.map : nullptr, sm.cs, X, out,
+                                        eacc);
     if (a.q.gam) {
         float *g = reinterpret_cast<float *>(a.q.gam + (size_t)head * a.q.gam_hs);
         for (int i = threadIdx.x; i < a.q.gam_n; i += kThreads) g[i] = 1.0f;
@@ -135,6 +138,8 @@ __global__ void __launch_bounds__(kThreads) qcopy_kernel(const CodecArgs a) {
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads) damp_select_kernel(const CodecArgs a) {
     __shared__ CodecSmem<DK, DV> cs;
+    extern __shared__ __align__(16) unsigned char dyn[];
+    ExactSmem<DK, DV> &X = *reinterpret_cast<ExactSmem<DK, DV> *>(dyn);
     __shared__ double score[DK];
     __shared__ int sel[DK];
     using T = Tile<DK, DV>;
@@ -147,13 +152,13 @@ __global__ void __launch_bounds__(kThreads) damp_select_kernel(const CodecArgs a
     for (int n = 0; n < a.n_states; ++n) {
         float R[T::RPT][16];
         tile_load_global<DK, DV>(R, a.S_in + ((size_t)n * a.H + h) * DK * DV);
-        codec_quantize<DK, DV, true>(R, a.r, a.K, a.smoothing, 0, nullptr, cs, none, eacc);
+        codec_quantize_exact<DK, DV, true>(R, a.r, a.K, a.smoothing, 0, nullptr, cs, X, none, eacc);
     }
     if (cg == 0) {
 #pragma unroll
         for (int r = 0; r < T::RPT; ++r) score[row0 + r] = eacc[r];
     }
-    __syncthreads();
+    cbar();
     if (t < DK) {
         const double E = score[t];
         a.energy[(size_t)h * DK + t] = E;
@@ -189,8 +194,24 @@ __global__ void __launch_bounds__(kThreads) damp_select_kernel(const CodecArgs a
      : ((dk) == 64 && (dv) == 128) ? KERN<64, 128>     \
                                    : KERN<128, 64>)
 
+static size_t exact_bytes(int dk, int dv) {
+    if (dk == 64 && dv == 64) return sizeof(ExactSmem<64, 64>);
+    if (dk == 64 && dv == 128) return sizeof(ExactSmem<64, 128>);
+    if (dk == 128 && dv == 64) return sizeof(ExactSmem<128, 64>);
+    return sizeof(ExactSmem<128, 128>);
+}
+
+template <typename K>
+static cudaError_t allow_smem(K kern, size_t bytes) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 cudaError_t launch_quantize(const CodecArgs &a, int dk, int dv, int heads, cudaStream_t s) {
-    LQ_PICK(dk, dv, quantize_kernel)<<<heads, kThreads, 0, s>>>(a);
+    auto kern = LQ_PICK(dk, dv, quantize_kernel);
+    const size_t sm = exact_bytes(dk, dv);
+    cudaError_t e = allow_smem(kern, sm);
+    if (e != cudaSuccess) return e;
+    kern<<<heads, kThreads, sm, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -205,7 +226,11 @@ cudaError_t launch_qcopy(const CodecArgs &a, int dk, int dv, int heads, cudaStre
 }
 
 cudaError_t launch_damp_select(const CodecArgs &a, int dk, int dv, cudaStream_t s) {
-    LQ_PICK(dk, dv, damp_select_kernel)<<<a.H, kThreads, 0, s>>>(a);
+    auto kern = LQ_PICK(dk, dv, damp_select_kernel);
+    const size_t sm = exact_bytes(dk, dv);
+    cudaError_t e = allow_smem(kern, sm);
+    if (e != cudaSuccess) return e;
+    kern<<<a.H, kThreads, sm, s>>>(a);
     return cudaGetLastError();
 }
 

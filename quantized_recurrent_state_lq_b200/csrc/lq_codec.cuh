@@ -120,22 +120,19 @@ __device__ __forceinline__ void tile_cols_matvec(const float (&R)[Tile<DK, DV>::
     }
 }
 
-// Full codec on the register tile R (destroyed).  `map` is the shared row map
-// (slot >= 0 for INT8 rows, -1-p for BF16 row p); with P == 0 it may be null.
-// ENERGY: instead of writing codes, add sum_c (R - Deq)^2 of the residual to
-// eacc[r] (DAMP calibration); in that mode nothing is written.
-template <int DK, int DV, bool ENERGY>
-__device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, int K, int smoothing, int P,
-                               const int *map, CodecSmem<DK, DV> &cs, const CodecOut &out,
-                               double (&eacc)[Tile<DK, DV>::RPT]) {
+// Step 1 in FP32 on the register tile: R becomes the residual.  (The window
+// flush uses this path; its input is itself an FP32 result.)  With WRITE the
+// compensators go to `out`.  Returns the barrier-buffer index to continue with.
+template <int DK, int DV, bool WRITE>
+__device__ int codec_compensators_fp32(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, int K,
+                                       CodecSmem<DK, DV> &cs, const CodecOut &out) {
     using T = Tile<DK, DV>;
     constexpr int RPT = T::RPT, CG = T::CG;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int cg = t % CG, rg = t / CG;
     const int row0 = rg * RPT;
+    constexpr bool ENERGY = !WRITE;
     int buf = 0;
-
-    // 1. Compensator tokens.
     for (int j = 0; j < r_comp; ++j) {
         float w[16];
         const float w0 = (float)(1.0 / sqrt((double)DV));
@@ -185,6 +182,130 @@ __device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, in
 #pragma unroll
             for (int q = 0; q < 16; ++q) R[r][q] = fmaf(-c[r], w[q], R[r][q]);
     }
+    return buf;
+}
+
+// Double-precision scratch of the exact compensator extraction.
+template <int DK, int DV>
+struct ExactSmem {
+    double R[DK][DV];
+    double z[DK];
+    double w[DV];
+    double part[kThreads];
+    double red[kWarps];
+};
+
+// Step 1 in double, as the oracle computes it: the residual lives in shared
+// memory in double; z = R w / |R w|, w = R^T z / |R^T z| (K times), w and
+// c = R w rounded to float when stored, R <- R - c w^T in double; the float
+// residual comes back into the tile.  Used where the codec's input is an exact
+// FP32 array (lq_quantize_state, lq_state_init, DAMP calibration), so that the
+// compensators -- which decide every code -- agree with the oracle's to double
+// rounding.
+template <int DK, int DV, bool WRITE>
+__device__ void codec_compensators_fp64(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, int K,
+                                        ExactSmem<DK, DV> &X, const CodecOut &out) {
+    using T = Tile<DK, DV>;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
+    constexpr int TPC = kThreads / DV;   // threads per column in R^T z
+    constexpr int RPTC = DK / TPC;       // rows each of them sums
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) X.R[row0 + r][T::col(cg, q) + u] = (double)R[r][4 * q + u];
+    cbar();
+    for (int j = 0; j < r_comp; ++j) {
+        if (t < DV) X.w[t] = 1.0 / sqrt((double)DV);
+        cbar();
+        bool zero = false;
+        for (int it = 0; it < K; ++it) {
+            for (int i = warp; i < DK; i += kWarps) {
+                double acc = 0.0;
+#pragma unroll
+                for (int k = 0; k < DV / 32; ++k) acc = fma(X.R[i][lane + 32 * k], X.w[lane + 32 * k], acc);
+                acc = warp_sum_d(acc);
+                if (lane == 0) X.z[i] = acc;
+            }
+            cbar();
+            const double nz = sqrt(block_sum_d(t < DK ? X.z[t] * X.z[t] : 0.0, X.red));
+            if (nz == 0.0) { zero = true; break; }
+            if (t < DK) X.z[t] = X.z[t] / nz;
+            cbar();
+            {
+                const int c = t % DV, h = t / DV;
+                double acc = 0.0;
+                for (int i = h * RPTC; i < (h + 1) * RPTC; ++i) acc = fma(X.R[i][c], X.z[i], acc);
+                X.part[t] = acc;
+            }
+            cbar();
+            if (t < DV) {
+                double a = 0.0;
+#pragma unroll
+                for (int hh = 0; hh < TPC; ++hh) a += X.part[t + hh * DV];
+                X.w[t] = a;
+            }
+            const double nw = sqrt(block_sum_d(t < DV ? X.w[t] * X.w[t] : 0.0, X.red));
+            if (nw == 0.0) { zero = true; break; }
+            if (t < DV) X.w[t] = X.w[t] / nw;
+            cbar();
+        }
+        if (zero) {
+            if (WRITE) {
+                if (t < DV) out.cw[j * out.cw_stride + t] = 0.f;
+                if (t < DK) out.ck[j * out.ck_stride + t] = 0.f;
+            }
+            cbar();
+            continue;
+        }
+        if (t < DV) {
+            const float wf = (float)X.w[t];
+            X.w[t] = (double)wf;
+            if (WRITE) out.cw[j * out.cw_stride + t] = wf;
+        }
+        cbar();
+        for (int i = warp; i < DK; i += kWarps) {
+            double acc = 0.0;
+#pragma unroll
+            for (int k = 0; k < DV / 32; ++k) acc = fma(X.R[i][lane + 32 * k], X.w[lane + 32 * k], acc);
+            acc = warp_sum_d(acc);
+            if (lane == 0) {
+                const float cf = (float)acc;
+                X.z[i] = (double)cf;
+                if (WRITE) out.ck[j * out.ck_stride + i] = cf;
+            }
+        }
+        cbar();
+        for (int e = t; e < DK * DV; e += kThreads) {
+            const int i = e / DV, c = e % DV;
+            X.R[i][c] -= X.z[i] * X.w[c];
+        }
+        cbar();
+    }
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) R[r][4 * q + u] = (float)X.R[row0 + r][T::col(cg, q) + u];
+    cbar();
+}
+
+// Steps 2-4 on the residual tile R (destroyed).  `map` is the shared row map
+// (slot >= 0 for INT8 rows, -1-p for BF16 row p); with P == 0 it may be null.
+// ENERGY: instead of writing codes, add sum_c (R - Deq)^2 of the residual to
+// eacc[r] (DAMP calibration); in that mode nothing is written.
+template <int DK, int DV, bool ENERGY>
+__device__ void codec_finish(float (&R)[Tile<DK, DV>::RPT][16], int smoothing, int P, const int *map,
+                             CodecSmem<DK, DV> &cs, const CodecOut &out, double (&eacc)[Tile<DK, DV>::RPT],
+                             int buf) {
+    using T = Tile<DK, DV>;
+    constexpr int RPT = T::RPT, CG = T::CG;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int cg = t % CG, rg = t / CG;
+    const int row0 = rg * RPT;
 
     // 2. BF16 rows and 3. smoothing scales; x = R / m in place (ENERGY keeps R).
     float m[RPT];
@@ -295,6 +416,24 @@ __device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, in
         }
     }
     cbar();
+}
+
+// The whole quantizer with the FP32 compensator step (window flush).
+template <int DK, int DV, bool ENERGY>
+__device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, int K, int smoothing, int P,
+                               const int *map, CodecSmem<DK, DV> &cs, const CodecOut &out,
+                               double (&eacc)[Tile<DK, DV>::RPT]) {
+    const int buf = codec_compensators_fp32<DK, DV, !ENERGY>(R, r_comp, K, cs, out);
+    codec_finish<DK, DV, ENERGY>(R, smoothing, P, map, cs, out, eacc, buf);
+}
+
+// The whole quantizer with the double-precision compensator step.
+template <int DK, int DV, bool ENERGY>
+__device__ void codec_quantize_exact(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, int K, int smoothing, int P,
+                                     const int *map, CodecSmem<DK, DV> &cs, ExactSmem<DK, DV> &X,
+                                     const CodecOut &out, double (&eacc)[Tile<DK, DV>::RPT]) {
+    codec_compensators_fp64<DK, DV, !ENERGY>(R, r_comp, K, X, out);
+    codec_finish<DK, DV, ENERGY>(R, smoothing, P, map, cs, out, eacc, 0);
 }
 
 // Reconstruct a head's current state into the tile:

@@ -84,8 +84,18 @@ def rel_inf_rows(a: np.ndarray, ref: np.ndarray, axis=-1) -> np.ndarray:
     return num / np.maximum(den, 1e-30)
 
 
-# Codes bar: bit-exact except 1 LSB on at most 0.01% of the entries compared.
+# Codes bar where both sides quantize the SAME float32 state (lq_quantize_state,
+# lq_state_init): bit-exact except 1 LSB on at most 0.01% of the entries.
 CODE_FLIP_FRAC = 1e-4
+# Codes after a window flush: the GPU quantizes its own FP32 end-of-window
+# state, which differs from the oracle's double-precision one by ~1e-7
+# relative (FP32 buffered updates and reconstruction).  A code can then differ
+# wherever the oracle's x/s lies within that perturbation of a rounding
+# boundary -- after the unconverged power iteration amplifies it by up to
+# 1/(1 - sigma_{j+1}/sigma_j) (measured ~10) and the 127-level scale:
+# 2 * 127 * 1e-7 * 10 * (cancellation of compensators, ~10) ~ 3e-4.  Bar:
+# 1 LSB on at most 0.1% of the entries.
+FLUSH_FLIP_FRAC = 1e-3
 
 
 def compare_codes(gpu: np.ndarray, orc: np.ndarray, ratio: np.ndarray | None, tie_eps: float = 1e-3):
@@ -104,10 +114,10 @@ def compare_codes(gpu: np.ndarray, orc: np.ndarray, ratio: np.ndarray | None, ti
     return out
 
 
-def assert_code_bar(stats: dict, label: str = ""):
+def assert_code_bar(stats: dict, label: str = "", frac: float = CODE_FLIP_FRAC):
     assert stats["max_diff"] <= 1, f"{label}: a code differs by {stats['max_diff']} LSB"
-    assert stats["n"] <= CODE_FLIP_FRAC * stats["total"] + 1, \
-        f"{label}: {stats['n']}/{stats['total']} codes differ (bar {CODE_FLIP_FRAC:.0e})"
+    assert stats["n"] <= frac * stats["total"] + 1, \
+        f"{label}: {stats['n']}/{stats['total']} codes differ (bar {frac:.0e})"
 
 
 def oracle_ratios(cfg: lq.Config, S_heads: np.ndarray, hp_rows_heads) -> np.ndarray:

@@ -125,7 +125,7 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label=""):
           f"flips {stats['flips']}/{stats['codes']} ({stats['at_tie']} at ties)")
     assert stats["out"] < OUT_REL
     assert stats["state"] < STATE_REL
-    U.assert_code_bar({"n": stats["flips"], "total": stats["codes"], "max_diff": 0}, label)
+    U.assert_code_bar({"n": stats["flips"], "total": stats["codes"], "max_diff": 0}, label, U.FLUSH_FLIP_FRAC)
     return stats
 
 

@@ -167,6 +167,30 @@ int lq_dequantize_state(const lq_config *cfg, const lq_qstate_view *in,
                         const int32_t *h_hp_row_ids, float *d_S, void *stream);
 
 /*
+ * lq_quantize_state without any device allocation (the method's pages have no
+ * counterpart to this call; it exists for callers of this library).
+ *
+ * lq_quantize_state keeps the BF16 row list on the device in a temporary it
+ * allocates on `stream`.  Some callers cannot let a library allocate: engines
+ * whose allocator owns all device memory (it is reserved up front, and an
+ * outside cudaMallocAsync would fail or fragment it) and processes that must
+ * not allocate after start-up.  This variant is the same computation with the
+ * row list held in a fixed array of LQ_STATIC_ROWS_MAX int32 values compiled
+ * into the library (a file-scope __device__ array, present on every GPU that
+ * loads the library until the process exits).  Same arguments, results and
+ * errors as lq_quantize_state, plus:
+ *  - LQ_ERR_UNSUPPORTED when H * n_hp_rows > LQ_STATIC_ROWS_MAX;
+ *  - the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture;
+ *  - every call, on every stream, shares the one array and overwrites it:
+ *    calls that overlap on the GPU race with each other.
+ */
+#define LQ_STATIC_ROWS_MAX 8192
+int lq_quantize_state_static(const lq_config *cfg, const float *d_S, const int32_t *h_hp_row_ids,
+                             lq_qstate_view *out, void *stream);
+
+/*
  * DAMP channel risk (offline calibration; DAMP abstract: error energy and
  * decay-based persistence pick the high-risk channels).  For each head h:
  *   E[h,i]  = sum_n sum_c (R - Deq(R))_ic^2 over the n_states FP32 states

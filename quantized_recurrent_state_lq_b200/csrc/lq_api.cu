@@ -352,6 +352,55 @@ int lq_quantize_state(const lq_config *cfg, const float *d_S, const int32_t *h_h
     return rc;
 }
 
+// Row lists of lq_quantize_state_static: a fixed device array instead of a
+// per-call allocation.  Host code must not use the symbol itself as a device
+// address; the address is looked up once per device with that device current.
+static __device__ __align__(256) int32_t g_static_rows[LQ_STATIC_ROWS_MAX];
+
+static int static_rows_ptr(int32_t **out) {
+    constexpr int kMaxDev = 64;
+    static int32_t *ptr[kMaxDev] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return LQ_ERR_CUDA;
+    if (!ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_rows) != cudaSuccess || !p) return LQ_ERR_CUDA;
+        ptr[dev] = static_cast<int32_t *>(p);
+    }
+    *out = ptr[dev];
+    return LQ_OK;
+}
+
+int lq_quantize_state_static(const lq_config *cfg, const float *d_S, const int32_t *h_hp_row_ids,
+                             lq_qstate_view *out, void *stream) {
+    if (!d_S || (reinterpret_cast<uintptr_t>(d_S) % 16)) return LQ_ERR_INVALID_ARG;
+    if (!cfg) return LQ_ERR_INVALID_ARG;
+    int rc = check_view(cfg, out);
+    if (rc) return rc;
+    if (cfg->B < 1 || cfg->H < 1) return LQ_ERR_SHAPE;
+    rc = check_codec_fields(cfg);
+    if (rc) return rc;
+    rc = check_hp_rows(cfg, h_hp_row_ids);
+    if (rc) return rc;
+    if ((long long)cfg->H * cfg->n_hp_rows > LQ_STATIC_ROWS_MAX) return LQ_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    lq::CodecArgs a{};
+    a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing; a.P = cfg->n_hp_rows;
+    if (cfg->n_hp_rows > 0) {
+        int32_t *rows = nullptr;
+        rc = static_rows_ptr(&rows);
+        if (rc) return rc;
+        // Every entry the kernel reads is written here; nothing needs clearing.
+        if (cudaMemcpyAsync(rows, h_hp_row_ids, (size_t)cfg->H * cfg->n_hp_rows * 4, cudaMemcpyHostToDevice, s) !=
+            cudaSuccess)
+            return LQ_ERR_CUDA;
+        a.hp_rows = rows;
+    }
+    a.S_in = d_S;
+    a.q = view_ptrs(cfg, out);
+    return cuda_rc(lq::launch_quantize(a, cfg->dk, cfg->dv, cfg->B * cfg->H, s));
+}
+
 int lq_dequantize_state(const lq_config *cfg, const lq_qstate_view *in, const int32_t *h_hp_row_ids, float *d_S,
                         void *stream) {
     if (!d_S || (reinterpret_cast<uintptr_t>(d_S) % 16)) return LQ_ERR_INVALID_ARG;

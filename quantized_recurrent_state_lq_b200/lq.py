@@ -32,8 +32,8 @@ LQ_MODE_FP32, LQ_MODE_INT8_STEP, LQ_MODE_INT8_WINDOW = 0, 1, 2
 EXPORTED = ["lq_workspace_bytes", "lq_config_check", "lq_state_init", "lq_decode_step",
             "lq_window_flush", "lq_state_buffered", "lq_state_export_fp32",
             "lq_state_export_view", "lq_state_import_view", "lq_quantize_state",
-            "lq_dequantize_state", "lq_damp_select", "lq_get_status", "lq_state_destroy",
-            "lq_strerror"]
+            "lq_dequantize_state", "lq_quantize_state_static", "lq_damp_select", "lq_get_status",
+            "lq_state_destroy", "lq_strerror"]
 
 
 class LqError(RuntimeError):
@@ -78,6 +78,7 @@ def lib():
             "lq_state_import_view": (C.c_int, [vp, viewp, vp]),
             "lq_quantize_state": (C.c_int, [cfgp, vp, vp, viewp, vp]),
             "lq_dequantize_state": (C.c_int, [cfgp, viewp, vp, vp, vp]),
+            "lq_quantize_state_static": (C.c_int, [cfgp, vp, vp, viewp, vp]),
             "lq_damp_select": (C.c_int, [cfgp, i32, vp, i32, vp, vp, vp, vp]),
             "lq_get_status": (C.c_int, [vp, vp]),
             "lq_state_destroy": (None, [vp]),
@@ -265,6 +266,21 @@ def lq_quantize_state(cfg: Config, S: torch.Tensor, view: dict, hp_rows=None, st
     v = _view_struct(cfg, view)
     _chk(lib().lq_quantize_state(C.byref(cfg.c()), C.c_void_p(p), p_rows, C.byref(v),
                                  C.c_void_p(_stream(stream))), "lq_quantize_state")
+
+
+LQ_STATIC_ROWS_MAX = 8192
+
+
+def lq_quantize_state_static(cfg: Config, S: torch.Tensor, view: dict, hp_rows=None, stream=None):
+    """lq_quantize_state for callers that must not let the library allocate
+    device memory: the BF16 row list goes to a fixed array inside liblq.so
+    (at most LQ_STATIC_ROWS_MAX = H * n_hp_rows entries) instead of a per-call
+    temporary.  Calls that overlap on the GPU share that array and race."""
+    p = _dev(S, "S", (cfg.B, cfg.H, cfg.dk, cfg.dv))
+    rows, p_rows = _host_rows(cfg, hp_rows)
+    v = _view_struct(cfg, view)
+    _chk(lib().lq_quantize_state_static(C.byref(cfg.c()), C.c_void_p(p), p_rows, C.byref(v),
+                                        C.c_void_p(_stream(stream))), "lq_quantize_state_static")
 
 
 def lq_dequantize_state(cfg: Config, view: dict, S: torch.Tensor, hp_rows=None, stream=None):

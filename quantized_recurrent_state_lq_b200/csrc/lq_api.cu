@@ -98,7 +98,7 @@ lq::QPtrs record_ptrs(const lq_state *st) {
     const Layout &L = st->L;
     lq::QPtrs q{};
     const size_t hs = (size_t)L.rec_bytes;
-    q.codes = st->rec + L.off_codes; q.codes_hs = hs;
+    q.codes = st->rec + L.off_codes; q.codes_hs = hs; q.codes_t = L.P == 0 ? 1 : 0;
     q.hp = st->rec + L.off_hp; q.hp_hs = hs;
     q.m = st->rec + L.off_m; q.m_hs = hs;
     q.s = st->rec + L.off_s; q.s_hs = hs;

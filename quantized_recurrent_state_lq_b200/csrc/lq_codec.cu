@@ -17,6 +17,7 @@ struct QSmem {
 __device__ __forceinline__ CodecOut codec_out_of(const QPtrs &q, int head) {
     CodecOut o;
     o.codes = reinterpret_cast<int8_t *>(q.codes + (size_t)head * q.codes_hs);
+    o.codes_t = q.codes_t;
     o.hp = reinterpret_cast<uint16_t *>(q.hp ? q.hp + (size_t)head * q.hp_hs : nullptr);
     o.m = reinterpret_cast<float *>(q.m + (size_t)head * q.m_hs);
     o.s = reinterpret_cast<float *>(q.s + (size_t)head * q.s_hs);
@@ -99,11 +100,19 @@ __global__ void __launch_bounds__(kThreads) qcopy_kernel(const CodecArgs a) {
     const int head = blockIdx.x, t = threadIdx.x;
     const QPtrs &x = a.q, &y = a.q2;
     const int P = a.P;
-    {
+    if (x.codes_t == y.codes_t) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x.codes + (size_t)head * x.codes_hs);
         uint4 *dst = reinterpret_cast<uint4 *>(y.codes + (size_t)head * y.codes_hs);
         const int n16 = (DK - P) * DV / 16;
         for (int e = t; e < n16; e += kThreads) dst[e] = src[e];
+    } else {   // row-major view <-> column-major swizzled record (P == 0)
+        const int8_t *src = reinterpret_cast<const int8_t *>(x.codes + (size_t)head * x.codes_hs);
+        int8_t *dst = reinterpret_cast<int8_t *>(y.codes + (size_t)head * y.codes_hs);
+        for (int e = t; e < DK * DV; e += kThreads) {
+            const int i = e / DV, c = e % DV;
+            const int rm = i * DV + c, cm = code_off_t(c, i, DK);
+            dst[y.codes_t ? cm : rm] = src[x.codes_t ? cm : rm];
+        }
     }
     if (P > 0) {
         const uint16_t *src = reinterpret_cast<const uint16_t *>(x.hp + (size_t)head * x.hp_hs);

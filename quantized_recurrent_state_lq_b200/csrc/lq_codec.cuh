@@ -48,7 +48,8 @@ struct CodecSmem {
 
 // Where the codec writes one head's quantized state.
 struct CodecOut {
-    int8_t *codes;     // [(DK-P)][DV]
+    int8_t *codes;     // [(DK-P)][DV] by slot, or (codes_t) value-column-major, swizzled
+    int codes_t;       // 1: code_off_t layout (no BF16 rows); 0: row-major by INT8 slot
     uint16_t *hp;      // [P][DV]
     float *m;          // [DK]
     float *s;          // [DV]
@@ -386,6 +387,9 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV>::RPT][16], int smoothing, i
     // Codes (or the error energy of the INT8 reconstruction).
     float sv[16];
     load_cols16<DK, DV>(cs.sc, sv);
+    uint32_t tpk[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) tpk[c] = 0u;
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         if (!int8row[r]) continue;
@@ -408,12 +412,32 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV>::RPT][16], int smoothing, i
 #pragma unroll
             for (int mm = CG / 2; mm >= 1; mm >>= 1) e += __shfl_xor_sync(0xffffffffu, e, mm);
             eacc[r] += e;
+        } else if (out.codes_t) {
+            // value-column-major: gather this thread's RPT consecutive rows of each column
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) tpk[4 * q + u] |= ((pk[q] >> (8 * u)) & 0xffu) << (8 * r);
         } else {
             const int slot = (P > 0) ? map[i] : i;
             uint32_t *dst = reinterpret_cast<uint32_t *>(out.codes + (size_t)slot * DV);
 #pragma unroll
             for (int q = 0; q < 4; ++q) dst[T::col(cg, q) / 4] = pk[q];
         }
+    }
+    if (!ENERGY && out.codes_t) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                int8_t *dst = out.codes + code_off_t(T::col(cg, q) + u, row0, DK);
+                if (RPT == 4) {
+                    *reinterpret_cast<uint32_t *>(dst) = tpk[4 * q + u];
+                } else {
+#pragma unroll
+                    for (int r = 0; r < RPT; ++r) dst[r] = (int8_t)((tpk[4 * q + u] >> (8 * r)) & 0xffu);
+                }
+            }
     }
     cbar();
 }
@@ -445,7 +469,7 @@ template <int DK, int DV>
 __device__ __forceinline__ bool tile_reconstruct(float (&R)[Tile<DK, DV>::RPT][16], const float *m_s,
                                                  const float *s_s, const uint16_t *hp_s, const int8_t *codes_s,
                                                  const float *ent, int P, const int *map, int E,
-                                                 const float *gam_s) {
+                                                 const float *gam_s, bool codes_t) {
     using T = Tile<DK, DV>;
     constexpr int RPT = T::RPT;
     const int t = threadIdx.x, cg = t % T::CG, rg = t / T::CG, row0 = rg * RPT;
@@ -455,7 +479,16 @@ __device__ __forceinline__ bool tile_reconstruct(float (&R)[Tile<DK, DV>::RPT][1
     for (int r = 0; r < RPT; ++r) {
         const int i = row0 + r;
         const int mp = (P > 0) ? map[i] : i;
-        if (mp >= 0) {
+        if (mp >= 0 && codes_t) {
+            const float mi = m_s[i];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float cf = (float)codes_s[code_off_t(T::col(cg, q) + u, i, DK)];
+                    R[r][4 * q + u] = (cf * sv[4 * q + u]) * mi;
+                }
+        } else if (mp >= 0) {
             const float mi = m_s[i];
             const uint32_t *row = reinterpret_cast<const uint32_t *>(codes_s + (size_t)mp * DV);
 #pragma unroll

@@ -52,6 +52,18 @@ __host__ inline Layout make_layout(int dk, int dv, int P, int r, int W, int kda)
     return L;
 }
 
+// INT8 codes without BF16 rows are stored value-column-major (row c holds the
+// dk codes of value column c) so that they are the row-major A operand of an
+// int8 tensor-core MMA over the key dimension; 16-byte chunks are XOR-swizzled
+// by the column so that 8 consecutive columns read with ldmatrix hit 8
+// different shared-memory bank groups.  With BF16 rows the codes stay
+// row-major by INT8 slot: [slot][c].
+__host__ __device__ __forceinline__ int code_swz(int c, int dk) { return dk >= 128 ? (c & 7) : ((c >> 1) & 3); }
+
+__host__ __device__ __forceinline__ int code_off_t(int c, int i, int dk) {
+    return c * dk + ((((i >> 4) ^ code_swz(c, dk)) << 4) | (i & 15));
+}
+
 // Named barrier over the 256 compute threads (warps 0..7) of a CTA; with a
 // 256-thread CTA it is a full barrier, with an extra producer warp it leaves
 // the producer out.

@@ -12,8 +12,9 @@
 //   u_t = beta_t (v_t - y_k),   o_t = y_q + u_t (k_t . q_t),
 // and (k_t / Gamma_t, u_t) is appended to the buffer.
 //
-// Buffering steps run decode_buffer_kernel (one CTA per head, the record head
-// staged by one bulk copy, the buffered entries streamed from global memory);
+// Buffering steps run decode_buffer_kernel (one CTA per head, four per SM: the
+// codes staged by one bulk copy and multiplied on the int8 tensor cores, the
+// buffered entries streamed from global memory);
 // the step that ends a window runs decode_flush_kernel (one CTA per head,
 // state rebuilt in registers and requantized).
 #include "lq_codec.cuh"
@@ -21,16 +22,32 @@
 
 namespace lq {
 
-// Shared memory of a buffering step (everything but the staged codes).
+// ---------------------------------------------------------------------------
+// Buffering step: one CTA of 8 warps per head, small enough (<= 64 registers,
+// ~30 KB of shared memory) for four CTAs per SM, so that the phases of four
+// heads interleave on each SM:
+//   * thread 0 stages the record head [m | s | BF16 rows | codes] (17 KB at
+//     d = 128) with one cp.async.bulk; every warp loads the first pair of its
+//     buffered entries into registers; the small step vectors are read.
+//   (a) x = Gamma_t (k, q), a = m * x; the per-vector maxima of |a|.   barrier
+//   (b) a_k, a_q as exact signed base-256 digits (4 each): the B operand.  barrier
+//   (c) codes: int8 tensor-core MMA (m16n8k32) of the value-column-major code
+//       tile with the digits, one warp per 16 value columns -- while the
+//       entry pairs are still arriving.  (With BF16 rows: SIMT, a warp per row.)
+//   (d) entries: pairs of entries per warp, the next pair prefetched, dot
+//       products reduced by a transpose-reduce butterfly.
+//   (e) per-warp partial column sums combined; output, append.           barrier
+// ---------------------------------------------------------------------------
 template <int DK, int DV>
 struct BufSmem {
-    float2 x2[DK];              // (Gamma k, Gamma q) by key row
-    float2 a2[DK];              // m * x2, by INT8 slot
-    float2 red[kWarps][DV];     // per-warp partial column sums
-    int rows[DK];               // DAMP: key row of INT8 slot j, then of BF16 row p
+    float2 x2[DK];                      // (Gamma k, Gamma q) by key row
+    float2 a2[DK];                      // m * x2 by INT8 slot (BF16-row layout)
+    float2 red[kWarps][DV];             // per-warp partial column sums (BF16 rows + entries)
+    float2 rc[DV];                      // codes part of (y_k, y_q)
+    int8_t dig[8][DK + 16];             // base-256 digits of a_k (rows 0-3) and a_q (rows 4-7)
+    int rows[DK];                       // DAMP: key row of INT8 slot j, then of BF16 row p
     float v[DV];
-    float gt[DK];               // Gamma_t (GDN: gt[0])
-    float kk[DK];
+    float amax[kWarps][2];
     float kqw[kWarps];
     uint64_t mbar;
 };
@@ -49,16 +66,51 @@ size_t buffer_smem_bytes(int dk, int dv, const Layout &L) {
     return fixed + (size_t)align_up(L.off_ent, 128);
 }
 
-// One buffering token of one head (n < W-1 tokens already buffered, or any n
-// with the flush left to lq_window_flush).  One CTA per head, 256 threads.
-//   * thread 0 stages the record head [m | s | BF16 rows | codes] with one
-//     cp.async.bulk (17 KB at d = 128) into shared memory;
-//   * the r + n buffered entries are read straight from global memory, one
-//     entry per warp (32 lanes x 16 bytes per half), two entries in flight per
-//     warp, while the codes are still arriving;
-//   * codes: one 32-bit word (4 columns) per lane and row, a warp per row.
-// The small footprint (~28 KB of shared memory, <= 64 registers) keeps 4+
-// CTAs resident per SM, which is what hides the load latency.
+// Sum V = 2 NE values (v[2e] = dot_k of entry e, v[2e+1] = dot_q) over the
+// warp: a transpose-reduce butterfly leaves each value's total in one lane
+// group (log2(V) halving steps, then plain steps), then every lane fetches all
+// V totals -- about V + 5 shuffles instead of 5 V.
+template <int NE>
+__device__ __forceinline__ void warp_reduce_dots(float (&v)[2 * NE]) {
+    constexpr int V = 2 * NE;
+    const int lane = threadIdx.x & 31;
+    float cur[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) cur[i] = v[i];
+    int n = V;
+    int mask = 16;
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        if (n > 1) {
+            const bool upper = (lane & mask) != 0;
+            const int h = n / 2;
+#pragma unroll
+            for (int i = 0; i < V / 2; ++i) {
+                if (i < h) {
+                    const float send = upper ? cur[i] : cur[i + h];
+                    const float keep = upper ? cur[i + h] : cur[i];
+                    cur[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+                }
+            }
+            n = h;
+        } else {
+            cur[0] += __shfl_xor_sync(0xffffffffu, cur[0], mask);
+        }
+        mask >>= 1;
+    }
+    // value i ended in the lanes whose top log2(V) bits (from bit 4 down) spell i
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        int src = 0, bit = 16;
+#pragma unroll
+        for (int k = V / 2; k >= 1; k >>= 1) {
+            if (i & k) src |= bit;
+            bit >>= 1;
+        }
+        v[i] = __shfl_sync(0xffffffffu, cur[0], src);
+    }
+}
+
 template <int DK, int DV, bool KDA, bool DAMP>
 __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -76,7 +128,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
     const float *ent_g = reinterpret_cast<const float *>(rec + L.off_ent);
     float *rec_ent = reinterpret_cast<float *>(rec + L.off_ent);
     float *rec_gam = reinterpret_cast<float *>(rec + L.off_gam);
-    constexpr int XPL = DK / 32;   // key elements per lane in an entry's dot product
+    constexpr int XPL = DK / 32;                 // key elements per lane in a dot product
+    constexpr int EF = DK + DV;                  // floats per entry
 
     if (t == 0) {
         mbar_init(&S.mbar, 1);
@@ -88,103 +141,145 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
         bulk_g2s(stage, rec, (uint32_t)L.off_ent, &S.mbar);
     }
 
-    // First two entries of this warp, in flight while the rest is set up.
-    float4 kbuf[2], ubuf[2];
-    float2 kbuf2[2];
+    // Entry pairs of this warp: entries 2 warp + 16 j + {0, 1}.
+    float4 kb[2], ub[2];
+    float2 kb2[2];
+    auto load_pair = [&](int e0) {
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
-        const int e = warp + p * kWarps;
-        if (e < E) {
-            const float *kt = ent_g + (size_t)e * (DK + DV);
-            if (XPL == 4) kbuf[p] = __ldcs(reinterpret_cast<const float4 *>(kt) + lane);
-            else kbuf2[p] = __ldcs(reinterpret_cast<const float2 *>(kt) + lane);
-            if (lane < DV / 4) ubuf[p] = __ldcs(reinterpret_cast<const float4 *>(kt + DK) + lane);
+        for (int p = 0; p < 2; ++p) {
+            const int e = e0 + p;
+            if (e < E) {
+                const float *kt = ent_g + (size_t)e * EF;
+                if (XPL == 4) kb[p] = __ldcs(reinterpret_cast<const float4 *>(kt) + lane);
+                else kb2[p] = __ldcs(reinterpret_cast<const float2 *>(kt) + lane);
+                if (lane < DV / 4) ub[p] = __ldcs(reinterpret_cast<const float4 *>(kt + DK) + lane);
+            }
         }
-    }
+    };
+    load_pair(2 * warp);
 
-    // Step inputs and Gamma_t.
-    float kqp = 0.f;
+    // (a) step inputs, Gamma_t, x, a = m * x.
+    float kqp = 0.f, gt = 1.f, kk = 0.f, ak_t = 0.f, aq_t = 0.f;
     if (t < DK) {
         const size_t qk = ((size_t)b * a.Hk + g) * DK;
-        const float kk = a.k[qk + t], qq = a.q[qk + t];
+        kk = a.k[qk + t];
+        const float qq = a.q[qk + t];
         const float gp = a.n > 0 ? (KDA ? rec_gam[t] : rec_gam[0]) : 1.0f;
-        const float gt = (KDA ? a.alpha[hv * DK + t] : a.alpha[hv]) * gp;
-        S.x2[t] = make_float2(gt * kk, gt * qq);
-        S.gt[t] = gt;
-        S.kk[t] = kk;
+        gt = (KDA ? a.alpha[hv * DK + t] : a.alpha[hv]) * gp;
+        const float2 x = make_float2(gt * kk, gt * qq);
+        S.x2[t] = x;
         kqp = kk * qq;
-        if (DAMP) S.rows[t] = a.slot_rows[(size_t)h * DK + t];
+        if (!DAMP) {
+            const float mi = reinterpret_cast<const float *>(rec + L.off_m)[t];
+            ak_t = mi * x.x;
+            aq_t = mi * x.y;
+        } else {
+            S.rows[t] = a.slot_rows[(size_t)h * DK + t];
+        }
     }
     if (t < DV) S.v[t] = a.v[hv * DV + t];
     const float beta = a.beta[hv];
     kqp = warp_sum(kqp);
+    if (!DAMP) {
+        float mk = fabsf(ak_t), mq = fabsf(aq_t);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+            mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+        }
+        if (lane == 0) {
+            S.amax[warp][0] = mk;
+            S.amax[warp][1] = mq;
+        }
+    }
     if (lane == 0) S.kqw[warp] = kqp;
     __syncthreads();
     float kq = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) kq += S.kqw[w];
-    // This lane's x values for the entry dot products.
-    float xk[XPL], xq[XPL];
-#pragma unroll
-    for (int u = 0; u < XPL; ++u) {
-        const float2 x = S.x2[XPL * lane + u];
-        xk[u] = x.x;
-        xq[u] = x.y;
-    }
 
-    // Entries: y += u_e (ktil_e . x), one warp per entry, loads kept two ahead.
-    float ek[4] = {0.f, 0.f, 0.f, 0.f}, eq[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int e0 = warp; e0 < E; e0 += 2 * kWarps) {
+    // (b) the tensor-core operand: a_k, a_q as exact signed base-256 digits of
+    // one fixed-point integer each, X = a * 2^(30 - e) with |a| < 2^e.
+    int ek_ = 0, eq_ = 0;
+    if (!DAMP) {
+        float mk = 0.f, mq = 0.f;
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const int e = e0 + p * kWarps;
-            if (e >= E) break;
-            float dk_, dq_;
-            if (XPL == 4) {
-                const float4 kv = kbuf[p];
-                dk_ = fmaf(kv.x, xk[0], fmaf(kv.y, xk[1 % XPL], fmaf(kv.z, xk[2 % XPL], kv.w * xk[3 % XPL])));
-                dq_ = fmaf(kv.x, xq[0], fmaf(kv.y, xq[1 % XPL], fmaf(kv.z, xq[2 % XPL], kv.w * xq[3 % XPL])));
-            } else {
-                const float2 kv = kbuf2[p];
-                dk_ = fmaf(kv.x, xk[0], kv.y * xk[1 % XPL]);
-                dq_ = fmaf(kv.x, xq[0], kv.y * xq[1 % XPL]);
-            }
-            const float4 uv = ubuf[p];
-            const int en = e + 2 * kWarps;   // refill this slot
-            if (en < E) {
-                const float *kt = ent_g + (size_t)en * (DK + DV);
-                if (XPL == 4) kbuf[p] = __ldcs(reinterpret_cast<const float4 *>(kt) + lane);
-                else kbuf2[p] = __ldcs(reinterpret_cast<const float2 *>(kt) + lane);
-                if (lane < DV / 4) ubuf[p] = __ldcs(reinterpret_cast<const float4 *>(kt + DK) + lane);
-            }
-            dk_ = warp_sum(dk_);
-            dq_ = warp_sum(dq_);
-            if (lane < DV / 4) {
-                ek[0] = fmaf(uv.x, dk_, ek[0]); ek[1] = fmaf(uv.y, dk_, ek[1]);
-                ek[2] = fmaf(uv.z, dk_, ek[2]); ek[3] = fmaf(uv.w, dk_, ek[3]);
-                eq[0] = fmaf(uv.x, dq_, eq[0]); eq[1] = fmaf(uv.y, dq_, eq[1]);
-                eq[2] = fmaf(uv.z, dq_, eq[2]); eq[3] = fmaf(uv.w, dq_, eq[3]);
+        for (int w = 0; w < kWarps; ++w) {
+            mk = fmaxf(mk, S.amax[w][0]);
+            mq = fmaxf(mq, S.amax[w][1]);
+        }
+        frexpf(mk, &ek_);
+        frexpf(mq, &eq_);
+        ek_ = max(ek_, -96);
+        eq_ = max(eq_, -96);
+        if (t < DK) {
+            const int xs[2] = {(int)rintf(ak_t * ldexpf(1.0f, 30 - ek_)), (int)rintf(aq_t * ldexpf(1.0f, 30 - eq_))};
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+                int X = xs[v];
+#pragma unroll
+                for (int dgt = 0; dgt < 3; ++dgt) {
+                    const int d = ((X + 128) & 255) - 128;
+                    S.dig[4 * v + dgt][t] = (int8_t)d;
+                    X = (X - d) >> 8;
+                }
+                S.dig[4 * v + 3][t] = (int8_t)X;
             }
         }
     }
-
-    // Codes staged: a = m * x by INT8 slot, then the dual GEMV.
     const bool ok = mbar_wait_bounded(&S.mbar, 0, a.status);
-    if (__syncthreads_or(!ok)) return;
-    const float *m_s = reinterpret_cast<const float *>(stage + L.off_m);
-    const float *s_s = reinterpret_cast<const float *>(stage + L.off_s);
-    if (t < NI) {
-        const int row = DAMP ? S.rows[t] : t;
-        const float mi = m_s[row];
+    if (DAMP && t < NI) {
+        const float *m_s = reinterpret_cast<const float *>(stage + L.off_m);
+        const int row = S.rows[t];
         const float2 x = S.x2[row];
-        S.a2[t] = make_float2(mi * x.x, mi * x.y);
+        S.a2[t] = make_float2(m_s[row] * x.x, m_s[row] * x.y);
     }
-    __syncthreads();
-    constexpr int LPR = DV / 4, RPP = 32 / LPR;
-    float ak[4] = {0.f, 0.f, 0.f, 0.f}, aq[4] = {0.f, 0.f, 0.f, 0.f};
-    {
+    if (__syncthreads_or(!ok)) return;
+    const float *s_s = reinterpret_cast<const float *>(stage + L.off_s);
+
+    // (c) codes.
+    float ek[4] = {0.f, 0.f, 0.f, 0.f}, eq[4] = {0.f, 0.f, 0.f, 0.f};
+    if (!DAMP) {
+        if (warp < DV / 16) {   // one warp per 16 value columns
+            const int c0 = 16 * warp;
+            const int gq = lane >> 2, tq = lane & 3;
+            const unsigned char *codes = stage + L.off_codes;
+            const int r = ((lane >> 3) & 1) * 8 + (lane & 7), blk = lane >> 4;
+            int d[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int ks = 0; ks < DK / 32; ++ks) {
+                const int c = c0 + r, chunk = 2 * ks + blk;
+                const uint32_t addr = smem_u32(codes + c * DK + ((chunk ^ code_swz(c, DK)) << 4));
+                uint32_t a0, a1, a2, a3;
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                             : "r"(addr));
+                const uint32_t b0 = *reinterpret_cast<const uint32_t *>(&S.dig[gq][32 * ks + 4 * tq]);
+                const uint32_t b1 = *reinterpret_cast<const uint32_t *>(&S.dig[gq][32 * ks + 16 + 4 * tq]);
+                asm volatile(
+                    "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                    "{%0,%1,%2,%3};"
+                    : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+                    : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+            }
+            // lane (gq, tq) holds digit columns 2tq, 2tq+1 of value columns c0+gq, c0+gq+8
+            const float w0 = (tq & 1) ? 65536.f : 1.f, w1 = (tq & 1) ? 16777216.f : 256.f;
+            float p0 = fmaf((float)d[1], w1, (float)d[0] * w0);
+            float p1 = fmaf((float)d[3], w1, (float)d[2] * w0);
+            p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+            p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
+            if ((tq & 1) == 0) {
+                const float inv = ldexpf(1.0f, (tq == 0 ? ek_ : eq_) - 30);
+                float *rc = reinterpret_cast<float *>(S.rc);
+                rc[2 * (c0 + gq) + (tq >> 1)] = s_s[c0 + gq] * (p0 * inv);
+                rc[2 * (c0 + gq + 8) + (tq >> 1)] = s_s[c0 + gq + 8] * (p1 * inv);
+            }
+        }
+    } else {
+        constexpr int LPR = DV / 4, RPP = 32 / LPR;
         const int cq = lane % LPR, rsub = lane / LPR;
         const unsigned char *codes = stage + L.off_codes;
+        float ak[4] = {0.f, 0.f, 0.f, 0.f}, aq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
         for (int j = warp * RPP + rsub; j < NI; j += kWarps * RPP) {
             const uint32_t w = *reinterpret_cast<const uint32_t *>(codes + (size_t)j * DV + 4 * cq);
@@ -204,10 +299,17 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
                 aq[u] += __shfl_xor_sync(0xffffffffu, aq[u], 16);
             }
         }
-    }
-    if (DAMP) {   // BF16 rows: one per warp, 4 columns per lane, unscaled x
+        if (lane < DV / 4) {
+            const float4 sc = *reinterpret_cast<const float4 *>(s_s + 4 * lane);
+            const float s4[4] = {sc.x, sc.y, sc.z, sc.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                ek[u] = s4[u] * ak[u];
+                eq[u] = s4[u] * aq[u];
+            }
+        }
         const uint16_t *hp = reinterpret_cast<const uint16_t *>(stage + L.off_hp);
-        for (int p = warp; p < P; p += kWarps) {
+        for (int p = warp; p < P; p += kWarps) {   // BF16 rows: unscaled x
             if (lane < DV / 4) {
                 const uint2 hb = *reinterpret_cast<const uint2 *>(hp + (size_t)p * DV + 4 * lane);
                 const float2 x = S.x2[S.rows[NI + p]];
@@ -220,17 +322,62 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
             }
         }
     }
-    // Per warp: s * (codes part) + (BF16 rows + entries part); one barrier.
-    if (lane < DV / 4) {
-        const float4 sc = *reinterpret_cast<const float4 *>(s_s + 4 * lane);
-        const float s4[4] = {sc.x, sc.y, sc.z, sc.w};
+
+    // (d) entries: y += u_e (ktil_e . x), a pair per warp step, next pair in flight.
+    {
+        float xk[XPL], xq[XPL];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            S.red[warp][4 * lane + u] = make_float2(fmaf(s4[u], ak[u], ek[u]), fmaf(s4[u], aq[u], eq[u]));
+        for (int u = 0; u < XPL; ++u) {
+            const float2 x = S.x2[XPL * lane + u];
+            xk[u] = x.x;
+            xq[u] = x.y;
+        }
+        for (int e0 = 2 * warp; e0 < E; e0 += 2 * kWarps) {
+            float d[4];
+            float4 uv[2];
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                float dk_ = 0.f, dq_ = 0.f;
+                if (e0 + p < E) {
+                    if (XPL == 4) {
+                        const float4 kv = kb[p];
+                        dk_ = fmaf(kv.x, xk[0], fmaf(kv.y, xk[1 % XPL], fmaf(kv.z, xk[2 % XPL], kv.w * xk[3 % XPL])));
+                        dq_ = fmaf(kv.x, xq[0], fmaf(kv.y, xq[1 % XPL], fmaf(kv.z, xq[2 % XPL], kv.w * xq[3 % XPL])));
+                    } else {
+                        const float2 kv = kb2[p];
+                        dk_ = fmaf(kv.x, xk[0], kv.y * xk[1 % XPL]);
+                        dq_ = fmaf(kv.x, xq[0], kv.y * xq[1 % XPL]);
+                    }
+                }
+                d[2 * p] = dk_;
+                d[2 * p + 1] = dq_;
+                uv[p] = ub[p];
+            }
+            const int ne = min(2, E - e0);
+            load_pair(e0 + 2 * kWarps);   // refill the registers while this pair is reduced
+            warp_reduce_dots<2>(d);
+            if (lane < DV / 4) {
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    if (p < ne) {
+                        ek[0] = fmaf(uv[p].x, d[2 * p], ek[0]); ek[1] = fmaf(uv[p].y, d[2 * p], ek[1]);
+                        ek[2] = fmaf(uv[p].z, d[2 * p], ek[2]); ek[3] = fmaf(uv[p].w, d[2 * p], ek[3]);
+                        eq[0] = fmaf(uv[p].x, d[2 * p + 1], eq[0]); eq[1] = fmaf(uv[p].y, d[2 * p + 1], eq[1]);
+                        eq[2] = fmaf(uv[p].z, d[2 * p + 1], eq[2]); eq[3] = fmaf(uv[p].w, d[2 * p + 1], eq[3]);
+                    }
+                }
+            }
+        }
+    }
+
+    // (e) combine, output, append.
+    if (lane < DV / 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) S.red[warp][4 * lane + u] = make_float2(ek[u], eq[u]);
     }
     __syncthreads();
     if (t < DV) {
-        float yk = 0.f, yq = 0.f;
+        float yk = DAMP ? 0.f : S.rc[t].x, yq = DAMP ? 0.f : S.rc[t].y;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
             const float2 p = S.red[w][t];
@@ -240,13 +387,13 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
         const float ut = beta * (S.v[t] - yk);
         const float o = fmaf(ut, kq, yq);
         a.o[hv * DV + t] = o;
-        rec_ent[(size_t)E * (DK + DV) + DK + t] = ut;
+        rec_ent[(size_t)E * EF + DK + t] = ut;
         if (!isfinite(o) || !isfinite(ut)) atomicOr(a.status, kStatusNonFinite);
     }
     if (t < DK) {
-        rec_ent[(size_t)E * (DK + DV) + t] = S.kk[t] / S.gt[t];
-        if (KDA) rec_gam[t] = S.gt[t];
-        else if (t == 0) rec_gam[0] = S.gt[0];
+        rec_ent[(size_t)E * EF + t] = kk / gt;
+        if (KDA) rec_gam[t] = gt;
+        else if (t == 0) rec_gam[0] = gt;
     }
 }
 
@@ -339,7 +486,7 @@ __global__ void __launch_bounds__(kThreads) decode_flush_kernel(const DecodeArgs
     const bool fin = tile_reconstruct<DK, DV>(
         R, reinterpret_cast<const float *>(stage + L.off_m), reinterpret_cast<const float *>(stage + L.off_s),
         reinterpret_cast<const uint16_t *>(stage + L.off_hp), reinterpret_cast<const int8_t *>(stage + L.off_codes),
-        reinterpret_cast<const float *>(stage + L.off_ent), P, DAMP ? F.map : nullptr, E, F.gam);
+        reinterpret_cast<const float *>(stage + L.off_ent), P, DAMP ? F.map : nullptr, E, F.gam, !DAMP);
     if (!fin) atomicOr(a.status, kStatusNonFinite);
 
     if (MODE == kExport) {
@@ -409,6 +556,7 @@ __global__ void __launch_bounds__(kThreads) decode_flush_kernel(const DecodeArgs
     }
     CodecOut out;
     out.codes = reinterpret_cast<int8_t *>(rec + L.off_codes);
+    out.codes_t = DAMP ? 0 : 1;
     out.hp = reinterpret_cast<uint16_t *>(rec + L.off_hp);
     out.m = reinterpret_cast<float *>(rec + L.off_m);
     out.s = reinterpret_cast<float *>(rec + L.off_s);

@@ -35,6 +35,7 @@ struct Fp32Args {
 // record layout and the plain lq_qstate_view arrays.
 struct QPtrs {
     unsigned char *codes; size_t codes_hs;
+    int codes_t;                                    // 1: column-major swizzled (record, no BF16 rows)
     unsigned char *hp;    size_t hp_hs;
     unsigned char *m;     size_t m_hs;
     unsigned char *s;     size_t s_hs;

@@ -71,18 +71,20 @@ __device__ __forceinline__ void load_cols16(const float *v, float (&o)[16]) {
 }
 
 // z[r] = sum_c R[r][c] w[c] for the thread's rows (w: the thread's 16 column
-// values); all CG lanes of a row group end with the full sums.
+// values); all CG lanes of a row group end with the full sums.  Packed FP32
+// FMAs over column pairs, then a transpose all-reduce over the row group.
 template <int DK, int DV>
 __device__ __forceinline__ void tile_rows_matvec(const float (&R)[Tile<DK, DV>::RPT][16], const float (&w)[16],
                                                  float (&z)[Tile<DK, DV>::RPT]) {
     using T = Tile<DK, DV>;
 #pragma unroll
     for (int r = 0; r < T::RPT; ++r) {
-        float acc = 0.f;
+        float2 acc = f2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) acc = fmaf(R[r][c], w[c], acc);
-        z[r] = shfl_xor_sum<T::CG>(acc);
+        for (int j = 0; j < 8; ++j) acc = ffma2(f2(R[r][2 * j], R[r][2 * j + 1]), f2(w[2 * j], w[2 * j + 1]), acc);
+        z[r] = acc.x + acc.y;
     }
+    xpose_allreduce<T::RPT, T::CG / 2, 1>(z);
 }
 
 // Column sums of R weighted by z, reduced over the tile.  Each warp ends with
@@ -96,20 +98,20 @@ __device__ __forceinline__ void tile_cols_matvec(const float (&R)[Tile<DK, DV>::
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5, cg = t % T::CG;
     float acc[16];
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        float a = 0.f;
+    for (int j = 0; j < 8; ++j) {
+        float2 a = f2(0.f, 0.f);
 #pragma unroll
-        for (int r = 0; r < T::RPT; ++r) a = fmaf(R[r][c], z[r], a);
-#pragma unroll
-        for (int m = T::CG; m < 32; m <<= 1) a += __shfl_xor_sync(0xffffffffu, a, m);
-        acc[c] = a;
+        for (int r = 0; r < T::RPT; ++r) a = ffma2(f2(R[r][2 * j], R[r][2 * j + 1]), f2(z[r], z[r]), a);
+        acc[2 * j] = a.x;
+        acc[2 * j + 1] = a.y;
     }
-    if (lane < T::CG) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<float4 *>(&cs.red[buf][warp][T::col(cg, q)]) =
-                make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
-    }
+    // over the warp's row groups: lanes differing in bits 16 .. CG
+    xpose_reduce<16, 16, T::CG>(acc);
+    constexpr int NR = 16 >> xpose_bits<16, T::CG>();   // tile columns left per lane
+    const int base = xpose_base<16, 16, T::CG>(lane);
+    float *dst = &cs.red[buf][warp][T::col(cg, base / 4) + base % 4];
+    if (NR == 4) *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2 % NR], acc[3 % NR]);
+    else *reinterpret_cast<float2 *>(dst) = make_float2(acc[0], acc[1 % NR]);
     cbar();
     mine = make_float4(0.f, 0.f, 0.f, 0.f);
     if (lane < DV / 4) {
@@ -146,13 +148,16 @@ __device__ int codec_compensators_fp32(float (&R)[Tile<DK, DV>::RPT][16], int r_
             float4 y;
             tile_cols_matvec<DK, DV>(R, z, cs, buf, y);
             buf ^= 1;
+            // |y|^2 accumulated in double (no overflow for any finite y); only
+            // the reciprocal of the norm is taken in FP32: it sets w's length,
+            // not its direction, and the next step normalises again.
             double ss = (double)y.x * y.x + (double)y.y * y.y + (double)y.z * y.z + (double)y.w * y.w;
-            const double nw = sqrt(warp_sum_d(ss));   // identical in every warp
-            if (nw == 0.0) { zero = true; break; }
-            const double inv = 1.0 / nw;
+            ss = warp_sum_d(ss);   // identical in every warp
+            if (ss == 0.0) { zero = true; break; }
+            const float inv = 1.0f / (float)sqrt(ss);
             if (lane < DV / 4)
                 *reinterpret_cast<float4 *>(&cs.wv[warp][4 * lane]) =
-                    make_float4((float)(y.x * inv), (float)(y.y * inv), (float)(y.z * inv), (float)(y.w * inv));
+                    make_float4(y.x * inv, y.y * inv, y.z * inv, y.w * inv);
             __syncwarp();
             load_cols16<DK, DV>(cs.wv[warp], w);
             __syncwarp();
@@ -181,7 +186,11 @@ __device__ int codec_compensators_fp32(float (&R)[Tile<DK, DV>::RPT][16], int r_
 #pragma unroll
         for (int r = 0; r < RPT; ++r)
 #pragma unroll
-            for (int q = 0; q < 16; ++q) R[r][q] = fmaf(-c[r], w[q], R[r][q]);
+            for (int q = 0; q < 8; ++q) {
+                const float2 o = ffma2(f2(-c[r], -c[r]), f2(w[2 * q], w[2 * q + 1]), f2(R[r][2 * q], R[r][2 * q + 1]));
+                R[r][2 * q] = o.x;
+                R[r][2 * q + 1] = o.y;
+            }
     }
     return buf;
 }
@@ -475,64 +484,96 @@ __device__ __forceinline__ bool tile_reconstruct(float (&R)[Tile<DK, DV>::RPT][1
     const int t = threadIdx.x, cg = t % T::CG, rg = t / T::CG, row0 = rg * RPT;
     float sv[16];
     load_cols16<DK, DV>(s_s, sv);
+    if (codes_t && RPT == 4) {
+        // value-column-major codes (no BF16 rows): the thread's 4 rows of one
+        // column are 4 consecutive bytes
+        float mi[4];
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-        const int i = row0 + r;
-        const int mp = (P > 0) ? map[i] : i;
-        if (mp >= 0 && codes_t) {
-            const float mi = m_s[i];
+        for (int r = 0; r < 4; ++r) mi[r] = m_s[row0 + r];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 4; ++q)
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float cf = (float)codes_s[code_off_t(T::col(cg, q) + u, i, DK)];
-                    R[r][4 * q + u] = (cf * sv[4 * q + u]) * mi;
-                }
-        } else if (mp >= 0) {
-            const float mi = m_s[i];
-            const uint32_t *row = reinterpret_cast<const uint32_t *>(codes_s + (size_t)mp * DV);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t w4 = *reinterpret_cast<const uint32_t *>(codes_s + code_off_t(T::col(cg, q) + u, row0, DK));
                 float f[4];
-                s8x4_to_f(row[T::col(cg, q) / 4], f);
+                s8x4_to_f(w4, f);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) R[r][4 * q + u] = (f[u] * sv[4 * q + u]) * mi;
+                for (int r = 0; r < 4; ++r) R[r % RPT][4 * q + u] = (f[r] * sv[4 * q + u]) * mi[r];
             }
-        } else {
-            const int p = -1 - mp;
+    } else {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint2 h = *reinterpret_cast<const uint2 *>(hp_s + (size_t)p * DV + T::col(cg, q));
-                R[r][4 * q] = bf16_to_f((uint16_t)(h.x & 0xffff));
-                R[r][4 * q + 1] = bf16_to_f((uint16_t)(h.x >> 16));
-                R[r][4 * q + 2] = bf16_to_f((uint16_t)(h.y & 0xffff));
-                R[r][4 * q + 3] = bf16_to_f((uint16_t)(h.y >> 16));
+        for (int r = 0; r < RPT; ++r) {
+            const int i = row0 + r;
+            const int mp = (P > 0) ? map[i] : i;
+            if (mp >= 0 && codes_t) {
+                const float mi = m_s[i];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float cf = (float)codes_s[code_off_t(T::col(cg, q) + u, i, DK)];
+                        R[r][4 * q + u] = (cf * sv[4 * q + u]) * mi;
+                    }
+            } else if (mp >= 0) {
+                const float mi = m_s[i];
+                const uint32_t *row = reinterpret_cast<const uint32_t *>(codes_s + (size_t)mp * DV);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float f[4];
+                    s8x4_to_f(row[T::col(cg, q) / 4], f);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) R[r][4 * q + u] = (f[u] * sv[4 * q + u]) * mi;
+                }
+            } else {
+                const int p = -1 - mp;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint2 h = *reinterpret_cast<const uint2 *>(hp_s + (size_t)p * DV + T::col(cg, q));
+                    R[r][4 * q] = bf16_to_f((uint16_t)(h.x & 0xffff));
+                    R[r][4 * q + 1] = bf16_to_f((uint16_t)(h.x >> 16));
+                    R[r][4 * q + 2] = bf16_to_f((uint16_t)(h.y & 0xffff));
+                    R[r][4 * q + 3] = bf16_to_f((uint16_t)(h.y >> 16));
+                }
             }
         }
     }
+    // buffered entries: R += ktil_e u_e^T, two columns per packed FMA
     for (int e = 0; e < E; ++e) {
         const float *kt = ent + (size_t)e * (DK + DV);
         float kv[RPT];
+        if (RPT == 4) {
+            const float4 k4 = *reinterpret_cast<const float4 *>(kt + row0);
+            kv[0] = k4.x; kv[1 % RPT] = k4.y; kv[2 % RPT] = k4.z; kv[3 % RPT] = k4.w;
+        } else {
 #pragma unroll
-        for (int r = 0; r < RPT; ++r) kv[r] = kt[row0 + r];
+            for (int r = 0; r < RPT; ++r) kv[r] = kt[row0 + r];
+        }
         float uv[16];
         load_cols16<DK, DV>(kt + DK, uv);
 #pragma unroll
         for (int r = 0; r < RPT; ++r)
 #pragma unroll
-            for (int q = 0; q < 16; ++q) R[r][q] = fmaf(kv[r], uv[q], R[r][q]);
+            for (int q = 0; q < 8; ++q) {
+                const float2 o = ffma2(f2(kv[r], kv[r]), f2(uv[2 * q], uv[2 * q + 1]), f2(R[r][2 * q], R[r][2 * q + 1]));
+                R[r][2 * q] = o.x;
+                R[r][2 * q + 1] = o.y;
+            }
     }
-    bool finite = true;
+    // Gamma, and a finiteness check that costs one packed FMA per pair:
+    // x * 0 is NaN exactly when x is not finite, and NaN propagates.
+    float2 chk = f2(0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         const float g = gam_s[row0 + r];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            R[r][q] *= g;
-            finite = finite && isfinite(R[r][q]);
+        for (int q = 0; q < 8; ++q) {
+            const float2 o = __fmul2_rn(f2(g, g), f2(R[r][2 * q], R[r][2 * q + 1]));
+            R[r][2 * q] = o.x;
+            R[r][2 * q + 1] = o.y;
+            chk = ffma2(o, f2(0.f, 0.f), chk);
         }
     }
-    return finite;
+    return chk.x == 0.f && chk.y == 0.f;
 }
 
 // Tile <-> row-major [DK][DV] global arrays.

@@ -153,6 +153,81 @@ __device__ __forceinline__ double warp_sum_d(double v) {
     return v;
 }
 
+// Transpose-reduce of V values per lane over the lanes that differ in bits
+// HI, HI/2, ..., LO (powers of two, LO <= HI <= 16).  At each of the first
+// log2(V) bits a lane keeps one half of its list and adds the other half,
+// received from its partner -- V/2 + V/4 + ... shuffles instead of V per bit;
+// any further bits are plain butterflies on the one value left.  Afterwards
+// v[0 .. V >> S) (S = the number of halving bits) hold the totals of the
+// entries xpose_base<V, HI, LO>(lane) + j.
+template <int HI, int LO>
+__host__ __device__ constexpr int xpose_bits() {
+    return HI < LO ? 0 : 1 + xpose_bits<HI / 2, LO>();
+}
+
+template <int V>
+__host__ __device__ constexpr int ilog2() {
+    return V <= 1 ? 0 : 1 + ilog2<V / 2>();
+}
+
+template <int V, int HI, int LO>
+__device__ __forceinline__ void xpose_reduce(float (&v)[V]) {
+    const int lane = threadIdx.x & 31;
+    constexpr int L = xpose_bits<HI, LO>();
+#pragma unroll
+    for (int l = 0; l < L; ++l) {
+        const int m = HI >> l;
+        const int n = V >> l;   // values still held before this bit
+        if (n > 1) {
+            const bool up = (lane & m) != 0;
+#pragma unroll
+            for (int i = 0; i < V / 2; ++i) {
+                if (i < n / 2) {
+                    const float send = up ? v[i] : v[i + n / 2];
+                    const float keep = up ? v[i + n / 2] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+        }
+    }
+}
+
+template <int V, int HI, int LO>
+__device__ __forceinline__ int xpose_base(int lane) {
+    constexpr int S = ilog2<V>() < xpose_bits<HI, LO>() ? ilog2<V>() : xpose_bits<HI, LO>();
+    int b = 0;
+#pragma unroll
+    for (int l = 0; l < S; ++l)
+        if (lane & (HI >> l)) b += V >> (l + 1);
+    return b;
+}
+
+// All-reduce of V values over the lanes differing in bits HI..LO, with
+// V <= 2^(number of bits): a transpose-reduce, then every lane gathers the V
+// totals (V shuffles).
+template <int V, int HI, int LO>
+__device__ __forceinline__ void xpose_allreduce(float (&v)[V]) {
+    static_assert(ilog2<V>() <= xpose_bits<HI, LO>(), "more values than lanes");
+    const int lane = threadIdx.x & 31;
+    xpose_reduce<V, HI, LO>(v);
+    const float mine = v[0];
+    constexpr int ALL = 2 * HI - LO;   // bits HI..LO
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        int src = lane & ~ALL;
+#pragma unroll
+        for (int l = 0; l < ilog2<V>(); ++l)
+            if (i & (V >> (l + 1))) src |= HI >> l;
+        v[i] = __shfl_sync(0xffffffffu, mine, src);
+    }
+}
+
+// Two FP32 fused multiply-adds per instruction (sm_100 packed FP32).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
 // Sum of one double per compute thread (warps 0..7); every compute thread
 // gets the result.  `scratch` holds kWarps doubles; two barriers inside.
 __device__ inline double block_sum_d(double v, double *scratch) {

@@ -501,33 +501,31 @@ __global__ void __launch_bounds__(kThreads) decode_flush_kernel(const DecodeArgs
             zk[r] = F.k[row0 + r];
             zq[r] = F.q[row0 + r];
         }
-        float acc[2][16];
+        // acc[0..16): the thread's column partials of S'^T k, acc[16..32): of S'^T q
+        float acc[32];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            float x = 0.f, y = 0.f;
+        for (int j = 0; j < 8; ++j) {
+            float2 ak = f2(0.f, 0.f), aq = f2(0.f, 0.f);
 #pragma unroll
             for (int r = 0; r < T::RPT; ++r) {
-                x = fmaf(R[r][c], zk[r], x);
-                y = fmaf(R[r][c], zq[r], y);
+                const float2 rv = f2(R[r][2 * j], R[r][2 * j + 1]);
+                ak = ffma2(rv, f2(zk[r], zk[r]), ak);
+                aq = ffma2(rv, f2(zq[r], zq[r]), aq);
             }
-#pragma unroll
-            for (int m = T::CG; m < 32; m <<= 1) {
-                x += __shfl_xor_sync(0xffffffffu, x, m);
-                y += __shfl_xor_sync(0xffffffffu, y, m);
-            }
-            acc[0][c] = x;
-            acc[1][c] = y;
+            acc[2 * j] = ak.x; acc[2 * j + 1] = ak.y;
+            acc[16 + 2 * j] = aq.x; acc[16 + 2 * j + 1] = aq.y;
         }
+        xpose_reduce<32, 16, T::CG>(acc);   // over the warp's row groups
         float(*rk)[DV] = F.cs.red[0];
         float(*rq)[DV] = F.cs.red[1];
-        if (lane < T::CG) {
+        {
+            constexpr int NR = 32 >> xpose_bits<16, T::CG>();
+            const int base = xpose_base<32, 16, T::CG>(lane);
+            float *dst = (base < 16 ? rk[warp] : rq[warp]);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                *reinterpret_cast<float4 *>(&rk[warp][T::col(cg, q)]) =
-                    make_float4(acc[0][4 * q], acc[0][4 * q + 1], acc[0][4 * q + 2], acc[0][4 * q + 3]);
-                *reinterpret_cast<float4 *>(&rq[warp][T::col(cg, q)]) =
-                    make_float4(acc[1][4 * q], acc[1][4 * q + 1], acc[1][4 * q + 2], acc[1][4 * q + 3]);
-            }
+            for (int gq = 0; gq < NR / 4; ++gq)
+                *reinterpret_cast<float4 *>(dst + T::col(cg, (base % 16) / 4 + gq)) =
+                    make_float4(acc[4 * gq], acc[4 * gq + 1], acc[4 * gq + 2], acc[4 * gq + 3]);
         }
         cbar();
         if (t < DV) {
@@ -551,7 +549,11 @@ __global__ void __launch_bounds__(kThreads) decode_flush_kernel(const DecodeArgs
         for (int r = 0; r < T::RPT; ++r) {
             const float kk = F.k[row0 + r];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) R[r][c] = fmaf(kk, uv[c], R[r][c]);
+            for (int c = 0; c < 8; ++c) {
+                const float2 o = ffma2(f2(kk, kk), f2(uv[2 * c], uv[2 * c + 1]), f2(R[r][2 * c], R[r][2 * c + 1]));
+                R[r][2 * c] = o.x;
+                R[r][2 * c + 1] = o.y;
+            }
         }
     }
     CodecOut out;

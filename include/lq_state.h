@@ -68,12 +68,15 @@ typedef enum {
     LQ_MODE_INT8_WINDOW = 2  /* INT8 state quantized once per window of W tokens */
 } lq_mode;
 
+/* Longest supported window (tokens buffered between two quantizations). */
+#define LQ_MAX_WINDOW 4096
+
 typedef struct {
     int32_t B, H, Hk;       /* batch, value heads, q/k heads (Hk divides H; GQA map h -> h*Hk/H) */
     int32_t dk, dv;         /* key / value head size */
     int32_t gate;           /* lq_gate */
     int32_t mode;           /* lq_mode */
-    int32_t W;              /* window length (tokens per quantization) */
+    int32_t W;              /* window length (tokens per quantization), 1 .. LQ_MAX_WINDOW */
     int32_t r;              /* compensator tokens per head, 0..min(dk,dv) */
     int32_t power_iters;    /* power-iteration steps per compensator (K), >= 0 */
     int32_t n_hp_rows;      /* P: BF16 key rows per head (DAMP layout), 0 = all INT8 */

@@ -61,6 +61,7 @@ int check_config(const lq_config *c) {
     if (rc) return rc;
     if (is_int8(c)) {
         if (c->W < 1) return LQ_ERR_INVALID_ARG;
+        if (c->W > LQ_MAX_WINDOW) return LQ_ERR_UNSUPPORTED;
         if (c->mode == LQ_MODE_INT8_STEP && c->W != 1) return LQ_ERR_INVALID_ARG;
         if (lq::decode_smem_bytes(c->dk, c->dv, layout_of(c)) > kMaxSmem) return LQ_ERR_UNSUPPORTED;
     } else if (c->n_hp_rows != 0) {

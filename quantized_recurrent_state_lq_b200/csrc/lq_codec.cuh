@@ -1,5 +1,6 @@
 // lq_codec.cuh -- the window-boundary quantizer on one head's FP32 state held
-// in registers across the 256 compute threads of a CTA.
+// in registers across the NT compute threads of a CTA (NT = 256 for the
+// stand-alone codec kernels, 128 for the window flush).
 //
 // Steps (LeapQuant project page: Compensator Tokens paragraph, then the
 // smoothing paragraph; STEPQuant article for key-row / value-column scales;
@@ -20,30 +21,31 @@
 // with CG = dv/16 column groups and thread t in column group t % CG, row group
 // t / CG.  The CG threads sharing rows are adjacent lanes, so every 16-byte
 // shared-memory access of a column group touches consecutive words (no bank
-// conflicts) and code rows leave as 32-byte contiguous segments.
+// conflicts).
 #pragma once
 
 #include "lq_common.cuh"
 
 namespace lq {
 
-template <int DK, int DV>
+template <int DK, int DV, int NT = kThreads>
 struct Tile {
     static constexpr int CG = DV / 16;
-    static constexpr int RG = kThreads / CG;
+    static constexpr int RG = NT / CG;
     static constexpr int RPT = DK / RG;
     static constexpr int RGW = 32 / CG;  // row groups per warp
+    static constexpr int NW = NT / 32;   // warps
     static_assert(RPT >= 1 && RG * RPT == DK, "tile shape");
     static_assert(CG <= 32 && (32 % CG) == 0, "column groups per warp");
     __device__ static int col(int cg, int q) { return 4 * cg + 4 * CG * q; }
 };
 
-template <int DK, int DV>
+template <int DK, int DV, int NT = kThreads>
 struct CodecSmem {
-    float red[2][kWarps][DV];   // cross-warp partial column sums (double-buffered)
-    float wv[kWarps][DV];       // per-warp copy of the current power-iteration vector
+    float red[2][NT / 32][DV];   // cross-warp partial column sums (double-buffered)
+    float wv[NT / 32][DV];       // per-warp copy of the current power-iteration vector
     float sc[DV];
-    double dred[kWarps];
+    double dred[NT / 32];
 };
 
 // Where the codec writes one head's quantized state.
@@ -73,10 +75,10 @@ __device__ __forceinline__ void load_cols16(const float *v, float (&o)[16]) {
 // z[r] = sum_c R[r][c] w[c] for the thread's rows (w: the thread's 16 column
 // values); all CG lanes of a row group end with the full sums.  Packed FP32
 // FMAs over column pairs, then a transpose all-reduce over the row group.
-template <int DK, int DV>
-__device__ __forceinline__ void tile_rows_matvec(const float (&R)[Tile<DK, DV>::RPT][16], const float (&w)[16],
-                                                 float (&z)[Tile<DK, DV>::RPT]) {
-    using T = Tile<DK, DV>;
+template <int DK, int DV, int NT>
+__device__ __forceinline__ void tile_rows_matvec(const float (&R)[Tile<DK, DV, NT>::RPT][16], const float (&w)[16],
+                                                 float (&z)[Tile<DK, DV, NT>::RPT]) {
+    using T = Tile<DK, DV, NT>;
 #pragma unroll
     for (int r = 0; r < T::RPT; ++r) {
         float2 acc = f2(0.f, 0.f);
@@ -87,14 +89,30 @@ __device__ __forceinline__ void tile_rows_matvec(const float (&R)[Tile<DK, DV>::
     xpose_allreduce<T::RPT, T::CG / 2, 1>(z);
 }
 
-// Column sums of R weighted by z, reduced over the tile.  Each warp ends with
-// the full vector y[DV] in its own wv[warp] (and lane-distributed in `mine`:
-// lane l holds y[4l .. 4l+3] for l < DV/4).  One barrier.
-template <int DK, int DV>
-__device__ __forceinline__ void tile_cols_matvec(const float (&R)[Tile<DK, DV>::RPT][16],
-                                                 const float (&z)[Tile<DK, DV>::RPT], CodecSmem<DK, DV> &cs,
+// Sum of NW per-warp float4 partials in a fixed tree order (the same bits in
+// every warp that computes it).
+template <int NW>
+__device__ __forceinline__ float4 sum_partials4(const float *base, int stride) {
+    float4 p[NW];
+#pragma unroll
+    for (int w = 0; w < NW; ++w) p[w] = *reinterpret_cast<const float4 *>(base + w * stride);
+#pragma unroll
+    for (int h = NW / 2; h >= 1; h >>= 1)
+#pragma unroll
+        for (int w = 0; w < h; ++w) {
+            p[w].x += p[w + h].x; p[w].y += p[w + h].y; p[w].z += p[w + h].z; p[w].w += p[w + h].w;
+        }
+    return p[0];
+}
+
+// Column sums of R weighted by z, reduced over the tile.  Every warp ends with
+// the full vector y[DV] lane-distributed in `mine` (lane l holds y[4l .. 4l+3]
+// for l < DV/4).  One barrier.
+template <int DK, int DV, int NT>
+__device__ __forceinline__ void tile_cols_matvec(const float (&R)[Tile<DK, DV, NT>::RPT][16],
+                                                 const float (&z)[Tile<DK, DV, NT>::RPT], CodecSmem<DK, DV, NT> &cs,
                                                  int buf, float4 &mine) {
-    using T = Tile<DK, DV>;
+    using T = Tile<DK, DV, NT>;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5, cg = t % T::CG;
     float acc[16];
 #pragma unroll
@@ -112,66 +130,68 @@ __device__ __forceinline__ void tile_cols_matvec(const float (&R)[Tile<DK, DV>::
     float *dst = &cs.red[buf][warp][T::col(cg, base / 4) + base % 4];
     if (NR == 4) *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2 % NR], acc[3 % NR]);
     else *reinterpret_cast<float2 *>(dst) = make_float2(acc[0], acc[1 % NR]);
-    cbar();
+    cbar<NT>();
     mine = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (lane < DV / 4) {
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const float4 p = *reinterpret_cast<const float4 *>(&cs.red[buf][w][4 * lane]);
-            mine.x += p.x; mine.y += p.y; mine.z += p.z; mine.w += p.w;
-        }
-    }
+    if (lane < DV / 4) mine = sum_partials4<T::NW>(&cs.red[buf][0][4 * lane], DV);
 }
 
 // Step 1 in FP32 on the register tile: R becomes the residual.  (The window
 // flush uses this path; its input is itself an FP32 result.)  With WRITE the
 // compensators go to `out`.  Returns the barrier-buffer index to continue with.
-template <int DK, int DV, bool WRITE>
-__device__ int codec_compensators_fp32(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, int K,
-                                       CodecSmem<DK, DV> &cs, const CodecOut &out) {
-    using T = Tile<DK, DV>;
+//
+// The power-iteration vector is normalised lazily: step k multiplies R by the
+// previous, unnormalised y and scales z = R y by 1/|y| afterwards, so the norm
+// (a double reduction, a square root and a reciprocal) runs alongside the next
+// matrix-vector product instead of before it.  The final w_j is y_K / |y_K|.
+template <int DK, int DV, bool WRITE, int NT = kThreads>
+__device__ int codec_compensators_fp32(float (&R)[Tile<DK, DV, NT>::RPT][16], int r_comp, int K,
+                                       CodecSmem<DK, DV, NT> &cs, const CodecOut &out) {
+    using T = Tile<DK, DV, NT>;
     constexpr int RPT = T::RPT, CG = T::CG;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int cg = t % CG, rg = t / CG;
     const int row0 = rg * RPT;
-    constexpr bool ENERGY = !WRITE;
     int buf = 0;
     for (int j = 0; j < r_comp; ++j) {
         float w[16];
         const float w0 = (float)(1.0 / sqrt((double)DV));
 #pragma unroll
         for (int c = 0; c < 16; ++c) w[c] = w0;
-        bool zero = false;
+        float inv = 1.0f;
+        bool zero = false;   // identical in every thread: every warp reduces the same partials
         for (int it = 0; it < K; ++it) {
             float z[RPT];
-            tile_rows_matvec<DK, DV>(R, w, z);
+            tile_rows_matvec<DK, DV, NT>(R, w, z);
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) z[r] *= inv;
             float4 y;
-            tile_cols_matvec<DK, DV>(R, z, cs, buf, y);
+            tile_cols_matvec<DK, DV, NT>(R, z, cs, buf, y);
             buf ^= 1;
-            // |y|^2 accumulated in double (no overflow for any finite y); only
-            // the reciprocal of the norm is taken in FP32: it sets w's length,
-            // not its direction, and the next step normalises again.
+            if (lane < DV / 4) *reinterpret_cast<float4 *>(&cs.wv[warp][4 * lane]) = y;
+            // |y|^2 accumulated in double; only the reciprocal of the norm is
+            // taken in FP32 (it sets w's length, not its direction).  A zero
+            // norm ends the extraction of this compensator; the remaining
+            // steps then run on zeros / NaN and are discarded.
             double ss = (double)y.x * y.x + (double)y.y * y.y + (double)y.z * y.z + (double)y.w * y.w;
-            ss = warp_sum_d(ss);   // identical in every warp
-            if (ss == 0.0) { zero = true; break; }
-            const float inv = 1.0f / (float)sqrt(ss);
-            if (lane < DV / 4)
-                *reinterpret_cast<float4 *>(&cs.wv[warp][4 * lane]) =
-                    make_float4(y.x * inv, y.y * inv, y.z * inv, y.w * inv);
+            ss = warp_sum_d(ss);
+            zero = zero || (ss == 0.0);
+            inv = 1.0f / (float)sqrt(ss);
             __syncwarp();
             load_cols16<DK, DV>(cs.wv[warp], w);
             __syncwarp();
         }
         if (zero) {
-            if (!ENERGY) {
+            if (WRITE) {
                 if (t < DV) out.cw[j * out.cw_stride + t] = 0.f;
                 if (t < DK) out.ck[j * out.ck_stride + t] = 0.f;
             }
             continue;
         }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) w[c] *= inv;
         float c[RPT];
-        tile_rows_matvec<DK, DV>(R, w, c);
-        if (!ENERGY) {
+        tile_rows_matvec<DK, DV, NT>(R, w, c);
+        if (WRITE) {
             if (warp == 0 && lane < CG) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -307,11 +327,11 @@ __device__ void codec_compensators_fp64(float (&R)[Tile<DK, DV>::RPT][16], int r
 // (slot >= 0 for INT8 rows, -1-p for BF16 row p); with P == 0 it may be null.
 // ENERGY: instead of writing codes, add sum_c (R - Deq)^2 of the residual to
 // eacc[r] (DAMP calibration); in that mode nothing is written.
-template <int DK, int DV, bool ENERGY>
-__device__ void codec_finish(float (&R)[Tile<DK, DV>::RPT][16], int smoothing, int P, const int *map,
-                             CodecSmem<DK, DV> &cs, const CodecOut &out, double (&eacc)[Tile<DK, DV>::RPT],
-                             int buf) {
-    using T = Tile<DK, DV>;
+template <int DK, int DV, bool ENERGY, int NT = kThreads>
+__device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothing, int P, const int *map,
+                             CodecSmem<DK, DV, NT> &cs, const CodecOut &out,
+                             double (&eacc)[Tile<DK, DV, NT>::RPT], int buf) {
+    using T = Tile<DK, DV, NT>;
     constexpr int RPT = T::RPT, CG = T::CG;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int cg = t % CG, rg = t / CG;
@@ -319,12 +339,12 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV>::RPT][16], int smoothing, i
 
     // 2. BF16 rows and 3. smoothing scales; x = R / m in place (ENERGY keeps R).
     float m[RPT];
-    bool int8row[RPT];
+    uint32_t int8mask = 0;   // bit r: row row0 + r is an INT8 row
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         const int i = row0 + r;
         const int mp = (P > 0) ? map[i] : i;
-        int8row[r] = mp >= 0;
+        if (mp >= 0) int8mask |= 1u << r;
         if (!ENERGY && mp < 0) {
             const int p = -1 - mp;
 #pragma unroll
@@ -334,18 +354,29 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV>::RPT][16], int smoothing, i
                 *reinterpret_cast<uint2 *>(out.hp + (size_t)p * DV + T::col(cg, q)) = make_uint2(lo, hi);
             }
         }
+        // row sum of squares in double over the row group's CG lanes (one row
+        // at a time: few registers beside the tile)
         double ss = 0.0;
 #pragma unroll
-        for (int q = 0; q < 16; ++q) ss += (double)R[r][q] * (double)R[r][q];
+        for (int q = 0; q < 16; ++q) ss = fma((double)R[r][q], (double)R[r][q], ss);
 #pragma unroll
         for (int mm = CG / 2; mm >= 1; mm >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, mm);
         float mi = 1.0f;
-        if (smoothing && int8row[r]) {
+        if (smoothing && mp >= 0) {
             mi = (float)sqrt(ss / (double)DV);
             if (mi == 0.0f) mi = 1.0f;
         }
         m[r] = mi;
-        if (!ENERGY && cg == 0) out.m[i] = mi;
+    }
+    if (!ENERGY && cg == 0) {
+        if (RPT % 4 == 0) {
+#pragma unroll
+            for (int r = 0; r < RPT; r += 4)
+                *reinterpret_cast<float4 *>(out.m + row0 + r) = make_float4(m[r], m[(r + 1) % RPT], m[(r + 2) % RPT], m[(r + 3) % RPT]);
+        } else {
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) out.m[row0 + r] = m[r];
+        }
     }
     // x = R / m (IEEE division, as the oracle); in place unless R is still
     // needed for the error energy.
@@ -364,100 +395,91 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV>::RPT][16], int smoothing, i
         for (int q = 0; q < 16; ++q) am[q] = 0.f;
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
-            if (!int8row[r]) continue;
+            if (!((int8mask >> r) & 1u)) continue;
 #pragma unroll
             for (int q = 0; q < 16; ++q) am[q] = fmaxf(am[q], fabsf(X(r, q)));
         }
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            float a = am[q];
-#pragma unroll
-            for (int mm = CG; mm < 32; mm <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, mm));
-            am[q] = a;
-        }
-        if (lane < CG) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<float4 *>(&cs.red[buf][warp][T::col(cg, q)]) =
-                    make_float4(am[4 * q], am[4 * q + 1], am[4 * q + 2], am[4 * q + 3]);
-        }
-        cbar();
+        xpose_reduce<16, 16, CG, true>(am);   // over the warp's row groups
+        constexpr int NR = 16 >> xpose_bits<16, CG>();
+        const int base = xpose_base<16, 16, CG>(lane);
+        float *dst = &cs.red[buf][warp][T::col(cg, base / 4) + base % 4];
+        if (NR == 4) *reinterpret_cast<float4 *>(dst) = make_float4(am[0], am[1], am[2 % NR], am[3 % NR]);
+        else *reinterpret_cast<float2 *>(dst) = make_float2(am[0], am[1 % NR]);
+        cbar<NT>();
         if (t < DV) {
             float a = 0.f;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) a = fmaxf(a, cs.red[buf][w][t]);
+            for (int w = 0; w < T::NW; ++w) a = fmaxf(a, cs.red[buf][w][t]);
             const float sc = a / 127.0f;
             cs.sc[t] = sc;
             if (!ENERGY) out.s[t] = sc;
         }
-        cbar();
+        cbar<NT>();
     }
 
     // Codes (or the error energy of the INT8 reconstruction).
     float sv[16];
     load_cols16<DK, DV>(cs.sc, sv);
-    uint32_t tpk[16];
+    auto code_of = [&](float x, float s) -> int {
+        return s != 0.f ? (int)fminf(fmaxf(rintf(x / s), -127.f), 127.f) : 0;
+    };
+    if (ENERGY) {
 #pragma unroll
-    for (int c = 0; c < 16; ++c) tpk[c] = 0u;
+        for (int r = 0; r < RPT; ++r) {
+            if (!((int8mask >> r) & 1u)) continue;
+            double e = 0.0;
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-        if (!int8row[r]) continue;
-        const int i = row0 + r;
-        uint32_t pk[4] = {0u, 0u, 0u, 0u};
-        double e = 0.0;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            float code = 0.f;
-            if (sv[q] != 0.f) code = fminf(fmaxf(rintf(X(r, q) / sv[q]), -127.f), 127.f);
-            if (ENERGY) {
-                const float dq = (code * sv[q]) * m[r];
+            for (int q = 0; q < 16; ++q) {
+                const float dq = ((float)code_of(X(r, q), sv[q]) * sv[q]) * m[r];
                 const double d = (double)R[r][q] - (double)dq;
                 e += d * d;
-            } else {
-                pk[q >> 2] |= ((uint32_t)((int)code & 0xff)) << (8 * (q & 3));
             }
-        }
-        if (ENERGY) {
 #pragma unroll
             for (int mm = CG / 2; mm >= 1; mm >>= 1) e += __shfl_xor_sync(0xffffffffu, e, mm);
             eacc[r] += e;
-        } else if (out.codes_t) {
-            // value-column-major: gather this thread's RPT consecutive rows of each column
+        }
+    } else if (out.codes_t) {
+        // value-column-major (no BF16 rows): the thread's RPT rows of one
+        // column are RPT consecutive bytes; one store per column
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 16; ++q) {
+            uint32_t lo = 0u, hi = 0u;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) tpk[4 * q + u] |= ((pk[q] >> (8 * u)) & 0xffu) << (8 * r);
-        } else {
+            for (int r = 0; r < RPT; ++r) {
+                const uint32_t b = (uint32_t)(code_of(R[r][q], sv[q]) & 0xff);
+                if (r < 4) lo |= b << (8 * r);
+                else hi |= b << (8 * (r - 4));
+            }
+            int8_t *dst = out.codes + code_off_t(T::col(cg, q / 4) + q % 4, row0, DK);
+            if (RPT == 8) *reinterpret_cast<uint2 *>(dst) = make_uint2(lo, hi);
+            else if (RPT == 4) *reinterpret_cast<uint32_t *>(dst) = lo;
+            else if (RPT == 2) *reinterpret_cast<uint16_t *>(dst) = (uint16_t)lo;
+            else *dst = (int8_t)lo;
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            if (!((int8mask >> r) & 1u)) continue;
+            const int i = row0 + r;
             const int slot = (P > 0) ? map[i] : i;
+            uint32_t pk[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int q = 0; q < 16; ++q) pk[q >> 2] |= ((uint32_t)(code_of(R[r][q], sv[q]) & 0xff)) << (8 * (q & 3));
             uint32_t *dst = reinterpret_cast<uint32_t *>(out.codes + (size_t)slot * DV);
 #pragma unroll
             for (int q = 0; q < 4; ++q) dst[T::col(cg, q) / 4] = pk[q];
         }
     }
-    if (!ENERGY && out.codes_t) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                int8_t *dst = out.codes + code_off_t(T::col(cg, q) + u, row0, DK);
-                if (RPT == 4) {
-                    *reinterpret_cast<uint32_t *>(dst) = tpk[4 * q + u];
-                } else {
-#pragma unroll
-                    for (int r = 0; r < RPT; ++r) dst[r] = (int8_t)((tpk[4 * q + u] >> (8 * r)) & 0xffu);
-                }
-            }
-    }
-    cbar();
+    cbar<NT>();
 }
 
 // The whole quantizer with the FP32 compensator step (window flush).
-template <int DK, int DV, bool ENERGY>
-__device__ void codec_quantize(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, int K, int smoothing, int P,
-                               const int *map, CodecSmem<DK, DV> &cs, const CodecOut &out,
-                               double (&eacc)[Tile<DK, DV>::RPT]) {
-    const int buf = codec_compensators_fp32<DK, DV, !ENERGY>(R, r_comp, K, cs, out);
-    codec_finish<DK, DV, ENERGY>(R, smoothing, P, map, cs, out, eacc, buf);
+template <int DK, int DV, bool ENERGY, int NT = kThreads>
+__device__ void codec_quantize(float (&R)[Tile<DK, DV, NT>::RPT][16], int r_comp, int K, int smoothing, int P,
+                               const int *map, CodecSmem<DK, DV, NT> &cs, const CodecOut &out,
+                               double (&eacc)[Tile<DK, DV, NT>::RPT]) {
+    const int buf = codec_compensators_fp32<DK, DV, !ENERGY, NT>(R, r_comp, K, cs, out);
+    codec_finish<DK, DV, ENERGY, NT>(R, smoothing, P, map, cs, out, eacc, buf);
 }
 
 // The whole quantizer with the double-precision compensator step.
@@ -469,81 +491,105 @@ __device__ void codec_quantize_exact(float (&R)[Tile<DK, DV>::RPT][16], int r_co
     codec_finish<DK, DV, ENERGY>(R, smoothing, P, map, cs, out, eacc, 0);
 }
 
-// Reconstruct a head's current state into the tile:
-// R = Gamma * ( Deq(C, m, s) [or BF16 rows] + sum_{e<E} ktil_e u_e^T ).
+// Reconstruction of a head's current state into the tile, in three parts:
+//   tile_dequant:      R = Deq(C, m, s) [BF16 rows widened]
+//   tile_add_entries:  R += sum_e ktil_e u_e^T over n entries [n][DK+DV]
+//   tile_gamma:        R *= Gamma (by key row); true if every value is finite
 // The arrays may live in shared or global memory: m_s [DK], s_s [DV],
-// hp_s [P][DV], codes_s [DK-P][DV], ent [E][DK+DV], gam_s [DK].
-// Returns true if every value is finite.
-template <int DK, int DV>
-__device__ __forceinline__ bool tile_reconstruct(float (&R)[Tile<DK, DV>::RPT][16], const float *m_s,
-                                                 const float *s_s, const uint16_t *hp_s, const int8_t *codes_s,
-                                                 const float *ent, int P, const int *map, int E,
-                                                 const float *gam_s, bool codes_t) {
-    using T = Tile<DK, DV>;
+// hp_s [P][DV], codes_s (layout per codes_t), gam_s [DK].
+template <int DK, int DV, int NT>
+__device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][16], const float *m_s,
+                                             const float *s_s, const uint16_t *hp_s, const int8_t *codes_s, int P,
+                                             const int *map, bool codes_t) {
+    using T = Tile<DK, DV, NT>;
     constexpr int RPT = T::RPT;
     const int t = threadIdx.x, cg = t % T::CG, rg = t / T::CG, row0 = rg * RPT;
     float sv[16];
     load_cols16<DK, DV>(s_s, sv);
-    if (codes_t && RPT == 4) {
-        // value-column-major codes (no BF16 rows): the thread's 4 rows of one
-        // column are 4 consecutive bytes
-        float mi[4];
+    if (codes_t && (RPT == 4 || RPT == 8)) {
+        // value-column-major codes (no BF16 rows): the thread's RPT rows of
+        // one column are RPT consecutive bytes
+        float mi[RPT];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) mi[r] = m_s[row0 + r];
+        for (int r = 0; r < RPT; ++r) mi[r] = m_s[row0 + r];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const uint32_t w4 = *reinterpret_cast<const uint32_t *>(codes_s + code_off_t(T::col(cg, q) + u, row0, DK));
-                float f[4];
-                s8x4_to_f(w4, f);
+                const int8_t *src = codes_s + code_off_t(T::col(cg, q) + u, row0, DK);
+                uint32_t wd[2];
+                if (RPT == 8) {
+                    const uint2 v2 = *reinterpret_cast<const uint2 *>(src);
+                    wd[0] = v2.x;
+                    wd[1] = v2.y;
+                } else {
+                    wd[0] = *reinterpret_cast<const uint32_t *>(src);
+                    wd[1] = 0u;
+                }
 #pragma unroll
-                for (int r = 0; r < 4; ++r) R[r % RPT][4 * q + u] = (f[r] * sv[4 * q + u]) * mi[r];
-            }
-    } else {
-#pragma unroll
-        for (int r = 0; r < RPT; ++r) {
-            const int i = row0 + r;
-            const int mp = (P > 0) ? map[i] : i;
-            if (mp >= 0 && codes_t) {
-                const float mi = m_s[i];
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float cf = (float)codes_s[code_off_t(T::col(cg, q) + u, i, DK)];
-                        R[r][4 * q + u] = (cf * sv[4 * q + u]) * mi;
-                    }
-            } else if (mp >= 0) {
-                const float mi = m_s[i];
-                const uint32_t *row = reinterpret_cast<const uint32_t *>(codes_s + (size_t)mp * DV);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int h = 0; h < RPT / 4; ++h) {
                     float f[4];
-                    s8x4_to_f(row[T::col(cg, q) / 4], f);
+                    s8x4_to_f(wd[h], f);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) R[r][4 * q + u] = (f[u] * sv[4 * q + u]) * mi;
+                    for (int k = 0; k < 4; ++k) {
+                        const int r = 4 * h + k;
+                        R[r % RPT][4 * q + u] = (f[k] * sv[4 * q + u]) * mi[r % RPT];
+                    }
                 }
-            } else {
-                const int p = -1 - mp;
+            }
+        return;
+    }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint2 h = *reinterpret_cast<const uint2 *>(hp_s + (size_t)p * DV + T::col(cg, q));
-                    R[r][4 * q] = bf16_to_f((uint16_t)(h.x & 0xffff));
-                    R[r][4 * q + 1] = bf16_to_f((uint16_t)(h.x >> 16));
-                    R[r][4 * q + 2] = bf16_to_f((uint16_t)(h.y & 0xffff));
-                    R[r][4 * q + 3] = bf16_to_f((uint16_t)(h.y >> 16));
+    for (int r = 0; r < RPT; ++r) {
+        const int i = row0 + r;
+        const int mp = (P > 0) ? map[i] : i;
+        if (mp >= 0 && codes_t) {
+            const float mi = m_s[i];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float cf = (float)codes_s[code_off_t(T::col(cg, q) + u, i, DK)];
+                    R[r][4 * q + u] = (cf * sv[4 * q + u]) * mi;
                 }
+        } else if (mp >= 0) {
+            const float mi = m_s[i];
+            const uint32_t *row = reinterpret_cast<const uint32_t *>(codes_s + (size_t)mp * DV);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float f[4];
+                s8x4_to_f(row[T::col(cg, q) / 4], f);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) R[r][4 * q + u] = (f[u] * sv[4 * q + u]) * mi;
+            }
+        } else {
+            const int p = -1 - mp;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint2 h = *reinterpret_cast<const uint2 *>(hp_s + (size_t)p * DV + T::col(cg, q));
+                R[r][4 * q] = bf16_to_f((uint16_t)(h.x & 0xffff));
+                R[r][4 * q + 1] = bf16_to_f((uint16_t)(h.x >> 16));
+                R[r][4 * q + 2] = bf16_to_f((uint16_t)(h.y & 0xffff));
+                R[r][4 * q + 3] = bf16_to_f((uint16_t)(h.y >> 16));
             }
         }
     }
-    // buffered entries: R += ktil_e u_e^T, two columns per packed FMA
-    for (int e = 0; e < E; ++e) {
+}
+
+template <int DK, int DV, int NT>
+__device__ __forceinline__ void tile_add_entries(float (&R)[Tile<DK, DV, NT>::RPT][16], const float *ent, int n) {
+    using T = Tile<DK, DV, NT>;
+    constexpr int RPT = T::RPT;
+    const int row0 = (threadIdx.x / T::CG) * RPT;
+    for (int e = 0; e < n; ++e) {
         const float *kt = ent + (size_t)e * (DK + DV);
         float kv[RPT];
-        if (RPT == 4) {
-            const float4 k4 = *reinterpret_cast<const float4 *>(kt + row0);
-            kv[0] = k4.x; kv[1 % RPT] = k4.y; kv[2 % RPT] = k4.z; kv[3 % RPT] = k4.w;
+        if (RPT % 4 == 0) {
+#pragma unroll
+            for (int r = 0; r < RPT; r += 4) {
+                const float4 k4 = *reinterpret_cast<const float4 *>(kt + row0 + r);
+                kv[r] = k4.x; kv[(r + 1) % RPT] = k4.y; kv[(r + 2) % RPT] = k4.z; kv[(r + 3) % RPT] = k4.w;
+            }
         } else {
 #pragma unroll
             for (int r = 0; r < RPT; ++r) kv[r] = kt[row0 + r];
@@ -559,11 +605,17 @@ __device__ __forceinline__ bool tile_reconstruct(float (&R)[Tile<DK, DV>::RPT][1
                 R[r][2 * q + 1] = o.y;
             }
     }
-    // Gamma, and a finiteness check that costs one packed FMA per pair:
-    // x * 0 is NaN exactly when x is not finite, and NaN propagates.
+}
+
+// Gamma, and a finiteness check that costs one packed FMA per pair: x * 0 is
+// NaN exactly when x is not finite, and NaN propagates.
+template <int DK, int DV, int NT>
+__device__ __forceinline__ bool tile_gamma(float (&R)[Tile<DK, DV, NT>::RPT][16], const float *gam_s) {
+    using T = Tile<DK, DV, NT>;
+    const int row0 = (threadIdx.x / T::CG) * T::RPT;
     float2 chk = f2(0.f, 0.f);
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
+    for (int r = 0; r < T::RPT; ++r) {
         const float g = gam_s[row0 + r];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -577,9 +629,9 @@ __device__ __forceinline__ bool tile_reconstruct(float (&R)[Tile<DK, DV>::RPT][1
 }
 
 // Tile <-> row-major [DK][DV] global arrays.
-template <int DK, int DV>
-__device__ __forceinline__ void tile_load_global(float (&R)[Tile<DK, DV>::RPT][16], const float *src) {
-    using T = Tile<DK, DV>;
+template <int DK, int DV, int NT = kThreads>
+__device__ __forceinline__ void tile_load_global(float (&R)[Tile<DK, DV, NT>::RPT][16], const float *src) {
+    using T = Tile<DK, DV, NT>;
     const int t = threadIdx.x, cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
 #pragma unroll
     for (int r = 0; r < T::RPT; ++r)
@@ -590,9 +642,9 @@ __device__ __forceinline__ void tile_load_global(float (&R)[Tile<DK, DV>::RPT][1
         }
 }
 
-template <int DK, int DV>
-__device__ __forceinline__ void tile_store_global(const float (&R)[Tile<DK, DV>::RPT][16], float *dst) {
-    using T = Tile<DK, DV>;
+template <int DK, int DV, int NT = kThreads>
+__device__ __forceinline__ void tile_store_global(const float (&R)[Tile<DK, DV, NT>::RPT][16], float *dst) {
+    using T = Tile<DK, DV, NT>;
     const int t = threadIdx.x, cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
 #pragma unroll
     for (int r = 0; r < T::RPT; ++r)

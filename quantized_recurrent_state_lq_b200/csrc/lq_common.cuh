@@ -64,10 +64,11 @@ __host__ __device__ __forceinline__ int code_off_t(int c, int i, int dk) {
     return c * dk + ((((i >> 4) ^ code_swz(c, dk)) << 4) | (i & 15));
 }
 
-// Named barrier over the 256 compute threads (warps 0..7) of a CTA; with a
-// 256-thread CTA it is a full barrier, with an extra producer warp it leaves
-// the producer out.
-__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// Named barrier over the NT compute threads (warps 0 .. NT/32-1) of a CTA;
+// with an NT-thread CTA it is a full barrier, with extra warps it leaves them
+// out.
+template <int NT = kThreads>
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
 
 // ---------------------------------------------------------------------------
 // PTX wrappers: mbarrier + cp.async.bulk (global -> shared, no multicast).
@@ -170,8 +171,14 @@ __host__ __device__ constexpr int ilog2() {
     return V <= 1 ? 0 : 1 + ilog2<V / 2>();
 }
 
-template <int V, int HI, int LO>
-__device__ __forceinline__ void xpose_reduce(float (&v)[V]) {
+template <bool MAX, typename F>
+__device__ __forceinline__ F xpose_op(F a, F b) {
+    if constexpr (MAX) return fmax(a, b);   // fmaxf / fmax: a NaN operand is ignored
+    else return a + b;
+}
+
+template <int V, int HI, int LO, bool MAX = false, typename F>
+__device__ __forceinline__ void xpose_reduce(F (&v)[V]) {
     const int lane = threadIdx.x & 31;
     constexpr int L = xpose_bits<HI, LO>();
 #pragma unroll
@@ -183,13 +190,13 @@ __device__ __forceinline__ void xpose_reduce(float (&v)[V]) {
 #pragma unroll
             for (int i = 0; i < V / 2; ++i) {
                 if (i < n / 2) {
-                    const float send = up ? v[i] : v[i + n / 2];
-                    const float keep = up ? v[i + n / 2] : v[i];
-                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                    const F send = up ? v[i] : v[i + n / 2];
+                    const F keep = up ? v[i + n / 2] : v[i];
+                    v[i] = xpose_op<MAX>(keep, __shfl_xor_sync(0xffffffffu, send, m));
                 }
             }
         } else {
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+            v[0] = xpose_op<MAX>(v[0], __shfl_xor_sync(0xffffffffu, v[0], m));
         }
     }
 }
@@ -207,12 +214,12 @@ __device__ __forceinline__ int xpose_base(int lane) {
 // All-reduce of V values over the lanes differing in bits HI..LO, with
 // V <= 2^(number of bits): a transpose-reduce, then every lane gathers the V
 // totals (V shuffles).
-template <int V, int HI, int LO>
-__device__ __forceinline__ void xpose_allreduce(float (&v)[V]) {
+template <int V, int HI, int LO, typename F>
+__device__ __forceinline__ void xpose_allreduce(F (&v)[V]) {
     static_assert(ilog2<V>() <= xpose_bits<HI, LO>(), "more values than lanes");
     const int lane = threadIdx.x & 31;
     xpose_reduce<V, HI, LO>(v);
-    const float mine = v[0];
+    const F mine = v[0];
     constexpr int ALL = 2 * HI - LO;   // bits HI..LO
 #pragma unroll
     for (int i = 0; i < V; ++i) {
@@ -268,10 +275,11 @@ __device__ __forceinline__ void s8x4_to_f(uint32_t w, float f[4]) {
 
 // Build the key-row map of one head in shared memory: map[i] = INT8 slot of
 // row i (rows in increasing order, BF16 rows skipped) or -1-p for the p-th
-// BF16 row.  Run by the 256 compute threads; needs DK <= 256.  Ends with a
+// BF16 row.  Run by the NT compute threads; needs DK <= NT.  Ends with a
 // barrier over them.
-template <int DK>
+template <int DK, int NT = kThreads>
 __device__ inline void build_row_map(const int *hp_rows_h, int P, int *map, int *scratch_w) {
+    static_assert(DK <= NT, "one thread per key row");
     const int i = threadIdx.x;
     int p_of = -1;
     if (i < DK) {
@@ -282,11 +290,11 @@ __device__ inline void build_row_map(const int *hp_rows_h, int P, int *map, int 
     const uint32_t bal = __ballot_sync(0xffffffffu, hp);
     const int lane = i & 31, warp = i >> 5;
     if (lane == 0) scratch_w[warp] = __popc(bal);
-    cbar();
+    cbar<NT>();
     int before = __popc(bal & ((1u << lane) - 1u));
     for (int w = 0; w < warp; ++w) before += scratch_w[w];
     if (i < DK) map[i] = hp ? (-1 - p_of) : (i - before);
-    cbar();
+    cbar<NT>();
 }
 
 }  // namespace lq

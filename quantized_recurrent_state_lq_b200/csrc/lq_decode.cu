@@ -398,8 +398,11 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
 }
 
 // ---------------------------------------------------------------------------
-// Window-end step: one CTA per head.  The record prefix (m, s, BF16 rows,
-// codes, r+n entries) is staged with one bulk copy; the tile
+// Window-end step: one CTA of 128 threads per head, three per SM (a 128-row
+// tile is 128 registers a thread).  The record prefix (m, s, BF16 rows,
+// codes) is staged with one bulk copy and the r+n entries stream through two
+// shared-memory buffers of kFlushChunk entries, one chunk in flight while the
+// previous one is applied; the tile
 //   S' = Gamma_t [Deq + sum_e ktil_e u_e^T]
 // is built in registers, the step's outputs come from it (y_k = S'^T k_t,
 // y_q = S'^T q_t), S_t = S' + k_t u_t^T is quantized in place (new
@@ -407,15 +410,20 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
 // kExport instead writes the current state Gamma [Deq + buffer] (no token);
 // kFlushOnly ends the window without a token (lq_window_flush).
 // ---------------------------------------------------------------------------
+constexpr int kFlushThreads = 128;
+constexpr int kFlushWarps = kFlushThreads / 32;
+constexpr int kFlushChunk = 16;
+
 template <int DK, int DV>
 struct FlushSmem {
     float k[DK], q[DK], gam[DK];
     float u[DV];
-    float kqw[kWarps];
+    float kqw[kFlushWarps];
     int map[DK];
-    int wscr[kWarps];
-    CodecSmem<DK, DV> cs;
-    uint64_t mbar;
+    int wscr[kFlushWarps];
+    CodecSmem<DK, DV, kFlushThreads> cs;
+    uint64_t mbar_pre;
+    uint64_t mbar_ent[2];
 };
 
 template <int DK, int DV>
@@ -423,44 +431,69 @@ __host__ __device__ constexpr size_t flush_fixed_bytes() {
     return (sizeof(FlushSmem<DK, DV>) + 127) / 128 * 128;
 }
 
+__host__ __device__ inline size_t flush_chunk_bytes(int dk, int dv) { return (size_t)kFlushChunk * (dk + dv) * 4; }
+
 size_t flush_smem_bytes(int dk, int dv, const Layout &L) {
     size_t fixed = 0;
     if (dk == 64 && dv == 64) fixed = flush_fixed_bytes<64, 64>();
     if (dk == 64 && dv == 128) fixed = flush_fixed_bytes<64, 128>();
     if (dk == 128 && dv == 64) fixed = flush_fixed_bytes<128, 64>();
     if (dk == 128 && dv == 128) fixed = flush_fixed_bytes<128, 128>();
-    return fixed + (size_t)align_up(L.off_ent + (L.r + L.W) * (L.dk + L.dv) * 4, 128);
+    return fixed + (size_t)align_up(L.off_ent, 128) + 2 * flush_chunk_bytes(dk, dv);
 }
 
 enum { kFlushStep = 0, kFlushOnly = 1, kExport = 2 };
 
 template <int DK, int DV, bool KDA, bool DAMP, int MODE>
-__global__ void __launch_bounds__(kThreads) decode_flush_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const DecodeArgs a) {
+    constexpr int NT = kFlushThreads;
+    constexpr int EF = DK + DV;   // floats per entry
     extern __shared__ __align__(128) unsigned char smem[];
-    using T = Tile<DK, DV>;
+    using T = Tile<DK, DV, NT>;
     FlushSmem<DK, DV> &F = *reinterpret_cast<FlushSmem<DK, DV> *>(smem);
-    unsigned char *stage = smem + flush_fixed_bytes<DK, DV>();
     const Layout &L = a.L;
+    unsigned char *stage = smem + flush_fixed_bytes<DK, DV>();
+    float *ebuf = reinterpret_cast<float *>(stage + align_up(L.off_ent, 128));   // [2][kFlushChunk][EF]
     const int head = blockIdx.x;
     const int b = head / a.H, h = head - b * a.H, g = (h * a.Hk) / a.H;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
     const int P = DAMP ? L.P : 0;
     const int E = L.r + a.n;
+    const int nch = (E + kFlushChunk - 1) / kFlushChunk;
     unsigned char *rec = a.rec + (size_t)head * L.rec_bytes;
     float *rec_ent = reinterpret_cast<float *>(rec + L.off_ent);
     float *rec_gam = reinterpret_cast<float *>(rec + L.off_gam);
     const size_t hv = (size_t)b * a.H + h;
 
+    // chunk c (entries [c*kFlushChunk, ...)) goes to buffer c & 1; its
+    // barrier completes once per use, use c >> 1, parity (c >> 1) & 1
+    auto issue_chunk = [&](int c) {
+        const int n = min(kFlushChunk, E - c * kFlushChunk);
+        const uint32_t bytes = (uint32_t)(n * EF * 4);
+        mbar_arrive_expect_tx(&F.mbar_ent[c & 1], bytes);
+        bulk_g2s(ebuf + (size_t)(c & 1) * kFlushChunk * EF, rec_ent + (size_t)c * kFlushChunk * EF, bytes,
+                 &F.mbar_ent[c & 1]);
+    };
+    // after a failed wait: let the copies still in flight land (bounded)
+    // before the CTA's shared memory is released
+    auto drain = [&](int from, int issued) {
+        if (t == 0)
+            for (int c = from; c < issued; ++c) mbar_wait_bounded(&F.mbar_ent[c & 1], (c >> 1) & 1, nullptr);
+    };
+
     if (t == 0) {
-        mbar_init(&F.mbar, 1);
+        mbar_init(&F.mbar_pre, 1);
+        mbar_init(&F.mbar_ent[0], 1);
+        mbar_init(&F.mbar_ent[1], 1);
         fence_mbar_init();
     }
     __syncthreads();
+    int issued = min(nch, 2);
     if (t == 0) {
-        const uint32_t bytes = (uint32_t)(L.off_ent + E * (DK + DV) * 4);
-        mbar_arrive_expect_tx(&F.mbar, bytes);
-        bulk_g2s(stage, rec, bytes, &F.mbar);
+        mbar_arrive_expect_tx(&F.mbar_pre, (uint32_t)L.off_ent);
+        bulk_g2s(stage, rec, (uint32_t)L.off_ent, &F.mbar_pre);
+        for (int c = 0; c < issued; ++c) issue_chunk(c);
     }
     float kqp = 0.f;
     if (t < DK) {
@@ -478,60 +511,70 @@ __global__ void __launch_bounds__(kThreads) decode_flush_kernel(const DecodeArgs
     }
     kqp = warp_sum(kqp);
     if (lane == 0) F.kqw[warp] = kqp;
-    if (DAMP) build_row_map<DK>(a.hp_rows + (size_t)h * P, P, F.map, F.wscr);
-    const bool okw = mbar_wait_bounded(&F.mbar, 0, a.status);
-    if (__syncthreads_or(!okw)) return;
+    if (DAMP) build_row_map<DK, NT>(a.hp_rows + (size_t)h * P, P, F.map, F.wscr);
+    const bool okw = mbar_wait_bounded(&F.mbar_pre, 0, a.status);
+    if (__syncthreads_or(!okw)) {
+        drain(0, issued);
+        return;
+    }
 
     float R[T::RPT][16];
-    const bool fin = tile_reconstruct<DK, DV>(
-        R, reinterpret_cast<const float *>(stage + L.off_m), reinterpret_cast<const float *>(stage + L.off_s),
-        reinterpret_cast<const uint16_t *>(stage + L.off_hp), reinterpret_cast<const int8_t *>(stage + L.off_codes),
-        reinterpret_cast<const float *>(stage + L.off_ent), P, DAMP ? F.map : nullptr, E, F.gam, !DAMP);
+    tile_dequant<DK, DV, NT>(R, reinterpret_cast<const float *>(stage + L.off_m),
+                             reinterpret_cast<const float *>(stage + L.off_s),
+                             reinterpret_cast<const uint16_t *>(stage + L.off_hp),
+                             reinterpret_cast<const int8_t *>(stage + L.off_codes), P, DAMP ? F.map : nullptr, !DAMP);
+    for (int c = 0; c < nch; ++c) {
+        const bool ok = mbar_wait_bounded(&F.mbar_ent[c & 1], (c >> 1) & 1, a.status);
+        // also the barrier after which buffer (c+1) & 1 -- chunk c-1 -- is free
+        if (__syncthreads_or(!ok)) {
+            drain(c + 1, issued);
+            return;
+        }
+        if (c >= 1 && c + 1 < nch) {
+            if (t == 0) issue_chunk(c + 1);
+            ++issued;
+        }
+        tile_add_entries<DK, DV, NT>(R, ebuf + (size_t)(c & 1) * kFlushChunk * EF, min(kFlushChunk, E - c * kFlushChunk));
+    }
+    const bool fin = tile_gamma<DK, DV, NT>(R, F.gam);
     if (!fin) atomicOr(a.status, kStatusNonFinite);
 
     if (MODE == kExport) {
-        tile_store_global<DK, DV>(R, a.S_out + (size_t)head * DK * DV);
+        tile_store_global<DK, DV, NT>(R, a.S_out + (size_t)head * DK * DV);
         return;
     }
     if (MODE == kFlushStep) {
-        // y_k = S'^T k, y_q = S'^T q over the tile, one barrier.
-        float zk[T::RPT], zq[T::RPT];
-#pragma unroll
-        for (int r = 0; r < T::RPT; ++r) {
-            zk[r] = F.k[row0 + r];
-            zq[r] = F.q[row0 + r];
-        }
-        // acc[0..16): the thread's column partials of S'^T k, acc[16..32): of S'^T q
-        float acc[32];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float2 ak = f2(0.f, 0.f), aq = f2(0.f, 0.f);
-#pragma unroll
-            for (int r = 0; r < T::RPT; ++r) {
-                const float2 rv = f2(R[r][2 * j], R[r][2 * j + 1]);
-                ak = ffma2(rv, f2(zk[r], zk[r]), ak);
-                aq = ffma2(rv, f2(zq[r], zq[r]), aq);
-            }
-            acc[2 * j] = ak.x; acc[2 * j + 1] = ak.y;
-            acc[16 + 2 * j] = aq.x; acc[16 + 2 * j + 1] = aq.y;
-        }
-        xpose_reduce<32, 16, T::CG>(acc);   // over the warp's row groups
+        // y_k = S'^T k, y_q = S'^T q over the tile (one vector at a time, to
+        // keep the registers beside the tile few), one barrier.
         float(*rk)[DV] = F.cs.red[0];
         float(*rq)[DV] = F.cs.red[1];
-        {
-            constexpr int NR = 32 >> xpose_bits<16, T::CG>();
-            const int base = xpose_base<32, 16, T::CG>(lane);
-            float *dst = (base < 16 ? rk[warp] : rq[warp]);
+#pragma unroll 1
+        for (int vsel = 0; vsel < 2; ++vsel) {
+            const float *xs = vsel ? F.q : F.k;
+            float zx[T::RPT];
 #pragma unroll
-            for (int gq = 0; gq < NR / 4; ++gq)
-                *reinterpret_cast<float4 *>(dst + T::col(cg, (base % 16) / 4 + gq)) =
-                    make_float4(acc[4 * gq], acc[4 * gq + 1], acc[4 * gq + 2], acc[4 * gq + 3]);
+            for (int r = 0; r < T::RPT; ++r) zx[r] = xs[row0 + r];
+            float acc[16];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float2 ax = f2(0.f, 0.f);
+#pragma unroll
+                for (int r = 0; r < T::RPT; ++r) ax = ffma2(f2(R[r][2 * j], R[r][2 * j + 1]), f2(zx[r], zx[r]), ax);
+                acc[2 * j] = ax.x;
+                acc[2 * j + 1] = ax.y;
+            }
+            xpose_reduce<16, 16, T::CG>(acc);   // over the warp's row groups
+            constexpr int NR = 16 >> xpose_bits<16, T::CG>();
+            const int base = xpose_base<16, 16, T::CG>(lane);
+            float *dst = (vsel ? rq[warp] : rk[warp]) + T::col(cg, base / 4) + base % 4;
+            if (NR == 4) *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2 % NR], acc[3 % NR]);
+            else *reinterpret_cast<float2 *>(dst) = make_float2(acc[0], acc[1 % NR]);
         }
-        cbar();
+        cbar<NT>();
         if (t < DV) {
             float yk = 0.f, yq = 0.f, kq = 0.f;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) {
+            for (int w = 0; w < kFlushWarps; ++w) {
                 yk += rk[w][t];
                 yq += rq[w][t];
                 kq += F.kqw[w];
@@ -542,7 +585,7 @@ __global__ void __launch_bounds__(kThreads) decode_flush_kernel(const DecodeArgs
             F.u[t] = ut;
             if (!isfinite(o) || !isfinite(ut)) atomicOr(a.status, kStatusNonFinite);
         }
-        cbar();
+        cbar<NT>();
         float uv[16];
         load_cols16<DK, DV>(F.u, uv);
 #pragma unroll
@@ -567,7 +610,7 @@ __global__ void __launch_bounds__(kThreads) decode_flush_kernel(const DecodeArgs
     out.cw = rec_ent + DK;
     out.cw_stride = DK + DV;
     double eacc[T::RPT];
-    codec_quantize<DK, DV, false>(R, L.r, a.K, a.smoothing, P, DAMP ? F.map : nullptr, F.cs, out, eacc);
+    codec_quantize<DK, DV, false, NT>(R, L.r, a.K, a.smoothing, P, DAMP ? F.map : nullptr, F.cs, out, eacc);
     if (KDA) {
         if (t < DK) rec_gam[t] = 1.0f;
     } else if (t == 0) {
@@ -687,7 +730,7 @@ static cudaError_t launch_flush_t(const DecodeArgs &a, int heads, cudaStream_t s
     static size_t done = 0;
     cudaError_t e = set_smem(kern, sm, done);
     if (e != cudaSuccess) return e;
-    kern<<<heads, kThreads, sm, s>>>(a);
+    kern<<<heads, kFlushThreads, sm, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -269,6 +269,7 @@ def lq_quantize_state(cfg: Config, S: torch.Tensor, view: dict, hp_rows=None, st
 
 
 LQ_STATIC_ROWS_MAX = 8192
+LQ_MAX_WINDOW = 4096
 
 
 def lq_quantize_state_static(cfg: Config, S: torch.Tensor, view: dict, hp_rows=None, stream=None):

@@ -68,13 +68,23 @@ def test_workspace_size_matches_record_layout(L):
     ("W", 0, lq.LQ_ERR_INVALID_ARG), ("r", 129, lq.LQ_ERR_INVALID_ARG), ("r", -1, lq.LQ_ERR_INVALID_ARG),
     ("power_iters", -1, lq.LQ_ERR_INVALID_ARG), ("n_hp_rows", 128, lq.LQ_ERR_INVALID_ARG),
     ("smoothing", 2, lq.LQ_ERR_INVALID_ARG), ("fused_flush", 7, lq.LQ_ERR_INVALID_ARG),
-    ("W", 400, lq.LQ_ERR_UNSUPPORTED),
+    ("W", 4097, lq.LQ_ERR_UNSUPPORTED),
 ])
 def test_config_errors(L, field, value, code):
     cfg = lq.Config.from_workload(configs.GDN_SERVING)
     setattr(cfg, field, value)
     assert lq.lq_config_check(cfg) == code
     assert lq.lq_workspace_bytes(cfg) == 0
+
+
+def test_long_windows_are_accepted(L):
+    # the window's buffered entries stream from the workspace; nothing of
+    # their size has to fit in shared memory
+    for W in (400, 4096):
+        cfg = lq.Config.from_workload(configs.GDN_SERVING)
+        cfg.W = W
+        assert lq.lq_config_check(cfg) == lq.LQ_OK
+        assert lq.lq_workspace_bytes(cfg) > 0
 
 
 def test_step_mode_requires_window_one(L):

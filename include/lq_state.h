@@ -211,6 +211,23 @@ int lq_damp_select(const lq_config *cfg, int32_t n_states, const float *d_states
                    int32_t n_gate_samples, const float *d_gates, double *d_energy,
                    int32_t *d_rows, void *stream);
 
+/*
+ * Self-test of the library's internal division (no counterpart in the papers:
+ * a check of an implementation detail).  The codec divides by a per-row
+ * smoothing scale and a per-column quantization scale many times over; it
+ * does so from one correctly rounded reciprocal y = RN(1/b) per divisor and
+ * Markstein's FMA correction step, falling back to IEEE division near the
+ * subnormal range.  This call runs that routine and the IEEE division on
+ * the same operands so that a test can require them to agree bit for bit:
+ *   d_fast[i] = the routine's a[i] / b[i];
+ *   d_pair[i] = the two-lane variant's a[i] / b[i & ~1] (pairs share b);
+ *   d_ieee[i] = IEEE RN a[i] / b[i].
+ * All arrays are device arrays of n floats (n even, >= 0); b[i] > 0.
+ * Returns LQ_OK, LQ_ERR_INVALID_ARG or LQ_ERR_CUDA.
+ */
+int lq_selftest_division(const float *d_a, const float *d_b, float *d_fast, float *d_pair, float *d_ieee,
+                         int32_t n, void *stream);
+
 /* Synchronize `stream` and return the sticky device status of this state:
  * LQ_OK, LQ_ERR_NONFINITE or LQ_ERR_TIMEOUT. */
 int lq_get_status(lq_state *st, void *stream);

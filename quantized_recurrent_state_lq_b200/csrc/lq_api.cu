@@ -442,6 +442,13 @@ int lq_damp_select(const lq_config *cfg, int32_t n_states, const float *d_states
     return cuda_rc(lq::launch_damp_select(a, cfg->dk, cfg->dv, static_cast<cudaStream_t>(stream)));
 }
 
+int lq_selftest_division(const float *d_a, const float *d_b, float *d_fast, float *d_pair, float *d_ieee,
+                         int32_t n, void *stream) {
+    if (n < 0 || (n & 1)) return LQ_ERR_INVALID_ARG;
+    if (n > 0 && (!d_a || !d_b || !d_fast || !d_pair || !d_ieee)) return LQ_ERR_INVALID_ARG;
+    return cuda_rc(lq::launch_div_selftest(d_a, d_b, d_fast, d_pair, d_ieee, n, static_cast<cudaStream_t>(stream)));
+}
+
 int lq_get_status(lq_state *st, void *stream) {
     if (!st) return LQ_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -243,4 +243,26 @@ cudaError_t launch_damp_select(const CodecArgs &a, int dk, int dv, cudaStream_t 
     return cudaGetLastError();
 }
 
+// The codec's division routine beside IEEE division (lq_selftest_division).
+__global__ void div_selftest_kernel(const float *a, const float *b, float *fast, float *pair, float *ieee, int n) {
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;   // pair index
+    if (2 * j >= n) return;
+    const int i0 = 2 * j, i1 = 2 * j + 1;
+    fast[i0] = div_rn(a[i0], b[i0], __frcp_rn(b[i0]));
+    fast[i1] = div_rn(a[i1], b[i1], __frcp_rn(b[i1]));
+    const float2 p = div2_rn(f2(a[i0], a[i1]), b[i0], __frcp_rn(b[i0]));
+    pair[i0] = p.x;
+    pair[i1] = p.y;
+    ieee[i0] = __fdiv_rn(a[i0], b[i0]);
+    ieee[i1] = __fdiv_rn(a[i1], b[i1]);
+}
+
+cudaError_t launch_div_selftest(const float *a, const float *b, float *fast, float *pair, float *ieee, int n,
+                                cudaStream_t s) {
+    const int pairs = n / 2;
+    if (pairs == 0) return cudaSuccess;
+    div_selftest_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(a, b, fast, pair, ieee, n);
+    return cudaGetLastError();
+}
+
 }  // namespace lq

@@ -45,6 +45,7 @@ struct CodecSmem {
     float red[2][NT / 32][DV];   // cross-warp partial column sums (double-buffered)
     float wv[NT / 32][DV];       // per-warp copy of the current power-iteration vector
     float sc[DV];
+    float ysc[DV];               // RN(1 / sc)
     double dred[NT / 32];
 };
 
@@ -340,6 +341,7 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
     // 2. BF16 rows and 3. smoothing scales; x = R / m in place (ENERGY keeps R).
     float m[RPT];
     uint32_t int8mask = 0;   // bit r: row row0 + r is an INT8 row
+    float minabs = INFINITY;  // smallest |R| of the thread's elements
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         const int i = row0 + r;
@@ -358,7 +360,10 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
         // at a time: few registers beside the tile)
         double ss = 0.0;
 #pragma unroll
-        for (int q = 0; q < 16; ++q) ss = fma((double)R[r][q], (double)R[r][q], ss);
+        for (int q = 0; q < 16; ++q) {
+            ss = fma((double)R[r][q], (double)R[r][q], ss);
+            minabs = fminf(minabs, fabsf(R[r][q]));
+        }
 #pragma unroll
         for (int mm = CG / 2; mm >= 1; mm >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, mm);
         float mi = 1.0f;
@@ -378,15 +383,36 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
             for (int r = 0; r < RPT; ++r) out.m[row0 + r] = m[r];
         }
     }
-    // x = R / m (IEEE division, as the oracle); in place unless R is still
-    // needed for the error energy.
+    // x = R / m, correctly rounded (the oracle's IEEE division).  When every
+    // element of the thread is at least 2^-79 in size and every row scale
+    // lies in [2^-20, 2^20], the reciprocal-and-correction division (div_rn)
+    // is exact for all of them -- m is 1 or the row RMS, so |x| <= sqrt(dv)
+    // or the division is by 1 -- and one branch-free loop of packed
+    // operations does it; otherwise the thread divides.  In place unless R
+    // is still needed for the error energy.
     if (!ENERGY) {
+        bool fast = minabs >= 0x1p-79f;
 #pragma unroll
-        for (int r = 0; r < RPT; ++r)
+        for (int r = 0; r < RPT; ++r) fast = fast && m[r] >= 0x1p-20f && m[r] <= 0x1p20f;
+        if (fast) {
 #pragma unroll
-            for (int q = 0; q < 16; ++q) R[r][q] = R[r][q] / m[r];
+            for (int r = 0; r < RPT; ++r) {
+                const float ym = __frcp_rn(m[r]);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float2 x = div2_rn_unchecked(f2(R[r][2 * q], R[r][2 * q + 1]), m[r], ym);
+                    R[r][2 * q] = x.x;
+                    R[r][2 * q + 1] = x.y;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < RPT; ++r)
+#pragma unroll
+                for (int q = 0; q < 16; ++q) R[r][q] = __fdiv_rn(R[r][q], m[r]);
+        }
     }
-    auto X = [&](int r, int q) -> float { return ENERGY ? R[r][q] / m[r] : R[r][q]; };
+    auto X = [&](int r, int q) -> float { return ENERGY ? __fdiv_rn(R[r][q], m[r]) : R[r][q]; };
 
     // 4. Column scales over INT8 rows.
     {
@@ -412,16 +438,27 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
             for (int w = 0; w < T::NW; ++w) a = fmaxf(a, cs.red[buf][w][t]);
             const float sc = a / 127.0f;
             cs.sc[t] = sc;
+            cs.ysc[t] = __frcp_rn(sc);
             if (!ENERGY) out.s[t] = sc;
         }
         cbar<NT>();
     }
 
     // Codes (or the error energy of the INT8 reconstruction).
-    float sv[16];
-    load_cols16<DK, DV>(cs.sc, sv);
-    auto code_of = [&](float x, float s) -> int {
-        return s != 0.f ? (int)fminf(fmaxf(rintf(x / s), -127.f), 127.f) : 0;
+    // C = clamp(rne(x / s)), the quotient correctly rounded as in the oracle.
+    // For a column scale in [2^-20, 2^20] (col_fast) the reciprocal-and-
+    // correction quotient is exact for |x| >= 2^-79 (|x / s| <= 127 for INT8
+    // rows); below that, exact or not, it is under 2^-58 in size and rounds
+    // to code 0 like the exact one: no branch per element.  Other scales (0
+    // included) take IEEE division.  s and 1/s come from shared memory.
+    auto col_fast = [](float sc) -> bool { return sc >= 0x1p-20f && sc <= 0x1p20f; };
+    auto clamp_code = [](float qt) -> uint32_t {
+        return (uint32_t)((int)fminf(fmaxf(rintf(qt), -127.f), 127.f) & 0xff);
+    };
+    auto code_fast = [&](float x, float sc, float ysc) -> uint32_t { return clamp_code(div_rn_unchecked(x, sc, ysc)); };
+    auto code_ieee = [&](float x, float sc) -> uint32_t { return sc != 0.f ? clamp_code(__fdiv_rn(x, sc)) : 0u; };
+    auto code_of = [&](float x, float sc, float ysc) -> uint32_t {
+        return col_fast(sc) ? code_fast(x, sc, ysc) : code_ieee(x, sc);
     };
     if (ENERGY) {
 #pragma unroll
@@ -429,10 +466,17 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
             if (!((int8mask >> r) & 1u)) continue;
             double e = 0.0;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const float dq = ((float)code_of(X(r, q), sv[q]) * sv[q]) * m[r];
-                const double d = (double)R[r][q] - (double)dq;
-                e += d * d;
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 s4 = *reinterpret_cast<const float4 *>(&cs.sc[T::col(cg, q4)]);
+                const float4 y4 = *reinterpret_cast<const float4 *>(&cs.ysc[T::col(cg, q4)]);
+                const float sa[4] = {s4.x, s4.y, s4.z, s4.w}, ya[4] = {y4.x, y4.y, y4.z, y4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int q = 4 * q4 + u;
+                    const float dq = ((float)(int8_t)code_of(X(r, q), sa[u], ya[u]) * sa[u]) * m[r];
+                    const double d = (double)R[r][q] - (double)dq;
+                    e += d * d;
+                }
             }
 #pragma unroll
             for (int mm = CG / 2; mm >= 1; mm >>= 1) e += __shfl_xor_sync(0xffffffffu, e, mm);
@@ -443,14 +487,25 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
         // column are RPT consecutive bytes; one store per column
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
+            const int col = T::col(cg, q / 4) + q % 4;
+            const float sc = cs.sc[col], ysc = cs.ysc[col];
             uint32_t lo = 0u, hi = 0u;
+            if (col_fast(sc)) {
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const uint32_t b = (uint32_t)(code_of(R[r][q], sv[q]) & 0xff);
-                if (r < 4) lo |= b << (8 * r);
-                else hi |= b << (8 * (r - 4));
+                for (int r = 0; r < RPT; ++r) {
+                    const uint32_t b = code_fast(R[r][q], sc, ysc);
+                    if (r < 4) lo |= b << (8 * r);
+                    else hi |= b << (8 * (r - 4));
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    const uint32_t b = code_ieee(R[r][q], sc);
+                    if (r < 4) lo |= b << (8 * r);
+                    else hi |= b << (8 * (r - 4));
+                }
             }
-            int8_t *dst = out.codes + code_off_t(T::col(cg, q / 4) + q % 4, row0, DK);
+            int8_t *dst = out.codes + code_off_t(col, row0, DK);
             if (RPT == 8) *reinterpret_cast<uint2 *>(dst) = make_uint2(lo, hi);
             else if (RPT == 4) *reinterpret_cast<uint32_t *>(dst) = lo;
             else if (RPT == 2) *reinterpret_cast<uint16_t *>(dst) = (uint16_t)lo;
@@ -462,12 +517,16 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
             if (!((int8mask >> r) & 1u)) continue;
             const int i = row0 + r;
             const int slot = (P > 0) ? map[i] : i;
-            uint32_t pk[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int q = 0; q < 16; ++q) pk[q >> 2] |= ((uint32_t)(code_of(R[r][q], sv[q]) & 0xff)) << (8 * (q & 3));
             uint32_t *dst = reinterpret_cast<uint32_t *>(out.codes + (size_t)slot * DV);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) dst[T::col(cg, q) / 4] = pk[q];
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 s4 = *reinterpret_cast<const float4 *>(&cs.sc[T::col(cg, q4)]);
+                const float4 y4 = *reinterpret_cast<const float4 *>(&cs.ysc[T::col(cg, q4)]);
+                const uint32_t pk = code_of(R[r][4 * q4], s4.x, y4.x) | (code_of(R[r][4 * q4 + 1], s4.y, y4.y) << 8) |
+                                    (code_of(R[r][4 * q4 + 2], s4.z, y4.z) << 16) |
+                                    (code_of(R[r][4 * q4 + 3], s4.w, y4.w) << 24);
+                dst[T::col(cg, q4) / 4] = pk;
+            }
         }
     }
     cbar<NT>();

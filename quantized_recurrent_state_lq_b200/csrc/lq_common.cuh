@@ -231,9 +231,49 @@ __device__ __forceinline__ void xpose_allreduce(F (&v)[V]) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Correctly rounded a / b from a precomputed y = RN(1/b), three operations:
+//   q = RN(a y);  r = a - b q (exact, one FMA);  q' = RN(q + r y).
+// Markstein's correction step (P. Markstein, IBM J. Res. Dev. 34(1), 1990;
+// also Muller et al., Handbook of Floating-Point Arithmetic, section on
+// FMA-based division): q' is the IEEE quotient whenever the residual r is
+// exact, i.e. away from the subnormal range.  The guard keeps a, q' and y
+// well inside the normal range (|a|, |q'| >= 2^-100, |q'| <= 2^126,
+// b <= 2^100); everything else -- zeros included -- takes the IEEE division.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool div_fast_ok(float a, float q, float b) {
+    return fabsf(a) >= 0x1p-100f && fabsf(q) >= 0x1p-100f && fabsf(q) <= 0x1p126f && b <= 0x1p100f;
+}
+
+// The three operations alone, for callers that have established the range.
+__device__ __forceinline__ float div_rn_unchecked(float a, float b, float y) {
+    const float q = __fmul_rn(a, y);
+    const float r = __fmaf_rn(-q, b, a);
+    return __fmaf_rn(r, y, q);
+}
+
+__device__ __forceinline__ float div_rn(float a, float b, float y) {
+    const float q2 = div_rn_unchecked(a, b, y);
+    return div_fast_ok(a, q2, b) ? q2 : __fdiv_rn(a, b);
+}
+
 // Two FP32 fused multiply-adds per instruction (sm_100 packed FP32).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// div_rn on a pair of dividends sharing the divisor.
+__device__ __forceinline__ float2 div2_rn_unchecked(float2 a, float b, float y) {
+    const float2 q = __fmul2_rn(a, f2(y, y));
+    const float2 r = __ffma2_rn(q, f2(-b, -b), a);
+    return __ffma2_rn(r, f2(y, y), q);
+}
+
+__device__ __forceinline__ float2 div2_rn(float2 a, float b, float y) {
+    float2 q2 = div2_rn_unchecked(a, b, y);
+    if (!div_fast_ok(a.x, q2.x, b)) q2.x = __fdiv_rn(a.x, b);
+    if (!div_fast_ok(a.y, q2.y, b)) q2.y = __fdiv_rn(a.y, b);
+    return q2;
+}
 
 // Sum of one double per compute thread (warps 0..7); every compute thread
 // gets the result.  `scratch` holds kWarps doubles; two barriers inside.

@@ -71,4 +71,7 @@ cudaError_t launch_dequantize(const CodecArgs &a, int dk, int dv, int heads, cud
 cudaError_t launch_qcopy(const CodecArgs &a, int dk, int dv, int heads, cudaStream_t s);
 cudaError_t launch_damp_select(const CodecArgs &a, int dk, int dv, cudaStream_t s);
 
+cudaError_t launch_div_selftest(const float *a, const float *b, float *fast, float *pair, float *ieee, int n,
+                                cudaStream_t s);
+
 }  // namespace lq

@@ -33,7 +33,7 @@ EXPORTED = ["lq_workspace_bytes", "lq_config_check", "lq_state_init", "lq_decode
             "lq_window_flush", "lq_state_buffered", "lq_state_export_fp32",
             "lq_state_export_view", "lq_state_import_view", "lq_quantize_state",
             "lq_dequantize_state", "lq_quantize_state_static", "lq_damp_select", "lq_get_status",
-            "lq_state_destroy", "lq_strerror"]
+            "lq_state_destroy", "lq_strerror", "lq_selftest_division"]
 
 
 class LqError(RuntimeError):
@@ -83,6 +83,7 @@ def lib():
             "lq_get_status": (C.c_int, [vp, vp]),
             "lq_state_destroy": (None, [vp]),
             "lq_strerror": (C.c_char_p, [C.c_int]),
+            "lq_selftest_division": (C.c_int, [vp, vp, vp, vp, vp, i32, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -282,6 +283,20 @@ def lq_quantize_state_static(cfg: Config, S: torch.Tensor, view: dict, hp_rows=N
     v = _view_struct(cfg, view)
     _chk(lib().lq_quantize_state_static(C.byref(cfg.c()), C.c_void_p(p), p_rows, C.byref(v),
                                         C.c_void_p(_stream(stream))), "lq_quantize_state_static")
+
+
+def lq_selftest_division(a: torch.Tensor, b: torch.Tensor, stream=None):
+    """Run the codec's division routine and IEEE division on the same device
+    operands (float32, same even length; pairs b[2j] == b[2j+1] for the
+    two-lane variant).  Returns (fast, pair, ieee)."""
+    n = a.numel()
+    pa = _dev(a, "a", (n,))
+    pb = _dev(b, "b", (n,))
+    fast, pair, ieee = (torch.empty_like(a) for _ in range(3))
+    _chk(lib().lq_selftest_division(C.c_void_p(pa), C.c_void_p(pb), C.c_void_p(fast.data_ptr()),
+                                    C.c_void_p(pair.data_ptr()), C.c_void_p(ieee.data_ptr()), n,
+                                    C.c_void_p(_stream(stream))), "lq_selftest_division")
+    return fast, pair, ieee
 
 
 def lq_dequantize_state(cfg: Config, view: dict, S: torch.Tensor, hp_rows=None, stream=None):

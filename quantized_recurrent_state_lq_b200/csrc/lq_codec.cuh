@@ -9,7 +9,8 @@
 //      w = 1/sqrt(dv); K times { w = R^T (R w), normalised };  c = R w;
 //      R <- R - c w^T.  (R^T R w normalised is the oracle's z = Rw/|Rw|,
 //      w = R^T z/|R^T z| without the intermediate scaling, which only changes
-//      rounding; norms are accumulated in double.)
+//      rounding.  The FP64 path accumulates norms in double; the FP32 path
+//      takes them in FP32 when safely in range.)
 //   2. BF16 rows: bf16_rne(R_i) for the head's listed key rows.
 //   3. m_i = sqrt(mean_c R_ic^2) (double accumulation), 1 if zero or if
 //      smoothing is off;  x = R / m.
@@ -168,15 +169,39 @@ __device__ int codec_compensators_fp32(float (&R)[Tile<DK, DV, NT>::RPT][16], in
             float4 y;
             tile_cols_matvec<DK, DV, NT>(R, z, cs, buf, y);
             buf ^= 1;
-            if (lane < DV / 4) *reinterpret_cast<float4 *>(&cs.wv[warp][4 * lane]) = y;
-            // |y|^2 accumulated in double; only the reciprocal of the norm is
-            // taken in FP32 (it sets w's length, not its direction).  A zero
-            // norm ends the extraction of this compensator; the remaining
-            // steps then run on zeros / NaN and are discarded.
-            double ss = (double)y.x * y.x + (double)y.y * y.y + (double)y.z * y.z + (double)y.w * y.w;
-            ss = warp_sum_d(ss);
-            zero = zero || (ss == 0.0);
-            inv = 1.0f / (float)sqrt(ss);
+            if (it + 1 < K) {
+                // 1/|y| only sets the next step's length, not its direction:
+                // FP32 sum and reciprocal square root while |y|^2 is
+                // comfortably inside the FP32 range, else the sum again in
+                // double.  A zero norm ends the extraction of this
+                // compensator; the remaining steps then run on zeros / NaN and
+                // are discarded.  (The sums are identical in every lane and
+                // warp, so the branch is uniform.)
+                if (lane < DV / 4) *reinterpret_cast<float4 *>(&cs.wv[warp][4 * lane]) = y;
+                float ssf = fmaf(y.x, y.x, fmaf(y.y, y.y, fmaf(y.z, y.z, y.w * y.w)));
+                ssf = warp_sum(ssf);
+                if (ssf >= 0x1p-100f && ssf <= 0x1p100f) {
+                    inv = rsqrtf(ssf);
+                } else {
+                    double ss = (double)y.x * y.x + (double)y.y * y.y + (double)y.z * y.z + (double)y.w * y.w;
+                    ss = warp_sum_d(ss);
+                    zero = zero || (ss == 0.0);
+                    inv = (float)(1.0 / sqrt(ss));
+                }
+            } else {
+                // The final w_j = y_K / |y_K| with the norm and the division in
+                // double: unlike the per-step scales, |w_j| enters the removed
+                // term c_j w_j^T = R w_j w_j^T squared, and that term can
+                // exceed the residual by the ratio of the first to the
+                // (r+1)-th singular value.
+                double ss = (double)y.x * y.x + (double)y.y * y.y + (double)y.z * y.z + (double)y.w * y.w;
+                ss = warp_sum_d(ss);
+                zero = zero || (ss == 0.0);
+                const double invd = 1.0 / sqrt(ss);
+                if (lane < DV / 4)
+                    *reinterpret_cast<float4 *>(&cs.wv[warp][4 * lane]) =
+                        make_float4((float)(y.x * invd), (float)(y.y * invd), (float)(y.z * invd), (float)(y.w * invd));
+            }
             __syncwarp();
             load_cols16<DK, DV>(cs.wv[warp], w);
             __syncwarp();
@@ -188,8 +213,6 @@ __device__ int codec_compensators_fp32(float (&R)[Tile<DK, DV, NT>::RPT][16], in
             }
             continue;
         }
-#pragma unroll
-        for (int c = 0; c < 16; ++c) w[c] *= inv;
         float c[RPT];
         tile_rows_matvec<DK, DV, NT>(R, w, c);
         if (WRITE) {

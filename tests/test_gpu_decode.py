@@ -107,8 +107,7 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label=""):
             stats["flips"] += c["n"]
             stats["codes"] += c["total"]
             stats["at_tie"] += c["at_tie"]
-            np.testing.assert_allclose(got["m"], ref["view"]["m"], rtol=STATE_REL)
-            np.testing.assert_allclose(got["s"], ref["view"]["s"], rtol=STATE_REL)
+            U.assert_flush_params(cfg, got, ref["view"], ref["S_pre"], hr, label, rel=STATE_REL)
             scale = np.abs(ref["S_pre"]).max(axis=(1, 2))
             for j in range(cfg.r):
                 pg = np.einsum("hi,hc->hic", got["c"][:, j], got["w"][:, j])

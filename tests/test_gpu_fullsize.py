@@ -104,5 +104,4 @@ def test_full_size_sampled_heads(wl):
     c = U.compare_codes(got["codes"], ref["view"]["codes"], ratio)
     print(f"{wl.name}: flushed codes {c}")
     U.assert_code_bar(c, wl.name + " flushed", U.FLUSH_FLIP_FRAC)
-    np.testing.assert_allclose(got["s"], ref["view"]["s"], rtol=1e-3)
-    np.testing.assert_allclose(got["m"], ref["view"]["m"], rtol=1e-3)
+    U.assert_flush_params(sub, got, ref["view"], ref["S_pre"], hr, wl.name + " flushed")

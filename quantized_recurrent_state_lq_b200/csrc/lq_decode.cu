@@ -38,17 +38,23 @@ namespace lq {
 //       products reduced by a transpose-reduce butterfly.
 //   (e) per-warp partial column sums combined; output, append.           barrier
 // ---------------------------------------------------------------------------
+// Warps of a buffering CTA: 4 warps and ~31 KB of shared memory let 7 heads
+// be in flight on an SM (the per-head critical path -- step inputs, the
+// staged codes, the tensor-core GEMV, the entry stream -- is latency-bound).
+constexpr int kBufWarps = 4;
+constexpr int kBufThreads = kBufWarps * 32;
+
 template <int DK, int DV>
 struct BufSmem {
     float2 x2[DK];                      // (Gamma k, Gamma q) by key row
     float2 a2[DK];                      // m * x2 by INT8 slot (BF16-row layout)
-    float2 red[kWarps][DV];             // per-warp partial column sums (BF16 rows + entries)
+    float2 red[kBufWarps][DV];             // per-warp partial column sums (BF16 rows + entries)
     float2 rc[DV];                      // codes part of (y_k, y_q)
     int8_t dig[8][DK + 16];             // base-256 digits of a_k (rows 0-3) and a_q (rows 4-7)
     int rows[DK];                       // DAMP: key row of INT8 slot j, then of BF16 row p
     float v[DV];
-    float amax[kWarps][2];
-    float kqw[kWarps];
+    float amax[kBufWarps][2];
+    float kqw[kBufWarps];
     uint64_t mbar;
 };
 
@@ -112,7 +118,7 @@ __device__ __forceinline__ void warp_reduce_dots(float (&v)[2 * NE]) {
 }
 
 template <int DK, int DV, bool KDA, bool DAMP>
-__global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     BufSmem<DK, DV> &S = *reinterpret_cast<BufSmem<DK, DV> *>(smem);
     unsigned char *stage = smem + buf_fixed_bytes<DK, DV>();
@@ -196,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
     __syncthreads();
     float kq = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) kq += S.kqw[w];
+    for (int w = 0; w < kBufWarps; ++w) kq += S.kqw[w];
 
     // (b) the tensor-core operand: a_k, a_q as exact signed base-256 digits of
     // one fixed-point integer each, X = a * 2^(30 - e) with |a| < 2^e.
@@ -204,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
     if (!DAMP) {
         float mk = 0.f, mq = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < kBufWarps; ++w) {
             mk = fmaxf(mk, S.amax[w][0]);
             mq = fmaxf(mq, S.amax[w][1]);
         }
@@ -240,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
     // (c) codes.
     float ek[4] = {0.f, 0.f, 0.f, 0.f}, eq[4] = {0.f, 0.f, 0.f, 0.f};
     if (!DAMP) {
-        if (warp < DV / 16) {   // one warp per 16 value columns
-            const int c0 = 16 * warp;
+        for (int cb = warp; cb < DV / 16; cb += kBufWarps) {   // a warp per 16 value columns
+            const int c0 = 16 * cb;
             const int gq = lane >> 2, tq = lane & 3;
             const unsigned char *codes = stage + L.off_codes;
             const int r = ((lane >> 3) & 1) * 8 + (lane & 7), blk = lane >> 4;
@@ -281,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
         const unsigned char *codes = stage + L.off_codes;
         float ak[4] = {0.f, 0.f, 0.f, 0.f}, aq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
-        for (int j = warp * RPP + rsub; j < NI; j += kWarps * RPP) {
+        for (int j = warp * RPP + rsub; j < NI; j += kBufWarps * RPP) {
             const uint32_t w = *reinterpret_cast<const uint32_t *>(codes + (size_t)j * DV + 4 * cq);
             const float2 av = S.a2[j];
             float f[4];
@@ -309,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
             }
         }
         const uint16_t *hp = reinterpret_cast<const uint16_t *>(stage + L.off_hp);
-        for (int p = warp; p < P; p += kWarps) {   // BF16 rows: unscaled x
+        for (int p = warp; p < P; p += kBufWarps) {   // BF16 rows: unscaled x
             if (lane < DV / 4) {
                 const uint2 hb = *reinterpret_cast<const uint2 *>(hp + (size_t)p * DV + 4 * lane);
                 const float2 x = S.x2[S.rows[NI + p]];
@@ -332,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
             xk[u] = x.x;
             xq[u] = x.y;
         }
-        for (int e0 = 2 * warp; e0 < E; e0 += 2 * kWarps) {
+        for (int e0 = 2 * warp; e0 < E; e0 += 2 * kBufWarps) {
             float d[4];
             float4 uv[2];
 #pragma unroll
@@ -354,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
                 uv[p] = ub[p];
             }
             const int ne = min(2, E - e0);
-            load_pair(e0 + 2 * kWarps);   // refill the registers while this pair is reduced
+            load_pair(e0 + 2 * kBufWarps);   // refill the registers while this pair is reduced
             warp_reduce_dots<2>(d);
             if (lane < DV / 4) {
 #pragma unroll
@@ -379,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_buffer_kernel(const Decode
     if (t < DV) {
         float yk = DAMP ? 0.f : S.rc[t].x, yq = DAMP ? 0.f : S.rc[t].y;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < kBufWarps; ++w) {
             const float2 p = S.red[w][t];
             yk += p.x;
             yq += p.y;
@@ -719,7 +725,7 @@ static cudaError_t launch_buffer_t(const DecodeArgs &a, int heads, cudaStream_t 
     static size_t done = 0;
     cudaError_t e = set_smem(kern, sm, done);
     if (e != cudaSuccess) return e;
-    kern<<<heads, kThreads, sm, s>>>(a);
+    kern<<<heads, kBufThreads, sm, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -574,21 +574,22 @@ __device__ void codec_quantize_exact(float (&R)[Tile<DK, DV>::RPT][16], int r_co
 }
 
 // Reconstruction of a head's current state into the tile, in three parts:
-//   tile_dequant:      R = Deq(C, m, s) [BF16 rows widened]
+//   tile_dequant:      R = Deq(C, m, s) [BF16 rows widened]  (ADD: R += ...)
 //   tile_add_entries:  R += sum_e ktil_e u_e^T over n entries [n][DK+DV]
 //   tile_gamma:        R *= Gamma (by key row); true if every value is finite
 // The arrays may live in shared or global memory: m_s [DK], s_s [DV],
 // hp_s [P][DV], codes_s (layout per codes_t), gam_s [DK].
-template <int DK, int DV, int NT>
+template <int DK, int DV, int NT, bool ADD = false>
 __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][16], const float *m_s,
                                              const float *s_s, const uint16_t *hp_s, const int8_t *codes_s, int P,
                                              const int *map, bool codes_t) {
     using T = Tile<DK, DV, NT>;
     constexpr int RPT = T::RPT;
     const int t = threadIdx.x, cg = t % T::CG, rg = t / T::CG, row0 = rg * RPT;
-    float sv[16];
-    load_cols16<DK, DV>(s_s, sv);
+    auto put = [&](int r, int q, float v) { R[r][q] = ADD ? R[r][q] + v : v; };
     if (codes_t && (RPT == 4 || RPT == 8)) {
+        float sv[16];
+        load_cols16<DK, DV>(s_s, sv);
         // value-column-major codes (no BF16 rows): the thread's RPT rows of
         // one column are RPT consecutive bytes
         float mi[RPT];
@@ -615,7 +616,7 @@ __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][1
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const int r = 4 * h + k;
-                        R[r % RPT][4 * q + u] = (f[k] * sv[4 * q + u]) * mi[r % RPT];
+                        put(r % RPT, 4 * q + u, (f[k] * sv[4 * q + u]) * mi[r % RPT]);
                     }
                 }
             }
@@ -628,31 +629,36 @@ __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][1
         if (mp >= 0 && codes_t) {
             const float mi = m_s[i];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < 4; ++q) {
+                const float4 s4 = *reinterpret_cast<const float4 *>(s_s + T::col(cg, q));
+                const float sq[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const float cf = (float)codes_s[code_off_t(T::col(cg, q) + u, i, DK)];
-                    R[r][4 * q + u] = (cf * sv[4 * q + u]) * mi;
+                    put(r, 4 * q + u, (cf * sq[u]) * mi);
                 }
+            }
         } else if (mp >= 0) {
             const float mi = m_s[i];
             const uint32_t *row = reinterpret_cast<const uint32_t *>(codes_s + (size_t)mp * DV);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
+                const float4 s4 = *reinterpret_cast<const float4 *>(s_s + T::col(cg, q));
+                const float sq[4] = {s4.x, s4.y, s4.z, s4.w};
                 float f[4];
                 s8x4_to_f(row[T::col(cg, q) / 4], f);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) R[r][4 * q + u] = (f[u] * sv[4 * q + u]) * mi;
+                for (int u = 0; u < 4; ++u) put(r, 4 * q + u, (f[u] * sq[u]) * mi);
             }
         } else {
             const int p = -1 - mp;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const uint2 h = *reinterpret_cast<const uint2 *>(hp_s + (size_t)p * DV + T::col(cg, q));
-                R[r][4 * q] = bf16_to_f((uint16_t)(h.x & 0xffff));
-                R[r][4 * q + 1] = bf16_to_f((uint16_t)(h.x >> 16));
-                R[r][4 * q + 2] = bf16_to_f((uint16_t)(h.y & 0xffff));
-                R[r][4 * q + 3] = bf16_to_f((uint16_t)(h.y >> 16));
+                put(r, 4 * q, bf16_to_f((uint16_t)(h.x & 0xffff)));
+                put(r, 4 * q + 1, bf16_to_f((uint16_t)(h.x >> 16)));
+                put(r, 4 * q + 2, bf16_to_f((uint16_t)(h.y & 0xffff)));
+                put(r, 4 * q + 3, bf16_to_f((uint16_t)(h.y >> 16)));
             }
         }
     }

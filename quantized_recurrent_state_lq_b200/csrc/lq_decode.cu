@@ -18,6 +18,7 @@
 // the step that ends a window runs decode_flush_kernel (one CTA per head,
 // state rebuilt in registers and requantized).
 #include "lq_codec.cuh"
+#include "lq_tc.cuh"
 #include "lq_kernels.h"
 
 namespace lq {
@@ -418,7 +419,7 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
 // ---------------------------------------------------------------------------
 constexpr int kFlushThreads = 128;
 constexpr int kFlushWarps = kFlushThreads / 32;
-constexpr int kFlushChunk = 16;
+constexpr int kFlushChunk = 8;   // entries per staged chunk: one TF32 MMA K-block
 
 template <int DK, int DV>
 struct FlushSmem {
@@ -430,6 +431,8 @@ struct FlushSmem {
     CodecSmem<DK, DV, kFlushThreads> cs;
     uint64_t mbar_pre;
     uint64_t mbar_ent[2];
+    uint64_t mbar_mma[2];
+    uint32_t tmem_base;
 };
 
 template <int DK, int DV>
@@ -437,7 +440,21 @@ __host__ __device__ constexpr size_t flush_fixed_bytes() {
     return (sizeof(FlushSmem<DK, DV>) + 127) / 128 * 128;
 }
 
+// Shared memory of the flush, in this order (all 128-byte aligned):
+//   FlushSmem | work area | record prefix
+// d_k = 128 (tensor-core reconstruction): the work area holds two operand
+// buffers, each the TF32 big / small parts of one chunk's ktil^T [dk][8] and
+// u^T [dv][8] in K-major core-matrix layout; the entries come from global
+// memory into registers one chunk ahead.  They come before the prefix so that
+// everything a descriptor can address stays inside the allocation.
+// d_k = 64: the work area stages the entries, two chunk buffers
+// [kFlushChunk][dk+dv] filled by bulk copies.
+// Either way the work area doubles as the accumulator's transposition scratch.
+__host__ __device__ inline size_t flush_ops_bytes(int dk, int dv) { return (size_t)2 * (dk + dv) * 32; }
 __host__ __device__ inline size_t flush_chunk_bytes(int dk, int dv) { return (size_t)kFlushChunk * (dk + dv) * 4; }
+__host__ __device__ inline size_t flush_work_bytes(int dk, int dv) {
+    return dk == 128 ? 2 * flush_ops_bytes(dk, dv) : 2 * flush_chunk_bytes(dk, dv);
+}
 
 size_t flush_smem_bytes(int dk, int dv, const Layout &L) {
     size_t fixed = 0;
@@ -445,7 +462,7 @@ size_t flush_smem_bytes(int dk, int dv, const Layout &L) {
     if (dk == 64 && dv == 128) fixed = flush_fixed_bytes<64, 128>();
     if (dk == 128 && dv == 64) fixed = flush_fixed_bytes<128, 64>();
     if (dk == 128 && dv == 128) fixed = flush_fixed_bytes<128, 128>();
-    return fixed + (size_t)align_up(L.off_ent, 128) + 2 * flush_chunk_bytes(dk, dv);
+    return fixed + flush_work_bytes(dk, dv) + (size_t)align_up(L.off_ent, 128);
 }
 
 enum { kFlushStep = 0, kFlushOnly = 1, kExport = 2 };
@@ -458,8 +475,9 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
     using T = Tile<DK, DV, NT>;
     FlushSmem<DK, DV> &F = *reinterpret_cast<FlushSmem<DK, DV> *>(smem);
     const Layout &L = a.L;
-    unsigned char *stage = smem + flush_fixed_bytes<DK, DV>();
-    float *ebuf = reinterpret_cast<float *>(stage + align_up(L.off_ent, 128));   // [2][kFlushChunk][EF]
+    unsigned char *work = smem + flush_fixed_bytes<DK, DV>();
+    float *ebuf = reinterpret_cast<float *>(work);   // d_k = 64: [2][kFlushChunk][EF]
+    unsigned char *stage = work + flush_work_bytes(DK, DV);
     const int head = blockIdx.x;
     const int b = head / a.H, h = head - b * a.H, g = (h * a.Hk) / a.H;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -492,10 +510,12 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
         mbar_init(&F.mbar_pre, 1);
         mbar_init(&F.mbar_ent[0], 1);
         mbar_init(&F.mbar_ent[1], 1);
+        mbar_init(&F.mbar_mma[0], 1);
+        mbar_init(&F.mbar_mma[1], 1);
         fence_mbar_init();
     }
     __syncthreads();
-    int issued = min(nch, 2);
+    int issued = DK == 128 ? 0 : min(nch, 2);   // entry chunks bulk-copied (d_k = 64)
     if (t == 0) {
         mbar_arrive_expect_tx(&F.mbar_pre, (uint32_t)L.off_ent);
         bulk_g2s(stage, rec, (uint32_t)L.off_ent, &F.mbar_pre);
@@ -524,24 +544,168 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
         return;
     }
 
+    // R = sum_e ktil_e u_e^T over the r + n entries, then += Deq, then * Gamma.
     float R[T::RPT][16];
-    tile_dequant<DK, DV, NT>(R, reinterpret_cast<const float *>(stage + L.off_m),
-                             reinterpret_cast<const float *>(stage + L.off_s),
-                             reinterpret_cast<const uint16_t *>(stage + L.off_hp),
-                             reinterpret_cast<const int8_t *>(stage + L.off_codes), P, DAMP ? F.map : nullptr, !DAMP);
-    for (int c = 0; c < nch; ++c) {
-        const bool ok = mbar_wait_bounded(&F.mbar_ent[c & 1], (c >> 1) & 1, a.status);
-        // also the barrier after which buffer (c+1) & 1 -- chunk c-1 -- is free
-        if (__syncthreads_or(!ok)) {
-            drain(c + 1, issued);
-            return;
+    auto zero_tile = [&]() {
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r)
+#pragma unroll
+            for (int q = 0; q < 16; ++q) R[r][q] = 0.f;
+    };
+    if constexpr (DK == 128) {
+        // On the tensor cores: per chunk of 8 entries, A = ktil^T [128][8] and
+        // B = u^T [DV][8] split into TF32 big + small parts, three MMAs (big
+        // big, big small, small big) accumulating D [128][DV] in tensor
+        // memory.  The entries of chunk c+1 are loaded into registers while
+        // chunk c is converted; operand buffer c & 1 is reused once the MMAs
+        // of chunk c-2, committed to mbar_mma[c & 1], have completed.
+        if (nch == 0) {
+            zero_tile();
+        } else {
+            constexpr uint32_t TCOLS = DV;   // 64 or 128 columns: a power of two >= 32
+            constexpr uint32_t IDESC = umma_idesc_tf32(DK, DV);
+            constexpr int OPW = (int)((2 * (DK + DV) * 32) / 4);   // words per operand buffer
+            if (warp == 0) {
+                tmem_alloc(&F.tmem_base, TCOLS);
+                tmem_relinquish();
+            }
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            const uint32_t tmem = F.tmem_base;
+            // row x of a K-major [rows][8] TF32 operand: 16 bytes (4 words) per
+            // core-matrix row, core matrices of 8 rows 128 bytes (32 words)
+            // apart (SBO), the second 16 bytes of K rows*16 bytes further (LBO)
+            auto put_row = [&](uint32_t *big, uint32_t *small, int rows, int x, const float (&src)[8]) {
+                uint32_t hb[8], hs[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) tf32_split(src[e], hb[e], hs[e]);
+                uint32_t *pb = big + (x >> 3) * 32 + (x & 7) * 4;
+                uint32_t *ps = small + (x >> 3) * 32 + (x & 7) * 4;
+                *reinterpret_cast<uint4 *>(pb) = make_uint4(hb[0], hb[1], hb[2], hb[3]);
+                *reinterpret_cast<uint4 *>(pb + rows * 4) = make_uint4(hb[4], hb[5], hb[6], hb[7]);
+                *reinterpret_cast<uint4 *>(ps) = make_uint4(hs[0], hs[1], hs[2], hs[3]);
+                *reinterpret_cast<uint4 *>(ps + rows * 4) = make_uint4(hs[4], hs[5], hs[6], hs[7]);
+            };
+            // chunk entries of this thread's key row / value column, a ring of
+            // PF chunks in registers (slot = chunk % PF, a compile-time index
+            // inside the unrolled loop): loads run PF chunks ahead of use
+            constexpr int PF = 1;
+            float xa[PF][8], xb[PF][8];
+            auto load_chunk = [&](int c, float (&ya)[8], float (&yb)[8]) {
+                const int n = min(kFlushChunk, E - c * kFlushChunk);
+                const float *src = rec_ent + (size_t)c * kFlushChunk * EF;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    ya[e] = e < n ? __ldcs(src + e * EF + t) : 0.f;
+                    yb[e] = (e < n && t < DV) ? __ldcs(src + e * EF + DK + t) : 0.f;
+                }
+            };
+#pragma unroll
+            for (int s2 = 0; s2 < PF; ++s2)
+                if (s2 < nch) load_chunk(s2, xa[s2], xb[s2]);
+            int c = 0;   // chunks committed
+            bool ok = true;
+            for (int c0 = 0; c0 < nch && ok; c0 += PF) {
+#pragma unroll
+                for (int s2 = 0; s2 < PF; ++s2) {
+                    const int cc = c0 + s2;
+                    if (cc < nch && ok) {
+                        uint32_t *opA_big = reinterpret_cast<uint32_t *>(work) + (cc & 1) * OPW;
+                        uint32_t *opA_small = opA_big + DK * 8;
+                        uint32_t *opB_big = opA_small + DK * 8;
+                        uint32_t *opB_small = opB_big + DV * 8;
+                        const bool okc =
+                            cc < 2 || mbar_wait_bounded(&F.mbar_mma[cc & 1], ((cc >> 1) - 1) & 1, a.status);
+                        if (__syncthreads_or(!okc)) {
+                            ok = false;
+                        } else {
+                            put_row(opA_big, opA_small, DK, t, xa[s2]);
+                            if (t < DV) put_row(opB_big, opB_small, DV, t, xb[s2]);
+                            if (cc + PF < nch) load_chunk(cc + PF, xa[s2], xb[s2]);
+                            fence_async_smem();
+                            tc_fence_before();
+                            __syncthreads();
+                            if (t == 0) {
+                                tc_fence_after();
+                                const uint64_t ab = umma_smem_desc(opA_big, DK * 16, 128);
+                                const uint64_t as = umma_smem_desc(opA_small, DK * 16, 128);
+                                const uint64_t bb = umma_smem_desc(opB_big, DV * 16, 128);
+                                const uint64_t bs = umma_smem_desc(opB_small, DV * 16, 128);
+                                umma_tf32(tmem, ab, bb, IDESC, cc > 0 ? 1u : 0u);
+                                umma_tf32(tmem, ab, bs, IDESC, 1u);
+                                umma_tf32(tmem, as, bb, IDESC, 1u);
+                                umma_commit(&F.mbar_mma[cc & 1]);
+                            }
+                            c = cc + 1;
+                        }
+                    }
+                }
+            }
+            // chunks 0 .. c-1 were committed; the last commit completes after
+            // every earlier MMA
+            bool okm = c == 0 || mbar_wait_bounded(&F.mbar_mma[(c - 1) & 1], ((c - 1) >> 1) & 1, a.status);
+            okm = !__syncthreads_or(!okm) && ok;
+            tc_fence_after();
+            if (okm) {
+                // D -> register tile in four slices of DV/4 columns through
+                // the work area (both operand buffers, consumed): thread l of
+                // warp w holds D row 32 w + l of the slice
+                constexpr int SW = DV / 4, SP = SW + 4;   // slice width, padded row pitch
+                float *scr = reinterpret_cast<float *>(work);
+#pragma unroll
+                for (int qs = 0; qs < 4; ++qs) {
+                    uint32_t v[SW];
+                    tmem_ld_32x32b<SW>(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(qs * SW), v);
+                    tmem_ld_wait();
+                    float *rowp = scr + (size_t)(32 * warp + lane) * SP;
+#pragma unroll
+                    for (int j = 0; j < SW / 4; ++j)
+                        *reinterpret_cast<float4 *>(rowp + 4 * j) =
+                            make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                        __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                    __syncthreads();
+#pragma unroll
+                    for (int r = 0; r < T::RPT; ++r) {
+                        const float4 f = *reinterpret_cast<const float4 *>(scr + (size_t)(row0 + r) * SP + 4 * cg);
+                        R[r][4 * qs] = f.x;
+                        R[r][4 * qs + 1] = f.y;
+                        R[r][4 * qs + 2] = f.z;
+                        R[r][4 * qs + 3] = f.w;
+                    }
+                    __syncthreads();
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+            if (warp == 0) {
+                tc_fence_after();
+                tmem_dealloc(tmem, TCOLS);
+            }
+            if (!okm) return;
         }
-        if (c >= 1 && c + 1 < nch) {
-            if (t == 0) issue_chunk(c + 1);
-            ++issued;
+    } else {
+        zero_tile();
+        for (int c = 0; c < nch; ++c) {
+            const bool ok = mbar_wait_bounded(&F.mbar_ent[c & 1], (c >> 1) & 1, a.status);
+            // also the barrier after which buffer (c+1) & 1 -- chunk c-1 -- is free
+            if (__syncthreads_or(!ok)) {
+                drain(c + 1, issued);
+                return;
+            }
+            if (c >= 1 && c + 1 < nch) {
+                if (t == 0) issue_chunk(c + 1);
+                ++issued;
+            }
+            tile_add_entries<DK, DV, NT>(R, ebuf + (size_t)(c & 1) * kFlushChunk * EF,
+                                         min(kFlushChunk, E - c * kFlushChunk));
         }
-        tile_add_entries<DK, DV, NT>(R, ebuf + (size_t)(c & 1) * kFlushChunk * EF, min(kFlushChunk, E - c * kFlushChunk));
     }
+    tile_dequant<DK, DV, NT, true>(R, reinterpret_cast<const float *>(stage + L.off_m),
+                                   reinterpret_cast<const float *>(stage + L.off_s),
+                                   reinterpret_cast<const uint16_t *>(stage + L.off_hp),
+                                   reinterpret_cast<const int8_t *>(stage + L.off_codes), P, DAMP ? F.map : nullptr,
+                                   !DAMP);
     const bool fin = tile_gamma<DK, DV, NT>(R, F.gam);
     if (!fin) atomicOr(a.status, kStatusNonFinite);
 

@@ -1,0 +1,118 @@
+// lq_tc.cuh -- 5th-generation tensor-core (tcgen05) helpers for sm_100a: tensor
+// memory allocation, shared-memory operand descriptors, TF32 MMA issue,
+// completion tracking and accumulator loads.
+//
+// Formats (from the PTX ISA's tcgen05 chapter; the same bit layouts as
+// CUTLASS's UMMA::SmemDescriptor / UMMA::InstrDescriptor for sm100):
+//   shared-memory descriptor, 64 bits:
+//     [0,14)  start address >> 4      [16,30) leading byte offset >> 4
+//     [32,46) stride byte offset >> 4 [46,48) version = 1
+//     [49,52) base offset = 0         [52]    LBO mode = 0
+//     [61,64) layout: 0 = no swizzle
+//   A K-major operand without swizzle is made of 8-row x 16-byte core
+//   matrices: row r of a core matrix at +16 r, the next 8 rows at +SBO, the
+//   next 16 bytes along K at +LBO.
+//   instruction descriptor, 32 bits (.kind::tf32, dense):
+//     [4,6) D format: 1 = F32   [7,10) A format: 2 = TF32   [10,13) B format: 2
+//     [15] A major: 0 = K       [16] B major: 0 = K
+//     [17,23) N >> 3            [24,29) M >> 4
+#pragma once
+
+#include "lq_common.cuh"
+
+namespace lq {
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Generic-proxy shared-memory writes become visible to the tensor core (async
+// proxy) after this fence and a barrier.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ uint64_t umma_smem_desc(const void *base, uint32_t lbo, uint32_t sbo) {
+    const uint64_t a = (uint64_t)((smem_u32(base) & 0x3FFFFu) >> 4);
+    return a | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) |
+           (1ull << 46);
+}
+
+__host__ __device__ constexpr uint32_t umma_idesc_tf32(int M, int N) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D (tensor memory) = A B^T (+ D if accumulate), A [M][K], B [N][K] K-major.
+// Issued by one thread.
+__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// One arrival on the mbarrier once every tcgen05.mma this thread issued before
+// has completed (its operand reads included).
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Thread l of the warp reads tensor-memory lane (taddr.lane + l), columns
+// taddr.col .. taddr.col + N - 1 (shape 32x32b, N = 16 or 32).
+template <int N>
+__device__ __forceinline__ void tmem_ld_32x32b(uint32_t taddr, uint32_t (&v)[N]);
+
+template <>
+__device__ __forceinline__ void tmem_ld_32x32b<32>(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld_32x32b<16>(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// x = big + small with big, small representable in TF32: big = x rounded to
+// nearest (ties away from zero) at TF32's 10 stored mantissa bits -- add half a
+// TF32 unit to the bit pattern, clear the 13 low bits -- the rest x - big
+// (exact) truncated to TF32.  Integer and FP32 ALU operations only (the
+// conversion instruction runs at a lower rate); the three products
+// big*big + big*small + small*big of a 3-pass TF32 MMA carry about 22 bits of
+// each operand.  (Finite x below the FP32 maximum; no operand here comes close.)
+__device__ __forceinline__ void tf32_split(float x, uint32_t &big, uint32_t &small) {
+    big = (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
+    const float rest = x - __uint_as_float(big);
+    small = __float_as_uint(rest) & 0xFFFFE000u;
+}
+
+}  // namespace lq

@@ -116,11 +116,11 @@ def compare_codes(gpu: np.ndarray, orc: np.ndarray, ratio: np.ndarray | None, ti
 
 def assert_flush_params(cfg: lq.Config, got: dict, want: dict, S_pre: np.ndarray, hp_rows, label: str = "",
                         rel: float = 1e-3, guard: float = 1e-2):
-    """m, s and the compensators of a flush, judged by the window-start state
-    they produce.  With the oracle's codes and BF16 rows on both sides (flips
-    are counted on their own), Deq(C; m, s) + sum_j c_j w_j^T from the GPU's
-    parameters must match the oracle's within `rel` of max|S_pre| per head --
-    the FP32-state bar.  Per-element m, s are only guarded against gross error
+    """m, s, BF16 rows and the compensators of a flush, judged by the
+    window-start state they produce.  With the oracle's codes on both sides
+    (flips are counted on their own), Deq(C; m, s, BF16 rows) + sum_j c_j w_j^T
+    from the GPU's parameters must match the oracle's within `rel` of
+    max|S_pre| per head -- the FP32-state bar.  Per-element m, s are only guarded against gross error
     (`guard` relative): an FP32 power iteration on a state whose leading
     singular values dwarf the residual moves a residual column's amax by far
     more, relatively, than it moves the state.  `got`/`want` are oracle-layout
@@ -132,9 +132,9 @@ def assert_flush_params(cfg: lq.Config, got: dict, want: dict, S_pre: np.ndarray
     worst = 0.0
     for h in range(nh):
         hr = None if hp_rows is None else hp_rows[h]
-        base = {"codes": want["codes"][h], "hp": want["hp"][h]}
-        mine = dict(base, m=got["m"][h], s=got["s"][h], c=got["c"][h], w=got["w"][h])
-        ref = dict(base, m=want["m"][h], s=want["s"][h], c=want["c"][h], w=want["w"][h])
+        base = {"codes": want["codes"][h]}
+        mine = dict(base, hp=got["hp"][h], m=got["m"][h], s=got["s"][h], c=got["c"][h], w=got["w"][h])
+        ref = dict(base, hp=want["hp"][h], m=want["m"][h], s=want["s"][h], c=want["c"][h], w=want["w"][h])
         dg = O.dequantize(oc, mine, hp_rows=hr)
         dr = O.dequantize(oc, ref, hp_rows=hr)
         e = float(np.abs(dg - dr).max() / max(np.abs(S_pre[h]).max(), 1e-30))

@@ -114,9 +114,15 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label=""):
                 pw = np.einsum("hi,hc->hic", ref["view"]["c"][:, j], ref["view"]["w"][:, j])
                 assert (np.abs(pg - pw).max(axis=(1, 2)) <= STATE_REL * scale).all()
             if cfg.n_hp_rows:
-                hpg = got["hp"][:, :cfg.n_hp_rows].view(np.int16).astype(np.int32)
-                hpw = ref["view"]["hp"][:, :cfg.n_hp_rows].view(np.int16).astype(np.int32)
-                assert np.abs(hpg - hpw).max() <= 1   # one bf16 ulp at a rounding tie
+                # BF16 rows enter the window-start state check above; per
+                # element: one bf16 ulp (a rounding tie), or -- for elements
+                # far below the head's largest -- within the state bar of it
+                hpg = got["hp"][:, :cfg.n_hp_rows]
+                hpw = ref["view"]["hp"][:, :cfg.n_hp_rows]
+                ulps = np.abs(hpg.view(np.int16).astype(np.int32) - hpw.view(np.int16).astype(np.int32))
+                f = lambda x: (x.astype(np.uint32) << 16).view(np.float32)
+                dv = np.abs(f(hpg) - f(hpw))
+                assert ((ulps <= 1) | (dv <= STATE_REL * scale[:, None, None])).all()
         ov = ref["view"]
         t0 += n
     assert lq.lq_get_status(st) == lq.LQ_OK

@@ -306,7 +306,8 @@ def run_ours(args, wl, world, rank, pg):
                     "frac_of_measured": step_bytes * args.steps / dt / 1e9 / peaks["hbm_gbs"],
                     "algorithmic_bytes_per_step": step_bytes},
             "kernels": {"decode_buffering_mean_s": t_buf, "decode_flushing_mean_s": t_flush},
-            "roofline": roof, "gpu_launches": wl.W * args.steps, "clocks": clk.summary()}
+            "roofline": roof, "gpu_launches": wl.W * args.steps, "clocks": clk.summary(),
+            "state_bits_per_value": traffic.bits_per_value(wl)}
 
     e2e_steps = max(1, min(args.steps, 5))
     dte, h2d, d2h = e2e_measure(r, e2e_steps, stream)

@@ -60,3 +60,15 @@ def fp32_step_bytes(wl: Workload) -> float:
 
 def step_int8_bytes(wl: Workload) -> float:
     return io_bytes(wl) + 2 * state_bytes(wl)
+
+
+def bits_per_value(wl: Workload) -> dict:
+    """Effective bits per state value of the window-start state (the DAMP
+    abstract reports its state-storage saving; it gives no definition, so both
+    readings are reported): `payload` counts the codes and the BF16 rows only,
+    (8 (dk-P) + 16 P) / dk; `total` adds the FP32 smoothing and column scales
+    and the r compensators, 32 (dk + dv) (1 + r) / (dk dv).  The transient
+    window buffer is excluded (it is the method's FP32 update stream)."""
+    payload = (8 * (wl.dk - wl.P) + 16 * wl.P) / wl.dk
+    total = payload + 32 * (wl.dk + wl.dv) * (1 + wl.r) / (wl.dk * wl.dv)
+    return {"payload": payload, "total": total, "fp32_reference": 32.0}

@@ -148,3 +148,15 @@ def test_strerror_covers_every_status(L):
     for code in range(-8, 1):
         assert lq.strerror(code) != "unknown status"
     assert lq.strerror(-99) == "unknown status"
+
+
+def test_effective_bits_per_state_value():
+    # payload: codes + BF16 rows; total: + FP32 m, s and r compensators
+    # (8 (dk-P) + 16 P) / dk and 32 (dk + dv)(1 + r) / (dk dv)
+    from quantized_recurrent_state_lq_b200 import traffic
+    b = traffic.bits_per_value(configs.GDN_DAMP)          # P = 16 of 128 rows, r = 2
+    assert b["payload"] == pytest.approx(9.0) and b["total"] == pytest.approx(10.5)
+    b = traffic.bits_per_value(configs.GDN_PREFIX_CACHE)  # r = 4
+    assert b["payload"] == pytest.approx(8.0) and b["total"] == pytest.approx(10.5)
+    b = traffic.bits_per_value(configs.TINY_GDN)          # d = 64, r = 2
+    assert b["payload"] == pytest.approx(8.0) and b["total"] == pytest.approx(11.0)

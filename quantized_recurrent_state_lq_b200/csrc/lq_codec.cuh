@@ -475,8 +475,13 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
     // to code 0 like the exact one: no branch per element.  Other scales (0
     // included) take IEEE division.  s and 1/s come from shared memory.
     auto col_fast = [](float sc) -> bool { return sc >= 0x1p-20f && sc <= 0x1p20f; };
+    // clamp, then round half to even and convert with one FP32 add of
+    // 1.5 * 2^23 (the sum's last bit is the integer, RN does the rounding) and
+    // an integer subtract: no conversion-pipe instructions.  Clamping first is
+    // equivalent to clamping the rounded value (127 is an integer).
     auto clamp_code = [](float qt) -> uint32_t {
-        return (uint32_t)((int)fminf(fmaxf(rintf(qt), -127.f), 127.f) & 0xff);
+        const float cq = fminf(fmaxf(qt, -127.f), 127.f) + 12582912.0f;
+        return (uint32_t)(__float_as_int(cq) - 0x4B400000) & 0xffu;
     };
     auto code_fast = [&](float x, float sc, float ysc) -> uint32_t { return clamp_code(div_rn_unchecked(x, sc, ysc)); };
     auto code_ieee = [&](float x, float sc) -> uint32_t { return sc != 0.f ? clamp_code(__fdiv_rn(x, sc)) : 0u; };

@@ -142,6 +142,7 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label=""):
     ("kda", 1, 3, 3, 64, 128, 5, 2),        # dk != dv, odd window
     ("gdn", 2, 2, 2, 128, 64, 6, 3),
     ("gdn", 1, 2, 2, 128, 128, 64, 4),      # 85 KB staged: above the 48 KB default
+    ("kda", 1, 2, 2, 128, 128, 200, 4),     # 26 entry chunks per flush, a ragged last one
 ])
 def test_windowed_teacher_forced(fused, gate, B, H, Hk, dk, dv, W, r):
     U.require_gpu()

@@ -65,6 +65,7 @@ typedef struct {
     int smoothing; /* 1: per-row RMS smoothing; 0: m_i = 1 */
     int P;         /* BF16 key rows per head (DAMP); 0 = none */
     int quantize;  /* 0: identity quantizer (FP32-state mode); 1: INT8 */
+    int bf16_buffer; /* 1: each token's update is kept in BF16 (see lqo_step_bf16) */
 } lqo_cfg;
 
 /* A quantized view of one head.  codes are [dk][dv] with the BF16 rows' codes
@@ -130,6 +131,49 @@ float lqo_bf16_to_float(uint16_t h)
     float f;
     memcpy(&f, &u, 4);
     return f;
+}
+
+/* One token with the window's buffered updates kept in BF16 (the
+ * traffic-lean buffer): as lqo_step, except that the rank-one update enters
+ * the state rounded, the way the windowed kernels store it -- the key side
+ * divided by the window's decay so far, ktil = k / Gamma_t, and the value side
+ * u, each rounded to BF16 (round to nearest even) from FP32:
+ *     S <- S' + (Gamma_t * bf16(ktil)) bf16(u)^T,   o = S^T q.
+ * Gamma_t = a_t * Gamma_{t-1} (per key row for KDA, one value for GDN) is
+ * carried in FP32 in gam[] (1 at the window start), and ktil and u are formed
+ * in FP32 before rounding: BF16 rounding decides the stored bits, so it is
+ * taken in the kernels' precision. */
+void lqo_step_bf16(const lqo_cfg *cfg, double *S, float *gam, const float *q, const float *k,
+                   const float *v, float beta, const float *alpha, double *o)
+{
+    const int dk = cfg->dk, dv = cfg->dv, ga = cfg->gate ? dk : 1;
+    double *u = (double *)malloc(sizeof(double) * dv);
+    double *kg = (double *)malloc(sizeof(double) * dk);
+    for (int j = 0; j < ga; ++j) gam[j] = alpha[j] * gam[j];
+    for (int i = 0; i < dk; ++i) {
+        const double d = cfg->gate ? (double)alpha[i] : (double)alpha[0];
+        for (int c = 0; c < dv; ++c) S[i * dv + c] *= d;
+    }
+    for (int c = 0; c < dv; ++c) {
+        double y = 0.0;
+        for (int i = 0; i < dk; ++i) y += (double)k[i] * S[i * dv + c];
+        const float uf = (float)((double)beta * ((double)v[c] - y));
+        u[c] = (double)lqo_bf16_to_float(lqo_bf16_rne(uf));
+    }
+    for (int i = 0; i < dk; ++i) {
+        const float g = cfg->gate ? gam[i] : gam[0];
+        const float kt = k[i] / g;
+        kg[i] = (double)g * (double)lqo_bf16_to_float(lqo_bf16_rne(kt));
+    }
+    for (int i = 0; i < dk; ++i)
+        for (int c = 0; c < dv; ++c) S[i * dv + c] += kg[i] * u[c];
+    for (int c = 0; c < dv; ++c) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i) acc += S[i * dv + c] * (double)q[i];
+        o[c] = acc;
+    }
+    free(u);
+    free(kg);
 }
 
 static int is_hp_row(const int *hp_rows, int P, int i)
@@ -321,10 +365,19 @@ void lqo_run(const lqo_cfg *cfg, int nh, const int *hp_rows, int from_view,
             for (int e = 0; e < dk * dv; ++e) S[e] = (double)S0[(size_t)h * dk * dv + e];
         }
         int n = 0;
+        float gam[512];
+        for (int j = 0; j < ga; ++j) gam[j] = 1.0f;
         for (int t = 0; t < T; ++t) {
             const size_t th = (size_t)t * nh + h;
-            lqo_step(cfg, S, q + th * dk, k + th * dk, v + th * dv, beta[th],
-                     alpha + th * ga, o + th * dv);
+            if (cfg->quantize && cfg->bf16_buffer) {
+                if (n == 0)
+                    for (int j = 0; j < ga; ++j) gam[j] = 1.0f;
+                lqo_step_bf16(cfg, S, gam, q + th * dk, k + th * dk, v + th * dv, beta[th],
+                              alpha + th * ga, o + th * dv);
+            } else {
+                lqo_step(cfg, S, q + th * dk, k + th * dk, v + th * dv, beta[th],
+                         alpha + th * ga, o + th * dv);
+            }
             n += 1;
             if (cfg->quantize && n == cfg->W && (t < T - 1 || flush_last)) {
                 if (S_pre) memcpy(S_pre + (size_t)h * dk * dv, S, sizeof(double) * dk * dv);

@@ -82,6 +82,12 @@ typedef struct {
     int32_t n_hp_rows;      /* P: BF16 key rows per head (DAMP layout), 0 = all INT8 */
     int32_t smoothing;      /* 1: per-key-row RMS smoothing; 0: none (m = 1) */
     int32_t fused_flush;    /* 1: the call that buffers the W-th token also flushes */
+    int32_t buffer_bf16;    /* 1 (INT8_WINDOW only): keep each buffered token's update in BF16 --
+                               bf16(k/Gamma) and bf16(u), formed in FP32, the state carrying the
+                               rounded term from that token on (its own output included);
+                               compensators stay FP32.  Halves the window buffer's bytes.
+                               Not built together with BF16 rows (n_hp_rows > 0:
+                               LQ_ERR_UNSUPPORTED).  0: FP32 buffer (the method as stated). */
 } lq_config;
 
 /* A quantized state in plain arrays (all device pointers, caller-owned):

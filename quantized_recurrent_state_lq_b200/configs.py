@@ -50,6 +50,7 @@ class Workload:
     seed: int = 0
     calib_prefills: int = 0
     calib_tokens: int = 0
+    buffer_bf16: int = 0         # 1: the traffic-lean BF16 window buffer (an option, not a config)
 
     @property
     def heads(self) -> int:

@@ -35,7 +35,8 @@ bool is_int8(const lq_config *c) { return c->mode == LQ_MODE_INT8_STEP || c->mod
 
 Layout layout_of(const lq_config *c) {
     const int W = c->mode == LQ_MODE_INT8_STEP ? 1 : c->W;
-    return lq::make_layout(c->dk, c->dv, c->n_hp_rows, c->r, W, c->gate == LQ_GATE_CHANNEL);
+    return lq::make_layout(c->dk, c->dv, c->n_hp_rows, c->r, W, c->gate == LQ_GATE_CHANNEL,
+                           c->mode == LQ_MODE_INT8_WINDOW && c->buffer_bf16 == 1);
 }
 
 int check_codec_fields(const lq_config *c) {
@@ -57,6 +58,9 @@ int check_config(const lq_config *c) {
     if (c->mode != LQ_MODE_FP32 && c->mode != LQ_MODE_INT8_STEP && c->mode != LQ_MODE_INT8_WINDOW)
         return LQ_ERR_INVALID_ARG;
     if (c->fused_flush != 0 && c->fused_flush != 1) return LQ_ERR_INVALID_ARG;
+    if (c->buffer_bf16 != 0 && c->buffer_bf16 != 1) return LQ_ERR_INVALID_ARG;
+    if (c->buffer_bf16 == 1 && c->mode != LQ_MODE_INT8_WINDOW) return LQ_ERR_INVALID_ARG;
+    if (c->buffer_bf16 == 1 && c->n_hp_rows > 0) return LQ_ERR_UNSUPPORTED;   // not built with BF16 rows
     int rc = check_codec_fields(c);
     if (rc) return rc;
     if (is_int8(c)) {

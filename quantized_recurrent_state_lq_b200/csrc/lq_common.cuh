@@ -21,31 +21,33 @@ constexpr int kStatusTimeout = 2;
 //   m       f32   [dk]              smoothing scale per key row (1 on BF16 rows)
 //   s       f32   [dv]              quantization scale per value column
 //   hp      u16   [P][dv]           BF16 rows (order of the head's row list)
-//   codes   int8  [dk-P][dv]        INT8 rows in increasing key-row order
-//   ent     f32   [r+W][dk+dv]      entry e = (key side [dk], value side [dv]);
-//                                   e < r: compensator (c_e, w_e);
-//                                   r <= e < r+n: buffered token (k/Gamma, u)
+//   codes   int8  [dk-P][dv]        INT8 codes (layout: code_off_t below)
+//   comps   f32   [r][dk+dv]        compensator j = (c_j [dk], w_j [dv])
+//   tokens  f32 or bf16 [W][dk+dv]  buffered token tau = (k_tau/Gamma_tau, u_tau)
 //   gam     f32   [dk] (KDA) / [4] (GDN)   cumulative decay since window start
-// A decode step reads [hp, codes, r+n entries] -- one contiguous byte range --
-// as a stream of bulk copies; m, s are read with the step's small vectors.
+// Entries e < r are the compensators, e = r + tau the buffered tokens; with
+// FP32 tokens both form one array [r+W][dk+dv].  A decode step reads
+// [m .. codes] with one bulk copy and the r + n entries as coalesced streams.
 // ---------------------------------------------------------------------------
 struct Layout {
     int dk, dv, P, r, W, kda;
-    int off_m, off_s, off_hp, off_codes, off_ent, off_gam;
+    int tok_bf16;   // buffered tokens stored in BF16
+    int off_m, off_s, off_hp, off_codes, off_ent, off_tok, off_gam;
     int rec_bytes;
 };
 
 __host__ __device__ inline int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-__host__ inline Layout make_layout(int dk, int dv, int P, int r, int W, int kda) {
+__host__ inline Layout make_layout(int dk, int dv, int P, int r, int W, int kda, int tok_bf16 = 0) {
     Layout L;
-    L.dk = dk; L.dv = dv; L.P = P; L.r = r; L.W = W; L.kda = kda;
+    L.dk = dk; L.dv = dv; L.P = P; L.r = r; L.W = W; L.kda = kda; L.tok_bf16 = tok_bf16;
     L.off_m = 0;
     L.off_s = dk * 4;
     L.off_hp = (dk + dv) * 4;
     L.off_codes = L.off_hp + P * dv * 2;
     L.off_ent = align_up(L.off_codes + (dk - P) * dv, 16);
-    int o = L.off_ent + (r + W) * (dk + dv) * 4;
+    L.off_tok = L.off_ent + r * (dk + dv) * 4;
+    int o = L.off_tok + W * (dk + dv) * (tok_bf16 ? 2 : 4);
     L.off_gam = align_up(o, 16);
     o = L.off_gam + (kda ? dk : 4) * 4;
     L.rec_bytes = align_up(o, 128);
@@ -299,6 +301,15 @@ __device__ __forceinline__ uint16_t bf16_rne(float x) {
 }
 
 __device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+__device__ __forceinline__ float4 bf16x4_to_f4(uint2 w) {
+    return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u), __uint_as_float(w.y << 16),
+                       __uint_as_float(w.y & 0xffff0000u));
+}
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+// x rounded to BF16 (nearest even), as an FP32 value
+__device__ __forceinline__ float bf16_round(float x) { return bf16_to_f(bf16_rne(x)); }
 
 // Signed bytes of a 32-bit word -> floats (exact).  Each byte, offset to
 // unsigned, is placed in the low mantissa byte of 2^23 (bit pattern

@@ -118,7 +118,7 @@ __device__ __forceinline__ void warp_reduce_dots(float (&v)[2 * NE]) {
     }
 }
 
-template <int DK, int DV, bool KDA, bool DAMP>
+template <int DK, int DV, bool KDA, bool DAMP, bool TB>
 __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     BufSmem<DK, DV> &S = *reinterpret_cast<BufSmem<DK, DV> *>(smem);
@@ -134,9 +134,11 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
     unsigned char *rec = a.rec + (size_t)head * L.rec_bytes;
     const float *ent_g = reinterpret_cast<const float *>(rec + L.off_ent);
     float *rec_ent = reinterpret_cast<float *>(rec + L.off_ent);
+    uint16_t *rec_tok16 = reinterpret_cast<uint16_t *>(rec + L.off_tok);   // BF16 tokens
     float *rec_gam = reinterpret_cast<float *>(rec + L.off_gam);
+    constexpr bool tb = TB;   // buffered tokens in BF16
     constexpr int XPL = DK / 32;                 // key elements per lane in a dot product
-    constexpr int EF = DK + DV;                  // floats per entry
+    constexpr int EF = DK + DV;                  // elements per entry
 
     if (t == 0) {
         mbar_init(&S.mbar, 1);
@@ -151,16 +153,34 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
     // Entry pairs of this warp: entries 2 warp + 16 j + {0, 1}.
     float4 kb[2], ub[2];
     float2 kb2[2];
+    // (FP32 entries -- the compensators, and FP32 tokens -- form one array;
+    // BF16 tokens are widened on load)
+    auto load_fp32 = [&](int p, int e) {
+        const float *kt = ent_g + (size_t)e * EF;
+        if (XPL == 4) kb[p] = __ldcs(reinterpret_cast<const float4 *>(kt) + lane);
+        else kb2[p] = __ldcs(reinterpret_cast<const float2 *>(kt) + lane);
+        if (lane < DV / 4) ub[p] = __ldcs(reinterpret_cast<const float4 *>(kt + DK) + lane);
+    };
+    auto load_bf16 = [&](int p, int e) {
+        const uint16_t *kt = rec_tok16 + (size_t)(e - L.r) * EF;
+        if (XPL == 4) kb[p] = bf16x4_to_f4(__ldcs(reinterpret_cast<const uint2 *>(kt) + lane));
+        else kb2[p] = bf16x2_to_f2(__ldcs(reinterpret_cast<const unsigned int *>(kt) + lane));
+        if (lane < DV / 4) ub[p] = bf16x4_to_f4(__ldcs(reinterpret_cast<const uint2 *>(kt + DK) + lane));
+    };
+    // (with BF16 tokens the type is decided per pair: a pair of tokens loads
+    // without branches between its loads)
     auto load_pair = [&](int e0) {
+        if (!tb || e0 + 1 < L.r) {
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const int e = e0 + p;
-            if (e < E) {
-                const float *kt = ent_g + (size_t)e * EF;
-                if (XPL == 4) kb[p] = __ldcs(reinterpret_cast<const float4 *>(kt) + lane);
-                else kb2[p] = __ldcs(reinterpret_cast<const float2 *>(kt) + lane);
-                if (lane < DV / 4) ub[p] = __ldcs(reinterpret_cast<const float4 *>(kt + DK) + lane);
-            }
+            for (int p = 0; p < 2; ++p)
+                if (e0 + p < E) load_fp32(p, e0 + p);
+        } else if (e0 >= L.r) {
+#pragma unroll
+            for (int p = 0; p < 2; ++p)
+                if (e0 + p < E) load_bf16(p, e0 + p);
+        } else {
+            if (e0 < E) load_fp32(0, e0);
+            if (e0 + 1 < E) load_bf16(1, e0 + 1);
         }
     };
     load_pair(2 * warp);
@@ -175,7 +195,8 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
         gt = (KDA ? a.alpha[hv * DK + t] : a.alpha[hv]) * gp;
         const float2 x = make_float2(gt * kk, gt * qq);
         S.x2[t] = x;
-        kqp = kk * qq;
+        // the key of the update the state carries: k, or Gamma bf16(k / Gamma)
+        kqp = (tb ? gt * bf16_round(kk / gt) : kk) * qq;
         if (!DAMP) {
             const float mi = reinterpret_cast<const float *>(rec + L.off_m)[t];
             ak_t = mi * x.x;
@@ -391,14 +412,21 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
             yk += p.x;
             yq += p.y;
         }
-        const float ut = beta * (S.v[t] - yk);
+        float ut = beta * (S.v[t] - yk);
+        if (tb) {
+            const uint16_t uh = bf16_rne(ut);
+            rec_tok16[(size_t)a.n * EF + DK + t] = uh;
+            ut = bf16_to_f(uh);
+        } else {
+            rec_ent[(size_t)E * EF + DK + t] = ut;
+        }
         const float o = fmaf(ut, kq, yq);
         a.o[hv * DV + t] = o;
-        rec_ent[(size_t)E * EF + DK + t] = ut;
         if (!isfinite(o) || !isfinite(ut)) atomicOr(a.status, kStatusNonFinite);
     }
     if (t < DK) {
-        rec_ent[(size_t)E * EF + t] = kk / gt;
+        if (tb) rec_tok16[(size_t)a.n * EF + t] = bf16_rne(kk / gt);
+        else rec_ent[(size_t)E * EF + t] = kk / gt;
         if (KDA) rec_gam[t] = gt;
         else if (t == 0) rec_gam[0] = gt;
     }
@@ -423,14 +451,13 @@ constexpr int kFlushChunk = 8;   // entries per staged chunk: one TF32 MMA K-blo
 
 template <int DK, int DV>
 struct FlushSmem {
-    float k[DK], q[DK], gam[DK];
+    float k[DK], ke[DK], q[DK], gam[DK];
     float u[DV];
     float kqw[kFlushWarps];
     int map[DK];
     int wscr[kFlushWarps];
     CodecSmem<DK, DV, kFlushThreads> cs;
     uint64_t mbar_pre;
-    uint64_t mbar_ent[2];
     uint64_t mbar_mma[2];
     uint32_t tmem_base;
 };
@@ -446,15 +473,11 @@ __host__ __device__ constexpr size_t flush_fixed_bytes() {
 // buffers, each the TF32 big / small parts of one chunk's ktil^T [dk][8] and
 // u^T [dv][8] in K-major core-matrix layout; the entries come from global
 // memory into registers one chunk ahead.  They come before the prefix so that
-// everything a descriptor can address stays inside the allocation.
-// d_k = 64: the work area stages the entries, two chunk buffers
-// [kFlushChunk][dk+dv] filled by bulk copies.
-// Either way the work area doubles as the accumulator's transposition scratch.
+// everything a descriptor can address stays inside the allocation; afterwards
+// the work area is the accumulator's transposition scratch.  d_k = 64 needs
+// no work area.
 __host__ __device__ inline size_t flush_ops_bytes(int dk, int dv) { return (size_t)2 * (dk + dv) * 32; }
-__host__ __device__ inline size_t flush_chunk_bytes(int dk, int dv) { return (size_t)kFlushChunk * (dk + dv) * 4; }
-__host__ __device__ inline size_t flush_work_bytes(int dk, int dv) {
-    return dk == 128 ? 2 * flush_ops_bytes(dk, dv) : 2 * flush_chunk_bytes(dk, dv);
-}
+__host__ __device__ inline size_t flush_work_bytes(int dk, int dv) { return dk == 128 ? 2 * flush_ops_bytes(dk, dv) : 0; }
 
 size_t flush_smem_bytes(int dk, int dv, const Layout &L) {
     size_t fixed = 0;
@@ -467,7 +490,7 @@ size_t flush_smem_bytes(int dk, int dv, const Layout &L) {
 
 enum { kFlushStep = 0, kFlushOnly = 1, kExport = 2 };
 
-template <int DK, int DV, bool KDA, bool DAMP, int MODE>
+template <int DK, int DV, bool KDA, bool DAMP, int MODE, bool TB>
 __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const DecodeArgs a) {
     constexpr int NT = kFlushThreads;
     constexpr int EF = DK + DV;   // floats per entry
@@ -476,7 +499,6 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
     FlushSmem<DK, DV> &F = *reinterpret_cast<FlushSmem<DK, DV> *>(smem);
     const Layout &L = a.L;
     unsigned char *work = smem + flush_fixed_bytes<DK, DV>();
-    float *ebuf = reinterpret_cast<float *>(work);   // d_k = 64: [2][kFlushChunk][EF]
     unsigned char *stage = work + flush_work_bytes(DK, DV);
     const int head = blockIdx.x;
     const int b = head / a.H, h = head - b * a.H, g = (h * a.Hk) / a.H;
@@ -487,39 +509,26 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
     const int nch = (E + kFlushChunk - 1) / kFlushChunk;
     unsigned char *rec = a.rec + (size_t)head * L.rec_bytes;
     float *rec_ent = reinterpret_cast<float *>(rec + L.off_ent);
+    const uint16_t *rec_tok16 = reinterpret_cast<const uint16_t *>(rec + L.off_tok);
     float *rec_gam = reinterpret_cast<float *>(rec + L.off_gam);
     const size_t hv = (size_t)b * a.H + h;
-
-    // chunk c (entries [c*kFlushChunk, ...)) goes to buffer c & 1; its
-    // barrier completes once per use, use c >> 1, parity (c >> 1) & 1
-    auto issue_chunk = [&](int c) {
-        const int n = min(kFlushChunk, E - c * kFlushChunk);
-        const uint32_t bytes = (uint32_t)(n * EF * 4);
-        mbar_arrive_expect_tx(&F.mbar_ent[c & 1], bytes);
-        bulk_g2s(ebuf + (size_t)(c & 1) * kFlushChunk * EF, rec_ent + (size_t)c * kFlushChunk * EF, bytes,
-                 &F.mbar_ent[c & 1]);
-    };
-    // after a failed wait: let the copies still in flight land (bounded)
-    // before the CTA's shared memory is released
-    auto drain = [&](int from, int issued) {
-        if (t == 0)
-            for (int c = from; c < issued; ++c) mbar_wait_bounded(&F.mbar_ent[c & 1], (c >> 1) & 1, nullptr);
+    constexpr bool tb = TB;   // buffered tokens in BF16
+    // element x of entry e (e < r: a compensator, else buffered token e - r)
+    auto entry_at = [&](int e, int x) -> float {
+        if (!tb || e < L.r) return __ldcs(rec_ent + (size_t)e * EF + x);
+        return bf16_to_f(__ldcs(rec_tok16 + (size_t)(e - L.r) * EF + x));
     };
 
     if (t == 0) {
         mbar_init(&F.mbar_pre, 1);
-        mbar_init(&F.mbar_ent[0], 1);
-        mbar_init(&F.mbar_ent[1], 1);
         mbar_init(&F.mbar_mma[0], 1);
         mbar_init(&F.mbar_mma[1], 1);
         fence_mbar_init();
     }
     __syncthreads();
-    int issued = DK == 128 ? 0 : min(nch, 2);   // entry chunks bulk-copied (d_k = 64)
     if (t == 0) {
         mbar_arrive_expect_tx(&F.mbar_pre, (uint32_t)L.off_ent);
         bulk_g2s(stage, rec, (uint32_t)L.off_ent, &F.mbar_pre);
-        for (int c = 0; c < issued; ++c) issue_chunk(c);
     }
     float kqp = 0.f;
     if (t < DK) {
@@ -529,9 +538,12 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
             const size_t qk = ((size_t)b * a.Hk + g) * DK;
             const float kk = a.k[qk + t], qq = a.q[qk + t];
             gt = (KDA ? a.alpha[hv * DK + t] : a.alpha[hv]) * gp;
+            // the key of the update the state takes: k, or Gamma bf16(k / Gamma)
+            const float ke = tb ? gt * bf16_round(kk / gt) : kk;
             F.k[t] = kk;
+            F.ke[t] = ke;
             F.q[t] = qq;
-            kqp = kk * qq;
+            kqp = ke * qq;
         }
         F.gam[t] = gt;
     }
@@ -539,10 +551,7 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
     if (lane == 0) F.kqw[warp] = kqp;
     if (DAMP) build_row_map<DK, NT>(a.hp_rows + (size_t)h * P, P, F.map, F.wscr);
     const bool okw = mbar_wait_bounded(&F.mbar_pre, 0, a.status);
-    if (__syncthreads_or(!okw)) {
-        drain(0, issued);
-        return;
-    }
+    if (__syncthreads_or(!okw)) return;
 
     // R = sum_e ktil_e u_e^T over the r + n entries, then += Deq, then * Gamma.
     float R[T::RPT][16];
@@ -587,60 +596,70 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
                 *reinterpret_cast<uint4 *>(ps) = make_uint4(hs[0], hs[1], hs[2], hs[3]);
                 *reinterpret_cast<uint4 *>(ps + rows * 4) = make_uint4(hs[4], hs[5], hs[6], hs[7]);
             };
-            // chunk entries of this thread's key row / value column, a ring of
-            // PF chunks in registers (slot = chunk % PF, a compile-time index
-            // inside the unrolled loop): loads run PF chunks ahead of use
-            constexpr int PF = 1;
-            float xa[PF][8], xb[PF][8];
-            auto load_chunk = [&](int c, float (&ya)[8], float (&yb)[8]) {
+            // this thread's key row (A) / value column (B) of a chunk's entries,
+            // loaded one chunk ahead of its conversion
+            float xa[8], xb[8];
+            // (the FP32-or-BF16 choice is made per chunk, so that the common
+            // all-token chunk issues its 16 loads without branches between them)
+            auto load_chunk = [&](int c) {
                 const int n = min(kFlushChunk, E - c * kFlushChunk);
-                const float *src = rec_ent + (size_t)c * kFlushChunk * EF;
+                if (tb && c * kFlushChunk >= L.r) {
+                    const uint16_t *src = rec_tok16 + (size_t)(c * kFlushChunk - L.r) * EF;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    ya[e] = e < n ? __ldcs(src + e * EF + t) : 0.f;
-                    yb[e] = (e < n && t < DV) ? __ldcs(src + e * EF + DK + t) : 0.f;
-                }
-            };
+                    for (int e = 0; e < 8; ++e) {
+                        xa[e] = e < n ? bf16_to_f(__ldcs(src + e * EF + t)) : 0.f;
+                        xb[e] = (e < n && t < DV) ? bf16_to_f(__ldcs(src + e * EF + DK + t)) : 0.f;
+                    }
+                } else if (!tb) {
+                    const float *src = rec_ent + (size_t)c * kFlushChunk * EF;
 #pragma unroll
-            for (int s2 = 0; s2 < PF; ++s2)
-                if (s2 < nch) load_chunk(s2, xa[s2], xb[s2]);
-            int c = 0;   // chunks committed
-            bool ok = true;
-            for (int c0 = 0; c0 < nch && ok; c0 += PF) {
+                    for (int e = 0; e < 8; ++e) {
+                        xa[e] = e < n ? __ldcs(src + e * EF + t) : 0.f;
+                        xb[e] = (e < n && t < DV) ? __ldcs(src + e * EF + DK + t) : 0.f;
+                    }
+                } else {
 #pragma unroll
-                for (int s2 = 0; s2 < PF; ++s2) {
-                    const int cc = c0 + s2;
-                    if (cc < nch && ok) {
-                        uint32_t *opA_big = reinterpret_cast<uint32_t *>(work) + (cc & 1) * OPW;
-                        uint32_t *opA_small = opA_big + DK * 8;
-                        uint32_t *opB_big = opA_small + DK * 8;
-                        uint32_t *opB_small = opB_big + DV * 8;
-                        const bool okc =
-                            cc < 2 || mbar_wait_bounded(&F.mbar_mma[cc & 1], ((cc >> 1) - 1) & 1, a.status);
-                        if (__syncthreads_or(!okc)) {
-                            ok = false;
-                        } else {
-                            put_row(opA_big, opA_small, DK, t, xa[s2]);
-                            if (t < DV) put_row(opB_big, opB_small, DV, t, xb[s2]);
-                            if (cc + PF < nch) load_chunk(cc + PF, xa[s2], xb[s2]);
-                            fence_async_smem();
-                            tc_fence_before();
-                            __syncthreads();
-                            if (t == 0) {
-                                tc_fence_after();
-                                const uint64_t ab = umma_smem_desc(opA_big, DK * 16, 128);
-                                const uint64_t as = umma_smem_desc(opA_small, DK * 16, 128);
-                                const uint64_t bb = umma_smem_desc(opB_big, DV * 16, 128);
-                                const uint64_t bs = umma_smem_desc(opB_small, DV * 16, 128);
-                                umma_tf32(tmem, ab, bb, IDESC, cc > 0 ? 1u : 0u);
-                                umma_tf32(tmem, ab, bs, IDESC, 1u);
-                                umma_tf32(tmem, as, bb, IDESC, 1u);
-                                umma_commit(&F.mbar_mma[cc & 1]);
-                            }
-                            c = cc + 1;
-                        }
+                    for (int e = 0; e < 8; ++e) {
+                        xa[e] = e < n ? entry_at(c * kFlushChunk + e, t) : 0.f;
+                        xb[e] = (e < n && t < DV) ? entry_at(c * kFlushChunk + e, DK + t) : 0.f;
                     }
                 }
+            };
+            load_chunk(0);
+            int c = 0;   // chunks committed
+            bool ok = true;
+            for (int cc = 0; cc < nch; ++cc) {
+                uint32_t *opA_big = reinterpret_cast<uint32_t *>(work) + (cc & 1) * OPW;
+                uint32_t *opA_small = opA_big + DK * 8;
+                uint32_t *opB_big = opA_small + DK * 8;
+                uint32_t *opB_small = opB_big + DV * 8;
+                const bool okc = cc < 2 || mbar_wait_bounded(&F.mbar_mma[cc & 1], ((cc >> 1) - 1) & 1, a.status);
+                if (__syncthreads_or(!okc)) {
+                    ok = false;
+                    break;
+                }
+                put_row(opA_big, opA_small, DK, t, xa);
+                if (t < DV) put_row(opB_big, opB_small, DV, t, xb);
+                if (cc + 1 < nch) load_chunk(cc + 1);
+                fence_async_smem();
+                tc_fence_before();
+                __syncthreads();
+                if (t == 0) {
+                    tc_fence_after();
+                    const uint64_t ab = umma_smem_desc(opA_big, DK * 16, 128);
+                    const uint64_t bb = umma_smem_desc(opB_big, DV * 16, 128);
+                    umma_tf32(tmem, ab, bb, IDESC, cc > 0 ? 1u : 0u);
+                    // BF16 tokens are exact in TF32 (the small parts are zero):
+                    // a chunk of them needs the big x big pass only
+                    if (!tb || cc * kFlushChunk < L.r) {
+                        const uint64_t as = umma_smem_desc(opA_small, DK * 16, 128);
+                        const uint64_t bs = umma_smem_desc(opB_small, DV * 16, 128);
+                        umma_tf32(tmem, ab, bs, IDESC, 1u);
+                        umma_tf32(tmem, as, bb, IDESC, 1u);
+                    }
+                    umma_commit(&F.mbar_mma[cc & 1]);
+                }
+                c = cc + 1;
             }
             // chunks 0 .. c-1 were committed; the last commit completes after
             // every earlier MMA
@@ -685,20 +704,25 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
             if (!okm) return;
         }
     } else {
+        // d_k = 64: the entries straight from memory (every thread of the CTA
+        // reads the same rows: cached), packed FP32 FMAs on the tile
         zero_tile();
-        for (int c = 0; c < nch; ++c) {
-            const bool ok = mbar_wait_bounded(&F.mbar_ent[c & 1], (c >> 1) & 1, a.status);
-            // also the barrier after which buffer (c+1) & 1 -- chunk c-1 -- is free
-            if (__syncthreads_or(!ok)) {
-                drain(c + 1, issued);
-                return;
-            }
-            if (c >= 1 && c + 1 < nch) {
-                if (t == 0) issue_chunk(c + 1);
-                ++issued;
-            }
-            tile_add_entries<DK, DV, NT>(R, ebuf + (size_t)(c & 1) * kFlushChunk * EF,
-                                         min(kFlushChunk, E - c * kFlushChunk));
+        for (int e = 0; e < E; ++e) {
+            float kv[T::RPT], uv[16];
+#pragma unroll
+            for (int r = 0; r < T::RPT; ++r) kv[r] = entry_at(e, row0 + r);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) uv[4 * q + u] = entry_at(e, DK + T::col(cg, q) + u);
+#pragma unroll
+            for (int r = 0; r < T::RPT; ++r)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float2 o = ffma2(f2(kv[r], kv[r]), f2(uv[2 * q], uv[2 * q + 1]), f2(R[r][2 * q], R[r][2 * q + 1]));
+                    R[r][2 * q] = o.x;
+                    R[r][2 * q + 1] = o.y;
+                }
         }
     }
     tile_dequant<DK, DV, NT, true>(R, reinterpret_cast<const float *>(stage + L.off_m),
@@ -749,7 +773,8 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
                 yq += rq[w][t];
                 kq += F.kqw[w];
             }
-            const float ut = a.beta[hv] * (a.v[hv * DV + t] - yk);
+            float ut = a.beta[hv] * (a.v[hv * DV + t] - yk);
+            if (tb) ut = bf16_round(ut);   // the update the state takes: u or bf16(u)
             const float o = fmaf(ut, kq, yq);
             a.o[hv * DV + t] = o;
             F.u[t] = ut;
@@ -760,7 +785,7 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
         load_cols16<DK, DV>(F.u, uv);
 #pragma unroll
         for (int r = 0; r < T::RPT; ++r) {
-            const float kk = F.k[row0 + r];
+            const float kk = F.ke[row0 + r];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const float2 o = ffma2(f2(kk, kk), f2(uv[2 * c], uv[2 * c + 1]), f2(R[r][2 * c], R[r][2 * c + 1]));
@@ -882,21 +907,34 @@ static cudaError_t set_smem(K kern, size_t bytes, size_t &done) {
     return e;
 }
 
-template <int DK, int DV, bool KDA, bool DAMP>
+// Shared-memory carveout of the buffering kernel: 85% of the SM's 228 KB,
+// rounded up by the driver to the 196 KB configuration, leaves ~60 KB of L1
+// for the streamed entries and step inputs and room for 7 CTAs of ~27 KB
+// (measured: the 228 KB configuration that 8 CTAs would need, with 28 KB of
+// L1, is ~9% slower).
+constexpr int kBufCarveoutPct = 85;
+
+template <int DK, int DV, bool KDA, bool DAMP, bool TB>
 static cudaError_t launch_buffer_t(const DecodeArgs &a, int heads, cudaStream_t s) {
     const size_t sm = buffer_smem_bytes(DK, DV, a.L);
-    auto kern = decode_buffer_kernel<DK, DV, KDA, DAMP>;
+    auto kern = decode_buffer_kernel<DK, DV, KDA, DAMP, TB>;
     static size_t done = 0;
+    static bool carved = false;
     cudaError_t e = set_smem(kern, sm, done);
     if (e != cudaSuccess) return e;
+    if (!carved) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, kBufCarveoutPct);
+        if (e != cudaSuccess) return e;
+        carved = true;
+    }
     kern<<<heads, kBufThreads, sm, s>>>(a);
     return cudaGetLastError();
 }
 
-template <int DK, int DV, bool KDA, bool DAMP, int MODE>
+template <int DK, int DV, bool KDA, bool DAMP, int MODE, bool TB>
 static cudaError_t launch_flush_t(const DecodeArgs &a, int heads, cudaStream_t s) {
     const size_t sm = flush_smem_bytes(DK, DV, a.L);
-    auto kern = decode_flush_kernel<DK, DV, KDA, DAMP, MODE>;
+    auto kern = decode_flush_kernel<DK, DV, KDA, DAMP, MODE, TB>;
     static size_t done = 0;
     cudaError_t e = set_smem(kern, sm, done);
     if (e != cudaSuccess) return e;
@@ -910,18 +948,32 @@ static cudaError_t launch_flush_t(const DecodeArgs &a, int heads, cudaStream_t s
      : ((dk) == 64 && (dv) == 128) ? FN<64, 128>       \
                                    : FN<128, 64>)
 
+// BF16 tokens are built without BF16 rows (the configuration check rejects
+// the combination).
 template <int DK, int DV>
 static cudaError_t buffer_dispatch(const DecodeArgs &a, int heads, bool kda, bool damp, cudaStream_t s) {
-    if (kda) return damp ? launch_buffer_t<DK, DV, true, true>(a, heads, s) : launch_buffer_t<DK, DV, true, false>(a, heads, s);
-    return damp ? launch_buffer_t<DK, DV, false, true>(a, heads, s) : launch_buffer_t<DK, DV, false, false>(a, heads, s);
+    const bool tb = a.L.tok_bf16 != 0;
+    if (kda) {
+        if (damp) return launch_buffer_t<DK, DV, true, true, false>(a, heads, s);
+        return tb ? launch_buffer_t<DK, DV, true, false, true>(a, heads, s)
+                  : launch_buffer_t<DK, DV, true, false, false>(a, heads, s);
+    }
+    if (damp) return launch_buffer_t<DK, DV, false, true, false>(a, heads, s);
+    return tb ? launch_buffer_t<DK, DV, false, false, true>(a, heads, s)
+              : launch_buffer_t<DK, DV, false, false, false>(a, heads, s);
 }
 
 template <int DK, int DV, int MODE>
 static cudaError_t flush_mode_dispatch(const DecodeArgs &a, int heads, bool kda, bool damp, cudaStream_t s) {
-    if (kda) return damp ? launch_flush_t<DK, DV, true, true, MODE>(a, heads, s)
-                         : launch_flush_t<DK, DV, true, false, MODE>(a, heads, s);
-    return damp ? launch_flush_t<DK, DV, false, true, MODE>(a, heads, s)
-                : launch_flush_t<DK, DV, false, false, MODE>(a, heads, s);
+    const bool tb = a.L.tok_bf16 != 0;
+    if (kda) {
+        if (damp) return launch_flush_t<DK, DV, true, true, MODE, false>(a, heads, s);
+        return tb ? launch_flush_t<DK, DV, true, false, MODE, true>(a, heads, s)
+                  : launch_flush_t<DK, DV, true, false, MODE, false>(a, heads, s);
+    }
+    if (damp) return launch_flush_t<DK, DV, false, true, MODE, false>(a, heads, s);
+    return tb ? launch_flush_t<DK, DV, false, false, MODE, true>(a, heads, s)
+              : launch_flush_t<DK, DV, false, false, MODE, false>(a, heads, s);
 }
 
 template <int DK, int DV>

@@ -6,7 +6,8 @@ Per head and token of a window (n tokens already buffered, 0 <= n < W):
           beta, the gate (1 or dk floats)
   state   INT8 codes (dk-P)*dv, BF16 rows 2*P*dv, m and s (dk+dv)*4,
           r compensators r*(dk+dv)*4, the n buffered entries n*(dk+dv)*4
-  append  one entry (dk+dv)*4 and Gamma written (read too when n > 0)
+          (n*(dk+dv)*2 with the BF16 buffer)
+  append  one entry (dk+dv)*4 (or *2) and Gamma written (read too when n > 0)
 At the window end the new state is written once: codes, BF16 rows, m, s and
 the compensators.
 """
@@ -31,9 +32,14 @@ def gamma_bytes(wl: Workload, n: int) -> int:
     return 4 * g * (2 if n > 0 else 1)
 
 
+def token_entry_bytes(wl: Workload) -> int:
+    """One buffered token (ktil, u): FP32, or BF16 with the traffic-lean buffer."""
+    return (2 if wl.buffer_bf16 else 4) * (wl.dk + wl.dv)
+
+
 def decode_launch_bytes(wl: Workload, n: int, flush: bool = False) -> float:
     """Bytes per head of the decode launch that buffers token n+1 of a window."""
-    e = 4 * (wl.dk + wl.dv)
+    e = token_entry_bytes(wl)
     b = io_bytes(wl) + state_bytes(wl) + n * e
     if flush:
         b += state_bytes(wl)           # the new window-start state is written once

@@ -160,3 +160,38 @@ def test_effective_bits_per_state_value():
     assert b["payload"] == pytest.approx(8.0) and b["total"] == pytest.approx(10.5)
     b = traffic.bits_per_value(configs.TINY_GDN)          # d = 64, r = 2
     assert b["payload"] == pytest.approx(8.0) and b["total"] == pytest.approx(11.0)
+
+
+def test_bf16_buffer_config(L):
+    cfg = lq.Config.from_workload(configs.GDN_PREFIX_CACHE)
+    full = lq.lq_workspace_bytes(cfg)
+    cfg.buffer_bf16 = 1
+    assert lq.lq_config_check(cfg) == lq.LQ_OK
+    lean = lq.lq_workspace_bytes(cfg)
+    # the W buffered tokens take half the bytes
+    wl = configs.GDN_PREFIX_CACHE
+    saved = wl.heads * wl.W * (wl.dk + wl.dv) * 2
+    assert full - lean == pytest.approx(saved, rel=0.01)
+    cfg.buffer_bf16 = 2
+    assert lq.lq_config_check(cfg) == lq.LQ_ERR_INVALID_ARG
+    for mode in ("fp32", "step"):
+        c2 = lq.Config.from_workload(configs.GDN_PREFIX_CACHE, mode=mode)
+        c2.buffer_bf16 = 1
+        assert lq.lq_config_check(c2) == lq.LQ_ERR_INVALID_ARG
+
+
+def test_bf16_buffer_with_bf16_rows_is_not_built(L):
+    cfg = lq.Config.from_workload(configs.GDN_DAMP)      # P = 16 BF16 rows
+    cfg.buffer_bf16 = 1
+    assert lq.lq_config_check(cfg) == lq.LQ_ERR_UNSUPPORTED
+
+
+def test_bf16_buffer_traffic_model():
+    # the window buffer's bytes halve; everything else is unchanged
+    from quantized_recurrent_state_lq_b200 import traffic
+    wl = configs.GDN_PREFIX_CACHE
+    lean = wl.with_(buffer_bf16=1)
+    assert traffic.token_entry_bytes(lean) * 2 == traffic.token_entry_bytes(wl) == 4 * (wl.dk + wl.dv)
+    n = 10
+    d = traffic.decode_launch_bytes(wl, n) - traffic.decode_launch_bytes(lean, n)
+    assert d == (n + 1) * 2 * (wl.dk + wl.dv)     # n entries read + one appended

@@ -17,9 +17,9 @@ STATE_REL = 1e-3   # FP32 state: max relative error per head
 TIE_EPS = 1e-3     # a flip this close to a rounding tie is counted as "at a tie"
 
 
-def _workload(gate, B, H, Hk, dk, dv, W, r, seed, P=0):
+def _workload(gate, B, H, Hk, dk, dv, W, r, seed, P=0, bf16=0):
     return configs.TINY_GDN.with_(gate=gate, B=B, H=H, Hk=Hk, dk=dk, dv=dv, W=W, r=r, seed=seed, P=P,
-                                  n_out_rows=3, n_out_cols=3, out_lo=10.0, out_hi=50.0)
+                                  n_out_rows=3, n_out_cols=3, out_lo=10.0, out_hi=50.0, buffer_bf16=bf16)
 
 
 def _rows_for(wl):
@@ -149,6 +149,22 @@ def test_windowed_teacher_forced(fused, gate, B, H, Hk, dk, dv, W, r):
     wl = _workload(gate, B, H, Hk, dk, dv, W, r, seed=31 + W)
     T = 3 * W + W // 2   # three windows and a ragged tail
     _teacher_forced(wl, T, fused, label=f"window {gate} d{dk}x{dv} W{W} r{r} fused{int(fused)}")
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("gate,B,H,Hk,dk,dv,W,r", [
+    ("gdn", 2, 2, 2, 128, 128, 64, 4),      # the benchmark's shape: one-pass tensor-core chunks
+    ("kda", 2, 3, 3, 128, 128, 32, 4),
+    ("gdn", 1, 2, 2, 64, 64, 16, 2),        # d = 64: the tile reads the BF16 entries directly
+    ("kda", 1, 3, 3, 128, 64, 5, 3),
+])
+def test_windowed_bf16_buffer_teacher_forced(fused, gate, B, H, Hk, dk, dv, W, r):
+    """The traffic-lean buffer: tokens' updates kept as bf16(k/Gamma), bf16(u);
+    the oracle's BF16-buffer mode takes the same rounding decisions in FP32."""
+    U.require_gpu()
+    wl = _workload(gate, B, H, Hk, dk, dv, W, r, seed=61 + W, bf16=1)
+    T = 2 * W + W // 2 + 1
+    _teacher_forced(wl, T, fused, label=f"bf16 buffer {gate} d{dk}x{dv} W{W} r{r} fused{int(fused)}")
 
 
 def test_damp_rows_teacher_forced():

@@ -54,6 +54,7 @@ struct BufSmem {
     int8_t dig[8][DK + 16];             // base-256 digits of a_k (rows 0-3) and a_q (rows 4-7)
     int rows[DK];                       // DAMP: key row of INT8 slot j, then of BF16 row p
     float v[DV];
+    float qk[DK];                       // q (BF16 buffer: k . q is formed at the end)
     float amax[kBufWarps][2];
     float kqw[kBufWarps];
     uint64_t mbar;
@@ -195,8 +196,10 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
         gt = (KDA ? a.alpha[hv * DK + t] : a.alpha[hv]) * gp;
         const float2 x = make_float2(gt * kk, gt * qq);
         S.x2[t] = x;
-        // the key of the update the state carries: k, or Gamma bf16(k / Gamma)
-        kqp = (tb ? gt * bf16_round(kk / gt) : kk) * qq;
+        // k . q for the output (BF16 buffer: Gamma bf16(k / Gamma) . q, formed
+        // at the end, next to the reduction it feeds)
+        kqp = tb ? 0.f : kk * qq;
+        if (tb) S.qk[t] = qq;
         if (!DAMP) {
             const float mi = reinterpret_cast<const float *>(rec + L.off_m)[t];
             ak_t = mi * x.x;
@@ -403,7 +406,23 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
 #pragma unroll
         for (int u = 0; u < 4; ++u) S.red[warp][4 * lane + u] = make_float2(ek[u], eq[u]);
     }
+    uint16_t khat = 0;
+    if (tb) {
+        // the key of the update the state carries: Gamma bf16(k / Gamma)
+        float kqh = 0.f;
+        if (t < DK) {
+            khat = bf16_rne(kk / gt);
+            kqh = (gt * bf16_to_f(khat)) * S.qk[t];
+        }
+        kqh = warp_sum(kqh);
+        if (lane == 0) S.kqw[warp] = kqh;
+    }
     __syncthreads();
+    if (tb) {
+        kq = 0.f;
+#pragma unroll
+        for (int w = 0; w < kBufWarps; ++w) kq += S.kqw[w];
+    }
     if (t < DV) {
         float yk = DAMP ? 0.f : S.rc[t].x, yq = DAMP ? 0.f : S.rc[t].y;
 #pragma unroll
@@ -425,7 +444,7 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
         if (!isfinite(o) || !isfinite(ut)) atomicOr(a.status, kStatusNonFinite);
     }
     if (t < DK) {
-        if (tb) rec_tok16[(size_t)a.n * EF + t] = bf16_rne(kk / gt);
+        if (tb) rec_tok16[(size_t)a.n * EF + t] = khat;
         else rec_ent[(size_t)E * EF + t] = kk / gt;
         if (KDA) rec_gam[t] = gt;
         else if (t == 0) rec_gam[0] = gt;

@@ -8,7 +8,7 @@
  * arrays and writes plain host arrays.
  *
  * Precision: all floating-point arithmetic is double, except the steps that
- * turn a value into an integer code (x = R/m, s = a/127, code = rne(x/s)),
+ * turn a value into an integer code (x = R/m, s = a/qmax, code = rne(x/s)),
  * which are taken in float, the precision the CUDA kernels decide them in.
  * Stored quantities that the method keeps in float (compensator vectors,
  * scales, the residual handed to the quantizer) are rounded to float at the
@@ -40,9 +40,12 @@
  *            energy and decay persistence are stored at higher precision.
  *
  * Readings where the pages are silent (each also listed in the design notes):
- *  - quantizer: symmetric, no zero point, codes in [-127, 127], round half to
- *    even, one scale per value column s_c = amax_c / 127 of the smoothed
- *    residual, one smoothing scale per key row m_i = RMS of row i.
+ *  - quantizer: symmetric, no zero point, codes in [-qmax, qmax], round half
+ *    to even, one scale per value column s_c = amax_c / qmax of the smoothed
+ *    residual, one smoothing scale per key row m_i = RMS of row i.  The b-bit
+ *    state (b = 8, 6 or 4: the LeapQuant page's 8-, 6- and 4-bit rows of its
+ *    results table) takes qmax = 2^(b-1) - 1 = 127, 31 or 7; the most
+ *    negative code of each width is left unused, as for INT8.
  *  - compensators: power iteration on the residual, start w = 1/sqrt(d_v),
  *    K steps of z = R w / |R w|, w = R^T z / |R^T z|; then c = R w and
  *    R <- R - c w^T; repeated r times (deflation).  A zero norm gives a zero
@@ -66,7 +69,15 @@ typedef struct {
     int P;         /* BF16 key rows per head (DAMP); 0 = none */
     int quantize;  /* 0: identity quantizer (FP32-state mode); 1: INT8 */
     int bf16_buffer; /* 1: each token's update is kept in BF16 (see lqo_step_bf16) */
+    int bits;      /* code width of the quantized state: 8 (0 reads as 8), 6 or 4 */
 } lqo_cfg;
+
+/* Largest code magnitude of a b-bit symmetric quantizer. */
+static int lqo_qmax(const lqo_cfg *cfg)
+{
+    const int b = cfg->bits == 0 ? 8 : cfg->bits;
+    return (1 << (b - 1)) - 1;
+}
 
 /* A quantized view of one head.  codes are [dk][dv] with the BF16 rows' codes
  * left at 0; hp holds the BF16 rows in the order of hp_rows. */
@@ -267,7 +278,8 @@ void lqo_quantize(const lqo_cfg *cfg, const int *hp_rows, const float *S,
             const float ax = fabsf(x[i * dv + c]);
             if (ax > a) a = ax;
         }
-        const float sc = a / 127.0f;
+        const float qmax = (float)lqo_qmax(cfg);
+        const float sc = a / qmax;
         out->s[c] = sc;
         for (int i = 0; i < dk; ++i) {
             int8_t code = 0;
@@ -275,8 +287,8 @@ void lqo_quantize(const lqo_cfg *cfg, const int *hp_rows, const float *S,
             if (!is_hp_row(hp_rows, P, i) && sc != 0.0f) {
                 const float qf = x[i * dv + c] / sc;   /* float division */
                 float rq = rintf(qf);                  /* round half to even */
-                if (rq > 127.0f) rq = 127.0f;
-                if (rq < -127.0f) rq = -127.0f;
+                if (rq > qmax) rq = qmax;
+                if (rq < -qmax) rq = -qmax;
                 code = (int8_t)rq;
                 rt = (double)x[i * dv + c] / (double)sc;
             }

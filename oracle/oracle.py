@@ -35,7 +35,8 @@ def build(force: bool = False) -> str:
 
 class _Cfg(C.Structure):
     _fields_ = [(n, C.c_int) for n in
-                ("dk", "dv", "gate", "W", "r", "K", "smoothing", "P", "quantize", "bf16_buffer")]
+                ("dk", "dv", "gate", "W", "r", "K", "smoothing", "P", "quantize", "bf16_buffer",
+                 "bits")]
 
 
 class _Views(C.Structure):
@@ -71,10 +72,12 @@ class Cfg:
     P: int = 0
     quantize: int = 1
     bf16_buffer: int = 0   # 1: buffered updates kept in BF16 (lqo_step_bf16)
+    bits: int = 8          # code width of the quantized state: 8, 6 or 4
 
     def c(self) -> _Cfg:
         return _Cfg(self.dk, self.dv, 1 if self.gate == "kda" else 0, self.W,
-                    self.r, self.K, self.smoothing, self.P, self.quantize, self.bf16_buffer)
+                    self.r, self.K, self.smoothing, self.P, self.quantize, self.bf16_buffer,
+                    self.bits)
 
     @property
     def ga(self) -> int:

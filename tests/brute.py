@@ -41,9 +41,9 @@ def power_closed_form(R: np.ndarray, K: int) -> np.ndarray:
     return x / np.linalg.norm(x)
 
 
-def codes_exhaustive(x: np.ndarray, s: np.ndarray) -> np.ndarray:
-    """argmin over k in [-127, 127] of |x/s - k|, ties to the even k."""
-    levels = np.arange(-127, 128, dtype=np.float64)
+def codes_exhaustive(x: np.ndarray, s: np.ndarray, qmax: int = 127) -> np.ndarray:
+    """argmin over k in [-qmax, qmax] of |x/s - k|, ties to the even k."""
+    levels = np.arange(-qmax, qmax + 1, dtype=np.float64)
     out = np.zeros(x.shape, np.int64)
     for i in range(x.shape[0]):
         for c in range(x.shape[1]):
@@ -58,8 +58,8 @@ def codes_exhaustive(x: np.ndarray, s: np.ndarray) -> np.ndarray:
     return out
 
 
-def quantize(S: np.ndarray, r: int, K: int, smoothing: bool = True):
-    """Brute-force quantizer Q on one head (no BF16 rows).
+def quantize(S: np.ndarray, r: int, K: int, smoothing: bool = True, qmax: int = 127):
+    """Brute-force quantizer Q on one head (no BF16 rows), codes in [-qmax, qmax].
 
     Float rounding happens where the method stores a float: compensator
     vectors, the residual handed to the codec, m and s, and x = R/m.
@@ -79,8 +79,8 @@ def quantize(S: np.ndarray, r: int, K: int, smoothing: bool = True):
         m = np.ones(R.shape[0], f32)
     x = (R32 / m[:, None]).astype(f32)
     a = np.abs(x).max(axis=0).astype(f32)
-    s = (a / f32(127)).astype(f32)
-    codes = codes_exhaustive(x, s)
+    s = (a / f32(qmax)).astype(f32)
+    codes = codes_exhaustive(x, s, qmax)
     dk, dv = R.shape
     return {"codes": codes, "m": m, "s": s, "c": np.array(cs, f32).reshape(r, dk),
             "w": np.array(ws, f32).reshape(r, dv), "R32": R32, "x": x}
@@ -94,14 +94,15 @@ def dequantize(view) -> np.ndarray:
     return S
 
 
-def run_windowed(S0, toks, W: int, r: int, K: int, gate: str, smoothing=True, quantize_on=True):
+def run_windowed(S0, toks, W: int, r: int, K: int, gate: str, smoothing=True, quantize_on=True,
+                 qmax: int = 127):
     """Whole windowed decode of one head with literal matrices.
 
     toks: list of (q, k, v, beta, alpha).  Returns (outputs, last view).
     """
     view = None
     if quantize_on:
-        view = quantize(S0, r, K, smoothing)
+        view = quantize(S0, r, K, smoothing, qmax)
         S = dequantize(view)
     else:
         S = np.asarray(S0, np.float64)
@@ -113,7 +114,7 @@ def run_windowed(S0, toks, W: int, r: int, K: int, gate: str, smoothing=True, qu
         outs.append(o)
         n += 1
         if quantize_on and n == W:
-            view = quantize(Sp.T.astype(f32), r, K, smoothing)
+            view = quantize(Sp.T.astype(f32), r, K, smoothing, qmax)
             Sp = dequantize(view).T.copy()
             n = 0
     return np.array(outs), view

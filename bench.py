@@ -118,7 +118,8 @@ def oracle_sample_seconds(wl, heads: int, threads: int, seed_offset: int = 0):
     import numpy as np
     from oracle import oracle as O
     sw = wl.with_(B=max(1, heads // wl.H + (heads % wl.H > 0)), seed=wl.seed + seed_offset)
-    oc = O.Cfg(dk=wl.dk, dv=wl.dv, gate=wl.gate, W=wl.W, r=wl.r, K=wl.K, smoothing=wl.smoothing, P=wl.P)
+    oc = O.Cfg(dk=wl.dk, dv=wl.dv, gate=wl.gate, W=wl.W, r=wl.r, K=wl.K, smoothing=wl.smoothing, P=wl.P,
+               bf16_buffer=wl.buffer_bf16, bits=wl.bits)
     pre = gen.token_inputs(sw, 16, stream="prefill")
     S0 = O.prefill(O.Cfg(dk=wl.dk, dv=wl.dv, gate=wl.gate, quantize=0), O.per_head_inputs(pre, wl.H),
                    nthreads=threads).astype(np.float32).reshape(sw.B, wl.H, wl.dk, wl.dv)
@@ -185,6 +186,8 @@ def profile_traffic(wl):
     for f in sorted(os.listdir(csrc)):
         h.update(open(os.path.join(csrc, f), "rb").read())
     if kv.get("csrc_sha256", "").strip() != h.hexdigest()[:16] or kv.get("workload", "").strip() != wl.name:
+        return None
+    if wl.bits != 8 or wl.buffer_bf16:   # the capture is of the INT8 state with the FP32 buffer
         return None
     try:
         return float(kv["dram_bytes_per_launch_full"])
@@ -261,12 +264,10 @@ def mode_throughput(wl, S0, mode: str, windows: int, stream):
     return v
 
 
-def bf16_buffer_variant(wl, S0, stream, peak_gbs: float, windows: int = 3) -> dict:
-    """The traffic-lean option on the same inputs: buffered token updates kept
-    in BF16 (halves the window buffer's bytes; not the method as stated).
-    Whole-window throughput by graph replay, and the buffering launch's
-    achieved algorithmic bandwidth."""
-    wv = wl.with_(buffer_bf16=1)
+def variant(wv, S0, stream, peak_gbs: float, note: str, windows: int = 3) -> dict:
+    """Another configuration of the window step on the same inputs: whole-window
+    throughput by graph replay, and the buffering launch's achieved
+    algorithmic bandwidth."""
     r = runner.WindowRunner(wv, S0, tokens=wv.W * min(2, wv.T // wv.W))
     r.capture()
     for k in range(2):
@@ -276,7 +277,7 @@ def bf16_buffer_variant(wl, S0, stream, peak_gbs: float, windows: int = 3) -> di
     t_buf, t_flush = kernel_times(r, 1, stream)
     rc = lq.lq_get_status(r.st)
     if rc != lq.LQ_OK:
-        raise lq.LqError(rc, "bf16-buffer variant status")
+        raise lq.LqError(rc, f"variant status ({note})")
     launch_bytes = traffic.nonflush_launch_bytes(wv) * wv.heads
     del r
     torch.cuda.empty_cache()
@@ -284,7 +285,11 @@ def bf16_buffer_variant(wl, S0, stream, peak_gbs: float, windows: int = 3) -> di
             "decode_buffering_mean_s": t_buf, "decode_flushing_mean_s": t_flush,
             "buffering_roofline_frac": launch_bytes / t_buf / 1e9 / peak_gbs,
             "algorithmic_bytes_per_step": traffic.window_bytes(wv) * wv.heads,
-            "note": "option: buffered token updates stored as bf16(k/Gamma), bf16(u)"}
+            "state_bits_per_value": traffic.bits_per_value(wv), "note": note}
+
+
+def state_dtype(wl) -> str:
+    return "int8" if wl.bits == 8 else f"int{wl.bits} (bit-packed)"
 
 
 def run_ours(args, wl, world, rank, pg):
@@ -322,7 +327,7 @@ def run_ours(args, wl, world, rank, pg):
             "peak_source": f"{peak_src} hbm_gbs (copy kernel)"}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * dt_max / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "state_dtype": "int8", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "state_dtype": state_dtype(wl), "data": "synthetic",
             "config": {"workload": wl.name, "gate": wl.gate, "prefill": wl.prefill, "B": wl.B, "H": wl.H, "Hk": wl.Hk, "dk": wl.dk,
                        "dv": wl.dv, "W": wl.W, "r": wl.r, "K": wl.K, "P": wl.P, "step": "one window per head",
                        "l2": "state + buffers + inputs larger than L2 (no flush needed)",
@@ -343,7 +348,7 @@ def run_ours(args, wl, world, rank, pg):
     del r
     torch.cuda.empty_cache()
 
-    if not args.no_modes and wl.P == 0 and not wl.buffer_bf16:
+    if not args.no_modes and wl.P == 0 and not wl.buffer_bf16 and wl.bits == 8:
         modes = {"window_int8": value / world}
         modes["fp32_state"] = mode_throughput(wl, S0, "fp32", 4, stream)
         modes["per_step_int8"] = mode_throughput(wl, S0, "step", 2, stream)
@@ -351,7 +356,12 @@ def run_ours(args, wl, world, rank, pg):
         modes["naive_per_step_int8"] = mode_throughput(nv, S0, "step", 2, stream)
         modes["window_vs_fp32_speedup"] = modes["window_int8"] / modes["fp32_state"]
         line["modes_per_gpu"] = modes
-        line["buffer_bf16_per_gpu"] = bf16_buffer_variant(wl, S0, stream, peaks["hbm_gbs"])
+        line["buffer_bf16_per_gpu"] = variant(wl.with_(buffer_bf16=1), S0, stream, peaks["hbm_gbs"],
+                                              "option: buffered token updates stored as bf16(k/Gamma), bf16(u)")
+        line["low_bit_states_per_gpu"] = {
+            f"int{b}": variant(wl.with_(bits=b), S0, stream, peaks["hbm_gbs"],
+                               f"{b}-bit window-start state (codes in +-{(1 << (b - 1)) - 1}, bit-packed)")
+            for b in (6, 4)}
 
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(wl)
@@ -373,6 +383,8 @@ def main():
     ap.add_argument("--prefill", type=int, default=None, help="override the prefill length (profiling runs)")
     ap.add_argument("--buffer-bf16", action="store_true",
                     help="run the traffic-lean option (buffered token updates in BF16) as the main line")
+    ap.add_argument("--bits", type=int, choices=[8, 6, 4], default=8,
+                    help="code width of the quantized state for the main line (6, 4: bit-packed)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -383,6 +395,8 @@ def main():
         wl = wl.with_(prefill=args.prefill)
     if args.buffer_bf16:
         wl = wl.with_(buffer_bf16=1)
+    if args.bits != 8:
+        wl = wl.with_(bits=args.bits)
     world, rank, local, pg = dist_setup()
     try:
         if args.impl == "reference":

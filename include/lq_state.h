@@ -88,10 +88,18 @@ typedef struct {
                                compensators stay FP32.  Halves the window buffer's bytes.
                                Not built together with BF16 rows (n_hp_rows > 0:
                                LQ_ERR_UNSUPPORTED).  0: FP32 buffer (the method as stated). */
+    int32_t state_bits;     /* code width of the quantized state (INT8 modes and the codec): 8 (0
+                               reads as 8), 6 or 4 -- the LeapQuant page's 8-, 6- and 4-bit states:
+                               the same quantizer with codes in [-qmax, qmax], qmax = 2^(b-1) - 1
+                               (127, 31, 7), s_c = amax_c / qmax.  6 and 4 are bit-packed in the
+                               workspace (0.75 and 0.5 bytes a code); views (lq_qstate_view) keep
+                               one code per int8 byte.  Not built with BF16 rows (n_hp_rows > 0:
+                               LQ_ERR_UNSUPPORTED); FP32 mode takes 0 or 8 only. */
 } lq_config;
 
 /* A quantized state in plain arrays (all device pointers, caller-owned):
  *   codes     int8   [B,H,dk-P,dv]  INT8 key rows in increasing row order, dv contiguous
+ *                                   (one code per byte also with state_bits 6 or 4)
  *   bf16_rows uint16 [B,H,P,dv]     BF16 bit patterns of the rows listed in hp_row_ids
  *   m         float  [B,H,dk]       smoothing scale per key row (1 on BF16 rows)
  *   s         float  [B,H,dv]       quantization scale per value column
@@ -158,7 +166,8 @@ int lq_state_export_fp32(const lq_state *st, float *d_S, void *stream);
 
 /* Copy the window-start quantized state out to / in from plain arrays (layout of
  * lq_qstate_view, for this state's B and H).  Import starts a new window
- * (buffer emptied, Gamma = 1).  INT8 modes only.  Used for checkpoint/resume. */
+ * (buffer emptied, Gamma = 1); with state_bits 6 or 4 it saturates codes to
+ * +-qmax.  INT8 modes only.  Used for checkpoint/resume. */
 int lq_state_export_view(const lq_state *st, const lq_qstate_view *out, void *stream);
 int lq_state_import_view(lq_state *st, const lq_qstate_view *in, void *stream);
 

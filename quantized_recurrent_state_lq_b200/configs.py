@@ -51,6 +51,7 @@ class Workload:
     calib_prefills: int = 0
     calib_tokens: int = 0
     buffer_bf16: int = 0         # 1: the traffic-lean BF16 window buffer (an option, not a config)
+    bits: int = 8                # code width of the quantized state: 8, or the packed 6 / 4 bits
 
     @property
     def heads(self) -> int:

@@ -33,15 +33,21 @@ size_t align_sz(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool is_int8(const lq_config *c) { return c->mode == LQ_MODE_INT8_STEP || c->mode == LQ_MODE_INT8_WINDOW; }
 
+// Code width of the quantized state (0 reads as 8).
+int bits_of(const lq_config *c) { return c->state_bits == 0 ? 8 : c->state_bits; }
+
 Layout layout_of(const lq_config *c) {
     const int W = c->mode == LQ_MODE_INT8_STEP ? 1 : c->W;
     return lq::make_layout(c->dk, c->dv, c->n_hp_rows, c->r, W, c->gate == LQ_GATE_CHANNEL,
-                           c->mode == LQ_MODE_INT8_WINDOW && c->buffer_bf16 == 1);
+                           c->mode == LQ_MODE_INT8_WINDOW && c->buffer_bf16 == 1, bits_of(c));
 }
 
 int check_codec_fields(const lq_config *c) {
     if (c->dk != 64 && c->dk != 128) return LQ_ERR_UNSUPPORTED;
     if (c->dv != 64 && c->dv != 128) return LQ_ERR_UNSUPPORTED;
+    const int bits = bits_of(c);
+    if (bits != 8 && bits != 6 && bits != 4) return LQ_ERR_INVALID_ARG;
+    if (bits != 8 && c->n_hp_rows > 0) return LQ_ERR_UNSUPPORTED;   // packed codes: no BF16 rows
     if (c->r < 0 || c->r > (c->dk < c->dv ? c->dk : c->dv)) return LQ_ERR_INVALID_ARG;
     if (c->power_iters < 0 || c->power_iters > 1000) return LQ_ERR_INVALID_ARG;
     if (c->n_hp_rows < 0 || c->n_hp_rows >= c->dk) return LQ_ERR_INVALID_ARG;
@@ -61,6 +67,7 @@ int check_config(const lq_config *c) {
     if (c->buffer_bf16 != 0 && c->buffer_bf16 != 1) return LQ_ERR_INVALID_ARG;
     if (c->buffer_bf16 == 1 && c->mode != LQ_MODE_INT8_WINDOW) return LQ_ERR_INVALID_ARG;
     if (c->buffer_bf16 == 1 && c->n_hp_rows > 0) return LQ_ERR_UNSUPPORTED;   // not built with BF16 rows
+    if (c->mode == LQ_MODE_FP32 && c->state_bits != 0 && c->state_bits != 8) return LQ_ERR_INVALID_ARG;
     int rc = check_codec_fields(c);
     if (rc) return rc;
     if (is_int8(c)) {
@@ -219,7 +226,7 @@ int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_
         if (is_int8(cfg)) {
             lq::CodecArgs a{};
             a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing;
-            a.P = cfg->n_hp_rows; a.hp_rows = st->hp_rows; a.S_in = d_S0;
+            a.P = cfg->n_hp_rows; a.hp_rows = st->hp_rows; a.S_in = d_S0; a.bits = bits_of(cfg);
             a.q = record_ptrs(st);
             a.status = st->status;
             e = lq::launch_quantize(a, cfg->dk, cfg->dv, (int)st->heads, s);
@@ -296,7 +303,7 @@ int lq_state_export_view(const lq_state *st, const lq_qstate_view *out, void *st
     int rc = check_view(&st->cfg, out);
     if (rc) return rc;
     lq::CodecArgs a{};
-    a.H = st->cfg.H; a.r = st->cfg.r; a.P = st->cfg.n_hp_rows;
+    a.H = st->cfg.H; a.r = st->cfg.r; a.P = st->cfg.n_hp_rows; a.bits = bits_of(&st->cfg);
     a.q = record_ptrs(st);
     a.q.gam = nullptr;
     a.q2 = view_ptrs(&st->cfg, out);
@@ -309,7 +316,7 @@ int lq_state_import_view(lq_state *st, const lq_qstate_view *in, void *stream) {
     int rc = check_view(&st->cfg, in);
     if (rc) return rc;
     lq::CodecArgs a{};
-    a.H = st->cfg.H; a.r = st->cfg.r; a.P = st->cfg.n_hp_rows;
+    a.H = st->cfg.H; a.r = st->cfg.r; a.P = st->cfg.n_hp_rows; a.bits = bits_of(&st->cfg);
     a.q = view_ptrs(&st->cfg, in);
     a.q2 = record_ptrs(st);
     rc = cuda_rc(lq::launch_qcopy(a, st->cfg.dk, st->cfg.dv, (int)st->heads, static_cast<cudaStream_t>(stream)));
@@ -326,6 +333,7 @@ static int codec_common(const lq_config *cfg, const int32_t *h_rows, lq::CodecAr
     rc = check_hp_rows(cfg, h_rows);
     if (rc) return rc;
     a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing; a.P = cfg->n_hp_rows;
+    a.bits = bits_of(cfg);
     *d_rows = nullptr;
     if (cfg->n_hp_rows > 0) {
         const size_t nb = (size_t)cfg->H * cfg->n_hp_rows * 4;
@@ -391,6 +399,7 @@ int lq_quantize_state_static(const lq_config *cfg, const float *d_S, const int32
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     lq::CodecArgs a{};
     a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing; a.P = cfg->n_hp_rows;
+    a.bits = bits_of(cfg);
     if (cfg->n_hp_rows > 0) {
         int32_t *rows = nullptr;
         rc = static_rows_ptr(&rows);
@@ -434,8 +443,10 @@ int lq_damp_select(const lq_config *cfg, int32_t n_states, const float *d_states
     int rc = check_codec_fields(cfg);
     if (rc) return rc;
     if (cfg->n_hp_rows < 1) return LQ_ERR_INVALID_ARG;
+    if (bits_of(cfg) != 8) return LQ_ERR_UNSUPPORTED;   // the selection scores INT8 error energy
     lq::CodecArgs a{};
     a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing; a.P = cfg->n_hp_rows;
+    a.bits = 8;
     a.S_in = d_states;
     a.n_states = n_states;
     a.n_gate_samples = n_gate_samples;

@@ -28,7 +28,7 @@ __device__ __forceinline__ CodecOut codec_out_of(const QPtrs &q, int head) {
     return o;
 }
 
-template <int DK, int DV>
+template <int DK, int DV, int BITS>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const CodecArgs a) {
     __shared__ QSmem<DK, DV> sm;
     extern __shared__ __align__(16) unsigned char dyn[];
@@ -40,8 +40,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const CodecArgs a) {
     tile_load_global<DK, DV>(R, a.S_in + (size_t)head * DK * DV);
     const CodecOut out = codec_out_of(a.q, head);
     double eacc[T::RPT];
-    codec_quantize_exact<DK, DV, false>(R, a.r, a.K, a.smoothing, a.P, a.P > 0 ? sm.map : nullptr, sm.cs, X, out,
-                                        eacc);
+    codec_quantize_exact<DK, DV, false, BITS>(R, a.r, a.K, a.smoothing, a.P, a.P > 0 ? sm.map : nullptr, sm.cs, X,
+                                              out, eacc);
     if (a.q.gam) {
         float *g = reinterpret_cast<float *>(a.q.gam + (size_t)head * a.q.gam_hs);
         for (int i = threadIdx.x; i < a.q.gam_n; i += kThreads) g[i] = 1.0f;
@@ -94,13 +94,39 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(const CodecArgs a)
 }
 
 // Copy a quantized state from q to q2 (same head numbering), setting q2's
-// Gamma to 1 when it has one.
+// Gamma to 1 when it has one.  Row-major (view) codes are one per byte; a
+// record's 4 / 6-bit codes are packed (an 8-row group per thread), and codes
+// entering one are saturated to +-qmax.
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads) qcopy_kernel(const CodecArgs a) {
     const int head = blockIdx.x, t = threadIdx.x;
     const QPtrs &x = a.q, &y = a.q2;
     const int P = a.P;
-    if (x.codes_t == y.codes_t) {
+    if (a.bits < 8 && x.codes_t != y.codes_t) {
+        const int qmax = (1 << (a.bits - 1)) - 1;
+        const int8_t *src = reinterpret_cast<const int8_t *>(x.codes + (size_t)head * x.codes_hs);
+        int8_t *dst = reinterpret_cast<int8_t *>(y.codes + (size_t)head * y.codes_hs);
+        for (int e = t; e < (DK / 8) * DV; e += kThreads) {
+            const int g = e / DV, c = e % DV;
+            if (x.codes_t) {   // record -> view
+                const unsigned char *pk = reinterpret_cast<const unsigned char *>(src);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    dst[(size_t)(8 * g + k) * DV + c] = (int8_t)packed_code(pk, c, 8 * g + k, DK, DV, a.bits);
+            } else {           // view -> record
+                uint32_t nw = 0u, pw = 0u;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int v = max(-qmax, min(qmax, (int)src[(size_t)(8 * g + k) * DV + c]));
+                    nw |= ((uint32_t)v & 15u) << (4 * k);
+                    pw |= (((uint32_t)v >> 4) & 3u) << (2 * k);
+                }
+                unsigned char *pk = reinterpret_cast<unsigned char *>(dst);
+                *reinterpret_cast<uint32_t *>(pk + nib_off(c, g, DK)) = nw;
+                if (a.bits == 6) *reinterpret_cast<uint16_t *>(pk + pair_off(c, g, DK, DV)) = (uint16_t)pw;
+            }
+        }
+    } else if (x.codes_t == y.codes_t) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x.codes + (size_t)head * x.codes_hs);
         uint4 *dst = reinterpret_cast<uint4 *>(y.codes + (size_t)head * y.codes_hs);
         const int n16 = (DK - P) * DV / 16;
@@ -215,8 +241,18 @@ static cudaError_t allow_smem(K kern, size_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+using CodecKernel = void (*)(const CodecArgs);
+
+template <int BITS>
+static CodecKernel pick_quantize(int dk, int dv) {
+    if (dk == 128 && dv == 128) return quantize_kernel<128, 128, BITS>;
+    if (dk == 64 && dv == 64) return quantize_kernel<64, 64, BITS>;
+    if (dk == 64 && dv == 128) return quantize_kernel<64, 128, BITS>;
+    return quantize_kernel<128, 64, BITS>;
+}
+
 cudaError_t launch_quantize(const CodecArgs &a, int dk, int dv, int heads, cudaStream_t s) {
-    auto kern = LQ_PICK(dk, dv, quantize_kernel);
+    auto kern = a.bits == 4 ? pick_quantize<4>(dk, dv) : a.bits == 6 ? pick_quantize<6>(dk, dv) : pick_quantize<8>(dk, dv);
     const size_t sm = exact_bytes(dk, dv);
     cudaError_t e = allow_smem(kern, sm);
     if (e != cudaSuccess) return e;

@@ -14,7 +14,9 @@
 //   2. BF16 rows: bf16_rne(R_i) for the head's listed key rows.
 //   3. m_i = sqrt(mean_c R_ic^2) (double accumulation), 1 if zero or if
 //      smoothing is off;  x = R / m.
-//   4. s_c = max_i |x_ic| / 127 over INT8 rows;  C = clamp(rne(x / s), +-127).
+//   4. s_c = max_i |x_ic| / qmax over INT8 rows;  C = clamp(rne(x / s), +-qmax),
+//      qmax = 2^(b-1) - 1 for b-bit codes (127, 31, 7: the LeapQuant page's
+//      8-, 6- and 4-bit states).
 //
 // Tile layout: a thread owns RPT consecutive key rows and 16 value columns, in
 // four groups of four adjacent columns spaced CG*4 apart:
@@ -53,7 +55,8 @@ struct CodecSmem {
 // Where the codec writes one head's quantized state.
 struct CodecOut {
     int8_t *codes;     // [(DK-P)][DV] by slot, or (codes_t) value-column-major, swizzled
-    int codes_t;       // 1: code_off_t layout (no BF16 rows); 0: row-major by INT8 slot
+    int codes_t;       // 1: code_off_t layout, or the packed planes of 4 / 6-bit codes (no
+                       //    BF16 rows); 0: row-major by INT8 slot, one code per byte
     uint16_t *hp;      // [P][DV]
     float *m;          // [DK]
     float *s;          // [DV]
@@ -351,12 +354,14 @@ __device__ void codec_compensators_fp64(float (&R)[Tile<DK, DV>::RPT][16], int r
 // (slot >= 0 for INT8 rows, -1-p for BF16 row p); with P == 0 it may be null.
 // ENERGY: instead of writing codes, add sum_c (R - Deq)^2 of the residual to
 // eacc[r] (DAMP calibration); in that mode nothing is written.
-template <int DK, int DV, bool ENERGY, int NT = kThreads>
+template <int DK, int DV, bool ENERGY, int NT = kThreads, int BITS = 8>
 __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothing, int P, const int *map,
                              CodecSmem<DK, DV, NT> &cs, const CodecOut &out,
                              double (&eacc)[Tile<DK, DV, NT>::RPT], int buf) {
     using T = Tile<DK, DV, NT>;
     constexpr int RPT = T::RPT, CG = T::CG;
+    constexpr float kQmax = (float)((1 << (BITS - 1)) - 1);   // 127, 31 or 7
+    static_assert(BITS == 8 || BITS == 6 || BITS == 4, "code widths");
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int cg = t % CG, rg = t / CG;
     const int row0 = rg * RPT;
@@ -459,7 +464,7 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
             float a = 0.f;
 #pragma unroll
             for (int w = 0; w < T::NW; ++w) a = fmaxf(a, cs.red[buf][w][t]);
-            const float sc = a / 127.0f;
+            const float sc = a / kQmax;
             cs.sc[t] = sc;
             cs.ysc[t] = __frcp_rn(sc);
             if (!ENERGY) out.s[t] = sc;
@@ -470,7 +475,7 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
     // Codes (or the error energy of the INT8 reconstruction).
     // C = clamp(rne(x / s)), the quotient correctly rounded as in the oracle.
     // For a column scale in [2^-20, 2^20] (col_fast) the reciprocal-and-
-    // correction quotient is exact for |x| >= 2^-79 (|x / s| <= 127 for INT8
+    // correction quotient is exact for |x| >= 2^-79 (|x / s| <= qmax for INT8
     // rows); below that, exact or not, it is under 2^-58 in size and rounds
     // to code 0 like the exact one: no branch per element.  Other scales (0
     // included) take IEEE division.  s and 1/s come from shared memory.
@@ -478,9 +483,9 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
     // clamp, then round half to even and convert with one FP32 add of
     // 1.5 * 2^23 (the sum's last bit is the integer, RN does the rounding) and
     // an integer subtract: no conversion-pipe instructions.  Clamping first is
-    // equivalent to clamping the rounded value (127 is an integer).
+    // equivalent to clamping the rounded value (qmax is an integer).
     auto clamp_code = [](float qt) -> uint32_t {
-        const float cq = fminf(fmaxf(qt, -127.f), 127.f) + 12582912.0f;
+        const float cq = fminf(fmaxf(qt, -kQmax), kQmax) + 12582912.0f;
         return (uint32_t)(__float_as_int(cq) - 0x4B400000) & 0xffu;
     };
     auto code_fast = [&](float x, float sc, float ysc) -> uint32_t { return clamp_code(div_rn_unchecked(x, sc, ysc)); };
@@ -509,6 +514,41 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
 #pragma unroll
             for (int mm = CG / 2; mm >= 1; mm >>= 1) e += __shfl_xor_sync(0xffffffffu, e, mm);
             eacc[r] += e;
+        }
+    } else if (BITS < 8 && out.codes_t) {
+        // packed 4 / 6-bit planes (no BF16 rows; the codes_t layout): the
+        // RPT rows of one column go into the nibble / pair words of their
+        // 8-row group, the 8 / RPT row groups of a code group (lanes CG
+        // apart in one warp) OR their words together and the first stores.
+        static_assert(RPT <= 8, "an 8-row code group spans whole row groups");
+        constexpr int GT = 8 / RPT;
+        unsigned char *base = reinterpret_cast<unsigned char *>(out.codes);
+        const int g = row0 >> 3, k0 = row0 & 7;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const int col = T::col(cg, q / 4) + q % 4;
+            const float sc = cs.sc[col], ysc = cs.ysc[col];
+            uint32_t nw = 0u, pw = 0u;
+            auto put = [&](int r, uint32_t b) {
+                nw |= (b & 15u) << (4 * (k0 + r));
+                pw |= ((b >> 4) & 3u) << (2 * (k0 + r));
+            };
+            if (col_fast(sc)) {   // one decision per column, as for INT8
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) put(r, code_fast(R[r][q], sc, ysc));
+            } else {
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) put(r, code_ieee(R[r][q], sc));
+            }
+#pragma unroll
+            for (int o = CG; o < CG * GT; o <<= 1) {
+                nw |= __shfl_xor_sync(0xffffffffu, nw, o);
+                if (BITS == 6) pw |= __shfl_xor_sync(0xffffffffu, pw, o);
+            }
+            if (k0 == 0) {
+                *reinterpret_cast<uint32_t *>(base + nib_off(col, g, DK)) = nw;
+                if (BITS == 6) *reinterpret_cast<uint16_t *>(base + pair_off(col, g, DK, DV)) = (uint16_t)pw;
+            }
         }
     } else if (out.codes_t) {
         // value-column-major (no BF16 rows): the thread's RPT rows of one
@@ -561,21 +601,21 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
 }
 
 // The whole quantizer with the FP32 compensator step (window flush).
-template <int DK, int DV, bool ENERGY, int NT = kThreads>
+template <int DK, int DV, bool ENERGY, int NT = kThreads, int BITS = 8>
 __device__ void codec_quantize(float (&R)[Tile<DK, DV, NT>::RPT][16], int r_comp, int K, int smoothing, int P,
                                const int *map, CodecSmem<DK, DV, NT> &cs, const CodecOut &out,
                                double (&eacc)[Tile<DK, DV, NT>::RPT]) {
     const int buf = codec_compensators_fp32<DK, DV, !ENERGY, NT>(R, r_comp, K, cs, out);
-    codec_finish<DK, DV, ENERGY, NT>(R, smoothing, P, map, cs, out, eacc, buf);
+    codec_finish<DK, DV, ENERGY, NT, BITS>(R, smoothing, P, map, cs, out, eacc, buf);
 }
 
 // The whole quantizer with the double-precision compensator step.
-template <int DK, int DV, bool ENERGY>
+template <int DK, int DV, bool ENERGY, int BITS = 8>
 __device__ void codec_quantize_exact(float (&R)[Tile<DK, DV>::RPT][16], int r_comp, int K, int smoothing, int P,
                                      const int *map, CodecSmem<DK, DV> &cs, ExactSmem<DK, DV> &X,
                                      const CodecOut &out, double (&eacc)[Tile<DK, DV>::RPT]) {
     codec_compensators_fp64<DK, DV, !ENERGY>(R, r_comp, K, X, out);
-    codec_finish<DK, DV, ENERGY>(R, smoothing, P, map, cs, out, eacc, 0);
+    codec_finish<DK, DV, ENERGY, kThreads, BITS>(R, smoothing, P, map, cs, out, eacc, 0);
 }
 
 // Reconstruction of a head's current state into the tile, in three parts:
@@ -583,8 +623,9 @@ __device__ void codec_quantize_exact(float (&R)[Tile<DK, DV>::RPT][16], int r_co
 //   tile_add_entries:  R += sum_e ktil_e u_e^T over n entries [n][DK+DV]
 //   tile_gamma:        R *= Gamma (by key row); true if every value is finite
 // The arrays may live in shared or global memory: m_s [DK], s_s [DV],
-// hp_s [P][DV], codes_s (layout per codes_t), gam_s [DK].
-template <int DK, int DV, int NT, bool ADD = false>
+// hp_s [P][DV], codes_s (layout per codes_t; BITS < 8: the packed planes),
+// gam_s [DK].
+template <int DK, int DV, int NT, bool ADD = false, int BITS = 8>
 __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][16], const float *m_s,
                                              const float *s_s, const uint16_t *hp_s, const int8_t *codes_s, int P,
                                              const int *map, bool codes_t) {
@@ -592,6 +633,50 @@ __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][1
     constexpr int RPT = T::RPT;
     const int t = threadIdx.x, cg = t % T::CG, rg = t / T::CG, row0 = rg * RPT;
     auto put = [&](int r, int q, float v) { R[r][q] = ADD ? R[r][q] + v : v; };
+    if (BITS < 8) {
+        // packed 4 / 6-bit codes: the thread's rows lie in one 8-row group,
+        // unpacked to signed bytes c * 2^(8-BITS), scaled back exactly
+        static_assert(RPT <= 8, "rows of a thread within one code group");
+        constexpr float kInv = BITS == 4 ? 0.0625f : 0.25f;
+        const unsigned char *cb = reinterpret_cast<const unsigned char *>(codes_s);
+        const int g = row0 >> 3, k0 = row0 & 7;
+        float sv[16];
+        load_cols16<DK, DV>(s_s, sv);
+        float mi[RPT];
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) mi[r] = m_s[row0 + r];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int col = T::col(cg, q) + u;
+                const uint32_t nib = *reinterpret_cast<const uint32_t *>(cb + nib_off(col, g, DK));
+                const uint32_t pr =
+                    BITS == 6 ? spread_pairs(*reinterpret_cast<const uint16_t *>(cb + pair_off(col, g, DK, DV)), false)
+                              : 0u;
+                uint32_t lo, hi;
+                unpack_group<(BITS < 8 ? BITS : 4)>(nib, pr, lo, hi);
+                if (RPT == 8) {
+                    float fl[4], fh[4];
+                    s8x4_to_f(lo, fl);
+                    s8x4_to_f(hi, fh);
+#pragma unroll
+                    for (int r = 0; r < RPT; ++r) {
+                        const float cf = ((r & 1) ? fh[r >> 1] : fl[r >> 1]) * kInv;
+                        put(r, 4 * q + u, (cf * sv[4 * q + u]) * mi[r]);
+                    }
+                } else {
+#pragma unroll
+                    for (int r = 0; r < RPT; ++r) {
+                        const int k = k0 + r;
+                        const uint32_t w = (k & 1) ? hi : lo;
+                        const float cf = (float)(int8_t)((w >> (8 * (k >> 1))) & 0xffu) * kInv;
+                        put(r, 4 * q + u, (cf * sv[4 * q + u]) * mi[r]);
+                    }
+                }
+            }
+        return;
+    }
     if (codes_t && (RPT == 4 || RPT == 8)) {
         float sv[16];
         load_cols16<DK, DV>(s_s, sv);

@@ -21,7 +21,8 @@ constexpr int kStatusTimeout = 2;
 //   m       f32   [dk]              smoothing scale per key row (1 on BF16 rows)
 //   s       f32   [dv]              quantization scale per value column
 //   hp      u16   [P][dv]           BF16 rows (order of the head's row list)
-//   codes   int8  [dk-P][dv]        INT8 codes (layout: code_off_t below)
+//   codes   int8  [dk-P][dv]        INT8 codes (layout: code_off_t below), or
+//                                   4 / 6-bit codes bit-packed (nib_off, pair_off)
 //   comps   f32   [r][dk+dv]        compensator j = (c_j [dk], w_j [dv])
 //   tokens  f32 or bf16 [W][dk+dv]  buffered token tau = (k_tau/Gamma_tau, u_tau)
 //   gam     f32   [dk] (KDA) / [4] (GDN)   cumulative decay since window start
@@ -32,20 +33,21 @@ constexpr int kStatusTimeout = 2;
 struct Layout {
     int dk, dv, P, r, W, kda;
     int tok_bf16;   // buffered tokens stored in BF16
+    int bits;       // code width: 8, 6 or 4 (6 and 4 bit-packed, no BF16 rows)
     int off_m, off_s, off_hp, off_codes, off_ent, off_tok, off_gam;
     int rec_bytes;
 };
 
 __host__ __device__ inline int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-__host__ inline Layout make_layout(int dk, int dv, int P, int r, int W, int kda, int tok_bf16 = 0) {
+__host__ inline Layout make_layout(int dk, int dv, int P, int r, int W, int kda, int tok_bf16 = 0, int bits = 8) {
     Layout L;
-    L.dk = dk; L.dv = dv; L.P = P; L.r = r; L.W = W; L.kda = kda; L.tok_bf16 = tok_bf16;
+    L.dk = dk; L.dv = dv; L.P = P; L.r = r; L.W = W; L.kda = kda; L.tok_bf16 = tok_bf16; L.bits = bits;
     L.off_m = 0;
     L.off_s = dk * 4;
     L.off_hp = (dk + dv) * 4;
     L.off_codes = L.off_hp + P * dv * 2;
-    L.off_ent = align_up(L.off_codes + (dk - P) * dv, 16);
+    L.off_ent = align_up(L.off_codes + (dk - P) * dv * bits / 8, 16);
     L.off_tok = L.off_ent + r * (dk + dv) * 4;
     int o = L.off_tok + W * (dk + dv) * (tok_bf16 ? 2 : 4);
     L.off_gam = align_up(o, 16);
@@ -60,10 +62,73 @@ __host__ inline Layout make_layout(int dk, int dv, int P, int r, int W, int kda,
 // by the column so that 8 consecutive columns read with ldmatrix hit 8
 // different shared-memory bank groups.  With BF16 rows the codes stay
 // row-major by INT8 slot: [slot][c].
-__host__ __device__ __forceinline__ int code_swz(int c, int dk) { return dk >= 128 ? (c & 7) : ((c >> 1) & 3); }
+// Chunk swizzle of a column-major plane whose columns are `row_bytes` (16 ..
+// 128) long: the 16-byte chunk index is XORed with bits of the column so that
+// the same chunk of 8 consecutive columns covers all 8 bank groups of 128 bytes.
+__host__ __device__ __forceinline__ int chunk_swz(int c, int row_bytes) {
+    return row_bytes >= 128 ? (c & 7) : row_bytes == 64 ? ((c >> 1) & 3) : row_bytes == 32 ? ((c >> 2) & 1) : 0;
+}
+
+__host__ __device__ __forceinline__ int code_swz(int c, int dk) { return chunk_swz(c, dk); }
 
 __host__ __device__ __forceinline__ int code_off_t(int c, int i, int dk) {
     return c * dk + ((((i >> 4) ^ code_swz(c, dk)) << 4) | (i & 15));
+}
+
+// 4- and 6-bit codes (no BF16 rows), value-column-major and swizzled like the
+// INT8 codes, in groups of 8 key rows g = i / 8:
+//   nibble plane [dv][dk/2]: the low 4 bits of each code; a group is one
+//     32-bit word (row 8g+k in bits 4k .. 4k+3) at byte nib_off(c, g);
+//   pair plane [dv][dk/4] (6-bit only, after the nibble plane): bits 4-5 of
+//     each code; a group is one 16-bit word (row 8g+k in bits 2k, 2k+1) at
+//     byte pair_off(c, g).  Groups g and g+4 of a 64-row block share a 32-bit
+//     word, so that one shared-memory matrix load hands a lane the pair bits
+//     of both 32-row halves it multiplies.
+__host__ __device__ __forceinline__ int nib_off(int c, int g, int dk) {
+    const int rb = dk / 2, b = 4 * g;
+    return c * rb + ((((b >> 4) ^ chunk_swz(c, rb)) << 4) | (b & 15));
+}
+
+__host__ __device__ __forceinline__ int pair_off(int c, int g, int dk, int dv) {
+    const int rb = dk / 4, b = 16 * (g >> 3) + 4 * (g & 3) + 2 * ((g >> 2) & 1);
+    return dv * (dk / 2) + c * rb + ((((b >> 4) ^ chunk_swz(c, rb)) << 4) | (b & 15));
+}
+
+// Position of key row i in the contraction order of the packed tensor-core
+// GEMV: a lane's nibble word of 32-row block i / 32 holds rows 8tq .. 8tq+7,
+// whose even rows fill MMA k-slots 4tq .. 4tq+3 and odd rows 16+4tq .. 16+4tq+3.
+__host__ __device__ __forceinline__ int lowbit_kslot(int i) {
+    return (i & ~31) | ((i & 1) << 4) | (((i >> 3) & 3) << 2) | ((i >> 1) & 3);
+}
+
+// An 8-row group as signed bytes c * 2^(8 - BITS) (exact: the code sits in the
+// byte's top BITS bits): lo = rows 0, 2, 4, 6, hi = rows 1, 3, 5, 7 (byte j =
+// row 2j resp. 2j+1).  `pairs` is the group's 16-bit pair word spread as bytes
+// [p0, p0, p1, p1] (spread_pairs).
+__device__ __forceinline__ uint32_t spread_pairs(uint32_t w32, bool high_half) {
+    return __byte_perm(w32, 0u, high_half ? 0x3322u : 0x1100u);
+}
+
+template <int BITS>
+__device__ __forceinline__ void unpack_group(uint32_t nib, uint32_t pairs, uint32_t &lo, uint32_t &hi) {
+    static_assert(BITS == 4 || BITS == 6, "packed widths");
+    if (BITS == 4) {
+        lo = (nib << 4) & 0xF0F0F0F0u;
+        hi = nib & 0xF0F0F0F0u;
+    } else {
+        lo = ((nib << 2) & 0x3C3C3C3Cu) | ((pairs << 6) & 0x00C000C0u) | ((pairs << 2) & 0xC000C000u);
+        hi = ((nib >> 2) & 0x3C3C3C3Cu) | ((pairs << 4) & 0x00C000C0u) | (pairs & 0xC000C000u);
+    }
+}
+
+// Code of key row i, column c in a packed plane set (any width; 8 = code_off_t).
+__device__ __forceinline__ int packed_code(const unsigned char *codes, int c, int i, int dk, int dv, int bits) {
+    if (bits == 8) return (int)(int8_t)codes[code_off_t(c, i, dk)];
+    const int g = i >> 3, k = i & 7;
+    const uint32_t nib = (codes[nib_off(c, g, dk) + (k >> 1)] >> (4 * (k & 1))) & 15u;
+    if (bits == 4) return ((int)(nib << 28)) >> 28;
+    const uint32_t pr = (*reinterpret_cast<const uint16_t *>(codes + pair_off(c, g, dk, dv)) >> (2 * k)) & 3u;
+    return ((int)((nib | (pr << 4)) << 26)) >> 26;
 }
 
 // Named barrier over the NT compute threads (warps 0 .. NT/32-1) of a CTA;

@@ -35,7 +35,8 @@ struct Fp32Args {
 // record layout and the plain lq_qstate_view arrays.
 struct QPtrs {
     unsigned char *codes; size_t codes_hs;
-    int codes_t;                                    // 1: column-major swizzled (record, no BF16 rows)
+    int codes_t;                                    // 1: column-major swizzled (record, no BF16 rows;
+                                                    //    4 / 6-bit codes packed, CodecArgs::bits)
     unsigned char *hp;    size_t hp_hs;
     unsigned char *m;     size_t m_hs;
     unsigned char *s;     size_t s_hs;
@@ -46,6 +47,7 @@ struct QPtrs {
 
 struct CodecArgs {
     int H, r, K, smoothing, P;
+    int bits;             // code width: 8, 6 or 4 (the quantizer's qmax; packing of codes_t stores)
     const int *hp_rows;   // [H][P] (device), may be null when P == 0
     const float *S_in;    // [heads][dk][dv]
     float *S_out;         // [heads][dk][dv]
@@ -60,6 +62,21 @@ struct CodecArgs {
 };
 
 size_t decode_smem_bytes(int dk, int dv, const Layout &L);
+size_t buffer_smem_bytes_of(int dk, int dv, const Layout &L);
+size_t flush_smem_bytes_of(int dk, int dv, const Layout &L);
+// Per code width (L.bits): launch_decode / launch_flush dispatch to these.
+cudaError_t launch_decode_b8(const DecodeArgs &a, int dk, int dv, int heads, bool kda, bool flush, bool damp,
+                             cudaStream_t s);
+cudaError_t launch_decode_b6(const DecodeArgs &a, int dk, int dv, int heads, bool kda, bool flush, bool damp,
+                             cudaStream_t s);
+cudaError_t launch_decode_b4(const DecodeArgs &a, int dk, int dv, int heads, bool kda, bool flush, bool damp,
+                             cudaStream_t s);
+cudaError_t launch_flush_b8(const DecodeArgs &a, int dk, int dv, int heads, bool kda, bool damp, bool exp,
+                            cudaStream_t s);
+cudaError_t launch_flush_b6(const DecodeArgs &a, int dk, int dv, int heads, bool kda, bool damp, bool exp,
+                            cudaStream_t s);
+cudaError_t launch_flush_b4(const DecodeArgs &a, int dk, int dv, int heads, bool kda, bool damp, bool exp,
+                            cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int dk, int dv, int heads, bool kda, bool flush, bool damp,
                           cudaStream_t s);
 cudaError_t launch_flush(const DecodeArgs &a, int dk, int dv, int heads, bool kda, bool damp, bool exp,

@@ -45,7 +45,7 @@ class LqError(RuntimeError):
 class lq_config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in ("B", "H", "Hk", "dk", "dv", "gate", "mode", "W", "r",
                                           "power_iters", "n_hp_rows", "smoothing", "fused_flush",
-                                          "buffer_bf16")]
+                                          "buffer_bf16", "state_bits")]
 
 
 class lq_qstate_view(C.Structure):
@@ -119,13 +119,14 @@ class Config:
     smoothing: int = 1
     fused_flush: int = 1
     buffer_bf16: int = 0         # 1: buffered token updates kept in BF16 (window mode)
+    state_bits: int = 8          # code width of the quantized state: 8, 6 or 4 (bit-packed)
 
     def c(self) -> lq_config:
         gate = {"gdn": LQ_GATE_SCALAR, "kda": LQ_GATE_CHANNEL}[self.gate]
         mode = {"fp32": LQ_MODE_FP32, "step": LQ_MODE_INT8_STEP, "window": LQ_MODE_INT8_WINDOW}[self.mode]
         return lq_config(self.B, self.H, self.Hk, self.dk, self.dv, gate, mode, self.W, self.r,
                          self.power_iters, self.n_hp_rows, self.smoothing, self.fused_flush,
-                         self.buffer_bf16)
+                         self.buffer_bf16, self.state_bits)
 
     @property
     def heads(self) -> int:
@@ -140,7 +141,8 @@ class Config:
         base = dict(B=wl.B, H=wl.H, Hk=wl.Hk, dk=wl.dk, dv=wl.dv, gate=wl.gate, mode=mode,
                     W=(1 if mode == "step" else wl.W), r=wl.r, power_iters=wl.K,
                     n_hp_rows=(wl.P if mode != "fp32" else 0), smoothing=wl.smoothing,
-                    buffer_bf16=(wl.buffer_bf16 if mode == "window" else 0))
+                    buffer_bf16=(wl.buffer_bf16 if mode == "window" else 0),
+                    state_bits=(wl.bits if mode != "fp32" else 8))
         base.update(kw)
         return Config(**base)
 

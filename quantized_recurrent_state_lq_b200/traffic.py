@@ -4,7 +4,8 @@ what a kernel happens to move -- used for the roofline figures.
 Per head and token of a window (n tokens already buffered, 0 <= n < W):
   IO      q, k read once per q/k head (shared by H/Hk value heads), v and o,
           beta, the gate (1 or dk floats)
-  state   INT8 codes (dk-P)*dv, BF16 rows 2*P*dv, m and s (dk+dv)*4,
+  state   codes (dk-P)*dv*bits/8 (INT8, or packed 6 / 4 bits), BF16 rows 2*P*dv,
+          m and s (dk+dv)*4,
           r compensators r*(dk+dv)*4, the n buffered entries n*(dk+dv)*4
           (n*(dk+dv)*2 with the BF16 buffer)
   append  one entry (dk+dv)*4 (or *2) and Gamma written (read too when n > 0)
@@ -24,7 +25,8 @@ def io_bytes(wl: Workload) -> float:
 
 def state_bytes(wl: Workload, P: int | None = None) -> int:
     P = wl.P if P is None else P
-    return (wl.dk - P) * wl.dv + 2 * P * wl.dv + 4 * (wl.dk + wl.dv) + 4 * wl.r * (wl.dk + wl.dv)
+    return ((wl.dk - P) * wl.dv * wl.bits // 8 + 2 * P * wl.dv + 4 * (wl.dk + wl.dv)
+            + 4 * wl.r * (wl.dk + wl.dv))
 
 
 def gamma_bytes(wl: Workload, n: int) -> int:
@@ -72,9 +74,9 @@ def bits_per_value(wl: Workload) -> dict:
     """Effective bits per state value of the window-start state (the DAMP
     abstract reports its state-storage saving; it gives no definition, so both
     readings are reported): `payload` counts the codes and the BF16 rows only,
-    (8 (dk-P) + 16 P) / dk; `total` adds the FP32 smoothing and column scales
+    (bits (dk-P) + 16 P) / dk; `total` adds the FP32 smoothing and column scales
     and the r compensators, 32 (dk + dv) (1 + r) / (dk dv).  The transient
     window buffer is excluded (it is the method's FP32 update stream)."""
-    payload = (8 * (wl.dk - wl.P) + 16 * wl.P) / wl.dk
+    payload = (wl.bits * (wl.dk - wl.P) + 16 * wl.P) / wl.dk
     total = payload + 32 * (wl.dk + wl.dv) * (1 + wl.r) / (wl.dk * wl.dv)
     return {"payload": payload, "total": total, "fp32_reference": 32.0}

@@ -25,7 +25,8 @@ def require_gpu():
 def ocfg(cfg: lq.Config, quantize: int = 1) -> O.Cfg:
     return O.Cfg(dk=cfg.dk, dv=cfg.dv, gate=cfg.gate, W=cfg.W, r=cfg.r, K=cfg.power_iters,
                  smoothing=cfg.smoothing, P=cfg.n_hp_rows, quantize=quantize,
-                 bf16_buffer=cfg.buffer_bf16 if (quantize and cfg.mode == "window") else 0)
+                 bf16_buffer=cfg.buffer_bf16 if (quantize and cfg.mode == "window") else 0,
+                 bits=cfg.state_bits if quantize else 8)
 
 
 def head_rows(cfg: lq.Config, hp_rows):

@@ -195,3 +195,47 @@ def test_bf16_buffer_traffic_model():
     n = 10
     d = traffic.decode_launch_bytes(wl, n) - traffic.decode_launch_bytes(lean, n)
     assert d == (n + 1) * 2 * (wl.dk + wl.dv)     # n entries read + one appended
+
+
+def test_state_bits_config(L):
+    base = lq.Config.from_workload(configs.GDN_PREFIX_CACHE)
+    full = lq.lq_workspace_bytes(base)
+    wl = configs.GDN_PREFIX_CACHE
+    for bits, code_bytes in ((8, 1.0), (6, 0.75), (4, 0.5)):
+        for mode in ("window", "step"):
+            c = lq.Config.from_workload(wl.with_(bits=bits), mode=mode)
+            assert c.state_bits == bits
+            assert lq.lq_config_check(c) == lq.LQ_OK
+        c = lq.Config.from_workload(wl.with_(bits=bits))
+        # the codes shrink to bits / 8 bytes each; nothing else changes (records
+        # are 128-byte aligned)
+        saved = wl.heads * wl.dk * wl.dv * (1 - code_bytes)
+        assert full - lq.lq_workspace_bytes(c) == pytest.approx(saved, abs=wl.heads * 128)
+    zero = lq.Config.from_workload(wl)
+    zero.state_bits = 0                                   # reads as 8
+    assert lq.lq_config_check(zero) == lq.LQ_OK and lq.lq_workspace_bytes(zero) == full
+    for bad in (1, 2, 3, 5, 7, 9, 16, -4):
+        c = lq.Config.from_workload(wl)
+        c.state_bits = bad
+        assert lq.lq_config_check(c) == lq.LQ_ERR_INVALID_ARG
+    f = lq.Config.from_workload(wl, mode="fp32")
+    f.state_bits = 4
+    assert lq.lq_config_check(f) == lq.LQ_ERR_INVALID_ARG
+
+
+def test_packed_codes_with_bf16_rows_are_not_built(L):
+    cfg = lq.Config.from_workload(configs.GDN_DAMP)       # P = 16 BF16 rows
+    for bits in (6, 4):
+        cfg.state_bits = bits
+        assert lq.lq_config_check(cfg) == lq.LQ_ERR_UNSUPPORTED
+
+
+def test_low_bit_traffic_and_bits_per_value():
+    from quantized_recurrent_state_lq_b200 import traffic
+    wl = configs.GDN_PREFIX_CACHE                          # d = 128, r = 4
+    for bits in (6, 4):
+        lb = wl.with_(bits=bits)
+        assert traffic.state_bytes(wl) - traffic.state_bytes(lb) == wl.dk * wl.dv * (8 - bits) // 8
+        b = traffic.bits_per_value(lb)
+        assert b["payload"] == pytest.approx(bits)
+        assert b["total"] == pytest.approx(bits + 2.5)     # 32 * 256 * 5 / 16384

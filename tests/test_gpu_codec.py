@@ -101,6 +101,82 @@ def test_dequantize_matches_oracle(B, H, dk, dv, r, K, smoothing, P):
     assert err.max() < 1e-6, err.max()
 
 
+@pytest.mark.parametrize("bits", [4, 6])
+@pytest.mark.parametrize("B,H,dk,dv,r,K,smoothing", [
+    (2, 3, 128, 128, 4, 8, 1), (1, 5, 64, 64, 2, 8, 1), (2, 2, 64, 128, 2, 8, 1), (2, 2, 128, 64, 3, 8, 1),
+    (2, 3, 128, 128, 0, 8, 0),
+])
+def test_quantize_low_bit_matches_oracle(bits, B, H, dk, dv, r, K, smoothing):
+    """6- and 4-bit codes (qmax 31, 7) against the oracle's quantizer, and the
+    workspace's bit-packed copy of them: lq_state_init packs what
+    lq_quantize_state writes one per byte, lq_state_export_view unpacks it,
+    lq_state_export_fp32 dequantizes the packed planes."""
+    U.require_gpu()
+    qmax = (1 << (bits - 1)) - 1
+    cfg = lq.Config(B=B, H=H, Hk=H, dk=dk, dv=dv, W=4, r=r, power_iters=K, smoothing=smoothing, state_bits=bits)
+    S = gen.random_state(B * H, dk, dv, seed=21 + dk + dv + r + bits).reshape(B, H, dk, dv)
+    view = lq.alloc_view(cfg)
+    lq.lq_quantize_state(cfg, S.cuda(), view)
+    torch.cuda.synchronize()
+    got = U.gpu_view_to_oracle(cfg, view, None)
+    oc = U.ocfg(cfg)
+    Sn = S.numpy().reshape(B * H, dk, dv)
+    flips = total = 0
+    for h in range(B * H):
+        want = O.quantize(oc, Sn[h], want_ratio=True)
+        assert np.abs(want["codes"]).max() == qmax
+        c = U.compare_codes(got["codes"][h], want["codes"], want["ratio"], TIE_EPS)
+        assert c["max_diff"] <= 1, (h, c)
+        flips += c["n"]
+        total += c["total"]
+        np.testing.assert_allclose(got["m"][h], want["m"], rtol=SCALE_REL)
+        np.testing.assert_allclose(got["s"][h], want["s"], rtol=SCALE_REL, atol=1e-30)
+    assert flips <= CODE_FLIP_FRAC * total + 1
+    # packed in the workspace, unpacked on export: the same codes bit for bit
+    st = lq.lq_state_init(cfg, S.cuda())
+    ev = lq.alloc_view(cfg)
+    lq.lq_state_export_view(st, ev)
+    for k in view:
+        assert torch.equal(ev[k], view[k]), k
+    # the packed planes dequantized (export at the window start) equal the
+    # one-per-byte view dequantized
+    a = torch.empty((B, H, dk, dv), device="cuda")
+    b = torch.empty_like(a)
+    lq.lq_state_export_fp32(st, a)
+    lq.lq_dequantize_state(cfg, view, b)
+    torch.testing.assert_close(a, b, rtol=1e-6, atol=1e-6 * b.abs().max().item())
+
+
+@pytest.mark.parametrize("bits", [4, 6])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64)])
+def test_packed_import_export_every_code(bits, dk, dv):
+    """Every code value of the width at every position survives import (pack)
+    and export (unpack); codes beyond +-qmax are saturated on import."""
+    U.require_gpu()
+    qmax = (1 << (bits - 1)) - 1
+    cfg = lq.Config(B=2, H=2, Hk=2, dk=dk, dv=dv, W=4, r=1, state_bits=bits)
+    S0 = gen.random_state(4, dk, dv, seed=2).reshape(2, 2, dk, dv).cuda()
+    st = lq.lq_state_init(cfg, S0)
+    v = lq.alloc_view(cfg)
+    lq.lq_state_export_view(st, v)
+    g = torch.Generator().manual_seed(bits * 1000 + dk + dv)
+    codes = torch.randint(-qmax, qmax + 1, tuple(v["codes"].shape), generator=g, dtype=torch.int8)
+    flat = codes.view(-1)
+    flat[: 2 * qmax + 1] = torch.arange(-qmax, qmax + 1, dtype=torch.int8)
+    v["codes"].copy_(codes)
+    lq.lq_state_import_view(st, v)
+    back = lq.alloc_view(cfg)
+    lq.lq_state_export_view(st, back)
+    assert torch.equal(back["codes"].cpu(), codes)
+    wide = codes.clone()
+    wide.view(-1)[:4] = torch.tensor([127, -127, qmax + 1, -qmax - 1], dtype=torch.int8)
+    v["codes"].copy_(wide)
+    lq.lq_state_import_view(st, v)
+    lq.lq_state_export_view(st, back)
+    want = wide.clamp(-qmax, qmax)
+    assert torch.equal(back["codes"].cpu(), want)
+
+
 def test_view_export_import_roundtrip():
     U.require_gpu()
     cfg = lq.Config(B=2, H=3, Hk=3, dk=128, dv=128, W=4, r=2, n_hp_rows=8)

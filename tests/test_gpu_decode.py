@@ -17,9 +17,10 @@ STATE_REL = 1e-3   # FP32 state: max relative error per head
 TIE_EPS = 1e-3     # a flip this close to a rounding tie is counted as "at a tie"
 
 
-def _workload(gate, B, H, Hk, dk, dv, W, r, seed, P=0, bf16=0):
+def _workload(gate, B, H, Hk, dk, dv, W, r, seed, P=0, bf16=0, bits=8):
     return configs.TINY_GDN.with_(gate=gate, B=B, H=H, Hk=Hk, dk=dk, dv=dv, W=W, r=r, seed=seed, P=P,
-                                  n_out_rows=3, n_out_cols=3, out_lo=10.0, out_hi=50.0, buffer_bf16=bf16)
+                                  n_out_rows=3, n_out_cols=3, out_lo=10.0, out_hi=50.0, buffer_bf16=bf16,
+                                  bits=bits)
 
 
 def _rows_for(wl):
@@ -165,6 +166,33 @@ def test_windowed_bf16_buffer_teacher_forced(fused, gate, B, H, Hk, dk, dv, W, r
     wl = _workload(gate, B, H, Hk, dk, dv, W, r, seed=61 + W, bf16=1)
     T = 2 * W + W // 2 + 1
     _teacher_forced(wl, T, fused, label=f"bf16 buffer {gate} d{dk}x{dv} W{W} r{r} fused{int(fused)}")
+
+
+@pytest.mark.parametrize("bits", [4, 6])
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("gate,B,H,Hk,dk,dv,W,r,bf16", [
+    ("gdn", 2, 4, 2, 128, 128, 8, 4, 0),    # GQA, d = 128: two packed k-pairs per column
+    ("kda", 2, 3, 3, 128, 128, 32, 4, 0),
+    ("gdn", 1, 2, 2, 64, 64, 16, 2, 0),     # d = 64: one k-pair, a single pair-plane chunk
+    ("kda", 1, 3, 3, 64, 128, 5, 2, 0),     # odd window
+    ("gdn", 2, 2, 2, 128, 64, 6, 3, 0),
+    ("gdn", 2, 2, 2, 128, 128, 16, 4, 1),   # with the BF16 window buffer
+])
+def test_windowed_low_bit_teacher_forced(bits, fused, gate, B, H, Hk, dk, dv, W, r, bf16):
+    """6- and 4-bit states (codes in +-31 / +-7, bit-packed in the workspace):
+    the same teacher-forced bars as INT8 -- outputs and pre-flush state within
+    1e-3 of the oracle's low-bit mode, codes exact but for rounding ties."""
+    U.require_gpu()
+    wl = _workload(gate, B, H, Hk, dk, dv, W, r, seed=71 + W + bits, bf16=bf16, bits=bits)
+    T = 2 * W + W // 2 + 1
+    _teacher_forced(wl, T, fused, label=f"{bits}-bit {gate} d{dk}x{dv} W{W} r{r} bf16{bf16} fused{int(fused)}")
+
+
+@pytest.mark.parametrize("bits", [4, 6])
+def test_per_step_low_bit_mode(bits):
+    U.require_gpu()
+    wl = _workload("gdn", 2, 2, 2, 128, 128, 1, 4, seed=45 + bits, bits=bits)
+    _teacher_forced(wl, 10, True, mode="step", label=f"per-step {bits}-bit")
 
 
 def test_damp_rows_teacher_forced():

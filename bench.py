@@ -172,20 +172,32 @@ def run_reference(args, wl, world, rank, pg):
 
 # ---------------------------------------------------------------- GPU leg
 
+def kernel_sources_sha(names) -> str:
+    """sha256 prefix of the listed csrc files (in the order given): the
+    sources the profiled kernel is built from."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "quantized_recurrent_state_lq_b200", "csrc")
+    try:
+        for f in names:
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    except OSError:
+        return "missing"
+    return h.hexdigest()[:16] if names else "none"
+
+
 def profile_traffic(wl):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, if it was taken on the current kernel sources; else None."""
-    import hashlib
+    summary, if it was taken on the current sources of that kernel (the files
+    listed under `sources:`); else None."""
     path = os.path.join(ROOT, "profiles", "decode_window_traffic.txt")
     try:
         kv = dict(line.split(":", 1) for line in open(path) if ":" in line)
     except OSError:
         return None
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "quantized_recurrent_state_lq_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        h.update(open(os.path.join(csrc, f), "rb").read())
-    if kv.get("csrc_sha256", "").strip() != h.hexdigest()[:16] or kv.get("workload", "").strip() != wl.name:
+    if kv.get("sources_sha256", "").strip() != kernel_sources_sha(kv.get("sources", "").split()):
+        return None
+    if kv.get("workload", "").strip() != wl.name:
         return None
     if wl.bits != 8 or wl.buffer_bf16:   # the capture is of the INT8 state with the FP32 buffer
         return None

@@ -300,6 +300,63 @@ def variant(wv, S0, stream, peak_gbs: float, note: str, windows: int = 3) -> dic
             "state_bits_per_value": traffic.bits_per_value(wv), "note": note}
 
 
+# FP32 arithmetic peak of the B200 used for ALU-bound kernels: 148 SMs x 128
+# FP32 lanes x 2 flops per FMA x the 1965 MHz maximum SM clock.
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def prefill_line(wl, stream, chunks: int = 32, tokens: int = 64) -> dict:
+    """The chunked prefill (lq_prefill) of the workload's heads: `chunks`
+    calls of `tokens` tokens each from one seeded draw of `tokens` tokens
+    (the kernel's work does not depend on the values), the state carried in
+    place; beside it the token-by-token FP32-state kernel on one call's worth
+    of tokens.  CUDA events on the launching stream."""
+    cfg = lq.Config(B=wl.B, H=wl.H, Hk=wl.Hk, dk=wl.dk, dv=wl.dv, gate=wl.gate, mode="fp32", r=0)
+    tok = gen.token_inputs(wl, tokens, stream="prefill", device="cuda")
+    S = torch.zeros((wl.B, wl.H, wl.dk, wl.dv), device="cuda")
+    run = lambda: lq.lq_prefill(cfg, tok["q"], tok["k"], tok["v"], tok["beta"], tok["alpha"], S0=S, S_out=S)
+    for _ in range(2):
+        run()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(chunks):
+        run()
+    ev1.record(stream)
+    ev1.synchronize()
+    dt = ev0.elapsed_time(ev1) / 1e3
+    T = chunks * tokens
+    if not bool(torch.isfinite(S).all()):
+        raise lq.LqError(lq.LQ_ERR_NONFINITE, "prefill")
+    # the recurrent FP32-state kernel on `tokens` tokens
+    st = lq.lq_state_init(cfg, S)
+    o = torch.empty((wl.B, wl.H, wl.dv), device="cuda")
+    step = lambda t: lq.lq_decode_step(st, tok["q"][t], tok["k"][t], tok["v"][t], tok["beta"][t],
+                                       tok["alpha"][t], o)
+    for t in range(4):
+        step(t)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for t in range(tokens):
+        step(t)
+    ev1.record(stream)
+    ev1.synchronize()
+    dtr = ev0.elapsed_time(ev1) / 1e3 * (T / tokens)
+    lq.lq_state_destroy(st)
+    flops = traffic.prefill_flops(wl, T) * wl.heads
+    achieved = flops / dt / 1e12
+    del tok, S
+    torch.cuda.empty_cache()
+    return {"tokens": T, "heads": wl.heads, "chunk": traffic.PREFILL_CHUNK, "seconds": dt,
+            "value": wl.heads * T / dt, "unit": "state updates/s",
+            "recurrent_fp32_seconds": dtr, "speedup_vs_recurrent": dtr / dt,
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                         "frac": achieved / FP32_PEAK_TFLOPS, "traffic": None,
+                         "kernel": "prefill_kernel (chunked WY form, FP32 FMA)",
+                         "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"},
+            "note": f"{chunks} calls of one {tokens}-token draw; recurrent time from {tokens} tokens x {T // tokens}"}
+
+
 def state_dtype(wl) -> str:
     return "int8" if wl.bits == 8 else f"int{wl.bits} (bit-packed)"
 
@@ -374,6 +431,9 @@ def run_ours(args, wl, world, rank, pg):
             f"int{b}": variant(wl.with_(bits=b), S0, stream, peaks["hbm_gbs"],
                                f"{b}-bit window-start state (codes in +-{(1 << (b - 1)) - 1}, bit-packed)")
             for b in (6, 4)}
+
+    if not args.no_modes:
+        line["prefill_per_gpu"] = prefill_line(wl, stream)
 
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(wl)

@@ -209,6 +209,32 @@ int lq_quantize_state_static(const lq_config *cfg, const float *d_S, const int32
                              lq_qstate_view *out, void *stream);
 
 /*
+ * Chunked prefill, the step before the windowed decode: T tokens of the
+ * recurrence S_t = (I - b k k^T) D_t S_{t-1} + b k v^T, o_t = S_t^T q_t (the
+ * rule lq_decode_step follows in FP32 mode; LinQuant appendix Table 3,
+ * key-rows form) for all B*H heads, from d_S0 (FP32 [B,H,dk,dv]; NULL = the
+ * zero state) to d_S_out [B,H,dk,dv] (may equal d_S0).  Chunks of
+ * LQ_PREFILL_CHUNK tokens in WY form: the chunk's rank-one updates become
+ * pseudo-values u by forward substitution, with every decay factor
+ * 2^(g_t - g_i), i <= t, from cumulative log2 decays (at most 1 for gates in
+ * (0, 1]; gates are floored at 2^-150).  FP32 arithmetic.
+ *   inputs, token-major stacks of decode-step inputs: q, k [T,B,Hk,dk],
+ *     v [T,B,H,dv], beta [T,B,H], alpha [T,B,H] (GDN) or [T,B,H,dk] (KDA)
+ *   d_o [T,B,H,dv] receives every token's output (NULL: not written)
+ * cfg supplies B, H, Hk, dk, dv and gate (mode and codec fields unused).
+ * T = 0 writes S0 (or zeros) to d_S_out.  To decode from the result with a
+ * quantized state, pass d_S_out to lq_state_init, which quantizes it
+ * (compensators, smoothing, codes).  Device pointers, caller-owned;
+ * asynchronous on `stream`; LQ_ERR_INVALID_ARG for a NULL input with T > 0,
+ * T < 0 or misaligned (not 4-byte) pointers, LQ_ERR_SHAPE / _UNSUPPORTED as
+ * for lq_config_check.
+ */
+#define LQ_PREFILL_CHUNK 16
+int lq_prefill(const lq_config *cfg, int32_t T, const float *d_q, const float *d_k, const float *d_v,
+               const float *d_beta, const float *d_alpha, const float *d_S0, float *d_S_out, float *d_o,
+               void *stream);
+
+/*
  * DAMP channel risk (offline calibration; DAMP abstract: error energy and
  * decay-based persistence pick the high-risk channels).  For each head h:
  *   E[h,i]  = sum_n sum_c (R - Deq(R))_ic^2 over the n_states FP32 states

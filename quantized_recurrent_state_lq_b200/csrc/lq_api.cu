@@ -8,6 +8,7 @@
 
 #include "../../include/lq_state.h"
 #include "lq_kernels.h"
+#include "lq_prefill.h"
 
 using lq::Layout;
 
@@ -455,6 +456,30 @@ int lq_damp_select(const lq_config *cfg, int32_t n_states, const float *d_states
     a.energy = d_energy;
     a.rows_out = d_rows;
     return cuda_rc(lq::launch_damp_select(a, cfg->dk, cfg->dv, static_cast<cudaStream_t>(stream)));
+}
+
+int lq_prefill(const lq_config *cfg, int32_t T, const float *d_q, const float *d_k, const float *d_v,
+               const float *d_beta, const float *d_alpha, const float *d_S0, float *d_S_out, float *d_o,
+               void *stream) {
+    if (!cfg || !d_S_out || T < 0) return LQ_ERR_INVALID_ARG;
+    if (cfg->B < 1 || cfg->H < 1 || cfg->Hk < 1) return LQ_ERR_SHAPE;
+    if (cfg->Hk > cfg->H || cfg->H % cfg->Hk != 0) return LQ_ERR_SHAPE;
+    if ((long long)cfg->B * cfg->H > (1ll << 31) - 1) return LQ_ERR_SHAPE;
+    if (cfg->gate != LQ_GATE_SCALAR && cfg->gate != LQ_GATE_CHANNEL) return LQ_ERR_INVALID_ARG;
+    if (cfg->dk != 64 && cfg->dk != 128) return LQ_ERR_UNSUPPORTED;
+    if (cfg->dv != 64 && cfg->dv != 128) return LQ_ERR_UNSUPPORTED;
+    if (T > 0 && (!d_q || !d_k || !d_v || !d_beta || !d_alpha)) return LQ_ERR_INVALID_ARG;
+    const uintptr_t al = reinterpret_cast<uintptr_t>(d_q) | reinterpret_cast<uintptr_t>(d_k) |
+                         reinterpret_cast<uintptr_t>(d_v) | reinterpret_cast<uintptr_t>(d_beta) |
+                         reinterpret_cast<uintptr_t>(d_alpha) | reinterpret_cast<uintptr_t>(d_S0) |
+                         reinterpret_cast<uintptr_t>(d_S_out) | reinterpret_cast<uintptr_t>(d_o);
+    if (al & 3) return LQ_ERR_INVALID_ARG;
+    lq::PrefillArgs a{};
+    a.B = cfg->B; a.H = cfg->H; a.Hk = cfg->Hk; a.T = T;
+    a.q = d_q; a.k = d_k; a.v = d_v; a.beta = d_beta; a.alpha = d_alpha;
+    a.S0 = d_S0; a.S_out = d_S_out; a.o = d_o; a.status = nullptr;
+    return cuda_rc(lq::launch_prefill(a, cfg->dk, cfg->dv, cfg->B * cfg->H, cfg->gate == LQ_GATE_CHANNEL,
+                                      static_cast<cudaStream_t>(stream)));
 }
 
 int lq_selftest_division(const float *d_a, const float *d_b, float *d_fast, float *d_pair, float *d_ieee,

@@ -33,7 +33,7 @@ EXPORTED = ["lq_workspace_bytes", "lq_config_check", "lq_state_init", "lq_decode
             "lq_window_flush", "lq_state_buffered", "lq_state_export_fp32",
             "lq_state_export_view", "lq_state_import_view", "lq_quantize_state",
             "lq_dequantize_state", "lq_quantize_state_static", "lq_damp_select", "lq_get_status",
-            "lq_state_destroy", "lq_strerror", "lq_selftest_division"]
+            "lq_state_destroy", "lq_strerror", "lq_selftest_division", "lq_prefill"]
 
 
 class LqError(RuntimeError):
@@ -85,6 +85,7 @@ def lib():
             "lq_state_destroy": (None, [vp]),
             "lq_strerror": (C.c_char_p, [C.c_int]),
             "lq_selftest_division": (C.c_int, [vp, vp, vp, vp, vp, i32, vp]),
+            "lq_prefill": (C.c_int, [cfgp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -289,6 +290,30 @@ def lq_quantize_state_static(cfg: Config, S: torch.Tensor, view: dict, hp_rows=N
     v = _view_struct(cfg, view)
     _chk(lib().lq_quantize_state_static(C.byref(cfg.c()), C.c_void_p(p), p_rows, C.byref(v),
                                         C.c_void_p(_stream(stream))), "lq_quantize_state_static")
+
+
+LQ_PREFILL_CHUNK = 16
+
+
+def lq_prefill(cfg: Config, q, k, v, beta, alpha, S0=None, S_out=None, o=None, stream=None) -> torch.Tensor:
+    """Chunked prefill of T tokens (inputs [T, ...] stacks of decode-step
+    inputs) from S0 (None: zero state) into S_out (allocated when None; may be
+    S0); o [T,B,H,dv] receives the outputs when given.  Returns S_out."""
+    T = q.shape[0]
+    B, H, Hk, dk, dv = cfg.B, cfg.H, cfg.Hk, cfg.dk, cfg.dv
+    shapes = {"q": (T, B, Hk, dk), "k": (T, B, Hk, dk), "v": (T, B, H, dv), "beta": (T, B, H),
+              "alpha": (T, B, H, dk) if cfg.gate == "kda" else (T, B, H)}
+    ptr = {n: _dev(t, n, shapes[n]) for n, t in (("q", q), ("k", k), ("v", v), ("beta", beta), ("alpha", alpha))}
+    if S_out is None:
+        S_out = torch.empty((B, H, dk, dv), device=q.device)
+    p_out = _dev(S_out, "S_out", (B, H, dk, dv))
+    p_s0 = _dev(S0, "S0", (B, H, dk, dv)) if S0 is not None else None
+    p_o = _dev(o, "o", (T, B, H, dv)) if o is not None else None
+    _chk(lib().lq_prefill(C.byref(cfg.c()), C.c_int32(T), C.c_void_p(ptr["q"]), C.c_void_p(ptr["k"]),
+                          C.c_void_p(ptr["v"]), C.c_void_p(ptr["beta"]), C.c_void_p(ptr["alpha"]),
+                          C.c_void_p(p_s0), C.c_void_p(p_out), C.c_void_p(p_o), C.c_void_p(_stream(stream))),
+         "lq_prefill")
+    return S_out
 
 
 def lq_selftest_division(a: torch.Tensor, b: torch.Tensor, stream=None):

@@ -2,7 +2,8 @@
 the DAMP rows, and runs windowed decode steps through the C ABI.
 
 Every numerical step runs in liblq.so kernels: the prefill that produces the
-initial state uses the FP32-state decode kernel, the initial quantization uses
+initial state uses the chunked prefill (lq_prefill; or, on request, the
+FP32-state decode kernel token by token), the initial quantization uses
 lq_state_init, the DAMP choice uses lq_damp_select.  torch provides device
 memory, the seeded input draws (inputs.py), streams and CUDA graphs.
 """
@@ -16,8 +17,11 @@ from .configs import Workload
 
 
 def gpu_prefill(wl: Workload, *, tokens: int | None = None, batch: int | None = None, stream: str = "prefill",
-                chunk: int = 64, device="cuda", capture_heads=None, keep_inputs: bool = False):
-    """FP32-state recurrence from zero over `tokens` generator tokens on the GPU.
+                chunk: int = 64, device="cuda", capture_heads=None, keep_inputs: bool = False,
+                method: str = "chunked"):
+    """FP32 recurrence from zero over `tokens` generator tokens on the GPU:
+    `method` "chunked" runs lq_prefill on each generator chunk, "recurrent"
+    the FP32-state decode kernel one token at a time.
 
     Returns the state [batch, H, dk, dv] (float32, no outliers yet) and, if
     capture_heads lists (b, h) pairs, those heads' inputs on the host in the
@@ -27,25 +31,31 @@ def gpu_prefill(wl: Workload, *, tokens: int | None = None, batch: int | None = 
     B = wl.B if batch is None else batch
     cfg = lq.Config(B=B, H=wl.H, Hk=wl.Hk, dk=wl.dk, dv=wl.dv, gate=wl.gate, mode="fp32", r=0, n_hp_rows=0)
     S0 = torch.zeros((B, wl.H, wl.dk, wl.dv), device=device)
-    st = lq.lq_state_init(cfg, S0)
+    st = lq.lq_state_init(cfg, S0) if method != "chunked" else None
     o = torch.empty((B, wl.H, wl.dv), device=device)
     captured = []
     bsel = None
     if capture_heads:
         bsel = torch.tensor(sorted({b for b, _ in capture_heads}), device=device)
+    S = torch.zeros_like(S0)
     for c in range((T + chunk - 1) // chunk):
         n = min(chunk, T - c * chunk)
         tok = gen.token_inputs(wl, n, stream=stream, chunk=c, batch=B, device=device)
-        for t in range(n):
-            lq.lq_decode_step(st, tok["q"][t], tok["k"][t], tok["v"][t], tok["beta"][t], tok["alpha"][t], o)
+        if method == "chunked":
+            lq.lq_prefill(cfg, tok["q"], tok["k"], tok["v"], tok["beta"], tok["alpha"], S0=S, S_out=S)
+        else:
+            for t in range(n):
+                lq.lq_decode_step(st, tok["q"][t], tok["k"][t], tok["v"][t], tok["beta"][t], tok["alpha"][t], o)
         if bsel is not None:
             captured.append({k: v.index_select(1, bsel).cpu() for k, v in tok.items()})
-    S = torch.empty_like(S0)
-    lq.lq_state_export_fp32(st, S)
-    rc = lq.lq_get_status(st)
-    if rc != lq.LQ_OK:
-        raise lq.LqError(rc, "prefill")
-    lq.lq_state_destroy(st)
+    if st is not None:
+        lq.lq_state_export_fp32(st, S)
+        rc = lq.lq_get_status(st)
+        if rc != lq.LQ_OK:
+            raise lq.LqError(rc, "prefill")
+        lq.lq_state_destroy(st)
+    elif not bool(torch.isfinite(S).all()):
+        raise lq.LqError(lq.LQ_ERR_NONFINITE, "prefill")
     if bsel is None:
         return S, None
     cap = {k: torch.cat([c[k] for c in captured], dim=0) for k in captured[0]}
@@ -58,7 +68,7 @@ def initial_state(wl: Workload, **kw):
 
 
 def damp_rows(wl: Workload, device="cuda") -> torch.Tensor:
-    """Offline DAMP calibration on the GPU: calibration prefills (FP32 kernel),
+    """Offline DAMP calibration on the GPU: calibration prefills (lq_prefill),
     the workload's outliers, then lq_damp_select.  Returns rows [H, P] (host)."""
     n, T = wl.calib_prefills, wl.calib_tokens
     states, _ = gpu_prefill(wl, tokens=T, batch=n, stream="calib", device=device)

@@ -80,3 +80,26 @@ def bits_per_value(wl: Workload) -> dict:
     payload = (wl.bits * (wl.dk - wl.P) + 16 * wl.P) / wl.dk
     total = payload + 32 * (wl.dk + wl.dv) * (1 + wl.r) / (wl.dk * wl.dv)
     return {"payload": payload, "total": total, "fp32_reference": 32.0}
+
+
+PREFILL_CHUNK = 16
+
+
+def prefill_flops(wl: Workload, T: int) -> float:
+    """Floating-point operations per head of the chunked prefill over T tokens
+    (chunks of 16; counted as the kernel evaluates them, an FMA as 2):
+      S^T (Gamma k), S^T (Gamma q), the state update      3 x 2 C dk dv + dk dv
+      decayed keys / queries / update keys                3 C dk (+ 3 C dk exp2 for KDA)
+      pair matrices A, P (i <= t)                         C(C+1)/2 x dk x (4, KDA 6 + 1 exp2)
+      forward substitution, outputs                       C(C-1)/2 dv 2 + C(C+1)/2 dv 2 + 3 C dv
+    exp2 counted as one operation."""
+    C = PREFILL_CHUNK
+    n = (T + C - 1) // C
+    dk, dv = wl.dk, wl.dv
+    kda = wl.gate == "kda"
+    pairs = C * (C + 1) // 2
+    per = (3 * 2 * C * dk * dv + dk * dv
+           + 3 * C * dk * (2 if kda else 1)
+           + pairs * dk * (7 if kda else 4)
+           + (C * (C - 1) // 2) * dv * 2 + pairs * dv * 2 + 3 * C * dv)
+    return float(n * per)

@@ -239,3 +239,33 @@ def test_low_bit_traffic_and_bits_per_value():
         b = traffic.bits_per_value(lb)
         assert b["payload"] == pytest.approx(bits)
         assert b["total"] == pytest.approx(bits + 2.5)     # 32 * 256 * 5 / 16384
+
+
+def test_prefill_argument_checks(L):
+    """lq_prefill validates on the host and launches nothing on error."""
+    cfg = lq.Config(B=2, H=4, Hk=2, dk=128, dv=128, gate="kda", mode="fp32", r=0)
+    p = C.c_void_p(256)
+    args = lambda T=8, q=p, out=p, **kw: (C.byref(kw.get("c", cfg).c()), C.c_int32(T), q, p, p, p, p, None,
+                                          out, None, None)
+    assert L.lq_prefill(*args(T=-1)) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_prefill(*args(out=None)) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_prefill(*args(q=None)) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_prefill(*args(q=C.c_void_p(258))) == lq.LQ_ERR_INVALID_ARG     # not 4-byte aligned
+    for bad, code in ((dict(dk=96), lq.LQ_ERR_UNSUPPORTED), (dict(Hk=3), lq.LQ_ERR_SHAPE),
+                      (dict(B=0), lq.LQ_ERR_SHAPE), (dict(H=2, Hk=4), lq.LQ_ERR_SHAPE)):
+        c2 = lq.Config(**{**cfg.__dict__, **bad})
+        assert L.lq_prefill(*args(c=c2)) == code, bad
+    assert L.lq_prefill(None, C.c_int32(1), p, p, p, p, p, None, p, None, None) == lq.LQ_ERR_INVALID_ARG
+
+
+def test_prefill_flops_model():
+    """Arithmetic of the chunked prefill per head and chunk (the ALU roofline's
+    numerator): the three dk x dv products dominate."""
+    from quantized_recurrent_state_lq_b200 import traffic
+    wl = configs.KDA_B256
+    f = traffic.prefill_flops(wl, 2048)
+    C16 = 16
+    big = 3 * 2 * C16 * wl.dk * wl.dv * (2048 // C16)
+    assert big < f < 1.25 * big
+    g = traffic.prefill_flops(configs.GDN_PREFIX_CACHE, 2048)
+    assert g < f                                  # KDA's per-channel pair decays cost more

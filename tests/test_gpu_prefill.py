@@ -1,0 +1,134 @@
+"""GPU parity of the chunked prefill (lq_prefill) against the oracle's plain
+recurrence on the same seeded inputs: outputs of every token and the final
+state, from zero and from a given state, with ragged last chunks, strong and
+vanishing decays, GQA, and the full-size prefill of the benchmark's KDA
+workload on sampled heads; then the quantized state it hands to the decode."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from quantized_recurrent_state_lq_b200 import configs, inputs as gen, lq, runner
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+OUT_REL = 1e-3     # per output vector (b, h, t), as the decode
+STATE_REL = 1e-3   # per head
+
+
+def _cfg(wl):
+    return lq.Config(B=wl.B, H=wl.H, Hk=wl.Hk, dk=wl.dk, dv=wl.dv, gate=wl.gate, mode="fp32", r=0)
+
+
+def _check(wl, tok, S0, label):
+    cfg = _cfg(wl)
+    T = tok["q"].shape[0]
+    nh = wl.B * wl.H
+    o = torch.full((T, wl.B, wl.H, wl.dv), float("nan"), device="cuda")
+    S = lq.lq_prefill(cfg, tok["q"], tok["k"], tok["v"], tok["beta"], tok["alpha"],
+                      S0=None if S0 is None else S0.cuda(), o=o)
+    torch.cuda.synchronize()
+    oc = O.Cfg(dk=wl.dk, dv=wl.dv, gate=wl.gate, quantize=0, W=max(T, 1))
+    ref = O.run(oc, O.per_head_inputs(tok, wl.H),
+                S0=None if S0 is None else S0.numpy().reshape(nh, wl.dk, wl.dv))
+    if T:
+        eo = U.rel_inf_rows(o.cpu().numpy().reshape(T * nh, wl.dv), ref["o"].reshape(T * nh, wl.dv))
+        assert eo.max() < OUT_REL, f"{label}: outputs {eo.max():.2e}"
+    es = U.rel_inf_rows(S.cpu().numpy().reshape(nh, -1), ref["S"].reshape(nh, -1))
+    assert es.max() < STATE_REL, f"{label}: state {es.max():.2e}"
+    print(f"{label}: out {eo.max() if T else 0:.2e} state {es.max():.2e}")
+    return S
+
+
+@pytest.mark.parametrize("gate,B,H,Hk,dk,dv", [
+    ("gdn", 1, 2, 2, 64, 64), ("gdn", 2, 4, 2, 128, 128), ("kda", 2, 3, 3, 128, 128),
+    ("kda", 1, 3, 3, 64, 128), ("gdn", 2, 2, 2, 128, 64),
+])
+@pytest.mark.parametrize("T", [1, 15, 16, 17, 50])
+def test_prefill_matches_recurrence(gate, B, H, Hk, dk, dv, T):
+    U.require_gpu()
+    wl = configs.TINY_GDN.with_(gate=gate, B=B, H=H, Hk=Hk, dk=dk, dv=dv, seed=5 + T)
+    tok = gen.token_inputs(wl, T, stream="prefill", device="cuda")
+    _check(wl, tok, None, f"prefill {gate} d{dk}x{dv} T{T} from zero")
+    S0 = gen.random_state(B * H, dk, dv, seed=T).reshape(B, H, dk, dv)
+    _check(wl, tok, S0, f"prefill {gate} d{dk}x{dv} T{T} from S0")
+
+
+def test_prefill_long_kda_strong_decay():
+    """KDA over 300 tokens with the benchmark's per-channel decays (mu in
+    U(-6, -1): per-step log decays down to ~-1.3) -- cumulative decays far
+    below FP32's range within a run, never formed as ratios above 1."""
+    U.require_gpu()
+    wl = configs.KDA_B256.with_(B=1, H=4, Hk=4, seed=9)
+    tok = gen.token_inputs(wl, 300, stream="prefill", device="cuda")
+    _check(wl, tok, None, "prefill kda T300")
+
+
+def test_prefill_vanishing_and_unit_gates():
+    """Gates of exactly 0 (state wiped), 1e-30, and 1 (no decay) mid-run."""
+    U.require_gpu()
+    for gate in ("gdn", "kda"):
+        wl = configs.TINY_GDN.with_(gate=gate, B=1, H=2, Hk=2, dk=64, dv=64, seed=3)
+        tok = gen.token_inputs(wl, 40, stream="prefill", device="cuda")
+        a = tok["alpha"]
+        a[5] = 0.0
+        a[6] = 1e-30
+        a[20:24] = 1.0
+        S0 = gen.random_state(2, 64, 64, seed=4).reshape(1, 2, 64, 64)
+        _check(wl, tok, S0, f"prefill {gate} vanishing gates")
+
+
+def test_prefill_zero_tokens_and_in_place():
+    U.require_gpu()
+    wl = configs.TINY_GDN.with_(B=2, H=2, Hk=2, dk=128, dv=128, seed=1)
+    cfg = _cfg(wl)
+    tok = gen.token_inputs(wl, 0, stream="prefill", device="cuda")
+    S0 = gen.random_state(4, 128, 128, seed=2).reshape(2, 2, 128, 128).cuda()
+    out = lq.lq_prefill(cfg, tok["q"], tok["k"], tok["v"], tok["beta"], tok["alpha"], S0=S0)
+    assert torch.equal(out, S0)
+    out = lq.lq_prefill(cfg, tok["q"], tok["k"], tok["v"], tok["beta"], tok["alpha"])
+    assert torch.count_nonzero(out) == 0
+    # in place, in two calls, equals one call over the concatenated tokens
+    tok = gen.token_inputs(wl, 40, stream="prefill", device="cuda")
+    one = lq.lq_prefill(cfg, tok["q"], tok["k"], tok["v"], tok["beta"], tok["alpha"], S0=S0)
+    S = S0.clone()
+    for sl in (slice(0, 23), slice(23, 40)):
+        lq.lq_prefill(cfg, tok["q"][sl], tok["k"][sl], tok["v"][sl], tok["beta"][sl], tok["alpha"][sl],
+                      S0=S, S_out=S)
+    torch.testing.assert_close(S, one, rtol=1e-5, atol=1e-5 * one.abs().max().item())
+
+
+def test_full_size_kda_prefill_sampled_heads():
+    """The benchmark's KDA workload (B=256, H=32, d=128): its 2048-token prefill
+    over all 8192 heads in the runner's launch configuration, 4 sampled heads
+    against the oracle's recurrence; then the quantized state the decode
+    starts from (lq_state_init of the result) against the oracle's quantizer
+    on the oracle's state -- codes within the flush bar (the inputs differ by
+    the prefill's rounding)."""
+    U.require_gpu()
+    wl = configs.KDA_B256
+    heads = [(0, 0), (17, 5), (128, 31), (255, 16)]
+    S, cap = runner.gpu_prefill(wl, capture_heads=heads)
+    bsel = sorted({b for b, _ in heads})
+    nh = len(heads)
+    ph = O.per_head_inputs(cap, wl.H, heads=[(bsel.index(b), h) for b, h in heads])
+    oc = O.Cfg(dk=wl.dk, dv=wl.dv, gate=wl.gate, quantize=0)
+    ref = O.prefill(oc, ph)
+    got = torch.stack([S[b, h] for b, h in heads]).cpu().numpy()
+    es = U.rel_inf_rows(got.reshape(nh, -1), ref.reshape(nh, -1))
+    print(f"full-size KDA prefill: state {es.max():.2e}")
+    assert es.max() < STATE_REL
+    # ends in Q(S): the window-start state of the decode
+    cfg = lq.Config.from_workload(wl.with_(B=1, H=nh, Hk=nh))
+    view = lq.alloc_view(cfg)
+    lq.lq_quantize_state(cfg, torch.from_numpy(got).reshape(1, nh, wl.dk, wl.dv).cuda(), view)
+    gv = U.gpu_view_to_oracle(cfg, view, None)
+    flips = total = 0
+    for i in range(nh):
+        want = O.quantize(U.ocfg(cfg), ref[i].astype(np.float32), want_ratio=True)
+        c = U.compare_codes(gv["codes"][i], want["codes"], want["ratio"], 1e-3)
+        assert c["max_diff"] <= 1
+        flips += c["n"]
+        total += c["total"]
+    assert flips <= U.FLUSH_FLIP_FRAC * total + 1, (flips, total)

@@ -70,6 +70,11 @@ typedef struct {
     int quantize;  /* 0: identity quantizer (FP32-state mode); 1: INT8 */
     int bf16_buffer; /* 1: each token's update is kept in BF16 (see lqo_step_bf16) */
     int bits;      /* code width of the quantized state: 8 (0 reads as 8), 6 or 4 */
+    /* smoothing == 2 (static, fitted offline; see lqo_fit_static): the
+     * head's key-row scales [dk] and value-column scales [dv] (lqo_run: the
+     * arrays of all heads, [nh][dk] and [nh][dv]) */
+    const float *static_m;
+    const float *static_s;
 } lqo_cfg;
 
 /* Largest code magnitude of a b-bit symmetric quantizer. */
@@ -257,10 +262,13 @@ void lqo_quantize(const lqo_cfg *cfg, const int *hp_rows, const float *S,
         for (int c = 0; c < dv; ++c) out->hp[(size_t)p * dv + c] = lqo_bf16_rne(R32[i * dv + c]);
     }
 
-    /* Smoothing: per key row RMS of the residual. */
+    /* Smoothing: per key row RMS of the residual (static scales: the
+     * head's fitted ones). */
     for (int i = 0; i < dk; ++i) {
         float mi = 1.0f;
-        if (cfg->smoothing && !is_hp_row(hp_rows, P, i)) {
+        if (cfg->smoothing == 2) {
+            mi = cfg->static_m[i];
+        } else if (cfg->smoothing && !is_hp_row(hp_rows, P, i)) {
             double ss = 0.0;
             for (int c = 0; c < dv; ++c) ss += (double)R32[i * dv + c] * (double)R32[i * dv + c];
             mi = (float)sqrt(ss / (double)dv);
@@ -279,7 +287,7 @@ void lqo_quantize(const lqo_cfg *cfg, const int *hp_rows, const float *S,
             if (ax > a) a = ax;
         }
         const float qmax = (float)lqo_qmax(cfg);
-        const float sc = a / qmax;
+        const float sc = cfg->smoothing == 2 ? cfg->static_s[c] : a / qmax;
         out->s[c] = sc;
         for (int i = 0; i < dk; ++i) {
             int8_t code = 0;
@@ -365,14 +373,20 @@ void lqo_run(const lqo_cfg *cfg, int nh, const int *hp_rows, int from_view,
     const int dk = cfg->dk, dv = cfg->dv, ga = cfg->gate ? dk : 1;
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
     for (int h = 0; h < nh; ++h) {
+        lqo_cfg hc = *cfg;     /* this head's static scales, if any */
+        if (cfg->smoothing == 2) {
+            hc.static_m = cfg->static_m + (size_t)h * dk;
+            hc.static_s = cfg->static_s + (size_t)h * dv;
+        }
+        const lqo_cfg *hcfg = &hc;
         double *S = S_out + (size_t)h * dk * dv;
         float *F = (float *)malloc(sizeof(float) * dk * dv);
-        const int *hr = hp_rows ? hp_rows + (size_t)h * cfg->P : NULL;
+        const int *hr = hp_rows ? hp_rows + (size_t)h * hcfg->P : NULL;
         lqo_view vh;
-        view_of(cfg, view, h, &vh);
-        if (cfg->quantize) {
-            if (!from_view) lqo_quantize(cfg, hr, S0 + (size_t)h * dk * dv, &vh, NULL);
-            lqo_dequantize(cfg, hr, &vh, S);
+        view_of(hcfg, view, h, &vh);
+        if (hcfg->quantize) {
+            if (!from_view) lqo_quantize(hcfg, hr, S0 + (size_t)h * dk * dv, &vh, NULL);
+            lqo_dequantize(hcfg, hr, &vh, S);
         } else {
             for (int e = 0; e < dk * dv; ++e) S[e] = (double)S0[(size_t)h * dk * dv + e];
         }
@@ -381,21 +395,21 @@ void lqo_run(const lqo_cfg *cfg, int nh, const int *hp_rows, int from_view,
         for (int j = 0; j < ga; ++j) gam[j] = 1.0f;
         for (int t = 0; t < T; ++t) {
             const size_t th = (size_t)t * nh + h;
-            if (cfg->quantize && cfg->bf16_buffer) {
+            if (hcfg->quantize && hcfg->bf16_buffer) {
                 if (n == 0)
                     for (int j = 0; j < ga; ++j) gam[j] = 1.0f;
-                lqo_step_bf16(cfg, S, gam, q + th * dk, k + th * dk, v + th * dv, beta[th],
+                lqo_step_bf16(hcfg, S, gam, q + th * dk, k + th * dk, v + th * dv, beta[th],
                               alpha + th * ga, o + th * dv);
             } else {
-                lqo_step(cfg, S, q + th * dk, k + th * dk, v + th * dv, beta[th],
+                lqo_step(hcfg, S, q + th * dk, k + th * dk, v + th * dv, beta[th],
                          alpha + th * ga, o + th * dv);
             }
             n += 1;
-            if (cfg->quantize && n == cfg->W && (t < T - 1 || flush_last)) {
+            if (hcfg->quantize && n == hcfg->W && (t < T - 1 || flush_last)) {
                 if (S_pre) memcpy(S_pre + (size_t)h * dk * dv, S, sizeof(double) * dk * dv);
                 to_float(S, F, dk * dv);
-                lqo_quantize(cfg, hr, F, &vh, NULL);
-                lqo_dequantize(cfg, hr, &vh, S);
+                lqo_quantize(hcfg, hr, F, &vh, NULL);
+                lqo_dequantize(hcfg, hr, &vh, S);
                 n = 0;
             }
         }
@@ -465,4 +479,146 @@ void lqo_damp_select(int dk, int P, const double *score, int *rows)
     for (int i = 0; i < dk; ++i)
         if (taken[i]) rows[n++] = i;
     free(taken);
+}
+
+/* ------------------------------------------------------------------ */
+/* Static key-row / value-column scales fitted offline [STEP].         */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The STEPQuant article says the scales are fitted jointly, offline, from
+ * state distributions and each key row's impact on the output error, with no
+ * formula.  Reading taken here (the plainest one that fits the quantizer
+ * above):
+ *  - fitted per head on n calibration states, on the residual the quantizer
+ *    sees (after the cfg->r compensators);
+ *  - objective: sum over states, rows, columns of weight_i (R_ic - Deq_ic)^2,
+ *    Deq_ic = (clamp(rne((R_ic / m_i) / s_c)) s_c) m_i as at run time; the
+ *    row weight carries the row's impact (the caller passes e.g. the decay
+ *    persistence 1 / (1 - mean gate), NULL = 1);
+ *  - start: m_i = RMS of row i over all states (1 if 0), s_c = the largest
+ *    |R_ic / m_i| over all states and rows / qmax;
+ *  - LQO_FIT_ROUNDS rounds of coordinate descent, each first over the
+ *    columns then over the rows: s_c takes the best of s_c0 x (1 - j/16),
+ *    j = 0..11, for the current m; then m_i the best of m_i0 x {1/2, 5/8, 3/4,
+ *    7/8, 1, 5/4, 3/2, 7/4, 2} for the current s (ties to the first
+ *    candidate); the current value is always a candidate, so the objective
+ *    never increases.
+ * Errors are accumulated in double, states outer, then rows (column step) or
+ * columns (row step); every float step is the quantizer's.
+ */
+#define LQO_FIT_ROUNDS 3
+#define LQO_FIT_NCOL 12
+#define LQO_FIT_NROW 9
+static const float lqo_fit_rowgrid[LQO_FIT_NROW] = {0.5f, 0.625f, 0.75f, 0.875f, 1.0f, 1.25f, 1.5f, 1.75f, 2.0f};
+
+static double lqo_fit_err(float R, float m, float s, float qmax)
+{
+    float dq = 0.0f;
+    if (s != 0.0f) {
+        const float x = R / m;
+        float rq = rintf(x / s);
+        if (rq > qmax) rq = qmax;
+        if (rq < -qmax) rq = -qmax;
+        dq = (rq * s) * m;
+    }
+    const double d = (double)R - (double)dq;
+    return d * d;
+}
+
+/* Residuals R [n][dk][dv] (float) of n states after the r compensators. */
+static void lqo_residuals(const lqo_cfg *cfg, int n, const float *states, float *R)
+{
+    const int dk = cfg->dk, dv = cfg->dv, r = cfg->r;
+    lqo_cfg c2 = *cfg;
+    c2.P = 0;
+    c2.smoothing = 1;
+    lqo_view v;
+    v.codes = (int8_t *)malloc(dk * dv);
+    v.m = (float *)malloc(sizeof(float) * dk);
+    v.s = (float *)malloc(sizeof(float) * dv);
+    v.c = (float *)malloc(sizeof(float) * (r > 0 ? r : 1) * dk);
+    v.w = (float *)malloc(sizeof(float) * (r > 0 ? r : 1) * dv);
+    v.hp = NULL;
+    double *D = (double *)malloc(sizeof(double) * dk * dv);
+    for (int t = 0; t < n; ++t) {
+        const float *S = states + (size_t)t * dk * dv;
+        lqo_quantize(&c2, NULL, S, &v, NULL);
+        for (int e = 0; e < dk * dv; ++e) D[e] = (double)S[e];
+        for (int j = 0; j < r; ++j)
+            for (int i = 0; i < dk; ++i)
+                for (int c = 0; c < dv; ++c)
+                    D[i * dv + c] -= (double)v.c[j * dk + i] * (double)v.w[j * dv + c];
+        for (int e = 0; e < dk * dv; ++e) R[(size_t)t * dk * dv + e] = (float)D[e];
+    }
+    free(v.codes); free(v.m); free(v.s); free(v.c); free(v.w); free(D);
+}
+
+/* Fit one head: m [dk], s [dv]; obj [LQO_FIT_ROUNDS + 1] (nullable) receives
+ * the objective at the start and after every round. */
+void lqo_fit_static(const lqo_cfg *cfg, int n, const float *states, const double *weight,
+                    float *m, float *s, double *obj)
+{
+    const int dk = cfg->dk, dv = cfg->dv;
+    const float qmax = (float)lqo_qmax(cfg);
+    float *R = (float *)malloc(sizeof(float) * (size_t)n * dk * dv);
+    float *m0 = (float *)malloc(sizeof(float) * dk);
+    float *s0 = (float *)malloc(sizeof(float) * dv);
+    lqo_residuals(cfg, n, states, R);
+#define RES(t, i, c) R[((size_t)(t) * dk + (i)) * dv + (c)]
+    for (int i = 0; i < dk; ++i) {
+        double ss = 0.0;
+        for (int t = 0; t < n; ++t)
+            for (int c = 0; c < dv; ++c) ss += (double)RES(t, i, c) * (double)RES(t, i, c);
+        float mi = (float)sqrt(ss / ((double)n * dv));
+        if (mi == 0.0f) mi = 1.0f;
+        m0[i] = m[i] = mi;
+    }
+    for (int c = 0; c < dv; ++c) {
+        float a = 0.0f;
+        for (int t = 0; t < n; ++t)
+            for (int i = 0; i < dk; ++i) {
+                const float ax = fabsf(RES(t, i, c) / m[i]);
+                if (ax > a) a = ax;
+            }
+        s0[c] = s[c] = a / qmax;
+    }
+    for (int round = 0; round <= LQO_FIT_ROUNDS; ++round) {
+        if (obj) {
+            double e = 0.0;
+            for (int t = 0; t < n; ++t)
+                for (int i = 0; i < dk; ++i)
+                    for (int c = 0; c < dv; ++c)
+                        e += (weight ? weight[i] : 1.0) * lqo_fit_err(RES(t, i, c), m[i], s[c], qmax);
+            obj[round] = e;
+        }
+        if (round == LQO_FIT_ROUNDS) break;
+        for (int c = 0; c < dv; ++c) {
+            double best = INFINITY;
+            float sb = s[c];
+            for (int j = 0; j < LQO_FIT_NCOL; ++j) {
+                const float sc = s0[c] * (1.0f - (float)j / 16.0f);
+                double e = 0.0;
+                for (int t = 0; t < n; ++t)
+                    for (int i = 0; i < dk; ++i)
+                        e += (weight ? weight[i] : 1.0) * lqo_fit_err(RES(t, i, c), m[i], sc, qmax);
+                if (e < best) { best = e; sb = sc; }
+            }
+            s[c] = sb;
+        }
+        for (int i = 0; i < dk; ++i) {
+            double best = INFINITY;
+            float mb = m[i];
+            for (int j = 0; j < LQO_FIT_NROW; ++j) {
+                const float mi = m0[i] * lqo_fit_rowgrid[j];
+                double e = 0.0;
+                for (int t = 0; t < n; ++t)
+                    for (int c = 0; c < dv; ++c) e += lqo_fit_err(RES(t, i, c), mi, s[c], qmax);
+                if (e < best) { best = e; mb = mi; }
+            }
+            m[i] = mb;
+        }
+    }
+#undef RES
+    free(R); free(m0); free(s0);
 }

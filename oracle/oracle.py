@@ -36,7 +36,7 @@ def build(force: bool = False) -> str:
 class _Cfg(C.Structure):
     _fields_ = [(n, C.c_int) for n in
                 ("dk", "dv", "gate", "W", "r", "K", "smoothing", "P", "quantize", "bf16_buffer",
-                 "bits")]
+                 "bits")] + [("static_m", C.c_void_p), ("static_s", C.c_void_p)]
 
 
 class _Views(C.Structure):
@@ -73,11 +73,18 @@ class Cfg:
     quantize: int = 1
     bf16_buffer: int = 0   # 1: buffered updates kept in BF16 (lqo_step_bf16)
     bits: int = 8          # code width of the quantized state: 8, 6 or 4
+    static_m: object = None   # smoothing 2: fitted key-row scales [dk] ([nh, dk] for run)
+    static_s: object = None   # and value-column scales [dv] ([nh, dv] for run)
 
     def c(self) -> _Cfg:
+        sm = ss = None
+        if self.smoothing == 2:
+            self._sm = _f32(self.static_m)
+            self._ss = _f32(self.static_s)
+            sm, ss = self._sm.ctypes.data, self._ss.ctypes.data
         return _Cfg(self.dk, self.dv, 1 if self.gate == "kda" else 0, self.W,
                     self.r, self.K, self.smoothing, self.P, self.quantize, self.bf16_buffer,
-                    self.bits)
+                    self.bits, sm, ss)
 
     @property
     def ga(self) -> int:
@@ -201,6 +208,24 @@ def prefill(cfg: Cfg, inputs: dict, S0=None, nthreads: int | None = None) -> np.
     """Plain FP recurrence from S0 (zeros by default); returns the state, float64."""
     c2 = Cfg(**{**cfg.__dict__, "quantize": 0})
     return run(c2, inputs, S0=S0, nthreads=nthreads)["S"]
+
+
+FIT_ROUNDS = 3
+
+
+def fit_static(cfg: Cfg, states, weight=None) -> dict:
+    """Static key-row / value-column scales of one head fitted on calibration
+    states [n, dk, dv] (lqo_fit_static).  Returns m [dk], s [dv] and the
+    objective after the start and after every round."""
+    st = _f32(states)
+    m = np.zeros(cfg.dk, np.float32)
+    s = np.zeros(cfg.dv, np.float32)
+    obj = np.zeros(FIT_ROUNDS + 1, np.float64)
+    w = None if weight is None else np.ascontiguousarray(np.asarray(weight, np.float64))
+    lib().lqo_fit_static(C.byref(cfg.c()), C.c_int(st.shape[0]), _p(st, C.c_float),
+                         _p(w, C.c_double) if w is not None else None, _p(m, C.c_float),
+                         _p(s, C.c_float), _p(obj, C.c_double))
+    return {"m": m, "s": s, "obj": obj}
 
 
 def damp_energy(cfg: Cfg, states) -> np.ndarray:

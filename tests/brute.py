@@ -118,3 +118,69 @@ def run_windowed(S0, toks, W: int, r: int, K: int, gate: str, smoothing=True, qu
             Sp = dequantize(view).T.copy()
             n = 0
     return np.array(outs), view
+
+
+ROWGRID = [0.5, 0.625, 0.75, 0.875, 1.0, 1.25, 1.5, 1.75, 2.0]
+COLGRID = [1.0 - j / 16.0 for j in range(12)]
+
+
+def _fit_err(R, m, s, qmax):
+    """(R - Deq)^2 in double for one float32 entry under scales m, s."""
+    dq = f32(0)
+    if s != 0:
+        x = f32(R) / f32(m)
+        rq = np.float32(np.rint(f32(x) / f32(s)))
+        rq = f32(min(max(rq, -qmax), qmax))
+        dq = f32(f32(rq * f32(s)) * f32(m))
+    d = float(R) - float(dq)
+    return d * d
+
+
+def fit_static(R, weight, qmax, rounds=3):
+    """Coordinate descent for static scales on residuals R [n, dk, dv]
+    (float32), written out loop by loop: start from the rows' RMS and the
+    columns' amax / qmax; per round the columns (s0 x COLGRID), then the rows
+    (m0 x ROWGRID), first best candidate kept."""
+    n, dk, dv = R.shape
+    w = np.ones(dk) if weight is None else np.asarray(weight, np.float64)
+    m0 = np.zeros(dk, f32)
+    for i in range(dk):
+        ss = 0.0
+        for t in range(n):
+            for c in range(dv):
+                ss += float(R[t, i, c]) * float(R[t, i, c])
+        mi = f32(np.sqrt(ss / (n * dv)))
+        m0[i] = mi if mi != 0 else f32(1)
+    m = m0.copy()
+    s0 = np.zeros(dv, f32)
+    for c in range(dv):
+        a = f32(0)
+        for t in range(n):
+            for i in range(dk):
+                a = max(a, f32(abs(f32(R[t, i, c]) / m[i])))
+        s0[c] = f32(a / f32(qmax))
+    s = s0.copy()
+    for _ in range(rounds):
+        for c in range(dv):
+            best, sb = np.inf, s[c]
+            for g in COLGRID:
+                sc = f32(s0[c] * f32(g))
+                e = 0.0
+                for t in range(n):
+                    for i in range(dk):
+                        e += w[i] * _fit_err(R[t, i, c], m[i], sc, qmax)
+                if e < best:
+                    best, sb = e, sc
+            s[c] = sb
+        for i in range(dk):
+            best, mb = np.inf, m[i]
+            for g in ROWGRID:
+                mi = f32(m0[i] * f32(g))
+                e = 0.0
+                for t in range(n):
+                    for c in range(dv):
+                        e += _fit_err(R[t, i, c], mi, s[c], qmax)
+                if e < best:
+                    best, mb = e, mi
+            m[i] = mb
+    return m, s

@@ -80,7 +80,10 @@ typedef struct {
     int32_t r;              /* compensator tokens per head, 0..min(dk,dv) */
     int32_t power_iters;    /* power-iteration steps per compensator (K), >= 0 */
     int32_t n_hp_rows;      /* P: BF16 key rows per head (DAMP layout), 0 = all INT8 */
-    int32_t smoothing;      /* 1: per-key-row RMS smoothing; 0: none (m = 1) */
+    int32_t smoothing;      /* 1: per-key-row RMS smoothing, column scales from each window's
+                               amax; 0: none (m = 1); 2: fixed key-row and value-column scales
+                               fitted offline (STEPQuant article; lq_fit_static_scales), given
+                               to lq_state_init_static -- INT8 modes, no BF16 rows */
     int32_t fused_flush;    /* 1: the call that buffers the W-th token also flushes */
     int32_t buffer_bf16;    /* 1 (INT8_WINDOW only): keep each buffered token's update in BF16 --
                                bf16(k/Gamma) and bf16(u), formed in FP32, the state carrying the
@@ -136,6 +139,19 @@ int lq_config_check(const lq_config *cfg);
  */
 int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_t bytes,
                   const float *d_S0, const int32_t *h_hp_row_ids, void *stream);
+
+/*
+ * lq_state_init for smoothing = 2: the quantizer keeps the given per-head
+ * scales at every window boundary -- key rows d_static_m [H,dk] (positive,
+ * finite) and value columns d_static_s [H,dv] (>= 0, finite; a zero column
+ * quantizes to 0), e.g. from lq_fit_static_scales -- instead of the window's
+ * row RMS and column amax; codes beyond +-qmax saturate.  The scales are
+ * copied into the workspace (lq_workspace_bytes counts them).  No BF16 rows.
+ * Errors as lq_state_init; LQ_ERR_INVALID_ARG for NULL or misaligned scales
+ * or smoothing != 2 (and lq_state_init with smoothing = 2).
+ */
+int lq_state_init_static(lq_state **out, const lq_config *cfg, void *d_workspace, size_t bytes,
+                         const float *d_S0, const float *d_static_m, const float *d_static_s, void *stream);
 
 /*
  * Decode one token for all B*H heads:  q, k [B,Hk,dk], v [B,H,dv], beta [B,H],
@@ -207,6 +223,25 @@ int lq_dequantize_state(const lq_config *cfg, const lq_qstate_view *in,
 #define LQ_STATIC_ROWS_MAX 8192
 int lq_quantize_state_static(const lq_config *cfg, const float *d_S, const int32_t *h_hp_row_ids,
                              lq_qstate_view *out, void *stream);
+
+/*
+ * Static scales for smoothing = 2 (offline; STEPQuant article: key-row and
+ * value-column scales fitted jointly from the state distribution and each key
+ * row's impact on the output error).  Per head h, on the residuals of the
+ * n_states calibration states d_states [n_states,H,dk,dv] after cfg->r
+ * compensators (K = cfg->power_iters, FP64 extraction), minimise
+ *   sum_states sum_i sum_c w_i (R_ic - (clamp(rne((R_ic/m_i)/s_c)) s_c) m_i)^2
+ * (codes of cfg->state_bits) over d_m [H,dk] and d_s [H,dv], by 3 rounds of
+ * coordinate descent from m_i = RMS of row i over the states (1 if 0), s_c =
+ * max |R_ic / m_i| / qmax: each column takes the best of s_c0 (1 - j/16),
+ * j = 0..11, then each row the best of m_i0 x {1/2, 5/8, 3/4, 7/8, 1, 5/4,
+ * 3/2, 7/4, 2} (first best kept; the objective never increases).  Row weights
+ * d_row_weight [H,dk] (double; NULL = 1) carry each row's impact, e.g. the
+ * persistence 1 / (1 - mean decay).  A stream-ordered temporary of
+ * n_states*H*dk*dv floats holds the residuals.  No BF16 rows.
+ */
+int lq_fit_static_scales(const lq_config *cfg, int32_t n_states, const float *d_states,
+                         const double *d_row_weight, float *d_m, float *d_s, void *stream);
 
 /*
  * Chunked prefill, the step before the windowed decode: T tokens of the

@@ -622,3 +622,20 @@ void lqo_fit_static(const lqo_cfg *cfg, int n, const float *states, const double
 #undef RES
     free(R); free(m0); free(s0);
 }
+
+/* The fit's objective for given scales m [dk], s [dv] on one head's states. */
+double lqo_fit_objective(const lqo_cfg *cfg, int n, const float *states, const double *weight,
+                         const float *m, const float *s)
+{
+    const int dk = cfg->dk, dv = cfg->dv;
+    const float qmax = (float)lqo_qmax(cfg);
+    float *R = (float *)malloc(sizeof(float) * (size_t)n * dk * dv);
+    lqo_residuals(cfg, n, states, R);
+    double e = 0.0;
+    for (int t = 0; t < n; ++t)
+        for (int i = 0; i < dk; ++i)
+            for (int c = 0; c < dv; ++c)
+                e += (weight ? weight[i] : 1.0) * lqo_fit_err(R[((size_t)t * dk + i) * dv + c], m[i], s[c], qmax);
+    free(R);
+    return e;
+}

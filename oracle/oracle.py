@@ -78,7 +78,7 @@ class Cfg:
 
     def c(self) -> _Cfg:
         sm = ss = None
-        if self.smoothing == 2:
+        if self.smoothing == 2 and self.static_m is not None:
             self._sm = _f32(self.static_m)
             self._ss = _f32(self.static_s)
             sm, ss = self._sm.ctypes.data, self._ss.ctypes.data
@@ -226,6 +226,16 @@ def fit_static(cfg: Cfg, states, weight=None) -> dict:
                          _p(w, C.c_double) if w is not None else None, _p(m, C.c_float),
                          _p(s, C.c_float), _p(obj, C.c_double))
     return {"m": m, "s": s, "obj": obj}
+
+
+def fit_objective(cfg: Cfg, states, m, s, weight=None) -> float:
+    """The fit's weighted error of scales m [dk], s [dv] on states [n, dk, dv]."""
+    st = _f32(states)
+    w = None if weight is None else np.ascontiguousarray(np.asarray(weight, np.float64))
+    fn = lib().lqo_fit_objective
+    fn.restype = C.c_double
+    return fn(C.byref(cfg.c()), C.c_int(st.shape[0]), _p(st, C.c_float),
+              _p(w, C.c_double) if w is not None else None, _p(_f32(m), C.c_float), _p(_f32(s), C.c_float))
 
 
 def damp_energy(cfg: Cfg, states) -> np.ndarray:

@@ -20,6 +20,7 @@ struct lq_state {
     int *status;
     int *hp_rows;
     int *slot_rows;
+    float *static_ms;   // smoothing 2: [H][dk+dv] fixed key-row and value-column scales
     unsigned char *rec;
     size_t heads;
     int n;  // tokens buffered in the current window
@@ -52,7 +53,8 @@ int check_codec_fields(const lq_config *c) {
     if (c->r < 0 || c->r > (c->dk < c->dv ? c->dk : c->dv)) return LQ_ERR_INVALID_ARG;
     if (c->power_iters < 0 || c->power_iters > 1000) return LQ_ERR_INVALID_ARG;
     if (c->n_hp_rows < 0 || c->n_hp_rows >= c->dk) return LQ_ERR_INVALID_ARG;
-    if (c->smoothing != 0 && c->smoothing != 1) return LQ_ERR_INVALID_ARG;
+    if (c->smoothing < 0 || c->smoothing > 2) return LQ_ERR_INVALID_ARG;
+    if (c->smoothing == 2 && c->n_hp_rows > 0) return LQ_ERR_UNSUPPORTED;   // static scales: no BF16 rows
     return LQ_OK;
 }
 
@@ -69,6 +71,7 @@ int check_config(const lq_config *c) {
     if (c->buffer_bf16 == 1 && c->mode != LQ_MODE_INT8_WINDOW) return LQ_ERR_INVALID_ARG;
     if (c->buffer_bf16 == 1 && c->n_hp_rows > 0) return LQ_ERR_UNSUPPORTED;   // not built with BF16 rows
     if (c->mode == LQ_MODE_FP32 && c->state_bits != 0 && c->state_bits != 8) return LQ_ERR_INVALID_ARG;
+    if (c->mode == LQ_MODE_FP32 && c->smoothing == 2) return LQ_ERR_INVALID_ARG;
     int rc = check_codec_fields(c);
     if (rc) return rc;
     if (is_int8(c)) {
@@ -86,6 +89,10 @@ size_t hp_bytes(const lq_config *c) { return align_sz((size_t)c->H * c->n_hp_row
 
 size_t slot_bytes(const lq_config *c) {
     return c->n_hp_rows > 0 ? align_sz((size_t)c->H * c->dk * 4, kAlign) : 0;
+}
+
+size_t static_bytes(const lq_config *c) {
+    return c->smoothing == 2 ? align_sz((size_t)c->H * (c->dk + c->dv) * 4, kAlign) : 0;
 }
 
 size_t record_bytes(const lq_config *c) {
@@ -168,15 +175,18 @@ int lq_config_check(const lq_config *cfg) { return check_config(cfg); }
 
 size_t lq_workspace_bytes(const lq_config *cfg) {
     if (check_config(cfg) != LQ_OK) return 0;
-    return kAlign + hp_bytes(cfg) + slot_bytes(cfg) + (size_t)cfg->B * cfg->H * record_bytes(cfg);
+    return kAlign + hp_bytes(cfg) + slot_bytes(cfg) + static_bytes(cfg) +
+           (size_t)cfg->B * cfg->H * record_bytes(cfg);
 }
 
-int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_t bytes, const float *d_S0,
-                  const int32_t *h_hp_row_ids, void *stream) {
+static int state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_t bytes, const float *d_S0,
+                      const int32_t *h_hp_row_ids, const float *d_static_m, const float *d_static_s, void *stream) {
     if (!out) return LQ_ERR_INVALID_ARG;
     *out = nullptr;
     int rc = check_config(cfg);
     if (rc) return rc;
+    if ((cfg->smoothing == 2) != (d_static_m != nullptr)) return LQ_ERR_INVALID_ARG;
+    if (cfg->smoothing == 2 && !d_static_s) return LQ_ERR_INVALID_ARG;
     if (!d_workspace || !d_S0) return LQ_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(d_workspace) % kAlign) return LQ_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(d_S0) % 16) return LQ_ERR_INVALID_ARG;
@@ -193,7 +203,10 @@ int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_
     st->status = reinterpret_cast<int *>(st->ws);
     st->hp_rows = reinterpret_cast<int *>(st->ws + kAlign);
     st->slot_rows = reinterpret_cast<int *>(st->ws + kAlign + hp_bytes(cfg));
-    st->rec = st->ws + kAlign + hp_bytes(cfg) + slot_bytes(cfg);
+    st->static_ms = cfg->smoothing == 2
+                        ? reinterpret_cast<float *>(st->ws + kAlign + hp_bytes(cfg) + slot_bytes(cfg))
+                        : nullptr;
+    st->rec = st->ws + kAlign + hp_bytes(cfg) + slot_bytes(cfg) + static_bytes(cfg);
     st->heads = (size_t)cfg->B * cfg->H;
     st->n = 0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -223,11 +236,20 @@ int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_
                             cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && cfg->n_hp_rows > 0)
         e = cudaMemcpyAsync(st->slot_rows, slots, (size_t)cfg->H * cfg->dk * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && st->static_ms) {   // [H][dk] and [H][dv] -> [H][dk+dv]
+        const size_t pitch = (size_t)(cfg->dk + cfg->dv) * 4;
+        e = cudaMemcpy2DAsync(st->static_ms, pitch, d_static_m, (size_t)cfg->dk * 4, (size_t)cfg->dk * 4, cfg->H,
+                              cudaMemcpyDeviceToDevice, s);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(st->static_ms + cfg->dk, pitch, d_static_s, (size_t)cfg->dv * 4,
+                                  (size_t)cfg->dv * 4, cfg->H, cudaMemcpyDeviceToDevice, s);
+    }
     if (e == cudaSuccess) {
         if (is_int8(cfg)) {
             lq::CodecArgs a{};
             a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing;
             a.P = cfg->n_hp_rows; a.hp_rows = st->hp_rows; a.S_in = d_S0; a.bits = bits_of(cfg);
+            a.static_ms = st->static_ms;
             a.q = record_ptrs(st);
             a.status = st->status;
             e = lq::launch_quantize(a, cfg->dk, cfg->dv, (int)st->heads, s);
@@ -243,6 +265,19 @@ int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_
     }
     *out = st;
     return LQ_OK;
+}
+
+int lq_state_init(lq_state **out, const lq_config *cfg, void *d_workspace, size_t bytes, const float *d_S0,
+                  const int32_t *h_hp_row_ids, void *stream) {
+    return state_init(out, cfg, d_workspace, bytes, d_S0, h_hp_row_ids, nullptr, nullptr, stream);
+}
+
+int lq_state_init_static(lq_state **out, const lq_config *cfg, void *d_workspace, size_t bytes, const float *d_S0,
+                         const float *d_static_m, const float *d_static_s, void *stream) {
+    if (!d_static_m || !d_static_s) return LQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_static_m) | reinterpret_cast<uintptr_t>(d_static_s)) & 3)
+        return LQ_ERR_INVALID_ARG;
+    return state_init(out, cfg, d_workspace, bytes, d_S0, nullptr, d_static_m, d_static_s, stream);
 }
 
 int lq_decode_step(lq_state *st, const float *d_q, const float *d_k, const float *d_v, const float *d_beta,
@@ -352,6 +387,7 @@ int lq_quantize_state(const lq_config *cfg, const float *d_S, const int32_t *h_h
                       void *stream) {
     if (!d_S || (reinterpret_cast<uintptr_t>(d_S) % 16)) return LQ_ERR_INVALID_ARG;
     if (!cfg) return LQ_ERR_INVALID_ARG;
+    if (cfg->smoothing == 2) return LQ_ERR_UNSUPPORTED;   // fixed scales live in a decode state
     int rc = check_view(cfg, out);
     if (rc) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -397,6 +433,7 @@ int lq_quantize_state_static(const lq_config *cfg, const float *d_S, const int32
     rc = check_hp_rows(cfg, h_hp_row_ids);
     if (rc) return rc;
     if ((long long)cfg->H * cfg->n_hp_rows > LQ_STATIC_ROWS_MAX) return LQ_ERR_UNSUPPORTED;
+    if (cfg->smoothing == 2) return LQ_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     lq::CodecArgs a{};
     a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing; a.P = cfg->n_hp_rows;
@@ -445,6 +482,7 @@ int lq_damp_select(const lq_config *cfg, int32_t n_states, const float *d_states
     if (rc) return rc;
     if (cfg->n_hp_rows < 1) return LQ_ERR_INVALID_ARG;
     if (bits_of(cfg) != 8) return LQ_ERR_UNSUPPORTED;   // the selection scores INT8 error energy
+    if (cfg->smoothing == 2) return LQ_ERR_UNSUPPORTED;
     lq::CodecArgs a{};
     a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing; a.P = cfg->n_hp_rows;
     a.bits = 8;
@@ -456,6 +494,24 @@ int lq_damp_select(const lq_config *cfg, int32_t n_states, const float *d_states
     a.energy = d_energy;
     a.rows_out = d_rows;
     return cuda_rc(lq::launch_damp_select(a, cfg->dk, cfg->dv, static_cast<cudaStream_t>(stream)));
+}
+
+int lq_fit_static_scales(const lq_config *cfg, int32_t n_states, const float *d_states, const double *d_row_weight,
+                         float *d_m, float *d_s, void *stream) {
+    if (!cfg || !d_states || !d_m || !d_s || n_states < 1) return LQ_ERR_INVALID_ARG;
+    if (cfg->H < 1) return LQ_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(d_states) % 16) return LQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_m) | reinterpret_cast<uintptr_t>(d_s)) & 3) return LQ_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(d_row_weight) & 7) return LQ_ERR_INVALID_ARG;
+    int rc = check_codec_fields(cfg);
+    if (rc) return rc;
+    if (cfg->n_hp_rows != 0) return LQ_ERR_UNSUPPORTED;
+    if ((long long)n_states * cfg->H > (1ll << 31) - 1) return LQ_ERR_SHAPE;
+    lq::CodecArgs a{};
+    a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.bits = bits_of(cfg);
+    a.S_in = d_states;
+    return cuda_rc(lq::launch_fit_static(a, cfg->dk, cfg->dv, n_states, d_row_weight, d_m, d_s,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 int lq_prefill(const lq_config *cfg, int32_t T, const float *d_q, const float *d_k, const float *d_v,

@@ -15,7 +15,7 @@ struct QSmem {
 };
 
 __device__ __forceinline__ CodecOut codec_out_of(const QPtrs &q, int head) {
-    CodecOut o;
+    CodecOut o{};
     o.codes = reinterpret_cast<int8_t *>(q.codes + (size_t)head * q.codes_hs);
     o.codes_t = q.codes_t;
     o.hp = reinterpret_cast<uint16_t *>(q.hp ? q.hp + (size_t)head * q.hp_hs : nullptr);
@@ -39,6 +39,12 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const CodecArgs a) {
     float R[T::RPT][16];
     tile_load_global<DK, DV>(R, a.S_in + (size_t)head * DK * DV);
     const CodecOut out = codec_out_of(a.q, head);
+    if (a.smoothing == 2) {   // the fixed scales, read back by the codec
+        const float *ms = a.static_ms + (size_t)h * (DK + DV);
+        for (int i = threadIdx.x; i < DK; i += kThreads) out.m[i] = ms[i];
+        for (int c = threadIdx.x; c < DV; c += kThreads) out.s[c] = ms[DK + c];
+        __syncthreads();
+    }
     double eacc[T::RPT];
     codec_quantize_exact<DK, DV, false, BITS>(R, a.r, a.K, a.smoothing, a.P, a.P > 0 ? sm.map : nullptr, sm.cs, X,
                                               out, eacc);
@@ -223,6 +229,126 @@ __global__ void __launch_bounds__(kThreads) damp_select_kernel(const CodecArgs a
     }
 }
 
+// ---------------------------------------------------------------------------
+// Static key-row / value-column scales fitted offline (STEPQuant article: the
+// scales are fitted jointly from the state distribution and each key row's
+// impact on the output error).  Reading: per head, on the residuals of n
+// calibration states after the r compensators, minimise
+//   sum_states sum_i sum_c w_i (R_ic - (clamp(rne((R_ic / m_i) / s_c)) s_c) m_i)^2
+// by kFitRounds rounds of coordinate descent from m_i = RMS of row i over all
+// states (1 if 0) and s_c = max |R_ic / m_i| / qmax: every column takes the
+// best of s_c0 (1 - j/16), j < 12, then every row the best of m_i0 x
+// kFitRowGrid (first best kept).  Errors in double, states outer, then rows
+// (column step) or columns (row step); explicit roundings (no contraction).
+// ---------------------------------------------------------------------------
+constexpr int kFitRounds = 3;
+constexpr int kFitNCol = 12;
+constexpr int kFitNRow = 9;
+__constant__ float kFitRowGrid[kFitNRow] = {0.5f, 0.625f, 0.75f, 0.875f, 1.0f, 1.25f, 1.5f, 1.75f, 2.0f};
+
+// Residual of one calibration state after the compensators (FP64 extraction),
+// float, to the scratch array [n][H][DK][DV].
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads) fit_residual_kernel(const CodecArgs a) {
+    extern __shared__ __align__(16) unsigned char dyn[];
+    ExactSmem<DK, DV> &X = *reinterpret_cast<ExactSmem<DK, DV> *>(dyn);
+    using T = Tile<DK, DV>;
+    const size_t idx = blockIdx.x;   // state * H + head
+    float R[T::RPT][16];
+    tile_load_global<DK, DV>(R, a.S_in + idx * DK * DV);
+    CodecOut none{};
+    codec_compensators_fp64<DK, DV, false>(R, a.r, a.K, X, none);
+    tile_store_global<DK, DV>(R, a.S_out + idx * DK * DV);
+}
+
+__device__ __forceinline__ double fit_err(float R, float m, float s, float qmax) {
+    float dq = 0.0f;
+    if (s != 0.0f) {
+        const float x = __fdiv_rn(R, m);
+        const float rq = fminf(fmaxf(rintf(__fdiv_rn(x, s)), -qmax), qmax);
+        dq = __fmul_rn(__fmul_rn(rq, s), m);
+    }
+    const double d = __dsub_rn((double)R, (double)dq);
+    return __dmul_rn(d, d);
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads) fit_static_kernel(const CodecArgs a, const float *res, int n,
+                                                              const double *weight, float *m_out, float *s_out) {
+    __shared__ float m0[DK], m[DK], s0[DV], s[DV];
+    __shared__ double w[DK];
+    __shared__ double err[kFitNRow > kFitNCol ? kFitNRow : kFitNCol][DK > DV ? DK : DV];
+    const int h = blockIdx.x, t = threadIdx.x, H = a.H;
+    const float qmax = (float)((1 << (a.bits - 1)) - 1);
+    auto Rv = [&](int st, int i, int c) -> float { return res[(((size_t)st * H + h) * DK + i) * DV + c]; };
+    if (t < DK) {
+        w[t] = weight ? weight[(size_t)h * DK + t] : 1.0;
+        double ss = 0.0;
+        for (int st = 0; st < n; ++st)
+            for (int c = 0; c < DV; ++c) {
+                const double r = (double)Rv(st, t, c);
+                ss = __dadd_rn(ss, __dmul_rn(r, r));
+            }
+        float mi = (float)sqrt(__ddiv_rn(ss, (double)n * DV));
+        if (mi == 0.0f) mi = 1.0f;
+        m0[t] = m[t] = mi;
+    }
+    __syncthreads();
+    if (t < DV) {
+        float amax = 0.0f;
+        for (int st = 0; st < n; ++st)
+            for (int i = 0; i < DK; ++i) amax = fmaxf(amax, fabsf(__fdiv_rn(Rv(st, i, t), m[i])));
+        s0[t] = s[t] = __fdiv_rn(amax, qmax);
+    }
+    __syncthreads();
+    for (int round = 0; round < kFitRounds; ++round) {
+        // columns: every (column, candidate) pair by one thread
+        for (int p = t; p < DV * kFitNCol; p += kThreads) {
+            const int c = p % DV, j = p / DV;
+            const float sc = __fmul_rn(s0[c], 1.0f - (float)j / 16.0f);
+            double e = 0.0;
+            for (int st = 0; st < n; ++st)
+                for (int i = 0; i < DK; ++i) e = __dadd_rn(e, __dmul_rn(w[i], fit_err(Rv(st, i, c), m[i], sc, qmax)));
+            err[j][c] = e;
+        }
+        __syncthreads();
+        if (t < DV) {
+            double best = INFINITY;
+            float sb = s[t];
+            for (int j = 0; j < kFitNCol; ++j)
+                if (err[j][t] < best) {
+                    best = err[j][t];
+                    sb = __fmul_rn(s0[t], 1.0f - (float)j / 16.0f);
+                }
+            s[t] = sb;
+        }
+        __syncthreads();
+        // rows
+        for (int p = t; p < DK * kFitNRow; p += kThreads) {
+            const int i = p % DK, j = p / DK;
+            const float mi = __fmul_rn(m0[i], kFitRowGrid[j]);
+            double e = 0.0;
+            for (int st = 0; st < n; ++st)
+                for (int c = 0; c < DV; ++c) e = __dadd_rn(e, fit_err(Rv(st, i, c), mi, s[c], qmax));
+            err[j][i] = e;
+        }
+        __syncthreads();
+        if (t < DK) {
+            double best = INFINITY;
+            float mb = m[t];
+            for (int j = 0; j < kFitNRow; ++j)
+                if (err[j][t] < best) {
+                    best = err[j][t];
+                    mb = __fmul_rn(m0[t], kFitRowGrid[j]);
+                }
+            m[t] = mb;
+        }
+        __syncthreads();
+    }
+    if (t < DK) m_out[(size_t)h * DK + t] = m[t];
+    if (t < DV) s_out[(size_t)h * DV + t] = s[t];
+}
+
 #define LQ_PICK(dk, dv, KERN)                          \
     (((dk) == 128 && (dv) == 128)  ? KERN<128, 128>    \
      : ((dk) == 64 && (dv) == 64)  ? KERN<64, 64>      \
@@ -277,6 +403,38 @@ cudaError_t launch_damp_select(const CodecArgs &a, int dk, int dv, cudaStream_t 
     if (e != cudaSuccess) return e;
     kern<<<a.H, kThreads, sm, s>>>(a);
     return cudaGetLastError();
+}
+
+template <int DK, int DV>
+static cudaError_t fit_static_t(const CodecArgs &a, int n, const double *weight, float *m, float *sc,
+                                cudaStream_t s) {
+    float *res = nullptr;
+    const size_t nb = (size_t)n * a.H * DK * DV * sizeof(float);
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&res), nb, s);
+    if (e != cudaSuccess) return e;
+    auto rk = fit_residual_kernel<DK, DV>;
+    const size_t sm = sizeof(ExactSmem<DK, DV>);
+    e = allow_smem(rk, sm);
+    CodecArgs b = a;
+    b.S_out = res;
+    if (e == cudaSuccess) {
+        rk<<<n * a.H, kThreads, sm, s>>>(b);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+        fit_static_kernel<DK, DV><<<a.H, kThreads, 0, s>>>(a, res, n, weight, m, sc);
+        e = cudaGetLastError();
+    }
+    const cudaError_t f = cudaFreeAsync(res, s);
+    return e != cudaSuccess ? e : f;
+}
+
+cudaError_t launch_fit_static(const CodecArgs &a, int dk, int dv, int n, const double *weight, float *m,
+                              float *sc, cudaStream_t s) {
+    if (dk == 128 && dv == 128) return fit_static_t<128, 128>(a, n, weight, m, sc, s);
+    if (dk == 64 && dv == 64) return fit_static_t<64, 64>(a, n, weight, m, sc, s);
+    if (dk == 64 && dv == 128) return fit_static_t<64, 128>(a, n, weight, m, sc, s);
+    return fit_static_t<128, 64>(a, n, weight, m, sc, s);
 }
 
 // The codec's division routine beside IEEE division (lq_selftest_division).

@@ -13,8 +13,10 @@
 //      takes them in FP32 when safely in range.)
 //   2. BF16 rows: bf16_rne(R_i) for the head's listed key rows.
 //   3. m_i = sqrt(mean_c R_ic^2) (double accumulation), 1 if zero or if
-//      smoothing is off;  x = R / m.
-//   4. s_c = max_i |x_ic| / qmax over INT8 rows;  C = clamp(rne(x / s), +-qmax),
+//      smoothing is off, the head's fixed scale with smoothing 2 (fitted
+//      offline, STEPQuant article);  x = R / m.
+//   4. s_c = max_i |x_ic| / qmax over INT8 rows (fixed with smoothing 2);
+//      C = clamp(rne(x / s), +-qmax),
 //      qmax = 2^(b-1) - 1 for b-bit codes (127, 31, 7: the LeapQuant page's
 //      8-, 6- and 4-bit states).
 //
@@ -65,6 +67,9 @@ struct CodecOut {
     float *cw;         // w_j at cw + j*cw_stride, [DV] each
     int cw_stride;
 };
+// With smoothing 2 the scales are fixed: the codec reads them from m and s
+// (the record's, which hold them from lq_state_init on) and writes them back
+// unchanged.
 
 template <int DK, int DV>
 __device__ __forceinline__ void load_cols16(const float *v, float (&o)[16]) {
@@ -384,20 +389,23 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
                 *reinterpret_cast<uint2 *>(out.hp + (size_t)p * DV + T::col(cg, q)) = make_uint2(lo, hi);
             }
         }
-        // row sum of squares in double over the row group's CG lanes (one row
-        // at a time: few registers beside the tile)
-        double ss = 0.0;
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            ss = fma((double)R[r][q], (double)R[r][q], ss);
-            minabs = fminf(minabs, fabsf(R[r][q]));
-        }
-#pragma unroll
-        for (int mm = CG / 2; mm >= 1; mm >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, mm);
+        for (int q = 0; q < 16; ++q) minabs = fminf(minabs, fabsf(R[r][q]));
         float mi = 1.0f;
-        if (smoothing && mp >= 0) {
-            mi = (float)sqrt(ss / (double)DV);
-            if (mi == 0.0f) mi = 1.0f;
+        if (smoothing == 2) {
+            mi = out.m[i];   // fixed (fitted offline)
+        } else {
+            // row sum of squares in double over the row group's CG lanes (one
+            // row at a time: few registers beside the tile)
+            double ss = 0.0;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) ss = fma((double)R[r][q], (double)R[r][q], ss);
+#pragma unroll
+            for (int mm = CG / 2; mm >= 1; mm >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, mm);
+            if (smoothing && mp >= 0) {
+                mi = (float)sqrt(ss / (double)DV);
+                if (mi == 0.0f) mi = 1.0f;
+            }
         }
         m[r] = mi;
     }
@@ -442,8 +450,16 @@ __device__ void codec_finish(float (&R)[Tile<DK, DV, NT>::RPT][16], int smoothin
     }
     auto X = [&](int r, int q) -> float { return ENERGY ? __fdiv_rn(R[r][q], m[r]) : R[r][q]; };
 
-    // 4. Column scales over INT8 rows.
-    {
+    // 4. Column scales over INT8 rows (fixed ones with smoothing 2).
+    if (smoothing == 2) {
+        if (t < DV) {
+            const float sc = out.s[t];
+            cs.sc[t] = sc;
+            cs.ysc[t] = __frcp_rn(sc);
+            if (!ENERGY) out.s[t] = sc;
+        }
+        cbar<NT>();
+    } else {
         float am[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) am[q] = 0.f;

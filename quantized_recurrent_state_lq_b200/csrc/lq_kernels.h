@@ -48,6 +48,7 @@ struct QPtrs {
 struct CodecArgs {
     int H, r, K, smoothing, P;
     int bits;             // code width: 8, 6 or 4 (the quantizer's qmax; packing of codes_t stores)
+    const float *static_ms;   // smoothing 2: per head h, key-row then value-column scales [H][dk+dv]
     const int *hp_rows;   // [H][P] (device), may be null when P == 0
     const float *S_in;    // [heads][dk][dv]
     float *S_out;         // [heads][dk][dv]
@@ -87,6 +88,8 @@ cudaError_t launch_quantize(const CodecArgs &a, int dk, int dv, int heads, cudaS
 cudaError_t launch_dequantize(const CodecArgs &a, int dk, int dv, int heads, cudaStream_t s);
 cudaError_t launch_qcopy(const CodecArgs &a, int dk, int dv, int heads, cudaStream_t s);
 cudaError_t launch_damp_select(const CodecArgs &a, int dk, int dv, cudaStream_t s);
+cudaError_t launch_fit_static(const CodecArgs &a, int dk, int dv, int n, const double *weight, float *m,
+                              float *sc, cudaStream_t s);
 
 cudaError_t launch_div_selftest(const float *a, const float *b, float *fast, float *pair, float *ieee, int n,
                                 cudaStream_t s);

@@ -33,7 +33,8 @@ EXPORTED = ["lq_workspace_bytes", "lq_config_check", "lq_state_init", "lq_decode
             "lq_window_flush", "lq_state_buffered", "lq_state_export_fp32",
             "lq_state_export_view", "lq_state_import_view", "lq_quantize_state",
             "lq_dequantize_state", "lq_quantize_state_static", "lq_damp_select", "lq_get_status",
-            "lq_state_destroy", "lq_strerror", "lq_selftest_division", "lq_prefill"]
+            "lq_state_destroy", "lq_strerror", "lq_selftest_division", "lq_prefill",
+            "lq_state_init_static", "lq_fit_static_scales"]
 
 
 class LqError(RuntimeError):
@@ -86,6 +87,8 @@ def lib():
             "lq_strerror": (C.c_char_p, [C.c_int]),
             "lq_selftest_division": (C.c_int, [vp, vp, vp, vp, vp, i32, vp]),
             "lq_prefill": (C.c_int, [cfgp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+            "lq_state_init_static": (C.c_int, [C.POINTER(vp), cfgp, vp, sz, vp, vp, vp, vp]),
+            "lq_fit_static_scales": (C.c_int, [cfgp, i32, vp, vp, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -219,19 +222,44 @@ class LqState:
 
 
 def lq_state_init(cfg: Config, S0: torch.Tensor, hp_rows=None, workspace: torch.Tensor | None = None,
-                  stream=None) -> LqState:
+                  stream=None, static_m: torch.Tensor | None = None,
+                  static_s: torch.Tensor | None = None) -> LqState:
+    """lq_state_init, or lq_state_init_static when the scales are given
+    (cfg.smoothing = 2: static_m [H, dk], static_s [H, dv])."""
     nbytes = lq_workspace_bytes(cfg)
     if nbytes == 0:
         _chk(lq_config_check(cfg), "lq_config_check")
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=S0.device)
     p_s0 = _dev(S0, "S0", (cfg.B, cfg.H, cfg.dk, cfg.dv))
-    rows, p_rows = _host_rows(cfg, hp_rows)
     h = C.c_void_p()
-    _chk(lib().lq_state_init(C.byref(h), C.byref(cfg.c()), C.c_void_p(workspace.data_ptr()),
-                             workspace.numel() * workspace.element_size(), C.c_void_p(p_s0), p_rows,
+    ws = (C.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size())
+    if static_m is not None or static_s is not None:
+        pm = _dev(static_m, "static_m", (cfg.H, cfg.dk))
+        ps = _dev(static_s, "static_s", (cfg.H, cfg.dv))
+        _chk(lib().lq_state_init_static(C.byref(h), C.byref(cfg.c()), *ws, C.c_void_p(p_s0), C.c_void_p(pm),
+                                        C.c_void_p(ps), C.c_void_p(_stream(stream))), "lq_state_init_static")
+        return LqState(cfg, h.value, workspace, None)
+    rows, p_rows = _host_rows(cfg, hp_rows)
+    _chk(lib().lq_state_init(C.byref(h), C.byref(cfg.c()), *ws, C.c_void_p(p_s0), p_rows,
                              C.c_void_p(_stream(stream))), "lq_state_init")
     return LqState(cfg, h.value, workspace, rows)
+
+
+def lq_fit_static_scales(cfg: Config, states: torch.Tensor, row_weight: torch.Tensor | None = None,
+                         stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Static scales (smoothing 2) of every head from calibration states
+    [n, H, dk, dv]; row_weight [H, dk] float64 or None.  Returns (m [H, dk],
+    s [H, dv])."""
+    n = states.shape[0]
+    p_st = _dev(states, "states", (n, cfg.H, cfg.dk, cfg.dv))
+    p_w = _dev(row_weight, "row_weight", (cfg.H, cfg.dk), torch.float64) if row_weight is not None else None
+    m = torch.empty((cfg.H, cfg.dk), device=states.device)
+    s = torch.empty((cfg.H, cfg.dv), device=states.device)
+    _chk(lib().lq_fit_static_scales(C.byref(cfg.c()), C.c_int32(n), C.c_void_p(p_st), C.c_void_p(p_w),
+                                    C.c_void_p(m.data_ptr()), C.c_void_p(s.data_ptr()),
+                                    C.c_void_p(_stream(stream))), "lq_fit_static_scales")
+    return m, s
 
 
 def lq_decode_step(st: LqState, q, k, v, beta, alpha, o, stream=None):

@@ -151,13 +151,15 @@ def assert_code_bar(stats: dict, label: str = "", frac: float = CODE_FLIP_FRAC):
         f"{label}: {stats['n']}/{stats['total']} codes differ (bar {frac:.0e})"
 
 
-def oracle_ratios(cfg: lq.Config, S_heads: np.ndarray, hp_rows_heads) -> np.ndarray:
-    """x/s behind every oracle code, for float32 states S_heads [nh, dk, dv]."""
+def oracle_ratios(cfg: lq.Config, S_heads: np.ndarray, hp_rows_heads, head_cfg=None) -> np.ndarray:
+    """x/s behind every oracle code, for float32 states S_heads [nh, dk, dv]
+    (head_cfg(h): the oracle config of head h, for per-head fixed scales)."""
     oc = ocfg(cfg)
     out = np.zeros(S_heads.shape, np.float64)
     for h in range(S_heads.shape[0]):
         rows = None if hp_rows_heads is None else hp_rows_heads[h]
-        out[h] = O.quantize(oc, S_heads[h].astype(f32), hp_rows=rows, want_ratio=True)["ratio"]
+        c = oc if head_cfg is None else head_cfg(h)
+        out[h] = O.quantize(c, S_heads[h].astype(f32), hp_rows=rows, want_ratio=True)["ratio"]
     return out
 
 

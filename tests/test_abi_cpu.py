@@ -67,7 +67,7 @@ def test_workspace_size_matches_record_layout(L):
     ("Hk", 3, lq.LQ_ERR_SHAPE), ("B", 0, lq.LQ_ERR_SHAPE), ("H", 0, lq.LQ_ERR_SHAPE),
     ("W", 0, lq.LQ_ERR_INVALID_ARG), ("r", 129, lq.LQ_ERR_INVALID_ARG), ("r", -1, lq.LQ_ERR_INVALID_ARG),
     ("power_iters", -1, lq.LQ_ERR_INVALID_ARG), ("n_hp_rows", 128, lq.LQ_ERR_INVALID_ARG),
-    ("smoothing", 2, lq.LQ_ERR_INVALID_ARG), ("fused_flush", 7, lq.LQ_ERR_INVALID_ARG),
+    ("smoothing", 3, lq.LQ_ERR_INVALID_ARG), ("fused_flush", 7, lq.LQ_ERR_INVALID_ARG),
     ("W", 4097, lq.LQ_ERR_UNSUPPORTED),
 ])
 def test_config_errors(L, field, value, code):
@@ -269,3 +269,34 @@ def test_prefill_flops_model():
     assert big < f < 1.25 * big
     g = traffic.prefill_flops(configs.GDN_PREFIX_CACHE, 2048)
     assert g < f                                  # KDA's per-channel pair decays cost more
+
+
+def test_static_scales_config(L):
+    wl = configs.KDA_B256
+    c = lq.Config.from_workload(wl, smoothing=2)
+    assert lq.lq_config_check(c) == lq.LQ_OK
+    base = lq.lq_workspace_bytes(lq.Config.from_workload(wl))
+    # the [H][dk+dv] table of fixed scales, 256-byte aligned
+    assert lq.lq_workspace_bytes(c) - base == (wl.H * (wl.dk + wl.dv) * 4 + 255) // 256 * 256
+    f = lq.Config.from_workload(wl, mode="fp32", smoothing=2)
+    assert lq.lq_config_check(f) == lq.LQ_ERR_INVALID_ARG
+    d = lq.Config.from_workload(configs.GDN_DAMP, smoothing=2)
+    assert lq.lq_config_check(d) == lq.LQ_ERR_UNSUPPORTED          # no BF16 rows with fixed scales
+    # the state init needs the scales, the static init needs smoothing 2
+    h = C.c_void_p()
+    p = C.c_void_p(256)
+    assert L.lq_state_init(C.byref(h), C.byref(c.c()), p, C.c_size_t(1 << 40), p, None, None) == \
+        lq.LQ_ERR_INVALID_ARG
+    c1 = lq.Config.from_workload(wl)
+    assert L.lq_state_init_static(C.byref(h), C.byref(c1.c()), p, C.c_size_t(1 << 40), p, p, p, None) == \
+        lq.LQ_ERR_INVALID_ARG
+    assert L.lq_state_init_static(C.byref(h), C.byref(c.c()), p, C.c_size_t(1 << 40), p, None, p, None) == \
+        lq.LQ_ERR_INVALID_ARG
+    # the stateless quantizer has no scale arguments
+    assert L.lq_quantize_state(C.byref(c.c()), p, None, None, None) in (lq.LQ_ERR_INVALID_ARG,
+                                                                      lq.LQ_ERR_UNSUPPORTED)
+    # the fit's argument checks
+    assert L.lq_fit_static_scales(C.byref(c.c()), C.c_int32(0), p, None, p, p, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_fit_static_scales(C.byref(c.c()), C.c_int32(4), p, C.c_void_p(260), p, p, None) == \
+        lq.LQ_ERR_INVALID_ARG
+    assert L.lq_fit_static_scales(C.byref(d.c()), C.c_int32(4), p, None, p, p, None) == lq.LQ_ERR_UNSUPPORTED

@@ -2,6 +2,8 @@
 inputs: FP32-state mode, windowed INT8 (teacher-forced per window: each window
 starts from the oracle's window-start view, imported into the GPU state),
 per-step INT8, naive INT8, DAMP rows, partial windows and error paths."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -56,8 +58,11 @@ def test_fp32_mode_matches_oracle(gate, B, H, Hk, dk, dv):
     assert serr.max() < STATE_REL
 
 
-def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label=""):
-    """Run T tokens window by window; each window starts from the oracle's view."""
+def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=None):
+    """Run T tokens window by window; each window starts from the oracle's view.
+    static = (m [H, dk], s [H, dv]) numpy arrays: fixed scales (smoothing 2)."""
+    if static is not None:
+        smoothing = 2
     cfg = lq.Config.from_workload(wl, mode=mode, fused_flush=int(fused), smoothing=smoothing)
     if mode == "step":
         cfg.W = 1
@@ -68,11 +73,20 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label=""):
     tok = gen.token_inputs(wl, T, device="cuda")
     ph = O.per_head_inputs(tok, wl.H)
     oc = U.ocfg(cfg)
-    st = lq.lq_state_init(cfg, torch.from_numpy(S0).cuda(), hp_rows=rows)
+    if static is None:
+        st = lq.lq_state_init(cfg, torch.from_numpy(S0).cuda(), hp_rows=rows)
+        head_cfg = lambda h: oc
+    else:
+        sm, ss = (np.ascontiguousarray(x, np.float32) for x in static)
+        st = lq.lq_state_init(cfg, torch.from_numpy(S0).cuda(), static_m=torch.from_numpy(sm).cuda(),
+                              static_s=torch.from_numpy(ss).cuda())
+        oc.static_m = np.tile(sm, (wl.B, 1))        # per oracle head (b, h)
+        oc.static_s = np.tile(ss, (wl.B, 1))
+        head_cfg = lambda h: dataclasses.replace(oc, static_m=oc.static_m[h], static_s=oc.static_s[h])
     # window-start view of the oracle
     ov = O.empty_views(oc, nh)
     for h in range(nh):
-        q = O.quantize(oc, S0.reshape(nh, wl.dk, wl.dv)[h], hp_rows=None if hr is None else hr[h])
+        q = O.quantize(head_cfg(h), S0.reshape(nh, wl.dk, wl.dv)[h], hp_rows=None if hr is None else hr[h])
         for k in ov:
             ov[k][h][...] = np.asarray(q[k]).reshape(ov[k][h].shape)
     W = cfg.W
@@ -82,7 +96,7 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label=""):
     while t0 < T:
         n = min(W, T - t0)
         sl = {k: v[t0:t0 + n] for k, v in ph.items()}
-        ref = O.run(oc, sl, view=ov, hp_rows=hr, flush_last=(n == W))
+        ref = O.run(oc, sl, view=ov, hp_rows=hr, flush_last=(n == W))   # oc: all heads' fixed scales
         lq.lq_state_import_view(st, U.oracle_view_to_gpu(cfg, ov, rows))
         for t in range(n):
             last = t == n - 1
@@ -102,7 +116,7 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label=""):
             gv = lq.alloc_view(cfg)
             lq.lq_state_export_view(st, gv)
             got = U.gpu_view_to_oracle(cfg, gv, rows)
-            ratio = U.oracle_ratios(cfg, ref["S_pre"].astype(np.float32), hr)
+            ratio = U.oracle_ratios(cfg, ref["S_pre"].astype(np.float32), hr, head_cfg=head_cfg)
             c = U.compare_codes(got["codes"], ref["view"]["codes"], ratio, TIE_EPS)
             assert c["max_diff"] <= 1, f"{label}: window {t0 // W}: {c}"
             stats["flips"] += c["n"]

@@ -94,3 +94,10 @@ def test_fit_row_weight_scale_invariant_and_used(orc):
     m, s = brute.fit_static(R, w, 7)
     np.testing.assert_array_equal(a["m"], m)
     np.testing.assert_array_equal(a["s"], s)
+
+
+def test_fit_objective_function_matches_fit(orc):
+    S = gen.random_state(4, 16, 16, seed=7, n_out=2, out_factor=20.0).numpy()
+    cfg = orc.Cfg(dk=16, dv=16, r=1, K=8, bits=8)
+    res = orc.fit_static(cfg, S)
+    assert orc.fit_objective(cfg, S, res["m"], res["s"]) == pytest.approx(res["obj"][-1], rel=1e-12)

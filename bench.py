@@ -276,11 +276,11 @@ def mode_throughput(wl, S0, mode: str, windows: int, stream):
     return v
 
 
-def variant(wv, S0, stream, peak_gbs: float, note: str, windows: int = 3) -> dict:
+def variant(wv, S0, stream, peak_gbs: float, note: str, windows: int = 3, static=None) -> dict:
     """Another configuration of the window step on the same inputs: whole-window
     throughput by graph replay, and the buffering launch's achieved
     algorithmic bandwidth."""
-    r = runner.WindowRunner(wv, S0, tokens=wv.W * min(2, wv.T // wv.W))
+    r = runner.WindowRunner(wv, S0, tokens=wv.W * min(2, wv.T // wv.W), static=static)
     r.capture()
     for k in range(2):
         r.replay(k)
@@ -431,6 +431,12 @@ def run_ours(args, wl, world, rank, pg):
             f"int{b}": variant(wl.with_(bits=b), S0, stream, peaks["hbm_gbs"],
                                f"{b}-bit window-start state (codes in +-{(1 << (b - 1)) - 1}, bit-packed)")
             for b in (6, 4)}
+        line["static_scales_per_gpu"] = {
+            f"int{b}": variant(wl.with_(smoothing=2, bits=b), S0, stream, peaks["hbm_gbs"],
+                               f"{b}-bit state, fixed key-row / value-column scales fitted offline on 8 "
+                               "calibration prefills (not timed)",
+                               static=runner.static_scales(wl.with_(bits=b)))
+            for b in (8, 4)}
 
     if not args.no_modes:
         line["prefill_per_gpu"] = prefill_line(wl, stream)

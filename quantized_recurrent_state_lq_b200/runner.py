@@ -86,18 +86,41 @@ def damp_rows(wl: Workload, device="cuda") -> torch.Tensor:
     return rows.cpu()
 
 
+def static_scales(wl: Workload, n: int = 8, tokens: int | None = None, device="cuda"):
+    """Offline fit of fixed key-row / value-column scales (smoothing 2) on the
+    GPU: n calibration prefills of the workload's prefill length (calibration
+    draws, the workload's outliers), rows weighted by their decay persistence
+    1 / (1 - mean gate) (per key channel for KDA; one value per head for GDN),
+    then lq_fit_static_scales.  Returns (m [H, dk], s [H, dv]) on the device."""
+    T = wl.prefill if tokens is None else tokens
+    states, _ = gpu_prefill(wl, tokens=T, batch=n, stream="calib", device=device)
+    states = gen.apply_outliers(states, wl).contiguous()
+    tok = gen.token_inputs(wl, min(T, 256), stream="calib", batch=n, device=device)
+    a = tok["alpha"].double()
+    mean = a.mean(dim=(0, 1))                                      # [H] or [H, dk]
+    if wl.gate != "kda":
+        mean = mean[:, None].expand(wl.H, wl.dk)
+    weight = (1.0 / (1.0 - mean)).contiguous()
+    cfg = lq.Config(B=1, H=wl.H, Hk=wl.H, dk=wl.dk, dv=wl.dv, gate=wl.gate, r=wl.r, power_iters=wl.K,
+                    state_bits=wl.bits, smoothing=2)
+    return lq.lq_fit_static_scales(cfg, states, row_weight=weight)
+
+
 class WindowRunner:
     """Holds a decode state, the decode inputs of T tokens and one CUDA graph
     per window of W tokens (the W-th call also flushes)."""
 
     def __init__(self, wl: Workload, S0: torch.Tensor, *, mode: str = "window", hp_rows=None,
-                 tokens: int | None = None, device="cuda"):
+                 tokens: int | None = None, device="cuda", static=None):
         self.wl = wl
         self.cfg = lq.Config.from_workload(wl, mode=mode)
         self.W = wl.W          # tokens per graph; in step mode every call also requantizes
         self.T = wl.T if tokens is None else tokens
         self.hp_rows = hp_rows
-        self.st = lq.lq_state_init(self.cfg, S0.contiguous(), hp_rows=hp_rows)
+        if static is not None:   # fixed scales (smoothing 2): (m [H, dk], s [H, dv])
+            self.st = lq.lq_state_init(self.cfg, S0.contiguous(), static_m=static[0], static_s=static[1])
+        else:
+            self.st = lq.lq_state_init(self.cfg, S0.contiguous(), hp_rows=hp_rows)
         self.tok = gen.token_inputs(wl, self.T, device=device)
         self.out = torch.empty((self.T, wl.B, wl.H, wl.dv), device=device)
         self.graphs = {}

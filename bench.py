@@ -236,25 +236,55 @@ def kernel_times(r: runner.WindowRunner, windows: int, stream):
 
 
 def e2e_measure(r: runner.WindowRunner, steps: int, stream):
-    """Whole windows through the C ABI with HOST inputs and outputs: pinned
-    host -> device copy of the window's inputs, the W calls, and the device ->
-    host copy of its outputs, all inside the timed region."""
+    """Whole windows through the C ABI with HOST inputs and outputs: every
+    window's inputs are copied from pinned host memory to the device and its
+    outputs back, all inside the timed region.  The copies are pipelined with
+    the decode: window k+1's inputs go up on a copy stream into the other of
+    two input slots while window k runs, and window k's outputs come down on a
+    third stream while window k+1 runs (events order every reuse of a slot)."""
     W = r.W
     keys = ["q", "k", "v", "beta", "alpha"]
     host_in = {k: torch.empty_like(r.tok[k][:W], device="cpu").pin_memory() for k in keys}
     for k in keys:
         host_in[k].copy_(r.tok[k][:W])
-    host_out = torch.empty_like(r.out[:W], device="cpu").pin_memory()
+    host_out = [torch.empty_like(r.out[:W], device="cpu").pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = host_out.numel() * host_out.element_size()
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_ready, used, out_ready, out_free = [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    slot_tok = lambda sl: {k: r.tok[k][sl * W:(sl + 1) * W] for k in keys}
+
+    def upload(sl):
+        with torch.cuda.stream(up):
+            dst = slot_tok(sl)
+            for key in keys:
+                dst[key].copy_(host_in[key], non_blocking=True)
+            in_ready[sl].record(up)
+
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
+    up.wait_event(ev0)
+    upload(0)
     for k in range(steps):
-        for key in keys:
-            r.tok[key][:W].copy_(host_in[key], non_blocking=True)
-        r.replay(0)
-        host_out.copy_(r.out[:W], non_blocking=True)
+        sl = k % 2
+        if k + 1 < steps:
+            if k >= 1:
+                up.wait_event(used[1 - sl])     # window k-1 is done reading that slot
+            upload(1 - sl)
+        stream.wait_event(in_ready[sl])
+        if k >= 2:
+            stream.wait_event(out_free[sl])     # window k-2's outputs are down
+        r.replay(sl)
+        used[sl].record(stream)
+        out_ready[sl].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(out_ready[sl])
+            host_out[sl].copy_(r.out[sl * W:(sl + 1) * W], non_blocking=True)
+            out_free[sl].record(down)
+    stream.wait_stream(down)
+    stream.wait_stream(up)
     ev1.record(stream)
     ev1.synchronize()
     dt = ev0.elapsed_time(ev1) / 1e3

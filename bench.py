@@ -375,15 +375,20 @@ def prefill_line(wl, stream, chunks: int = 32, tokens: int = 64) -> dict:
     lq.lq_state_destroy(st)
     flops = traffic.prefill_flops(wl, T) * wl.heads
     achieved = flops / dt / 1e12
+    peaks, src = measured_peaks()
+    # FP32-accurate products as three TF32 passes: the TF32 peak (the measured
+    # bf16 peak x the nominal 1.1 / 2.25 ratio) / 3
+    peak = peaks["bf16_tflops"] * 1.1 / 2.25 / 3
     del tok, S
     torch.cuda.empty_cache()
     return {"tokens": T, "heads": wl.heads, "chunk": traffic.PREFILL_CHUNK, "seconds": dt,
             "value": wl.heads * T / dt, "unit": "state updates/s",
             "recurrent_fp32_seconds": dtr, "speedup_vs_recurrent": dtr / dt,
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
-                         "frac": achieved / FP32_PEAK_TFLOPS, "traffic": None,
-                         "kernel": "prefill_kernel (chunked WY form, FP32 FMA)",
-                         "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "kernel": "prefill_tc_kernel (chunked WY form; d_k x d_v products as mma.sync TF32 x3)",
+                         "peak_source": f"{src} bf16 burst x 1.1/2.25 (TF32) / 3 passes",
+                         "fp32_alu_frac": achieved / FP32_PEAK_TFLOPS},
             "note": f"{chunks} calls of one {tokens}-token draw; recurrent time from {tokens} tokens x {T // tokens}"}
 
 

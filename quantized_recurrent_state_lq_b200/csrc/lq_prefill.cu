@@ -18,11 +18,11 @@
 // Every decay factor is 2^(g_t - g_i) with i <= t, or 2^g_t: never above 1
 // for gates in (0, 1], so nothing overflows however strong the decay.
 //
-// One CTA of 2 dv threads per head (two per SM): thread (c, half) holds key
-// rows half * dk/2 .. + dk/2 of value column c of the state in registers for
-// the whole run; the chunk's keys, queries and decays are staged in shared memory
-// and read as broadcasts.  FP32 arithmetic (FMA), the products ordered as
-// written above.
+// One CTA of 2 dv threads per head (two per SM), the state in registers for
+// the whole run (below); the chunk's keys, queries and decays are staged in
+// shared memory.  The three d_k x d_v products run on the tensor cores in
+// three TF32 passes (FP32-level accuracy); the pair matrices, the forward
+// substitution and the outputs in FP32.
 #include "lq_common.cuh"
 #include "lq_prefill.h"
 
@@ -30,63 +30,108 @@ namespace lq {
 
 constexpr int kChunk = 16;
 
-template <int DK, int DV, bool KDA>
-struct PrefillSmem {
-    static constexpr int GC = KDA ? DK : 1;   // decay channels
-    static constexpr int CP = kChunk + 1;     // padded row: column access free of bank conflicts
-    float kg_t[DK][kChunk];   // (Gamma_t k_t)^T, rows read as float4
-    float qg_t[DK][kChunk];   // (Gamma_t q_t)^T
-    float kh_t[DK][kChunk];   // (Gamma_C / Gamma_t k_t)^T
-    float k[DK][CP];          // k^T, q^T as staged
-    float q[DK][CP];
-    float g[GC][CP];          // cumulative log2 decay within the chunk, per channel
-    float v[kChunk][DV];
-    float beta[kChunk];
-    float A[kChunk][kChunk];
-    float P[kChunk][kChunk];
-    float yp[2][kChunk][DV];  // per row half: S^T (Gamma_t k_t)
-    float op[2][kChunk][DV];  // per row half: S^T (Gamma_t q_t)
-    float glast[DK];          // Gamma_C per key row
-};
+// ---------------------------------------------------------------------------
+// The chunk step on the tensor cores.  Warp w owns value columns
+// 16w .. 16w+15 and keeps S^T for them in registers as mma.sync m16n8k8
+// accumulator tiles (M = 16 columns, N = 8 key rows per tile): thread (g, q)
+// of a tile holds S[8nb+2q][c0+g], S[8nb+2q+1][c0+g], S[8nb+2q][c0+g+8],
+// S[8nb+2q+1][c0+g+8].  Read with the key rows of each 8-row block ordered
+// 0, 2, 4, 6, 1, 3, 5, 7, the same registers are the A operand (M = columns,
+// K = rows) of S^T (Gamma k)^T, so the products need no data movement:
+//   Y^T = S^T Kg^T, Oi^T = S^T Qg^T   (M = 16 columns, N = 8 tokens, K = rows)
+//   S^T <- Gamma_C S^T + U^T Kh        (M = 16 columns, N = 8 rows, K = tokens)
+// Every product is three TF32 MMAs (big x big + big x small + small x big of
+// the operands' split, FP32-level accuracy).  Each warp holds all key rows of
+// its columns, so no product needs a reduction across warps; the forward
+// substitution of the pseudo-values runs one column per lane of the warp.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 
-template <int DK, int DV>
-size_t prefill_smem_bytes_t(bool kda) {
-    return kda ? sizeof(PrefillSmem<DK, DV, true>) : sizeof(PrefillSmem<DK, DV, false>);
+// x = big + small, both TF32 (big rounded to nearest, small the exact rest
+// truncated): integer operations only.
+__device__ __forceinline__ void split_tf32(float x, uint32_t &big, uint32_t &small) {
+    big = (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
+    small = __float_as_uint(x - __uint_as_float(big)) & 0xFFFFE000u;
+}
+
+// D += A B in three TF32 passes; A given split, B as two floats.
+__device__ __forceinline__ void mma3(float (&d)[4], const uint32_t (&ab)[4], const uint32_t (&as)[4], float b0,
+                                     float b1) {
+    uint32_t bb0, bs0, bb1, bs1;
+    split_tf32(b0, bb0, bs0);
+    split_tf32(b1, bb1, bs1);
+    mma_tf32_16x8x8(d, as, bb0, bb1);
+    mma_tf32_16x8x8(d, ab, bs0, bs1);
+    mma_tf32_16x8x8(d, ab, bb0, bb1);
 }
 
 template <int DK, int DV, bool KDA>
-__global__ void __launch_bounds__(2 * DV, 2) prefill_kernel(const PrefillArgs a) {
-    constexpr int NT = 2 * DV, RH = DK / 2, C = kChunk;
-    using Sm = PrefillSmem<DK, DV, KDA>;
+struct PrefillTcSmem {
+    static constexpr int GC = KDA ? DK : 1;
+    static constexpr int CP = kChunk + 1;   // transposed rows, padded
+    static constexpr int KP = DK + 8;       // token rows of the MMA operands, padded
+    static constexpr int VP = DV + 8;
+    alignas(16) float kg[kChunk][KP];       // Gamma_t k_t (read as float2)
+    alignas(16) float qg[kChunk][KP];       // Gamma_t q_t
+    float kh[kChunk][KP];                   // Gamma_C / Gamma_t k_t
+    float y[kChunk][VP], oi[kChunk][VP];    // S^T (Gamma k), S^T (Gamma q)
+    float u[kChunk][VP];                    // pseudo-values
+    float v[kChunk][DV];
+    float kT[DK][CP], qT[DK][CP];           // raw k^T, q^T (pair matrices)
+    float g[GC][CP];                        // cumulative log2 decay
+    float beta[kChunk];
+    float A[kChunk][kChunk], P[kChunk][kChunk];
+    float glast[DK];
+};
+
+template <int DK, int DV, bool KDA>
+__global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs a) {
+    constexpr int NT = 2 * DV, C = kChunk, NB = DK / 8;
+    using Sm = PrefillTcSmem<DK, DV, KDA>;
     constexpr int GC = Sm::GC;
     (void)GC;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Sm &S = *reinterpret_cast<Sm *>(smem_raw);
     const int head = blockIdx.x;
-    const int b = head / a.H, h = head - b * a.H, g = (h * a.Hk) / a.H;
-    const int t = threadIdx.x, c = t % DV, half = t / DV, r0 = half * RH;
+    const int b = head / a.H, h = head - b * a.H, gk = (h * a.Hk) / a.H;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int gq = lane >> 2, tq = lane & 3, c0 = 16 * warp;
     const size_t state_off = (size_t)head * DK * DV;
 
-    float Sr[RH];
+    // S^T tiles: st[nb][0..3] = S[8nb+2tq][c0+gq], S[8nb+2tq+1][c0+gq],
+    //                           S[8nb+2tq][c0+gq+8], S[8nb+2tq+1][c0+gq+8]
+    float st[NB][4];
 #pragma unroll
-    for (int j = 0; j < RH; ++j) Sr[j] = a.S0 ? a.S0[state_off + (size_t)(r0 + j) * DV + c] : 0.0f;
+    for (int nb = 0; nb < NB; ++nb) {
+        const int r = 8 * nb + 2 * tq;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int rr = r + (e & 1), cc = c0 + gq + 8 * (e >> 1);
+            st[nb][e] = a.S0 ? a.S0[state_off + (size_t)rr * DV + cc] : 0.0f;
+        }
+    }
 
     const int nchunks = (a.T + C - 1) / C;
     for (int ch = 0; ch < nchunks; ++ch) {
         const int t0 = ch * C;
-        // (0) the chunk's inputs; tokens past T are identity steps (b = 0,
-        // decay 1, zero vectors) and write nothing
+        // (0) inputs; tokens past T are identity steps
         for (int e = t; e < C * DK; e += NT) {
             const int tt = e / DK, r = e % DK, tok = t0 + tt;
             float kv = 0.f, qv = 0.f, gl = 0.f;
             if (tok < a.T) {
-                const size_t qk = (((size_t)tok * a.B + b) * a.Hk + g) * DK + r;
+                const size_t qk = (((size_t)tok * a.B + b) * a.Hk + gk) * DK + r;
                 kv = a.k[qk];
                 qv = a.q[qk];
                 if (KDA) gl = fmaxf(log2f(a.alpha[(((size_t)tok * a.B + b) * a.H + h) * DK + r]), -150.0f);
             }
-            S.k[r][tt] = kv;
-            S.q[r][tt] = qv;
+            S.kT[r][tt] = kv;
+            S.qT[r][tt] = qv;
             if (KDA) S.g[r][tt] = gl;
         }
         for (int e = t; e < C * DV; e += NT) {
@@ -100,7 +145,7 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_kernel(const PrefillArgs a)
             if (!KDA) S.g[0][t] = tok < a.T ? fmaxf(log2f(a.alpha[bh]), -150.0f) : 0.f;
         }
         __syncthreads();
-        // (1) cumulative log2 decay per channel
+        // (1) cumulative log2 decay
         if (t < GC) {
             float acc = 0.f;
 #pragma unroll
@@ -112,14 +157,14 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_kernel(const PrefillArgs a)
         }
         __syncthreads();
         if (!KDA && t < DK && t > 0) S.glast[t] = S.glast[0];
-        // (2) decayed keys / queries, and the chunk's pair matrices
+        // (2) decayed operands (token-major) and the pair matrices
         for (int e = t; e < C * DK; e += NT) {
-            const int tt = e % C, r = e / C;
+            const int r = e % DK, tt = e / DK;
             const float gt = S.g[KDA ? r : 0][tt], gC = S.g[KDA ? r : 0][C - 1];
             const float et = exp2f(gt);
-            S.kg_t[r][tt] = S.k[r][tt] * et;
-            S.qg_t[r][tt] = S.q[r][tt] * et;
-            S.kh_t[r][tt] = S.k[r][tt] * exp2f(gC - gt);
+            S.kg[tt][r] = S.kT[r][tt] * et;
+            S.qg[tt][r] = S.qT[r][tt] * et;
+            S.kh[tt][r] = S.kT[r][tt] * exp2f(gC - gt);
         }
         for (int pr = t; pr < C * C; pr += NT) {
             const int ti = pr / C, ii = pr % C;
@@ -128,15 +173,15 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_kernel(const PrefillArgs a)
                 if (KDA) {
 #pragma unroll 8
                     for (int r = 0; r < DK; ++r) {
-                        const float f = exp2f(S.g[r][ti] - S.g[r][ii]) * S.k[r][ii];
-                        dkk = fmaf(S.k[r][ti], f, dkk);
-                        dqk = fmaf(S.q[r][ti], f, dqk);
+                        const float f = exp2f(S.g[r][ti] - S.g[r][ii]) * S.kT[r][ii];
+                        dkk = fmaf(S.kT[r][ti], f, dkk);
+                        dqk = fmaf(S.qT[r][ti], f, dqk);
                     }
                 } else {
 #pragma unroll 8
                     for (int r = 0; r < DK; ++r) {
-                        dkk = fmaf(S.k[r][ti], S.k[r][ii], dkk);
-                        dqk = fmaf(S.q[r][ti], S.k[r][ii], dqk);
+                        dkk = fmaf(S.kT[r][ti], S.kT[r][ii], dkk);
+                        dqk = fmaf(S.qT[r][ti], S.kT[r][ii], dqk);
                     }
                     const float f = exp2f(S.g[0][ti] - S.g[0][ii]);
                     dkk *= f;
@@ -147,82 +192,112 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_kernel(const PrefillArgs a)
             S.P[ti][ii] = ii <= ti ? dqk : 0.f;
         }
         __syncthreads();
-        // (3) S^T (Gamma_t k_t) and S^T (Gamma_t q_t) over this thread's rows,
-        // one product at a time (few accumulators beside the state)
-#pragma unroll 1
-        for (int which = 0; which < 2; ++which) {
-            float y[C];
+        // (3) Y^T = S^T Kg^T and Oi^T = S^T Qg^T on the tensor cores
+        {
+            float dy[2][4] = {}, dq[2][4] = {};
 #pragma unroll
-            for (int tt = 0; tt < C; ++tt) y[tt] = 0.f;
-            const float(*xt)[C] = which ? S.qg_t : S.kg_t;
+            for (int kb = 0; kb < NB; ++kb) {
+                uint32_t ab[4], as[4];
+                // A: rows 8kb+2tq (k = tq) and 8kb+2tq+1 (k = tq+4)
+                split_tf32(st[kb][0], ab[0], as[0]);
+                split_tf32(st[kb][2], ab[1], as[1]);
+                split_tf32(st[kb][1], ab[2], as[2]);
+                split_tf32(st[kb][3], ab[3], as[3]);
 #pragma unroll
-            for (int jj = 0; jj < RH; ++jj) {
-                const float s = Sr[jj];
-                const float4 *xr = reinterpret_cast<const float4 *>(xt[r0 + jj]);
-#pragma unroll
-                for (int u = 0; u < C / 4; ++u) {
-                    const float4 xv = xr[u];
-                    y[4 * u] = fmaf(xv.x, s, y[4 * u]);
-                    y[4 * u + 1] = fmaf(xv.y, s, y[4 * u + 1]);
-                    y[4 * u + 2] = fmaf(xv.z, s, y[4 * u + 2]);
-                    y[4 * u + 3] = fmaf(xv.w, s, y[4 * u + 3]);
+                for (int nt = 0; nt < 2; ++nt) {
+                    const float2 kv = *reinterpret_cast<const float2 *>(&S.kg[8 * nt + gq][8 * kb + 2 * tq]);
+                    const float2 qv = *reinterpret_cast<const float2 *>(&S.qg[8 * nt + gq][8 * kb + 2 * tq]);
+                    mma3(dy[nt], ab, as, kv.x, kv.y);
+                    mma3(dq[nt], ab, as, qv.x, qv.y);
                 }
             }
-            float(*dst)[DV] = which ? S.op[half] : S.yp[half];
 #pragma unroll
-            for (int tt = 0; tt < C; ++tt) dst[tt][c] = y[tt];
+            for (int nt = 0; nt < 2; ++nt) {
+                const int tt = 8 * nt + 2 * tq;
+                S.y[tt][c0 + gq] = dy[nt][0];
+                S.y[tt + 1][c0 + gq] = dy[nt][1];
+                S.y[tt][c0 + gq + 8] = dy[nt][2];
+                S.y[tt + 1][c0 + gq + 8] = dy[nt][3];
+                S.oi[tt][c0 + gq] = dq[nt][0];
+                S.oi[tt + 1][c0 + gq] = dq[nt][1];
+                S.oi[tt][c0 + gq + 8] = dq[nt][2];
+                S.oi[tt + 1][c0 + gq + 8] = dq[nt][3];
+            }
         }
-        __syncthreads();
-        // (4) pseudo-values by forward substitution (both halves of a column
-        // compute them), outputs (half 0)
-        float u[C];
-#pragma unroll
-        for (int tt = 0; tt < C; ++tt) {
-            float x = S.beta[tt] * (S.v[tt][c] - (S.yp[0][tt][c] + S.yp[1][tt][c]));
-#pragma unroll
-            for (int i = 0; i < tt; ++i) x = fmaf(-S.A[tt][i], u[i], x);
-            u[tt] = x;
-        }
-        if (half == 0 && a.o) {
+        __syncwarp();
+        // (4) pseudo-values by forward substitution and the outputs, a column per lane
+        if (lane < 16) {
+            const int cc = c0 + lane;
+            float u[C];
 #pragma unroll
             for (int tt = 0; tt < C; ++tt) {
-                const int tok = t0 + tt;
-                float x = S.op[0][tt][c] + S.op[1][tt][c];
+                float x = S.beta[tt] * (S.v[tt][cc] - S.y[tt][cc]);
 #pragma unroll
-                for (int i = 0; i <= tt; ++i) x = fmaf(S.P[tt][i], u[i], x);
-                if (tok < a.T) a.o[(((size_t)tok * a.B + b) * a.H + h) * DV + c] = x;
+                for (int i = 0; i < tt; ++i) x = fmaf(-S.A[tt][i], u[i], x);
+                u[tt] = x;
+                S.u[tt][cc] = x;
+            }
+            if (a.o) {
+#pragma unroll
+                for (int tt = 0; tt < C; ++tt) {
+                    const int tok = t0 + tt;
+                    float x = S.oi[tt][cc];
+#pragma unroll
+                    for (int i = 0; i <= tt; ++i) x = fmaf(S.P[tt][i], u[i], x);
+                    if (tok < a.T) a.o[(((size_t)tok * a.B + b) * a.H + h) * DV + cc] = x;
+                }
             }
         }
-        // (5) the state after the chunk
+        __syncwarp();
+        // (5) S^T <- Gamma_C S^T + U^T Kh on the tensor cores
+        {
+            uint32_t ub[2][4], us[2][4];
 #pragma unroll
-        for (int j = 0; j < RH; ++j) {
-            const float4 *kr = reinterpret_cast<const float4 *>(S.kh_t[r0 + j]);
-            float s = S.glast[r0 + j] * Sr[j];
-#pragma unroll
-            for (int uu = 0; uu < C / 4; ++uu) {
-                const float4 kv = kr[uu];
-                s = fmaf(kv.x, u[4 * uu], s);
-                s = fmaf(kv.y, u[4 * uu + 1], s);
-                s = fmaf(kv.z, u[4 * uu + 2], s);
-                s = fmaf(kv.w, u[4 * uu + 3], s);
+            for (int kt = 0; kt < 2; ++kt) {
+                const int tt = 8 * kt + tq;
+                split_tf32(S.u[tt][c0 + gq], ub[kt][0], us[kt][0]);
+                split_tf32(S.u[tt][c0 + gq + 8], ub[kt][1], us[kt][1]);
+                split_tf32(S.u[tt + 4][c0 + gq], ub[kt][2], us[kt][2]);
+                split_tf32(S.u[tt + 4][c0 + gq + 8], ub[kt][3], us[kt][3]);
             }
-            Sr[j] = s;
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int r = 8 * nb + 2 * tq;
+                const float g0 = S.glast[r], g1 = S.glast[r + 1];
+                st[nb][0] *= g0;
+                st[nb][1] *= g1;
+                st[nb][2] *= g0;
+                st[nb][3] *= g1;
+#pragma unroll
+                for (int kt = 0; kt < 2; ++kt)
+                    mma3(st[nb], ub[kt], us[kt], S.kh[8 * kt + tq][8 * nb + gq], S.kh[8 * kt + tq + 4][8 * nb + gq]);
+            }
         }
         __syncthreads();
     }
     bool fin = true;
 #pragma unroll
-    for (int j = 0; j < RH; ++j) {
-        fin = fin && isfinite(Sr[j]);
-        a.S_out[state_off + (size_t)(r0 + j) * DV + c] = Sr[j];
+    for (int nb = 0; nb < NB; ++nb) {
+        const int r = 8 * nb + 2 * tq;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int rr = r + (e & 1), cc = c0 + gq + 8 * (e >> 1);
+            fin = fin && isfinite(st[nb][e]);
+            a.S_out[state_off + (size_t)rr * DV + cc] = st[nb][e];
+        }
     }
     if (!fin && a.status) atomicOr(a.status, kStatusNonFinite);
 }
 
 template <int DK, int DV>
+size_t prefill_smem_bytes_t(bool kda) {
+    return kda ? sizeof(PrefillTcSmem<DK, DV, true>) : sizeof(PrefillTcSmem<DK, DV, false>);
+}
+
+template <int DK, int DV>
 static cudaError_t prefill_dispatch(const PrefillArgs &a, int heads, bool kda, cudaStream_t s) {
     const size_t sm = prefill_smem_bytes_t<DK, DV>(kda);
-    auto kern = kda ? prefill_kernel<DK, DV, true> : prefill_kernel<DK, DV, false>;
+    auto kern = kda ? prefill_tc_kernel<DK, DV, true> : prefill_tc_kernel<DK, DV, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     kern<<<heads, 2 * DV, sm, s>>>(a);

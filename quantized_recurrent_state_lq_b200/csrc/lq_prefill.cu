@@ -76,11 +76,12 @@ struct PrefillTcSmem {
     static constexpr int GC = KDA ? DK : 1;
     static constexpr int CP = kChunk + 1;   // transposed rows, padded
     static constexpr int KP = DK + 8;       // token rows of the MMA operands, padded
-    static constexpr int VP = DV + 8;
+    static constexpr int VP = DV + 8;       // u: A-fragment reads free of bank conflicts
+    static constexpr int YP = DV + 4;       // y, oi: fragment stores free of bank conflicts
     alignas(16) float kg[kChunk][KP];       // Gamma_t k_t (read as float2)
     alignas(16) float qg[kChunk][KP];       // Gamma_t q_t
     float kh[kChunk][KP];                   // Gamma_C / Gamma_t k_t
-    float y[kChunk][VP], oi[kChunk][VP];    // S^T (Gamma k), S^T (Gamma q)
+    float y[kChunk][YP], oi[kChunk][YP];    // S^T (Gamma k), S^T (Gamma q)
     float u[kChunk][VP];                    // pseudo-values
     float v[kChunk][DV];
     float kT[DK][CP], qT[DK][CP];           // raw k^T, q^T (pair matrices)

@@ -2,8 +2,9 @@
 times (whole batch, CUDA-graph replay of one window, fused flush), on a sample
 of heads the oracle recomputes one by one.
 
-1. The GPU prefill (FP32-state kernel, all heads, the full prefill length) is
-   compared with the oracle's prefill of the sampled heads on the same inputs.
+1. The GPU prefill (the chunked prefill, all heads, the full prefill length)
+   is compared with the oracle's prefill of the sampled heads on the same
+   inputs.
 2. The sampled heads' initial states are replaced by the oracle's, both sides
    quantize them (codes compared with the rounding-tie slack).
 3. The sampled heads' window-start views are set to the oracle's (teacher
@@ -37,7 +38,13 @@ def _rows(wl):
                         for _ in range(wl.H)]).int().numpy()
 
 
-@pytest.mark.parametrize("wl", configs.WORKLOADS[1:], ids=lambda w: w.name)
+def _wid(w):
+    return w.name + (f"-{w.bits}bit" if w.bits != 8 else "") + ("-bf16buf" if w.buffer_bf16 else "")
+
+
+@pytest.mark.parametrize("wl", configs.WORKLOADS[1:] + [configs.KDA_B256.with_(bits=4),
+                                                        configs.GDN_PREFIX_CACHE.with_(bits=6),
+                                                        configs.GDN_PREFIX_CACHE.with_(buffer_bf16=1)], ids=_wid)
 def test_full_size_sampled_heads(wl):
     U.require_gpu()
     heads = _sample(wl)
@@ -50,7 +57,7 @@ def test_full_size_sampled_heads(wl):
     idx_h = torch.tensor([h for _, h in heads])
     got0 = S[idx_b.cuda(), idx_h.cuda()].cpu().numpy()
     e0 = U.rel_inf_rows(got0.reshape(len(heads), -1), pre.reshape(len(heads), -1))
-    print(f"{wl.name}: prefill ({wl.prefill} tokens, FP32 kernel) max rel err {e0.max():.2e}")
+    print(f"{_wid(wl)}: prefill ({wl.prefill} tokens, chunked) max rel err {e0.max():.2e}")
     assert e0.max() < 1e-3
 
     # both sides start from the oracle's prefilled state of the sampled heads

@@ -146,6 +146,23 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
             if (!KDA) S.g[0][t] = tok < a.T ? fmaxf(log2f(a.alpha[bh]), -150.0f) : 0.f;
         }
         __syncthreads();
+        // the next chunk's input lines into L2 while this chunk computes: per
+        // token k, q (one q/k head), v and a per-channel gate, 128-byte lines
+        {
+            constexpr int LK = DK / 32, LV = DV / 32;          // lines per vector
+            constexpr int LT = 2 * LK + LV + (KDA ? LK : 0);   // lines per token
+            const int tok = t0 + C + t / LT, l = t % LT;
+            if (t < C * LT && tok < a.T) {
+                const float *p;
+                const size_t qk = (((size_t)tok * a.B + b) * a.Hk + gk) * DK;
+                const size_t hv = ((size_t)tok * a.B + b) * a.H + h;
+                if (l < LK) p = a.k + qk + 32 * l;
+                else if (l < 2 * LK) p = a.q + qk + 32 * (l - LK);
+                else if (l < 2 * LK + LV) p = a.v + hv * DV + 32 * (l - 2 * LK);
+                else p = a.alpha + hv * DK + 32 * (l - 2 * LK - LV);
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+            }
+        }
         // (1) cumulative log2 decay
         if (t < GC) {
             float acc = 0.f;

@@ -183,7 +183,8 @@ int lq_state_export_fp32(const lq_state *st, float *d_S, void *stream);
 /* Copy the window-start quantized state out to / in from plain arrays (layout of
  * lq_qstate_view, for this state's B and H).  Import starts a new window
  * (buffer emptied, Gamma = 1); with state_bits 6 or 4 it saturates codes to
- * +-qmax.  INT8 modes only.  Used for checkpoint/resume. */
+ * +-qmax; with smoothing = 2 the imported m and s are the fixed scales from
+ * then on.  INT8 modes only.  Used for checkpoint/resume. */
 int lq_state_export_view(const lq_state *st, const lq_qstate_view *out, void *stream);
 int lq_state_import_view(lq_state *st, const lq_qstate_view *in, void *stream);
 
@@ -262,7 +263,7 @@ int lq_fit_static_scales(const lq_config *cfg, int32_t n_states, const float *d_
  * quantized state, pass d_S_out to lq_state_init, which quantizes it
  * (compensators, smoothing, codes).  Device pointers, caller-owned;
  * asynchronous on `stream`; LQ_ERR_INVALID_ARG for a NULL input with T > 0,
- * T < 0 or misaligned (not 4-byte) pointers, LQ_ERR_SHAPE / _UNSUPPORTED as
+ * T < 0 or T > 2^30, misaligned (not 4-byte) pointers, LQ_ERR_SHAPE / _UNSUPPORTED as
  * for lq_config_check.
  */
 #define LQ_PREFILL_CHUNK 16

@@ -517,7 +517,7 @@ int lq_fit_static_scales(const lq_config *cfg, int32_t n_states, const float *d_
 int lq_prefill(const lq_config *cfg, int32_t T, const float *d_q, const float *d_k, const float *d_v,
                const float *d_beta, const float *d_alpha, const float *d_S0, float *d_S_out, float *d_o,
                void *stream) {
-    if (!cfg || !d_S_out || T < 0) return LQ_ERR_INVALID_ARG;
+    if (!cfg || !d_S_out || T < 0 || T > (1 << 30)) return LQ_ERR_INVALID_ARG;
     if (cfg->B < 1 || cfg->H < 1 || cfg->Hk < 1) return LQ_ERR_SHAPE;
     if (cfg->Hk > cfg->H || cfg->H % cfg->Hk != 0) return LQ_ERR_SHAPE;
     if ((long long)cfg->B * cfg->H > (1ll << 31) - 1) return LQ_ERR_SHAPE;

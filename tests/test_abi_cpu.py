@@ -248,6 +248,7 @@ def test_prefill_argument_checks(L):
     args = lambda T=8, q=p, out=p, **kw: (C.byref(kw.get("c", cfg).c()), C.c_int32(T), q, p, p, p, p, None,
                                           out, None, None)
     assert L.lq_prefill(*args(T=-1)) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_prefill(*args(T=(1 << 30) + 1)) == lq.LQ_ERR_INVALID_ARG
     assert L.lq_prefill(*args(out=None)) == lq.LQ_ERR_INVALID_ARG
     assert L.lq_prefill(*args(q=None)) == lq.LQ_ERR_INVALID_ARG
     assert L.lq_prefill(*args(q=C.c_void_p(258))) == lq.LQ_ERR_INVALID_ARG     # not 4-byte aligned

@@ -172,15 +172,24 @@ def run_reference(args, wl, world, rank, pg):
 
 # ---------------------------------------------------------------- GPU leg
 
+def _code_only(text: str) -> str:
+    """C / C++ source without comments, trailing blanks and empty lines (the
+    sources carry no comment markers inside string literals)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_sources_sha(names) -> str:
-    """sha256 prefix of the listed csrc files (in the order given): the
-    sources the profiled kernel is built from."""
+    """sha256 prefix of the listed csrc files' code (in the order given,
+    comments left out): the sources the profiled kernel is built from."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quantized_recurrent_state_lq_b200", "csrc")
     try:
         for f in names:
-            h.update(open(os.path.join(csrc, f), "rb").read())
+            h.update(_code_only(open(os.path.join(csrc, f)).read()).encode())
     except OSError:
         return "missing"
     return h.hexdigest()[:16] if names else "none"

@@ -1,8 +1,9 @@
 // lq_decode.cuh -- decode-step kernels (templates; instantiated per code width
 // by lq_decode_b8.cu, lq_decode_b6.cu and lq_decode_b4.cu).
 //
-// Windowed INT8 decode (LeapQuant project page, window paragraph): within a
-// window the INT8 state is read, never written.  With Gamma_t the product of
+// Windowed INT8 (or bit-packed 6 / 4-bit) decode (LeapQuant project page,
+// window paragraph): within a window the quantized state is read, never
+// written.  With Gamma_t the product of
 // the decays since the window start, ktil_tau = k_tau / Gamma_tau and the
 // compensators (c_j, w_j) treated as buffer entries with ktil = c_j, u = w_j
 // (Compensator Tokens paragraph), the recurrence of the LinQuant appendix
@@ -13,7 +14,7 @@
 //   u_t = beta_t (v_t - y_k),   o_t = y_q + u_t (k_t . q_t),
 // and (k_t / Gamma_t, u_t) is appended to the buffer.
 //
-// Buffering steps run decode_buffer_kernel (one CTA per head, four per SM: the
+// Buffering steps run decode_buffer_kernel (one CTA per head, seven per SM: the
 // codes staged by one bulk copy and multiplied on the int8 tensor cores, the
 // buffered entries streamed from global memory);
 // the step that ends a window runs decode_flush_kernel (one CTA per head,
@@ -27,22 +28,25 @@
 namespace lq {
 
 // ---------------------------------------------------------------------------
-// Buffering step: one CTA of 8 warps per head, small enough (<= 64 registers,
-// ~30 KB of shared memory) for four CTAs per SM, so that the phases of four
-// heads interleave on each SM:
+// Buffering step: one CTA of 4 warps per head, small enough (<= 72 registers,
+// ~27 KB of shared memory at d = 128) for seven CTAs per SM, so that the
+// phases of seven heads interleave on each SM:
 //   * thread 0 stages the record head [m | s | BF16 rows | codes] (17 KB at
-//     d = 128) with one cp.async.bulk; every warp loads the first pair of its
+//     d = 128 with INT8 codes, 13 / 9 KB with 6 / 4-bit) with one
+//     cp.async.bulk; every warp loads the first pair of its
 //     buffered entries into registers; the small step vectors are read.
 //   (a) x = Gamma_t (k, q), a = m * x; the per-vector maxima of |a|.   barrier
 //   (b) a_k, a_q as exact signed base-256 digits (4 each): the B operand.  barrier
 //   (c) codes: int8 tensor-core MMA (m16n8k32) of the value-column-major code
 //       tile with the digits, one warp per 16 value columns -- while the
-//       entry pairs are still arriving.  (With BF16 rows: SIMT, a warp per row.)
+//       entry pairs are still arriving (packed codes are unpacked to signed
+//       bytes c * 2^(8-b) in registers first).  (With BF16 rows: SIMT, a
+//       warp per row.)
 //   (d) entries: pairs of entries per warp, the next pair prefetched, dot
 //       products reduced by a transpose-reduce butterfly.
 //   (e) per-warp partial column sums combined; output, append.           barrier
 // ---------------------------------------------------------------------------
-// Warps of a buffering CTA: 4 warps and ~31 KB of shared memory let 7 heads
+// Warps of a buffering CTA: 4 warps and ~27 KB of shared memory let 7 heads
 // be in flight on an SM (the per-head critical path -- step inputs, the
 // staged codes, the tensor-core GEMV, the entry stream -- is latency-bound).
 constexpr int kBufWarps = 4;

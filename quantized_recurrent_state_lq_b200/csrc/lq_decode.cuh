@@ -154,7 +154,20 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
         fence_mbar_init();
     }
     __syncthreads();
-    if (t == 0) {
+    // Programmatic dependent launch: the next step's grid may start once every
+    // CTA of this one has begun, and this grid may have started while the
+    // previous launch on the stream finishes.  Within a window the buffering
+    // steps never write the record prefix (m, s, BF16 rows, codes), so after
+    // one (n > 0) the prefix is staged before waiting for the previous grid;
+    // everything else -- the entries and Gamma the previous step wrote, the
+    // step's inputs -- is read after the wait.
+    asm volatile("griddepcontrol.launch_dependents;");
+    if (t == 0 && a.n > 0) {
+        mbar_arrive_expect_tx(&S.mbar, (uint32_t)L.off_ent);
+        bulk_g2s(stage, rec, (uint32_t)L.off_ent, &S.mbar);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (t == 0 && a.n == 0) {
         mbar_arrive_expect_tx(&S.mbar, (uint32_t)L.off_ent);
         bulk_g2s(stage, rec, (uint32_t)L.off_ent, &S.mbar);
     }
@@ -924,7 +937,20 @@ static cudaError_t launch_buffer_t(const DecodeArgs &a, int heads, cudaStream_t 
         if (e != cudaSuccess) return e;
         carved = true;
     }
-    kern<<<heads, kBufThreads, sm, s>>>(a);
+    // launched as a programmatic dependent of the previous launch on the
+    // stream (the kernel waits for it before reading what it wrote)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)heads);
+    cfg.blockDim = dim3(kBufThreads);
+    cfg.dynamicSmemBytes = sm;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -301,3 +301,14 @@ def test_static_scales_config(L):
     assert L.lq_fit_static_scales(C.byref(c.c()), C.c_int32(4), p, C.c_void_p(260), p, p, None) == \
         lq.LQ_ERR_INVALID_ARG
     assert L.lq_fit_static_scales(C.byref(d.c()), C.c_int32(4), p, None, p, p, None) == lq.LQ_ERR_UNSUPPORTED
+
+
+def test_profiled_source_hash_ignores_comments_only():
+    """The traffic figure of the ncu record is tied to the profiled kernel's
+    code: a comment or blank-line edit keeps the hash, a code edit changes it."""
+    import bench
+    code = "int f(int x) {\n    return x + 1;  // add one\n}\n/* block\n comment */\n"
+    same = "// header\nint f(int x) {\n\n    return x + 1;\n}\n"
+    other = "int f(int x) {\n    return x + 2;\n}\n"
+    assert bench._code_only(code) == bench._code_only(same)
+    assert bench._code_only(code) != bench._code_only(other)

@@ -312,3 +312,20 @@ def test_profiled_source_hash_ignores_comments_only():
     other = "int f(int x) {\n    return x + 2;\n}\n"
     assert bench._code_only(code) == bench._code_only(same)
     assert bench._code_only(code) != bench._code_only(other)
+
+
+def test_binding_constants_match_the_header():
+    """Every #define and enum value of include/lq_state.h that the binding
+    mirrors has the header's value, and lq_config has the header's fields in
+    the header's order."""
+    text = open(HEADER).read()
+    for name, val in re.findall(r"#define (LQ_[A-Z_]+) (\d+)", text):
+        if hasattr(lq, name):
+            assert getattr(lq, name) == int(val), name
+    for name, val in re.findall(r"\b(LQ_[A-Z_]+)\s*=\s*(-?\d+)", text):
+        if hasattr(lq, name):
+            assert getattr(lq, name) == int(val), name
+    body = re.search(r"typedef struct \{(.*?)\} lq_config;", text, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = [f.strip() for decl in re.findall(r"int32_t ([^;]+);", body) for f in decl.split(",")]
+    assert fields == [n for n, _ in lq.lq_config._fields_]

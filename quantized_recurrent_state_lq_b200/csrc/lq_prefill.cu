@@ -25,6 +25,7 @@
 // substitution and the outputs in FP32.
 #include "lq_common.cuh"
 #include "lq_prefill.h"
+#include "lq_tc.cuh"
 
 namespace lq {
 
@@ -53,19 +54,12 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// x = big + small, both TF32 (big rounded to nearest, small the exact rest
-// truncated): integer operations only.
-__device__ __forceinline__ void split_tf32(float x, uint32_t &big, uint32_t &small) {
-    big = (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
-    small = __float_as_uint(x - __uint_as_float(big)) & 0xFFFFE000u;
-}
-
 // D += A B in three TF32 passes; A given split, B as two floats.
 __device__ __forceinline__ void mma3(float (&d)[4], const uint32_t (&ab)[4], const uint32_t (&as)[4], float b0,
                                      float b1) {
     uint32_t bb0, bs0, bb1, bs1;
-    split_tf32(b0, bb0, bs0);
-    split_tf32(b1, bb1, bs1);
+    tf32_split(b0, bb0, bs0);
+    tf32_split(b1, bb1, bs1);
     mma_tf32_16x8x8(d, as, bb0, bb1);
     mma_tf32_16x8x8(d, ab, bs0, bs1);
     mma_tf32_16x8x8(d, ab, bb0, bb1);
@@ -217,10 +211,10 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
             for (int kb = 0; kb < NB; ++kb) {
                 uint32_t ab[4], as[4];
                 // A: rows 8kb+2tq (k = tq) and 8kb+2tq+1 (k = tq+4)
-                split_tf32(st[kb][0], ab[0], as[0]);
-                split_tf32(st[kb][2], ab[1], as[1]);
-                split_tf32(st[kb][1], ab[2], as[2]);
-                split_tf32(st[kb][3], ab[3], as[3]);
+                tf32_split(st[kb][0], ab[0], as[0]);
+                tf32_split(st[kb][2], ab[1], as[1]);
+                tf32_split(st[kb][1], ab[2], as[2]);
+                tf32_split(st[kb][3], ab[3], as[3]);
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     const float2 kv = *reinterpret_cast<const float2 *>(&S.kg[8 * nt + gq][8 * kb + 2 * tq]);
@@ -273,10 +267,10 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
 #pragma unroll
             for (int kt = 0; kt < 2; ++kt) {
                 const int tt = 8 * kt + tq;
-                split_tf32(S.u[tt][c0 + gq], ub[kt][0], us[kt][0]);
-                split_tf32(S.u[tt][c0 + gq + 8], ub[kt][1], us[kt][1]);
-                split_tf32(S.u[tt + 4][c0 + gq], ub[kt][2], us[kt][2]);
-                split_tf32(S.u[tt + 4][c0 + gq + 8], ub[kt][3], us[kt][3]);
+                tf32_split(S.u[tt][c0 + gq], ub[kt][0], us[kt][0]);
+                tf32_split(S.u[tt][c0 + gq + 8], ub[kt][1], us[kt][1]);
+                tf32_split(S.u[tt + 4][c0 + gq], ub[kt][2], us[kt][2]);
+                tf32_split(S.u[tt + 4][c0 + gq + 8], ub[kt][3], us[kt][3]);
             }
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {

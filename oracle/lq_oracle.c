@@ -149,23 +149,43 @@ float lqo_bf16_to_float(uint16_t h)
     return f;
 }
 
+/* The window's decay product as the BF16 buffer keys against it: an FP32
+ * significand chain G_t = a_t G_{t-1} whose exponent is kept apart -- when the
+ * product falls below 2^-64 it is taken as (a_t 2^64) G_{t-1} instead (the
+ * same rounding, 64 binades up), and when even that is below 2^-64 (one
+ * token's decay under 2^-128) the chain restarts at 1.  Only the rounding
+ * of k / G depends on it: the token's contribution is G bf16(k / G), so the
+ * exponent kept apart cancels, and the state itself decays exactly (in
+ * double).  Reading of the BF16-buffer option for decays whose product leaves
+ * the FP32 range (the pages store the buffered updates in higher precision
+ * and say nothing of a decay's range). */
+static float lqo_gate_chain(float a, float g)
+{
+    float p = a * g;
+    if (p >= 0.0f && p < 0x1p-64f) {
+        p = (a * 0x1p64f) * g;
+        if (!(p >= 0x1p-64f)) p = 1.0f;
+    }
+    return p;
+}
+
 /* One token with the window's buffered updates kept in BF16 (the
  * traffic-lean buffer): as lqo_step, except that the rank-one update enters
  * the state rounded, the way the windowed kernels store it -- the key side
- * divided by the window's decay so far, ktil = k / Gamma_t, and the value side
+ * divided by the window's decay so far, ktil = k / G_t, and the value side
  * u, each rounded to BF16 (round to nearest even) from FP32:
- *     S <- S' + (Gamma_t * bf16(ktil)) bf16(u)^T,   o = S^T q.
- * Gamma_t = a_t * Gamma_{t-1} (per key row for KDA, one value for GDN) is
- * carried in FP32 in gam[] (1 at the window start), and ktil and u are formed
- * in FP32 before rounding: BF16 rounding decides the stored bits, so it is
- * taken in the kernels' precision. */
+ *     S <- S' + (G_t * bf16(ktil)) bf16(u)^T,   o = S^T q.
+ * G_t (per key row for KDA, one value for GDN) is the decay chain of
+ * lqo_gate_chain carried in FP32 in gam[] (1 at the window start), and ktil
+ * and u are formed in FP32 before rounding: BF16 rounding decides the stored
+ * bits, so it is taken in the kernels' precision. */
 void lqo_step_bf16(const lqo_cfg *cfg, double *S, float *gam, const float *q, const float *k,
                    const float *v, float beta, const float *alpha, double *o)
 {
     const int dk = cfg->dk, dv = cfg->dv, ga = cfg->gate ? dk : 1;
     double *u = (double *)malloc(sizeof(double) * dv);
     double *kg = (double *)malloc(sizeof(double) * dk);
-    for (int j = 0; j < ga; ++j) gam[j] = alpha[j] * gam[j];
+    for (int j = 0; j < ga; ++j) gam[j] = lqo_gate_chain(alpha[j], gam[j]);
     for (int i = 0; i < dk; ++i) {
         const double d = cfg->gate ? (double)alpha[i] : (double)alpha[0];
         for (int c = 0; c < dv; ++c) S[i * dv + c] *= d;
@@ -460,6 +480,22 @@ void lqo_damp_energy(const lqo_cfg *cfg, int n, const float *states, double *E)
         }
     }
     free(v.codes); free(v.m); free(v.s); free(v.c); free(v.w); free(R);
+}
+
+/* DAMP's risk score of every key row of one head [DAMP]: the calibration
+ * error energy E_i times the row's decay persistence 1 / (1 - a_i), with a_i
+ * the mean decay over the n calibration samples gates [n][ga] -- of the row's
+ * own channel for KDA (ga = dk), of the head for GDN (ga = 1, the same factor
+ * for every row).  Means accumulate in double in sample order. */
+void lqo_damp_score(int dk, int ga, int n, const float *gates, const double *E, double *score)
+{
+    for (int i = 0; i < dk; ++i) {
+        const int c = ga == 1 ? 0 : i;
+        double mean = 0.0;
+        for (int s = 0; s < n; ++s) mean += (double)gates[(size_t)s * ga + c];
+        mean /= (double)n;
+        score[i] = E[i] * (1.0 / (1.0 - mean));
+    }
 }
 
 /* Top-P rows by score, ties to the lower index, returned in increasing row

@@ -247,6 +247,20 @@ def damp_energy(cfg: Cfg, states) -> np.ndarray:
     return E
 
 
+def damp_score(E, gates) -> np.ndarray:
+    """DAMP risk score per key row: E [dk] (calibration error energy) times
+    1 / (1 - mean decay); gates [n, ga] are the calibration decays of the head
+    (ga = dk per channel for KDA, 1 for GDN) (lqo_damp_score)."""
+    e = np.ascontiguousarray(np.asarray(E, dtype=np.float64))
+    g = _f32(gates)
+    if g.ndim == 1:
+        g = g[:, None]
+    out = np.zeros(e.shape[0], np.float64)
+    lib().lqo_damp_score(C.c_int(e.shape[0]), C.c_int(g.shape[1]), C.c_int(g.shape[0]), _p(g, C.c_float),
+                         _p(e, C.c_double), _p(out, C.c_double))
+    return out
+
+
 def damp_select(score, P: int) -> np.ndarray:
     """Top-P rows by score (ties to the lower index), in increasing row order."""
     sc = np.ascontiguousarray(np.asarray(score, dtype=np.float64))

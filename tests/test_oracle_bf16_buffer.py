@@ -104,3 +104,58 @@ def test_many_tokens_within_the_rounding_bound(gate):
     dS = np.linalg.norm(b["S"][0] - a["S"][0])
     assert dS <= bound_S
     assert dS > 0                                          # the rounding did happen
+
+
+def test_zero_decay_restarts_the_key_chain():
+    """A decay of exactly 0 wipes the state; the token then enters with the
+    key chain restarted at 1: S = bf16(k) bf16(beta v)^T (y = 0 on the wiped
+    state), o = S^T q -- finite, where k / Gamma with Gamma = 0 is not."""
+    rng = np.random.default_rng(4)
+    d = 8
+    for gate in ("gdn", "kda"):
+        _, c16 = cfgs(d, d, 16, gate)
+        q = rng.standard_normal((2, 1, d)).astype(f32)
+        k = rng.standard_normal((2, 1, d)).astype(f32)
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+        v = rng.standard_normal((2, 1, d)).astype(f32)
+        beta = np.array([[0.6], [0.8]], f32)
+        shape = (2, 1, d) if gate == "kda" else (2, 1)
+        alpha = np.full(shape, 0.7, f32)
+        alpha[1] = 0.0
+        got = run(c16, q, k, v, beta, alpha)
+        u = bf16((np.float32(beta[1, 0]) * v[1, 0]).astype(f32)).astype(np.float64)
+        S = np.outer(bf16(k[1, 0]).astype(np.float64), u)
+        np.testing.assert_allclose(got["S"][0], S, rtol=1e-15, atol=0)
+        np.testing.assert_allclose(got["o"][1, 0], S.T @ q[1, 0].astype(np.float64), rtol=1e-12, atol=1e-300)
+
+
+@pytest.mark.parametrize("gate", ["gdn", "kda"])
+def test_power_of_two_decays_past_the_fp32_range(gate):
+    """Decays of 2^-10 a token for 30 tokens take Gamma to 2^-300, far below
+    FP32.  With a power-of-two decay chain, G bf16(k / G) = bf16(k) exactly
+    (scaling by a power of two commutes with rounding), so each token enters
+    as bf16(k) bf16(u)^T with u = bf16(fp32(beta (v - y))) and the state
+    decaying exactly: the whole window has this closed form, finite."""
+    rng = np.random.default_rng(5)
+    d, T = 8, 30
+    _, c16 = cfgs(d, d, 64, gate)
+    q = rng.standard_normal((T, 1, d)).astype(f32)
+    k = rng.standard_normal((T, 1, d)).astype(f32)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, 1, d)).astype(f32)
+    beta = (1 / (1 + np.exp(-rng.standard_normal((T, 1))))).astype(f32)
+    shape = (T, 1, d) if gate == "kda" else (T, 1)
+    alpha = np.full(shape, 2.0 ** -10, f32)
+    if gate == "kda":
+        alpha[:, :, ::2] = 0.5                              # channels at different depths
+    got = run(c16, q, k, v, beta, alpha)
+    S = np.zeros((d, d))
+    for t in range(T):
+        a = alpha[t, 0].astype(np.float64)
+        S = (a[:, None] if gate == "kda" else a) * S
+        y = S.T @ k[t, 0].astype(np.float64)
+        u = bf16((np.float64(beta[t, 0]) * (v[t, 0].astype(np.float64) - y)).astype(f32)).astype(np.float64)
+        S = S + np.outer(bf16(k[t, 0]).astype(np.float64), u)
+        np.testing.assert_allclose(got["o"][t, 0], S.T @ q[t, 0].astype(np.float64), rtol=1e-12, atol=1e-300)
+    assert np.isfinite(got["S"]).all()
+    np.testing.assert_allclose(got["S"][0], S, rtol=1e-12, atol=1e-300)

@@ -345,3 +345,25 @@ def test_damp_energy_definition(orc):
         deq = ((b["codes"].astype(f32) * b["s"]).astype(f32) * b["m"][:, None]).astype(f32)
         want += ((b["R32"].astype(np.float64) - deq.astype(np.float64)) ** 2).sum(axis=1)
     np.testing.assert_allclose(E, want, rtol=1e-3)
+
+
+@pytest.mark.parametrize("case", GOLD["damp_scores"], ids=lambda c: c["name"])
+def test_damp_score_hand_worked(orc, case):
+    """DAMP abstract: rows are chosen by error energy and decay persistence;
+    the worked cases (exact binary fractions) include one where per-channel
+    persistence (KDA) reorders rows that energy alone ranks the other way."""
+    score = orc.damp_score(case["E"], np.asarray(case["gates"], f32))
+    np.testing.assert_array_equal(score, np.asarray(case["score"]))
+    np.testing.assert_array_equal(orc.damp_select(score, case["P"]), case["rows"])
+    by_energy = orc.damp_select(np.asarray(case["E"]), case["P"])
+    assert (not np.array_equal(by_energy, case["rows"])) == (case["gate"] == "kda")
+
+
+def test_damp_score_persistence_limits(orc):
+    """Decays of 0 leave the energy unchanged; a mean decay of 1 - 2^-j
+    multiplies it by exactly 2^j; GDN's one decay scales every row alike."""
+    E = np.array([1.0, 2.0, 3.0, 5.0])
+    np.testing.assert_array_equal(orc.damp_score(E, np.zeros((3, 4), f32)), E)
+    g = np.array([[1 - 2.0 ** -1, 1 - 2.0 ** -2, 1 - 2.0 ** -3, 1 - 2.0 ** -10]], f32)
+    np.testing.assert_array_equal(orc.damp_score(E, g), E * np.array([2.0, 4.0, 8.0, 1024.0]))
+    np.testing.assert_array_equal(orc.damp_score(E, np.full((5, 1), 0.75, f32)), 4.0 * E)

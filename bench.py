@@ -135,16 +135,24 @@ def oracle_sample_seconds(wl, heads: int, threads: int, seed_offset: int = 0):
     return dt
 
 
-def cpu_baseline(wl, target_s: float = 12.0):
+def cpu_baseline(wl, target_s: float = 12.0, target_1t_s: float = 6.0):
+    """The oracle on all host cores (OpenMP across heads), and beside it on one
+    thread, each on a bounded sample of the workload's heads."""
     threads = os.cpu_count() or 1
     probe = 32
     dt = oracle_sample_seconds(wl, probe, threads)
     heads = int(max(probe, min(100000, probe * target_s / max(dt, 1e-3))))
     dt = oracle_sample_seconds(wl, heads, threads, seed_offset=1)
     value = heads * wl.W / dt
+    probe1 = 4
+    d1 = oracle_sample_seconds(wl, probe1, 1)
+    heads1 = int(max(probe1, min(4096, probe1 * target_1t_s / max(d1, 1e-3))))
+    d1 = oracle_sample_seconds(wl, heads1, 1, seed_offset=2)
     return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{heads} heads of {wl.name} x one window ({wl.W} tokens + flush), "
-                      f"includes the oracle's initial quantization; {dt:.1f} s"}
+                      f"includes the oracle's initial quantization; {dt:.1f} s",
+            "single_thread": {"value": heads1 * wl.W / d1, "unit": UNIT, "cores": 1, "kind": "oracle",
+                              "sample": f"{heads1} heads x one window on one thread; {d1:.1f} s"}}
 
 
 def run_reference(args, wl, world, rank, pg):
@@ -315,11 +323,11 @@ def mode_throughput(wl, S0, mode: str, windows: int, stream):
     return v
 
 
-def variant(wv, S0, stream, peak_gbs: float, note: str, windows: int = 3, static=None) -> dict:
+def variant(wv, S0, stream, peak_gbs: float, note: str, windows: int = 3, static=None, hp_rows=None) -> dict:
     """Another configuration of the window step on the same inputs: whole-window
     throughput by graph replay, and the buffering launch's achieved
     algorithmic bandwidth."""
-    r = runner.WindowRunner(wv, S0, tokens=wv.W * min(2, wv.T // wv.W), static=static)
+    r = runner.WindowRunner(wv, S0, tokens=wv.W * min(2, wv.T // wv.W), static=static, hp_rows=hp_rows)
     r.capture()
     for k in range(2):
         r.replay(k)
@@ -332,11 +340,31 @@ def variant(wv, S0, stream, peak_gbs: float, note: str, windows: int = 3, static
     launch_bytes = traffic.nonflush_launch_bytes(wv) * wv.heads
     del r
     torch.cuda.empty_cache()
+    step_bytes = traffic.window_bytes(wv) * wv.heads
     return {"value": wv.heads * wv.W * windows / dt, "unit": UNIT, "ms_per_step": 1e3 * dt / windows,
             "decode_buffering_mean_s": t_buf, "decode_flushing_mean_s": t_flush,
             "buffering_roofline_frac": launch_bytes / t_buf / 1e9 / peak_gbs,
-            "algorithmic_bytes_per_step": traffic.window_bytes(wv) * wv.heads,
+            "algorithmic_bytes_per_step": step_bytes,
+            "hbm": {"achieved_tbs": step_bytes * windows / dt / 1e12, "frac_of_8tbs": step_bytes * windows / dt / 8e12,
+                    "frac_of_measured": step_bytes * windows / dt / 1e9 / peak_gbs},
             "state_bits_per_value": traffic.bits_per_value(wv), "note": note}
+
+
+def workload_line(wl, stream, peak_gbs: float, windows: int = 6) -> dict:
+    """Another benchmark workload at its full size (its own initial state from
+    the GPU prefill, BF16 rows from the DAMP calibration where it has them):
+    the same whole-window measurement, with the clocks sampled over it."""
+    rows = runner.damp_rows(wl) if wl.P else None
+    S0, _ = runner.initial_state(wl)
+    dev = torch.cuda.current_device()
+    with ClockSampler(dev) as clk:
+        out = variant(wl, S0, stream, peak_gbs, f"workload {wl.name}", windows=windows, hp_rows=rows)
+    out["clocks"] = clk.summary()
+    out["config"] = {"workload": wl.name, "gate": wl.gate, "B": wl.B, "H": wl.H, "Hk": wl.Hk, "dk": wl.dk,
+                     "dv": wl.dv, "W": wl.W, "r": wl.r, "P": wl.P}
+    del S0
+    torch.cuda.empty_cache()
+    return out
 
 
 # FP32 arithmetic peak of the B200 used for ALU-bound kernels: 148 SMs x 128
@@ -484,6 +512,10 @@ def run_ours(args, wl, world, rank, pg):
 
     if not args.no_modes:
         line["prefill_per_gpu"] = prefill_line(wl, stream)
+        # the other two large workloads of the benchmark set, whole windows
+        for other in (configs.KDA_B256, configs.GDN_DAMP):
+            if other.name != wl.name:
+                line[other.name.split("_h")[0] + "_per_gpu"] = workload_line(other, stream, peaks["hbm_gbs"])
 
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(wl)

@@ -158,7 +158,13 @@ int lq_state_init_static(lq_state **out, const lq_config *cfg, void *d_workspace
  * alpha [B,H] (GDN) or [B,H,dk] (KDA)  ->  o [B,H,dv].
  * INT8_WINDOW: the output comes from the window-start INT8 state, its
  * compensators and the buffered updates; the new update (k_t / Gamma_t, u_t)
- * is appended to the buffer and the INT8 state is not written.  With
+ * is appended to the buffer and the INT8 state is not written.  Decay guard:
+ * Gamma_t (per key channel for KDA) is held as G_t * sigma_t with G_t in
+ * [2^-64, 1] keying the buffer and sigma_t a power of two (or 0) scaling the
+ * INT8 state; when a decay product would fall below 2^-64 the buffered keys
+ * of that channel are rescaled by 2^-64 in place (exact), or zeroed when one
+ * token's decay takes it below 2^-128 -- so any decays in [0, 1] and any
+ * window length up to LQ_MAX_WINDOW keep the buffered keys finite.  With
  * fused_flush = 1 the call that buffers the W-th token also reconstructs and
  * requantizes the state (the window ends); with fused_flush = 0 a call with W
  * tokens already buffered returns LQ_ERR_WINDOW_FULL and launches nothing.
@@ -184,7 +190,9 @@ int lq_state_export_fp32(const lq_state *st, float *d_S, void *stream);
  * lq_qstate_view, for this state's B and H).  Import starts a new window
  * (buffer emptied, Gamma = 1); with state_bits 6 or 4 it saturates codes to
  * +-qmax; with smoothing = 2 the imported m and s are the fixed scales from
- * then on.  INT8 modes only.  Used for checkpoint/resume. */
+ * then on.  INT8 modes only.  Used for checkpoint/resume.  Export is taken at
+ * a window boundary: with tokens buffered it returns LQ_ERR_UNSUPPORTED (the
+ * decay guard of lq_decode_step may have rescaled the stored compensators). */
 int lq_state_export_view(const lq_state *st, const lq_qstate_view *out, void *stream);
 int lq_state_import_view(lq_state *st, const lq_qstate_view *in, void *stream);
 
@@ -218,6 +226,8 @@ int lq_dequantize_state(const lq_config *cfg, const lq_qstate_view *in,
  *  - the first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture;
+ *  - every call copies h_hp_row_ids into the array with cudaMemcpyAsync on
+ *    `stream` (from the caller's host memory, read by that copy);
  *  - every call, on every stream, shares the one array and overwrites it:
  *    calls that overlap on the GPU race with each other.
  */
@@ -236,13 +246,16 @@ int lq_quantize_state_static(const lq_config *cfg, const float *d_S, const int32
  * coordinate descent from m_i = RMS of row i over the states (1 if 0), s_c =
  * max |R_ic / m_i| / qmax: each column takes the best of s_c0 (1 - j/16),
  * j = 0..11, then each row the best of m_i0 x {1/2, 5/8, 3/4, 7/8, 1, 5/4,
- * 3/2, 7/4, 2} (first best kept; the objective never increases).  Row weights
- * d_row_weight [H,dk] (double; NULL = 1) carry each row's impact, e.g. the
- * persistence 1 / (1 - mean decay).  A stream-ordered temporary of
+ * 3/2, 7/4, 2} (first best kept; the objective never increases).  Row weight
+ * w_i = each row's impact, read as its decay persistence 1 / (1 - mean decay)
+ * (DAMP abstract: decay persistence), from the calibration decays d_gates
+ * [n_gate_samples,H,1] (GDN, cfg->gate scalar: one weight per head) or
+ * [n_gate_samples,H,dk] (KDA: per key channel), the mean taken in double in
+ * sample order; d_gates NULL: w_i = 1.  A stream-ordered temporary of
  * n_states*H*dk*dv floats holds the residuals.  No BF16 rows.
  */
 int lq_fit_static_scales(const lq_config *cfg, int32_t n_states, const float *d_states,
-                         const double *d_row_weight, float *d_m, float *d_s, void *stream);
+                         int32_t n_gate_samples, const float *d_gates, float *d_m, float *d_s, void *stream);
 
 /*
  * Chunked prefill, the step before the windowed decode: T tokens of the
@@ -305,6 +318,22 @@ int lq_damp_select(const lq_config *cfg, int32_t n_states, const float *d_states
  */
 int lq_selftest_division(const float *d_a, const float *d_b, float *d_fast, float *d_pair, float *d_ieee,
                          int32_t n, void *stream);
+
+/*
+ * Self-test of failure detection (not part of the method; no page describes
+ * it).  Every staging copy of the decode kernels waits on an mbarrier with a
+ * time limit, and a wait that runs out raises the state's timeout status
+ * instead of hanging.  This call makes one such wait run out on purpose: one
+ * 32-thread block arms an mbarrier for 32 bytes, issues a single 16-byte bulk
+ * copy of the state's first workspace bytes (read only), and waits at most
+ * limit_ns nanoseconds (1e3 .. 1e9) for a phase that cannot complete; it then
+ * raises the timeout bit of this state's status word and returns, waiting a
+ * further (bounded) while for nothing.  Afterwards lq_get_status(st) returns
+ * LQ_ERR_TIMEOUT (the status is sticky).  Nothing else is written.
+ * LQ_ERR_INVALID_ARG for a null state or a limit out of range; LQ_ERR_CUDA
+ * if the launch fails.
+ */
+int lq_selftest_wait(lq_state *st, int64_t limit_ns, void *stream);
 
 /* Synchronize `stream` and return the sticky device status of this state:
  * LQ_OK, LQ_ERR_NONFINITE or LQ_ERR_TIMEOUT. */

@@ -124,7 +124,7 @@ lq::QPtrs record_ptrs(const lq_state *st) {
     q.s = st->rec + L.off_s; q.s_hs = hs;
     q.ck = st->rec + L.off_ent; q.ck_hs = hs; q.ck_js = L.dk + L.dv;
     q.cw = st->rec + L.off_ent + (size_t)L.dk * 4; q.cw_hs = hs; q.cw_js = L.dk + L.dv;
-    q.gam = st->rec + L.off_gam; q.gam_hs = hs; q.gam_n = L.kda ? L.dk : 1;
+    q.gam = st->rec + L.off_gam; q.gam_hs = hs; q.gam_n = L.kda ? 2 * L.dk : 2;   // G and sigma
     return q;
 }
 
@@ -336,6 +336,9 @@ int lq_state_export_fp32(const lq_state *st, float *d_S, void *stream) {
 int lq_state_export_view(const lq_state *st, const lq_qstate_view *out, void *stream) {
     if (!st) return LQ_ERR_INVALID_ARG;
     if (!is_int8(&st->cfg)) return LQ_ERR_INVALID_ARG;
+    // mid-window the record's compensators may carry the decay guard's
+    // rescaling; the window-start view is only whole at a window boundary
+    if (st->n > 0) return LQ_ERR_UNSUPPORTED;
     int rc = check_view(&st->cfg, out);
     if (rc) return rc;
     lq::CodecArgs a{};
@@ -423,8 +426,11 @@ static int static_rows_ptr(int32_t **out) {
 
 int lq_quantize_state_static(const lq_config *cfg, const float *d_S, const int32_t *h_hp_row_ids,
                              lq_qstate_view *out, void *stream) {
+    // the same checks in the same order as lq_quantize_state, then the size
+    // of the fixed row-list array
     if (!d_S || (reinterpret_cast<uintptr_t>(d_S) % 16)) return LQ_ERR_INVALID_ARG;
     if (!cfg) return LQ_ERR_INVALID_ARG;
+    if (cfg->smoothing == 2) return LQ_ERR_UNSUPPORTED;
     int rc = check_view(cfg, out);
     if (rc) return rc;
     if (cfg->B < 1 || cfg->H < 1) return LQ_ERR_SHAPE;
@@ -433,7 +439,6 @@ int lq_quantize_state_static(const lq_config *cfg, const float *d_S, const int32
     rc = check_hp_rows(cfg, h_hp_row_ids);
     if (rc) return rc;
     if ((long long)cfg->H * cfg->n_hp_rows > LQ_STATIC_ROWS_MAX) return LQ_ERR_UNSUPPORTED;
-    if (cfg->smoothing == 2) return LQ_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     lq::CodecArgs a{};
     a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.smoothing = cfg->smoothing; a.P = cfg->n_hp_rows;
@@ -496,13 +501,14 @@ int lq_damp_select(const lq_config *cfg, int32_t n_states, const float *d_states
     return cuda_rc(lq::launch_damp_select(a, cfg->dk, cfg->dv, static_cast<cudaStream_t>(stream)));
 }
 
-int lq_fit_static_scales(const lq_config *cfg, int32_t n_states, const float *d_states, const double *d_row_weight,
-                         float *d_m, float *d_s, void *stream) {
+int lq_fit_static_scales(const lq_config *cfg, int32_t n_states, const float *d_states, int32_t n_gate_samples,
+                         const float *d_gates, float *d_m, float *d_s, void *stream) {
     if (!cfg || !d_states || !d_m || !d_s || n_states < 1) return LQ_ERR_INVALID_ARG;
     if (cfg->H < 1) return LQ_ERR_SHAPE;
     if (reinterpret_cast<uintptr_t>(d_states) % 16) return LQ_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(d_m) | reinterpret_cast<uintptr_t>(d_s)) & 3) return LQ_ERR_INVALID_ARG;
-    if (reinterpret_cast<uintptr_t>(d_row_weight) & 7) return LQ_ERR_INVALID_ARG;
+    if (d_gates && ((reinterpret_cast<uintptr_t>(d_gates) & 3) || n_gate_samples < 1)) return LQ_ERR_INVALID_ARG;
+    if (cfg->gate != LQ_GATE_SCALAR && cfg->gate != LQ_GATE_CHANNEL) return LQ_ERR_INVALID_ARG;
     int rc = check_codec_fields(cfg);
     if (rc) return rc;
     if (cfg->n_hp_rows != 0) return LQ_ERR_UNSUPPORTED;
@@ -510,8 +516,10 @@ int lq_fit_static_scales(const lq_config *cfg, int32_t n_states, const float *d_
     lq::CodecArgs a{};
     a.H = cfg->H; a.r = cfg->r; a.K = cfg->power_iters; a.bits = bits_of(cfg);
     a.S_in = d_states;
-    return cuda_rc(lq::launch_fit_static(a, cfg->dk, cfg->dv, n_states, d_row_weight, d_m, d_s,
-                                         static_cast<cudaStream_t>(stream)));
+    a.gates = d_gates;
+    a.n_gate_samples = d_gates ? n_gate_samples : 0;
+    a.gate_per_channel = cfg->gate == LQ_GATE_CHANNEL;
+    return cuda_rc(lq::launch_fit_static(a, cfg->dk, cfg->dv, n_states, d_m, d_s, static_cast<cudaStream_t>(stream)));
 }
 
 int lq_prefill(const lq_config *cfg, int32_t T, const float *d_q, const float *d_k, const float *d_v,
@@ -543,6 +551,12 @@ int lq_selftest_division(const float *d_a, const float *d_b, float *d_fast, floa
     if (n < 0 || (n & 1)) return LQ_ERR_INVALID_ARG;
     if (n > 0 && (!d_a || !d_b || !d_fast || !d_pair || !d_ieee)) return LQ_ERR_INVALID_ARG;
     return cuda_rc(lq::launch_div_selftest(d_a, d_b, d_fast, d_pair, d_ieee, n, static_cast<cudaStream_t>(stream)));
+}
+
+int lq_selftest_wait(lq_state *st, int64_t limit_ns, void *stream) {
+    if (!st || limit_ns < 1000 || limit_ns > 1000000000) return LQ_ERR_INVALID_ARG;
+    return cuda_rc(lq::launch_wait_selftest(st->rec, st->status, (unsigned long long)limit_ns,
+                                            static_cast<cudaStream_t>(stream)));
 }
 
 int lq_get_status(lq_state *st, void *stream) {

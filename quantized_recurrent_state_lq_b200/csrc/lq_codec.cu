@@ -274,7 +274,7 @@ __device__ __forceinline__ double fit_err(float R, float m, float s, float qmax)
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads) fit_static_kernel(const CodecArgs a, const float *res, int n,
-                                                              const double *weight, float *m_out, float *s_out) {
+                                                              float *m_out, float *s_out) {
     __shared__ float m0[DK], m[DK], s0[DV], s[DV];
     __shared__ double w[DK];
     __shared__ double err[kFitNRow > kFitNCol ? kFitNRow : kFitNCol][DK > DV ? DK : DV];
@@ -282,7 +282,19 @@ __global__ void __launch_bounds__(kThreads) fit_static_kernel(const CodecArgs a,
     const float qmax = (float)((1 << (a.bits - 1)) - 1);
     auto Rv = [&](int st, int i, int c) -> float { return res[(((size_t)st * H + h) * DK + i) * DV + c]; };
     if (t < DK) {
-        w[t] = weight ? weight[(size_t)h * DK + t] : 1.0;
+        // row weight: the decay persistence 1 / (1 - mean calibration decay)
+        // of the row's channel (KDA) or of the head (GDN), as DAMP scores rows
+        double wt = 1.0;
+        if (a.gates) {
+            const int ga = a.gate_per_channel ? DK : 1;
+            const int col = a.gate_per_channel ? t : 0;
+            double mean = 0.0;
+            for (int sidx = 0; sidx < a.n_gate_samples; ++sidx)
+                mean += (double)a.gates[((size_t)sidx * a.H + h) * ga + col];
+            mean /= (double)a.n_gate_samples;
+            wt = 1.0 / (1.0 - mean);
+        }
+        w[t] = wt;
         double ss = 0.0;
         for (int st = 0; st < n; ++st)
             for (int c = 0; c < DV; ++c) {
@@ -406,8 +418,7 @@ cudaError_t launch_damp_select(const CodecArgs &a, int dk, int dv, cudaStream_t 
 }
 
 template <int DK, int DV>
-static cudaError_t fit_static_t(const CodecArgs &a, int n, const double *weight, float *m, float *sc,
-                                cudaStream_t s) {
+static cudaError_t fit_static_t(const CodecArgs &a, int n, float *m, float *sc, cudaStream_t s) {
     float *res = nullptr;
     const size_t nb = (size_t)n * a.H * DK * DV * sizeof(float);
     cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&res), nb, s);
@@ -422,19 +433,18 @@ static cudaError_t fit_static_t(const CodecArgs &a, int n, const double *weight,
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
-        fit_static_kernel<DK, DV><<<a.H, kThreads, 0, s>>>(a, res, n, weight, m, sc);
+        fit_static_kernel<DK, DV><<<a.H, kThreads, 0, s>>>(a, res, n, m, sc);
         e = cudaGetLastError();
     }
     const cudaError_t f = cudaFreeAsync(res, s);
     return e != cudaSuccess ? e : f;
 }
 
-cudaError_t launch_fit_static(const CodecArgs &a, int dk, int dv, int n, const double *weight, float *m,
-                              float *sc, cudaStream_t s) {
-    if (dk == 128 && dv == 128) return fit_static_t<128, 128>(a, n, weight, m, sc, s);
-    if (dk == 64 && dv == 64) return fit_static_t<64, 64>(a, n, weight, m, sc, s);
-    if (dk == 64 && dv == 128) return fit_static_t<64, 128>(a, n, weight, m, sc, s);
-    return fit_static_t<128, 64>(a, n, weight, m, sc, s);
+cudaError_t launch_fit_static(const CodecArgs &a, int dk, int dv, int n, float *m, float *sc, cudaStream_t s) {
+    if (dk == 128 && dv == 128) return fit_static_t<128, 128>(a, n, m, sc, s);
+    if (dk == 64 && dv == 64) return fit_static_t<64, 64>(a, n, m, sc, s);
+    if (dk == 64 && dv == 128) return fit_static_t<64, 128>(a, n, m, sc, s);
+    return fit_static_t<128, 64>(a, n, m, sc, s);
 }
 
 // The codec's division routine beside IEEE division (lq_selftest_division).
@@ -456,6 +466,32 @@ cudaError_t launch_div_selftest(const float *a, const float *b, float *fast, flo
     const int pairs = n / 2;
     if (pairs == 0) return cudaSuccess;
     div_selftest_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(a, b, fast, pair, ieee, n);
+    return cudaGetLastError();
+}
+
+// The bounded wait of the staging copies, made to run out: the mbarrier is
+// armed for 32 bytes and receives one 16-byte copy, so its phase never
+// completes; mbar_wait_bounded gives up after limit_ns, raises the timeout
+// status bit and returns (the copy itself has landed by then).
+__global__ void __launch_bounds__(32) wait_selftest_kernel(const unsigned char *src, int *status,
+                                                           unsigned long long limit_ns) {
+    __shared__ __align__(16) unsigned char buf[16];
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(&bar, 32u);
+        bulk_g2s(buf, src, 16u, &bar);
+        mbar_wait_bounded(&bar, 0, status, limit_ns);
+    }
+}
+
+cudaError_t launch_wait_selftest(const unsigned char *src, int *status, unsigned long long limit_ns,
+                                 cudaStream_t s) {
+    wait_selftest_kernel<<<1, 32, 0, s>>>(src, status, limit_ns);
     return cudaGetLastError();
 }
 

@@ -640,11 +640,12 @@ __device__ void codec_quantize_exact(float (&R)[Tile<DK, DV>::RPT][16], int r_co
 //   tile_gamma:        R *= Gamma (by key row); true if every value is finite
 // The arrays may live in shared or global memory: m_s [DK], s_s [DV],
 // hp_s [P][DV], codes_s (layout per codes_t; BITS < 8: the packed planes),
-// gam_s [DK].
+// gam_s [DK]; sig_s [DK] (nullable) scales every key row, quantized or BF16
+// (the decode kernels' decay guard).
 template <int DK, int DV, int NT, bool ADD = false, int BITS = 8>
 __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][16], const float *m_s,
                                              const float *s_s, const uint16_t *hp_s, const int8_t *codes_s, int P,
-                                             const int *map, bool codes_t) {
+                                             const int *map, bool codes_t, const float *sig_s = nullptr) {
     using T = Tile<DK, DV, NT>;
     constexpr int RPT = T::RPT;
     const int t = threadIdx.x, cg = t % T::CG, rg = t / T::CG, row0 = rg * RPT;
@@ -660,7 +661,7 @@ __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][1
         load_cols16<DK, DV>(s_s, sv);
         float mi[RPT];
 #pragma unroll
-        for (int r = 0; r < RPT; ++r) mi[r] = m_s[row0 + r];
+        for (int r = 0; r < RPT; ++r) mi[r] = sig_s ? m_s[row0 + r] * sig_s[row0 + r] : m_s[row0 + r];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
@@ -700,7 +701,7 @@ __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][1
         // one column are RPT consecutive bytes
         float mi[RPT];
 #pragma unroll
-        for (int r = 0; r < RPT; ++r) mi[r] = m_s[row0 + r];
+        for (int r = 0; r < RPT; ++r) mi[r] = sig_s ? m_s[row0 + r] * sig_s[row0 + r] : m_s[row0 + r];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
@@ -733,7 +734,7 @@ __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][1
         const int i = row0 + r;
         const int mp = (P > 0) ? map[i] : i;
         if (mp >= 0 && codes_t) {
-            const float mi = m_s[i];
+            const float mi = sig_s ? m_s[i] * sig_s[i] : m_s[i];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float4 s4 = *reinterpret_cast<const float4 *>(s_s + T::col(cg, q));
@@ -745,7 +746,7 @@ __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][1
                 }
             }
         } else if (mp >= 0) {
-            const float mi = m_s[i];
+            const float mi = sig_s ? m_s[i] * sig_s[i] : m_s[i];
             const uint32_t *row = reinterpret_cast<const uint32_t *>(codes_s + (size_t)mp * DV);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -758,13 +759,14 @@ __device__ __forceinline__ void tile_dequant(float (&R)[Tile<DK, DV, NT>::RPT][1
             }
         } else {
             const int p = -1 - mp;
+            const float sg = sig_s ? sig_s[i] : 1.0f;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const uint2 h = *reinterpret_cast<const uint2 *>(hp_s + (size_t)p * DV + T::col(cg, q));
-                put(r, 4 * q, bf16_to_f((uint16_t)(h.x & 0xffff)));
-                put(r, 4 * q + 1, bf16_to_f((uint16_t)(h.x >> 16)));
-                put(r, 4 * q + 2, bf16_to_f((uint16_t)(h.y & 0xffff)));
-                put(r, 4 * q + 3, bf16_to_f((uint16_t)(h.y >> 16)));
+                put(r, 4 * q, bf16_to_f((uint16_t)(h.x & 0xffff)) * sg);
+                put(r, 4 * q + 1, bf16_to_f((uint16_t)(h.x >> 16)) * sg);
+                put(r, 4 * q + 2, bf16_to_f((uint16_t)(h.y & 0xffff)) * sg);
+                put(r, 4 * q + 3, bf16_to_f((uint16_t)(h.y >> 16)) * sg);
             }
         }
     }

@@ -24,11 +24,27 @@ constexpr int kStatusTimeout = 2;
 //   codes   int8  [dk-P][dv]        INT8 codes (layout: code_off_t below), or
 //                                   4 / 6-bit codes bit-packed (nib_off, pair_off)
 //   comps   f32   [r][dk+dv]        compensator j = (c_j [dk], w_j [dv])
-//   tokens  f32 or bf16 [W][dk+dv]  buffered token tau = (k_tau/Gamma_tau, u_tau)
-//   gam     f32   [dk] (KDA) / [4] (GDN)   cumulative decay since window start
+//   tokens  f32 or bf16 [W][dk+dv]  buffered token tau = (k_tau/G_tau, u_tau)
+//   gam     f32   [2][dk] (KDA) / [4] (GDN)   the decay since the window start
+//                                   as G [dk] (GDN: [0]) and sigma [dk] ([1])
 // Entries e < r are the compensators, e = r + tau the buffered tokens; with
 // FP32 tokens both form one array [r+W][dk+dv].  A decode step reads
 // [m .. codes] with one bulk copy and the r + n entries as coalesced streams.
+//
+// Decay guard.  The product Gamma_t of a window's decays can leave the FP32
+// range for strong decays or long windows (a KDA channel at a = 0.73 passes
+// 2^-126 after ~280 tokens; a gate of 0 ends it at once), and the buffered
+// keys k / Gamma would overflow.  The kernels therefore carry Gamma_t, per
+// key channel, as G_t * sigma_t: G_t in [2^-64, 1] (1 at the window start)
+// keys the buffer (ktil = k / G, contribution ktil_tau u_tau^T G_t), and
+// sigma_t, a power of two or 0, scales the quantized state alone
+// (S_t = sigma_t G_t Deq + G_t [sum_j c_j w_j^T + sum_tau ktil_tau u_tau^T]).
+// When a step's product a_t G_{t-1} falls below 2^-64, G is rescaled by 2^64
+// and every buffered entry's key side (compensators included) and sigma by
+// 2^-64 -- all exact -- or, when one step's decay takes it below 2^-128, the
+// channel restarts: G = 1, and the entries' key side and sigma become 0
+// (what they multiply is below 2^-128 of its size).  gate_chain takes that
+// decision.
 // ---------------------------------------------------------------------------
 struct Layout {
     int dk, dv, P, r, W, kda;
@@ -51,7 +67,7 @@ __host__ inline Layout make_layout(int dk, int dv, int P, int r, int W, int kda,
     L.off_tok = L.off_ent + r * (dk + dv) * 4;
     int o = L.off_tok + W * (dk + dv) * (tok_bf16 ? 2 : 4);
     L.off_gam = align_up(o, 16);
-    o = L.off_gam + (kda ? dk : 4) * 4;
+    o = L.off_gam + (kda ? 2 * dk : 4) * 4;
     L.rec_bytes = align_up(o, 128);
     return L;
 }
@@ -129,6 +145,28 @@ __device__ __forceinline__ int packed_code(const unsigned char *codes, int c, in
     if (bits == 4) return ((int)(nib << 28)) >> 28;
     const uint32_t pr = (*reinterpret_cast<const uint16_t *>(codes + pair_off(c, g, dk, dv)) >> (2 * k)) & 3u;
     return ((int)((nib | (pr << 4)) << 26)) >> 26;
+}
+
+// One step of the decay guard (see the record layout): from the step's decay
+// a and the carried G_{t-1} in [2^-64, 1], the new G_t and the factor rho
+// applied to the buffered entries' key side and to sigma -- 1, 2^-64 (an
+// exact rescaling) or 0 (a restart).  a * 2^64 and the rescaled product are
+// exact scalings of a and of the in-range product.  NaN and negative decays
+// take the plain product (they reach the outputs and the status word).
+__host__ __device__ __forceinline__ float gate_chain(float a, float gp, float &rho) {
+    float g = a * gp;
+    rho = 1.0f;
+    if (g >= 0.0f && g < 0x1p-64f) {
+        const float g2 = (a * 0x1p64f) * gp;
+        if (g2 >= 0x1p-64f) {
+            g = g2;
+            rho = 0x1p-64f;
+        } else {
+            g = 1.0f;
+            rho = 0.0f;
+        }
+    }
+    return g;
 }
 
 // Named barrier over the NT compute threads (warps 0 .. NT/32-1) of a CTA;

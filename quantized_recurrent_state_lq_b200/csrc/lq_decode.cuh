@@ -54,7 +54,7 @@ constexpr int kBufThreads = kBufWarps * 32;
 
 template <int DK, int DV>
 struct BufSmem {
-    float2 x2[DK];                      // (Gamma k, Gamma q) by key row
+    float2 x2[DK];                      // (G k, G q) by key row (G: the guarded decay)
     float2 a2[DK];                      // m * x2 by INT8 slot (BF16-row layout)
     float2 red[kBufWarps][DV];             // per-warp partial column sums (BF16 rows + entries)
     float2 rc[DV];                      // codes part of (y_k, y_q)
@@ -62,6 +62,7 @@ struct BufSmem {
     int rows[DK];                       // DAMP: key row of INT8 slot j, then of BF16 row p
     float v[DV];
     float qk[DK];                       // q (BF16 buffer: k . q is formed at the end)
+    int rebase;                         // decay guard: some key channel rescales its entries this step
     float amax[kBufWarps][2];
     float kqw[kBufWarps];
     uint64_t mbar;
@@ -144,7 +145,8 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
     const float *ent_g = reinterpret_cast<const float *>(rec + L.off_ent);
     float *rec_ent = reinterpret_cast<float *>(rec + L.off_ent);
     uint16_t *rec_tok16 = reinterpret_cast<uint16_t *>(rec + L.off_tok);   // BF16 tokens
-    float *rec_gam = reinterpret_cast<float *>(rec + L.off_gam);
+    float *rec_gam = reinterpret_cast<float *>(rec + L.off_gam);   // G
+    float *rec_sig = rec_gam + (KDA ? DK : 1);                       // sigma
     constexpr bool tb = TB;   // buffered tokens in BF16
     constexpr int XPL = DK / 32;                 // key elements per lane in a dot product
     constexpr int EF = DK + DV;                  // elements per entry
@@ -152,7 +154,15 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
     if (t == 0) {
         mbar_init(&S.mbar, 1);
         fence_mbar_init();
+        S.rebase = 0;
     }
+    // Decay guard scratch in shared arrays this variant leaves unused: this
+    // step's factor rho per key row (DAMP: the q row array, never used with
+    // DAMP's BF16 rows; else the DAMP-only activation array) and, for DAMP,
+    // sigma per key row (in the digit array, which only the tensor-core GEMV
+    // of the other variants uses).
+    float *rho_s = DAMP ? S.qk : reinterpret_cast<float *>(S.a2);
+    float *sig_s = reinterpret_cast<float *>(&S.dig[0][0]);
     __syncthreads();
     // Programmatic dependent launch: the next step's grid may start once every
     // CTA of this one has begun, and this grid may have started while the
@@ -207,26 +217,32 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
     };
     load_pair(2 * warp);
 
-    // (a) step inputs, Gamma_t, x, a = m * x.
-    float kqp = 0.f, gt = 1.f, kk = 0.f, ak_t = 0.f, aq_t = 0.f;
+    // (a) step inputs, the guarded decay (G_t, sigma_t, the entries' rescaling
+    // rho), x = G_t (k, q), a = m * sigma_t * x.
+    float kqp = 0.f, gt = 1.f, kk = 0.f, ak_t = 0.f, aq_t = 0.f, sg = 1.f, rho = 1.f;
     if (t < DK) {
         const size_t qk = ((size_t)b * a.Hk + g) * DK;
         kk = a.k[qk + t];
         const float qq = a.q[qk + t];
         const float gp = a.n > 0 ? (KDA ? rec_gam[t] : rec_gam[0]) : 1.0f;
-        gt = (KDA ? a.alpha[hv * DK + t] : a.alpha[hv]) * gp;
+        const float sp = a.n > 0 ? (KDA ? rec_sig[t] : rec_sig[0]) : 1.0f;
+        gt = gate_chain(KDA ? a.alpha[hv * DK + t] : a.alpha[hv], gp, rho);
+        sg = sp * rho;
         const float2 x = make_float2(gt * kk, gt * qq);
         S.x2[t] = x;
+        rho_s[t] = rho;
+        if (rho != 1.f) S.rebase = 1;
         // k . q for the output (BF16 buffer: Gamma bf16(k / Gamma) . q, formed
         // at the end, next to the reduction it feeds)
         kqp = tb ? 0.f : kk * qq;
         if (tb) S.qk[t] = qq;
         if (!DAMP) {
             const float mi = reinterpret_cast<const float *>(rec + L.off_m)[t];
-            ak_t = mi * x.x;
-            aq_t = mi * x.y;
+            ak_t = mi * (sg * x.x);
+            aq_t = mi * (sg * x.y);
         } else {
             S.rows[t] = a.slot_rows[(size_t)h * DK + t];
+            sig_s[t] = sg;
         }
     }
     if (t < DV) S.v[t] = a.v[hv * DV + t];
@@ -246,6 +262,8 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
     }
     if (lane == 0) S.kqw[warp] = kqp;
     __syncthreads();
+    // a rescaling of the buffered keys this step (rare: the decay passed 2^-64)
+    const bool rebase = S.rebase != 0;
     float kq = 0.f;
 #pragma unroll
     for (int w = 0; w < kBufWarps; ++w) kq += S.kqw[w];
@@ -285,7 +303,8 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
         const float *m_s = reinterpret_cast<const float *>(stage + L.off_m);
         const int row = S.rows[t];
         const float2 x = S.x2[row];
-        S.a2[t] = make_float2(m_s[row] * x.x, m_s[row] * x.y);
+        const float ms = m_s[row] * sig_s[row];
+        S.a2[t] = make_float2(ms * x.x, ms * x.y);
     }
     if (__syncthreads_or(!ok)) return;
     const float *s_s = reinterpret_cast<const float *>(stage + L.off_s);
@@ -412,7 +431,8 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
         for (int p = warp; p < P; p += kBufWarps) {   // BF16 rows: unscaled x
             if (lane < DV / 4) {
                 const uint2 hb = *reinterpret_cast<const uint2 *>(hp + (size_t)p * DV + 4 * lane);
-                const float2 x = S.x2[S.rows[NI + p]];
+                const int row = S.rows[NI + p];
+                const float2 x = make_float2(S.x2[row].x * sig_s[row], S.x2[row].y * sig_s[row]);
                 const float f0 = bf16_to_f((uint16_t)(hb.x & 0xffff)), f1 = bf16_to_f((uint16_t)(hb.x >> 16));
                 const float f2 = bf16_to_f((uint16_t)(hb.y & 0xffff)), f3 = bf16_to_f((uint16_t)(hb.y >> 16));
                 ek[0] = fmaf(f0, x.x, ek[0]); ek[1] = fmaf(f1, x.x, ek[1]);
@@ -432,7 +452,38 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
             xk[u] = x.x;
             xq[u] = x.y;
         }
+        // decay guard: the entries' key side rescaled by rho (exact) in
+        // registers and written back, once for this step and the rest of the
+        // window (entries E - 1 and before; this step's own is appended below)
+        auto rescale = [&](int p, int e) {
+            float rl[XPL];
+#pragma unroll
+            for (int u = 0; u < XPL; ++u) rl[u] = rho_s[XPL * lane + u];
+            if (XPL == 4) {
+                kb[p] = make_float4(kb[p].x * rl[0], kb[p].y * rl[1 % XPL], kb[p].z * rl[2 % XPL], kb[p].w * rl[3 % XPL]);
+                if (!tb || e < L.r) {
+                    reinterpret_cast<float4 *>(rec_ent + (size_t)e * EF)[lane] = kb[p];
+                } else {
+                    const uint32_t lo = (uint32_t)bf16_rne(kb[p].x) | ((uint32_t)bf16_rne(kb[p].y) << 16);
+                    const uint32_t hi = (uint32_t)bf16_rne(kb[p].z) | ((uint32_t)bf16_rne(kb[p].w) << 16);
+                    reinterpret_cast<uint2 *>(rec_tok16 + (size_t)(e - L.r) * EF)[lane] = make_uint2(lo, hi);
+                }
+            } else {
+                kb2[p] = make_float2(kb2[p].x * rl[0], kb2[p].y * rl[1 % XPL]);
+                if (!tb || e < L.r) {
+                    reinterpret_cast<float2 *>(rec_ent + (size_t)e * EF)[lane] = kb2[p];
+                } else {
+                    reinterpret_cast<uint32_t *>(rec_tok16 + (size_t)(e - L.r) * EF)[lane] =
+                        (uint32_t)bf16_rne(kb2[p].x) | ((uint32_t)bf16_rne(kb2[p].y) << 16);
+                }
+            }
+        };
         for (int e0 = 2 * warp; e0 < E; e0 += 2 * kBufWarps) {
+            if (rebase) {
+#pragma unroll
+                for (int p = 0; p < 2; ++p)
+                    if (e0 + p < E) rescale(p, e0 + p);
+            }
             float d[4];
             float4 uv[2];
 #pragma unroll
@@ -515,8 +566,13 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
     if (t < DK) {
         if (tb) rec_tok16[(size_t)a.n * EF + t] = khat;
         else rec_ent[(size_t)E * EF + t] = kk / gt;
-        if (KDA) rec_gam[t] = gt;
-        else if (t == 0) rec_gam[0] = gt;
+        if (KDA) {
+            rec_gam[t] = gt;
+            rec_sig[t] = sg;
+        } else if (t == 0) {
+            rec_gam[0] = gt;
+            rec_sig[0] = sg;
+        }
     }
 }
 
@@ -539,7 +595,7 @@ constexpr int kFlushChunk = 8;   // entries per staged chunk: one TF32 MMA K-blo
 
 template <int DK, int DV>
 struct FlushSmem {
-    float k[DK], ke[DK], q[DK], gam[DK];
+    float k[DK], ke[DK], q[DK], gam[DK], sig[DK];
     float u[DV];
     float kqw[kFlushWarps];
     int map[DK];
@@ -599,7 +655,8 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
     unsigned char *rec = a.rec + (size_t)head * L.rec_bytes;
     float *rec_ent = reinterpret_cast<float *>(rec + L.off_ent);
     const uint16_t *rec_tok16 = reinterpret_cast<const uint16_t *>(rec + L.off_tok);
-    float *rec_gam = reinterpret_cast<float *>(rec + L.off_gam);
+    float *rec_gam = reinterpret_cast<float *>(rec + L.off_gam);   // G
+    float *rec_sig = rec_gam + (KDA ? DK : 1);                       // sigma
     const size_t hv = (size_t)b * a.H + h;
     constexpr bool tb = TB;   // buffered tokens in BF16
     // element x of entry e (e < r: a compensator, else buffered token e - r)
@@ -621,20 +678,29 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
     }
     float kqp = 0.f;
     if (t < DK) {
+        // the buffer is keyed to G and the quantized state scaled by sigma G
+        // (decay guard); the tile is G [sigma Deq + entries], times this
+        // step's decay for a window-end token (a product: it may underflow)
         const float gp = a.n > 0 ? (KDA ? rec_gam[t] : rec_gam[0]) : 1.0f;
+        const float sp = a.n > 0 ? (KDA ? rec_sig[t] : rec_sig[0]) : 1.0f;
         float gt = gp;
         if (MODE == kFlushStep) {
             const size_t qk = ((size_t)b * a.Hk + g) * DK;
             const float kk = a.k[qk + t], qq = a.q[qk + t];
-            gt = (KDA ? a.alpha[hv * DK + t] : a.alpha[hv]) * gp;
-            // the key of the update the state takes: k, or Gamma bf16(k / Gamma)
-            const float ke = tb ? gt * bf16_round(kk / gt) : kk;
+            const float at = KDA ? a.alpha[hv * DK + t] : a.alpha[hv];
+            gt = at * gp;
+            // the key of the update the state takes: k, or G bf16(k / G) with
+            // the guarded G a buffering step would key this token to
+            float rho;
+            const float gc = gate_chain(at, gp, rho);
+            const float ke = tb ? gc * bf16_round(kk / gc) : kk;
             F.k[t] = kk;
             F.ke[t] = ke;
             F.q[t] = qq;
             kqp = ke * qq;
         }
         F.gam[t] = gt;
+        F.sig[t] = sp;
     }
     kqp = warp_sum(kqp);
     if (lane == 0) F.kqw[warp] = kqp;
@@ -818,7 +884,7 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
                                    reinterpret_cast<const float *>(stage + L.off_s),
                                    reinterpret_cast<const uint16_t *>(stage + L.off_hp),
                                    reinterpret_cast<const int8_t *>(stage + L.off_codes), P, DAMP ? F.map : nullptr,
-                                   !DAMP);
+                                   !DAMP, F.sig);
     const bool fin = tile_gamma<DK, DV, NT>(R, F.gam);
     if (!fin) atomicOr(a.status, kStatusNonFinite);
 
@@ -896,9 +962,13 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
     double eacc[T::RPT];
     codec_quantize<DK, DV, false, NT, BITS>(R, L.r, a.K, a.smoothing, P, DAMP ? F.map : nullptr, F.cs, out, eacc);
     if (KDA) {
-        if (t < DK) rec_gam[t] = 1.0f;
+        if (t < DK) {
+            rec_gam[t] = 1.0f;
+            rec_sig[t] = 1.0f;
+        }
     } else if (t == 0) {
         rec_gam[0] = 1.0f;
+        rec_sig[0] = 1.0f;
     }
 }
 

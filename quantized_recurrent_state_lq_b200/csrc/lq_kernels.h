@@ -42,7 +42,7 @@ struct QPtrs {
     unsigned char *s;     size_t s_hs;
     unsigned char *ck;    size_t ck_hs; int ck_js;
     unsigned char *cw;    size_t cw_hs; int cw_js;
-    unsigned char *gam;   size_t gam_hs; int gam_n;   // set to 1 after writing (may be null)
+    unsigned char *gam;   size_t gam_hs; int gam_n;   // decay guard (G, sigma): set to 1 after writing (may be null)
 };
 
 struct CodecArgs {
@@ -55,7 +55,7 @@ struct CodecArgs {
     QPtrs q;              // destination (quantize) or source (dequantize)
     QPtrs q2;             // second target for copies (view <-> record)
     int *status;
-    // DAMP selection
+    // DAMP selection and the static-scale fit's row weights
     int n_states, n_gate_samples, gate_per_channel;
     const float *gates;   // [n_gate_samples][H][1 or dk]
     double *energy;       // [H][dk]
@@ -88,10 +88,11 @@ cudaError_t launch_quantize(const CodecArgs &a, int dk, int dv, int heads, cudaS
 cudaError_t launch_dequantize(const CodecArgs &a, int dk, int dv, int heads, cudaStream_t s);
 cudaError_t launch_qcopy(const CodecArgs &a, int dk, int dv, int heads, cudaStream_t s);
 cudaError_t launch_damp_select(const CodecArgs &a, int dk, int dv, cudaStream_t s);
-cudaError_t launch_fit_static(const CodecArgs &a, int dk, int dv, int n, const double *weight, float *m,
-                              float *sc, cudaStream_t s);
+cudaError_t launch_fit_static(const CodecArgs &a, int dk, int dv, int n, float *m, float *sc, cudaStream_t s);
 
 cudaError_t launch_div_selftest(const float *a, const float *b, float *fast, float *pair, float *ieee, int n,
                                 cudaStream_t s);
+cudaError_t launch_wait_selftest(const unsigned char *src, int *status, unsigned long long limit_ns,
+                                 cudaStream_t s);
 
 }  // namespace lq

@@ -104,15 +104,16 @@ __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.
 
 // x = big + small with big, small representable in TF32: big = x rounded to
 // nearest (ties away from zero) at TF32's 10 stored mantissa bits -- add half a
-// TF32 unit to the bit pattern, clear the 13 low bits -- the rest x - big
-// (exact) truncated to TF32.  Integer and FP32 ALU operations only (the
-// conversion instruction runs at a lower rate); the three products
-// big*big + big*small + small*big of a 3-pass TF32 MMA carry about 22 bits of
-// each operand.  (Finite x below the FP32 maximum; no operand here comes close.)
+// TF32 unit to the bit pattern, clear the 13 low bits -- and small the rest
+// x - big (exact) rounded the same way, so |x - big - small| <= 2^-22 |x|.
+// Integer and FP32 ALU operations only (the conversion instruction runs at a
+// lower rate); the three products big*big + big*small + small*big of a 3-pass
+// TF32 MMA carry about 22 bits of each operand.  (Finite x below the FP32
+// maximum; no operand here comes close.)
 __device__ __forceinline__ void tf32_split(float x, uint32_t &big, uint32_t &small) {
     big = (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
     const float rest = x - __uint_as_float(big);
-    small = __float_as_uint(rest) & 0xFFFFE000u;
+    small = (__float_as_uint(rest) + 0x1000u) & 0xFFFFE000u;
 }
 
 }  // namespace lq

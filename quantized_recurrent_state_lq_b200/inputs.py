@@ -82,6 +82,32 @@ def token_inputs(wl: Workload, T: int, *, stream: str = "decode", chunk: int = 0
             "beta": beta.contiguous(), "alpha": alpha.contiguous()}
 
 
+def strong_decays(shape, mu: float, seed: int, device="cpu") -> torch.Tensor:
+    """Decays exp(-softplus(N(mu, 0.5))) of the given shape (per key channel
+    for KDA): mu = -1 is the strongest end of the KDA workload's range."""
+    g = torch.Generator().manual_seed(seed)
+    z = torch.randn(tuple(shape), generator=g, dtype=torch.float32) * 0.5 + mu
+    return torch.exp(-torch.nn.functional.softplus(z)).to(device)
+
+
+def with_vanishing_decays(alpha: torch.Tensor, seed: int, n: int = 6) -> torch.Tensor:
+    """A copy of decays alpha [T, B, H] or [T, B, H, dk] with n seeded tokens'
+    decays set to 1e-30 (even tokens) or exactly 0 (odd): one key channel of
+    them for KDA, and for KDA every channel of the middle token at 1e-30."""
+    a = alpha.clone()
+    T = a.shape[0]
+    g = torch.Generator().manual_seed(seed)
+    for t in torch.randperm(T, generator=g)[:n].tolist():
+        val = 0.0 if t % 2 else 1e-30
+        if a.dim() == 4:
+            a[t, ..., int(torch.randint(a.shape[-1], (1,), generator=g))] = val
+        else:
+            a[t] = val
+    if a.dim() == 4:
+        a[T // 2] = 1e-30
+    return a
+
+
 def outlier_spec(wl: Workload) -> dict:
     """Outlier key rows / value columns per head and their factors (CPU tensors).
 

@@ -34,7 +34,7 @@ EXPORTED = ["lq_workspace_bytes", "lq_config_check", "lq_state_init", "lq_decode
             "lq_state_export_view", "lq_state_import_view", "lq_quantize_state",
             "lq_dequantize_state", "lq_quantize_state_static", "lq_damp_select", "lq_get_status",
             "lq_state_destroy", "lq_strerror", "lq_selftest_division", "lq_prefill",
-            "lq_state_init_static", "lq_fit_static_scales"]
+            "lq_state_init_static", "lq_fit_static_scales", "lq_selftest_wait"]
 
 
 class LqError(RuntimeError):
@@ -88,7 +88,8 @@ def lib():
             "lq_selftest_division": (C.c_int, [vp, vp, vp, vp, vp, i32, vp]),
             "lq_prefill": (C.c_int, [cfgp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
             "lq_state_init_static": (C.c_int, [C.POINTER(vp), cfgp, vp, sz, vp, vp, vp, vp]),
-            "lq_fit_static_scales": (C.c_int, [cfgp, i32, vp, vp, vp, vp, vp]),
+            "lq_fit_static_scales": (C.c_int, [cfgp, i32, vp, i32, vp, vp, vp, vp]),
+            "lq_selftest_wait": (C.c_int, [vp, C.c_int64, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -246,18 +247,22 @@ def lq_state_init(cfg: Config, S0: torch.Tensor, hp_rows=None, workspace: torch.
     return LqState(cfg, h.value, workspace, rows)
 
 
-def lq_fit_static_scales(cfg: Config, states: torch.Tensor, row_weight: torch.Tensor | None = None,
+def lq_fit_static_scales(cfg: Config, states: torch.Tensor, gates: torch.Tensor | None = None,
                          stream=None) -> tuple[torch.Tensor, torch.Tensor]:
     """Static scales (smoothing 2) of every head from calibration states
-    [n, H, dk, dv]; row_weight [H, dk] float64 or None.  Returns (m [H, dk],
-    s [H, dv])."""
+    [n, H, dk, dv]; gates [n_samples, H, 1 | dk] (the calibration decays that
+    weight the rows by their persistence) or None (unweighted).  Returns
+    (m [H, dk], s [H, dv])."""
     n = states.shape[0]
     p_st = _dev(states, "states", (n, cfg.H, cfg.dk, cfg.dv))
-    p_w = _dev(row_weight, "row_weight", (cfg.H, cfg.dk), torch.float64) if row_weight is not None else None
+    ng, p_g = 0, None
+    if gates is not None:
+        ng = gates.shape[0]
+        p_g = _dev(gates, "gates", (ng, cfg.H, cfg.dk if cfg.gate == "kda" else 1))
     m = torch.empty((cfg.H, cfg.dk), device=states.device)
     s = torch.empty((cfg.H, cfg.dv), device=states.device)
-    _chk(lib().lq_fit_static_scales(C.byref(cfg.c()), C.c_int32(n), C.c_void_p(p_st), C.c_void_p(p_w),
-                                    C.c_void_p(m.data_ptr()), C.c_void_p(s.data_ptr()),
+    _chk(lib().lq_fit_static_scales(C.byref(cfg.c()), C.c_int32(n), C.c_void_p(p_st), C.c_int32(ng),
+                                    C.c_void_p(p_g), C.c_void_p(m.data_ptr()), C.c_void_p(s.data_ptr()),
                                     C.c_void_p(_stream(stream))), "lq_fit_static_scales")
     return m, s
 
@@ -376,6 +381,12 @@ def lq_damp_select(cfg: Config, states: torch.Tensor, gates: torch.Tensor, energ
     pr = _dev(rows, "rows", (cfg.H, cfg.n_hp_rows), torch.int32)
     _chk(lib().lq_damp_select(C.byref(cfg.c()), n, C.c_void_p(ps), ng, C.c_void_p(pg), C.c_void_p(pe),
                               C.c_void_p(pr), C.c_void_p(_stream(stream))), "lq_damp_select")
+
+
+def lq_selftest_wait(st: LqState, limit_ns: int = 1_000_000, stream=None):
+    """Make one bounded device wait run out on purpose (failure-detection self-test)."""
+    _chk(lib().lq_selftest_wait(st.handle, C.c_int64(limit_ns), C.c_void_p(_stream(stream))),
+         "lq_selftest_wait")
 
 
 def lq_get_status(st: LqState, stream=None) -> int:

@@ -90,20 +90,17 @@ def static_scales(wl: Workload, n: int = 8, tokens: int | None = None, device="c
     """Offline fit of fixed key-row / value-column scales (smoothing 2) on the
     GPU: n calibration prefills of the workload's prefill length (calibration
     draws, the workload's outliers), rows weighted by their decay persistence
-    1 / (1 - mean gate) (per key channel for KDA; one value per head for GDN),
-    then lq_fit_static_scales.  Returns (m [H, dk], s [H, dv]) on the device."""
+    (lq_fit_static_scales forms it from the calibration decays: per key channel
+    for KDA, one value per head for GDN).  Returns (m [H, dk], s [H, dv]) on
+    the device."""
     T = wl.prefill if tokens is None else tokens
     states, _ = gpu_prefill(wl, tokens=T, batch=n, stream="calib", device=device)
     states = gen.apply_outliers(states, wl).contiguous()
     tok = gen.token_inputs(wl, min(T, 256), stream="calib", batch=n, device=device)
-    a = tok["alpha"].double()
-    mean = a.mean(dim=(0, 1))                                      # [H] or [H, dk]
-    if wl.gate != "kda":
-        mean = mean[:, None].expand(wl.H, wl.dk)
-    weight = (1.0 / (1.0 - mean)).contiguous()
+    gates = tok["alpha"].reshape(-1, wl.H, wl.dk if wl.gate == "kda" else 1).contiguous()
     cfg = lq.Config(B=1, H=wl.H, Hk=wl.H, dk=wl.dk, dv=wl.dv, gate=wl.gate, r=wl.r, power_iters=wl.K,
                     state_bits=wl.bits, smoothing=2)
-    return lq.lq_fit_static_scales(cfg, states, row_weight=weight)
+    return lq.lq_fit_static_scales(cfg, states, gates=gates)
 
 
 class WindowRunner:

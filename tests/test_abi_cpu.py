@@ -55,7 +55,8 @@ def test_workspace_size_matches_record_layout(L):
     wl = configs.KDA_B256
     cfg = lq.Config.from_workload(wl)
     dk, dv, r, W = wl.dk, wl.dv, wl.r, wl.W
-    payload = (dk * dv) + 4 * (dk + dv) + 4 * (r + W) * (dk + dv) + 4 * dk
+    # codes, m and s, entries, and the decay guard's G and sigma per key channel
+    payload = (dk * dv) + 4 * (dk + dv) + 4 * (r + W) * (dk + dv) + 2 * 4 * dk
     per_head = (lq.lq_workspace_bytes(cfg) - 256) / wl.heads
     assert payload <= per_head <= payload + 128 + 64
     fp = lq.Config.from_workload(wl, mode="fp32")
@@ -134,6 +135,10 @@ def test_null_handles_and_pointers(L):
     assert L.lq_window_flush(None, None) == lq.LQ_ERR_INVALID_ARG
     assert L.lq_state_export_fp32(None, C.c_void_p(16), None) == lq.LQ_ERR_INVALID_ARG
     assert L.lq_get_status(None, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_selftest_wait(None, 1000000, None) == lq.LQ_ERR_INVALID_ARG
+    fake = C.c_void_p(0x7f0000000000)    # never dereferenced: the limit is checked first
+    assert L.lq_selftest_wait(fake, 999, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_selftest_wait(fake, 2000000000, None) == lq.LQ_ERR_INVALID_ARG
     assert L.lq_state_buffered(None) == 0
     L.lq_state_destroy(None)
     cfg = lq.Config.from_workload(configs.TINY_GDN)
@@ -297,10 +302,12 @@ def test_static_scales_config(L):
     assert L.lq_quantize_state(C.byref(c.c()), p, None, None, None) in (lq.LQ_ERR_INVALID_ARG,
                                                                       lq.LQ_ERR_UNSUPPORTED)
     # the fit's argument checks
-    assert L.lq_fit_static_scales(C.byref(c.c()), C.c_int32(0), p, None, p, p, None) == lq.LQ_ERR_INVALID_ARG
-    assert L.lq_fit_static_scales(C.byref(c.c()), C.c_int32(4), p, C.c_void_p(260), p, p, None) == \
-        lq.LQ_ERR_INVALID_ARG
-    assert L.lq_fit_static_scales(C.byref(d.c()), C.c_int32(4), p, None, p, p, None) == lq.LQ_ERR_UNSUPPORTED
+    fit = lambda cfg, n, ng, g: L.lq_fit_static_scales(C.byref(cfg.c()), C.c_int32(n), p, C.c_int32(ng), g, p, p,
+                                                       None)
+    assert fit(c, 0, 0, None) == lq.LQ_ERR_INVALID_ARG
+    assert fit(c, 4, 8, C.c_void_p(258)) == lq.LQ_ERR_INVALID_ARG      # misaligned decays
+    assert fit(c, 4, 0, p) == lq.LQ_ERR_INVALID_ARG                    # decays without samples
+    assert fit(d, 4, 0, None) == lq.LQ_ERR_UNSUPPORTED
 
 
 def test_profiled_source_hash_ignores_comments_only():
@@ -329,3 +336,29 @@ def test_binding_constants_match_the_header():
     body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
     fields = [f.strip() for decl in re.findall(r"int32_t ([^;]+);", body) for f in decl.split(",")]
     assert fields == [n for n, _ in lq.lq_config._fields_]
+
+
+def test_static_quantize_checks_match_the_allocating_call(L):
+    """lq_quantize_state_static returns the same status as lq_quantize_state
+    for the same bad arguments (its checks run in the same order), before any
+    device access; fake device addresses are never touched."""
+    base = lq.Config.from_workload(configs.GDN_SERVING)
+    good_view = lq.lq_qstate_view(*([C.c_void_p(0x7f0000000000)] * 6))
+    bad_view = lq.lq_qstate_view(None, None, None, None, None, None)
+    S = C.c_void_p(0x7f1000000000)
+    cases = []
+    c = lq.Config(**base.__dict__)
+    c.smoothing = 2
+    cases += [(c, bad_view, S), (c, good_view, S)]
+    c = lq.Config(**base.__dict__)
+    cases += [(c, bad_view, S), (c, good_view, C.c_void_p(0x7f1000000004)), (c, good_view, None)]
+    c = lq.Config(**base.__dict__)
+    c.dk = 96
+    cases += [(c, good_view, S)]
+    c = lq.Config(**base.__dict__)
+    c.B = 0
+    cases += [(c, good_view, S)]
+    for cfg, view, s in cases:
+        a = L.lq_quantize_state(C.byref(cfg.c()), s, None, C.byref(view), None)
+        b = L.lq_quantize_state_static(C.byref(cfg.c()), s, None, C.byref(view), None)
+        assert a == b != lq.LQ_OK, (cfg.__dict__, a, b)

@@ -16,7 +16,6 @@ pytestmark = pytest.mark.gpu
 
 OUT_REL = 1e-3     # outputs: max relative error per output vector (b, h, t)
 STATE_REL = 1e-3   # FP32 state: max relative error per head
-TIE_EPS = 1e-3     # a flip this close to a rounding tie is counted as "at a tie"
 
 
 def _workload(gate, B, H, Hk, dk, dv, W, r, seed, P=0, bf16=0, bits=8):
@@ -58,9 +57,11 @@ def test_fp32_mode_matches_oracle(gate, B, H, Hk, dk, dv):
     assert serr.max() < STATE_REL
 
 
-def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=None):
+def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=None, alpha=None):
+    flip_frac = U.LONG_ACCUMULATION_FLIP_FRAC if wl.W >= 200 else U.FLUSH_FLIP_FRAC
     """Run T tokens window by window; each window starts from the oracle's view.
-    static = (m [H, dk], s [H, dv]) numpy arrays: fixed scales (smoothing 2)."""
+    static = (m [H, dk], s [H, dv]) numpy arrays: fixed scales (smoothing 2).
+    alpha(tok): replaces the generator's decays (a device tensor of their shape)."""
     if static is not None:
         smoothing = 2
     cfg = lq.Config.from_workload(wl, mode=mode, fused_flush=int(fused), smoothing=smoothing)
@@ -71,6 +72,8 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=N
     nh = wl.B * wl.H
     S0 = U.prefill_state(wl, 64)
     tok = gen.token_inputs(wl, T, device="cuda")
+    if alpha is not None:
+        tok["alpha"] = alpha(tok).contiguous()
     ph = O.per_head_inputs(tok, wl.H)
     oc = U.ocfg(cfg)
     if static is None:
@@ -90,7 +93,8 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=N
         for k in ov:
             ov[k][h][...] = np.asarray(q[k]).reshape(ov[k][h].shape)
     W = cfg.W
-    stats = {"out": 0.0, "state": 0.0, "flips": 0, "codes": 0, "at_tie": 0}
+    stats = {"out": 0.0, "state": 0.0, "flips": 0, "codes": 0, "band_used": 0.0, "bound_used": 0.0,
+             "flips_bf16_tie": 0, "undetermined": 0}
     o = torch.empty((wl.B, wl.H, wl.dv), device="cuda")
     t0 = 0
     while t0 < T:
@@ -98,13 +102,15 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=N
         sl = {k: v[t0:t0 + n] for k, v in ph.items()}
         ref = O.run(oc, sl, view=ov, hp_rows=hr, flush_last=(n == W))   # oc: all heads' fixed scales
         lq.lq_state_import_view(st, U.oracle_view_to_gpu(cfg, ov, rows))
+        S_g = None
         for t in range(n):
             last = t == n - 1
             if last and n == W and not fused and mode == "window":
                 lq.lq_decode_step(st, *U.step_args(tok, t0 + t), o)
                 S = torch.empty((wl.B, wl.H, wl.dk, wl.dv), device="cuda")
                 lq.lq_state_export_fp32(st, S)
-                e = U.rel_inf_rows(S.cpu().numpy().reshape(nh, -1), ref["S_pre"].reshape(nh, -1))
+                S_g = S.cpu().numpy().reshape(nh, wl.dk, wl.dv).astype(np.float64)
+                e = U.rel_inf_rows(S_g.reshape(nh, -1), ref["S_pre"].reshape(nh, -1))
                 stats["state"] = max(stats["state"], float(e.max()))
                 lq.lq_window_flush(st)
             else:
@@ -117,11 +123,33 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=N
             lq.lq_state_export_view(st, gv)
             got = U.gpu_view_to_oracle(cfg, gv, rows)
             ratio = U.oracle_ratios(cfg, ref["S_pre"].astype(np.float32), hr, head_cfg=head_cfg)
-            c = U.compare_codes(got["codes"], ref["view"]["codes"], ratio, TIE_EPS)
-            assert c["max_diff"] <= 1, f"{label}: window {t0 // W}: {c}"
-            stats["flips"] += c["n"]
-            stats["codes"] += c["total"]
-            stats["at_tie"] += c["at_tie"]
+            for h in range(nh):
+                hrh = None if hr is None else hr[h]
+                # the GPU's pre-flush FP32 state: measured (separate flush) or
+                # bounded from the arithmetic that forms it (flush fused into
+                # the W-th step); the measured difference must obey the bound
+                bound, risk = U.window_state_bound(head_cfg(h), U.head_view(ov, h),
+                                                   {k: v[:, h] for k, v in sl.items()}, hp_rows=hrh, risk_cols=True)
+                if S_g is not None:
+                    dS = np.abs(S_g[h] - ref["S_pre"][h])
+                    used = float((dS / bound).max())
+                    assert used <= 1.0, f"{label}: head {h}: pre-flush state error above its bound ({used:.2f})"
+                    stats["bound_used"] = max(stats["bound_used"], used)
+                else:
+                    dS = bound
+                c = U.check_quantized(head_cfg(h), U.head_view(got, h), U.head_view(ref["view"], h), ratio[h],
+                                      ref["S_pre"][h], dS, hp_rows=hrh, label=f"{label} window {t0 // W} head {h}",
+                                      risk_cols=risk)
+                if risk.any():
+                    # a buffered u at a BF16 rounding tie moves its column of
+                    # the state by a BF16 step, and through the compensators
+                    # every column: the window's flips are that tie's
+                    c = dict(c, n=0, n_risk=c["n"] + c["n_risk"])
+                stats["flips"] += c["n"]
+                stats["flips_bf16_tie"] += c["n_risk"]
+                stats["undetermined"] += c["n_undetermined"]
+                stats["codes"] += c["total"]
+                stats["band_used"] = max(stats["band_used"], c["band_used"])
             U.assert_flush_params(cfg, got, ref["view"], ref["S_pre"], hr, label, rel=STATE_REL)
             scale = np.abs(ref["S_pre"]).max(axis=(1, 2))
             for j in range(cfg.r):
@@ -141,11 +169,12 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=N
         ov = ref["view"]
         t0 += n
     assert lq.lq_get_status(st) == lq.LQ_OK
-    print(f"{label}: out {stats['out']:.2e} state {stats['state']:.2e} "
-          f"flips {stats['flips']}/{stats['codes']} ({stats['at_tie']} at ties)")
+    print(f"{label}: out {stats['out']:.2e} state {stats['state']:.2e} (bound used {stats['bound_used']:.2f}) "
+          f"flips {stats['flips']}/{stats['codes']} (band used {stats['band_used']:.2f}; "
+          f"{stats['flips_bf16_tie']} in BF16-tie columns, {stats['undetermined']} undetermined)")
     assert stats["out"] < OUT_REL
     assert stats["state"] < STATE_REL
-    U.assert_code_bar({"n": stats["flips"], "total": stats["codes"], "max_diff": 0}, label, U.FLUSH_FLIP_FRAC)
+    U.assert_code_bar({"n": stats["flips"], "total": stats["codes"]}, label, flip_frac)
     return stats
 
 
@@ -164,6 +193,37 @@ def test_windowed_teacher_forced(fused, gate, B, H, Hk, dk, dv, W, r):
     wl = _workload(gate, B, H, Hk, dk, dv, W, r, seed=31 + W)
     T = 3 * W + W // 2   # three windows and a ragged tail
     _teacher_forced(wl, T, fused, label=f"window {gate} d{dk}x{dv} W{W} r{r} fused{int(fused)}")
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("gate,H,W,bf16,mu", [
+    ("kda", 2, 512, 0, -1.0),     # strong channels: Gamma passes 2^-64 every ~110 tokens
+    ("kda", 2, 4096, 0, -1.0),    # the longest window: 2^-1900 by its end
+    ("kda", 2, 320, 1, -1.0),     # BF16 buffer: keys rounded against the guarded chain
+    ("gdn", 2, 4096, 0, None),    # the benchmark's GDN decays: Gamma ~2^-180 by the end
+])
+def test_long_windows_strong_decays(fused, gate, H, W, bf16, mu):
+    """Decay products far below the FP32 range within a window (the decay
+    guard of the buffering and flush kernels): outputs and the flushed state
+    against the oracle, which decays its double state directly."""
+    U.require_gpu()
+    wl = _workload(gate, 1, H, H, 128, 128, W, 4, seed=81 + W + bf16, bf16=bf16)
+    T = W + 3
+    dec = None if mu is None else (lambda tok: gen.strong_decays(tok["alpha"].shape, mu, 7, device="cuda"))
+    st = _teacher_forced(wl, T, fused, alpha=dec,
+                         label=f"long window {gate} W{W} bf16{bf16} fused{int(fused)}")
+    assert st["out"] < OUT_REL
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("gate,bf16", [("gdn", 0), ("kda", 0), ("kda", 1), ("gdn", 1)])
+def test_vanishing_decays(fused, gate, bf16):
+    """Decays of 1e-30 and exactly 0 inside a window: the channel (or head)
+    restarts, nothing overflows, outputs and flushes match the oracle."""
+    U.require_gpu()
+    wl = _workload(gate, 2, 2, 2, 128, 128, 16, 4, seed=91 + bf16, bf16=bf16)
+    _teacher_forced(wl, 2 * 16 + 5, fused, alpha=lambda tok: gen.with_vanishing_decays(tok["alpha"], 5),
+                    label=f"vanishing decays {gate} bf16{bf16} fused{int(fused)}")
 
 
 @pytest.mark.parametrize("fused", [False, True])
@@ -255,38 +315,75 @@ def test_free_running_tiny_workload():
     assert lq.lq_get_status(st) == lq.LQ_OK
 
 
+def _check_flush_vs_oracle(cfg, st, S_g, ref, ov_start, toks, label):
+    """The GPU state's view after a flush against the oracle's (`ref` from
+    O.run with flush_last), with the GPU's exported pre-flush state S_g [nh,
+    dk, dv]: the state within its derived bound, then the codes, scales and
+    compensators by check_quantized and the window-start state bar."""
+    oc = U.ocfg(cfg)
+    nh = cfg.B * cfg.H
+    gv = lq.alloc_view(cfg)
+    lq.lq_state_export_view(st, gv)
+    got = U.gpu_view_to_oracle(cfg, gv, None)
+    ratio = U.oracle_ratios(cfg, ref["S_pre"].astype(np.float32), None)
+    flips = total = 0
+    for h in range(nh):
+        bound = U.window_state_bound(oc, U.head_view(ov_start, h), {k: v[:, h] for k, v in toks.items()})
+        dS = np.abs(S_g[h] - ref["S_pre"][h])
+        assert (dS <= bound).all(), f"{label}: pre-flush state above its bound"
+        c = U.check_quantized(oc, U.head_view(got, h), U.head_view(ref["view"], h), ratio[h], ref["S_pre"][h], dS,
+                              label=f"{label} head {h}")
+        flips += c["n"]
+        total += c["total"]
+    U.assert_code_bar({"n": flips, "total": total}, label)
+    U.assert_flush_params(cfg, got, ref["view"], ref["S_pre"], None, label, rel=STATE_REL)
+
+
 def test_partial_window_flush_and_window_full():
+    """A full window, the call past it (refused), a flush; then two tokens and
+    a flush of the partial window (teacher-forced: the second window starts
+    from the oracle's view).  Each flush is held to the per-window bars."""
     U.require_gpu()
     wl = _workload("gdn", 1, 2, 2, 128, 128, 4, 2, seed=50)
     cfg = lq.Config.from_workload(wl, fused_flush=0)
     S0 = torch.from_numpy(U.prefill_state(wl, 32)).cuda()
     tok = gen.token_inputs(wl, 8, device="cuda")
+    oc = U.ocfg(cfg)
+    ph = O.per_head_inputs(tok, 2)
+    ov0 = O.empty_views(oc, 2)
+    for h in range(2):
+        q = O.quantize(oc, S0.cpu().numpy().reshape(2, 128, 128)[h])
+        for k in ov0:
+            ov0[k][h][...] = np.asarray(q[k]).reshape(ov0[k][h].shape)
     st = lq.lq_state_init(cfg, S0)
+    lq.lq_state_import_view(st, U.oracle_view_to_gpu(cfg, ov0, None))
     o = torch.empty((1, 2, 128), device="cuda")
     for t in range(4):
         lq.lq_decode_step(st, *U.step_args(tok, t), o)
     with pytest.raises(lq.LqError) as ei:
         lq.lq_decode_step(st, *U.step_args(tok, 4), o)
     assert ei.value.code == lq.LQ_ERR_WINDOW_FULL
+    Sg = torch.empty_like(S0)
+    lq.lq_state_export_fp32(st, Sg)
     lq.lq_window_flush(st)
     assert lq.lq_state_buffered(st) == 0
+    w1 = {k: v[:4] for k, v in ph.items()}
+    a = O.run(oc, w1, view=ov0, flush_last=True)
+    _check_flush_vs_oracle(cfg, st, Sg.cpu().numpy().reshape(2, 128, 128).astype(np.float64), a, ov0, w1,
+                           "full window")
+    # the second window starts from the oracle's view; two tokens, then a flush
+    lq.lq_state_import_view(st, U.oracle_view_to_gpu(cfg, a["view"], None))
     lq.lq_decode_step(st, *U.step_args(tok, 4), o)
     lq.lq_decode_step(st, *U.step_args(tok, 5), o)
     assert lq.lq_state_buffered(st) == 2
-    # oracle: window of 4, flush, then 2 tokens and a flush after 2
-    oc = U.ocfg(cfg)
-    ph = O.per_head_inputs(tok, 2)
-    a = O.run(oc, {k: v[:4] for k, v in ph.items()}, S0=S0.cpu().numpy().reshape(2, 128, 128), flush_last=True)
-    b = O.run(O.Cfg(**{**oc.__dict__, "W": 2}), {k: v[4:6] for k, v in ph.items()}, view=a["view"],
-              flush_last=True)
+    lq.lq_state_export_fp32(st, Sg)
     lq.lq_window_flush(st)
-    S = torch.empty_like(S0)
-    lq.lq_state_export_fp32(st, S)
-    deq = np.stack([O.dequantize(oc, {k: b["view"][k][h] for k in b["view"]}) for h in range(2)])
-    err = U.rel_inf_rows(S.cpu().numpy().reshape(2, -1), deq.reshape(2, -1))
-    # every window boundary may flip a few codes; compare within a few LSB-sized steps
-    assert err.max() < 2e-2, err
+    w2 = {k: v[4:6] for k, v in ph.items()}
+    b = O.run(O.Cfg(**{**oc.__dict__, "W": 2}), w2, view=a["view"], flush_last=True)
+    _check_flush_vs_oracle(cfg, st, Sg.cpu().numpy().reshape(2, 128, 128).astype(np.float64), b, a["view"], w2,
+                           "partial window")
     lq.lq_window_flush(st)   # nothing buffered: no-op
+    assert lq.lq_state_buffered(st) == 0
     assert lq.lq_get_status(st) == lq.LQ_OK
 
 

@@ -104,8 +104,9 @@ def test_full_size_kda_prefill_sampled_heads():
     over all 8192 heads in the runner's launch configuration, 4 sampled heads
     against the oracle's recurrence; then the quantized state the decode
     starts from (lq_state_init of the result) against the oracle's quantizer
-    on the oracle's state -- codes within the flush bar (the inputs differ by
-    the prefill's rounding)."""
+    on the oracle's state -- every differing code at a rounding tie within the
+    band the measured difference of the two input states allows, and their
+    count within the bar for states accumulated over long inputs."""
     U.require_gpu()
     wl = configs.KDA_B256
     heads = [(0, 0), (17, 5), (128, 31), (255, 16)]
@@ -126,9 +127,11 @@ def test_full_size_kda_prefill_sampled_heads():
     gv = U.gpu_view_to_oracle(cfg, view, None)
     flips = total = 0
     for i in range(nh):
-        want = O.quantize(U.ocfg(cfg), ref[i].astype(np.float32), want_ratio=True)
-        c = U.compare_codes(gv["codes"][i], want["codes"], want["ratio"], 1e-3)
-        assert c["max_diff"] <= 1
+        S_ref = ref[i].astype(np.float32).astype(np.float64)
+        want = O.quantize(U.ocfg(cfg), S_ref.astype(np.float32), want_ratio=True)
+        c = U.check_quantized(U.ocfg(cfg), U.head_view(gv, i), want, want["ratio"], S_ref,
+                              np.abs(got[i].astype(np.float64) - S_ref), label=f"prefill head {i}")
         flips += c["n"]
         total += c["total"]
-    assert flips <= U.FLUSH_FLIP_FRAC * total + 1, (flips, total)
+    print(f"full-size KDA prefill: quantized {flips}/{total} codes differ")
+    U.assert_code_bar({"n": flips, "total": total}, "prefill", U.LONG_ACCUMULATION_FLIP_FRAC)

@@ -15,29 +15,33 @@ from tests.test_gpu_decode import _teacher_forced, _workload
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("dk,dv,r,bits", [(128, 128, 2, 8), (128, 128, 0, 4), (64, 64, 2, 4), (64, 128, 1, 8),
-                                          (128, 64, 2, 6)])
-def test_fit_matches_oracle(dk, dv, r, bits):
-    """Both sides fit from their own residuals (FP64 compensators): the scales
-    agree exactly but where the residuals' last bits tip a near-tied
-    candidate; there the oracle's objective of the GPU's scales is within 1e-6
-    of its own optimum."""
+@pytest.mark.parametrize("dk,dv,r,bits,gate", [(128, 128, 2, 8, "kda"), (128, 128, 0, 4, "gdn"),
+                                               (64, 64, 2, 4, "kda"), (64, 128, 1, 8, "gdn"),
+                                               (128, 64, 2, 6, "kda")])
+def test_fit_matches_oracle(dk, dv, r, bits, gate):
+    """Both sides fit from their own residuals (FP64 compensators), rows
+    weighted by the decay persistence of seeded calibration decays (the oracle
+    forms it with its DAMP score of unit energies): the scales agree exactly
+    but where the residuals' last bits tip a near-tied candidate; there the
+    oracle's objective of the GPU's scales is within 1e-6 of its own optimum."""
     U.require_gpu()
-    n, H = 6, 3
+    n, H, ng = 6, 3, 40
     states = gen.random_state(n * H, dk, dv, seed=dk + dv + r + bits, n_out=2, out_factor=25.0).reshape(n, H, dk, dv)
-    w = torch.from_numpy(np.random.default_rng(bits).uniform(0.5, 3.0, (H, dk)))
-    cfg = lq.Config(B=1, H=H, Hk=H, dk=dk, dv=dv, r=r, power_iters=8, state_bits=bits)
-    m, s = lq.lq_fit_static_scales(cfg, states.cuda(), row_weight=w.cuda())
+    ga = dk if gate == "kda" else 1
+    gates = gen.strong_decays((ng, H, ga), -3.0, seed=bits + dk)
+    cfg = lq.Config(B=1, H=H, Hk=H, dk=dk, dv=dv, gate=gate, r=r, power_iters=8, state_bits=bits)
+    m, s = lq.lq_fit_static_scales(cfg, states.cuda(), gates=gates.cuda())
     m, s = m.cpu().numpy(), s.cpu().numpy()
     oc = O.Cfg(dk=dk, dv=dv, r=r, K=8, bits=bits)
     exact = total = 0
     for h in range(H):
         st = states[:, h].numpy()
-        want = O.fit_static(oc, st, weight=w[h].numpy())
+        w = O.damp_score(np.ones(dk), gates[:, h, :].numpy())
+        want = O.fit_static(oc, st, weight=w)
         same = np.concatenate([m[h] == want["m"], s[h] == want["s"]])
         exact += int(same.sum())
         total += same.size
-        ours = O.fit_objective(oc, st, m[h], s[h], weight=w[h].numpy())
+        ours = O.fit_objective(oc, st, m[h], s[h], weight=w)
         assert ours <= want["obj"][-1] * (1 + 1e-6), (h, ours, want["obj"][-1])
         assert ours < want["obj"][0]
     print(f"fit d{dk}x{dv} r{r} {bits}-bit: {exact}/{total} scales identical to the oracle's")

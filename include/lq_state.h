@@ -174,12 +174,41 @@ int lq_state_init_static(lq_state **out, const lq_config *cfg, void *d_workspace
 int lq_decode_step(lq_state *st, const float *d_q, const float *d_k, const float *d_v,
                    const float *d_beta, const float *d_alpha, float *d_o, void *stream);
 
+/*
+ * Staggered windows: give every batch entry its own window schedule.  The
+ * LeapQuant project page's window paragraph quantizes a sequence's state once
+ * every W of its tokens; it does not tie the sequences of a batch to common
+ * window ends (in serving they join at different times).  With phases, batch
+ * entry b ends a window at the lq_decode_step calls whose index `since`
+ * (counted from this call, from the last lq_window_flush, from 0) satisfies
+ * (since + h_phase[b]) mod W = W - 1: its first window holds W - h_phase[b]
+ * tokens, every later one W.  A step then ends the windows of the entries of
+ * one phase only, so the window-end work of 1/W of the batch (phases b mod W)
+ * runs beside the buffering of the rest instead of all of it in one step.
+ * The window-end launch goes to a higher-priority stream the state owns,
+ * forked from `stream` and joined back into it with events before the call
+ * returns (stream-ordered: the next call on `stream` sees its results).
+ *
+ * h_phase [B] (HOST): phases in [0, W); NULL removes the phases (common
+ * windows again).  INT8_WINDOW with fused_flush = 1 only, and only while
+ * every entry is at a window start (lq_state_buffered = 0): else
+ * LQ_ERR_UNSUPPORTED; a phase outside [0, W): LQ_ERR_INVALID_ARG.  Copies the
+ * phases into the workspace and synchronizes `stream` once.
+ * With phases, entry b holds min((since + h_phase[b]) mod W, since) tokens;
+ * lq_window_flush ends every entry's window and restarts the schedule
+ * (since = 0); lq_state_buffered returns the most any entry holds;
+ * lq_state_export_view and lq_state_import_view need every entry at a window
+ * start (LQ_ERR_UNSUPPORTED otherwise) and leave the schedule as it is.
+ */
+int lq_state_set_phases(lq_state *st, const int32_t *h_phase, void *stream);
+
 /* End the current window: reconstruct S = Gamma (Deq + comps + buffer) and
  * quantize it (new compensators, smoothing, codes); resets the buffer.  A no-op
  * with nothing buffered and in FP32 / INT8_STEP modes. */
 int lq_window_flush(lq_state *st, void *stream);
 
-/* Tokens buffered in the current window (host counter, no synchronization). */
+/* Tokens buffered in the current window (host counter, no synchronization);
+ * with window phases the most any batch entry holds. */
 int lq_state_buffered(const lq_state *st);
 
 /* Write the exact current state, Gamma (Deq + comps + buffer) in INT8 modes or

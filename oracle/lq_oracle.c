@@ -383,12 +383,16 @@ static void to_float(const double *S, float *F, int n)
  * made); S_pre [nh][dk][dv] (nullable) the state right before the last flush;
  * n_out [nh] the tokens buffered since the last window start.
  * flush_last: flush when the last token completes a window.
+ * phase [nh] (nullable): staggered windows -- head h's first window ends after
+ * W - phase[h] tokens, every later one after W (the page's rule of one
+ * requantization per W tokens of a sequence, with the sequences' window ends
+ * shifted against each other); NULL: every first window holds W tokens.
  */
 void lqo_run(const lqo_cfg *cfg, int nh, const int *hp_rows, int from_view,
              const float *S0, lqo_views *view, int T, const float *q,
              const float *k, const float *v, const float *beta,
              const float *alpha, double *o, double *S_out, double *S_pre,
-             int *n_out, int flush_last, int nthreads)
+             int *n_out, int flush_last, int nthreads, const int *phase)
 {
     const int dk = cfg->dk, dv = cfg->dv, ga = cfg->gate ? dk : 1;
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
@@ -411,6 +415,7 @@ void lqo_run(const lqo_cfg *cfg, int nh, const int *hp_rows, int from_view,
             for (int e = 0; e < dk * dv; ++e) S[e] = (double)S0[(size_t)h * dk * dv + e];
         }
         int n = 0;
+        int len = hcfg->W - (phase ? phase[h] : 0);   /* tokens of the current window */
         float gam[512];
         for (int j = 0; j < ga; ++j) gam[j] = 1.0f;
         for (int t = 0; t < T; ++t) {
@@ -425,12 +430,13 @@ void lqo_run(const lqo_cfg *cfg, int nh, const int *hp_rows, int from_view,
                          alpha + th * ga, o + th * dv);
             }
             n += 1;
-            if (hcfg->quantize && n == hcfg->W && (t < T - 1 || flush_last)) {
+            if (hcfg->quantize && n == len && (t < T - 1 || flush_last)) {
                 if (S_pre) memcpy(S_pre + (size_t)h * dk * dv, S, sizeof(double) * dk * dv);
                 to_float(S, F, dk * dv);
                 lqo_quantize(hcfg, hr, F, &vh, NULL);
                 lqo_dequantize(hcfg, hr, &vh, S);
                 n = 0;
+                len = hcfg->W;
             }
         }
         if (n_out) n_out[h] = n;

@@ -164,8 +164,11 @@ def dequantize(cfg: Cfg, view: dict, hp_rows=None) -> np.ndarray:
 
 
 def run(cfg: Cfg, inputs: dict, *, S0=None, view=None, hp_rows=None,
-        flush_last: bool = False, nthreads: int | None = None) -> dict:
+        flush_last: bool = False, nthreads: int | None = None, phase=None) -> dict:
     """Decode T tokens of nh independent heads.
+
+    phase [nh] (optional): staggered windows, head h's first window holding
+    W - phase[h] tokens (lqo_run).
 
     inputs: q, k [T, nh, dk]; v [T, nh, dv]; beta [T, nh]; alpha [T, nh] or
     [T, nh, dk] (already one entry per value head).  Give S0 [nh, dk, dv] or a
@@ -197,7 +200,8 @@ def run(cfg: Cfg, inputs: dict, *, S0=None, view=None, hp_rows=None,
                   _p(q, C.c_float), _p(k, C.c_float), _p(v, C.c_float),
                   _p(beta, C.c_float), _p(alpha, C.c_float), _p(o, C.c_double),
                   _p(S, C.c_double), _p(S_pre, C.c_double), _p(n, C.c_int),
-                  C.c_int(1 if flush_last else 0), C.c_int(nthreads or os.cpu_count() or 1))
+                  C.c_int(1 if flush_last else 0), C.c_int(nthreads or os.cpu_count() or 1),
+                  _p(_i32(phase), C.c_int) if phase is not None else None)
     if cfg.r == 0:
         views["c"] = views["c"][:, :0]
         views["w"] = views["w"][:, :0]

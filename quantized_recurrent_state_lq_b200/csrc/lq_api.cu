@@ -23,7 +23,18 @@ struct lq_state {
     float *static_ms;   // smoothing 2: [H][dk+dv] fixed key-row and value-column scales
     unsigned char *rec;
     size_t heads;
-    int n;  // tokens buffered in the current window
+    int n;  // tokens buffered in the current window (without window phases)
+    // Window phases (lq_state_set_phases): phase [B] and the batch entries
+    // ordered by phase in the workspace; on the host the phases and, per phase
+    // p, the range h_off[p] .. h_off[p+1] of d_order holding its entries.  The
+    // window-end launches run on `side`, forked from and joined back into the
+    // caller's stream by two events.
+    int phased;
+    long long since;   // steps since the last common window start
+    int *d_phase, *d_order;
+    int *h_phase, *h_off;
+    cudaStream_t side;
+    cudaEvent_t ev_fork, ev_join;
 };
 
 namespace {
@@ -95,6 +106,11 @@ size_t static_bytes(const lq_config *c) {
     return c->smoothing == 2 ? align_sz((size_t)c->H * (c->dk + c->dv) * 4, kAlign) : 0;
 }
 
+// Window mode: the phase array and the phase-ordered batch entries.
+size_t phase_bytes(const lq_config *c) {
+    return c->mode == LQ_MODE_INT8_WINDOW ? align_sz((size_t)2 * c->B * 4, kAlign) : 0;
+}
+
 size_t record_bytes(const lq_config *c) {
     if (is_int8(c)) return (size_t)layout_of(c).rec_bytes;
     return (size_t)c->dk * c->dv * 4;
@@ -164,7 +180,44 @@ lq::DecodeArgs decode_args(const lq_state *st) {
     a.hp_rows = st->hp_rows;
     a.slot_rows = st->slot_rows;
     a.status = st->status;
+    if (st->phased) {
+        const int W = st->L.W;
+        a.phase = st->d_phase;
+        a.n = st->since < W ? (int)st->since : W;
+        a.nmod = (int)(st->since % W);
+    }
     return a;
+}
+
+// Tokens batch entry b holds (every entry without phases).
+int entry_buffered(const lq_state *st, int phase) {
+    if (!st->phased) return st->n;
+    const int W = st->L.W;
+    const long long p = (st->since + phase) % W;
+    return (int)(p < st->since ? p : st->since);
+}
+
+// The most tokens any batch entry holds: 0 iff every entry is at a window start.
+int buffered_max(const lq_state *st) {
+    if (!st->phased) return st->n;
+    int m = 0;
+    for (int p = 0; p < st->L.W; ++p)
+        if (st->h_off[p + 1] > st->h_off[p]) {
+            const int v = entry_buffered(st, p);
+            m = v > m ? v : m;
+        }
+    return m;
+}
+
+void release(lq_state *st) {
+    if (st->side) {
+        cudaEventDestroy(st->ev_fork);
+        cudaEventDestroy(st->ev_join);
+        cudaStreamDestroy(st->side);
+    }
+    free(st->h_phase);
+    free(st->h_off);
+    delete st;
 }
 
 }  // namespace
@@ -175,7 +228,7 @@ int lq_config_check(const lq_config *cfg) { return check_config(cfg); }
 
 size_t lq_workspace_bytes(const lq_config *cfg) {
     if (check_config(cfg) != LQ_OK) return 0;
-    return kAlign + hp_bytes(cfg) + slot_bytes(cfg) + static_bytes(cfg) +
+    return kAlign + hp_bytes(cfg) + slot_bytes(cfg) + static_bytes(cfg) + phase_bytes(cfg) +
            (size_t)cfg->B * cfg->H * record_bytes(cfg);
 }
 
@@ -206,9 +259,16 @@ static int state_init(lq_state **out, const lq_config *cfg, void *d_workspace, s
     st->static_ms = cfg->smoothing == 2
                         ? reinterpret_cast<float *>(st->ws + kAlign + hp_bytes(cfg) + slot_bytes(cfg))
                         : nullptr;
-    st->rec = st->ws + kAlign + hp_bytes(cfg) + slot_bytes(cfg) + static_bytes(cfg);
+    st->d_phase = reinterpret_cast<int *>(st->ws + kAlign + hp_bytes(cfg) + slot_bytes(cfg) + static_bytes(cfg));
+    st->d_order = st->d_phase + cfg->B;
+    st->rec = st->ws + kAlign + hp_bytes(cfg) + slot_bytes(cfg) + static_bytes(cfg) + phase_bytes(cfg);
     st->heads = (size_t)cfg->B * cfg->H;
     st->n = 0;
+    st->phased = 0;
+    st->since = 0;
+    st->h_phase = st->h_off = nullptr;
+    st->side = nullptr;
+    st->ev_fork = st->ev_join = nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // Per head: the key row of every INT8 slot (increasing), then of every BF16 row.
     int32_t *slots = nullptr;
@@ -299,27 +359,122 @@ int lq_decode_step(lq_state *st, const float *d_q, const float *d_k, const float
         a.status = st->status;
         return cuda_rc(lq::launch_fp32_step(a, c.dk, c.dv, (int)st->heads, kda, s));
     }
-    if (st->n >= st->L.W) return LQ_ERR_WINDOW_FULL;
-    const bool flush = (c.mode == LQ_MODE_INT8_STEP) || (c.fused_flush && st->n + 1 == st->L.W);
     lq::DecodeArgs a = decode_args(st);
     a.q = d_q; a.k = d_k; a.v = d_v; a.beta = d_beta; a.alpha = d_alpha; a.o = d_o;
-    const int rc = cuda_rc(lq::launch_decode(a, c.dk, c.dv, (int)st->heads, kda, flush, c.n_hp_rows > 0, s));
+    const bool damp = c.n_hp_rows > 0;
+    if (st->phased) {
+        // The entries whose window ends at this step (phase W - 1 - since mod
+        // W) take the window-end kernel on the side stream, the others the
+        // buffering kernel (which skips the former) on `stream`.
+        const int W = st->L.W;
+        const int rho = W - 1 - a.nmod;
+        const int first = st->h_off[rho], cnt = st->h_off[rho + 1] - first;
+        cudaError_t e = cudaSuccess;
+        if (cnt > 0) {
+            e = cudaEventRecord(st->ev_fork, s);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(st->side, st->ev_fork, 0);
+            lq::DecodeArgs af = a;
+            af.flush_list = st->d_order + first;
+            if (e == cudaSuccess) e = lq::launch_decode(af, c.dk, c.dv, cnt * c.H, kda, true, damp, st->side);
+        }
+        if (e == cudaSuccess && cnt < c.B) e = lq::launch_decode(a, c.dk, c.dv, (int)st->heads, kda, false, damp, s);
+        if (e == cudaSuccess && cnt > 0) {
+            e = cudaEventRecord(st->ev_join, st->side);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(s, st->ev_join, 0);
+        }
+        if (e == cudaSuccess) st->since += 1;
+        return cuda_rc(e);
+    }
+    if (st->n >= st->L.W) return LQ_ERR_WINDOW_FULL;
+    const bool flush = (c.mode == LQ_MODE_INT8_STEP) || (c.fused_flush && st->n + 1 == st->L.W);
+    const int rc = cuda_rc(lq::launch_decode(a, c.dk, c.dv, (int)st->heads, kda, flush, damp, s));
     if (rc == LQ_OK) st->n = flush ? 0 : st->n + 1;
     return rc;
 }
 
+int lq_state_set_phases(lq_state *st, const int32_t *h_phase, void *stream) {
+    if (!st) return LQ_ERR_INVALID_ARG;
+    const lq_config &c = st->cfg;
+    if (c.mode != LQ_MODE_INT8_WINDOW || c.fused_flush != 1) return LQ_ERR_UNSUPPORTED;
+    if (buffered_max(st) > 0) return LQ_ERR_UNSUPPORTED;
+    const int W = st->L.W;
+    if (!h_phase) {
+        st->phased = 0;
+        st->n = 0;
+        return LQ_OK;
+    }
+    for (int b = 0; b < c.B; ++b)
+        if (h_phase[b] < 0 || h_phase[b] >= W) return LQ_ERR_INVALID_ARG;
+    int *ph = static_cast<int *>(malloc((size_t)c.B * sizeof(int)));
+    int *off = static_cast<int *>(calloc((size_t)W + 1, sizeof(int)));
+    int *order = static_cast<int *>(malloc((size_t)c.B * sizeof(int)));
+    if (!ph || !off || !order) {
+        free(ph); free(off); free(order);
+        return LQ_ERR_INVALID_ARG;
+    }
+    // counting sort of the entries by phase
+    for (int b = 0; b < c.B; ++b) {
+        ph[b] = h_phase[b];
+        off[ph[b] + 1] += 1;
+    }
+    for (int p = 0; p < W; ++p) off[p + 1] += off[p];
+    {
+        int *fill = static_cast<int *>(malloc((size_t)W * sizeof(int)));
+        if (!fill) {
+            free(ph); free(off); free(order);
+            return LQ_ERR_INVALID_ARG;
+        }
+        memcpy(fill, off, (size_t)W * sizeof(int));
+        for (int b = 0; b < c.B; ++b) order[fill[ph[b]]++] = b;
+        free(fill);
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (!st->side) {
+        int least = 0, greatest = 0;
+        e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+        if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&st->side, cudaStreamNonBlocking, greatest);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->ev_join, cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaMemcpyAsync(st->d_phase, ph, (size_t)c.B * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(st->d_order, order, (size_t)c.B * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    free(order);
+    if (e != cudaSuccess) {
+        free(ph); free(off);
+        return LQ_ERR_CUDA;
+    }
+    free(st->h_phase);
+    free(st->h_off);
+    st->h_phase = ph;
+    st->h_off = off;
+    st->phased = 1;
+    st->since = 0;
+    st->n = 0;
+    return LQ_OK;
+}
+
 int lq_window_flush(lq_state *st, void *stream) {
     if (!st) return LQ_ERR_INVALID_ARG;
-    if (st->cfg.mode != LQ_MODE_INT8_WINDOW || st->n == 0) return LQ_OK;
+    if (st->cfg.mode != LQ_MODE_INT8_WINDOW) return LQ_OK;
+    if (buffered_max(st) == 0) {
+        st->since = 0;   // (window phases: the schedule restarts all the same)
+        return LQ_OK;
+    }
+    // (window phases: entries with nothing buffered leave the launch at once)
     lq::DecodeArgs a = decode_args(st);
     const int rc = cuda_rc(lq::launch_flush(a, st->cfg.dk, st->cfg.dv, (int)st->heads,
                                             st->cfg.gate == LQ_GATE_CHANNEL, st->cfg.n_hp_rows > 0, false,
                                             static_cast<cudaStream_t>(stream)));
-    if (rc == LQ_OK) st->n = 0;
+    if (rc == LQ_OK) {
+        st->n = 0;
+        st->since = 0;
+    }
     return rc;
 }
 
-int lq_state_buffered(const lq_state *st) { return st ? st->n : 0; }
+int lq_state_buffered(const lq_state *st) { return st ? buffered_max(st) : 0; }
 
 int lq_state_export_fp32(const lq_state *st, float *d_S, void *stream) {
     if (!st || !d_S) return LQ_ERR_INVALID_ARG;
@@ -338,7 +493,7 @@ int lq_state_export_view(const lq_state *st, const lq_qstate_view *out, void *st
     if (!is_int8(&st->cfg)) return LQ_ERR_INVALID_ARG;
     // mid-window the record's compensators may carry the decay guard's
     // rescaling; the window-start view is only whole at a window boundary
-    if (st->n > 0) return LQ_ERR_UNSUPPORTED;
+    if (buffered_max(st) > 0) return LQ_ERR_UNSUPPORTED;
     int rc = check_view(&st->cfg, out);
     if (rc) return rc;
     lq::CodecArgs a{};
@@ -352,6 +507,8 @@ int lq_state_export_view(const lq_state *st, const lq_qstate_view *out, void *st
 int lq_state_import_view(lq_state *st, const lq_qstate_view *in, void *stream) {
     if (!st) return LQ_ERR_INVALID_ARG;
     if (!is_int8(&st->cfg)) return LQ_ERR_INVALID_ARG;
+    // with window phases the schedule goes on: every entry must be at a window start
+    if (st->phased && buffered_max(st) > 0) return LQ_ERR_UNSUPPORTED;
     int rc = check_view(&st->cfg, in);
     if (rc) return rc;
     lq::CodecArgs a{};
@@ -570,7 +727,9 @@ int lq_get_status(lq_state *st, void *stream) {
     return LQ_OK;
 }
 
-void lq_state_destroy(lq_state *st) { delete st; }
+void lq_state_destroy(lq_state *st) {
+    if (st) release(st);
+}
 
 const char *lq_strerror(int status) {
     switch (status) {

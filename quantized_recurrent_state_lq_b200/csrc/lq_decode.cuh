@@ -27,6 +27,20 @@
 
 namespace lq {
 
+// Tokens batch entry b holds in its current window, and whether its window
+// ends at this step (always false without window phases: the caller decides).
+struct EntryPos {
+    int n;
+    bool ends;
+};
+__device__ __forceinline__ EntryPos entry_pos(const DecodeArgs &a, int b) {
+    if (!a.phase) return {a.n, false};
+    int p = a.nmod + __ldg(a.phase + b);
+    if (p >= a.L.W) p -= a.L.W;
+    return {p < a.n ? p : a.n, p == a.L.W - 1};
+}
+
+
 // ---------------------------------------------------------------------------
 // Buffering step: one CTA of 4 warps per head, small enough (<= 72 registers,
 // ~27 KB of shared memory at d = 128) for seven CTAs per SM, so that the
@@ -139,7 +153,10 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int P = DAMP ? L.P : 0;
     const int NI = DK - P;
-    const int E = L.r + a.n;
+    const EntryPos pos = entry_pos(a, b);
+    if (pos.ends) return;   // staggered windows: this entry's flush launch takes the step
+    const int n = pos.n;
+    const int E = L.r + n;
     const size_t hv = (size_t)b * a.H + h;
     unsigned char *rec = a.rec + (size_t)head * L.rec_bytes;
     const float *ent_g = reinterpret_cast<const float *>(rec + L.off_ent);
@@ -172,12 +189,12 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
     // everything else -- the entries and Gamma the previous step wrote, the
     // step's inputs -- is read after the wait.
     asm volatile("griddepcontrol.launch_dependents;");
-    if (t == 0 && a.n > 0) {
+    if (t == 0 && n > 0) {
         mbar_arrive_expect_tx(&S.mbar, (uint32_t)L.off_ent);
         bulk_g2s(stage, rec, (uint32_t)L.off_ent, &S.mbar);
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (t == 0 && a.n == 0) {
+    if (t == 0 && n == 0) {
         mbar_arrive_expect_tx(&S.mbar, (uint32_t)L.off_ent);
         bulk_g2s(stage, rec, (uint32_t)L.off_ent, &S.mbar);
     }
@@ -224,8 +241,8 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
         const size_t qk = ((size_t)b * a.Hk + g) * DK;
         kk = a.k[qk + t];
         const float qq = a.q[qk + t];
-        const float gp = a.n > 0 ? (KDA ? rec_gam[t] : rec_gam[0]) : 1.0f;
-        const float sp = a.n > 0 ? (KDA ? rec_sig[t] : rec_sig[0]) : 1.0f;
+        const float gp = n > 0 ? (KDA ? rec_gam[t] : rec_gam[0]) : 1.0f;
+        const float sp = n > 0 ? (KDA ? rec_sig[t] : rec_sig[0]) : 1.0f;
         gt = gate_chain(KDA ? a.alpha[hv * DK + t] : a.alpha[hv], gp, rho);
         sg = sp * rho;
         const float2 x = make_float2(gt * kk, gt * qq);
@@ -554,7 +571,7 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
         float ut = beta * (S.v[t] - yk);
         if (tb) {
             const uint16_t uh = bf16_rne(ut);
-            rec_tok16[(size_t)a.n * EF + DK + t] = uh;
+            rec_tok16[(size_t)n * EF + DK + t] = uh;
             ut = bf16_to_f(uh);
         } else {
             rec_ent[(size_t)E * EF + DK + t] = ut;
@@ -564,7 +581,7 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
         if (!isfinite(o) || !isfinite(ut)) atomicOr(a.status, kStatusNonFinite);
     }
     if (t < DK) {
-        if (tb) rec_tok16[(size_t)a.n * EF + t] = khat;
+        if (tb) rec_tok16[(size_t)n * EF + t] = khat;
         else rec_ent[(size_t)E * EF + t] = kk / gt;
         if (KDA) {
             rec_gam[t] = gt;
@@ -645,12 +662,17 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
     const Layout &L = a.L;
     unsigned char *work = smem + flush_fixed_bytes<DK, DV>();
     unsigned char *stage = work + flush_work_bytes(DK, DV);
-    const int head = blockIdx.x;
-    const int b = head / a.H, h = head - b * a.H, g = (h * a.Hk) / a.H;
+    // (staggered windows: the grid covers the listed batch entries only)
+    const int b = a.flush_list ? __ldg(a.flush_list + blockIdx.x / a.H) : (int)(blockIdx.x / a.H);
+    const int h = (int)(blockIdx.x % a.H), g = (h * a.Hk) / a.H;
+    const int head = b * a.H + h;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int cg = t % T::CG, row0 = (t / T::CG) * T::RPT;
     const int P = DAMP ? L.P : 0;
-    const int E = L.r + a.n;
+    const int n = entry_pos(a, b).n;
+    // an explicit window end with nothing buffered leaves the state as it is
+    if (MODE == kFlushOnly && n == 0) return;
+    const int E = L.r + n;
     const int nch = (E + kFlushChunk - 1) / kFlushChunk;
     unsigned char *rec = a.rec + (size_t)head * L.rec_bytes;
     float *rec_ent = reinterpret_cast<float *>(rec + L.off_ent);
@@ -681,8 +703,8 @@ __global__ void __launch_bounds__(kFlushThreads, 3) decode_flush_kernel(const De
         // the buffer is keyed to G and the quantized state scaled by sigma G
         // (decay guard); the tile is G [sigma Deq + entries], times this
         // step's decay for a window-end token (a product: it may underflow)
-        const float gp = a.n > 0 ? (KDA ? rec_gam[t] : rec_gam[0]) : 1.0f;
-        const float sp = a.n > 0 ? (KDA ? rec_sig[t] : rec_sig[0]) : 1.0f;
+        const float gp = n > 0 ? (KDA ? rec_gam[t] : rec_gam[0]) : 1.0f;
+        const float sp = n > 0 ? (KDA ? rec_sig[t] : rec_sig[0]) : 1.0f;
         float gt = gp;
         if (MODE == kFlushStep) {
             const size_t qk = ((size_t)b * a.Hk + g) * DK;

@@ -20,6 +20,15 @@ struct DecodeArgs {
     const int *slot_rows; // [H][dk] (device): key row of INT8 slot j, then of BF16 row p
     int *status;
     float *S_out;         // export target [heads][dk][dv]
+    // Window phases (staggered windows): batch entry b ends its windows at the
+    // steps where (since + phase[b]) mod W = W - 1, since counting the steps
+    // from the last common window start; it then holds
+    // min((since + phase[b]) mod W, since) buffered tokens.  With phases, n is
+    // min(since, W) and nmod is since mod W; without (phase null) every entry
+    // holds n tokens.
+    const int *phase;       // [B] (device) or null
+    const int *flush_list;  // flush launches: the batch entries of the grid, H CTAs each (null: all heads)
+    int nmod;
 };
 
 struct Fp32Args {

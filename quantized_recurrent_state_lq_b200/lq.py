@@ -34,7 +34,7 @@ EXPORTED = ["lq_workspace_bytes", "lq_config_check", "lq_state_init", "lq_decode
             "lq_state_export_view", "lq_state_import_view", "lq_quantize_state",
             "lq_dequantize_state", "lq_quantize_state_static", "lq_damp_select", "lq_get_status",
             "lq_state_destroy", "lq_strerror", "lq_selftest_division", "lq_prefill",
-            "lq_state_init_static", "lq_fit_static_scales", "lq_selftest_wait"]
+            "lq_state_init_static", "lq_fit_static_scales", "lq_selftest_wait", "lq_state_set_phases"]
 
 
 class LqError(RuntimeError):
@@ -90,6 +90,7 @@ def lib():
             "lq_state_init_static": (C.c_int, [C.POINTER(vp), cfgp, vp, sz, vp, vp, vp, vp]),
             "lq_fit_static_scales": (C.c_int, [cfgp, i32, vp, i32, vp, vp, vp, vp]),
             "lq_selftest_wait": (C.c_int, [vp, C.c_int64, vp]),
+            "lq_state_set_phases": (C.c_int, [vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -275,6 +276,19 @@ def lq_decode_step(st: LqState, q, k, v, beta, alpha, o, stream=None):
             _dev(o, "o", (c.B, c.H, c.dv))]
     _chk(lib().lq_decode_step(st.handle, *[C.c_void_p(a) for a in args], C.c_void_p(_stream(stream))),
          "lq_decode_step")
+
+
+def lq_state_set_phases(st: LqState, phases, stream=None):
+    """Staggered windows: phases [B] (ints in [0, W)), or None to remove them."""
+    if phases is None:
+        _chk(lib().lq_state_set_phases(st.handle, None, C.c_void_p(_stream(stream))), "lq_state_set_phases")
+        return
+    vals = [int(x) for x in phases]
+    if len(vals) != st.cfg.B:
+        raise ValueError(f"phases: {len(vals)} values for B = {st.cfg.B}")
+    arr = (C.c_int32 * len(vals))(*vals)
+    _chk(lib().lq_state_set_phases(st.handle, C.cast(arr, C.c_void_p), C.c_void_p(_stream(stream))),
+         "lq_state_set_phases")
 
 
 def lq_window_flush(st: LqState, stream=None):

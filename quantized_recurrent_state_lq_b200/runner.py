@@ -108,7 +108,7 @@ class WindowRunner:
     per window of W tokens (the W-th call also flushes)."""
 
     def __init__(self, wl: Workload, S0: torch.Tensor, *, mode: str = "window", hp_rows=None,
-                 tokens: int | None = None, device="cuda", static=None):
+                 tokens: int | None = None, device="cuda", static=None, phases=None):
         self.wl = wl
         self.cfg = lq.Config.from_workload(wl, mode=mode)
         self.W = wl.W          # tokens per graph; in step mode every call also requantizes
@@ -118,6 +118,11 @@ class WindowRunner:
             self.st = lq.lq_state_init(self.cfg, S0.contiguous(), static_m=static[0], static_s=static[1])
         else:
             self.st = lq.lq_state_init(self.cfg, S0.contiguous(), hp_rows=hp_rows)
+        # staggered windows: batch entry b ends its windows at the steps where
+        # (step + phases[b]) mod W = W - 1 (lq_state_set_phases)
+        self.phases = phases
+        if phases is not None:
+            lq.lq_state_set_phases(self.st, phases)
         self.tok = gen.token_inputs(wl, self.T, device=device)
         self.out = torch.empty((self.T, wl.B, wl.H, wl.dv), device=device)
         self.graphs = {}
@@ -135,7 +140,9 @@ class WindowRunner:
             self.step_call(t)
 
     def capture(self):
-        """One graph per window slot; replays must start at a window boundary."""
+        """One graph per window slot; replays must start at a window boundary.
+        The warm-up runs window 0 eagerly: with phases it holds every entry's
+        shorter first window, and the graphs then hold full windows only."""
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):

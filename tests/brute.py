@@ -95,10 +95,11 @@ def dequantize(view) -> np.ndarray:
 
 
 def run_windowed(S0, toks, W: int, r: int, K: int, gate: str, smoothing=True, quantize_on=True,
-                 qmax: int = 127):
+                 qmax: int = 127, first: int | None = None):
     """Whole windowed decode of one head with literal matrices.
 
-    toks: list of (q, k, v, beta, alpha).  Returns (outputs, last view).
+    toks: list of (q, k, v, beta, alpha).  first: length of the first window
+    (W by default).  Returns (outputs, last view).
     """
     view = None
     if quantize_on:
@@ -109,14 +110,16 @@ def run_windowed(S0, toks, W: int, r: int, K: int, gate: str, smoothing=True, qu
     Sp = S.T.copy()
     outs = []
     n = 0
+    length = W if first is None else first
     for (q, k, v, beta, alpha) in toks:
         Sp, o = step_pages_form(Sp, q, k, v, beta, alpha, gate)
         outs.append(o)
         n += 1
-        if quantize_on and n == W:
+        if quantize_on and n == length:
             view = quantize(Sp.T.astype(f32), r, K, smoothing, qmax)
             Sp = dequantize(view).T.copy()
             n = 0
+            length = W
     return np.array(outs), view
 
 

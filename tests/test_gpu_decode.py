@@ -57,11 +57,14 @@ def test_fp32_mode_matches_oracle(gate, B, H, Hk, dk, dv):
     assert serr.max() < STATE_REL
 
 
-def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=None, alpha=None):
+def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=None, alpha=None, phase=0):
     flip_frac = U.LONG_ACCUMULATION_FLIP_FRAC if wl.W >= 200 else U.FLUSH_FLIP_FRAC
     """Run T tokens window by window; each window starts from the oracle's view.
     static = (m [H, dk], s [H, dv]) numpy arrays: fixed scales (smoothing 2).
-    alpha(tok): replaces the generator's decays (a device tensor of their shape)."""
+    alpha(tok): replaces the generator's decays (a device tensor of their shape).
+    phase: every batch entry's window phase (staggered windows, one phase for
+    all so that the windows still start together): the first window holds
+    W - phase tokens."""
     if static is not None:
         smoothing = 2
     cfg = lq.Config.from_workload(wl, mode=mode, fused_flush=int(fused), smoothing=smoothing)
@@ -93,19 +96,24 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=N
         for k in ov:
             ov[k][h][...] = np.asarray(q[k]).reshape(ov[k][h].shape)
     W = cfg.W
+    if phase:
+        lq.lq_state_set_phases(st, [phase] * wl.B)
     stats = {"out": 0.0, "state": 0.0, "flips": 0, "codes": 0, "band_used": 0.0, "bound_used": 0.0,
              "flips_bf16_tie": 0, "undetermined": 0}
     o = torch.empty((wl.B, wl.H, wl.dv), device="cuda")
     t0 = 0
     while t0 < T:
-        n = min(W, T - t0)
+        Lw = W - phase if t0 == 0 else W   # this window's length
+        flips0 = stats["flips"]
+        n = min(Lw, T - t0)
         sl = {k: v[t0:t0 + n] for k, v in ph.items()}
-        ref = O.run(oc, sl, view=ov, hp_rows=hr, flush_last=(n == W))   # oc: all heads' fixed scales
+        ref = O.run(oc, sl, view=ov, hp_rows=hr, flush_last=(n == Lw),   # oc: all heads' fixed scales
+                    phase=[phase] * nh if t0 == 0 else None)
         lq.lq_state_import_view(st, U.oracle_view_to_gpu(cfg, ov, rows))
         S_g = None
         for t in range(n):
             last = t == n - 1
-            if last and n == W and not fused and mode == "window":
+            if last and n == Lw and not fused and mode == "window":
                 lq.lq_decode_step(st, *U.step_args(tok, t0 + t), o)
                 S = torch.empty((wl.B, wl.H, wl.dk, wl.dv), device="cuda")
                 lq.lq_state_export_fp32(st, S)
@@ -117,8 +125,8 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=N
                 lq.lq_decode_step(st, *U.step_args(tok, t0 + t), o)
             e = U.rel_inf_rows(o.cpu().numpy().reshape(nh, wl.dv), ref["o"][t])
             stats["out"] = max(stats["out"], float(e.max()))
-        assert lq.lq_state_buffered(st) == (0 if n == W else n)
-        if n == W:
+        assert lq.lq_state_buffered(st) == (0 if n == Lw else n)
+        if n == Lw:
             gv = lq.alloc_view(cfg)
             lq.lq_state_export_view(st, gv)
             got = U.gpu_view_to_oracle(cfg, gv, rows)
@@ -166,6 +174,8 @@ def _teacher_forced(wl, T, fused, mode="window", smoothing=1, label="", static=N
                 f = lambda x: (x.astype(np.uint32) << 16).view(np.float32)
                 dv = np.abs(f(hpg) - f(hpw))
                 assert ((ulps <= 1) | (dv <= STATE_REL * scale[:, None, None])).all()
+        if n == Lw:
+            print(f"{label}: window at token {t0} ({n} tokens): {stats['flips'] - flips0} flips")
         ov = ref["view"]
         t0 += n
     assert lq.lq_get_status(st) == lq.LQ_OK

@@ -140,6 +140,7 @@ def test_null_handles_and_pointers(L):
     assert L.lq_selftest_wait(fake, 999, None) == lq.LQ_ERR_INVALID_ARG
     assert L.lq_selftest_wait(fake, 2000000000, None) == lq.LQ_ERR_INVALID_ARG
     assert L.lq_state_buffered(None) == 0
+    assert L.lq_state_set_phases(None, None, None) == lq.LQ_ERR_INVALID_ARG
     L.lq_state_destroy(None)
     cfg = lq.Config.from_workload(configs.TINY_GDN)
     view = lq.lq_qstate_view(None, None, None, None, None, None)

@@ -372,12 +372,12 @@ def workload_line(wl, stream, peak_gbs: float, windows: int = 6) -> dict:
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def prefill_line(wl, stream, chunks: int = 32, tokens: int = 64) -> dict:
-    """The chunked prefill (lq_prefill) of the workload's heads: `chunks`
-    calls of `tokens` tokens each from one seeded draw of `tokens` tokens
-    (the kernel's work does not depend on the values), the state carried in
-    place; beside it the token-by-token FP32-state kernel on one call's worth
-    of tokens.  CUDA events on the launching stream."""
+def prefill_line(wl, stream, chunks: int = 8, tokens: int = 256) -> dict:
+    """The chunked prefill (lq_prefill) of the workload's heads over its
+    prefill length: `chunks` calls of `tokens` tokens each from one seeded
+    draw of `tokens` tokens (the kernel's work does not depend on the values),
+    the state carried in place; beside it the token-by-token FP32-state kernel
+    on 64 tokens.  CUDA events on the launching stream."""
     cfg = lq.Config(B=wl.B, H=wl.H, Hk=wl.Hk, dk=wl.dk, dv=wl.dv, gate=wl.gate, mode="fp32", r=0)
     tok = gen.token_inputs(wl, tokens, stream="prefill", device="cuda")
     S = torch.zeros((wl.B, wl.H, wl.dk, wl.dv), device="cuda")
@@ -403,12 +403,13 @@ def prefill_line(wl, stream, chunks: int = 32, tokens: int = 64) -> dict:
     for t in range(4):
         step(t)
     torch.cuda.synchronize()
+    nrec = min(tokens, 64)
     ev0.record(stream)
-    for t in range(tokens):
+    for t in range(nrec):
         step(t)
     ev1.record(stream)
     ev1.synchronize()
-    dtr = ev0.elapsed_time(ev1) / 1e3 * (T / tokens)
+    dtr = ev0.elapsed_time(ev1) / 1e3 * (T / nrec)
     lq.lq_state_destroy(st)
     flops = traffic.prefill_flops(wl, T) * wl.heads
     achieved = flops / dt / 1e12
@@ -423,10 +424,13 @@ def prefill_line(wl, stream, chunks: int = 32, tokens: int = 64) -> dict:
             "recurrent_fp32_seconds": dtr, "speedup_vs_recurrent": dtr / dt,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": None,
-                         "kernel": "prefill_tc_kernel (chunked WY form; d_k x d_v products as mma.sync TF32 x3)",
+                         "kernel": ("prefill_umma_kernel (chunked WY form; the state in tensor memory, "
+                                    "products as tcgen05.mma TF32 x3, inputs by TMA tensor copies)"
+                                    if wl.dk == 128 and wl.dv == 128 else
+                                    "prefill_tc_kernel (chunked WY form; products as mma.sync TF32 x3)"),
                          "peak_source": f"{src} bf16 burst x 1.1/2.25 (TF32) / 3 passes",
                          "fp32_alu_frac": achieved / FP32_PEAK_TFLOPS},
-            "note": f"{chunks} calls of one {tokens}-token draw; recurrent time from {tokens} tokens x {T // tokens}"}
+            "note": f"{chunks} calls of one {tokens}-token draw; recurrent time from {nrec} tokens x {T // nrec}"}
 
 
 def state_dtype(wl) -> str:

@@ -23,6 +23,9 @@
 // shared memory.  The three d_k x d_v products run on the tensor cores in
 // three TF32 passes (FP32-level accuracy); the pair matrices, the forward
 // substitution and the outputs in FP32.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "lq_common.cuh"
 #include "lq_prefill.h"
 #include "lq_tc.cuh"
@@ -301,19 +304,673 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
     if (!fin && a.status) atomicOr(a.status, kStatusNonFinite);
 }
 
+
+// ---------------------------------------------------------------------------
+// d_k = d_v = 128: the chunk step on the fifth-generation tensor cores, in
+// chunks of kUChunk = 16 tokens, one CTA per head (one per SM: the state's
+// tensor memory) of 8 compute warps and one warp that issues the MMAs.  The chunk's pseudo-values are solved without the
+// state first: with A the strictly lower pair matrix above,
+//   (I + A) W = diag(b) Kg,   (I + A) Ut = diag(b) V     (rows = tokens)
+// by forward substitution (a key or value column per thread), so that
+//   U = Ut - W S,   O = Qg S + P U,   S <- diag(Gamma_C) S + Kh^T U
+// are products only, all on the tensor cores with the state in tensor memory
+// as S^T [d_v lanes x d_k columns] (FP32, the update's accumulator):
+//   group 1:  [Oi^T | U'^T] = S^T [Qg; -W]^T        (M = d_v, N = 32, K = d_k;
+//             A = S^T's TF32 big and small parts, also in tensor memory)
+//   group 2:  [S^T | O^T] += U^T [Kh; P]^T           (N = d_k + 16, K = 16
+//             tokens; A = U^T from shared memory, U = Ut + U')
+// each product in three TF32 passes (big x big + big x small + small x big);
+// stacking the two right-hand sides of each group makes it one MMA chain.
+// Everything that does not need the state -- the next chunk's decays, pair
+// matrices, substitution and operand splits -- runs on the compute warps while
+// a group is in flight (the MMA warp waits on mbarriers, so its issue time is
+// off their path): the next chunk's inputs arrive by bulk copies two chunks ahead
+// (two input slots), and the operands that group 2 may still read while the
+// next chunk's are written (Kh, P) have two slots.  Tensor memory: S^T
+// columns 0-127, O^T 128-143, U'^T 144-159, S^T's big and small parts
+// 256-383 and 384-511.
+// ---------------------------------------------------------------------------
+constexpr int kUChunk = 16;
+constexpr int kUCompute = 256;               // compute warps 0-7
+constexpr int kUThreads = kUCompute + 32;    // and the MMA warp
+
+template <bool KDA>
+struct alignas(128) PrefillUIn {   // one chunk's inputs (token rows padded against bank conflicts;
+                                   // tensor-copy destinations 128-byte aligned)
+    static constexpr int D = 128, C = kUChunk, RP = D + 4;
+    alignas(128) float k[C][RP];
+    alignas(128) float q[C][RP];
+    alignas(128) float g[KDA ? C : 1][KDA ? RP : C];   // decays -> cumulative log2 decay
+    alignas(128) float v[C][D];
+    float beta[C];
+};
+
+template <bool KDA>
+struct PrefillUSmem {
+    static constexpr int D = 128, C = kUChunk, RP = D + 4;
+    // MMA operands, TF32 big [0] and small [1], K-major core matrices: word
+    // (row x, k) at (k / 4) rows 4 + (x / 8) 32 + (x % 8) 4 + k % 4
+    alignas(128) uint32_t qw[2][2 * C * D];         // B of group 1: [Qg; -W] [N = 2C tokens][K = D key rows]
+    alignas(128) uint32_t khp[2][2][(D + C) * C];   // [slot]: B of group 2: [Kh; P] [N = D + C][K = C tokens]
+    alignas(128) uint32_t ut[2][D * C];             // A of group 2: U^T [M = D value columns][K = C tokens]
+    alignas(16) float ud[2][C][D];           // [slot]: Ut
+    alignas(16) float wst[C][RP];            // -W before its split
+    alignas(16) float fac[KDA ? 24 : 1][RP]; // KDA: the decay-factored pair operands (below)
+    PrefillUIn<KDA> in[2];                   // input slots: chunk c in slot c % 2
+    alignas(16) float A[C][C + 4];           // rows read as float4 (the last 4 columns unused)
+    alignas(16) float P[C][C + 4];
+    float gC[2][D];                          // [slot]: Gamma over the whole chunk, per key row
+    uint64_t mbar_in[2];       // input slot filled
+    uint64_t mbar_s, mbar_u;   // the state split / U^T written (compute warps -> MMA warp)
+    uint64_t mbar_yo, mbar_up; // group 1 / group 2 complete (tensor core -> compute warps)
+    uint32_t tmem_base;
+};
+
+__device__ __forceinline__ int umma_word(int rows, int x, int k) {
+    return (k >> 2) * rows * 4 + (x >> 3) * 32 + (x & 7) * 4 + (k & 3);
+}
+
+__device__ __forceinline__ void split4(float4 f, uint4 &big, uint4 &small) {
+    tf32_split(f.x, big.x, small.x);
+    tf32_split(f.y, big.y, small.y);
+    tf32_split(f.z, big.z, small.z);
+    tf32_split(f.w, big.w, small.w);
+}
+
+// Tensor maps of the token-major inputs [T][B][heads][D], one box = 16 token
+// rows of one head: k and q (of the q/k head), the KDA decays 132 floats wide
+// (the padded shared-memory rows; the 4 floats past D are out of bounds and
+// arrive as zeros), v 128 wide.  Rows past T arrive as zeros.
+struct alignas(64) PrefillMaps {
+    CUtensorMap k, q, v, g;
+};
+
+template <bool KDA>
+constexpr uint32_t prefill_load_bytes() {
+    return (uint32_t)(kUChunk * (PrefillUIn<KDA>::RP * 4 * (KDA ? 3 : 2) + 128 * 4));
+}
+
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int x, int y, int z, int w,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5}], [%6];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Named barrier of the compute warps (warps 0-7; the MMA warp stays out), and
+// its OR-reduction form.
+__device__ __forceinline__ void ubar() { asm volatile("bar.sync 1, %0;" ::"n"(kUCompute) : "memory"); }
+
+__device__ __forceinline__ bool ubar_or(bool v) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.s32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\t"
+        "selp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((int)v), "n"(kUCompute)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <bool KDA>
+__global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const PrefillArgs a,
+                                                                      const __grid_constant__ PrefillMaps mp) {
+    constexpr int D = 128, C = kUChunk, NT = kUCompute;
+    using Sm = PrefillUSmem<KDA>;
+    using In = PrefillUIn<KDA>;
+    extern __shared__ __align__(128) unsigned char smem_u[];
+    Sm &S = *reinterpret_cast<Sm *>(smem_u);
+    const int head = blockIdx.x;
+    const int b = head / a.H, h = head - b * a.H, gk = (h * a.Hk) / a.H;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int quad = warp & 3, half = (warp >> 2) & 1;   // tensor-memory lanes 32 quad.., column / token half
+    const int col = 32 * quad + lane;                    // the value column (tensor-memory lane) of this thread
+    const size_t state_off = (size_t)head * D * D;
+    const int nchunks = (a.T + C - 1) / C;
+    constexpr uint32_t cS = 0, cO = 128, cU = 144, cSb = 256, cSs = 384;
+    constexpr uint32_t IDESC_G1 = umma_idesc_tf32(128, 2 * C);
+    constexpr uint32_t IDESC_G2 = umma_idesc_tf32(128, D + C);
+    const bool want_o = a.o != nullptr;
+
+    if (t == 0) {
+        mbar_init(&S.mbar_in[0], 1);
+        mbar_init(&S.mbar_in[1], 1);
+        mbar_init(&S.mbar_yo, 1);
+        mbar_init(&S.mbar_up, 1);
+        mbar_init(&S.mbar_s, 1);
+        mbar_init(&S.mbar_u, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&S.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == kUCompute / 32) {
+        // The MMA warp: per chunk, group 1 once the state is split, group 2
+        // once U^T is in shared memory; completions go to mbar_yo / mbar_up.
+        if (lane == 0) {
+#pragma unroll 1
+            for (int ch = 0; ch < nchunks; ++ch) {
+                const int sl = ch & 1;
+                if (!mbar_wait_bounded(&S.mbar_s, (uint32_t)(ch & 1), a.status)) break;
+                tc_fence_after();
+                {   // 16 K-blocks of 8 key rows, three passes each; a K-block is
+                    // 8 x 2C x 4 bytes (1 KB) of each part of [Qg; -W]
+                    const uint64_t db = umma_smem_desc(&S.qw[0][0], 2 * C * 16, 128);
+                    const uint64_t ds = umma_smem_desc(&S.qw[1][0], 2 * C * 16, 128);
+#pragma unroll 1
+                    for (int kb = 0; kb < D / 8; ++kb) {
+                        const uint32_t ab = tmem + cSb + 8u * kb, as = tmem + cSs + 8u * kb;
+                        const uint64_t off = (uint64_t)(kb * 8 * 2 * C * 4) >> 4;
+                        umma_tf32_ta(tmem + cO, ab, db + off, IDESC_G1, kb > 0 ? 1u : 0u);
+                        umma_tf32_ta(tmem + cO, ab, ds + off, IDESC_G1, 1u);
+                        umma_tf32_ta(tmem + cO, as, db + off, IDESC_G1, 1u);
+                    }
+                    umma_commit(&S.mbar_yo);
+                }
+                if (!mbar_wait_bounded(&S.mbar_u, (uint32_t)(ch & 1), a.status)) break;
+                tc_fence_after();
+                {   // 2 K-blocks of 8 tokens, three passes each; a K-block is
+                    // 8 D x 4 words of U^T and 8 (D + C) x 4 words of [Kh; P]
+                    const uint64_t ub = umma_smem_desc(&S.ut[0][0], D * 16, 128);
+                    const uint64_t us = umma_smem_desc(&S.ut[1][0], D * 16, 128);
+                    const uint64_t hb = umma_smem_desc(&S.khp[sl][0][0], (D + C) * 16, 128);
+                    const uint64_t hs = umma_smem_desc(&S.khp[sl][1][0], (D + C) * 16, 128);
+#pragma unroll
+                    for (int kb = 0; kb < C / 8; ++kb) {
+                        const uint64_t ou = (uint64_t)(kb * 8 * D * 4) >> 4;
+                        const uint64_t oh = (uint64_t)(kb * 8 * (D + C) * 4) >> 4;
+                        umma_tf32(tmem + cS, ub + ou, hb + oh, IDESC_G2, 1u);
+                        umma_tf32(tmem + cS, ub + ou, hs + oh, IDESC_G2, 1u);
+                        umma_tf32(tmem + cS, us + ou, hb + oh, IDESC_G2, 1u);
+                    }
+                    umma_commit(&S.mbar_up);
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        const uint32_t trow = tmem + ((uint32_t)(32 * quad) << 16);   // this warp's 32 lanes
+
+        // Chunk c's token rows into input slot c % 2: one tensor copy per array
+        // (rows past T: zeros), completing on mbar_in[c % 2].  Starts with a
+        // barrier (the slot's previous contents have been read).
+        auto issue_load = [&](int c) {
+            In &I = S.in[c & 1];
+            const int t0 = c * C;
+            ubar();
+            if (t == 0) {
+                uint64_t *bar = &S.mbar_in[c & 1];
+                mbar_arrive_expect_tx(bar, prefill_load_bytes<KDA>());
+                tma_load_4d(&I.k[0][0], &mp.k, 0, gk, b, t0, bar);
+                tma_load_4d(&I.q[0][0], &mp.q, 0, gk, b, t0, bar);
+                tma_load_4d(&I.v[0][0], &mp.v, 0, h, b, t0, bar);
+                if (KDA) tma_load_4d(&I.g[0][0], &mp.g, 0, h, b, t0, bar);
+            }
+        };
+
+        // b_t (and GDN's decay, as log2) of chunk c's token t, loaded ahead of use
+        auto load_scalars = [&](int c, float &bet, float &gl) {
+            bet = 0.f;
+            gl = 0.f;
+            if (t < C && c * C + t < a.T) {
+                const size_t bh = ((size_t)(c * C + t) * a.B + b) * a.H + h;
+                bet = __ldg(a.beta + bh);
+                if (!KDA) gl = __ldg(a.alpha + bh);
+            }
+        };
+
+        // Chunk c, part 1 (no operand that a group may be reading): decays, pair
+        // matrices, and the substitution into -W (wst) and Ut (ud[c % 2]).
+        auto prep_solve = [&](int c, float bet, float gl) -> bool {
+            In &I = S.in[c & 1];
+            const int sl = c & 1;
+            const bool okw = mbar_wait_bounded(&S.mbar_in[sl], (uint32_t)((c >> 1) & 1), a.status);
+            if (ubar_or(!okw)) return false;
+            if (t < C) {
+                I.beta[t] = bet;
+                if (!KDA) I.g[0][t] = (c * C + t < a.T) ? fmaxf(log2f(gl), -150.0f) : 0.f;
+            }
+            if (KDA) {   // decays -> log2, floored at -150 (a decay of 0 wipes the state); 0 past T
+#pragma unroll
+                for (int j = 0; j < C * D / NT; ++j) {
+                    const int e = t + j * NT;
+                    float &x = I.g[e / D][e % D];
+                    x = c * C + e / D < a.T ? fmaxf(log2f(x), -150.0f) : 0.f;
+                }
+            }
+            ubar();
+            // cumulative log2 decay within the chunk, Gamma_C
+            if (KDA) {
+                if (t < D) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int tt = 0; tt < C; ++tt) {
+                        acc += I.g[tt][t];
+                        I.g[tt][t] = acc;
+                    }
+                    S.gC[sl][t] = exp2f(acc);
+                }
+            } else if (t == 0) {
+                float acc = 0.f;
+#pragma unroll
+                for (int tt = 0; tt < C; ++tt) {
+                    acc += I.g[0][tt];
+                    I.g[0][tt] = acc;
+                }
+                S.gC[sl][0] = exp2f(acc);
+            }
+            ubar();
+            if (!KDA) {
+                // pair matrices: warp w takes token rows w (lanes 0-15) and 15 - w
+                // (lanes 16-31), lane % 16 the column; the decay factor
+                // 2^(g_t - g_i) <= 1 is one value per pair
+                const int ti = lane < 16 ? warp : C - 1 - warp, ii = lane & 15;
+                float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), aq = ak;   // a partial sum per float4 lane
+#pragma unroll 4
+                for (int r4 = 0; r4 < D / 4; ++r4) {
+                    const float4 kt = *reinterpret_cast<const float4 *>(&I.k[ti][4 * r4]);
+                    const float4 qt = *reinterpret_cast<const float4 *>(&I.q[ti][4 * r4]);
+                    const float4 ki = *reinterpret_cast<const float4 *>(&I.k[ii][4 * r4]);
+                    ak = make_float4(fmaf(kt.x, ki.x, ak.x), fmaf(kt.y, ki.y, ak.y), fmaf(kt.z, ki.z, ak.z),
+                                     fmaf(kt.w, ki.w, ak.w));
+                    aq = make_float4(fmaf(qt.x, ki.x, aq.x), fmaf(qt.y, ki.y, aq.y), fmaf(qt.z, ki.z, aq.z),
+                                     fmaf(qt.w, ki.w, aq.w));
+                }
+                const float f = exp2f(fminf(I.g[0][ti] - I.g[0][ii], 0.f));
+                const float dkk = ((ak.x + ak.y) + (ak.z + ak.w)) * f, dqk = ((aq.x + aq.y) + (aq.z + aq.w)) * f;
+                S.A[ti][ii] = ii < ti ? I.beta[ti] * dkk : 0.f;
+                S.P[ti][ii] = ii <= ti ? dqk : 0.f;
+            } else {
+                // KDA: per-channel factors 2^(g_t - g_i).  Across the two
+                // 8-token halves (t >= 8 > 7 >= i) they factor through token 7,
+                // 2^(g_t - g_7) 2^(g_7 - g_i), both <= 1: rows 0-7 of fac hold
+                // k_i 2^(g_7 - g_i), rows 8-15 k_t 2^(g_t - g_7), rows 16-23
+                // q_t 2^(g_t - g_7) (t = 8 ..); within a half the factor is
+                // formed per pair.
+#pragma unroll
+                for (int j = 0; j < 24 * D / 4 / NT; ++j) {
+                    const int e = t + j * NT, row = e / (D / 4), r = 4 * (e % (D / 4));
+                    const float4 g7 = *reinterpret_cast<const float4 *>(&I.g[7][r]);
+                    const int tr = row < 16 ? row : row - 8;
+                    const float4 gr = *reinterpret_cast<const float4 *>(&I.g[tr][r]);
+                    const float4 x = *reinterpret_cast<const float4 *>(row < 16 ? &I.k[tr][r] : &I.q[tr][r]);
+                    float4 d = row < 8 ? make_float4(g7.x - gr.x, g7.y - gr.y, g7.z - gr.z, g7.w - gr.w)
+                                       : make_float4(gr.x - g7.x, gr.y - g7.y, gr.z - g7.z, gr.w - g7.w);
+                    *reinterpret_cast<float4 *>(&S.fac[row][r]) =
+                        make_float4(x.x * exp2f(d.x), x.y * exp2f(d.y), x.z * exp2f(d.z), x.w * exp2f(d.w));
+                }
+                ubar();
+                // warps 0-3: the two 8 x 8 diagonal blocks (4 rows x 8 columns
+                // a warp); 4-5: rows 8-15 x columns 0-7 from fac; 6-7: rows 0-7
+                // x columns 8-15, zero
+                int ti, ii;
+                float dkk = 0.f, dqk = 0.f;
+                if (warp < 4) {
+                    const int blk = 8 * (warp >> 1);
+                    ti = blk + 4 * (warp & 1) + (lane >> 3);
+                    ii = blk + (lane & 7);
+                    float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), aq = ak;
+#pragma unroll 4
+                    for (int r4 = 0; r4 < D / 4; ++r4) {
+                        const float4 kt = *reinterpret_cast<const float4 *>(&I.k[ti][4 * r4]);
+                        const float4 qt = *reinterpret_cast<const float4 *>(&I.q[ti][4 * r4]);
+                        float4 ki = *reinterpret_cast<const float4 *>(&I.k[ii][4 * r4]);
+                        const float4 gt = *reinterpret_cast<const float4 *>(&I.g[ti][4 * r4]);
+                        const float4 gi = *reinterpret_cast<const float4 *>(&I.g[ii][4 * r4]);
+                        // at most 1 where used (ii <= ti); clamped past the diagonal
+                        ki.x *= exp2f(fminf(gt.x - gi.x, 0.f));
+                        ki.y *= exp2f(fminf(gt.y - gi.y, 0.f));
+                        ki.z *= exp2f(fminf(gt.z - gi.z, 0.f));
+                        ki.w *= exp2f(fminf(gt.w - gi.w, 0.f));
+                        ak = make_float4(fmaf(kt.x, ki.x, ak.x), fmaf(kt.y, ki.y, ak.y), fmaf(kt.z, ki.z, ak.z),
+                                         fmaf(kt.w, ki.w, ak.w));
+                        aq = make_float4(fmaf(qt.x, ki.x, aq.x), fmaf(qt.y, ki.y, aq.y), fmaf(qt.z, ki.z, aq.z),
+                                         fmaf(qt.w, ki.w, aq.w));
+                    }
+                    dkk = (ak.x + ak.y) + (ak.z + ak.w);
+                    dqk = (aq.x + aq.y) + (aq.z + aq.w);
+                } else if (warp < 6) {
+                    ti = 8 + 4 * (warp - 4) + (lane >> 3);
+                    ii = lane & 7;
+                    float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), aq = ak;
+#pragma unroll 4
+                    for (int r4 = 0; r4 < D / 4; ++r4) {
+                        const float4 kt = *reinterpret_cast<const float4 *>(&S.fac[ti][4 * r4]);
+                        const float4 qt = *reinterpret_cast<const float4 *>(&S.fac[ti + 8][4 * r4]);
+                        const float4 ki = *reinterpret_cast<const float4 *>(&S.fac[ii][4 * r4]);
+                        ak = make_float4(fmaf(kt.x, ki.x, ak.x), fmaf(kt.y, ki.y, ak.y), fmaf(kt.z, ki.z, ak.z),
+                                         fmaf(kt.w, ki.w, ak.w));
+                        aq = make_float4(fmaf(qt.x, ki.x, aq.x), fmaf(qt.y, ki.y, aq.y), fmaf(qt.z, ki.z, aq.z),
+                                         fmaf(qt.w, ki.w, aq.w));
+                    }
+                    dkk = (ak.x + ak.y) + (ak.z + ak.w);
+                    dqk = (aq.x + aq.y) + (aq.z + aq.w);
+                } else {
+                    ti = 4 * (warp - 6) + (lane >> 3);
+                    ii = 8 + (lane & 7);
+                }
+                S.A[ti][ii] = ii < ti ? I.beta[ti] * dkk : 0.f;
+                S.P[ti][ii] = ii <= ti ? dqk : 0.f;
+            }
+            ubar();
+            // forward substitution, one column per thread: threads 0-127 the key
+            // column t of W (right side b Gamma k), 128-255 the value column of Ut
+            {
+                const int cc = t & (D - 1);
+                float x[C];
+#pragma unroll
+                for (int tt = 0; tt < C; ++tt) {   // the right-hand sides first (independent loads)
+                    if (t < D) x[tt] = I.beta[tt] * (I.k[tt][cc] * exp2f(KDA ? I.g[tt][cc] : I.g[0][tt]));
+                    else x[tt] = I.beta[tt] * I.v[tt][cc];
+                }
+#pragma unroll
+                for (int tt = 1; tt < C; ++tt) {
+                    float rhs = x[tt], x1 = 0.f;
+#pragma unroll
+                    for (int j = 0; 4 * j < tt; ++j) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(&S.A[tt][4 * j]);
+                        rhs = fmaf(-a4.x, x[4 * j], rhs);
+                        if (4 * j + 1 < tt) x1 = fmaf(-a4.y, x[4 * j + 1], x1);
+                        if (4 * j + 2 < tt) rhs = fmaf(-a4.z, x[4 * j + 2], rhs);
+                        if (4 * j + 3 < tt) x1 = fmaf(-a4.w, x[4 * j + 3], x1);
+                    }
+                    x[tt] = rhs + x1;
+                }
+                if (t < D) {
+#pragma unroll
+                    for (int tt = 0; tt < C; ++tt) S.wst[tt][cc] = -x[tt];
+                } else {
+#pragma unroll
+                    for (int tt = 0; tt < C; ++tt) S.ud[sl][tt][cc] = x[tt];
+                }
+            }
+            return true;
+        };
+
+        // Chunk c, part 2: the operand splits ([Qg; -W] single; [Kh; P] into
+        // slot c % 2), then chunk c + 2's inputs into the slot just read.  The
+        // caller guarantees that no group in flight reads qw or the slot written.
+        auto prep_operands = [&](int c) {
+            In &I = S.in[c & 1];
+            const int sl = c & 1;
+            ubar();
+            for (int e = t; e < C * D / 4; e += NT) {   // Qg, -W: token e % C, key rows 4 (e / C) ..
+                const int tt = e % C, r = 4 * (e / C);
+                const int wq = umma_word(2 * C, tt, r), ww = umma_word(2 * C, C + tt, r);
+                uint4 bb, bs;
+                split4(*reinterpret_cast<const float4 *>(&S.wst[tt][r]), bb, bs);
+                *reinterpret_cast<uint4 *>(&S.qw[0][ww]) = bb;
+                *reinterpret_cast<uint4 *>(&S.qw[1][ww]) = bs;
+                float4 qv = *reinterpret_cast<const float4 *>(&I.q[tt][r]);
+                float4 ev;
+                if (KDA) {
+                    const float4 gv = *reinterpret_cast<const float4 *>(&I.g[tt][r]);
+                    ev = make_float4(exp2f(gv.x), exp2f(gv.y), exp2f(gv.z), exp2f(gv.w));
+                } else {
+                    const float ee = exp2f(I.g[0][tt]);
+                    ev = make_float4(ee, ee, ee, ee);
+                }
+                qv = make_float4(qv.x * ev.x, qv.y * ev.y, qv.z * ev.z, qv.w * ev.w);
+                split4(qv, bb, bs);
+                *reinterpret_cast<uint4 *>(&S.qw[0][wq]) = bb;
+                *reinterpret_cast<uint4 *>(&S.qw[1][wq]) = bs;
+            }
+            for (int e = t; e < D * C / 4; e += NT) {   // Kh: key row e % D, tokens 4 (e / D) ..
+                const int r = e % D, t4 = 4 * (e / D);
+                const float glast = KDA ? I.g[C - 1][r] : I.g[0][C - 1];
+                float kh[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float gt = KDA ? I.g[t4 + j][r] : I.g[0][t4 + j];
+                    kh[j] = I.k[t4 + j][r] * exp2f(glast - gt);
+                }
+                uint4 bb, bs;
+                split4(make_float4(kh[0], kh[1], kh[2], kh[3]), bb, bs);
+                const int wd = umma_word(D + C, r, t4);
+                *reinterpret_cast<uint4 *>(&S.khp[sl][0][wd]) = bb;
+                *reinterpret_cast<uint4 *>(&S.khp[sl][1][wd]) = bs;
+            }
+            if (t < C * C / 4) {   // P: token t % C, columns 4 (t / C) ..
+                const int tt = t % C, i4 = 4 * (t / C);
+                uint4 bb, bs;
+                split4(*reinterpret_cast<const float4 *>(&S.P[tt][i4]), bb, bs);
+                const int wd = umma_word(D + C, D + tt, i4);
+                *reinterpret_cast<uint4 *>(&S.khp[sl][0][wd]) = bb;
+                *reinterpret_cast<uint4 *>(&S.khp[sl][1][wd]) = bs;
+            }
+            fence_async_smem();
+            if (c + 2 < nchunks) issue_load(c + 2);   // its barrier also orders the reads above
+        };
+
+        // The outputs of chunk c from O^T in tensor memory (tokens 8 half ..).
+        auto store_outputs = [&](int c) {
+            uint32_t w[8];
+            tmem_ld_32x32b<8>(trow + cO + 8u * half, w);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int tok = c * C + 8 * half + j;
+                if (tok < a.T) a.o[(((size_t)tok * a.B + b) * a.H + h) * D + col] = __uint_as_float(w[j]);
+            }
+        };
+
+        bool ok = true;
+        float bet = 0.f, gl = 0.f;
+        if (nchunks > 0) {   // the first two chunks' inputs in flight during the state's copy
+            load_scalars(0, bet, gl);
+            issue_load(0);
+            if (nchunks > 1) issue_load(1);
+        }
+        // S^T lane col = column col of S0; warp half `half` writes key rows 64 half ..
+#pragma unroll 1
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+            uint32_t w[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                w[j] = __float_as_uint(a.S0 ? a.S0[state_off + (size_t)(c0 + j) * D + col] : 0.0f);
+            tmem_st_32x32b_x32(trow + cS + c0, w);
+        }
+        tmem_st_wait();
+        if (nchunks > 0) {
+            ok = prep_solve(0, bet, gl);
+            if (ok) prep_operands(0);
+        }
+#pragma unroll 1
+        for (int ch = 0; ok && ch < nchunks; ++ch) {
+            const int sl = ch & 1;
+            if (ch + 1 < nchunks) load_scalars(ch + 1, bet, gl);
+            // (1) the previous chunk's group 2 is complete: its outputs, then S^T
+            // split into group 1's A operand and scaled by this chunk's Gamma
+            if (ch > 0) {
+                const bool okw = mbar_wait_bounded(&S.mbar_up, (uint32_t)((ch - 1) & 1), a.status);
+                if (ubar_or(!okw)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (want_o) store_outputs(ch - 1);
+            }
+#pragma unroll 1
+            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+                uint32_t w[32], wb[32], ws[32];
+                tmem_ld_32x32b<32>(trow + cS + (uint32_t)c0, w);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float x = __uint_as_float(w[j]);
+                    tf32_split(x, wb[j], ws[j]);
+                    w[j] = __float_as_uint(x * S.gC[sl][KDA ? c0 + j : 0]);
+                }
+                tmem_st_32x32b_x32(trow + cSb + (uint32_t)c0, wb);
+                tmem_st_32x32b_x32(trow + cSs + (uint32_t)c0, ws);
+                tmem_st_32x32b_x32(trow + cS + (uint32_t)c0, w);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            ubar();
+            if (t == 0) mbar_arrive(&S.mbar_s);   // (2) group 1 goes
+            // (3) while group 1 runs: the next chunk's decays, pairs and substitution
+            if (ch + 1 < nchunks && !prep_solve(ch + 1, bet, gl)) {
+                ok = false;
+                mbar_wait_bounded(&S.mbar_yo, (uint32_t)(ch & 1), a.status);   // group 1 is in flight
+                break;
+            }
+            // (4) group 1 complete: U = Ut + U' into the A operand of group 2
+            {
+                const bool okw = mbar_wait_bounded(&S.mbar_yo, (uint32_t)(ch & 1), a.status);
+                if (ubar_or(!okw)) {
+                    ok = false;
+                    break;
+                }
+            }
+            tc_fence_after();
+            {
+                uint32_t w[8];
+                tmem_ld_32x32b<8>(trow + cU + 8u * half, w);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j4 = 0; j4 < 2; ++j4) {
+                    const int tt = 8 * half + 4 * j4;
+                    float4 u;
+                    u.x = S.ud[sl][tt][col] + __uint_as_float(w[4 * j4]);
+                    u.y = S.ud[sl][tt + 1][col] + __uint_as_float(w[4 * j4 + 1]);
+                    u.z = S.ud[sl][tt + 2][col] + __uint_as_float(w[4 * j4 + 2]);
+                    u.w = S.ud[sl][tt + 3][col] + __uint_as_float(w[4 * j4 + 3]);
+                    uint4 bb, bs;
+                    split4(u, bb, bs);
+                    const int wd = umma_word(D, col, tt);
+                    *reinterpret_cast<uint4 *>(&S.ut[0][wd]) = bb;
+                    *reinterpret_cast<uint4 *>(&S.ut[1][wd]) = bs;
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            ubar();
+            if (t == 0) mbar_arrive(&S.mbar_u);   // (5) group 2 goes
+            // (6) while group 2 runs: the next chunk's operand splits (qw: read by
+            // group 1, complete; [Kh; P]: the other slot)
+            if (ch + 1 < nchunks) prep_operands(ch + 1);
+        }
+        // the last chunk's group 2, its outputs and the final state
+        if (ok && nchunks > 0) {
+            const bool okw = mbar_wait_bounded(&S.mbar_up, (uint32_t)((nchunks - 1) & 1), a.status);
+            ok = !ubar_or(!okw);
+            tc_fence_after();
+            if (ok && want_o) store_outputs(nchunks - 1);
+        }
+        if (ok) {
+            bool fin = true;
+#pragma unroll 1
+            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+                uint32_t w[32];
+                tmem_ld_32x32b<32>(trow + cS + (uint32_t)c0, w);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float x = __uint_as_float(w[j]);
+                    fin = fin && isfinite(x);
+                    a.S_out[state_off + (size_t)(c0 + j) * D + col] = x;
+                }
+            }
+            if (!fin && a.status) atomicOr(a.status, kStatusNonFinite);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
 template <int DK, int DV>
 size_t prefill_smem_bytes_t(bool kda) {
+    if (DK == 128 && DV == 128) return kda ? sizeof(PrefillUSmem<true>) : sizeof(PrefillUSmem<false>);
     return kda ? sizeof(PrefillTcSmem<DK, DV, true>) : sizeof(PrefillTcSmem<DK, DV, false>);
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once.
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        tried = true;
+    }
+    return fn;
+}
+
+// Token rows [T][B][NH][D] (FP32) as a 4-D map with boxes of `rows` tokens x
+// `width` floats of one (b, head).
+static bool encode_rows(CUtensorMap *m, const float *base, int T, int B, int NH, int D, int width, int rows) {
+    const auto enc = tensor_map_encoder();
+    if (!enc || !base) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)NH, (cuuint64_t)B, (cuuint64_t)(T > 0 ? T : 1)};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)NH * D * 4, (cuuint64_t)B * NH * D * 4};
+    const cuuint32_t box[4] = {(cuuint32_t)width, 1, 1, (cuuint32_t)rows};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int DK, int DV>
 static cudaError_t prefill_dispatch(const PrefillArgs &a, int heads, bool kda, cudaStream_t s) {
-    const size_t sm = prefill_smem_bytes_t<DK, DV>(kda);
-    auto kern = kda ? prefill_tc_kernel<DK, DV, true> : prefill_tc_kernel<DK, DV, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    kern<<<heads, 2 * DV, sm, s>>>(a);
-    return cudaGetLastError();
+    // the tensor-memory kernel reads token rows by tensor copies: 16-byte
+    // aligned k, q, v (and KDA's decays) and encodable maps; otherwise the
+    // register-state kernel
+    const uintptr_t al = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
+                         reinterpret_cast<uintptr_t>(a.v) | (kda ? reinterpret_cast<uintptr_t>(a.alpha) : 0);
+    if constexpr (DK == 128 && DV == 128) {
+        PrefillMaps mp{};
+        bool maps = al % 16 == 0 && a.T > 0;
+        if (maps) {
+            constexpr int RP = PrefillUIn<true>::RP;
+            maps = encode_rows(&mp.k, a.k, a.T, a.B, a.Hk, DK, RP, kUChunk) &&
+                   encode_rows(&mp.q, a.q, a.T, a.B, a.Hk, DK, RP, kUChunk) &&
+                   encode_rows(&mp.v, a.v, a.T, a.B, a.H, DV, DV, kUChunk) &&
+                   (!kda || encode_rows(&mp.g, a.alpha, a.T, a.B, a.H, DK, RP, kUChunk));
+        }
+        if (!maps && a.T > 0) {
+            const size_t sm = kda ? sizeof(PrefillTcSmem<DK, DV, true>) : sizeof(PrefillTcSmem<DK, DV, false>);
+            auto kern = kda ? prefill_tc_kernel<DK, DV, true> : prefill_tc_kernel<DK, DV, false>;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            if (e != cudaSuccess) return e;
+            kern<<<heads, 2 * DV, sm, s>>>(a);
+            return cudaGetLastError();
+        }
+        const size_t sm = kda ? sizeof(PrefillUSmem<true>) : sizeof(PrefillUSmem<false>);
+        auto kern = kda ? prefill_umma_kernel<true> : prefill_umma_kernel<false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        kern<<<heads, kUThreads, sm, s>>>(a, mp);
+        return cudaGetLastError();
+    } else {
+        const size_t sm = prefill_smem_bytes_t<DK, DV>(kda);
+        auto kern = kda ? prefill_tc_kernel<DK, DV, true> : prefill_tc_kernel<DK, DV, false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        kern<<<heads, 2 * DV, sm, s>>>(a);
+        return cudaGetLastError();
+    }
 }
 
 size_t prefill_smem_bytes(int dk, int dv, bool kda) {

@@ -65,6 +65,19 @@ __device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t adesc, uint6
         : "memory");
 }
 
+// D (tensor memory) = A B^T (+ D if accumulate) with A [M][K] in tensor memory
+// (lane m = row m, one 32-bit column per K element, from a_tmem) and B [N][K]
+// K-major in shared memory.  Issued by one thread.
+__device__ __forceinline__ void umma_tf32_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // One arrival on the mbarrier once every tcgen05.mma this thread issued before
 // has completed (its operand reads included).
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
@@ -73,7 +86,7 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
 }
 
 // Thread l of the warp reads tensor-memory lane (taddr.lane + l), columns
-// taddr.col .. taddr.col + N - 1 (shape 32x32b, N = 16 or 32).
+// taddr.col .. taddr.col + N - 1 (shape 32x32b, N = 8, 16 or 32).
 template <int N>
 __device__ __forceinline__ void tmem_ld_32x32b(uint32_t taddr, uint32_t (&v)[N]);
 
@@ -100,7 +113,30 @@ __device__ __forceinline__ void tmem_ld_32x32b<16>(uint32_t taddr, uint32_t (&v)
         : "r"(taddr));
 }
 
+template <>
+__device__ __forceinline__ void tmem_ld_32x32b<8>(uint32_t taddr, uint32_t (&v)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Thread l of the warp writes tensor-memory lane (taddr.lane + l), columns
+// taddr.col .. taddr.col + 31 (shape 32x32b).
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // x = big + small with big, small representable in TF32: big = x rounded to
 // nearest (ties away from zero) at TF32's 10 stored mantissa bits -- add half a

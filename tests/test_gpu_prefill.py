@@ -65,18 +65,41 @@ def test_prefill_long_kda_strong_decay():
     _check(wl, tok, None, "prefill kda T300")
 
 
-def test_prefill_vanishing_and_unit_gates():
-    """Gates of exactly 0 (state wiped), 1e-30, and 1 (no decay) mid-run."""
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_vanishing_and_unit_gates(d):
+    """Gates of exactly 0 (state wiped), 1e-30, and 1 (no decay) mid-run, in
+    the middle of a chunk and on a chunk's first and last tokens."""
     U.require_gpu()
     for gate in ("gdn", "kda"):
-        wl = configs.TINY_GDN.with_(gate=gate, B=1, H=2, Hk=2, dk=64, dv=64, seed=3)
+        wl = configs.TINY_GDN.with_(gate=gate, B=1, H=2, Hk=2, dk=d, dv=d, seed=3)
         tok = gen.token_inputs(wl, 40, stream="prefill", device="cuda")
         a = tok["alpha"]
         a[5] = 0.0
         a[6] = 1e-30
+        a[15] = 0.0
+        a[16] = 1e-30
         a[20:24] = 1.0
-        S0 = gen.random_state(2, 64, 64, seed=4).reshape(1, 2, 64, 64)
-        _check(wl, tok, S0, f"prefill {gate} vanishing gates")
+        S0 = gen.random_state(2, d, d, seed=4).reshape(1, 2, d, d)
+        _check(wl, tok, S0, f"prefill {gate} d{d} vanishing gates")
+
+
+@pytest.mark.parametrize("gate", ["gdn", "kda"])
+def test_prefill_rows_not_16_byte_aligned(gate):
+    """Inputs whose rows start 4 bytes past a 16-byte boundary (views into
+    a larger buffer): the call takes the kernel without bulk copies, with the
+    same results."""
+    U.require_gpu()
+    wl = configs.TINY_GDN.with_(gate=gate, B=2, H=2, Hk=2, dk=128, dv=128, seed=11)
+    tok = gen.token_inputs(wl, 37, stream="prefill", device="cuda")
+    shifted = {}
+    for name, x in tok.items():
+        buf = torch.empty(x.numel() + 1, device="cuda")
+        view = buf[1:].view(x.shape)
+        view.copy_(x)
+        shifted[name] = view
+    assert shifted["k"].data_ptr() % 16 == 4
+    S0 = gen.random_state(4, 128, 128, seed=6).reshape(2, 2, 128, 128)
+    _check(wl, shifted, S0, f"prefill {gate} rows at 4 mod 16")
 
 
 def test_prefill_zero_tokens_and_in_place():

@@ -543,6 +543,8 @@ def main():
                     help="run the traffic-lean option (buffered token updates in BF16) as the main line")
     ap.add_argument("--bits", type=int, choices=[8, 6, 4], default=8,
                     help="code width of the quantized state for the main line (6, 4: bit-packed)")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the chunked prefill of the workload's heads (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -559,6 +561,12 @@ def main():
     try:
         if args.impl == "reference":
             rc = run_reference(args, wl, world, rank, pg)
+        elif args.prefill_only:
+            line = {"workload": wl.name, "B": wl.B, "H": wl.H,
+                    "prefill_per_gpu": prefill_line(wl, torch.cuda.current_stream())}
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            rc = 0
         else:
             rc = run_ours(args, wl, world, rank, pg)
     finally:

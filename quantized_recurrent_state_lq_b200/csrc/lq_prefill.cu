@@ -18,11 +18,13 @@
 // Every decay factor is 2^(g_t - g_i) with i <= t, or 2^g_t: never above 1
 // for gates in (0, 1], so nothing overflows however strong the decay.
 //
-// One CTA of 2 dv threads per head (two per SM), the state in registers for
-// the whole run (below); the chunk's keys, queries and decays are staged in
-// shared memory.  The three d_k x d_v products run on the tensor cores in
-// three TF32 passes (FP32-level accuracy); the pair matrices, the forward
-// substitution and the outputs in FP32.
+// Two kernels, one CTA per head, products in three TF32 passes on the tensor
+// cores (FP32-level accuracy), pair matrices and substitutions in FP32:
+//   prefill_umma_kernel (d_k = d_v = 128, 16-byte aligned rows): the state in
+//     tensor memory, the products as tcgen05.mma chains issued by one warp
+//     while eight others prepare the next chunk; inputs by TMA tensor copies;
+//   prefill_tc_kernel (other shapes, other rows): the state in registers as
+//     mma.sync accumulator tiles, the chunk's inputs staged by plain loads.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

@@ -422,6 +422,22 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// The hardware base-2 exponential and logarithm (MUFU, ~2 ulp like exp2f /
+// log2f), results below 2^-126 flushed to zero: the decay factors they form
+// multiply keys and states of size <= 1, so a flushed factor changes a value
+// by less than 2^-126.
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float lg2_ftz(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <bool KDA>
 __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const PrefillArgs a,
                                                                       const __grid_constant__ PrefillMaps mp) {
@@ -544,14 +560,14 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
             if (ubar_or(!okw)) return false;
             if (t < C) {
                 I.beta[t] = bet;
-                if (!KDA) I.g[0][t] = (c * C + t < a.T) ? fmaxf(log2f(gl), -150.0f) : 0.f;
+                if (!KDA) I.g[0][t] = (c * C + t < a.T) ? fmaxf(lg2_ftz(gl), -150.0f) : 0.f;
             }
             if (KDA) {   // decays -> log2, floored at -150 (a decay of 0 wipes the state); 0 past T
 #pragma unroll
                 for (int j = 0; j < C * D / NT; ++j) {
                     const int e = t + j * NT;
                     float &x = I.g[e / D][e % D];
-                    x = c * C + e / D < a.T ? fmaxf(log2f(x), -150.0f) : 0.f;
+                    x = c * C + e / D < a.T ? fmaxf(lg2_ftz(x), -150.0f) : 0.f;
                 }
             }
             ubar();
@@ -564,7 +580,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                         acc += I.g[tt][t];
                         I.g[tt][t] = acc;
                     }
-                    S.gC[sl][t] = exp2f(acc);
+                    S.gC[sl][t] = ex2_ftz(acc);
                 }
             } else if (t == 0) {
                 float acc = 0.f;
@@ -573,7 +589,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                     acc += I.g[0][tt];
                     I.g[0][tt] = acc;
                 }
-                S.gC[sl][0] = exp2f(acc);
+                S.gC[sl][0] = ex2_ftz(acc);
             }
             ubar();
             if (!KDA) {
@@ -592,7 +608,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                     aq = make_float4(fmaf(qt.x, ki.x, aq.x), fmaf(qt.y, ki.y, aq.y), fmaf(qt.z, ki.z, aq.z),
                                      fmaf(qt.w, ki.w, aq.w));
                 }
-                const float f = exp2f(fminf(I.g[0][ti] - I.g[0][ii], 0.f));
+                const float f = ex2_ftz(fminf(I.g[0][ti] - I.g[0][ii], 0.f));
                 const float dkk = ((ak.x + ak.y) + (ak.z + ak.w)) * f, dqk = ((aq.x + aq.y) + (aq.z + aq.w)) * f;
                 S.A[ti][ii] = ii < ti ? I.beta[ti] * dkk : 0.f;
                 S.P[ti][ii] = ii <= ti ? dqk : 0.f;
@@ -613,7 +629,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                     float4 d = row < 8 ? make_float4(g7.x - gr.x, g7.y - gr.y, g7.z - gr.z, g7.w - gr.w)
                                        : make_float4(gr.x - g7.x, gr.y - g7.y, gr.z - g7.z, gr.w - g7.w);
                     *reinterpret_cast<float4 *>(&S.fac[row][r]) =
-                        make_float4(x.x * exp2f(d.x), x.y * exp2f(d.y), x.z * exp2f(d.z), x.w * exp2f(d.w));
+                        make_float4(x.x * ex2_ftz(d.x), x.y * ex2_ftz(d.y), x.z * ex2_ftz(d.z), x.w * ex2_ftz(d.w));
                 }
                 ubar();
                 // warps 0-3: the two 8 x 8 diagonal blocks (4 rows x 8 columns
@@ -634,10 +650,10 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                         const float4 gt = *reinterpret_cast<const float4 *>(&I.g[ti][4 * r4]);
                         const float4 gi = *reinterpret_cast<const float4 *>(&I.g[ii][4 * r4]);
                         // at most 1 where used (ii <= ti); clamped past the diagonal
-                        ki.x *= exp2f(fminf(gt.x - gi.x, 0.f));
-                        ki.y *= exp2f(fminf(gt.y - gi.y, 0.f));
-                        ki.z *= exp2f(fminf(gt.z - gi.z, 0.f));
-                        ki.w *= exp2f(fminf(gt.w - gi.w, 0.f));
+                        ki.x *= ex2_ftz(fminf(gt.x - gi.x, 0.f));
+                        ki.y *= ex2_ftz(fminf(gt.y - gi.y, 0.f));
+                        ki.z *= ex2_ftz(fminf(gt.z - gi.z, 0.f));
+                        ki.w *= ex2_ftz(fminf(gt.w - gi.w, 0.f));
                         ak = make_float4(fmaf(kt.x, ki.x, ak.x), fmaf(kt.y, ki.y, ak.y), fmaf(kt.z, ki.z, ak.z),
                                          fmaf(kt.w, ki.w, ak.w));
                         aq = make_float4(fmaf(qt.x, ki.x, aq.x), fmaf(qt.y, ki.y, aq.y), fmaf(qt.z, ki.z, aq.z),
@@ -676,7 +692,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                 float x[C];
 #pragma unroll
                 for (int tt = 0; tt < C; ++tt) {   // the right-hand sides first (independent loads)
-                    if (t < D) x[tt] = I.beta[tt] * (I.k[tt][cc] * exp2f(KDA ? I.g[tt][cc] : I.g[0][tt]));
+                    if (t < D) x[tt] = I.beta[tt] * (I.k[tt][cc] * ex2_ftz(KDA ? I.g[tt][cc] : I.g[0][tt]));
                     else x[tt] = I.beta[tt] * I.v[tt][cc];
                 }
 #pragma unroll
@@ -721,9 +737,9 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                 float4 ev;
                 if (KDA) {
                     const float4 gv = *reinterpret_cast<const float4 *>(&I.g[tt][r]);
-                    ev = make_float4(exp2f(gv.x), exp2f(gv.y), exp2f(gv.z), exp2f(gv.w));
+                    ev = make_float4(ex2_ftz(gv.x), ex2_ftz(gv.y), ex2_ftz(gv.z), ex2_ftz(gv.w));
                 } else {
-                    const float ee = exp2f(I.g[0][tt]);
+                    const float ee = ex2_ftz(I.g[0][tt]);
                     ev = make_float4(ee, ee, ee, ee);
                 }
                 qv = make_float4(qv.x * ev.x, qv.y * ev.y, qv.z * ev.z, qv.w * ev.w);
@@ -738,7 +754,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const float gt = KDA ? I.g[t4 + j][r] : I.g[0][t4 + j];
-                    kh[j] = I.k[t4 + j][r] * exp2f(glast - gt);
+                    kh[j] = I.k[t4 + j][r] * ex2_ftz(glast - gt);
                 }
                 uint4 bb, bs;
                 split4(make_float4(kh[0], kh[1], kh[2], kh[3]), bb, bs);

@@ -597,20 +597,20 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                 // (lanes 16-31), lane % 16 the column; the decay factor
                 // 2^(g_t - g_i) <= 1 is one value per pair
                 const int ti = lane < 16 ? warp : C - 1 - warp, ii = lane & 15;
-                float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), aq = ak;   // a partial sum per float4 lane
+                float2 ak0 = f2(0.f, 0.f), ak1 = ak0, aq0 = ak0, aq1 = ak0;   // packed partial sums
 #pragma unroll 4
                 for (int r4 = 0; r4 < D / 4; ++r4) {
                     const float4 kt = *reinterpret_cast<const float4 *>(&I.k[ti][4 * r4]);
                     const float4 qt = *reinterpret_cast<const float4 *>(&I.q[ti][4 * r4]);
                     const float4 ki = *reinterpret_cast<const float4 *>(&I.k[ii][4 * r4]);
-                    ak = make_float4(fmaf(kt.x, ki.x, ak.x), fmaf(kt.y, ki.y, ak.y), fmaf(kt.z, ki.z, ak.z),
-                                     fmaf(kt.w, ki.w, ak.w));
-                    aq = make_float4(fmaf(qt.x, ki.x, aq.x), fmaf(qt.y, ki.y, aq.y), fmaf(qt.z, ki.z, aq.z),
-                                     fmaf(qt.w, ki.w, aq.w));
+                    ak0 = ffma2(f2(kt.x, kt.y), f2(ki.x, ki.y), ak0);
+                    ak1 = ffma2(f2(kt.z, kt.w), f2(ki.z, ki.w), ak1);
+                    aq0 = ffma2(f2(qt.x, qt.y), f2(ki.x, ki.y), aq0);
+                    aq1 = ffma2(f2(qt.z, qt.w), f2(ki.z, ki.w), aq1);
                 }
                 const float f = ex2_ftz(fminf(I.g[0][ti] - I.g[0][ii], 0.f));
-                const float dkk = ((ak.x + ak.y) + (ak.z + ak.w)) * f, dqk = ((aq.x + aq.y) + (aq.z + aq.w)) * f;
-                S.A[ti][ii] = ii < ti ? I.beta[ti] * dkk : 0.f;
+                const float dkk = ((ak0.x + ak0.y) + (ak1.x + ak1.y)) * f, dqk = ((aq0.x + aq0.y) + (aq1.x + aq1.y)) * f;
+                S.A[ti][ii] = ii < ti ? -I.beta[ti] * dkk : 0.f;   // stored negated (the substitution adds)
                 S.P[ti][ii] = ii <= ti ? dqk : 0.f;
             } else {
                 // KDA: per-channel factors 2^(g_t - g_i).  Across the two
@@ -641,7 +641,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                     const int blk = 8 * (warp >> 1);
                     ti = blk + 4 * (warp & 1) + (lane >> 3);
                     ii = blk + (lane & 7);
-                    float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), aq = ak;
+                    float2 ak0 = f2(0.f, 0.f), ak1 = ak0, aq0 = ak0, aq1 = ak0;
 #pragma unroll 4
                     for (int r4 = 0; r4 < D / 4; ++r4) {
                         const float4 kt = *reinterpret_cast<const float4 *>(&I.k[ti][4 * r4]);
@@ -654,34 +654,34 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                         ki.y *= ex2_ftz(fminf(gt.y - gi.y, 0.f));
                         ki.z *= ex2_ftz(fminf(gt.z - gi.z, 0.f));
                         ki.w *= ex2_ftz(fminf(gt.w - gi.w, 0.f));
-                        ak = make_float4(fmaf(kt.x, ki.x, ak.x), fmaf(kt.y, ki.y, ak.y), fmaf(kt.z, ki.z, ak.z),
-                                         fmaf(kt.w, ki.w, ak.w));
-                        aq = make_float4(fmaf(qt.x, ki.x, aq.x), fmaf(qt.y, ki.y, aq.y), fmaf(qt.z, ki.z, aq.z),
-                                         fmaf(qt.w, ki.w, aq.w));
+                        ak0 = ffma2(f2(kt.x, kt.y), f2(ki.x, ki.y), ak0);
+                        ak1 = ffma2(f2(kt.z, kt.w), f2(ki.z, ki.w), ak1);
+                        aq0 = ffma2(f2(qt.x, qt.y), f2(ki.x, ki.y), aq0);
+                        aq1 = ffma2(f2(qt.z, qt.w), f2(ki.z, ki.w), aq1);
                     }
-                    dkk = (ak.x + ak.y) + (ak.z + ak.w);
-                    dqk = (aq.x + aq.y) + (aq.z + aq.w);
+                    dkk = (ak0.x + ak0.y) + (ak1.x + ak1.y);
+                    dqk = (aq0.x + aq0.y) + (aq1.x + aq1.y);
                 } else if (warp < 6) {
                     ti = 8 + 4 * (warp - 4) + (lane >> 3);
                     ii = lane & 7;
-                    float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), aq = ak;
+                    float2 ak0 = f2(0.f, 0.f), ak1 = ak0, aq0 = ak0, aq1 = ak0;
 #pragma unroll 4
                     for (int r4 = 0; r4 < D / 4; ++r4) {
                         const float4 kt = *reinterpret_cast<const float4 *>(&S.fac[ti][4 * r4]);
                         const float4 qt = *reinterpret_cast<const float4 *>(&S.fac[ti + 8][4 * r4]);
                         const float4 ki = *reinterpret_cast<const float4 *>(&S.fac[ii][4 * r4]);
-                        ak = make_float4(fmaf(kt.x, ki.x, ak.x), fmaf(kt.y, ki.y, ak.y), fmaf(kt.z, ki.z, ak.z),
-                                         fmaf(kt.w, ki.w, ak.w));
-                        aq = make_float4(fmaf(qt.x, ki.x, aq.x), fmaf(qt.y, ki.y, aq.y), fmaf(qt.z, ki.z, aq.z),
-                                         fmaf(qt.w, ki.w, aq.w));
+                        ak0 = ffma2(f2(kt.x, kt.y), f2(ki.x, ki.y), ak0);
+                        ak1 = ffma2(f2(kt.z, kt.w), f2(ki.z, ki.w), ak1);
+                        aq0 = ffma2(f2(qt.x, qt.y), f2(ki.x, ki.y), aq0);
+                        aq1 = ffma2(f2(qt.z, qt.w), f2(ki.z, ki.w), aq1);
                     }
-                    dkk = (ak.x + ak.y) + (ak.z + ak.w);
-                    dqk = (aq.x + aq.y) + (aq.z + aq.w);
+                    dkk = (ak0.x + ak0.y) + (ak1.x + ak1.y);
+                    dqk = (aq0.x + aq0.y) + (aq1.x + aq1.y);
                 } else {
                     ti = 4 * (warp - 6) + (lane >> 3);
                     ii = 8 + (lane & 7);
                 }
-                S.A[ti][ii] = ii < ti ? I.beta[ti] * dkk : 0.f;
+                S.A[ti][ii] = ii < ti ? -I.beta[ti] * dkk : 0.f;   // stored negated (the substitution adds)
                 S.P[ti][ii] = ii <= ti ? dqk : 0.f;
             }
             ubar();
@@ -695,18 +695,19 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                     if (t < D) x[tt] = I.beta[tt] * (I.k[tt][cc] * ex2_ftz(KDA ? I.g[tt][cc] : I.g[0][tt]));
                     else x[tt] = I.beta[tt] * I.v[tt][cc];
                 }
+                // x_t += sum_{i<t} (-A_ti) x_i, two terms per packed FMA (the
+                // entries past the diagonal are zero)
 #pragma unroll
                 for (int tt = 1; tt < C; ++tt) {
-                    float rhs = x[tt], x1 = 0.f;
+                    float2 acc = f2(x[tt], 0.f);
 #pragma unroll
                     for (int j = 0; 4 * j < tt; ++j) {
                         const float4 a4 = *reinterpret_cast<const float4 *>(&S.A[tt][4 * j]);
-                        rhs = fmaf(-a4.x, x[4 * j], rhs);
-                        if (4 * j + 1 < tt) x1 = fmaf(-a4.y, x[4 * j + 1], x1);
-                        if (4 * j + 2 < tt) rhs = fmaf(-a4.z, x[4 * j + 2], rhs);
-                        if (4 * j + 3 < tt) x1 = fmaf(-a4.w, x[4 * j + 3], x1);
+                        acc = ffma2(f2(a4.x, a4.y), f2(x[4 * j], 4 * j + 1 < tt ? x[4 * j + 1] : 0.f), acc);
+                        if (4 * j + 2 < tt)
+                            acc = ffma2(f2(a4.z, a4.w), f2(x[4 * j + 2], 4 * j + 3 < tt ? x[4 * j + 3] : 0.f), acc);
                     }
-                    x[tt] = rhs + x1;
+                    x[tt] = acc.x + acc.y;
                 }
                 if (t < D) {
 #pragma unroll

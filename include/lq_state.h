@@ -295,8 +295,12 @@ int lq_fit_static_scales(const lq_config *cfg, int32_t n_states, const float *d_
  * LQ_PREFILL_CHUNK tokens in WY form: the chunk's rank-one updates become
  * pseudo-values u by forward substitution, with every decay factor
  * 2^(g_t - g_i), i <= t, from cumulative log2 decays (at most 1 for gates in
- * (0, 1]; gates are floored at 2^-150).  FP32-level accuracy: the d_k x d_v
- * products run on the tensor cores in three TF32 passes, the rest in FP32.
+ * (0, 1]; gates are floored at 2^-150; factors below 2^-126 are flushed to
+ * zero).  FP32-level accuracy: the d_k x d_v products run on the tensor cores
+ * in three TF32 passes, the rest in FP32.  With dk = dv = 128 and q, k, v
+ * (and KDA's alpha) 16-byte aligned the state is held in tensor memory and
+ * the inputs arrive by tensor copies; other shapes and alignments take a
+ * register-state kernel -- the same results up to rounding order.
  *   inputs, token-major stacks of decode-step inputs: q, k [T,B,Hk,dk],
  *     v [T,B,H,dv], beta [T,B,H], alpha [T,B,H] (GDN) or [T,B,H,dk] (KDA)
  *   d_o [T,B,H,dv] receives every token's output (NULL: not written)

@@ -36,6 +36,22 @@ namespace lq {
 
 constexpr int kChunk = 16;
 
+// The hardware base-2 exponential and logarithm (MUFU, ~2 ulp like exp2f /
+// log2f), results below 2^-126 flushed to zero: the decay factors they form
+// multiply keys and states of size <= 1, so a flushed factor changes a value
+// by less than 2^-126.
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float lg2_ftz(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---------------------------------------------------------------------------
 // The chunk step on the tensor cores.  Warp w owns value columns
 // 16w .. 16w+15 and keeps S^T for them in registers as mma.sync m16n8k8
@@ -128,7 +144,7 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
                 const size_t qk = (((size_t)tok * a.B + b) * a.Hk + gk) * DK + r;
                 kv = a.k[qk];
                 qv = a.q[qk];
-                if (KDA) gl = fmaxf(log2f(a.alpha[(((size_t)tok * a.B + b) * a.H + h) * DK + r]), -150.0f);
+                if (KDA) gl = fmaxf(lg2_ftz(a.alpha[(((size_t)tok * a.B + b) * a.H + h) * DK + r]), -150.0f);
             }
             S.kT[r][tt] = kv;
             S.qT[r][tt] = qv;
@@ -142,7 +158,7 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
             const int tok = t0 + t;
             const size_t bh = ((size_t)tok * a.B + b) * a.H + h;
             S.beta[t] = tok < a.T ? a.beta[bh] : 0.f;
-            if (!KDA) S.g[0][t] = tok < a.T ? fmaxf(log2f(a.alpha[bh]), -150.0f) : 0.f;
+            if (!KDA) S.g[0][t] = tok < a.T ? fmaxf(lg2_ftz(a.alpha[bh]), -150.0f) : 0.f;
         }
         __syncthreads();
         // the next chunk's input lines into L2 while this chunk computes: per
@@ -170,7 +186,7 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
                 acc += S.g[t][tt];
                 S.g[t][tt] = acc;
             }
-            S.glast[KDA ? t : 0] = exp2f(acc);
+            S.glast[KDA ? t : 0] = ex2_ftz(acc);
         }
         __syncthreads();
         if (!KDA && t < DK && t > 0) S.glast[t] = S.glast[0];
@@ -178,10 +194,10 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
         for (int e = t; e < C * DK; e += NT) {
             const int r = e % DK, tt = e / DK;
             const float gt = S.g[KDA ? r : 0][tt], gC = S.g[KDA ? r : 0][C - 1];
-            const float et = exp2f(gt);
+            const float et = ex2_ftz(gt);
             S.kg[tt][r] = S.kT[r][tt] * et;
             S.qg[tt][r] = S.qT[r][tt] * et;
-            S.kh[tt][r] = S.kT[r][tt] * exp2f(gC - gt);
+            S.kh[tt][r] = S.kT[r][tt] * ex2_ftz(gC - gt);
         }
         for (int pr = t; pr < C * C; pr += NT) {
             const int ti = pr / C, ii = pr % C;
@@ -190,7 +206,7 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
                 if (KDA) {
 #pragma unroll 8
                     for (int r = 0; r < DK; ++r) {
-                        const float f = exp2f(S.g[r][ti] - S.g[r][ii]) * S.kT[r][ii];
+                        const float f = ex2_ftz(S.g[r][ti] - S.g[r][ii]) * S.kT[r][ii];
                         dkk = fmaf(S.kT[r][ti], f, dkk);
                         dqk = fmaf(S.qT[r][ti], f, dqk);
                     }
@@ -200,7 +216,7 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
                         dkk = fmaf(S.kT[r][ti], S.kT[r][ii], dkk);
                         dqk = fmaf(S.qT[r][ti], S.kT[r][ii], dqk);
                     }
-                    const float f = exp2f(S.g[0][ti] - S.g[0][ii]);
+                    const float f = ex2_ftz(S.g[0][ti] - S.g[0][ii]);
                     dkk *= f;
                     dqk *= f;
                 }
@@ -420,22 +436,6 @@ __device__ __forceinline__ bool ubar_or(bool v) {
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// The hardware base-2 exponential and logarithm (MUFU, ~2 ulp like exp2f /
-// log2f), results below 2^-126 flushed to zero: the decay factors they form
-// multiply keys and states of size <= 1, so a flushed factor changes a value
-// by less than 2^-126.
-__device__ __forceinline__ float ex2_ftz(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ float lg2_ftz(float x) {
-    float y;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
 }
 
 template <bool KDA>

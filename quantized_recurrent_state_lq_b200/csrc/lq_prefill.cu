@@ -593,25 +593,58 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
             }
             ubar();
             if (!KDA) {
-                // pair matrices: warp w takes token rows w (lanes 0-15) and 15 - w
-                // (lanes 16-31), lane % 16 the column; the decay factor
-                // 2^(g_t - g_i) <= 1 is one value per pair
-                const int ti = lane < 16 ? warp : C - 1 - warp, ii = lane & 15;
-                float2 ak0 = f2(0.f, 0.f), ak1 = ak0, aq0 = ak0, aq1 = ak0;   // packed partial sums
-#pragma unroll 4
-                for (int r4 = 0; r4 < D / 4; ++r4) {
-                    const float4 kt = *reinterpret_cast<const float4 *>(&I.k[ti][4 * r4]);
-                    const float4 qt = *reinterpret_cast<const float4 *>(&I.q[ti][4 * r4]);
-                    const float4 ki = *reinterpret_cast<const float4 *>(&I.k[ii][4 * r4]);
-                    ak0 = ffma2(f2(kt.x, kt.y), f2(ki.x, ki.y), ak0);
-                    ak1 = ffma2(f2(kt.z, kt.w), f2(ki.z, ki.w), ak1);
-                    aq0 = ffma2(f2(qt.x, qt.y), f2(ki.x, ki.y), aq0);
-                    aq1 = ffma2(f2(qt.z, qt.w), f2(ki.z, ki.w), aq1);
+                // pair matrices, one decay factor per pair: threads 0-143 take a
+                // 2 x 2 block of the lower triangle (blocks (a, b), b <= a, rows
+                // 2a, 2a+1, columns 2b, 2b+1) over a quarter of the channels
+                // (float4 groups 4 j + quarter), eight packed sums each; the
+                // quarters' partial sums meet in wst (free until the
+                // substitution), then every thread finishes one entry.
+                float *part = &S.wst[0][0];   // [kind][quarter][16][16]
+                if (t < 144) {
+                    const int bi = t >> 2, qu = t & 3;
+                    int ba = 0;
+                    while ((ba + 1) * (ba + 2) / 2 <= bi) ++ba;
+                    const int bb = bi - ba * (ba + 1) / 2;
+                    const int t0 = 2 * ba, i0 = 2 * bb;
+                    float2 kk00 = f2(0.f, 0.f), kk01 = kk00, kk10 = kk00, kk11 = kk00;
+                    float2 qk00 = kk00, qk01 = kk00, qk10 = kk00, qk11 = kk00;
+#pragma unroll 2
+                    for (int j = 0; j < D / 16; ++j) {
+                        const int r = 4 * (4 * j + qu);
+                        const float4 ka = *reinterpret_cast<const float4 *>(&I.k[t0][r]);
+                        const float4 kb = *reinterpret_cast<const float4 *>(&I.k[t0 + 1][r]);
+                        const float4 qa = *reinterpret_cast<const float4 *>(&I.q[t0][r]);
+                        const float4 qb = *reinterpret_cast<const float4 *>(&I.q[t0 + 1][r]);
+                        const float4 ia = *reinterpret_cast<const float4 *>(&I.k[i0][r]);
+                        const float4 ib = *reinterpret_cast<const float4 *>(&I.k[i0 + 1][r]);
+                        kk00 = ffma2(f2(ka.x, ka.y), f2(ia.x, ia.y), ffma2(f2(ka.z, ka.w), f2(ia.z, ia.w), kk00));
+                        kk01 = ffma2(f2(ka.x, ka.y), f2(ib.x, ib.y), ffma2(f2(ka.z, ka.w), f2(ib.z, ib.w), kk01));
+                        kk10 = ffma2(f2(kb.x, kb.y), f2(ia.x, ia.y), ffma2(f2(kb.z, kb.w), f2(ia.z, ia.w), kk10));
+                        kk11 = ffma2(f2(kb.x, kb.y), f2(ib.x, ib.y), ffma2(f2(kb.z, kb.w), f2(ib.z, ib.w), kk11));
+                        qk00 = ffma2(f2(qa.x, qa.y), f2(ia.x, ia.y), ffma2(f2(qa.z, qa.w), f2(ia.z, ia.w), qk00));
+                        qk01 = ffma2(f2(qa.x, qa.y), f2(ib.x, ib.y), ffma2(f2(qa.z, qa.w), f2(ib.z, ib.w), qk01));
+                        qk10 = ffma2(f2(qb.x, qb.y), f2(ia.x, ia.y), ffma2(f2(qb.z, qb.w), f2(ia.z, ia.w), qk10));
+                        qk11 = ffma2(f2(qb.x, qb.y), f2(ib.x, ib.y), ffma2(f2(qb.z, qb.w), f2(ib.z, ib.w), qk11));
+                    }
+                    float *pk = part + qu * 256, *pq = part + 1024 + qu * 256;
+                    pk[t0 * 16 + i0] = kk00.x + kk00.y;
+                    pk[t0 * 16 + i0 + 1] = kk01.x + kk01.y;
+                    pk[(t0 + 1) * 16 + i0] = kk10.x + kk10.y;
+                    pk[(t0 + 1) * 16 + i0 + 1] = kk11.x + kk11.y;
+                    pq[t0 * 16 + i0] = qk00.x + qk00.y;
+                    pq[t0 * 16 + i0 + 1] = qk01.x + qk01.y;
+                    pq[(t0 + 1) * 16 + i0] = qk10.x + qk10.y;
+                    pq[(t0 + 1) * 16 + i0 + 1] = qk11.x + qk11.y;
                 }
-                const float f = ex2_ftz(fminf(I.g[0][ti] - I.g[0][ii], 0.f));
-                const float dkk = ((ak0.x + ak0.y) + (ak1.x + ak1.y)) * f, dqk = ((aq0.x + aq0.y) + (aq1.x + aq1.y)) * f;
-                S.A[ti][ii] = ii < ti ? -I.beta[ti] * dkk : 0.f;   // stored negated (the substitution adds)
-                S.P[ti][ii] = ii <= ti ? dqk : 0.f;
+                ubar();
+                {   // entry (ti, ii) = (t / 16, t % 16)
+                    const int ti = t >> 4, ii = t & 15;
+                    const float f = ex2_ftz(fminf(I.g[0][ti] - I.g[0][ii], 0.f));
+                    const float dkk = ((part[t] + part[256 + t]) + (part[512 + t] + part[768 + t])) * f;
+                    const float dqk = ((part[1024 + t] + part[1280 + t]) + (part[1536 + t] + part[1792 + t])) * f;
+                    S.A[ti][ii] = ii < ti ? -I.beta[ti] * dkk : 0.f;   // stored negated (the substitution adds)
+                    S.P[ti][ii] = ii <= ti ? dqk : 0.f;
+                }
             } else {
                 // KDA: per-channel factors 2^(g_t - g_i).  Across the two
                 // 8-token halves (t >= 8 > 7 >= i) they factor through token 7,

@@ -326,8 +326,9 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
 // ---------------------------------------------------------------------------
 // d_k = d_v = 128: the chunk step on the fifth-generation tensor cores, in
 // chunks of kUChunk = 16 tokens, one CTA per head (one per SM: the state's
-// tensor memory) of 8 compute warps and one warp that issues the MMAs.  The chunk's pseudo-values are solved without the
-// state first: with A the strictly lower pair matrix above,
+// tensor memory) of a tensor-memory warpgroup and an 8-warp preparation
+// group.  The chunk's pseudo-values are solved without the state first: with
+// A the strictly lower pair matrix above,
 //   (I + A) W = diag(b) Kg,   (I + A) Ut = diag(b) V     (rows = tokens)
 // by forward substitution (a key or value column per thread), so that
 //   U = Ut - W S,   O = Qg S + P U,   S <- diag(Gamma_C) S + Kh^T U
@@ -339,18 +340,19 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
 //             tokens; A = U^T from shared memory, U = Ut + U')
 // each product in three TF32 passes (big x big + big x small + small x big);
 // stacking the two right-hand sides of each group makes it one MMA chain.
-// Everything that does not need the state -- the next chunk's decays, pair
-// matrices, substitution and operand splits -- runs on the compute warps while
-// a group is in flight (the MMA warp waits on mbarriers, so its issue time is
-// off their path): the next chunk's inputs arrive by bulk copies two chunks ahead
-// (two input slots), and the operands that group 2 may still read while the
-// next chunk's are written (Kh, P) have two slots.  Tensor memory: S^T
-// columns 0-127, O^T 128-143, U'^T 144-159, S^T's big and small parts
-// 256-383 and 384-511.
+// The tensor-memory warpgroup (warps 0-3, a value column per thread) splits
+// the state, issues both groups and forms U^T and the outputs; everything that
+// does not need the state -- the next chunk's decays, pair matrices,
+// substitution and operand splits -- runs meanwhile on the preparation group
+// (warps 4-11), the two handing buffers over by mbarriers.  The inputs arrive
+// by tensor copies two chunks ahead (two input slots); the buffers a chunk
+// reads after its group 1 (Ut, Gamma_C, [Kh; P]) have two slots.  Tensor
+// memory: S^T columns 0-127, O^T 128-143, U'^T 144-159, S^T's big and small
+// parts 256-383 and 384-511.
 // ---------------------------------------------------------------------------
 constexpr int kUChunk = 16;
-constexpr int kUCompute = 256;               // compute warps 0-7
-constexpr int kUThreads = kUCompute + 32;    // and the MMA warp
+constexpr int kUCompute = 256;               // the preparation group (warps 4-11)
+constexpr int kUThreads = 128 + kUCompute;   // after the tensor-memory warpgroup (warps 0-3)
 
 template <bool KDA>
 struct alignas(128) PrefillUIn {   // one chunk's inputs (token rows padded against bank conflicts;
@@ -379,8 +381,9 @@ struct PrefillUSmem {
     alignas(16) float P[C][C + 4];
     float gC[2][D];                          // [slot]: Gamma over the whole chunk, per key row
     uint64_t mbar_in[2];       // input slot filled
-    uint64_t mbar_s, mbar_u;   // the state split / U^T written (compute warps -> MMA warp)
-    uint64_t mbar_yo, mbar_up; // group 1 / group 2 complete (tensor core -> compute warps)
+    uint64_t mbar_ops;         // a chunk's operands written (preparation group -> tensor-memory warpgroup)
+    uint64_t mbar_yo;          // group 1 complete
+    uint64_t mbar_up[2];       // group 2 of an even / odd chunk complete
     uint32_t tmem_base;
 };
 
@@ -417,8 +420,7 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-// Named barrier of the compute warps (warps 0-7; the MMA warp stays out), and
-// its OR-reduction form.
+// Named barrier of the preparation group (warps 4-11), and its OR form.
 __device__ __forceinline__ void ubar() { asm volatile("bar.sync 1, %0;" ::"n"(kUCompute) : "memory"); }
 
 __device__ __forceinline__ bool ubar_or(bool v) {
@@ -430,6 +432,22 @@ __device__ __forceinline__ bool ubar_or(bool v) {
         "selp.s32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
         : "r"((int)v), "n"(kUCompute)
+        : "memory");
+    return r != 0;
+}
+
+// Named barrier of the tensor-memory warpgroup (warps 0-3), and its OR form.
+__device__ __forceinline__ void tbar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+__device__ __forceinline__ bool tbar_or(bool v) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.s32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 2, 128, p;\n\t"
+        "selp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((int)v)
         : "memory");
     return r != 0;
 }
@@ -448,9 +466,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
     Sm &S = *reinterpret_cast<Sm *>(smem_u);
     const int head = blockIdx.x;
     const int b = head / a.H, h = head - b * a.H, gk = (h * a.Hk) / a.H;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int quad = warp & 3, half = (warp >> 2) & 1;   // tensor-memory lanes 32 quad.., column / token half
-    const int col = 32 * quad + lane;                    // the value column (tensor-memory lane) of this thread
+    const int lane = threadIdx.x & 31;
     const size_t state_off = (size_t)head * D * D;
     const int nchunks = (a.T + C - 1) / C;
     constexpr uint32_t cS = 0, cO = 128, cU = 144, cSb = 256, cSs = 384;
@@ -458,16 +474,16 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
     constexpr uint32_t IDESC_G2 = umma_idesc_tf32(128, D + C);
     const bool want_o = a.o != nullptr;
 
-    if (t == 0) {
+    if (threadIdx.x == 0) {
         mbar_init(&S.mbar_in[0], 1);
         mbar_init(&S.mbar_in[1], 1);
+        mbar_init(&S.mbar_ops, 1);
         mbar_init(&S.mbar_yo, 1);
-        mbar_init(&S.mbar_up, 1);
-        mbar_init(&S.mbar_s, 1);
-        mbar_init(&S.mbar_u, 1);
+        mbar_init(&S.mbar_up[0], 1);
+        mbar_init(&S.mbar_up[1], 1);
         fence_mbar_init();
     }
-    if (warp == 0) {
+    if (threadIdx.x < 32) {
         tmem_alloc(&S.tmem_base, 512);
         tmem_relinquish();
     }
@@ -476,53 +492,160 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
 
-    if (warp == kUCompute / 32) {
-        // The MMA warp: per chunk, group 1 once the state is split, group 2
-        // once U^T is in shared memory; completions go to mbar_yo / mbar_up.
-        if (lane == 0) {
+    if (threadIdx.x < 128) {
+        // The tensor-memory warpgroup: thread t = value column t = tensor-memory
+        // lane t.  Per chunk: wait for the preparation group's operands, the
+        // previous chunk's outputs, the state split, group 1, U^T, group 2.
+        const int t = threadIdx.x, col = t;
+        const uint32_t trow = tmem + ((uint32_t)(t & ~31) << 16);   // this warp's 32 lanes
+        // S^T lane col = column col of S0
 #pragma unroll 1
-            for (int ch = 0; ch < nchunks; ++ch) {
-                const int sl = ch & 1;
-                if (!mbar_wait_bounded(&S.mbar_s, (uint32_t)(ch & 1), a.status)) break;
-                tc_fence_after();
-                {   // 16 K-blocks of 8 key rows, three passes each; a K-block is
-                    // 8 x 2C x 4 bytes (1 KB) of each part of [Qg; -W]
-                    const uint64_t db = umma_smem_desc(&S.qw[0][0], 2 * C * 16, 128);
-                    const uint64_t ds = umma_smem_desc(&S.qw[1][0], 2 * C * 16, 128);
-#pragma unroll 1
-                    for (int kb = 0; kb < D / 8; ++kb) {
-                        const uint32_t ab = tmem + cSb + 8u * kb, as = tmem + cSs + 8u * kb;
-                        const uint64_t off = (uint64_t)(kb * 8 * 2 * C * 4) >> 4;
-                        umma_tf32_ta(tmem + cO, ab, db + off, IDESC_G1, kb > 0 ? 1u : 0u);
-                        umma_tf32_ta(tmem + cO, ab, ds + off, IDESC_G1, 1u);
-                        umma_tf32_ta(tmem + cO, as, db + off, IDESC_G1, 1u);
-                    }
-                    umma_commit(&S.mbar_yo);
-                }
-                if (!mbar_wait_bounded(&S.mbar_u, (uint32_t)(ch & 1), a.status)) break;
-                tc_fence_after();
-                {   // 2 K-blocks of 8 tokens, three passes each; a K-block is
-                    // 8 D x 4 words of U^T and 8 (D + C) x 4 words of [Kh; P]
-                    const uint64_t ub = umma_smem_desc(&S.ut[0][0], D * 16, 128);
-                    const uint64_t us = umma_smem_desc(&S.ut[1][0], D * 16, 128);
-                    const uint64_t hb = umma_smem_desc(&S.khp[sl][0][0], (D + C) * 16, 128);
-                    const uint64_t hs = umma_smem_desc(&S.khp[sl][1][0], (D + C) * 16, 128);
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t w[32];
 #pragma unroll
-                    for (int kb = 0; kb < C / 8; ++kb) {
-                        const uint64_t ou = (uint64_t)(kb * 8 * D * 4) >> 4;
-                        const uint64_t oh = (uint64_t)(kb * 8 * (D + C) * 4) >> 4;
-                        umma_tf32(tmem + cS, ub + ou, hb + oh, IDESC_G2, 1u);
-                        umma_tf32(tmem + cS, ub + ou, hs + oh, IDESC_G2, 1u);
-                        umma_tf32(tmem + cS, us + ou, hb + oh, IDESC_G2, 1u);
-                    }
-                    umma_commit(&S.mbar_up);
+            for (int j = 0; j < 32; ++j)
+                w[j] = __float_as_uint(a.S0 ? a.S0[state_off + (size_t)(c0 + j) * D + col] : 0.0f);
+            tmem_st_32x32b_x32(trow + cS + c0, w);
+        }
+        tmem_st_wait();
+        // the outputs of chunk c from O^T in tensor memory
+        auto store_outputs = [&](int c) {
+            uint32_t w[16];
+            tmem_ld_32x32b<16>(trow + cO, w);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < C; ++j) {
+                const int tok = c * C + j;
+                if (tok < a.T) a.o[(((size_t)tok * a.B + b) * a.H + h) * D + col] = __uint_as_float(w[j]);
+            }
+        };
+        bool ok = true;
+#pragma unroll 1
+        for (int ch = 0; ch < nchunks; ++ch) {
+            const int sl = ch & 1;
+            {   // chunk ch's operands, and the previous chunk's group 2
+                bool okw = mbar_wait_bounded(&S.mbar_ops, (uint32_t)(ch & 1), a.status);
+                if (ch > 0 && okw)
+                    okw = mbar_wait_bounded(&S.mbar_up[(ch - 1) & 1], (uint32_t)(((ch - 1) >> 1) & 1), a.status);
+                if (tbar_or(!okw)) {
+                    ok = false;
+                    break;
                 }
             }
+            tc_fence_after();
+            if (ch > 0 && want_o) store_outputs(ch - 1);
+            // S^T split into group 1's A operand and scaled by this chunk's Gamma
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t w[32], wb[32], ws[32];
+                tmem_ld_32x32b<32>(trow + cS + (uint32_t)c0, w);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float x = __uint_as_float(w[j]);
+                    tf32_split(x, wb[j], ws[j]);
+                    w[j] = __float_as_uint(x * S.gC[sl][KDA ? c0 + j : 0]);
+                }
+                tmem_st_32x32b_x32(trow + cSb + (uint32_t)c0, wb);
+                tmem_st_32x32b_x32(trow + cSs + (uint32_t)c0, ws);
+                tmem_st_32x32b_x32(trow + cS + (uint32_t)c0, w);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            tbar();
+            if (t == 0) {   // group 1: 16 K-blocks of 8 key rows, three passes each
+                tc_fence_after();
+                const uint64_t db = umma_smem_desc(&S.qw[0][0], 2 * C * 16, 128);
+                const uint64_t ds = umma_smem_desc(&S.qw[1][0], 2 * C * 16, 128);
+#pragma unroll 1
+                for (int kb = 0; kb < D / 8; ++kb) {
+                    const uint32_t ab = tmem + cSb + 8u * kb, as = tmem + cSs + 8u * kb;
+                    const uint64_t off = (uint64_t)(kb * 8 * 2 * C * 4) >> 4;
+                    umma_tf32_ta(tmem + cO, ab, db + off, IDESC_G1, kb > 0 ? 1u : 0u);
+                    umma_tf32_ta(tmem + cO, ab, ds + off, IDESC_G1, 1u);
+                    umma_tf32_ta(tmem + cO, as, db + off, IDESC_G1, 1u);
+                }
+                umma_commit(&S.mbar_yo);
+            }
+            __syncwarp();
+            {
+                const bool okw = mbar_wait_bounded(&S.mbar_yo, (uint32_t)(ch & 1), a.status);
+                if (tbar_or(!okw)) {
+                    ok = false;
+                    break;
+                }
+            }
+            tc_fence_after();
+            {   // U = Ut + U' into group 2's A operand
+                uint32_t w[16];
+                tmem_ld_32x32b<16>(trow + cU, w);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j4 = 0; j4 < C / 4; ++j4) {
+                    const int tt = 4 * j4;
+                    float4 u;
+                    u.x = S.ud[sl][tt][col] + __uint_as_float(w[tt]);
+                    u.y = S.ud[sl][tt + 1][col] + __uint_as_float(w[tt + 1]);
+                    u.z = S.ud[sl][tt + 2][col] + __uint_as_float(w[tt + 2]);
+                    u.w = S.ud[sl][tt + 3][col] + __uint_as_float(w[tt + 3]);
+                    uint4 bb, bs;
+                    split4(u, bb, bs);
+                    const int wd = umma_word(D, col, tt);
+                    *reinterpret_cast<uint4 *>(&S.ut[0][wd]) = bb;
+                    *reinterpret_cast<uint4 *>(&S.ut[1][wd]) = bs;
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            tbar();
+            if (t == 0) {   // group 2: 2 K-blocks of 8 tokens, three passes each
+                tc_fence_after();
+                const uint64_t ub = umma_smem_desc(&S.ut[0][0], D * 16, 128);
+                const uint64_t us = umma_smem_desc(&S.ut[1][0], D * 16, 128);
+                const uint64_t hb = umma_smem_desc(&S.khp[sl][0][0], (D + C) * 16, 128);
+                const uint64_t hs = umma_smem_desc(&S.khp[sl][1][0], (D + C) * 16, 128);
+#pragma unroll
+                for (int kb = 0; kb < C / 8; ++kb) {
+                    const uint64_t ou = (uint64_t)(kb * 8 * D * 4) >> 4;
+                    const uint64_t oh = (uint64_t)(kb * 8 * (D + C) * 4) >> 4;
+                    umma_tf32(tmem + cS, ub + ou, hb + oh, IDESC_G2, 1u);
+                    umma_tf32(tmem + cS, ub + ou, hs + oh, IDESC_G2, 1u);
+                    umma_tf32(tmem + cS, us + ou, hb + oh, IDESC_G2, 1u);
+                }
+                umma_commit(&S.mbar_up[sl]);
+            }
+            __syncwarp();
         }
-        __syncwarp();
+        // the last chunk's group 2, its outputs and the final state
+        if (ok && nchunks > 0) {
+            const bool okw =
+                mbar_wait_bounded(&S.mbar_up[(nchunks - 1) & 1], (uint32_t)(((nchunks - 1) >> 1) & 1), a.status);
+            ok = !tbar_or(!okw);
+            tc_fence_after();
+            if (ok && want_o) store_outputs(nchunks - 1);
+        }
+        if (ok) {
+            bool fin = true;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t w[32];
+                tmem_ld_32x32b<32>(trow + cS + (uint32_t)c0, w);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float x = __uint_as_float(w[j]);
+                    fin = fin && isfinite(x);
+                    a.S_out[state_off + (size_t)(c0 + j) * D + col] = x;
+                }
+            }
+            if (!fin && a.status) atomicOr(a.status, kStatusNonFinite);
+        }
     } else {
-        const uint32_t trow = tmem + ((uint32_t)(32 * quad) << 16);   // this warp's 32 lanes
-
+        // The preparation group (warps 4-11; t, warp: its own thread and warp
+        // index): per chunk the decays, pair matrices, substitution and operand
+        // splits, into the buffers the tensor-memory warpgroup has finished
+        // with, then one arrival on mbar_ops.
+        const int t = threadIdx.x - 128, warp = t >> 5;
         // Chunk c's token rows into input slot c % 2: one tensor copy per array
         // (rows past T: zeros), completing on mbar_in[c % 2].  Starts with a
         // barrier (the slot's previous contents have been read).
@@ -808,142 +931,46 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
             if (c + 2 < nchunks) issue_load(c + 2);   // its barrier also orders the reads above
         };
 
-        // The outputs of chunk c from O^T in tensor memory (tokens 8 half ..).
-        auto store_outputs = [&](int c) {
-            uint32_t w[8];
-            tmem_ld_32x32b<8>(trow + cO + 8u * half, w);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int tok = c * C + 8 * half + j;
-                if (tok < a.T) a.o[(((size_t)tok * a.B + b) * a.H + h) * D + col] = __uint_as_float(w[j]);
-            }
-        };
-
         bool ok = true;
-        float bet = 0.f, gl = 0.f;
-        if (nchunks > 0) {   // the first two chunks' inputs in flight during the state's copy
+        float bet = 0.f, gl = 0.f, bet_n = 0.f, gl_n = 0.f;
+        if (nchunks > 0) {
             load_scalars(0, bet, gl);
             issue_load(0);
             if (nchunks > 1) issue_load(1);
         }
-        // S^T lane col = column col of S0; warp half `half` writes key rows 64 half ..
 #pragma unroll 1
-        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
-            uint32_t w[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                w[j] = __float_as_uint(a.S0 ? a.S0[state_off + (size_t)(c0 + j) * D + col] : 0.0f);
-            tmem_st_32x32b_x32(trow + cS + c0, w);
-        }
-        tmem_st_wait();
-        if (nchunks > 0) {
-            ok = prep_solve(0, bet, gl);
-            if (ok) prep_operands(0);
-        }
-#pragma unroll 1
-        for (int ch = 0; ok && ch < nchunks; ++ch) {
-            const int sl = ch & 1;
-            if (ch + 1 < nchunks) load_scalars(ch + 1, bet, gl);
-            // (1) the previous chunk's group 2 is complete: its outputs, then S^T
-            // split into group 1's A operand and scaled by this chunk's Gamma
-            if (ch > 0) {
-                const bool okw = mbar_wait_bounded(&S.mbar_up, (uint32_t)((ch - 1) & 1), a.status);
+        for (int c = 0; ok && c < nchunks; ++c) {
+            if (c + 1 < nchunks) load_scalars(c + 1, bet_n, gl_n);
+            // ud, gC and the [Kh; P] slot of c % 2 were last read by chunk c - 2
+            if (c >= 2) {
+                const bool okw = mbar_wait_bounded(&S.mbar_up[c & 1], (uint32_t)(((c - 2) >> 1) & 1), a.status);
                 if (ubar_or(!okw)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                if (want_o) store_outputs(ch - 1);
             }
-#pragma unroll 1
-            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
-                uint32_t w[32], wb[32], ws[32];
-                tmem_ld_32x32b<32>(trow + cS + (uint32_t)c0, w);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float x = __uint_as_float(w[j]);
-                    tf32_split(x, wb[j], ws[j]);
-                    w[j] = __float_as_uint(x * S.gC[sl][KDA ? c0 + j : 0]);
-                }
-                tmem_st_32x32b_x32(trow + cSb + (uint32_t)c0, wb);
-                tmem_st_32x32b_x32(trow + cSs + (uint32_t)c0, ws);
-                tmem_st_32x32b_x32(trow + cS + (uint32_t)c0, w);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            ubar();
-            if (t == 0) mbar_arrive(&S.mbar_s);   // (2) group 1 goes
-            // (3) while group 1 runs: the next chunk's decays, pairs and substitution
-            if (ch + 1 < nchunks && !prep_solve(ch + 1, bet, gl)) {
+            if (!prep_solve(c, bet, gl)) {
                 ok = false;
-                mbar_wait_bounded(&S.mbar_yo, (uint32_t)(ch & 1), a.status);   // group 1 is in flight
                 break;
             }
-            // (4) group 1 complete: U = Ut + U' into the A operand of group 2
-            {
-                const bool okw = mbar_wait_bounded(&S.mbar_yo, (uint32_t)(ch & 1), a.status);
+            // [Qg; -W] was last read by chunk c - 1's group 1
+            if (c >= 1) {
+                const bool okw = mbar_wait_bounded(&S.mbar_yo, (uint32_t)((c - 1) & 1), a.status);
                 if (ubar_or(!okw)) {
                     ok = false;
                     break;
                 }
             }
-            tc_fence_after();
-            {
-                uint32_t w[8];
-                tmem_ld_32x32b<8>(trow + cU + 8u * half, w);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j4 = 0; j4 < 2; ++j4) {
-                    const int tt = 8 * half + 4 * j4;
-                    float4 u;
-                    u.x = S.ud[sl][tt][col] + __uint_as_float(w[4 * j4]);
-                    u.y = S.ud[sl][tt + 1][col] + __uint_as_float(w[4 * j4 + 1]);
-                    u.z = S.ud[sl][tt + 2][col] + __uint_as_float(w[4 * j4 + 2]);
-                    u.w = S.ud[sl][tt + 3][col] + __uint_as_float(w[4 * j4 + 3]);
-                    uint4 bb, bs;
-                    split4(u, bb, bs);
-                    const int wd = umma_word(D, col, tt);
-                    *reinterpret_cast<uint4 *>(&S.ut[0][wd]) = bb;
-                    *reinterpret_cast<uint4 *>(&S.ut[1][wd]) = bs;
-                }
-            }
-            fence_async_smem();
-            tc_fence_before();
+            prep_operands(c);
             ubar();
-            if (t == 0) mbar_arrive(&S.mbar_u);   // (5) group 2 goes
-            // (6) while group 2 runs: the next chunk's operand splits (qw: read by
-            // group 1, complete; [Kh; P]: the other slot)
-            if (ch + 1 < nchunks) prep_operands(ch + 1);
-        }
-        // the last chunk's group 2, its outputs and the final state
-        if (ok && nchunks > 0) {
-            const bool okw = mbar_wait_bounded(&S.mbar_up, (uint32_t)((nchunks - 1) & 1), a.status);
-            ok = !ubar_or(!okw);
-            tc_fence_after();
-            if (ok && want_o) store_outputs(nchunks - 1);
-        }
-        if (ok) {
-            bool fin = true;
-#pragma unroll 1
-            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
-                uint32_t w[32];
-                tmem_ld_32x32b<32>(trow + cS + (uint32_t)c0, w);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float x = __uint_as_float(w[j]);
-                    fin = fin && isfinite(x);
-                    a.S_out[state_off + (size_t)(c0 + j) * D + col] = x;
-                }
-            }
-            if (!fin && a.status) atomicOr(a.status, kStatusNonFinite);
+            if (t == 0) mbar_arrive(&S.mbar_ops);
+            bet = bet_n;
+            gl = gl_n;
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (threadIdx.x < 32) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

@@ -335,7 +335,8 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
 // are products only, all on the tensor cores with the state in tensor memory
 // as S^T [d_v lanes x d_k columns] (FP32, the update's accumulator):
 //   group 1:  [Oi^T | U'^T] = S^T [Qg; -W]^T        (M = d_v, N = 32, K = d_k;
-//             A = S^T's TF32 big and small parts, also in tensor memory)
+//             A = S^T's TF32 big and small parts, also in tensor memory; the
+//             big part times both parts of B in one N = 64 MMA)
 //   group 2:  [S^T | O^T] += U^T [Kh; P]^T           (N = d_k + 16, K = 16
 //             tokens; A = U^T from shared memory, U = Ut + U')
 // each product in three TF32 passes (big x big + big x small + small x big);
@@ -347,8 +348,9 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
 // (warps 4-11), the two handing buffers over by mbarriers.  The inputs arrive
 // by tensor copies two chunks ahead (two input slots); the buffers a chunk
 // reads after its group 1 (Ut, Gamma_C, [Kh; P]) have two slots.  Tensor
-// memory: S^T columns 0-127, O^T 128-143, U'^T 144-159, S^T's big and small
-// parts 256-383 and 384-511.
+// memory: S^T columns 0-127; group 1's three passes as three [Oi^T | U'^T]
+// partials at 128, 160, 192 (their sum is the product; group 2 adds U^T P^T
+// onto the first); S^T's big and small parts 256-383 and 384-511.
 // ---------------------------------------------------------------------------
 constexpr int kUChunk = 16;
 constexpr int kUCompute = 256;               // the preparation group (warps 4-11)
@@ -370,7 +372,7 @@ struct PrefillUSmem {
     static constexpr int D = 128, C = kUChunk, RP = D + 4;
     // MMA operands, TF32 big [0] and small [1], K-major core matrices: word
     // (row x, k) at (k / 4) rows 4 + (x / 8) 32 + (x % 8) 4 + k % 4
-    alignas(128) uint32_t qw[2][2 * C * D];         // B of group 1: [Qg; -W] [N = 2C tokens][K = D key rows]
+    alignas(128) uint32_t qw[4 * C * D];            // B of group 1: [Qg; -W] big, then small: [N = 4C][K = D key rows]
     alignas(128) uint32_t khp[2][2][(D + C) * C];   // [slot]: B of group 2: [Kh; P] [N = D + C][K = C tokens]
     alignas(128) uint32_t ut[2][D * C];             // A of group 2: U^T [M = D value columns][K = C tokens]
     alignas(16) float ud[2][C][D];           // [slot]: Ut
@@ -469,8 +471,11 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
     const int lane = threadIdx.x & 31;
     const size_t state_off = (size_t)head * D * D;
     const int nchunks = (a.T + C - 1) / C;
+    // group 1 in two MMAs a K-block: S_big [Qg; -W]_big|small (N = 64) into
+    // cO .. cO+63 and S_small [Qg; -W]_big (N = 32) into cO+64 .. cO+95: three
+    // [Oi | U'] partials at cO, cO+32, cO+64; group 2 accumulates onto the first
     constexpr uint32_t cS = 0, cO = 128, cU = 144, cSb = 256, cSs = 384;
-    constexpr uint32_t IDESC_G1 = umma_idesc_tf32(128, 2 * C);
+    constexpr uint32_t IDESC_G1W = umma_idesc_tf32(128, 4 * C), IDESC_G1 = umma_idesc_tf32(128, 2 * C);
     constexpr uint32_t IDESC_G2 = umma_idesc_tf32(128, D + C);
     const bool want_o = a.o != nullptr;
 
@@ -510,13 +515,16 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
         tmem_st_wait();
         // the outputs of chunk c from O^T in tensor memory
         auto store_outputs = [&](int c) {
-            uint32_t w[16];
-            tmem_ld_32x32b<16>(trow + cO, w);
+            uint32_t w0[16], w1[16], w2[16];
+            tmem_ld_32x32b<16>(trow + cO, w0);
+            tmem_ld_32x32b<16>(trow + cO + 32, w1);
+            tmem_ld_32x32b<16>(trow + cO + 64, w2);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < C; ++j) {
                 const int tok = c * C + j;
-                if (tok < a.T) a.o[(((size_t)tok * a.B + b) * a.H + h) * D + col] = __uint_as_float(w[j]);
+                const float o = __uint_as_float(w0[j]) + (__uint_as_float(w1[j]) + __uint_as_float(w2[j]));
+                if (tok < a.T) a.o[(((size_t)tok * a.B + b) * a.H + h) * D + col] = o;
             }
         };
         bool ok = true;
@@ -553,17 +561,18 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
             tmem_st_wait();
             tc_fence_before();
             tbar();
-            if (t == 0) {   // group 1: 16 K-blocks of 8 key rows, three passes each
+            if (t == 0) {   // group 1: 16 K-blocks of 8 key rows, two MMAs each
                 tc_fence_after();
-                const uint64_t db = umma_smem_desc(&S.qw[0][0], 2 * C * 16, 128);
-                const uint64_t ds = umma_smem_desc(&S.qw[1][0], 2 * C * 16, 128);
+                // [4C rows][D]: a K-block is 8 x 4C x 4 bytes (2 KB); its first 2C
+                // rows are the big parts
+                const uint64_t dq = umma_smem_desc(&S.qw[0], 4 * C * 16, 128);
 #pragma unroll 1
                 for (int kb = 0; kb < D / 8; ++kb) {
                     const uint32_t ab = tmem + cSb + 8u * kb, as = tmem + cSs + 8u * kb;
-                    const uint64_t off = (uint64_t)(kb * 8 * 2 * C * 4) >> 4;
-                    umma_tf32_ta(tmem + cO, ab, db + off, IDESC_G1, kb > 0 ? 1u : 0u);
-                    umma_tf32_ta(tmem + cO, ab, ds + off, IDESC_G1, 1u);
-                    umma_tf32_ta(tmem + cO, as, db + off, IDESC_G1, 1u);
+                    const uint64_t off = (uint64_t)(kb * 8 * 4 * C * 4) >> 4;
+                    const uint32_t acc = kb > 0 ? 1u : 0u;
+                    umma_tf32_ta(tmem + cO, ab, dq + off, IDESC_G1W, acc);
+                    umma_tf32_ta(tmem + cO + 64, as, dq + off, IDESC_G1, acc);
                 }
                 umma_commit(&S.mbar_yo);
             }
@@ -576,18 +585,24 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                 }
             }
             tc_fence_after();
-            {   // U = Ut + U' into group 2's A operand
-                uint32_t w[16];
-                tmem_ld_32x32b<16>(trow + cU, w);
+            {   // U = Ut + U' (the three passes' sum) into group 2's A operand
+                uint32_t w0[16], w1[16], w2[16];
+                tmem_ld_32x32b<16>(trow + cU, w0);
+                tmem_ld_32x32b<16>(trow + cU + 32, w1);
+                tmem_ld_32x32b<16>(trow + cU + 64, w2);
                 tmem_ld_wait();
+                float w[16];
+#pragma unroll
+                for (int j = 0; j < C; ++j)
+                    w[j] = __uint_as_float(w0[j]) + (__uint_as_float(w1[j]) + __uint_as_float(w2[j]));
 #pragma unroll
                 for (int j4 = 0; j4 < C / 4; ++j4) {
                     const int tt = 4 * j4;
                     float4 u;
-                    u.x = S.ud[sl][tt][col] + __uint_as_float(w[tt]);
-                    u.y = S.ud[sl][tt + 1][col] + __uint_as_float(w[tt + 1]);
-                    u.z = S.ud[sl][tt + 2][col] + __uint_as_float(w[tt + 2]);
-                    u.w = S.ud[sl][tt + 3][col] + __uint_as_float(w[tt + 3]);
+                    u.x = S.ud[sl][tt][col] + w[tt];
+                    u.y = S.ud[sl][tt + 1][col] + w[tt + 1];
+                    u.z = S.ud[sl][tt + 2][col] + w[tt + 2];
+                    u.w = S.ud[sl][tt + 3][col] + w[tt + 3];
                     uint4 bb, bs;
                     split4(u, bb, bs);
                     const int wd = umma_word(D, col, tt);
@@ -885,11 +900,13 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
             ubar();
             for (int e = t; e < C * D / 4; e += NT) {   // Qg, -W: token e % C, key rows 4 (e / C) ..
                 const int tt = e % C, r = 4 * (e / C);
-                const int wq = umma_word(2 * C, tt, r), ww = umma_word(2 * C, C + tt, r);
+                // rows: Qg big tt, -W big C + tt, Qg small 2C + tt, -W small 3C + tt
+                const int wq = umma_word(4 * C, tt, r), ww = umma_word(4 * C, C + tt, r);
+                const int sq = umma_word(4 * C, 2 * C + tt, r), sw = umma_word(4 * C, 3 * C + tt, r);
                 uint4 bb, bs;
                 split4(*reinterpret_cast<const float4 *>(&S.wst[tt][r]), bb, bs);
-                *reinterpret_cast<uint4 *>(&S.qw[0][ww]) = bb;
-                *reinterpret_cast<uint4 *>(&S.qw[1][ww]) = bs;
+                *reinterpret_cast<uint4 *>(&S.qw[ww]) = bb;
+                *reinterpret_cast<uint4 *>(&S.qw[sw]) = bs;
                 float4 qv = *reinterpret_cast<const float4 *>(&I.q[tt][r]);
                 float4 ev;
                 if (KDA) {
@@ -901,8 +918,8 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                 }
                 qv = make_float4(qv.x * ev.x, qv.y * ev.y, qv.z * ev.z, qv.w * ev.w);
                 split4(qv, bb, bs);
-                *reinterpret_cast<uint4 *>(&S.qw[0][wq]) = bb;
-                *reinterpret_cast<uint4 *>(&S.qw[1][wq]) = bs;
+                *reinterpret_cast<uint4 *>(&S.qw[wq]) = bb;
+                *reinterpret_cast<uint4 *>(&S.qw[sq]) = bs;
             }
             for (int e = t; e < D * C / 4; e += NT) {   // Kh: key row e % D, tokens 4 (e / D) ..
                 const int r = e % D, t4 = 4 * (e / D);

@@ -353,8 +353,8 @@ __global__ void __launch_bounds__(2 * DV, 2) prefill_tc_kernel(const PrefillArgs
 // onto the first); S^T's big and small parts 256-383 and 384-511.
 // ---------------------------------------------------------------------------
 constexpr int kUChunk = 16;
-constexpr int kUCompute = 256;               // the preparation group (warps 4-11)
-constexpr int kUThreads = 128 + kUCompute;   // after the tensor-memory warpgroup (warps 0-3)
+constexpr int kUPrep = 256;               // the preparation group (warps 4-11)
+constexpr int kUThreads = 128 + kUPrep;   // after the tensor-memory warpgroup (warps 0-3)
 
 template <bool KDA>
 struct alignas(128) PrefillUIn {   // one chunk's inputs (token rows padded against bank conflicts;
@@ -423,7 +423,7 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
 }
 
 // Named barrier of the preparation group (warps 4-11), and its OR form.
-__device__ __forceinline__ void ubar() { asm volatile("bar.sync 1, %0;" ::"n"(kUCompute) : "memory"); }
+__device__ __forceinline__ void ubar() { asm volatile("bar.sync 1, %0;" ::"n"(kUPrep) : "memory"); }
 
 __device__ __forceinline__ bool ubar_or(bool v) {
     int r;
@@ -433,7 +433,7 @@ __device__ __forceinline__ bool ubar_or(bool v) {
         "bar.red.or.pred q, 1, %2, p;\n\t"
         "selp.s32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"((int)v), "n"(kUCompute)
+        : "r"((int)v), "n"(kUPrep)
         : "memory");
     return r != 0;
 }
@@ -461,7 +461,7 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 template <bool KDA>
 __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const PrefillArgs a,
                                                                       const __grid_constant__ PrefillMaps mp) {
-    constexpr int D = 128, C = kUChunk, NT = kUCompute;
+    constexpr int D = 128, C = kUChunk, NT = kUPrep;
     using Sm = PrefillUSmem<KDA>;
     using In = PrefillUIn<KDA>;
     extern __shared__ __align__(128) unsigned char smem_u[];

@@ -380,7 +380,7 @@ struct PrefillUSmem {
     alignas(16) float fac[KDA ? 24 : 1][RP]; // KDA: the decay-factored pair operands (below)
     PrefillUIn<KDA> in[2];                   // input slots: chunk c in slot c % 2
     alignas(16) float A[C][C + 4];           // rows read as float4 (the last 4 columns unused)
-    alignas(16) float P[C][C + 4];
+    alignas(16) float P[2][C][C + 4];        // [chunk % 2]: read by the tensor-memory warpgroup
     float gC[2][D];                          // [slot]: Gamma over the whole chunk, per key row
     uint64_t mbar_in[2];       // input slot filled
     uint64_t mbar_ops;         // a chunk's operands written (preparation group -> tensor-memory warpgroup)
@@ -577,6 +577,45 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                 umma_commit(&S.mbar_yo);
             }
             __syncwarp();
+            if (t >= 32) {   // while lane 0 issues: [Kh; P] of this chunk from its input slot
+                In &I = S.in[sl];
+                const int u = t - 32;   // 96 threads
+                for (int e = u; e < D * C / 4; e += 96) {   // Kh: key row e % D, tokens 4 (e / D) ..
+                    const int r = e % D, t4 = 4 * (e / D);
+                    const float glast = KDA ? I.g[C - 1][r] : I.g[0][C - 1];
+                    float kh[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float gt = KDA ? I.g[t4 + j][r] : I.g[0][t4 + j];
+                        kh[j] = I.k[t4 + j][r] * ex2_ftz(glast - gt);
+                    }
+                    uint4 bb, bs;
+                    split4(make_float4(kh[0], kh[1], kh[2], kh[3]), bb, bs);
+                    const int wd = umma_word(D + C, r, t4);
+                    *reinterpret_cast<uint4 *>(&S.khp[sl][0][wd]) = bb;
+                    *reinterpret_cast<uint4 *>(&S.khp[sl][1][wd]) = bs;
+                }
+                if (u < C * C / 4) {   // P: token u % C, columns 4 (u / C) ..
+                    const int tt = u % C, i4 = 4 * (u / C);
+                    uint4 bb, bs;
+                    split4(*reinterpret_cast<const float4 *>(&S.P[sl][tt][i4]), bb, bs);
+                    const int wd = umma_word(D + C, D + tt, i4);
+                    *reinterpret_cast<uint4 *>(&S.khp[sl][0][wd]) = bb;
+                    *reinterpret_cast<uint4 *>(&S.khp[sl][1][wd]) = bs;
+                }
+                fence_async_smem();
+            }
+            tbar();
+            if (t == 0 && ch + 2 < nchunks) {   // the slot's next contents: chunk ch + 2
+                In &I = S.in[sl];
+                const int t0 = (ch + 2) * C;
+                uint64_t *bar = &S.mbar_in[sl];
+                mbar_arrive_expect_tx(bar, prefill_load_bytes<KDA>());
+                tma_load_4d(&I.k[0][0], &mp.k, 0, gk, b, t0, bar);
+                tma_load_4d(&I.q[0][0], &mp.q, 0, gk, b, t0, bar);
+                tma_load_4d(&I.v[0][0], &mp.v, 0, h, b, t0, bar);
+                if (KDA) tma_load_4d(&I.g[0][0], &mp.g, 0, h, b, t0, bar);
+            }
             {
                 const bool okw = mbar_wait_bounded(&S.mbar_yo, (uint32_t)(ch & 1), a.status);
                 if (tbar_or(!okw)) {
@@ -781,7 +820,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                     const float dkk = ((part[t] + part[256 + t]) + (part[512 + t] + part[768 + t])) * f;
                     const float dqk = ((part[1024 + t] + part[1280 + t]) + (part[1536 + t] + part[1792 + t])) * f;
                     S.A[ti][ii] = ii < ti ? -I.beta[ti] * dkk : 0.f;   // stored negated (the substitution adds)
-                    S.P[ti][ii] = ii <= ti ? dqk : 0.f;
+                    S.P[sl][ti][ii] = ii <= ti ? dqk : 0.f;
                 }
             } else {
                 // KDA: per-channel factors 2^(g_t - g_i).  Across the two
@@ -853,7 +892,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                     ii = 8 + (lane & 7);
                 }
                 S.A[ti][ii] = ii < ti ? -I.beta[ti] * dkk : 0.f;   // stored negated (the substitution adds)
-                S.P[ti][ii] = ii <= ti ? dqk : 0.f;
+                S.P[sl][ti][ii] = ii <= ti ? dqk : 0.f;
             }
             ubar();
             // forward substitution, one column per thread: threads 0-127 the key
@@ -891,9 +930,9 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
             return true;
         };
 
-        // Chunk c, part 2: the operand splits ([Qg; -W] single; [Kh; P] into
-        // slot c % 2), then chunk c + 2's inputs into the slot just read.  The
-        // caller guarantees that no group in flight reads qw or the slot written.
+        // Chunk c, part 2: the split of [Qg; -W] (single; the caller guarantees
+        // that group 1 of the previous chunk is complete).  [Kh; P] and the
+        // reload of the input slot follow on the tensor-memory warpgroup.
         auto prep_operands = [&](int c) {
             In &I = S.in[c & 1];
             const int sl = c & 1;
@@ -921,31 +960,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                 *reinterpret_cast<uint4 *>(&S.qw[wq]) = bb;
                 *reinterpret_cast<uint4 *>(&S.qw[sq]) = bs;
             }
-            for (int e = t; e < D * C / 4; e += NT) {   // Kh: key row e % D, tokens 4 (e / D) ..
-                const int r = e % D, t4 = 4 * (e / D);
-                const float glast = KDA ? I.g[C - 1][r] : I.g[0][C - 1];
-                float kh[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float gt = KDA ? I.g[t4 + j][r] : I.g[0][t4 + j];
-                    kh[j] = I.k[t4 + j][r] * ex2_ftz(glast - gt);
-                }
-                uint4 bb, bs;
-                split4(make_float4(kh[0], kh[1], kh[2], kh[3]), bb, bs);
-                const int wd = umma_word(D + C, r, t4);
-                *reinterpret_cast<uint4 *>(&S.khp[sl][0][wd]) = bb;
-                *reinterpret_cast<uint4 *>(&S.khp[sl][1][wd]) = bs;
-            }
-            if (t < C * C / 4) {   // P: token t % C, columns 4 (t / C) ..
-                const int tt = t % C, i4 = 4 * (t / C);
-                uint4 bb, bs;
-                split4(*reinterpret_cast<const float4 *>(&S.P[tt][i4]), bb, bs);
-                const int wd = umma_word(D + C, D + tt, i4);
-                *reinterpret_cast<uint4 *>(&S.khp[sl][0][wd]) = bb;
-                *reinterpret_cast<uint4 *>(&S.khp[sl][1][wd]) = bs;
-            }
             fence_async_smem();
-            if (c + 2 < nchunks) issue_load(c + 2);   // its barrier also orders the reads above
         };
 
         bool ok = true;
@@ -958,7 +973,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
 #pragma unroll 1
         for (int c = 0; ok && c < nchunks; ++c) {
             if (c + 1 < nchunks) load_scalars(c + 1, bet_n, gl_n);
-            // ud, gC and the [Kh; P] slot of c % 2 were last read by chunk c - 2
+            // ud, gC and P of c % 2 were last read by chunk c - 2
             if (c >= 2) {
                 const bool okw = mbar_wait_bounded(&S.mbar_up[c & 1], (uint32_t)(((c - 2) >> 1) & 1), a.status);
                 if (ubar_or(!okw)) {

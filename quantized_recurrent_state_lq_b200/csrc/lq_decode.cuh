@@ -141,8 +141,16 @@ __device__ __forceinline__ void warp_reduce_dots(float (&v)[2 * NE]) {
     }
 }
 
+// GDN's BF16 buffered tokens at d = 128 stream four tokens per warp step (one
+// 16-byte load per lane covers a whole entry) in the registers of six CTAs per
+// SM.  (KDA's per-channel decay state leaves too few registers at that
+// occupancy: there the variant spills and runs 5% slower than the pairs.)
+template <int DK, int DV, bool KDA, bool TB>
+constexpr bool buf_quads() { return TB && !KDA && DK == 128 && DV == 128; }
+
 template <int DK, int DV, bool KDA, bool DAMP, bool TB, int BITS>
-__global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kBufThreads, buf_quads<DK, DV, KDA, TB>() ? 6 : 7)
+    decode_buffer_kernel(const DecodeArgs a) {
     static_assert(BITS == 8 || !DAMP, "packed codes are built without BF16 rows");
     extern __shared__ __align__(128) unsigned char smem[];
     BufSmem<DK, DV> &S = *reinterpret_cast<BufSmem<DK, DV> *>(smem);
@@ -232,7 +240,24 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
             if (e0 + 1 < E) load_bf16(1, e0 + 1);
         }
     };
-    load_pair(2 * warp);
+    constexpr bool Q4 = buf_quads<DK, DV, KDA, TB>();
+    // BF16 tokens in quads (Q4): token j's [k | u] is 256 bf16 = 512 bytes; lane
+    // l's 16-byte piece holds k channels 8 l .. 8 l + 7 (lanes 0-15) or u
+    // columns 8 (l - 16) .. (lanes 16-31).  The compensators (FP32) keep the pairs.
+    uint4 tkq[4];
+    auto load_quad = [&](int j0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (j0 + i < n) tkq[i] = __ldcs(reinterpret_cast<const uint4 *>(rec_tok16 + (size_t)(j0 + i) * EF) + lane);
+    };
+    if constexpr (Q4) {
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+            if (2 * warp + p < L.r) load_fp32(p, 2 * warp + p);
+        load_quad(4 * warp);
+    } else {
+        load_pair(2 * warp);
+    }
 
     // (a) step inputs, the guarded decay (G_t, sigma_t, the entries' rescaling
     // rho), x = G_t (k, q), a = m * sigma_t * x.
@@ -328,6 +353,7 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
 
     // (c) codes.
     float ek[4] = {0.f, 0.f, 0.f, 0.f}, eq[4] = {0.f, 0.f, 0.f, 0.f};
+    float R[Q4 ? 16 : 1];   // BF16 token quads' registers (below)
     if (!DAMP) {
         for (int cb = warp; cb < DV / 16; cb += kBufWarps) {   // a warp per 16 value columns
             const int c0 = 16 * cb;
@@ -495,43 +521,152 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
                 }
             }
         };
-        for (int e0 = 2 * warp; e0 < E; e0 += 2 * kBufWarps) {
-            if (rebase) {
+        if constexpr (!Q4) {
+            for (int e0 = 2 * warp; e0 < E; e0 += 2 * kBufWarps) {
+                if (rebase) {
 #pragma unroll
-                for (int p = 0; p < 2; ++p)
-                    if (e0 + p < E) rescale(p, e0 + p);
-            }
-            float d[4];
-            float4 uv[2];
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                float dk_ = 0.f, dq_ = 0.f;
-                if (e0 + p < E) {
-                    if (XPL == 4) {
-                        const float4 kv = kb[p];
-                        dk_ = fmaf(kv.x, xk[0], fmaf(kv.y, xk[1 % XPL], fmaf(kv.z, xk[2 % XPL], kv.w * xk[3 % XPL])));
-                        dq_ = fmaf(kv.x, xq[0], fmaf(kv.y, xq[1 % XPL], fmaf(kv.z, xq[2 % XPL], kv.w * xq[3 % XPL])));
-                    } else {
-                        const float2 kv = kb2[p];
-                        dk_ = fmaf(kv.x, xk[0], kv.y * xk[1 % XPL]);
-                        dq_ = fmaf(kv.x, xq[0], kv.y * xq[1 % XPL]);
-                    }
+                    for (int p = 0; p < 2; ++p)
+                        if (e0 + p < E) rescale(p, e0 + p);
                 }
-                d[2 * p] = dk_;
-                d[2 * p + 1] = dq_;
-                uv[p] = ub[p];
-            }
-            const int ne = min(2, E - e0);
-            load_pair(e0 + 2 * kBufWarps);   // refill the registers while this pair is reduced
-            warp_reduce_dots<2>(d);
-            if (lane < DV / 4) {
+                float d[4];
+                float4 uv[2];
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
-                    if (p < ne) {
-                        ek[0] = fmaf(uv[p].x, d[2 * p], ek[0]); ek[1] = fmaf(uv[p].y, d[2 * p], ek[1]);
-                        ek[2] = fmaf(uv[p].z, d[2 * p], ek[2]); ek[3] = fmaf(uv[p].w, d[2 * p], ek[3]);
-                        eq[0] = fmaf(uv[p].x, d[2 * p + 1], eq[0]); eq[1] = fmaf(uv[p].y, d[2 * p + 1], eq[1]);
-                        eq[2] = fmaf(uv[p].z, d[2 * p + 1], eq[2]); eq[3] = fmaf(uv[p].w, d[2 * p + 1], eq[3]);
+                    float dk_ = 0.f, dq_ = 0.f;
+                    if (e0 + p < E) {
+                        if (XPL == 4) {
+                            const float4 kv = kb[p];
+                            dk_ = fmaf(kv.x, xk[0], fmaf(kv.y, xk[1 % XPL], fmaf(kv.z, xk[2 % XPL], kv.w * xk[3 % XPL])));
+                            dq_ = fmaf(kv.x, xq[0], fmaf(kv.y, xq[1 % XPL], fmaf(kv.z, xq[2 % XPL], kv.w * xq[3 % XPL])));
+                        } else {
+                            const float2 kv = kb2[p];
+                            dk_ = fmaf(kv.x, xk[0], kv.y * xk[1 % XPL]);
+                            dq_ = fmaf(kv.x, xq[0], kv.y * xq[1 % XPL]);
+                        }
+                    }
+                    d[2 * p] = dk_;
+                    d[2 * p + 1] = dq_;
+                    uv[p] = ub[p];
+                }
+                const int ne = min(2, E - e0);
+                load_pair(e0 + 2 * kBufWarps);   // refill the registers while this pair is reduced
+                warp_reduce_dots<2>(d);
+                if (lane < DV / 4) {
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        if (p < ne) {
+                            ek[0] = fmaf(uv[p].x, d[2 * p], ek[0]); ek[1] = fmaf(uv[p].y, d[2 * p], ek[1]);
+                            ek[2] = fmaf(uv[p].z, d[2 * p], ek[2]); ek[3] = fmaf(uv[p].w, d[2 * p], ek[3]);
+                            eq[0] = fmaf(uv[p].x, d[2 * p + 1], eq[0]); eq[1] = fmaf(uv[p].y, d[2 * p + 1], eq[1]);
+                            eq[2] = fmaf(uv[p].z, d[2 * p + 1], eq[2]); eq[3] = fmaf(uv[p].w, d[2 * p + 1], eq[3]);
+                        }
+                    }
+                }
+            }
+        } else {
+            // compensators: FP32 pairs
+            for (int e0 = 2 * warp; e0 < L.r; e0 += 2 * kBufWarps) {
+                if (rebase) {
+#pragma unroll
+                    for (int p = 0; p < 2; ++p)
+                        if (e0 + p < L.r) rescale(p, e0 + p);
+                }
+                float d[4];
+                float4 uv[2];
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    float dk_ = 0.f, dq_ = 0.f;
+                    if (e0 + p < L.r) {
+                        const float4 kv = kb[p];
+                        dk_ = fmaf(kv.x, xk[0], fmaf(kv.y, xk[1], fmaf(kv.z, xk[2], kv.w * xk[3])));
+                        dq_ = fmaf(kv.x, xq[0], fmaf(kv.y, xq[1], fmaf(kv.z, xq[2], kv.w * xq[3])));
+                    }
+                    d[2 * p] = dk_;
+                    d[2 * p + 1] = dq_;
+                    uv[p] = ub[p];
+                }
+                const int ne = min(2, L.r - e0);
+#pragma unroll
+                for (int p = 0; p < 2; ++p)
+                    if (e0 + 2 * kBufWarps + p < L.r) load_fp32(p, e0 + 2 * kBufWarps + p);
+                warp_reduce_dots<2>(d);
+                if (lane < DV / 4) {
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        if (p < ne) {
+                            ek[0] = fmaf(uv[p].x, d[2 * p], ek[0]); ek[1] = fmaf(uv[p].y, d[2 * p], ek[1]);
+                            ek[2] = fmaf(uv[p].z, d[2 * p], ek[2]); ek[3] = fmaf(uv[p].w, d[2 * p], ek[3]);
+                            eq[0] = fmaf(uv[p].x, d[2 * p + 1], eq[0]); eq[1] = fmaf(uv[p].y, d[2 * p + 1], eq[1]);
+                            eq[2] = fmaf(uv[p].z, d[2 * p + 1], eq[2]); eq[3] = fmaf(uv[p].w, d[2 * p + 1], eq[3]);
+                        }
+                    }
+                }
+            }
+            if (lane < DV / 4) {   // the compensators' part, before the tokens' registers
+#pragma unroll
+                for (int u = 0; u < 4; ++u) S.red[warp][4 * lane + u] = make_float2(ek[u], eq[u]);
+            }
+            // tokens: BF16 quads.  R holds (G k, G q) of key channels 8 l ..
+            // 8 l + 7 on lanes l < 16, which form the dot products, and the
+            // sums of value columns 8 (l - 16) .. on lanes l >= 16.
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float2 x = lane < 16 ? S.x2[8 * lane + c] : make_float2(0.f, 0.f);
+                R[c] = x.x;
+                R[8 + c] = x.y;
+            }
+            for (int j0 = 4 * warp; j0 < n; j0 += 4 * kBufWarps) {
+                if (rebase && lane < 16) {   // the keys' rescaling, written back in BF16
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (j0 + i < n) {
+                            uint32_t w[4] = {tkq[i].x, tkq[i].y, tkq[i].z, tkq[i].w};
+#pragma unroll
+                            for (int c2 = 0; c2 < 4; ++c2) {
+                                const float2 f = bf16x2_to_f2(w[c2]);
+                                w[c2] = (uint32_t)bf16_rne(f.x * rho_s[8 * lane + 2 * c2]) |
+                                        ((uint32_t)bf16_rne(f.y * rho_s[8 * lane + 2 * c2 + 1]) << 16);
+                            }
+                            tkq[i] = make_uint4(w[0], w[1], w[2], w[3]);
+                            reinterpret_cast<uint4 *>(rec_tok16 + (size_t)(j0 + i) * EF)[lane] = tkq[i];
+                        }
+                    }
+                }
+                float d[8];
+                uint4 uk[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float dk_ = 0.f, dq_ = 0.f;
+                    if (j0 + i < n && lane < 16) {
+                        const uint32_t w[4] = {tkq[i].x, tkq[i].y, tkq[i].z, tkq[i].w};
+#pragma unroll
+                        for (int c2 = 0; c2 < 4; ++c2) {
+                            const float2 f = bf16x2_to_f2(w[c2]);
+                            dk_ = fmaf(f.x, R[2 * c2], fmaf(f.y, R[2 * c2 + 1], dk_));
+                            dq_ = fmaf(f.x, R[8 + 2 * c2], fmaf(f.y, R[8 + 2 * c2 + 1], dq_));
+                        }
+                    }
+                    d[2 * i] = dk_;
+                    d[2 * i + 1] = dq_;
+                    uk[i] = tkq[i];
+                }
+                const int ne = min(4, n - j0);
+                load_quad(j0 + 4 * kBufWarps);   // the next quad in flight while this one is reduced
+                warp_reduce_dots<4>(d);
+                if (lane >= 16) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (i < ne) {
+                            const uint32_t w[4] = {uk[i].x, uk[i].y, uk[i].z, uk[i].w};
+#pragma unroll
+                            for (int c2 = 0; c2 < 4; ++c2) {
+                                const float2 f = bf16x2_to_f2(w[c2]);
+                                R[2 * c2] = fmaf(f.x, d[2 * i], R[2 * c2]);
+                                R[2 * c2 + 1] = fmaf(f.y, d[2 * i], R[2 * c2 + 1]);
+                                R[8 + 2 * c2] = fmaf(f.x, d[2 * i + 1], R[8 + 2 * c2]);
+                                R[8 + 2 * c2 + 1] = fmaf(f.y, d[2 * i + 1], R[8 + 2 * c2 + 1]);
+                            }
+                        }
                     }
                 }
             }
@@ -539,9 +674,20 @@ __global__ void __launch_bounds__(kBufThreads, 7) decode_buffer_kernel(const Dec
     }
 
     // (e) combine, output, append.
-    if (lane < DV / 4) {
+    if constexpr (!Q4) {
+        if (lane < DV / 4) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) S.red[warp][4 * lane + u] = make_float2(ek[u], eq[u]);
+            for (int u = 0; u < 4; ++u) S.red[warp][4 * lane + u] = make_float2(ek[u], eq[u]);
+        }
+    } else {
+        __syncwarp();
+        if (lane >= 16) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float2 &r = S.red[warp][8 * (lane - 16) + c];
+                r = make_float2(r.x + R[c], r.y + R[8 + c]);
+            }
+        }
     }
     uint16_t khat = 0;
     if (tb) {

@@ -211,6 +211,7 @@ def test_windowed_teacher_forced(fused, gate, B, H, Hk, dk, dv, W, r):
     ("kda", 2, 4096, 0, -1.0),    # the longest window: 2^-1900 by its end
     ("kda", 2, 320, 1, -1.0),     # BF16 buffer: keys rounded against the guarded chain
     ("gdn", 2, 4096, 0, None),    # the benchmark's GDN decays: Gamma ~2^-180 by the end
+    ("gdn", 2, 320, 1, -1.0),     # BF16 buffer, whole-entry loads: re-based every ~140 tokens
 ])
 def test_long_windows_strong_decays(fused, gate, H, W, bf16, mu):
     """Decay products far below the FP32 range within a window (the decay

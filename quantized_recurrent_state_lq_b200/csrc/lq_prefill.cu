@@ -19,10 +19,12 @@
 // for gates in (0, 1], so nothing overflows however strong the decay.
 //
 // Two kernels, one CTA per head, products in three TF32 passes on the tensor
-// cores (FP32-level accuracy), pair matrices and substitutions in FP32:
+// cores (FP32-level accuracy), substitutions in FP32:
 //   prefill_umma_kernel (d_k = d_v = 128, 16-byte aligned rows): the state in
-//     tensor memory, the products as tcgen05.mma chains issued by one warp
-//     while eight others prepare the next chunk; inputs by TMA tensor copies;
+//     tensor memory, the products as tcgen05.mma chains issued by a
+//     tensor-memory warpgroup while eight other warps prepare the next chunk
+//     (GDN's pair matrices there on mma.sync, KDA's in FP32); inputs by TMA
+//     tensor copies;
 //   prefill_tc_kernel (other shapes, other rows): the state in registers as
 //     mma.sync accumulator tiles, the chunk's inputs staged by plain loads.
 #include <cuda.h>
@@ -770,55 +772,41 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
             }
             ubar();
             if (!KDA) {
-                // pair matrices, one decay factor per pair: threads 0-143 take a
-                // 2 x 2 block of the lower triangle (blocks (a, b), b <= a, rows
-                // 2a, 2a+1, columns 2b, 2b+1) over a quarter of the channels
-                // (float4 groups 4 j + quarter), eight packed sums each; the
-                // quarters' partial sums meet in wst (free until the
-                // substitution), then every thread finishes one entry.
-                float *part = &S.wst[0][0];   // [kind][quarter][16][16]
-                if (t < 144) {
-                    const int bi = t >> 2, qu = t & 3;
-                    int ba = 0;
-                    while ((ba + 1) * (ba + 2) / 2 <= bi) ++ba;
-                    const int bb = bi - ba * (ba + 1) / 2;
-                    const int t0 = 2 * ba, i0 = 2 * bb;
-                    float2 kk00 = f2(0.f, 0.f), kk01 = kk00, kk10 = kk00, kk11 = kk00;
-                    float2 qk00 = kk00, qk01 = kk00, qk10 = kk00, qk11 = kk00;
-#pragma unroll 2
-                    for (int j = 0; j < D / 16; ++j) {
-                        const int r = 4 * (4 * j + qu);
-                        const float4 ka = *reinterpret_cast<const float4 *>(&I.k[t0][r]);
-                        const float4 kb = *reinterpret_cast<const float4 *>(&I.k[t0 + 1][r]);
-                        const float4 qa = *reinterpret_cast<const float4 *>(&I.q[t0][r]);
-                        const float4 qb = *reinterpret_cast<const float4 *>(&I.q[t0 + 1][r]);
-                        const float4 ia = *reinterpret_cast<const float4 *>(&I.k[i0][r]);
-                        const float4 ib = *reinterpret_cast<const float4 *>(&I.k[i0 + 1][r]);
-                        kk00 = ffma2(f2(ka.x, ka.y), f2(ia.x, ia.y), ffma2(f2(ka.z, ka.w), f2(ia.z, ia.w), kk00));
-                        kk01 = ffma2(f2(ka.x, ka.y), f2(ib.x, ib.y), ffma2(f2(ka.z, ka.w), f2(ib.z, ib.w), kk01));
-                        kk10 = ffma2(f2(kb.x, kb.y), f2(ia.x, ia.y), ffma2(f2(kb.z, kb.w), f2(ia.z, ia.w), kk10));
-                        kk11 = ffma2(f2(kb.x, kb.y), f2(ib.x, ib.y), ffma2(f2(kb.z, kb.w), f2(ib.z, ib.w), kk11));
-                        qk00 = ffma2(f2(qa.x, qa.y), f2(ia.x, ia.y), ffma2(f2(qa.z, qa.w), f2(ia.z, ia.w), qk00));
-                        qk01 = ffma2(f2(qa.x, qa.y), f2(ib.x, ib.y), ffma2(f2(qa.z, qa.w), f2(ib.z, ib.w), qk01));
-                        qk10 = ffma2(f2(qb.x, qb.y), f2(ia.x, ia.y), ffma2(f2(qb.z, qb.w), f2(ia.z, ia.w), qk10));
-                        qk11 = ffma2(f2(qb.x, qb.y), f2(ib.x, ib.y), ffma2(f2(qb.z, qb.w), f2(ib.z, ib.w), qk11));
+                // pair matrices, one decay factor per pair: the products
+                // [K; Q] K^T (32 x 16, over the D key channels) on the tensor
+                // cores, mma.sync m16n8k8 in three TF32 passes (FP32-level
+                // accuracy).  Warp w takes the output tile of rows 16 (w / 2 % 2)
+                // .. (K for 0, Q for 1) and columns 8 (w % 2) .. over key
+                // channels 64 (w / 4) ..; the two halves' partial sums meet in
+                // wst (free until the substitution), then every thread
+                // finishes one entry.
+                float *part = &S.wst[0][0];   // [kind][channel half][16][16]
+                {
+                    const int mt = (warp >> 1) & 1, nt = warp & 1, kh = warp >> 2;
+                    const int gi = lane >> 2, tq = lane & 3;
+                    const float(*X)[In::RP] = mt ? I.q : I.k;
+                    const float *kr = &I.k[8 * nt + gi][0];
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const int k0 = (D / 2) * kh + 8 * ks + tq;
+                        uint32_t ab[4], as[4];
+                        tf32_split(X[gi][k0], ab[0], as[0]);
+                        tf32_split(X[gi + 8][k0], ab[1], as[1]);
+                        tf32_split(X[gi][k0 + 4], ab[2], as[2]);
+                        tf32_split(X[gi + 8][k0 + 4], ab[3], as[3]);
+                        mma3(d, ab, as, kr[k0], kr[k0 + 4]);
                     }
-                    float *pk = part + qu * 256, *pq = part + 1024 + qu * 256;
-                    pk[t0 * 16 + i0] = kk00.x + kk00.y;
-                    pk[t0 * 16 + i0 + 1] = kk01.x + kk01.y;
-                    pk[(t0 + 1) * 16 + i0] = kk10.x + kk10.y;
-                    pk[(t0 + 1) * 16 + i0 + 1] = kk11.x + kk11.y;
-                    pq[t0 * 16 + i0] = qk00.x + qk00.y;
-                    pq[t0 * 16 + i0 + 1] = qk01.x + qk01.y;
-                    pq[(t0 + 1) * 16 + i0] = qk10.x + qk10.y;
-                    pq[(t0 + 1) * 16 + i0 + 1] = qk11.x + qk11.y;
+                    float *pp = part + (2 * mt + kh) * 256 + 8 * nt + 2 * tq;
+                    *reinterpret_cast<float2 *>(pp + gi * 16) = make_float2(d[0], d[1]);
+                    *reinterpret_cast<float2 *>(pp + (gi + 8) * 16) = make_float2(d[2], d[3]);
                 }
                 ubar();
                 {   // entry (ti, ii) = (t / 16, t % 16)
                     const int ti = t >> 4, ii = t & 15;
                     const float f = ex2_ftz(fminf(I.g[0][ti] - I.g[0][ii], 0.f));
-                    const float dkk = ((part[t] + part[256 + t]) + (part[512 + t] + part[768 + t])) * f;
-                    const float dqk = ((part[1024 + t] + part[1280 + t]) + (part[1536 + t] + part[1792 + t])) * f;
+                    const float dkk = (part[t] + part[256 + t]) * f;
+                    const float dqk = (part[512 + t] + part[768 + t]) * f;
                     S.A[ti][ii] = ii < ti ? -I.beta[ti] * dkk : 0.f;   // stored negated (the substitution adds)
                     S.P[sl][ti][ii] = ii <= ti ? dqk : 0.f;
                 }

@@ -384,6 +384,7 @@ struct PrefillUSmem {
     alignas(16) float A[C][C + 4];           // rows read as float4 (the last 4 columns unused)
     alignas(16) float P[2][C][C + 4];        // [chunk % 2]: read by the tensor-memory warpgroup
     float gC[2][D];                          // [slot]: Gamma over the whole chunk, per key row
+    float bg[C];                             // GDN: b_t Gamma_t of the chunk being prepared
     uint64_t mbar_in[2];       // input slot filled
     uint64_t mbar_ops;         // a chunk's operands written (preparation group -> tensor-memory warpgroup)
     uint64_t mbar_yo;          // group 1 complete
@@ -809,6 +810,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                     const float dqk = (part[512 + t] + part[768 + t]) * f;
                     S.A[ti][ii] = ii < ti ? -I.beta[ti] * dkk : 0.f;   // stored negated (the substitution adds)
                     S.P[sl][ti][ii] = ii <= ti ? dqk : 0.f;
+                    if (t < C) S.bg[t] = I.beta[t] * ex2_ftz(I.g[0][t]);   // the substitution's key scale
                 }
             } else {
                 // KDA: per-channel factors 2^(g_t - g_i).  Across the two
@@ -890,7 +892,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                 float x[C];
 #pragma unroll
                 for (int tt = 0; tt < C; ++tt) {   // the right-hand sides first (independent loads)
-                    if (t < D) x[tt] = I.beta[tt] * (I.k[tt][cc] * ex2_ftz(KDA ? I.g[tt][cc] : I.g[0][tt]));
+                    if (t < D) x[tt] = KDA ? I.beta[tt] * (I.k[tt][cc] * ex2_ftz(I.g[tt][cc])) : S.bg[tt] * I.k[tt][cc];
                     else x[tt] = I.beta[tt] * I.v[tt][cc];
                 }
                 // x_t += sum_{i<t} (-A_ti) x_i, two terms per packed FMA (the

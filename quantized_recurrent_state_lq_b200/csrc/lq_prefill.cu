@@ -740,7 +740,19 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
             if (ubar_or(!okw)) return false;
             if (t < C) {
                 I.beta[t] = bet;
-                if (!KDA) I.g[0][t] = (c * C + t < a.T) ? fmaxf(lg2_ftz(gl), -150.0f) : 0.f;
+                if (!KDA) {
+                    // log2 decay, floored at -150 (a decay of 0 wipes the
+                    // state), 0 past T; then its cumulative sum within the
+                    // chunk as a shuffle scan over lanes 0-15, and Gamma_C
+                    float l = (c * C + t < a.T) ? fmaxf(lg2_ftz(gl), -150.0f) : 0.f;
+#pragma unroll
+                    for (int o = 1; o < C; o <<= 1) {
+                        const float v = __shfl_up_sync(0x0000ffffu, l, o);
+                        if (t >= o) l += v;
+                    }
+                    I.g[0][t] = l;
+                    if (t == C - 1) S.gC[sl][0] = ex2_ftz(l);
+                }
             }
             if (KDA) {   // decays -> log2, floored at -150 (a decay of 0 wipes the state); 0 past T
 #pragma unroll
@@ -751,7 +763,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                 }
             }
             ubar();
-            // cumulative log2 decay within the chunk, Gamma_C
+            // KDA: cumulative log2 decay within the chunk per key channel, Gamma_C
             if (KDA) {
                 if (t < D) {
                     float acc = 0.f;
@@ -762,16 +774,8 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                     }
                     S.gC[sl][t] = ex2_ftz(acc);
                 }
-            } else if (t == 0) {
-                float acc = 0.f;
-#pragma unroll
-                for (int tt = 0; tt < C; ++tt) {
-                    acc += I.g[0][tt];
-                    I.g[0][tt] = acc;
-                }
-                S.gC[sl][0] = ex2_ftz(acc);
+                ubar();
             }
-            ubar();
             if (!KDA) {
                 // pair matrices, one decay factor per pair: the products
                 // [K; Q] K^T (32 x 16, over the D key channels) on the tensor
@@ -787,8 +791,8 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                     const int gi = lane >> 2, tq = lane & 3;
                     const float(*X)[In::RP] = mt ? I.q : I.k;
                     const float *kr = &I.k[8 * nt + gi][0];
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+                    float d[4][4] = {};   // four accumulators (k-steps mod 4): shorter MMA chains
+#pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const int k0 = (D / 2) * kh + 8 * ks + tq;
                         uint32_t ab[4], as[4];
@@ -796,11 +800,14 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const Prefil
                         tf32_split(X[gi + 8][k0], ab[1], as[1]);
                         tf32_split(X[gi][k0 + 4], ab[2], as[2]);
                         tf32_split(X[gi + 8][k0 + 4], ab[3], as[3]);
-                        mma3(d, ab, as, kr[k0], kr[k0 + 4]);
+                        mma3(d[ks & 3], ab, as, kr[k0], kr[k0 + 4]);
                     }
+                    float e[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) e[j] = (d[0][j] + d[1][j]) + (d[2][j] + d[3][j]);
                     float *pp = part + (2 * mt + kh) * 256 + 8 * nt + 2 * tq;
-                    *reinterpret_cast<float2 *>(pp + gi * 16) = make_float2(d[0], d[1]);
-                    *reinterpret_cast<float2 *>(pp + (gi + 8) * 16) = make_float2(d[2], d[3]);
+                    *reinterpret_cast<float2 *>(pp + gi * 16) = make_float2(e[0], e[1]);
+                    *reinterpret_cast<float2 *>(pp + (gi + 8) * 16) = make_float2(e[2], e[3]);
                 }
                 ubar();
                 {   // entry (ti, ii) = (t / 16, t % 16)
